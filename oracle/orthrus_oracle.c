@@ -1,0 +1,694 @@
+/*
+ * Plain CPU oracle for the Orthrus dual-view decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg load this library.  The CUDA product path
+ * shares no code with it.
+ *
+ * Source: "Orthrus: Memory-Efficient Parallel Token Generation via Dual-View
+ * Diffusion" as described by the paper-notes page (zhangshuibai.github.io,
+ * spec-rl note 17): §2.1 (dual-view layer: per-layer extra W_Q/W_K/W_V, shared
+ * LM head, frozen backbone), §2.2-2.3 (one shared AR-only KV cache, transient
+ * diffusion K/V), §3.2 (diffusion-view mask: committed prefix before the
+ * anchor plus bidirectional attention inside the block), §4.1 (the cycle:
+ * parallel projection, AR verification, consensus and cache truncation),
+ * §4.2 (greedy consensus), §4.3 (rejection sampling at T>0).  The
+ * hotdry.top engineering page ("推理机制") restates the same cycle.
+ *
+ * Arithmetic is fp64 throughout.  Weights arrive as fp32 arrays holding the
+ * exact model values (bf16 values are exactly representable in fp32).  Every
+ * output element is computed by one loop in ascending index order, so a row
+ * of a block gives bit-for-bit the value that the same row gives alone.
+ *
+ * Readings where the pages are silent (each restated in the design notes):
+ *   - pre-norm decoder, RMSNorm eps 1e-6, no biases, no QK-norm, SwiGLU FFN
+ *     down(silu(gate a) * up a), rotate-half RoPE with inv_freq_i =
+ *     theta^(-2i/hd), attention scale 1/sqrt(hd), GQA head h -> kv head
+ *     h / (n_q / n_kv);
+ *   - the cache holds x_<t; the anchor's K/V come from the block;
+ *   - block row k (0-based) sits at position t+k and predicts position t+k+1;
+ *   - the verify input is [x_t, y_1 .. y_{K-1}], no bonus token, n in [1, K];
+ *   - ties in argmax go to the lowest index;
+ *   - sampling at T>0 is Gumbel-max over Philox4x32-10 uniforms keyed by
+ *     (seed, step, row, id, purpose); acceptance is u < p/q; the residual is
+ *     max(0, p - q) renormalised, falling back to argmax p if it has no mass.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OC_OK 0
+#define OC_ERR_ARG 1
+#define OC_ERR_NOMEM 2
+#define OC_ERR_CAPACITY 3
+
+enum { OC_PURPOSE_DRAFT = 1, OC_PURPOSE_ACCEPT = 2, OC_PURPOSE_RESIDUAL = 3, OC_PURPOSE_AR = 4 };
+
+typedef struct {
+    int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab, mask_id;
+    double rope_theta, rms_eps;
+} oc_cfg;
+
+typedef struct {
+    const float *attn_norm, *wq, *wk, *wv, *wq_diff, *wk_diff, *wv_diff;
+    const float *wo, *ffn_norm, *w_gate, *w_up, *w_down;
+} oc_layer;
+
+typedef struct {
+    const float *embed, *final_norm, *lm_head;
+    const oc_layer *layers;
+} oc_model;
+
+/* ------------------------------------------------------------------------ */
+/* Building blocks of the frozen backbone (paper notes §2.1: everything but   */
+/* W_Q/W_K/W_V is the unchanged pre-trained layer).                           */
+/* ------------------------------------------------------------------------ */
+
+/* y = x / sqrt(mean(x^2) + eps) * gain */
+void oc_rmsnorm(const double *x, const float *gain, int n, double eps, double *y)
+{
+    double ss = 0.0;
+    for (int i = 0; i < n; ++i) ss += x[i] * x[i];
+    double inv = 1.0 / sqrt(ss / n + eps);
+    for (int i = 0; i < n; ++i) y[i] = x[i] * inv * (double)gain[i];
+}
+
+/* y[r][o] = sum_i x[r][i] * W[o][i]   (W row-major [out][in]) */
+void oc_linear(const double *x, int R, int in, const float *W, int out, double *y)
+{
+    #pragma omp parallel for schedule(static) collapse(2) if ((long)R * out * in > 2000000)
+    for (int r = 0; r < R; ++r)
+        for (int o = 0; o < out; ++o) {
+            const double *xr = x + (size_t)r * in;
+            const float *w = W + (size_t)o * in;
+            double s = 0.0;
+            for (int i = 0; i < in; ++i) s += xr[i] * (double)w[i];
+            y[(size_t)r * out + o] = s;
+        }
+}
+
+/* Rotate-half rotary embedding of n_heads vectors of length hd at `pos`:
+ * pairs (i, i + hd/2) rotate by pos * theta^(-2i/hd). */
+void oc_rope(double *x, int n_heads, int hd, int pos, double theta)
+{
+    int half = hd / 2;
+    for (int i = 0; i < half; ++i) {
+        double inv_freq = pow(theta, -2.0 * i / hd);
+        double ang = (double)pos * inv_freq;
+        double c = cos(ang), s = sin(ang);
+        for (int h = 0; h < n_heads; ++h) {
+            double *v = x + (size_t)h * hd;
+            double a = v[i], b = v[i + half];
+            v[i] = a * c - b * s;
+            v[i + half] = b * c + a * s;
+        }
+    }
+}
+
+double oc_silu(double g) { return g / (1.0 + exp(-g)); }
+
+/*
+ * Dual-view attention for a block of R query rows at positions t .. t+R-1.
+ *   q      [R][n_q][hd]
+ *   kc, vc [>= t][n_kv][hd]  committed cache rows 0 .. t-1
+ *   kb, vb [R][n_kv][hd]     the block's own K/V
+ *   mode 0 (AR verify / prefill, paper notes §4.1 step 2): row r sees cache
+ *          rows [0, t) and block rows 0 .. r (causal);
+ *   mode 1 (diffusion draft, paper notes §3.2): row r sees cache rows [0, t)
+ *          and every block row (bidirectional inside the block).
+ *   o      [R][n_q][hd]
+ */
+void oc_attention(const double *q, int R, int n_q, int n_kv, int hd,
+                  const double *kc, const double *vc, int t,
+                  const double *kb, const double *vb, int mode, double *o)
+{
+    int g = n_q / n_kv;
+    double scale = 1.0 / sqrt((double)hd);
+    #pragma omp parallel for schedule(static) collapse(2) if ((long)R * n_q * (t + R) * hd > 1000000)
+    for (int r = 0; r < R; ++r)
+        for (int h = 0; h < n_q; ++h) {
+            int kvh = h / g;
+            int nblk = (mode == 0) ? r + 1 : R;
+            int nkeys = t + nblk;
+            const double *qv = q + ((size_t)r * n_q + h) * hd;
+            double *s = (double *)malloc(sizeof(double) * (size_t)(nkeys > 0 ? nkeys : 1));
+            double m = -INFINITY;
+            for (int j = 0; j < nkeys; ++j) {
+                const double *kv = (j < t) ? kc + ((size_t)j * n_kv + kvh) * hd
+                                           : kb + ((size_t)(j - t) * n_kv + kvh) * hd;
+                double d = 0.0;
+                for (int i = 0; i < hd; ++i) d += qv[i] * kv[i];
+                s[j] = d * scale;
+                if (s[j] > m) m = s[j];
+            }
+            double l = 0.0;
+            for (int j = 0; j < nkeys; ++j) { s[j] = exp(s[j] - m); l += s[j]; }
+            double *ov = o + ((size_t)r * n_q + h) * hd;
+            for (int i = 0; i < hd; ++i) ov[i] = 0.0;
+            for (int j = 0; j < nkeys; ++j) {
+                const double *vv = (j < t) ? vc + ((size_t)j * n_kv + kvh) * hd
+                                           : vb + ((size_t)(j - t) * n_kv + kvh) * hd;
+                double p = s[j] / l;
+                for (int i = 0; i < hd; ++i) ov[i] += p * vv[i];
+            }
+            free(s);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* One forward of either view over a block of R rows.                         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * view 0 = AR (frozen W_Q/W_K/W_V), view 1 = diffusion (W^diff); all other
+ * weights are shared (paper notes §2.1).
+ * mode 0: the block's K/V are written into the cache at positions t .. t+R-1
+ *         (the AR path is the only writer of the cache, §2.2) and rows attend
+ *         causally;
+ * mode 1: the block's K/V stay in a transient buffer that is freed on return
+ *         (they never enter the cache, §2.1/§2.3) and rows attend to the
+ *         whole block.
+ * kc, vc: [n_layers][cap][n_kv][hd]; rows [0, t) are the committed prefix.
+ * logits [R][vocab] and final_hidden [R][hidden] (after the final norm) may
+ * be NULL.
+ */
+int oc_forward(const oc_cfg *c, const oc_model *w, int view, int mode,
+               const int32_t *tokens, int R, int t,
+               double *kc, double *vc, int cap,
+               double *logits, double *final_hidden)
+{
+    if (!c || !w || !tokens || R <= 0 || t < 0 || (view != 0 && view != 1) || (mode != 0 && mode != 1))
+        return OC_ERR_ARG;
+    if (t + R > cap && mode == 0) return OC_ERR_CAPACITY;
+    if (t > cap) return OC_ERR_CAPACITY;
+    const int d = c->hidden, nq = c->n_q_heads, nkv = c->n_kv_heads, hd = c->head_dim;
+    const int F = c->ffn, V = c->vocab;
+    for (int r = 0; r < R; ++r)
+        if (tokens[r] < 0 || tokens[r] >= V) return OC_ERR_ARG;
+
+    size_t qn = (size_t)nq * hd, kn = (size_t)nkv * hd;
+    double *h = calloc((size_t)R * d, sizeof(double));
+    double *a = calloc((size_t)R * d, sizeof(double));
+    double *q = calloc((size_t)R * qn, sizeof(double));
+    double *k = calloc((size_t)R * kn, sizeof(double));
+    double *v = calloc((size_t)R * kn, sizeof(double));
+    double *o = calloc((size_t)R * qn, sizeof(double));
+    double *y = calloc((size_t)R * d, sizeof(double));
+    double *gt = calloc((size_t)R * F, sizeof(double));
+    double *up = calloc((size_t)R * F, sizeof(double));
+    int rc = OC_OK;
+    if (!h || !a || !q || !k || !v || !o || !y || !gt || !up) { rc = OC_ERR_NOMEM; goto done; }
+
+    for (int r = 0; r < R; ++r)
+        for (int i = 0; i < d; ++i) h[(size_t)r * d + i] = (double)w->embed[(size_t)tokens[r] * d + i];
+
+    for (int l = 0; l < c->n_layers; ++l) {
+        const oc_layer *L = &w->layers[l];
+        double *kcl = kc + (size_t)l * cap * kn, *vcl = vc + (size_t)l * cap * kn;
+        for (int r = 0; r < R; ++r) oc_rmsnorm(h + (size_t)r * d, L->attn_norm, d, c->rms_eps, a + (size_t)r * d);
+        oc_linear(a, R, d, view ? L->wq_diff : L->wq, nq * hd, q);
+        oc_linear(a, R, d, view ? L->wk_diff : L->wk, nkv * hd, k);
+        oc_linear(a, R, d, view ? L->wv_diff : L->wv, nkv * hd, v);
+        for (int r = 0; r < R; ++r) {
+            oc_rope(q + r * qn, nq, hd, t + r, c->rope_theta);
+            oc_rope(k + r * kn, nkv, hd, t + r, c->rope_theta);
+        }
+        if (mode == 0) {
+            memcpy(kcl + (size_t)t * kn, k, sizeof(double) * R * kn);
+            memcpy(vcl + (size_t)t * kn, v, sizeof(double) * R * kn);
+            oc_attention(q, R, nq, nkv, hd, kcl, vcl, t, kcl + (size_t)t * kn, vcl + (size_t)t * kn, 0, o);
+        } else {
+            oc_attention(q, R, nq, nkv, hd, kcl, vcl, t, k, v, 1, o);
+        }
+        oc_linear(o, R, nq * hd, L->wo, d, y);
+        for (size_t i = 0; i < (size_t)R * d; ++i) h[i] += y[i];
+        for (int r = 0; r < R; ++r) oc_rmsnorm(h + (size_t)r * d, L->ffn_norm, d, c->rms_eps, a + (size_t)r * d);
+        oc_linear(a, R, d, L->w_gate, F, gt);
+        oc_linear(a, R, d, L->w_up, F, up);
+        for (size_t i = 0; i < (size_t)R * F; ++i) gt[i] = oc_silu(gt[i]) * up[i];
+        oc_linear(gt, R, F, L->w_down, d, y);
+        for (size_t i = 0; i < (size_t)R * d; ++i) h[i] += y[i];
+    }
+    for (int r = 0; r < R; ++r) oc_rmsnorm(h + (size_t)r * d, w->final_norm, d, c->rms_eps, a + (size_t)r * d);
+    if (final_hidden) memcpy(final_hidden, a, sizeof(double) * R * d);
+    if (logits) oc_linear(a, R, d, w->lm_head, V, logits);
+done:
+    free(h); free(a); free(q); free(k); free(v); free(o); free(y); free(gt); free(up);
+    return rc;
+}
+
+/* AR causal forward over prompt[0 .. P-2]; returns the committed length
+ * P-1 (paper notes §2.2: the AR view pre-fills the shared cache). */
+int oc_prefill(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P,
+               double *kc, double *vc, int cap)
+{
+    if (P < 1) return -OC_ERR_ARG;
+    if (P == 1) return 0;
+    int rc = oc_forward(c, w, 0, 0, prompt, P - 1, 0, kc, vc, cap, NULL, NULL);
+    return rc ? -rc : P - 1;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Randomness: Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11), written    */
+/* from the published round function.                                         */
+/* ------------------------------------------------------------------------ */
+
+void oc_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4])
+{
+    uint32_t x0 = ctr_in[0], x1 = ctr_in[1], x2 = ctr_in[2], x3 = ctr_in[3];
+    uint32_t k0 = key_in[0], k1 = key_in[1];
+    for (int round = 0; round < 10; ++round) {
+        uint64_t p0 = (uint64_t)0xD2511F53u * x0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * x2;
+        uint32_t y0 = (uint32_t)(p1 >> 32) ^ x1 ^ k0;
+        uint32_t y1 = (uint32_t)p1;
+        uint32_t y2 = (uint32_t)(p0 >> 32) ^ x3 ^ k1;
+        uint32_t y3 = (uint32_t)p0;
+        x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+/* Uniform in (0, 1): counter (id, row, step, purpose), key (seed lo, hi),
+ * first output word, top 24 bits, centred in its cell. */
+double oc_uniform(uint64_t seed, uint32_t step, uint32_t row, uint32_t id, uint32_t purpose)
+{
+    uint32_t ctr[4] = { id, row, step, purpose };
+    uint32_t key[2] = { (uint32_t)seed, (uint32_t)(seed >> 32) };
+    uint32_t out[4];
+    oc_philox4x32_10(ctr, key, out);
+    return ((double)(out[0] >> 8) + 0.5) * (1.0 / 16777216.0);
+}
+
+double oc_gumbel(uint64_t seed, uint32_t step, uint32_t row, uint32_t id, uint32_t purpose)
+{
+    return -log(-log(oc_uniform(seed, step, row, id, purpose)));
+}
+
+/* Lowest index of the maximum; *margin (if given) = best - second best. */
+int oc_argmax(const double *x, int n, double *margin)
+{
+    int best = 0;
+    double b = x[0], second = -INFINITY;
+    for (int i = 1; i < n; ++i) {
+        if (x[i] > b) { second = b; b = x[i]; best = i; }
+        else if (x[i] > second) second = x[i];
+    }
+    if (margin) *margin = b - second;
+    return best;
+}
+
+/* p = softmax(z / T) */
+void oc_softmax_t(const double *z, int n, double T, double *p)
+{
+    double m = -INFINITY;
+    for (int i = 0; i < n; ++i) if (z[i] / T > m) m = z[i] / T;
+    double s = 0.0;
+    for (int i = 0; i < n; ++i) { p[i] = exp(z[i] / T - m); s += p[i]; }
+    for (int i = 0; i < n; ++i) p[i] /= s;
+}
+
+/* Gumbel-max draw from softmax(z/T) (one uniform per id). */
+int oc_sample_logits(const double *z, int n, double T, uint64_t seed, uint32_t step,
+                     uint32_t row, uint32_t purpose, double *margin)
+{
+    int best = 0;
+    double b = -INFINITY, second = -INFINITY;
+    for (int i = 0; i < n; ++i) {
+        double s = z[i] / T + oc_gumbel(seed, step, row, (uint32_t)i, purpose);
+        if (s > b) { second = b; b = s; best = i; }
+        else if (s > second) second = s;
+    }
+    if (margin) *margin = b - second;
+    return best;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Consensus (paper notes §4.1 step 3, §4.2, §4.3).                           */
+/* ------------------------------------------------------------------------ */
+
+/* Greedy: accept y_k while it equals the AR argmax g_k; at the first
+ * mismatch j emit g_j.  Emitted tokens go to `emit`; returns n in [1, K]. */
+int oc_consensus_greedy(const int32_t *draft, const int32_t *g, int K, int32_t *emit)
+{
+    for (int k = 0; k < K; ++k) {
+        emit[k] = g[k];
+        if (draft[k] != g[k]) return k + 1;
+    }
+    return K;
+}
+
+/* Leviathan/Chen acceptance probability of a draft with target mass p and
+ * draft mass q. */
+double oc_accept_prob(double p, double q)
+{
+    if (q <= 0.0) return 1.0;
+    double a = p / q;
+    return a < 1.0 ? a : 1.0;
+}
+
+/* Residual distribution norm(max(0, p - q)).  Returns 0 and fills r when it
+ * has mass; returns 1 (r untouched) when p <= q everywhere. */
+int oc_residual(const double *p, const double *q, int n, double *r)
+{
+    double s = 0.0;
+    for (int i = 0; i < n; ++i) { double d = p[i] - q[i]; s += d > 0.0 ? d : 0.0; }
+    if (!(s > 0.0)) return 1;
+    for (int i = 0; i < n; ++i) { double d = p[i] - q[i]; r[i] = (d > 0.0 ? d : 0.0) / s; }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* The three stages of one cycle.                                             */
+/* ------------------------------------------------------------------------ */
+
+/* Parallel projection (§4.1 step 1): block [anchor, mask x (K-1)] at
+ * positions t .. t+K-1 through the diffusion view.  Writes the K drafts; at
+ * T>0 also q_probs [K][V] = softmax(w/T) when given.  logits [K][V] may be
+ * NULL. */
+int oc_draft(const oc_cfg *c, const oc_model *w, double *kc, double *vc, int cap, int t,
+             int32_t anchor, int K, double T, uint64_t seed, uint32_t step,
+             int32_t *draft, double *q_probs, double *logits, double *min_margin)
+{
+    int V = c->vocab;
+    int32_t *blk = malloc(sizeof(int32_t) * K);
+    double *z = malloc(sizeof(double) * (size_t)K * V);
+    if (!blk || !z) { free(blk); free(z); return OC_ERR_NOMEM; }
+    blk[0] = anchor;
+    for (int k = 1; k < K; ++k) blk[k] = c->mask_id;
+    int rc = oc_forward(c, w, 1, 1, blk, K, t, kc, vc, cap, z, NULL);
+    if (rc == OC_OK) {
+        for (int k = 0; k < K; ++k) {
+            const double *zk = z + (size_t)k * V;
+            double mg;
+            if (T > 0.0) {
+                draft[k] = oc_sample_logits(zk, V, T, seed, step, (uint32_t)k, OC_PURPOSE_DRAFT, &mg);
+                if (q_probs) oc_softmax_t(zk, V, T, q_probs + (size_t)k * V);
+            } else {
+                draft[k] = oc_argmax(zk, V, &mg);
+            }
+            if (min_margin && mg < *min_margin) *min_margin = mg;
+        }
+        if (logits) memcpy(logits, z, sizeof(double) * (size_t)K * V);
+    }
+    free(blk); free(z);
+    return rc;
+}
+
+/* AR verification (§4.1 step 2): block [anchor, y_1 .. y_{K-1}] through the
+ * AR view, K/V written at t .. t+K-1.  Writes g [K] (argmax per row) and, at
+ * T>0, p_probs [K][V] = softmax(z/T).  logits may be NULL. */
+int oc_verify(const oc_cfg *c, const oc_model *w, double *kc, double *vc, int cap, int t,
+              int32_t anchor, const int32_t *draft, int K, double T,
+              int32_t *g, double *p_probs, double *logits, double *min_margin)
+{
+    int V = c->vocab;
+    int32_t *blk = malloc(sizeof(int32_t) * K);
+    double *z = malloc(sizeof(double) * (size_t)K * V);
+    if (!blk || !z) { free(blk); free(z); return OC_ERR_NOMEM; }
+    blk[0] = anchor;
+    for (int k = 1; k < K; ++k) blk[k] = draft[k - 1];
+    int rc = oc_forward(c, w, 0, 0, blk, K, t, kc, vc, cap, z, NULL);
+    if (rc == OC_OK) {
+        for (int k = 0; k < K; ++k) {
+            double mg;
+            g[k] = oc_argmax(z + (size_t)k * V, V, &mg);
+            if (T > 0.0 && p_probs) oc_softmax_t(z + (size_t)k * V, V, T, p_probs + (size_t)k * V);
+            if (min_margin && T <= 0.0 && mg < *min_margin) *min_margin = mg;
+        }
+        if (logits) memcpy(logits, z, sizeof(double) * (size_t)K * V);
+    }
+    free(blk); free(z);
+    return rc;
+}
+
+/* Consensus at T>0 (§4.3): accept y_k with probability min(1, p_k/q_k) using
+ * u_k; at the first rejection j draw the correction from norm(max(0, p_j -
+ * q_j)).  Returns n and fills emit. */
+int oc_consensus_sample(const double *p, const double *q, const int32_t *draft, const int32_t *g,
+                        int K, int V, uint64_t seed, uint32_t step, int32_t *emit,
+                        double *min_margin)
+{
+    double *r = malloc(sizeof(double) * V);
+    double *lr = malloc(sizeof(double) * V);
+    int n = K;
+    for (int k = 0; k < K; ++k) {
+        const double *pk = p + (size_t)k * V, *qk = q + (size_t)k * V;
+        double a = oc_accept_prob(pk[draft[k]], qk[draft[k]]);
+        double u = oc_uniform(seed, step, (uint32_t)k, 0, OC_PURPOSE_ACCEPT);
+        if (min_margin && fabs(u - a) < *min_margin) *min_margin = fabs(u - a);
+        if (u < a) { emit[k] = draft[k]; continue; }
+        if (oc_residual(pk, qk, V, r) == 0) {
+            for (int i = 0; i < V; ++i) lr[i] = r[i] > 0.0 ? log(r[i]) : -INFINITY;
+            double mg;
+            emit[k] = oc_sample_logits(lr, V, 1.0, seed, step, (uint32_t)k, OC_PURPOSE_RESIDUAL, &mg);
+        } else {
+            emit[k] = g[k];
+        }
+        n = k + 1;
+        break;
+    }
+    free(r); free(lr);
+    return n;
+}
+
+/*
+ * Whole decode from a prompt.  method 0 = plain AR (one AR forward per
+ * token), method 1 = Orthrus (draft, verify, consensus, commit per cycle).
+ * Stops once N tokens are out; out[N].  n_per_cycle (may be NULL) receives
+ * the tokens emitted by each cycle and *n_cycles their count.  *min_margin
+ * (may be NULL) receives the smallest argmax / acceptance decision margin
+ * seen, so callers can tell a decision that fp32 rounding could flip.
+ * kc_out / vc_out (may be NULL) receive the final committed cache
+ * [n_layers][cap][n_kv][hd], cap = P + N + K, rows beyond the committed length
+ * zeroed.  *t_out (may be NULL) receives the final committed length.
+ */
+int oc_generate(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P, int K, int N,
+                double T, uint64_t seed, int method, int32_t *out, int32_t *n_per_cycle,
+                int *n_cycles, double *min_margin, double *kc_out, double *vc_out, int *t_out)
+{
+    if (!c || !w || !prompt || P < 1 || N < 1 || K < 1 || (method != 0 && method != 1)) return OC_ERR_ARG;
+    const int V = c->vocab;
+    const int cap = P + N + K;
+    const size_t kn = (size_t)c->n_kv_heads * c->head_dim;
+    const size_t csz = (size_t)c->n_layers * cap * kn;
+    double *kc = calloc(csz, sizeof(double)), *vc = calloc(csz, sizeof(double));
+    int32_t *draft = malloc(sizeof(int32_t) * K), *g = malloc(sizeof(int32_t) * K);
+    int32_t *emit = malloc(sizeof(int32_t) * K);
+    double *p = NULL, *q = NULL, *z = malloc(sizeof(double) * V);
+    if (T > 0.0) { p = malloc(sizeof(double) * (size_t)K * V); q = malloc(sizeof(double) * (size_t)K * V); }
+    int rc = OC_OK;
+    if (!kc || !vc || !draft || !g || !emit || !z || (T > 0.0 && (!p || !q))) { rc = OC_ERR_NOMEM; goto done; }
+    if (min_margin) *min_margin = INFINITY;
+
+    int t = oc_prefill(c, w, prompt, P, kc, vc, cap);
+    if (t < 0) { rc = -t; goto done; }
+    int32_t anchor = prompt[P - 1];
+    int produced = 0, cycles = 0;
+    while (produced < N) {
+        int n;
+        if (method == 0) {
+            rc = oc_forward(c, w, 0, 0, &anchor, 1, t, kc, vc, cap, z, NULL);
+            if (rc) goto done;
+            double mg;
+            emit[0] = (T > 0.0) ? oc_sample_logits(z, V, T, seed, (uint32_t)produced, 0, OC_PURPOSE_AR, &mg)
+                                : oc_argmax(z, V, &mg);
+            if (min_margin && mg < *min_margin) *min_margin = mg;
+            n = 1;
+        } else {
+            rc = oc_draft(c, w, kc, vc, cap, t, anchor, K, T, seed, (uint32_t)cycles, draft, q, NULL, min_margin);
+            if (rc) goto done;
+            rc = oc_verify(c, w, kc, vc, cap, t, anchor, draft, K, T, g, p, NULL, min_margin);
+            if (rc) goto done;
+            n = (T > 0.0) ? oc_consensus_sample(p, q, draft, g, K, V, seed, (uint32_t)cycles, emit, min_margin)
+                          : oc_consensus_greedy(draft, g, K, emit);
+        }
+        /* commit (§4.1 step 3): keep cache rows t .. t+n-1 (already written by
+         * the AR forward for the accepted inputs), discard the rest. */
+        t += n;
+        anchor = emit[n - 1];
+        for (int i = 0; i < n && produced < N; ++i) out[produced++] = emit[i];
+        if (n_per_cycle) n_per_cycle[cycles] = n;
+        ++cycles;
+    }
+    if (n_cycles) *n_cycles = cycles;
+    if (t_out) *t_out = t;
+    if (kc_out || vc_out) {
+        for (int l = 0; l < c->n_layers; ++l) {
+            double *kl = kc + (size_t)l * cap * kn, *vl = vc + (size_t)l * cap * kn;
+            memset(kl + (size_t)t * kn, 0, sizeof(double) * (size_t)(cap - t) * kn);
+            memset(vl + (size_t)t * kn, 0, sizeof(double) * (size_t)(cap - t) * kn);
+        }
+        if (kc_out) memcpy(kc_out, kc, sizeof(double) * csz);
+        if (vc_out) memcpy(vc_out, vc, sizeof(double) * csz);
+    }
+done:
+    free(kc); free(vc); free(draft); free(g); free(emit); free(p); free(q); free(z);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Exact laws for the losslessness pin (paper notes §4.3, §9.1).              */
+/* ------------------------------------------------------------------------ */
+
+static long ipow(int b, int e) { long r = 1; while (e-- > 0) r *= b; return r; }
+
+/* Next-token distribution p_AR(. | seq[0 .. len-1]) at temperature T:
+ * prefill seq[0 .. len-2], then one AR row for seq[len-1]. */
+static int ar_next(const oc_cfg *c, const oc_model *w, const int32_t *seq, int len, double T, double *p)
+{
+    int cap = len;
+    size_t csz = (size_t)c->n_layers * cap * c->n_kv_heads * c->head_dim;
+    double *kc = calloc(csz, sizeof(double)), *vc = calloc(csz, sizeof(double));
+    double *z = malloc(sizeof(double) * c->vocab);
+    int rc = (!kc || !vc || !z) ? OC_ERR_NOMEM : OC_OK;
+    if (rc == OC_OK && len > 1) rc = oc_forward(c, w, 0, 0, seq, len - 1, 0, kc, vc, cap, NULL, NULL);
+    if (rc == OC_OK) rc = oc_forward(c, w, 0, 0, seq + len - 1, 1, len - 1, kc, vc, cap, z, NULL);
+    if (rc == OC_OK) oc_softmax_t(z, c->vocab, T, p);
+    free(kc); free(vc); free(z);
+    return rc;
+}
+
+/* dist[V^N]: probability of each first-N token string under plain AR
+ * sampling at temperature T after the prompt. */
+int oc_enumerate_ar(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P, int N,
+                    double T, double *dist)
+{
+    const int V = c->vocab;
+    long total = ipow(V, N);
+    int32_t *seq = malloc(sizeof(int32_t) * (P + N));
+    double *p = malloc(sizeof(double) * V);
+    double *mass = malloc(sizeof(double) * (size_t)total);   /* mass of each prefix, level by level */
+    double *next = malloc(sizeof(double) * (size_t)total);
+    if (!seq || !p || !mass || !next) { free(seq); free(p); free(mass); free(next); return OC_ERR_NOMEM; }
+    memcpy(seq, prompt, sizeof(int32_t) * P);
+    mass[0] = 1.0;
+    int rc = OC_OK;
+    for (int e = 0; e < N && rc == OC_OK; ++e) {
+        long cnt = ipow(V, e);
+        for (long idx = 0; idx < cnt; ++idx) {
+            long rem = idx;
+            for (int i = e - 1; i >= 0; --i) { seq[P + i] = (int32_t)(rem % V); rem /= V; }
+            rc = ar_next(c, w, seq, P + e, T, p);
+            if (rc) break;
+            for (int v = 0; v < V; ++v) next[idx * V + v] = mass[idx] * p[v];
+        }
+        memcpy(mass, next, sizeof(double) * (size_t)cnt * V);
+    }
+    if (rc == OC_OK) memcpy(dist, mass, sizeof(double) * (size_t)total);
+    free(seq); free(p); free(mass); free(next);
+    return rc;
+}
+
+/*
+ * dist[V^N]: exact probability of each first-N token string produced by the
+ * Orthrus cycle at temperature T > 0, under ideal randomness: drafts y_k drawn
+ * independently from q_k (one diffusion forward), acceptance with
+ * oc_accept_prob, correction from oc_residual (or argmax p when it has no
+ * mass).  The draft and verify distributions come from oc_draft /
+ * oc_verify-equivalent forwards.  planted_error = 1 replaces the residual by
+ * p itself (a known mistake that must break losslessness).
+ */
+int oc_enumerate_orthrus(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P, int K,
+                         int N, double T, int planted_error, double *dist)
+{
+    const int V = c->vocab;
+    const long total = ipow(V, N);
+    long ntuple = ipow(V, K);
+    int rc = OC_OK;
+    /* mass of states by number of emitted tokens e (< N), dense over V^e */
+    double **lvl = calloc(N, sizeof(double *));
+    int32_t *seq = malloc(sizeof(int32_t) * (P + N + K));
+    int32_t *blk = malloc(sizeof(int32_t) * K);
+    int32_t *y = malloc(sizeof(int32_t) * K);
+    double *qz = malloc(sizeof(double) * (size_t)K * V), *q = malloc(sizeof(double) * (size_t)K * V);
+    double *pz = malloc(sizeof(double) * (size_t)K * V), *p = malloc(sizeof(double) * (size_t)K * V);
+    double *r = malloc(sizeof(double) * V);
+    if (!lvl || !seq || !blk || !y || !qz || !q || !pz || !p || !r) { rc = OC_ERR_NOMEM; goto out; }
+    for (int e = 0; e < N; ++e) {
+        lvl[e] = calloc((size_t)ipow(V, e), sizeof(double));
+        if (!lvl[e]) { rc = OC_ERR_NOMEM; goto out; }
+    }
+    memset(dist, 0, sizeof(double) * (size_t)total);
+    memcpy(seq, prompt, sizeof(int32_t) * P);
+    lvl[0][0] = 1.0;
+    const int cap = P + N + K;
+    const size_t csz = (size_t)c->n_layers * cap * c->n_kv_heads * c->head_dim;
+    double *kc = calloc(csz, sizeof(double)), *vc = calloc(csz, sizeof(double));
+    if (!kc || !vc) { free(kc); free(vc); rc = OC_ERR_NOMEM; goto out; }
+
+    for (int e = 0; e < N && rc == OC_OK; ++e) {
+        long cnt = ipow(V, e);
+        for (long idx = 0; idx < cnt && rc == OC_OK; ++idx) {
+            double wstate = lvl[e][idx];
+            if (wstate == 0.0) continue;
+            long rem = idx;
+            for (int i = e - 1; i >= 0; --i) { seq[P + i] = (int32_t)(rem % V); rem /= V; }
+            int len = P + e;                         /* tokens known so far */
+            int t = len - 1;                         /* committed cache length */
+            int32_t anchor = seq[len - 1];
+            if (t > 0) rc = oc_forward(c, w, 0, 0, seq, t, 0, kc, vc, cap, NULL, NULL);
+            if (rc) break;
+            blk[0] = anchor;
+            for (int k = 1; k < K; ++k) blk[k] = c->mask_id;
+            rc = oc_forward(c, w, 1, 1, blk, K, t, kc, vc, cap, qz, NULL);
+            if (rc) break;
+            for (int k = 0; k < K; ++k) oc_softmax_t(qz + (size_t)k * V, V, T, q + (size_t)k * V);
+            long prev_ctx = -1;
+            for (long tup = 0; tup < ntuple && rc == OC_OK; ++tup) {
+                long rr = tup;
+                for (int k = K - 1; k >= 0; --k) { y[k] = (int32_t)(rr % V); rr /= V; }
+                double wq = 1.0;
+                for (int k = 0; k < K; ++k) wq *= q[(size_t)k * V + y[k]];
+                if (wq == 0.0) continue;
+                long ctx = tup / V;                  /* verify depends on y_1..y_{K-1} only */
+                if (ctx != prev_ctx) {
+                    blk[0] = anchor;
+                    for (int k = 1; k < K; ++k) blk[k] = y[k - 1];
+                    rc = oc_forward(c, w, 0, 0, blk, K, t, kc, vc, cap, pz, NULL);
+                    if (rc) break;
+                    for (int k = 0; k < K; ++k) oc_softmax_t(pz + (size_t)k * V, V, T, p + (size_t)k * V);
+                    prev_ctx = ctx;
+                }
+                double acc = 1.0;
+                int j;
+                for (j = 0; j < K; ++j) {
+                    const double *pj = p + (size_t)j * V, *qj = q + (size_t)j * V;
+                    double a = oc_accept_prob(pj[y[j]], qj[y[j]]);
+                    double rej = acc * (1.0 - a);
+                    if (rej > 0.0) {
+                        int none;
+                        if (planted_error) { memcpy(r, pj, sizeof(double) * V); none = 0; }
+                        else none = oc_residual(pj, qj, V, r);
+                        for (int cc = 0; cc < V; ++cc) {
+                            double pr = none ? (cc == oc_argmax(pj, V, NULL) ? 1.0 : 0.0) : r[cc];
+                            if (pr == 0.0) continue;
+                            /* emitted: y_0..y_{j-1}, cc  (j+1 tokens) */
+                            long ne = e + j + 1, nidx = idx;
+                            double m = wstate * wq * rej * pr;
+                            int lim = ne < N ? (int)ne : N;
+                            for (int i = e; i < lim; ++i) nidx = nidx * V + (i - e < j ? y[i - e] : cc);
+                            if (ne >= N) dist[nidx] += m; else lvl[ne][nidx] += m;
+                        }
+                    }
+                    acc *= a;
+                    if (acc == 0.0) break;
+                }
+                if (j == K && acc > 0.0) {
+                    long ne = e + K, nidx = idx;
+                    int lim = ne < N ? (int)ne : N;
+                    for (int i = e; i < lim; ++i) nidx = nidx * V + y[i - e];
+                    if (ne >= N) dist[nidx] += wstate * wq * acc; else lvl[ne][nidx] += wstate * wq * acc;
+                }
+            }
+        }
+    }
+    free(kc); free(vc);
+out:
+    if (lvl) for (int e = 0; e < N; ++e) free(lvl[e]);
+    free(lvl); free(seq); free(blk); free(y); free(qz); free(q); free(pz); free(p); free(r);
+    return rc;
+}

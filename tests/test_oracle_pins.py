@@ -1,0 +1,310 @@
+"""Pins of the CPU oracle against things other than itself: closed forms,
+invariants, library routines (torch, a HuggingFace Llama model), published
+known-answer vectors and exact enumeration of the sampled decode.
+
+Passages restated by the oracle: the paper-notes page on "Orthrus:
+Memory-Efficient Parallel Token Generation via Dual-View Diffusion", §2.1
+(dual-view layer), §3.2 (diffusion mask), §4.1-§4.3 (cycle, greedy and
+sampled consensus), §5.1 (TPF bounds), §9.1 (losslessness).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ------------------------------------------------------------------ RNG
+def test_philox_known_answers():
+    path = os.path.join(GOLDEN, "philox4x32_10_kat.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    assert len(rows) == 3
+    for r in rows:
+        v = [int(x, 16) for x in r]
+        assert oracle.philox4x32_10(v[0:4], v[4:6]) == v[6:10]
+
+
+def test_uniform_range_and_moments():
+    u = np.array([oracle.uniform(7, 3, r, i, oracle.PURPOSE_DRAFT) for r in range(4) for i in range(5000)])
+    assert (u > 0).all() and (u < 1).all()
+    assert abs(u.mean() - 0.5) < 0.01 and abs(u.var() - 1 / 12) < 0.005
+    # streams of different purposes / rows are different numbers
+    a = oracle.uniform(7, 3, 0, 0, oracle.PURPOSE_DRAFT)
+    assert a != oracle.uniform(7, 3, 0, 0, oracle.PURPOSE_ACCEPT)
+    assert a != oracle.uniform(7, 3, 1, 0, oracle.PURPOSE_DRAFT)
+    assert a != oracle.uniform(8, 3, 0, 0, oracle.PURPOSE_DRAFT)
+
+
+def test_gumbel_max_samples_softmax():
+    # Gumbel-max over one uniform per id is an exact sampler of softmax(z/T):
+    # chi-square over 20000 draws.
+    z = np.array([0.3, -1.0, 1.2, 0.0, 0.7, -0.4])
+    T = 0.8
+    p = np.exp(z / T - np.max(z / T)); p /= p.sum()
+    n = 20000
+    cnt = np.zeros(len(z))
+    for s in range(n):
+        i, _ = oracle.sample_logits(z, T, 11, s, 2, oracle.PURPOSE_DRAFT)
+        cnt[i] += 1
+    chi2 = ((cnt - n * p) ** 2 / (n * p)).sum()
+    assert chi2 < 25.0          # 5 dof: p-value ~1e-4
+
+
+# ------------------------------------------------------------------ blocks
+def test_rmsnorm_closed_form_and_torch():
+    for c in (0.5, -3.0, 1e-4):
+        y = oracle.rmsnorm(np.full(64, c), np.ones(64, np.float32), 1e-6)
+        assert np.allclose(y, math.copysign(1.0, c) / math.sqrt(1 + 1e-6 / c ** 2), rtol=1e-14, atol=0)
+    x = np.random.default_rng(0).standard_normal(64)
+    g = np.random.default_rng(1).standard_normal(64).astype(np.float32)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (64,), torch.from_numpy(g.astype(np.float64)), 1e-6)
+    assert np.allclose(oracle.rmsnorm(x, g, 1e-6), ref.numpy(), rtol=1e-13, atol=1e-15)
+
+
+def test_silu():
+    assert oracle.silu(0.0) == 0.0
+    for g in (-5.0, -0.3, 0.9, 4.0):
+        assert abs(oracle.silu(g) - torch.nn.functional.silu(torch.tensor(g, dtype=torch.float64)).item()) < 1e-15
+
+
+def test_rope_identity_norm_relative():
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((2, 16)); k = rng.standard_normal((2, 16))
+    assert np.array_equal(oracle.rope(q, 0), q)
+    for pos in (1, 7, 1000, 131071):
+        assert np.allclose(np.linalg.norm(oracle.rope(q, pos), axis=1), np.linalg.norm(q, axis=1), rtol=1e-13)
+    # q.k after RoPE depends only on the position difference
+    d1 = (oracle.rope(q, 10) * oracle.rope(k, 3)).sum(1)
+    d2 = (oracle.rope(q, 107) * oracle.rope(k, 100)).sum(1)
+    assert np.allclose(d1, d2, rtol=1e-11)
+    # a wrong pairing (adjacent instead of rotate-half) would break this:
+    # pair (0, 8) rotates by pos * theta^0 = pos radians
+    e = np.zeros((1, 16)); e[0, 0] = 1.0
+    r = oracle.rope(e, 2)
+    assert abs(r[0, 0] - math.cos(2)) < 1e-15 and abs(r[0, 8] - math.sin(2)) < 1e-15
+
+
+def _sdpa_reference(q, kc, vc, kb, vb, mode):
+    """torch scaled_dot_product_attention (library) with an explicit mask."""
+    R, nq, hd = q.shape
+    nkv = kb.shape[1]
+    keys = np.concatenate([kc, kb]) if kc is not None else kb
+    vals = np.concatenate([vc, vb]) if vc is not None else vb
+    t = 0 if kc is None else kc.shape[0]
+    g = nq // nkv
+    K = torch.from_numpy(np.repeat(keys, g, axis=1)).permute(1, 0, 2)
+    Vv = torch.from_numpy(np.repeat(vals, g, axis=1)).permute(1, 0, 2)
+    Q = torch.from_numpy(q).permute(1, 0, 2)
+    mask = torch.ones(R, t + R, dtype=torch.bool)
+    if mode == 0:
+        mask[:, t:] = torch.tril(torch.ones(R, R, dtype=torch.bool))
+    o = torch.nn.functional.scaled_dot_product_attention(Q, K, Vv, attn_mask=mask)
+    return o.permute(1, 0, 2).numpy()
+
+
+@pytest.mark.parametrize("t,R,mode", [(0, 1, 0), (0, 5, 1), (37, 4, 0), (37, 4, 1), (130, 8, 0), (130, 8, 1)])
+def test_attention_matches_torch_sdpa(t, R, mode):
+    rng = np.random.default_rng(t * 10 + R + mode)
+    nq, nkv, hd = 8, 2, 16
+    q = rng.standard_normal((R, nq, hd))
+    kc = rng.standard_normal((t, nkv, hd)) if t else None
+    vc = rng.standard_normal((t, nkv, hd)) if t else None
+    kb = rng.standard_normal((R, nkv, hd)); vb = rng.standard_normal((R, nkv, hd))
+    o = oracle.attention(q, kc, vc, kb, vb, mode)
+    assert np.allclose(o, _sdpa_reference(q, kc, vc, kb, vb, mode), rtol=1e-12, atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((1, 4, 8)); kb = rng.standard_normal((1, 2, 8)); vb = rng.standard_normal((1, 2, 8))
+    # one key: the output is that key's value row for every head of its group
+    o = oracle.attention(q, None, None, kb, vb, 0)
+    assert np.allclose(o[0, :2], vb[0, 0]) and np.allclose(o[0, 2:], vb[0, 1])
+    # identical keys: the output is the mean of the values
+    kc = np.repeat(kb, 9, axis=0); vc = rng.standard_normal((9, 2, 8))
+    o = oracle.attention(q, kc, vc, kb, vb, 0)
+    mean = np.concatenate([vc, vb]).mean(0)
+    assert np.allclose(o[0, :2], mean[0], rtol=1e-12) and np.allclose(o[0, 2:], mean[1], rtol=1e-12)
+    # with a one-row block the two masks coincide
+    o0 = oracle.attention(q, kc, vc, kb, vb, 0); o1 = oracle.attention(q, kc, vc, kb, vb, 1)
+    assert np.array_equal(o0, o1)
+
+
+# ------------------------------------------------------------------ model
+def _hf_llama(w):
+    from transformers import LlamaConfig, LlamaForCausalLM
+    s = w.shape
+    cfg = LlamaConfig(vocab_size=s.vocab, hidden_size=s.hidden, intermediate_size=s.ffn,
+                      num_hidden_layers=len(w.layers), num_attention_heads=s.n_q_heads,
+                      num_key_value_heads=s.n_kv_heads, head_dim=s.head_dim, rms_norm_eps=s.rms_eps,
+                      rope_theta=s.rope_theta, attention_bias=False, mlp_bias=False,
+                      tie_word_embeddings=False, max_position_embeddings=4096)
+    cfg._attn_implementation = "eager"
+    m = LlamaForCausalLM(cfg).double().eval()
+    T = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    with torch.no_grad():
+        m.model.embed_tokens.weight.copy_(T(w.embed)); m.lm_head.weight.copy_(T(w.lm_head))
+        m.model.norm.weight.copy_(T(w.final_norm))
+        for l, lw in enumerate(w.layers):
+            L = m.model.layers[l]
+            L.input_layernorm.weight.copy_(T(lw["attn_norm"])); L.post_attention_layernorm.weight.copy_(T(lw["ffn_norm"]))
+            L.self_attn.q_proj.weight.copy_(T(lw["wq"])); L.self_attn.k_proj.weight.copy_(T(lw["wk"]))
+            L.self_attn.v_proj.weight.copy_(T(lw["wv"])); L.self_attn.o_proj.weight.copy_(T(lw["wo"]))
+            L.mlp.gate_proj.weight.copy_(T(lw["w_gate"])); L.mlp.up_proj.weight.copy_(T(lw["w_up"]))
+            L.mlp.down_proj.weight.copy_(T(lw["w_down"]))
+    return m
+
+
+def test_ar_forward_matches_hf_llama():
+    """The AR view is a plain pre-norm Llama-style decoder: its prefill logits
+    equal those of the HuggingFace Llama model given the same weights (HF
+    builds its RoPE table in fp32, hence the 1e-6 tolerance; a dropped term or
+    wrong index gives errors of order 0.1)."""
+    w = synth.make_weights(synth.TINY, 0, random_gains=True)
+    pr = synth.make_prompt(synth.TINY, 40, 0)
+    hf = _hf_llama(w)
+    with torch.no_grad():
+        ref = hf(torch.from_numpy(pr.astype(np.int64))[None]).logits[0].numpy()
+    m = oracle.Model(w)
+    kc, vc = m.new_cache(64)
+    z = m.forward(0, 0, pr, 0, kc, vc)
+    assert np.abs(z - ref).max() < 1e-6 * max(1.0, np.abs(ref).max())
+
+
+def test_block_rows_equal_single_rows(tiny_weights, tiny_prompt):
+    """Row k of a causal block equals the same row run alone after the rows
+    before it were committed (bitwise: rows are computed independently)."""
+    m = oracle.Model(tiny_weights)
+    kc, vc = m.new_cache(64)
+    t = m.prefill(tiny_prompt, kc, vc)
+    blk = np.array([tiny_prompt[-1], 3, 77, 200, 9], np.int32)
+    z_blk = m.forward(0, 0, blk, t, kc.copy(), vc.copy())
+    kc2, vc2 = kc.copy(), vc.copy()
+    for k, tok in enumerate(blk):
+        z1 = m.forward(0, 0, [tok], t + k, kc2, vc2)
+        assert np.array_equal(z1[0], z_blk[k])
+
+
+def test_views_differ_only_by_qkv(tiny_weights, tiny_prompt):
+    """Diffusion weights equal to the AR ones make the two views the same
+    function when the masks coincide (one-row block)."""
+    w = synth.make_weights(synth.TINY, 0, diff_equals_ar=True)
+    m = oracle.Model(w)
+    kc, vc = m.new_cache(64)
+    t = m.prefill(tiny_prompt, kc, vc)
+    a = m.forward(0, 0, [tiny_prompt[-1]], t, kc.copy(), vc.copy())
+    b = m.forward(1, 1, [tiny_prompt[-1]], t, kc.copy(), vc.copy())
+    assert np.array_equal(a, b)
+    # and with the real (perturbed) diffusion weights they differ
+    m2 = oracle.Model(tiny_weights)
+    c = m2.forward(1, 1, [tiny_prompt[-1]], t, kc.copy(), vc.copy())
+    assert not np.array_equal(a, c)
+
+
+def test_draft_does_not_touch_cache(tiny_weights, tiny_prompt):
+    """Diffusion K/V are transient: a draft leaves the cache bit-identical."""
+    m = oracle.Model(tiny_weights)
+    kc, vc = m.new_cache(64)
+    t = m.prefill(tiny_prompt, kc, vc)
+    k0, v0 = kc.copy(), vc.copy()
+    m.draft(kc, vc, t, tiny_prompt[-1], 4)
+    assert np.array_equal(kc, k0) and np.array_equal(vc, v0)
+
+
+# ------------------------------------------------------------------ consensus
+def test_consensus_greedy_examples():
+    n, e = oracle.consensus_greedy([5, 6, 7, 8], [5, 6, 9, 1])
+    assert n == 3 and list(e) == [5, 6, 9]
+    n, e = oracle.consensus_greedy([5, 6, 7, 8], [5, 6, 7, 8])
+    assert n == 4 and list(e) == [5, 6, 7, 8]
+    n, e = oracle.consensus_greedy([4, 6], [5, 6])
+    assert n == 1 and list(e) == [5]
+
+
+def test_accept_and_residual():
+    assert oracle.accept_prob(0.2, 0.4) == 0.5 and oracle.accept_prob(0.4, 0.2) == 1.0
+    p = np.array([0.5, 0.3, 0.2]); q = np.array([0.2, 0.5, 0.3])
+    assert np.allclose(oracle.residual(p, q), [1.0, 0.0, 0.0])
+    assert oracle.residual(p, p) is None
+    # the identity behind losslessness: q*min(1,p/q) + (1-beta)*r == p
+    q = np.array([0.1, 0.6, 0.3]); p = np.array([0.3, 0.3, 0.4])
+    beta = sum(q[i] * oracle.accept_prob(p[i], q[i]) for i in range(3))
+    r = oracle.residual(p, q)
+    assert np.allclose([q[i] * oracle.accept_prob(p[i], q[i]) + (1 - beta) * r[i] for i in range(3)], p, atol=1e-15)
+
+
+@pytest.mark.parametrize("K", [1, 2, 4, 8])
+def test_greedy_orthrus_equals_ar(tiny_weights, tiny_prompt, K):
+    """Paper notes §4.2/§9.1: greedy Orthrus emits exactly the AR greedy
+    stream; every cycle is 2 forwards and emits 1..K tokens (§4.1, §5.1)."""
+    m = oracle.Model(tiny_weights)
+    a = m.generate(tiny_prompt, K, 32, 0.0, 0, "ar", want_cache=True)
+    o = m.generate(tiny_prompt, K, 32, 0.0, 0, "orthrus", want_cache=True)
+    assert np.array_equal(a["tokens"], o["tokens"])
+    n = o["n_per_cycle"]
+    assert (n >= 1).all() and (n <= K).all()
+    tpf = n.sum() / (2 * len(n))
+    assert 0.5 <= tpf <= K / 2
+    # the committed AR K/V are bit-identical to plain AR's
+    t = min(a["t"], o["t"])
+    assert np.array_equal(a["k_cache"][:, :t], o["k_cache"][:, :t])
+    assert np.array_equal(a["v_cache"][:, :t], o["v_cache"][:, :t])
+
+
+def test_k1_with_shared_weights_always_accepts(tiny_prompt):
+    w = synth.make_weights(synth.TINY, 0, diff_equals_ar=True)
+    m = oracle.Model(w)
+    o = m.generate(tiny_prompt, 1, 12, 0.0, 0, "orthrus")
+    assert (o["n_per_cycle"] == 1).all()
+    kc, vc = m.new_cache(64)
+    t = m.prefill(tiny_prompt, kc, vc)
+    d, _, _, _ = m.draft(kc, vc, t, tiny_prompt[-1], 1)
+    g, _, _, _ = m.verify(kc, vc, t, tiny_prompt[-1], d)
+    assert d[0] == g[0]
+
+
+@pytest.mark.parametrize("T", [1.0, 0.7])
+def test_sampled_orthrus_is_lossless_by_enumeration(T):
+    """Paper notes §4.3/§9.1: at T>0 the output law equals the AR law.  Exact
+    enumeration over every draft tuple and accept/reject branch on a micro
+    model (V=8, K=3, first 4 tokens): total variation below 1e-9; planting the
+    classic mistake (residual = p instead of norm(max(0, p - q))) breaks it."""
+    w = synth.make_weights(synth.MICRO, 0)
+    m = oracle.Model(w)
+    pr = synth.make_prompt(synth.MICRO, 3, 0)
+    pa = m.enumerate_ar(pr, 4, T)
+    po = m.enumerate_orthrus(pr, 3, 4, T)
+    assert abs(pa.sum() - 1) < 1e-12 and abs(po.sum() - 1) < 1e-12
+    assert 0.5 * np.abs(pa - po).sum() < 1e-9
+    pb = m.enumerate_orthrus(pr, 3, 4, T, planted_error=True)
+    assert 0.5 * np.abs(pa - pb).sum() > 1e-3
+    # a one-token block is lossless too (it reduces to one draft and one check)
+    assert 0.5 * np.abs(pa - m.enumerate_orthrus(pr, 1, 4, T)).sum() < 1e-9
+
+
+def test_sampler_matches_ar_law_monte_carlo():
+    """The oracle's real sampled decode (Philox uniforms, Gumbel drafts,
+    acceptance test, residual draw) against the exact AR law of the first two
+    tokens: chi-square over 6000 seeds on the micro model."""
+    w = synth.make_weights(synth.MICRO, 0)
+    m = oracle.Model(w)
+    pr = synth.make_prompt(synth.MICRO, 3, 0)
+    pa = m.enumerate_ar(pr, 2, 1.0)
+    n = 6000
+    cnt = np.zeros(64)
+    for s in range(n):
+        o = m.generate(pr, 3, 2, 1.0, s + 1, "orthrus")
+        cnt[o["tokens"][0] * 8 + o["tokens"][1]] += 1
+    e = n * pa
+    keep = e >= 5
+    chi2 = (((cnt - e) ** 2 / e)[keep]).sum() + ((cnt[~keep].sum() - e[~keep].sum()) ** 2 / max(e[~keep].sum(), 1e-9))
+    dof = keep.sum()
+    # p-value ~1e-4 threshold via Wilson-Hilferty
+    z = ((chi2 / dof) ** (1 / 3) - (1 - 2 / (9 * dof))) / math.sqrt(2 / (9 * dof))
+    assert z < 3.7, (chi2, dof)
