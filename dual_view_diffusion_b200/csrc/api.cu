@@ -1,0 +1,543 @@
+// C ABI of the dual-view decode library (declared in include/orthrus.h).
+//
+// Host orchestration only: argument checks, the workspace carve-up, and the
+// order of kernel launches for prefill, the draft forward (diffusion view),
+// the verify forward (AR view), consensus/commit and plain AR decoding
+// ("Orthrus: Memory-Efficient Parallel Token Generation via Dual-View
+// Diffusion", paper notes §2.1-§2.3 and §4.1-§4.3).  Every step of the
+// arithmetic runs in the kernels.
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <new>
+#include <type_traits>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+struct orthrus_ctx : orthrus::Ctx {};
+
+namespace orthrus {
+
+cudaError_t launch_set_int(int32_t *p, int v, cudaStream_t s);
+cudaError_t launch_lm_finalize_impl(const Ctx &c, int mode, int B, int K, float temperature, int32_t *tok_out,
+                                    const int32_t *given, cudaStream_t s);
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static bool valid_config(const orthrus_config_t &c)
+{
+    if (c.n_layers < 1 || c.hidden < 1 || c.n_q_heads < 1 || c.n_kv_heads < 1 || c.ffn < 1 || c.vocab < 2)
+        return false;
+    if (c.n_q_heads % c.n_kv_heads) return false;
+    if (c.head_dim != 16 && c.head_dim != 32 && c.head_dim != 64 && c.head_dim != 128) return false;
+    if (c.mask_token_id < 0 || c.mask_token_id >= c.vocab) return false;
+    if (c.dtype != ORTHRUS_BF16 && c.dtype != ORTHRUS_FP32) return false;
+    if (c.max_batch < 1 || c.max_batch > 128 || c.max_block < 1 || c.max_block > 4096) return false;
+    if (c.split_tokens < 64 || c.split_tokens % 64) return false;
+    if (c.max_seq < c.max_block + 1) return false;
+    if (!(c.rope_theta > 0.f) || !(c.rms_eps > 0.f)) return false;
+    return true;
+}
+
+// Largest split-partial buffer and ticket count any projection of this
+// model needs with up to `rows` token rows.
+static void gemm_scratch(const orthrus_config_t &c, int rows_body, int rows_lm, size_t *floats, int *tickets)
+{
+    const int d = c.hidden, hq = c.n_q_heads * c.head_dim, hk = c.n_kv_heads * c.head_dim;
+    struct Shape { int n_tiles, Kd, rows; };
+    const Shape shapes[] = {
+        {(hq + 2 * hk + kTileN - 1) / kTileN, d, rows_body},
+        {(d + kTileN - 1) / kTileN, hq, rows_body},
+        {(c.ffn + 63) / 64, d, rows_body},
+        {(d + kTileN - 1) / kTileN, c.ffn, rows_body},
+        {(c.vocab + kTileN - 1) / kTileN, d, rows_lm},
+    };
+    *floats = 0;
+    *tickets = 1;
+    for (const Shape &s : shapes) {
+        const int n_mt = (s.rows + kTileM - 1) / kTileM;
+        const int S = (use_tensor_cores(c) && s.Kd % kTileK == 0) ? choose_splits(s.n_tiles * kTileN, s.Kd) : 1;
+        if (S > 1) *floats = std::max(*floats, (size_t)n_mt * s.n_tiles * S * kTileM * kTileN);
+        *tickets = std::max(*tickets, n_mt * s.n_tiles);
+    }
+}
+
+size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
+{
+    const size_t es = c.dtype == ORTHRUS_BF16 ? 2 : 4;
+    const size_t d = c.hidden, hq = (size_t)c.n_q_heads * c.head_dim, hk = (size_t)c.n_kv_heads * c.head_dim;
+    const size_t F = c.ffn, L = c.n_layers, mb = c.max_batch;
+    const size_t R = mb * c.max_block;
+    const size_t Rw = std::max(R, (size_t)kPrefillChunk);
+    const size_t Rlm = std::max(R, 2 * mb);
+    const size_t n_splits = (c.max_seq + c.split_tokens - 1) / c.split_tokens;
+    const size_t n_vtiles = (c.vocab + kTileN - 1) / kTileN;
+    size_t gfloats;
+    int gtickets;
+    gemm_scratch(c, (int)Rw, (int)Rlm, &gfloats, &gtickets);
+
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off += align256(bytes); return o; };
+    const size_t o_h = take(Rw * d * 4), o_a = take(Rw * d * es), o_q = take(Rw * hq * es), o_o = take(Rw * hq * es);
+    const size_t o_act = take(Rw * F * es);
+    const size_t o_kd = take(L * R * hk * es), o_vd = take(L * R * hk * es);
+    const size_t o_fd = take(R * d * es), o_fv = take(R * d * es), o_rx = take(2 * mb * d * es);
+    // attention partials: [Rw][n_q][n_splits][hd] fp32 and [Rw][n_q][n_splits] float2
+    const size_t o_part = take(Rw * c.n_q_heads * n_splits * c.head_dim * 4);
+    const size_t o_ml = take(Rw * c.n_q_heads * n_splits * 8);
+    const size_t o_gp = take(std::max(gfloats, (size_t)1) * 4), o_gt = take((size_t)gtickets * 4);
+    const size_t o_lm = take(Rlm * n_vtiles * sizeof(LmPart));
+    const size_t o_tok = take(Rw * 4), o_pos = take(mb * 4), o_bt = take(mb * 4), o_pr = take(4);
+    const size_t o_dr = take(R * 4), o_lq = take(R * 4), o_lsq = take(R * 4), o_g = take(R * 4), o_lp = take(R * 4),
+                 o_lsp = take(R * 4);
+    const size_t o_rj = take(mb * 4), o_rt = take(mb * 4), o_any = take(4), o_err = take(4), o_prod = take(mb * 4),
+                 o_step = take(8), o_nb = take(mb * 4), o_tb = take(R * 4), o_ab = take(mb * 4);
+    const size_t total = off;
+    if (x) {
+        char *base = (char *)nullptr;
+        auto P = [&](size_t o) { return (void *)(base + o); };
+        x->h = (float *)P(o_h); x->a = P(o_a); x->q = P(o_q); x->attn_o = P(o_o); x->act = P(o_act);
+        x->k_diff = P(o_kd); x->v_diff = P(o_vd); x->fin_draft = P(o_fd); x->fin_verify = P(o_fv); x->res_x = P(o_rx);
+        x->attn_part = (float *)P(o_part); x->attn_ml = (float2 *)P(o_ml);
+        x->gemm_part = (float *)P(o_gp); x->gemm_part_floats = gfloats; x->gemm_ticket = (int *)P(o_gt);
+        x->gemm_tickets = gtickets; x->lm_part = (LmPart *)P(o_lm);
+        x->tok = (int32_t *)P(o_tok); x->pos0 = (int32_t *)P(o_pos); x->bt_rows = (int32_t *)P(o_bt);
+        x->prefill_row = (int32_t *)P(o_pr);
+        x->draft = (int32_t *)P(o_dr); x->logq = (float *)P(o_lq); x->lse_q = (float *)P(o_lsq);
+        x->g = (int32_t *)P(o_g); x->logp = (float *)P(o_lp); x->lse_p = (float *)P(o_lsp);
+        x->rej_row = (int32_t *)P(o_rj); x->res_tok = (int32_t *)P(o_rt); x->any_reject = (int *)P(o_any);
+        x->err = (unsigned *)P(o_err); x->produced = (int32_t *)P(o_prod); x->step = (int64_t *)P(o_step);
+        x->n_buf = (int32_t *)P(o_nb); x->tok_buf = (int32_t *)P(o_tb); x->anchor_buf = (int32_t *)P(o_ab);
+        x->R = (int)R; x->Rw = (int)Rw; x->n_splits = (int)n_splits; x->n_vtiles = (int)n_vtiles;
+        x->esize = (int)es;
+    }
+    return total;
+}
+
+static void rebase(Ctx *x, char *ws)
+{
+    auto fix = [&](auto *&p) { p = (std::remove_reference_t<decltype(p)>)(ws + (size_t)(const char *)p); };
+    fix(x->h); fix(x->a); fix(x->q); fix(x->attn_o); fix(x->act); fix(x->k_diff); fix(x->v_diff);
+    fix(x->fin_draft); fix(x->fin_verify); fix(x->res_x); fix(x->attn_part); fix(x->attn_ml); fix(x->gemm_part);
+    fix(x->gemm_ticket); fix(x->lm_part); fix(x->tok); fix(x->pos0); fix(x->bt_rows); fix(x->prefill_row);
+    fix(x->draft); fix(x->logq); fix(x->lse_q); fix(x->g); fix(x->logp); fix(x->lse_p); fix(x->rej_row);
+    fix(x->res_tok); fix(x->any_reject); fix(x->err); fix(x->produced); fix(x->step); fix(x->n_buf);
+    fix(x->tok_buf); fix(x->anchor_buf);
+}
+
+static KvView kv_view(const orthrus_kv_t &kv)
+{
+    return KvView{kv.k_pages, kv.v_pages, kv.block_table, kv.num_pages, kv.page_size, kv.max_pages_per_seq};
+}
+
+// Event probe (orthrus_set_probe): bracket a launch of the probed family in
+// the probed layer and view.
+struct ProbeScope {
+    Ctx &c;
+    bool on;
+    size_t slot;
+    cudaStream_t s;
+    ProbeScope(Ctx &c_, int family, int layer, int view, cudaStream_t s_)
+        : c(c_), on(!c_.probe_start.empty() && c_.probe_family == family && c_.probe_layer == layer &&
+                    c_.probe_view == view),
+          slot(0), s(s_)
+    {
+        if (on) {
+            slot = c.probe_hits++ % c.probe_start.size();
+            cudaEventRecord(c.probe_start[slot], s);
+        }
+    }
+    ~ProbeScope()
+    {
+        if (on) cudaEventRecord(c.probe_stop[slot], s);
+    }
+};
+
+// One forward of either view over B*K rows already embedded in c.h.
+//   view 0: AR W_Q/W_K/W_V, K/V written into the cache, causal (mode 0)
+//   view 1: diffusion W^diff, K/V into the transient buffer, block
+//           bidirectional (mode 1)
+// fin (nullable): final-norm rows for the LM head.
+static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int K, const int32_t *pos0,
+                           const int32_t *bt_rows, void *fin, cudaStream_t s)
+{
+    const orthrus_config_t &f = c.cfg;
+    const int M = B * K, hd = f.head_dim;
+    const size_t es = c.esize;
+    cudaError_t e;
+    for (int l = 0; l < f.n_layers; ++l) {
+        const orthrus_layer_weights_t &W = c.layers[l];
+        if ((e = launch_rmsnorm(c, c.h, W.attn_norm, c.a, M, s)) != cudaSuccess) return e;
+        GemmArgs q{};
+        q.x = c.a; q.M = M; q.Kd = f.hidden;
+        q.w[0] = view ? W.wq_diff : W.wq; q.w[1] = view ? W.wk_diff : W.wk; q.w[2] = view ? W.wv_diff : W.wv;
+        q.wrows[0] = f.n_q_heads * hd; q.wrows[1] = q.wrows[2] = f.n_kv_heads * hd;
+        q.N = q.wrows[0] + 2 * q.wrows[1];
+        q.epi = EPI_QKV; q.q_out = c.q; q.n_q = f.n_q_heads; q.n_kv = f.n_kv_heads; q.hd = hd; q.layer = l;
+        q.kv_to_cache = view == 0; q.k_blk = c.k_diff; q.v_blk = c.v_diff; q.rows_max = c.R;
+        q.kv = kv_view(kv); q.pos0 = pos0; q.bt_rows = bt_rows; q.K = K; q.rope_theta = (double)f.rope_theta;
+        {
+            ProbeScope ps(c, 0, l, view, s);
+            if ((e = launch_gemm(c, q, s)) != cudaSuccess) return e;
+        }
+
+        AttnArgs at{};
+        at.q = c.q; at.out = c.attn_o;
+        const size_t lay = (size_t)l * c.R * f.n_kv_heads * hd * es;
+        at.k_blk = (const char *)c.k_diff + lay; at.v_blk = (const char *)c.v_diff + lay;
+        at.kv = kv_view(kv); at.layer = l; at.seq_lens = pos0; at.bt_rows = bt_rows;
+        at.B = B; at.K = K; at.n_q = f.n_q_heads; at.n_kv = f.n_kv_heads; at.hd = hd; at.mode = view;
+        at.split_tokens = f.split_tokens; at.n_splits = c.n_splits; at.part = c.attn_part; at.ml = c.attn_ml;
+        at.err = c.err;
+        {
+            ProbeScope ps(c, 1, l, view, s);
+            if ((e = launch_attention(c, at, s)) != cudaSuccess) return e;
+        }
+
+        GemmArgs o{};
+        o.x = c.attn_o; o.M = M; o.N = f.hidden; o.Kd = f.n_q_heads * hd; o.w[0] = W.wo; o.wrows[0] = f.hidden;
+        o.epi = EPI_RESID; o.resid = c.h;
+        {
+            ProbeScope ps(c, 0, l, view, s);
+            if ((e = launch_gemm(c, o, s)) != cudaSuccess) return e;
+        }
+
+        if ((e = launch_rmsnorm(c, c.h, W.ffn_norm, c.a, M, s)) != cudaSuccess) return e;
+        GemmArgs gu{};
+        gu.x = c.a; gu.M = M; gu.N = f.ffn; gu.Kd = f.hidden; gu.w[0] = W.w_gate; gu.w[1] = W.w_up;
+        gu.wrows[0] = gu.wrows[1] = f.ffn; gu.epi = EPI_SWIGLU; gu.act = c.act;
+        {
+            ProbeScope ps(c, 0, l, view, s);
+            if ((e = launch_gemm(c, gu, s)) != cudaSuccess) return e;
+        }
+
+        GemmArgs dn{};
+        dn.x = c.act; dn.M = M; dn.N = f.hidden; dn.Kd = f.ffn; dn.w[0] = W.w_down; dn.wrows[0] = f.hidden;
+        dn.epi = EPI_RESID; dn.resid = c.h;
+        {
+            ProbeScope ps(c, 0, l, view, s);
+            if ((e = launch_gemm(c, dn, s)) != cudaSuccess) return e;
+        }
+    }
+    if (fin) return launch_rmsnorm(c, c.h, c.final_norm, fin, M, s);
+    return cudaSuccess;
+}
+
+static cudaError_t lm_head(Ctx &c, const void *fin, int B, int K, int lm_mode, float temperature, uint64_t seed,
+                           const int64_t *step, const int32_t *given, cudaStream_t s)
+{
+    GemmArgs g{};
+    g.x = fin; g.M = B * K; g.N = c.cfg.vocab; g.Kd = c.cfg.hidden; g.w[0] = c.lm_head; g.wrows[0] = c.cfg.vocab;
+    g.epi = EPI_LMHEAD; g.lm = c.lm_part; g.inv_temp = temperature > 0.f ? 1.0f / temperature : 0.f;
+    g.seed = seed; g.step = step; g.lm_mode = lm_mode; g.given = given; g.K = K;
+    return launch_gemm(c, g, s);
+}
+
+}  // namespace orthrus
+
+using namespace orthrus;
+
+#define CK(x)                                     \
+    do {                                          \
+        cudaError_t e_ = (x);                     \
+        if (e_ != cudaSuccess) return ORTHRUS_ERR_CUDA; \
+    } while (0)
+
+static bool kv_ok(const orthrus_ctx_t *c, const orthrus_kv_t *kv)
+{
+    if (!kv || !kv->k_pages || !kv->v_pages || !kv->block_table || !kv->seq_lens) return false;
+    if (kv->num_pages < 1 || kv->max_pages_per_seq < 1) return false;
+    const int ps_mult = (c->cfg.dtype == ORTHRUS_BF16 && c->cfg.head_dim == 128) ? 64 : 16;
+    if (kv->page_size < ps_mult || kv->page_size % ps_mult) return false;
+    return true;
+}
+
+extern "C" {
+
+const char *orthrus_status_string(orthrus_status_t s)
+{
+    switch (s) {
+    case ORTHRUS_OK: return "ok";
+    case ORTHRUS_ERR_INVALID_ARG: return "invalid argument";
+    case ORTHRUS_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ORTHRUS_ERR_CAPACITY: return "capacity exceeded";
+    case ORTHRUS_ERR_CUDA: return "CUDA runtime error";
+    case ORTHRUS_ERR_DEVICE_CHECK: return "device-side check failed";
+    case ORTHRUS_ERR_NONFINITE: return "non-finite log-sum-exp";
+    }
+    return "unknown status";
+}
+
+orthrus_status_t orthrus_workspace_size(const orthrus_config_t *cfg, size_t *bytes)
+{
+    if (!cfg || !bytes) return ORTHRUS_ERR_INVALID_ARG;
+    if (!valid_config(*cfg)) return ORTHRUS_ERR_INVALID_ARG;
+    *bytes = plan_workspace(*cfg, nullptr);
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_transient_bytes(const orthrus_config_t *cfg, int32_t batch, int32_t K, size_t *bytes)
+{
+    if (!cfg || !bytes || !valid_config(*cfg) || batch < 1 || K < 1) return ORTHRUS_ERR_INVALID_ARG;
+    if (batch > cfg->max_batch || K > cfg->max_block) return ORTHRUS_ERR_CAPACITY;
+    const size_t es = cfg->dtype == ORTHRUS_BF16 ? 2 : 4;
+    *bytes = (size_t)cfg->n_layers * batch * K * cfg->n_kv_heads * cfg->head_dim * 2 * es;
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_create(const orthrus_config_t *cfg, const orthrus_weights_t *w, void *workspace,
+                                size_t ws_bytes, orthrus_ctx_t **out)
+{
+    if (!cfg || !w || !workspace || !out || !w->embed || !w->final_norm || !w->lm_head || !w->layers)
+        return ORTHRUS_ERR_INVALID_ARG;
+    if (!valid_config(*cfg)) return ORTHRUS_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace % 256) return ORTHRUS_ERR_INVALID_ARG;
+    for (int l = 0; l < cfg->n_layers; ++l) {
+        const orthrus_layer_weights_t &L = w->layers[l];
+        if (!L.attn_norm || !L.wq || !L.wk || !L.wv || !L.wq_diff || !L.wk_diff || !L.wv_diff || !L.wo ||
+            !L.ffn_norm || !L.w_gate || !L.w_up || !L.w_down)
+            return ORTHRUS_ERR_INVALID_ARG;
+    }
+    orthrus_ctx_t *c = new (std::nothrow) orthrus_ctx_t();
+    if (!c) return ORTHRUS_ERR_CAPACITY;
+    c->cfg = *cfg;
+    const size_t need = plan_workspace(*cfg, c);
+    if (ws_bytes < need) { delete c; return ORTHRUS_ERR_CAPACITY; }
+    rebase(c, (char *)workspace);
+    c->layers.assign(w->layers, w->layers + cfg->n_layers);
+    c->embed = w->embed; c->final_norm = w->final_norm; c->lm_head = w->lm_head;
+    if (cudaGetDevice(&c->dev) != cudaSuccess || gemm_init_attributes() != cudaSuccess ||
+        attention_init_attributes() != cudaSuccess) {
+        delete c;
+        return ORTHRUS_ERR_CUDA;
+    }
+    std::vector<int32_t> ident(cfg->max_batch);
+    for (int b = 0; b < cfg->max_batch; ++b) ident[b] = b;
+    if (cudaMemset(workspace, 0, need) != cudaSuccess ||
+        cudaMemcpy(c->bt_rows, ident.data(), ident.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess) {
+        delete c;
+        return ORTHRUS_ERR_CUDA;
+    }
+    *out = c;
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_destroy(orthrus_ctx_t *c)
+{
+    if (!c) return ORTHRUS_ERR_INVALID_ARG;
+    delete c;
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_prefill(orthrus_ctx_t *c, const orthrus_kv_t *kv, const int32_t *tokens, int32_t stride,
+                                 const int32_t *lens, int32_t batch, int32_t *anchor_out, void *stream)
+{
+    if (!c || !kv_ok(c, kv) || !tokens || !lens || !anchor_out || batch < 1) return ORTHRUS_ERR_INVALID_ARG;
+    if (batch > c->cfg.max_batch) return ORTHRUS_ERR_CAPACITY;
+    cudaStream_t s = (cudaStream_t)stream;
+    for (int b = 0; b < batch; ++b) {
+        if (lens[b] < 1 || lens[b] > stride) return ORTHRUS_ERR_INVALID_ARG;
+        if (lens[b] - 1 + c->cfg.max_block > c->cfg.max_seq ||
+            lens[b] - 1 > kv->max_pages_per_seq * kv->page_size)
+            return ORTHRUS_ERR_CAPACITY;
+    }
+    for (int b = 0; b < batch; ++b) {
+        const int n = lens[b] - 1;
+        CK(launch_set_int(c->prefill_row, b, s));
+        c->launches += 1;
+        for (int p0 = 0; p0 < n; p0 += c->Rw) {
+            const int R = std::min(c->Rw, n - p0);
+            CK(launch_set_int(c->pos0, p0, s));
+            c->launches += 1;
+            CK(launch_embed(*c, 2, tokens + (size_t)b * stride + p0, nullptr, nullptr, 1, R, s));
+            CK(forward(*c, *kv, 0, 1, R, c->pos0, c->prefill_row, nullptr, s));
+        }
+        CK(launch_set_lens(*c, kv->seq_lens, b, n, anchor_out, tokens + (size_t)b * stride + n, s));
+        c->launches += 1;
+    }
+    return ORTHRUS_OK;
+}
+
+static orthrus_status_t check_step(orthrus_ctx_t *c, const orthrus_kv_t *kv, int batch, int K)
+{
+    if (!c || !kv_ok(c, kv) || batch < 1 || K < 1) return ORTHRUS_ERR_INVALID_ARG;
+    if (batch > c->cfg.max_batch || K > c->cfg.max_block) return ORTHRUS_ERR_CAPACITY;
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_draft_block(orthrus_ctx_t *c, const orthrus_kv_t *kv, const int32_t *anchor, int32_t batch,
+                                     int32_t K, float temperature, uint64_t seed, const int64_t *step, int32_t *draft,
+                                     void *stream)
+{
+    orthrus_status_t st = check_step(c, kv, batch, K);
+    if (st != ORTHRUS_OK) return st;
+    if (!anchor || !draft || (temperature > 0.f && !step) || temperature < 0.f) return ORTHRUS_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    CK(launch_embed(*c, 0, nullptr, anchor, nullptr, batch, K, s));
+    CK(forward(*c, *kv, 1, batch, K, kv->seq_lens, c->bt_rows, c->fin_draft, s));
+    CK(lm_head(*c, c->fin_draft, batch, K, 1, temperature, seed, step, nullptr, s));
+    CK(launch_lm_finalize_impl(*c, 1, batch, K, temperature, draft, nullptr, s));
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_verify_block(orthrus_ctx_t *c, const orthrus_kv_t *kv, const int32_t *anchor,
+                                      const int32_t *draft, int32_t batch, int32_t K, float temperature, void *stream)
+{
+    orthrus_status_t st = check_step(c, kv, batch, K);
+    if (st != ORTHRUS_OK) return st;
+    if (!anchor || !draft || temperature < 0.f) return ORTHRUS_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    CK(launch_embed(*c, 1, nullptr, anchor, draft, batch, K, s));
+    CK(forward(*c, *kv, 0, batch, K, kv->seq_lens, c->bt_rows, c->fin_verify, s));
+    CK(lm_head(*c, c->fin_verify, batch, K, 0, temperature, 0, nullptr, draft, s));
+    CK(launch_lm_finalize_impl(*c, 0, batch, K, temperature, nullptr, draft, s));
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_commit(orthrus_ctx_t *c, const orthrus_kv_t *kv, int32_t batch, int32_t K, float temperature,
+                                uint64_t seed, int64_t *step, const int32_t *force_n, int32_t *n_out,
+                                int32_t *tokens_out, int32_t *anchor_io, void *stream)
+{
+    orthrus_status_t st = check_step(c, kv, batch, K);
+    if (st != ORTHRUS_OK) return st;
+    if (!step || !n_out || !anchor_io || temperature < 0.f) return ORTHRUS_ERR_INVALID_ARG;
+    CK(launch_commit(*c, *kv, batch, K, temperature, seed, step, force_n, n_out, tokens_out, anchor_io, nullptr, 0, 0,
+                     (cudaStream_t)stream));
+    return ORTHRUS_OK;
+}
+
+static orthrus_status_t ar_step_impl(orthrus_ctx_t *c, const orthrus_kv_t *kv, int batch, float temperature,
+                                     uint64_t seed, int64_t *step, int32_t *token_out, int32_t *anchor_io,
+                                     int32_t *append, int stride, int amax, cudaStream_t s)
+{
+    CK(launch_embed(*c, 1, nullptr, anchor_io, nullptr, batch, 1, s));
+    CK(forward(*c, *kv, 0, batch, 1, kv->seq_lens, c->bt_rows, c->fin_verify, s));
+    CK(lm_head(*c, c->fin_verify, batch, 1, 2, temperature, seed, step, nullptr, s));
+    CK(launch_lm_finalize_impl(*c, 2, batch, 1, temperature, nullptr, nullptr, s));
+    CK(launch_ar_commit(*c, *kv, batch, step, token_out, anchor_io, append, stride, amax, s));
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_ar_step(orthrus_ctx_t *c, const orthrus_kv_t *kv, int32_t batch, float temperature,
+                                 uint64_t seed, int64_t *step, int32_t *token_out, int32_t *anchor_io, void *stream)
+{
+    orthrus_status_t st = check_step(c, kv, batch, 1);
+    if (st != ORTHRUS_OK) return st;
+    if (!step || !anchor_io || temperature < 0.f) return ORTHRUS_ERR_INVALID_ARG;
+    return ar_step_impl(c, kv, batch, temperature, seed, step, token_out, anchor_io, nullptr, 0, 0,
+                        (cudaStream_t)stream);
+}
+
+orthrus_status_t orthrus_set_probe(orthrus_ctx_t *c, int32_t family, int32_t layer, int32_t view,
+                                   void *const *starts, void *const *stops, int32_t n)
+{
+    if (!c || n < 0 || (n > 0 && (!starts || !stops))) return ORTHRUS_ERR_INVALID_ARG;
+    if (n > 0 && (family < 0 || family > 1 || layer < 0 || layer >= c->cfg.n_layers || view < 0 || view > 1))
+        return ORTHRUS_ERR_INVALID_ARG;
+    c->probe_start.clear();
+    c->probe_stop.clear();
+    c->probe_hits = 0;
+    for (int i = 0; i < n; ++i) {
+        if (!starts[i] || !stops[i]) { c->probe_start.clear(); c->probe_stop.clear(); return ORTHRUS_ERR_INVALID_ARG; }
+        c->probe_start.push_back((cudaEvent_t)starts[i]);
+        c->probe_stop.push_back((cudaEvent_t)stops[i]);
+    }
+    c->probe_family = family; c->probe_layer = layer; c->probe_view = view;
+    return ORTHRUS_OK;
+}
+
+uint64_t orthrus_launch_count(const orthrus_ctx_t *c) { return c ? c->launches : 0; }
+
+orthrus_status_t orthrus_check_error(orthrus_ctx_t *c, void *stream, uint32_t *bits)
+{
+    if (!c) return ORTHRUS_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned h = 0;
+    CK(cudaMemcpyAsync(&h, c->err, 4, cudaMemcpyDeviceToHost, s));
+    CK(cudaMemsetAsync(c->err, 0, 4, s));
+    CK(cudaStreamSynchronize(s));
+    if (bits) *bits = h;
+    if (h & ORTHRUS_DEVERR_NONFINITE) return ORTHRUS_ERR_NONFINITE;
+    if (h) return ORTHRUS_ERR_DEVICE_CHECK;
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_generate(orthrus_ctx_t *c, const orthrus_kv_t *kv, const int32_t *prompt, int32_t stride,
+                                  const int32_t *lens, int32_t batch, int32_t K, int32_t max_new, float temperature,
+                                  uint64_t seed, int32_t *out, orthrus_stats_t *stats, void *stream)
+{
+    if (!c || !prompt || !lens || !out || max_new < 1 || K < 0 || temperature < 0.f) return ORTHRUS_ERR_INVALID_ARG;
+    orthrus_status_t st = check_step(c, kv, batch, K > 0 ? K : 1);
+    if (st != ORTHRUS_OK) return st;
+    const int Kb = K > 0 ? K : 1;
+    for (int b = 0; b < batch; ++b) {
+        if (lens[b] < 1) return ORTHRUS_ERR_INVALID_ARG;
+        const long need = (long)lens[b] - 1 + max_new + Kb;
+        if (need > c->cfg.max_seq || need > (long)kv->max_pages_per_seq * kv->page_size) return ORTHRUS_ERR_CAPACITY;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    st = orthrus_prefill(c, kv, prompt, stride, lens, batch, c->anchor_buf, stream);
+    if (st != ORTHRUS_OK) return st;
+    CK(cudaMemsetAsync(c->produced, 0, (size_t)batch * 4, s));
+    CK(cudaMemsetAsync(c->step, 0, 8, s));
+    std::vector<int32_t> prod(batch);
+    orthrus_stats_t stt{};
+    for (int cycle = 0; cycle < max_new; ++cycle) {
+        if (K == 0) {
+            st = ar_step_impl(c, kv, batch, temperature, seed, c->step, nullptr, c->anchor_buf, out, max_new, max_new, s);
+            if (st != ORTHRUS_OK) return st;
+            stt.forwards += 1;
+        } else {
+            st = orthrus_draft_block(c, kv, c->anchor_buf, batch, K, temperature, seed, c->step, c->draft, stream);
+            if (st != ORTHRUS_OK) return st;
+            st = orthrus_verify_block(c, kv, c->anchor_buf, c->draft, batch, K, temperature, stream);
+            if (st != ORTHRUS_OK) return st;
+            CK(launch_commit(*c, *kv, batch, K, temperature, seed, c->step, nullptr, c->n_buf, c->tok_buf,
+                             c->anchor_buf, out, max_new, max_new, s));
+            stt.forwards += 2;
+        }
+        stt.cycles += 1;
+        CK(cudaMemcpyAsync(prod.data(), c->produced, (size_t)batch * 4, cudaMemcpyDeviceToHost, s));
+        CK(cudaStreamSynchronize(s));
+        const int mn = *std::min_element(prod.begin(), prod.end());
+        if (mn >= max_new) break;
+    }
+    for (int b = 0; b < batch; ++b) stt.tokens += std::min(prod[b], max_new);
+    stt.min_tokens = *std::min_element(prod.begin(), prod.end());
+    if (stats) *stats = stt;
+    return orthrus_check_error(c, stream, nullptr);
+}
+
+orthrus_status_t orthrus_dual_view_attention(orthrus_ctx_t *c, const orthrus_kv_t *kv, int32_t layer, int32_t mode,
+                                             const void *q, const void *k_blk, const void *v_blk, int32_t batch,
+                                             int32_t K, void *out, void *stream)
+{
+    orthrus_status_t st = check_step(c, kv, batch, K);
+    if (st != ORTHRUS_OK) return st;
+    if (!q || !out || (mode != 0 && mode != 1) || (mode == 1 && (!k_blk || !v_blk)) || layer < 0 ||
+        layer >= c->cfg.n_layers)
+        return ORTHRUS_ERR_INVALID_ARG;
+    const orthrus_config_t &f = c->cfg;
+    AttnArgs at{};
+    at.q = q; at.out = out; at.k_blk = k_blk; at.v_blk = v_blk; at.kv = kv_view(*kv); at.layer = layer;
+    at.seq_lens = kv->seq_lens; at.bt_rows = c->bt_rows; at.B = batch; at.K = K; at.n_q = f.n_q_heads;
+    at.n_kv = f.n_kv_heads; at.hd = f.head_dim; at.mode = mode; at.split_tokens = f.split_tokens;
+    at.n_splits = c->n_splits; at.part = c->attn_part; at.ml = c->attn_ml; at.err = c->err;
+    CK(launch_attention(*c, at, (cudaStream_t)stream));
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_debug_logits(orthrus_ctx_t *c, int32_t which, int32_t batch, int32_t K, float *logits,
+                                      void *stream)
+{
+    if (!c || !logits || (which != 0 && which != 1) || batch < 1 || K < 1) return ORTHRUS_ERR_INVALID_ARG;
+    if (batch * K > c->R) return ORTHRUS_ERR_CAPACITY;
+    CK(launch_logits_dump(*c, which ? c->fin_draft : c->fin_verify, batch * K, logits, (cudaStream_t)stream));
+    return ORTHRUS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,100 @@
+// Device helpers shared by the kernels of the dual-view decode library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/orthrus.h"
+
+namespace orthrus {
+
+using bf16 = __nv_bfloat16;
+
+// ---------------------------------------------------------------- dtype
+template <class T> __device__ __forceinline__ float to_f(T x);
+template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f<bf16>(bf16 x) { return __bfloat162float(x); }
+
+template <class T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
+
+// ---------------------------------------------------------------- errors
+__device__ __forceinline__ void raise_err(unsigned *err, unsigned bit) { atomicOr(err, bit); }
+
+// ---------------------------------------------------------------- RNG
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): ten rounds of two
+// 32x32->64 multiplies, key bumped by the Weyl constants between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k)
+{
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+        c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
+        k.x += 0x9E3779B9u;
+        k.y += 0xBB67AE85u;
+    }
+    return c;
+}
+
+enum Purpose : uint32_t { PURPOSE_DRAFT = 1, PURPOSE_ACCEPT = 2, PURPOSE_RESIDUAL = 3, PURPOSE_AR = 4 };
+
+// Uniform in (0,1) from counter (id, row, step, purpose) and key = seed:
+// top 24 bits of the first output word, centred in their cell.
+__device__ __forceinline__ float uniform01(uint64_t seed, uint32_t step, uint32_t row, uint32_t id,
+                                           uint32_t purpose)
+{
+    const uint4 o = philox4x32_10(make_uint4(id, row, step, purpose),
+                                  make_uint2((uint32_t)seed, (uint32_t)(seed >> 32)));
+    return ((float)(o.x >> 8) + 0.5f) * (1.0f / 16777216.0f);
+}
+
+__device__ __forceinline__ float gumbel(uint64_t seed, uint32_t step, uint32_t row, uint32_t id, uint32_t purpose)
+{
+    return -logf(-logf(uniform01(seed, step, row, id, purpose)));
+}
+
+// Row id used in the RNG counter: sequence b, block row k.
+__device__ __forceinline__ uint32_t rng_row(int b, int k) { return ((uint32_t)b << 16) | (uint32_t)k; }
+
+// ---------------------------------------------------------------- reductions
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// (value, index) max with the lowest index winning ties; NaN never wins.
+__device__ __forceinline__ void argmax_merge(float &v, int &i, float v2, int i2)
+{
+    if (v2 > v || (v2 == v && i2 < i)) { v = v2; i = i2; }
+}
+
+__device__ __forceinline__ void warp_argmax(float &v, int &i)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, i, o);
+        argmax_merge(v, i, v2, i2);
+    }
+}
+
+// ---------------------------------------------------------------- async copy
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// 16-byte cp.async; bytes = 0 zero-fills the destination.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N> __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+}  // namespace orthrus

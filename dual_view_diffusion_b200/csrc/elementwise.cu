@@ -1,0 +1,366 @@
+// Row-wise kernels of the decode cycle: block embedding, RMSNorm, the
+// LM-head reduction across vocab tiles, consensus and commit.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace orthrus {
+
+// ---------------------------------------------------------------- embedding
+// mode 0: draft block [anchor, mask x (K-1)] (paper notes §4.1 step 1)
+// mode 1: verify block [anchor, draft[0 .. K-2]] (§4.1 step 2)
+// mode 2: explicit tokens (prefill)
+template <class T>
+__global__ void embed_kernel(const T *embed, int d, int V, int mask_id, int mode, const int32_t *tokens,
+                             const int32_t *anchor, const int32_t *draft, int K, int32_t *tok_out, float *h,
+                             unsigned *err)
+{
+    const int row = blockIdx.x, b = row / K, k = row % K;
+    int tok;
+    if (mode == 2) tok = tokens[row];
+    else if (k == 0) tok = anchor[b];
+    else tok = mode == 0 ? mask_id : draft[b * K + k - 1];
+    if (tok < 0 || tok >= V) {
+        if (threadIdx.x == 0) raise_err(err, ORTHRUS_DEVERR_TOKEN);
+        tok = 0;
+    }
+    if (threadIdx.x == 0) tok_out[row] = tok;
+    const T *src = embed + (size_t)tok * d;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) h[(size_t)row * d + i] = to_f<T>(src[i]);
+}
+
+// ---------------------------------------------------------------- RMSNorm
+// out = h / sqrt(mean(h^2) + eps) * gain; fixed reduction order per row.
+template <class T>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const float *h, const T *gain, T *out, int d, float eps)
+{
+    __shared__ float red[8];
+    const int row = blockIdx.x, tid = threadIdx.x;
+    const float *x = h + (size_t)row * d;
+    float ss = 0.f;
+    for (int i = tid; i < d; i += 256) ss = fmaf(x[i], x[i], ss);
+    ss = warp_sum(ss);
+    if ((tid & 31) == 0) red[tid >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tot += red[w];
+    const float inv = 1.0f / sqrtf(tot / d + eps);
+    for (int i = tid; i < d; i += 256) out[(size_t)row * d + i] = from_f<T>(x[i] * inv * to_f<T>(gain[i]));
+}
+
+// ---------------------------------------------------------------- LM head
+// Merge the per-tile records of one row: global max / lowest argmax,
+// log-sum-exp of z/T (T = 1 when greedy), Gumbel winner, logit at the
+// given id.  mode 0 verify, 1 draft, 2 AR step, 3 residual resample.
+struct LmArgs {
+    const LmPart *part;
+    int n_vtiles, B, K, mode;
+    float inv_temp;
+    int32_t *draft, *draft_user, *g, *res_tok;
+    float *logq, *lse_q, *logp, *lse_p;
+    const int32_t *given, *rej_row;
+    unsigned *err;
+};
+
+__global__ void __launch_bounds__(256) lm_finalize_kernel(LmArgs a)
+{
+    const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    const int rows = a.mode == 3 ? a.B : a.B * a.K;
+    if (w >= rows) return;
+    if (a.mode == 3) {
+        const int j = a.rej_row[w];
+        if (j < 0) return;
+        const LmPart *p = a.part + (size_t)(2 * w) * a.n_vtiles;
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int i = lane; i < a.n_vtiles; i += 32) argmax_merge(bv, bi, p[i].gbest, p[i].garg);
+        warp_argmax(bv, bi);
+        if (lane == 0) a.res_tok[w] = bv > -INFINITY ? bi : a.g[w * a.K + j];
+        return;
+    }
+    const LmPart *p = a.part + (size_t)w * a.n_vtiles;
+    float zm = -INFINITY;
+    int za = 0x7fffffff;
+    float gb = -INFINITY, gz = 0.f;
+    int ga = 0x7fffffff;
+    float zid = NAN;
+    for (int i = lane; i < a.n_vtiles; i += 32) {
+        const LmPart q = p[i];
+        argmax_merge(zm, za, q.zmax, q.zarg);
+        if (q.gbest > gb || (q.gbest == gb && q.garg < ga)) { gb = q.gbest; ga = q.garg; gz = q.gz; }
+        if (!isnan(q.zid)) zid = q.zid;
+    }
+    warp_argmax(zm, za);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float gb2 = __shfl_xor_sync(0xffffffffu, gb, o);
+        const int ga2 = __shfl_xor_sync(0xffffffffu, ga, o);
+        const float gz2 = __shfl_xor_sync(0xffffffffu, gz, o);
+        if (gb2 > gb || (gb2 == gb && ga2 < ga)) { gb = gb2; ga = ga2; gz = gz2; }
+    }
+    const unsigned has = __ballot_sync(0xffffffffu, !isnan(zid));
+    if (has) zid = __shfl_sync(0xffffffffu, zid, __ffs(has) - 1);
+    const float it = a.inv_temp > 0.f ? a.inv_temp : 1.0f;
+    float s = 0.f;
+    for (int i = lane; i < a.n_vtiles; i += 32) s += p[i].zsum * expf((p[i].zmax - zm) * it);
+    s = warp_sum(s);
+    const float lse = zm * it + logf(s);
+    if (lane != 0) return;
+    if (!isfinite(lse)) raise_err(a.err, ORTHRUS_DEVERR_NONFINITE);
+    if (a.mode == 0) {
+        a.g[w] = za;
+        a.lse_p[w] = lse;
+        a.logp[w] = zid * it - lse;
+        if (a.given) a.draft[w] = a.given[w];
+    } else if (a.mode == 1) {
+        const int tok = a.inv_temp > 0.f ? ga : za;
+        a.draft[w] = tok;
+        if (a.draft_user) a.draft_user[w] = tok;
+        a.lse_q[w] = lse;
+        a.logq[w] = (a.inv_temp > 0.f ? gz : zm) * it - lse;
+    } else {
+        a.g[w] = a.inv_temp > 0.f ? ga : za;
+    }
+}
+
+// ---------------------------------------------------------------- commit
+struct CommitArgs {
+    int B, K;
+    float inv_temp;
+    uint64_t seed;
+    int64_t *step;
+    const int32_t *force_n;
+    const int32_t *draft, *g, *res_tok;
+    const float *logp, *logq;
+    int32_t *rej_row;
+    int *any_reject;
+    const void *fin_verify, *fin_draft;
+    void *res_x;
+    int d, esize;
+    int32_t *n_out, *tokens_out, *anchor_io, *seq_lens;
+    int32_t *append_out, *produced;
+    int append_stride, append_max;
+};
+
+// Decide n per sequence (paper notes §4.2 greedy, §4.3 sampled); for a
+// sampled rejection at row j, stage the two hidden rows the residual draw
+// needs (AR view, diffusion view).
+__global__ void commit_decide_kernel(CommitArgs a)
+{
+    const int b = blockIdx.x;
+    __shared__ int s_j;
+    if (threadIdx.x == 0) {
+        int n = a.K, j = -1;
+        if (a.force_n) {
+            n = min(max(a.force_n[b], 1), a.K);
+        } else if (a.inv_temp <= 0.f) {
+            for (int k = 0; k < a.K; ++k)
+                if (a.draft[b * a.K + k] != a.g[b * a.K + k]) { n = k + 1; break; }
+        } else {
+            const uint32_t step = (uint32_t)*a.step;
+            for (int k = 0; k < a.K; ++k) {
+                const float u = uniform01(a.seed, step, rng_row(b, k), 0, PURPOSE_ACCEPT);
+                if (!(logf(u) < a.logp[b * a.K + k] - a.logq[b * a.K + k])) { j = k; n = k + 1; break; }
+            }
+        }
+        a.n_out[b] = n;
+        if (a.rej_row) a.rej_row[b] = j;
+        if (j >= 0) atomicOr(a.any_reject, 1);
+        s_j = j;
+    }
+    __syncthreads();
+    if (s_j >= 0 && a.res_x) {
+        const size_t bytes = (size_t)a.d * a.esize;
+        const char *sv = (const char *)a.fin_verify + (size_t)(b * a.K + s_j) * bytes;
+        const char *sd = (const char *)a.fin_draft + (size_t)(b * a.K + s_j) * bytes;
+        char *dv = (char *)a.res_x + (size_t)(2 * b) * bytes;
+        for (size_t i = threadIdx.x; i < bytes; i += blockDim.x) { dv[i] = sv[i]; dv[bytes + i] = sd[i]; }
+    }
+}
+
+// Emit the tokens, advance the committed length (the accepted rows' AR K/V
+// are already in place: paper notes §4.1 step 3), bump the step counter.
+__global__ void commit_apply_kernel(CommitArgs a)
+{
+    const int b = threadIdx.x;
+    if (b < a.B) {
+        const int n = a.n_out[b];
+        const int j = a.rej_row ? a.rej_row[b] : -1;
+        const bool sampled = a.inv_temp > 0.f && !a.force_n;
+        int last = 0;
+        for (int i = 0; i < n; ++i) {
+            int tok;
+            if (!sampled) tok = a.g[b * a.K + i];
+            else tok = (i == j) ? a.res_tok[b] : a.draft[b * a.K + i];
+            if (a.tokens_out) a.tokens_out[b * a.K + i] = tok;
+            if (a.append_out) {
+                const int pos = a.produced[b] + i;
+                if (pos < a.append_max) a.append_out[(size_t)b * a.append_stride + pos] = tok;
+            }
+            last = tok;
+        }
+        if (a.append_out) a.produced[b] += n;
+        a.anchor_io[b] = last;
+        a.seq_lens[b] += n;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        *a.step += 1;
+        if (a.any_reject) *a.any_reject = 0;
+    }
+}
+
+// ---------------------------------------------------------------- AR step
+__global__ void ar_commit_kernel(int B, const int32_t *g, int64_t *step, int32_t *token_out, int32_t *anchor_io,
+                                 int32_t *seq_lens, int32_t *append_out, int32_t *produced, int stride, int amax)
+{
+    const int b = threadIdx.x;
+    if (b < B) {
+        const int tok = g[b];
+        if (token_out) token_out[b] = tok;
+        anchor_io[b] = tok;
+        seq_lens[b] += 1;
+        if (append_out) {
+            if (produced[b] < amax) append_out[(size_t)b * stride + produced[b]] = tok;
+            produced[b] += 1;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) *step += 1;
+}
+
+__global__ void set_lens_kernel(int32_t *seq_lens, int b, int value, int32_t *anchor_out, const int32_t *last_tok)
+{
+    seq_lens[b] = value;
+    if (anchor_out) anchor_out[b] = *last_tok;
+}
+
+__global__ void set_int_kernel(int32_t *p, int v) { *p = v; }
+
+// ---------------------------------------------------------------- host
+cudaError_t launch_embed(const Ctx &c, int mode, const int32_t *tokens, const int32_t *anchor, const int32_t *draft,
+                         int B, int K, cudaStream_t s)
+{
+    const int rows = B * K;
+    c.launches += 1;
+    if (c.cfg.dtype == ORTHRUS_BF16)
+        embed_kernel<bf16><<<rows, 256, 0, s>>>((const bf16 *)c.embed, c.cfg.hidden, c.cfg.vocab, c.cfg.mask_token_id,
+                                                 mode, tokens, anchor, draft, K, c.tok, c.h, c.err);
+    else
+        embed_kernel<float><<<rows, 256, 0, s>>>((const float *)c.embed, c.cfg.hidden, c.cfg.vocab,
+                                                  c.cfg.mask_token_id, mode, tokens, anchor, draft, K, c.tok, c.h,
+                                                  c.err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const Ctx &c, const float *h, const void *gain, void *out, int M, cudaStream_t s)
+{
+    c.launches += 1;
+    if (c.cfg.dtype == ORTHRUS_BF16)
+        rmsnorm_kernel<bf16><<<M, 256, 0, s>>>(h, (const bf16 *)gain, (bf16 *)out, c.cfg.hidden, c.cfg.rms_eps);
+    else
+        rmsnorm_kernel<float><<<M, 256, 0, s>>>(h, (const float *)gain, (float *)out, c.cfg.hidden, c.cfg.rms_eps);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lm_finalize_impl(const Ctx &c, int mode, int B, int K, float temperature, int32_t *tok_out,
+                                    const int32_t *given, cudaStream_t s)
+{
+    LmArgs a;
+    a.part = c.lm_part; a.n_vtiles = c.n_vtiles; a.B = B; a.K = K; a.mode = mode;
+    a.inv_temp = temperature > 0.f ? 1.0f / temperature : 0.f;
+    a.draft = c.draft; a.draft_user = tok_out; a.g = c.g; a.res_tok = c.res_tok;
+    a.logq = c.logq; a.lse_q = c.lse_q; a.logp = c.logp; a.lse_p = c.lse_p;
+    a.given = given; a.rej_row = c.rej_row; a.err = c.err;
+    const int rows = mode == 3 ? B : B * K;
+    c.launches += 1;
+    lm_finalize_kernel<<<(rows + 7) / 8, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lm_finalize(const Ctx &c, int mode, int B, int K, float temperature, uint64_t, const int64_t *,
+                               int32_t *tok_out, cudaStream_t s)
+{
+    return launch_lm_finalize_impl(c, mode, B, K, temperature, tok_out, mode == 0 ? tok_out : nullptr, s);
+}
+
+static CommitArgs commit_args(const Ctx &c, const orthrus_kv_t &kv, int B, int K, float temperature, uint64_t seed,
+                              int64_t *step, const int32_t *force_n, int32_t *n_out, int32_t *tokens_out,
+                              int32_t *anchor_io, int32_t *append_out, int append_stride, int append_max)
+{
+    CommitArgs a;
+    a.B = B; a.K = K; a.inv_temp = temperature > 0.f ? 1.0f / temperature : 0.f;
+    a.seed = seed; a.step = step; a.force_n = force_n;
+    a.draft = c.draft; a.g = c.g; a.res_tok = c.res_tok; a.logp = c.logp; a.logq = c.logq;
+    a.rej_row = c.rej_row; a.any_reject = c.any_reject;
+    a.fin_verify = c.fin_verify; a.fin_draft = c.fin_draft; a.res_x = c.res_x;
+    a.d = c.cfg.hidden; a.esize = c.esize;
+    a.n_out = n_out; a.tokens_out = tokens_out; a.anchor_io = anchor_io; a.seq_lens = kv.seq_lens;
+    a.append_out = append_out; a.produced = c.produced; a.append_stride = append_stride; a.append_max = append_max;
+    return a;
+}
+
+cudaError_t launch_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int K, float temperature, uint64_t seed,
+                          int64_t *step, const int32_t *force_n, int32_t *n_out, int32_t *tokens_out,
+                          int32_t *anchor_io, int32_t *append_out, int append_stride, int append_max,
+                          cudaStream_t s)
+{
+    CommitArgs a = commit_args(c, kv, B, K, temperature, seed, step, force_n, n_out, tokens_out, anchor_io,
+                               append_out, append_stride, append_max);
+    c.launches += 2;
+    commit_decide_kernel<<<B, 128, 0, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (temperature > 0.f && !force_n) {
+        // residual draw at the rejected row: one LM-head pass over the two
+        // staged hidden rows per sequence (skipped on device when nothing
+        // was rejected)
+        GemmArgs g{};
+        g.x = c.res_x; g.M = 2 * B; g.N = c.cfg.vocab; g.Kd = c.cfg.hidden;
+        g.w[0] = c.lm_head; g.wrows[0] = c.cfg.vocab;
+        g.epi = EPI_RESAMPLE; g.lm = c.lm_part; g.inv_temp = 1.0f / temperature; g.seed = seed; g.step = step;
+        g.lse_p = c.lse_p; g.lse_q = c.lse_q; g.rej_row = c.rej_row; g.any_flag = c.any_reject; g.K = K;
+        e = launch_gemm(c, g, s);
+        if (e != cudaSuccess) return e;
+        e = launch_lm_finalize_impl(c, 3, B, K, temperature, nullptr, nullptr, s);
+        if (e != cudaSuccess) return e;
+    }
+    commit_apply_kernel<<<1, 128, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ar_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int64_t *step, int32_t *token_out,
+                             int32_t *anchor_io, int32_t *append_out, int append_stride, int append_max,
+                             cudaStream_t s)
+{
+    c.launches += 1;
+    ar_commit_kernel<<<1, 128, 0, s>>>(B, c.g, step, token_out, anchor_io, kv.seq_lens, append_out, c.produced,
+                                       append_stride, append_max);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_set_lens(const Ctx &, int32_t *seq_lens, int b, int value, int32_t *anchor_out,
+                            const int32_t *last_tok, cudaStream_t s)
+{
+    set_lens_kernel<<<1, 1, 0, s>>>(seq_lens, b, value, anchor_out, last_tok);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_set_int(int32_t *p, int v, cudaStream_t s)
+{
+    set_int_kernel<<<1, 1, 0, s>>>(p, v);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_logits_dump(const Ctx &c, const void *fin, int M, float *logits, cudaStream_t s)
+{
+    GemmArgs g{};
+    g.x = fin; g.M = M; g.N = c.cfg.vocab; g.Kd = c.cfg.hidden;
+    g.w[0] = c.lm_head; g.wrows[0] = c.cfg.vocab;
+    g.epi = EPI_LOGITS; g.logits = logits;
+    return launch_gemm(c, g, s);
+}
+
+}  // namespace orthrus

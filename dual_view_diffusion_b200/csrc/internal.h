@@ -1,0 +1,179 @@
+// Internal declarations of the dual-view decode library: the context, the
+// workspace carve-up and the kernel launchers.  Not part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/orthrus.h"
+
+namespace orthrus {
+
+constexpr int kTileN = 128;          // GEMM tile: output features per tile
+constexpr int kTileM = 32;           // GEMM tile: token rows per tile
+constexpr int kTileK = 64;           // GEMM k chunk
+constexpr int kKeyTile = 64;         // attention: keys per tile
+constexpr int kPrefillChunk = 128;   // prefill rows per forward
+constexpr int kNumSMs = 148;         // B200
+
+// Per-(row, vocab tile) record of the fused LM-head epilogue.
+struct LmPart {
+    float zmax;   // max logit in the tile
+    float zsum;   // sum over the tile of exp((z - zmax) / T)
+    int zarg;     // lowest index attaining zmax
+    float gbest;  // best z/T + Gumbel (draft / AR sampling), or best residual score
+    int garg;     // its index
+    float gz;     // logit at garg
+    float zid;    // logit at the row's given id, NaN if the id is not in the tile
+    int pad;
+};
+
+enum Epi : int { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_LMHEAD = 3, EPI_RESAMPLE = 4, EPI_LOGITS = 5 };
+
+// Where an attention / QKV call reads positions and writes K/V.
+struct KvView {
+    void *k_pages, *v_pages;
+    const int32_t *block_table;
+    int num_pages, page_size, max_pages;
+};
+
+// One GEMM launch: Y[M][N] = X[M][Kd] . W^T with a fused epilogue.
+struct GemmArgs {
+    const void *x;           // [M][Kd] activations, dtype
+    int M, N, Kd;
+    // weight rows: concatenation of up to three matrices (QKV) or, for the
+    // SwiGLU epilogue, tile halves [0,64) from w[0] and [64,128) from w[1]
+    const void *w[3];
+    int wrows[3];
+    int splits;              // k segments per tile (fixed per matrix shape)
+    float *part;             // split partial tiles
+    int *ticket;             // per (m tile, n tile) arrival counters
+    unsigned *err;
+    int epi;
+    // EPI_RESID
+    float *resid;            // [M][N] fp32, += result
+    // EPI_SWIGLU
+    void *act;               // [M][N/2] dtype
+    // EPI_QKV
+    void *q_out;             // [M][n_q*hd]
+    int n_q, n_kv, hd, layer;
+    int kv_to_cache;         // 1: K/V into pages at (b, pos); 0: into k_blk/v_blk
+    void *k_blk, *v_blk;     // [n_layers][rows_max][n_kv][hd] when kv_to_cache == 0
+    int rows_max;
+    KvView kv;
+    const int32_t *pos0;     // [batch] position of block row 0
+    const int32_t *bt_rows;  // [batch] row of block_table for each batch entry
+    int K;                   // rows per sequence in this launch
+    double rope_theta;
+    // EPI_LMHEAD / EPI_RESAMPLE
+    LmPart *lm;              // [M][n_vtiles]
+    float inv_temp;          // 1/T (T > 0) or 0 for greedy
+    uint64_t seed;
+    const int64_t *step;
+    int lm_mode;             // 0 verify (zid from given ids), 1 draft (Gumbel), 2 AR sample
+    const int32_t *given;    // [M] id whose logit is wanted (verify), or null
+    const float *lse_p, *lse_q;   // EPI_RESAMPLE: per (b, k) row
+    const int32_t *rej_row;  // EPI_RESAMPLE: [batch] j or -1
+    const int *any_flag;     // EPI_RESAMPLE: skip everything when 0
+    float *logits;           // EPI_LOGITS: [M][N] fp32
+};
+
+struct AttnArgs {
+    const void *q;           // [B*K][n_q][hd]
+    void *out;               // [B*K][n_q][hd]
+    const void *k_blk, *v_blk;  // mode 1: [B*K][n_kv][hd]
+    KvView kv;
+    int layer;
+    const int32_t *seq_lens;  // [batch] t per sequence (positions of block row 0)
+    const int32_t *bt_rows;   // [batch] block-table row
+    int B, K, n_q, n_kv, hd, mode;
+    int split_tokens, n_splits;   // n_splits = buffer stride (max splits)
+    float *part;             // [B*K][n_q][n_splits][hd]
+    float2 *ml;              // [B*K][n_q][n_splits]
+    unsigned *err;
+};
+
+struct Ctx {
+    orthrus_config_t cfg;
+    std::vector<orthrus_layer_weights_t> layers;
+    const void *embed, *final_norm, *lm_head;
+    int esize;               // bytes per element of the dtype
+    int R;                   // decode rows: max_batch * max_block
+    int Rw;                  // rows of the forward buffers: max(R, prefill chunk)
+    int n_splits;            // attention split stride
+    int n_vtiles;            // LM-head vocab tiles
+    int dev;
+    // workspace carve-up (device pointers)
+    float *h;                // [Rw][d]
+    void *a;                 // [Rw][d]
+    void *q;                 // [Rw][n_q*hd]
+    void *attn_o;            // [Rw][n_q*hd]
+    void *act;               // [Rw][F]
+    void *k_diff, *v_diff;   // [n_layers][R][n_kv][hd]
+    void *fin_draft, *fin_verify;  // [R][d]
+    void *res_x;             // [2*max_batch][d]
+    float *attn_part;        // [Rw][n_q][n_splits][hd]
+    float2 *attn_ml;         // [Rw][n_q][n_splits]
+    float *gemm_part;
+    size_t gemm_part_floats;
+    int *gemm_ticket;
+    int gemm_tickets;
+    LmPart *lm_part;         // [max(R, 2*max_batch)][n_vtiles]
+    int32_t *tok;            // [Rw] block tokens
+    int32_t *pos0;           // [max_batch]
+    int32_t *bt_rows;        // [max_batch] identity rows 0..max_batch-1
+    int32_t *prefill_row;    // [1]
+    int32_t *draft;          // [R]
+    float *logq, *lse_q;     // [R]
+    int32_t *g;              // [R]
+    float *logp, *lse_p;     // [R]
+    int32_t *rej_row;        // [max_batch]
+    int32_t *res_tok;        // [max_batch]
+    int *any_reject;         // [1]
+    unsigned *err;           // [1]
+    int32_t *produced;       // [max_batch]
+    int64_t *step;           // [1]
+    int32_t *n_buf, *tok_buf, *anchor_buf;  // generate scratch
+    // host-side measurement state
+    mutable uint64_t launches = 0;
+    int probe_family = -1, probe_layer = -1, probe_view = -1;
+    std::vector<cudaEvent_t> probe_start, probe_stop;
+    uint64_t probe_hits = 0;
+};
+
+struct Layout {
+    size_t total;
+    size_t off[40];
+};
+
+// workspace carve-up shared by orthrus_workspace_size and orthrus_create
+size_t plan_workspace(const orthrus_config_t &c, Ctx *ctx);
+
+int choose_splits(int N, int Kd);
+bool use_tensor_cores(const orthrus_config_t &c);
+
+// ---------------------------------------------------------------- launchers
+cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s);
+cudaError_t gemm_init_attributes();
+cudaError_t attention_init_attributes();
+cudaError_t launch_attention(const Ctx &c, const AttnArgs &a, cudaStream_t s);
+cudaError_t launch_embed(const Ctx &c, int mode, const int32_t *tokens, const int32_t *anchor,
+                         const int32_t *draft, int B, int K, cudaStream_t s);
+cudaError_t launch_rmsnorm(const Ctx &c, const float *h, const void *gain, void *out, int M, cudaStream_t s);
+cudaError_t launch_lm_finalize(const Ctx &c, int mode, int B, int K, float temperature, uint64_t seed,
+                               const int64_t *step, int32_t *tok_out, cudaStream_t s);
+cudaError_t launch_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int K, float temperature, uint64_t seed,
+                          int64_t *step, const int32_t *force_n, int32_t *n_out, int32_t *tokens_out,
+                          int32_t *anchor_io, int32_t *append_out, int append_stride, int append_max,
+                          cudaStream_t s);
+cudaError_t launch_ar_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int64_t *step,
+                             int32_t *token_out, int32_t *anchor_io, int32_t *append_out, int append_stride,
+                             int append_max, cudaStream_t s);
+cudaError_t launch_set_lens(const Ctx &c, int32_t *seq_lens, int b, int value, int32_t *anchor_out,
+                            const int32_t *tokens, cudaStream_t s);
+cudaError_t launch_logits_dump(const Ctx &c, const void *fin, int M, float *logits, cudaStream_t s);
+
+}  // namespace orthrus

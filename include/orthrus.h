@@ -1,0 +1,275 @@
+/*
+ * orthrus.h — C ABI of the B200 (sm_100a) dual-view decode library.
+ *
+ * One decode cycle of Orthrus ("Orthrus: Memory-Efficient Parallel Token
+ * Generation via Dual-View Diffusion"; the paper-notes page, §4.1) is three
+ * calls on one CUDA stream:
+ *
+ *   orthrus_draft_block   parallel projection: the diffusion view reads the
+ *                         block [anchor, mask x (K-1)] and proposes K tokens
+ *                         (§4.1 step 1);
+ *   orthrus_verify_block  AR verification: the frozen AR view reads
+ *                         [anchor, y_1 .. y_{K-1}] in one causal forward and
+ *                         writes its K/V into the cache tail (§4.1 step 2);
+ *   orthrus_commit        consensus: greedy prefix match (§4.2) or rejection
+ *                         sampling at T>0 (§4.3); the committed length grows
+ *                         by the n in [1, K] emitted tokens (§4.1 step 3).
+ *
+ * orthrus_prefill builds the shared cache with the AR view (§2.2);
+ * orthrus_ar_step is one step of plain AR decoding with the same kernels
+ * (the baseline the method must reproduce exactly at T = 0, §4.2, §9.1);
+ * orthrus_generate drives the whole loop.
+ *
+ * Conventions for every entry point:
+ *   - Every pointer to tensor data is a DEVICE pointer owned by the caller
+ *     unless the comment says "host".  The library never allocates or frees
+ *     device memory: its scratch lives in the caller's workspace.
+ *   - `stream` is a cudaStream_t passed as void*; all work is enqueued on it
+ *     and the calls return without synchronising, except where stated.
+ *   - Matrices are row-major [out][in] (the nn.Linear layout), in the
+ *     config's dtype (bf16 or fp32).  Norm gains are [hidden] in that dtype.
+ *   - Argument and capacity errors are found on the host before any launch
+ *     and returned synchronously; nothing is enqueued then.  Problems that
+ *     only the device can see (a token id out of range, a sequence that
+ *     would overflow its pages, a non-finite log-sum-exp) set bits of a
+ *     device error word and skip the offending write; orthrus_check_error
+ *     and orthrus_generate report them as ORTHRUS_ERR_DEVICE_CHECK /
+ *     ORTHRUS_ERR_NONFINITE.  No call aborts the process.
+ *   - A context is bound to one stream at a time and is not thread-safe.
+ */
+#ifndef ORTHRUS_H
+#define ORTHRUS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ORTHRUS_OK = 0,
+    ORTHRUS_ERR_INVALID_ARG = 1,   /* null pointer, bad size or shape */
+    ORTHRUS_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim) */
+    ORTHRUS_ERR_CAPACITY = 3,      /* batch, K, length or workspace too large */
+    ORTHRUS_ERR_CUDA = 4,          /* a CUDA runtime call failed */
+    ORTHRUS_ERR_DEVICE_CHECK = 5,  /* a device-side bounds/id check fired */
+    ORTHRUS_ERR_NONFINITE = 6      /* a log-sum-exp came out NaN or inf */
+} orthrus_status_t;
+
+typedef enum { ORTHRUS_BF16 = 0, ORTHRUS_FP32 = 1 } orthrus_dtype_t;
+
+/* Device error-word bits (orthrus_check_error's *bits). */
+#define ORTHRUS_DEVERR_TOKEN     0x1   /* token id outside [0, vocab) */
+#define ORTHRUS_DEVERR_CAPACITY  0x2   /* position beyond the sequence's pages */
+#define ORTHRUS_DEVERR_NONFINITE 0x4   /* non-finite log-sum-exp */
+
+/*
+ * Model shape and run limits.  The decoder is the pages' frozen AR backbone
+ * (pre-norm, RMSNorm, rotary positions, grouped-query attention, SwiGLU FFN,
+ * no biases) with one extra W_Q/W_K/W_V per layer for the diffusion view
+ * (paper notes §2.1).
+ *   head_dim     must be 16, 32, 64 or 128; 128 for the bf16 tensor-core path.
+ *   mask_token_id  id of the mask token that fills block rows 1..K-1 of a
+ *                draft (paper notes §4.1 step 1); an ordinary embedding row.
+ *   max_batch, max_block   largest batch and block size K a call may use.
+ *   max_seq      largest committed length + K a sequence may reach; sizes the
+ *                attention split buffers only (never the diffusion K/V).
+ *   split_tokens KV positions per attention split, a multiple of 64; fixed
+ *                for a run so a row's result never depends on the block it
+ *                sits in.
+ */
+typedef struct {
+    int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab, mask_token_id;
+    int32_t dtype;                 /* orthrus_dtype_t */
+    int32_t max_batch, max_block, max_seq, split_tokens;
+    float rope_theta, rms_eps;
+} orthrus_config_t;
+
+/* Device pointers of one layer.  wq/wk/wv: AR view; *_diff: diffusion view
+ * (paper notes §2.1).  Shapes: wq [n_q*hd][hidden], wk/wv [n_kv*hd][hidden],
+ * wo [hidden][n_q*hd], w_gate/w_up [ffn][hidden], w_down [hidden][ffn]. */
+typedef struct {
+    const void *attn_norm, *wq, *wk, *wv, *wq_diff, *wk_diff, *wv_diff;
+    const void *wo, *ffn_norm, *w_gate, *w_up, *w_down;
+} orthrus_layer_weights_t;
+
+/* embed [vocab][hidden], lm_head [vocab][hidden] (may equal embed when the
+ * head is tied), final_norm [hidden]; `layers` is a HOST array of n_layers
+ * entries, copied by orthrus_create. */
+typedef struct {
+    const void *embed, *final_norm, *lm_head;
+    const orthrus_layer_weights_t *layers;
+} orthrus_weights_t;
+
+/*
+ * The one shared KV cache (paper notes §2.2-2.3): AR keys (after RoPE) and
+ * values only, paged.
+ *   k_pages, v_pages  [n_layers][num_pages][n_kv][page_size][head_dim], dtype
+ *   block_table       [max_batch][max_pages_per_seq] int32 page ids
+ *   seq_lens          [max_batch] int32 committed length t of each sequence
+ *                     (the anchor's own K/V are not in the cache)
+ * page_size must be a multiple of 16 (of 64 on the bf16 path).
+ */
+typedef struct {
+    void *k_pages, *v_pages;
+    int32_t *block_table;
+    int32_t *seq_lens;
+    int32_t num_pages, page_size, max_pages_per_seq;
+} orthrus_kv_t;
+
+typedef struct orthrus_ctx orthrus_ctx_t;
+
+/* Host-side statistics filled by orthrus_generate. */
+typedef struct {
+    int64_t cycles;         /* decode cycles (2 forwards each; 1 for plain AR) */
+    int64_t forwards;       /* forward passes run after prefill */
+    int64_t tokens;         /* tokens emitted, summed over the batch */
+    int64_t min_tokens;     /* smallest per-sequence count reached */
+} orthrus_stats_t;
+
+/* Bytes of workspace a context needs for `cfg` (device memory the caller
+ * allocates, 256-byte aligned).  Independent of any sequence length. */
+orthrus_status_t orthrus_workspace_size(const orthrus_config_t *cfg, size_t *bytes);
+
+/* Bytes of the transient diffusion K/V of one draft of `batch` sequences
+ * and block size K across all layers: n_layers*batch*K*n_kv*hd*2*sizeof(dtype).
+ * The pages state this is constant in the sequence length (~4.5 MiB for the
+ * Qwen3-8B shape at K = 32; paper notes §2.3, §9.5). */
+orthrus_status_t orthrus_transient_bytes(const orthrus_config_t *cfg, int32_t batch, int32_t K,
+                                         size_t *bytes);
+
+/* Validates cfg, copies cfg and the weight pointers (the weights themselves
+ * stay caller-owned and must outlive the context), carves the workspace and
+ * zeroes its counters on the current device.  Synchronous. */
+orthrus_status_t orthrus_create(const orthrus_config_t *cfg, const orthrus_weights_t *weights,
+                                void *workspace, size_t ws_bytes, orthrus_ctx_t **out);
+orthrus_status_t orthrus_destroy(orthrus_ctx_t *ctx);
+
+/*
+ * AR prefill (paper notes §2.2): for each b < batch, runs the AR view
+ * causally over tokens[b][0 .. lens[b]-2], writing their K/V into the
+ * sequence's pages, sets seq_lens[b] = lens[b]-1 and anchor_out[b] =
+ * tokens[b][lens[b]-1].  tokens: device [batch][tok_stride]; lens: HOST
+ * [batch], each in [1, max_seq - max_block].
+ */
+orthrus_status_t orthrus_prefill(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, const int32_t *tokens,
+                                 int32_t tok_stride, const int32_t *lens, int32_t batch,
+                                 int32_t *anchor_out, void *stream);
+
+/*
+ * Parallel projection (paper notes §4.1 step 1, §3.2 mask): per sequence b,
+ * the block [anchor[b], mask x (K-1)] at positions t..t+K-1 (t = seq_lens[b])
+ * goes through the diffusion view; each block row attends to cache rows
+ * [0, t) and to every block row.  The block's K/V stay in the workspace and
+ * never enter the cache.  Writes draft [batch][K] int32: argmax per row at
+ * temperature 0, else a Gumbel-max sample of softmax(logits/T) keyed by
+ * (seed, *step, row).  step: device int64 (read only).
+ */
+orthrus_status_t orthrus_draft_block(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, const int32_t *anchor,
+                                     int32_t batch, int32_t K, float temperature, uint64_t seed,
+                                     const int64_t *step, int32_t *draft, void *stream);
+
+/*
+ * AR verification (paper notes §4.1 step 2): per sequence, the block
+ * [anchor, draft[0..K-2]] at positions t..t+K-1 through the AR view, causal
+ * (row k sees cache rows [0, t+k]).  Its K/V are written into cache slots
+ * t..t+K-1 (beyond the committed length until orthrus_commit).  Results stay
+ * in the workspace for orthrus_commit.  The pages for t+K positions must
+ * exist in block_table.
+ */
+orthrus_status_t orthrus_verify_block(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, const int32_t *anchor,
+                                      const int32_t *draft, int32_t batch, int32_t K, float temperature,
+                                      void *stream);
+
+/*
+ * Consensus and commit (paper notes §4.1 step 3, §4.2, §4.3) after a draft
+ * and a verify with the same batch, K and temperature.  Greedy: accept draft
+ * tokens while they equal the AR argmax; at the first mismatch j emit the AR
+ * argmax.  T>0: accept row k iff u_k < p_k(y_k)/q_k(y_k); at the first
+ * rejection draw the correction from norm(max(0, p_j - q_j)).  Writes
+ * n_out [batch] (in [1, K]), tokens_out [batch][K] (first n valid),
+ * anchor_io[b] = last emitted token, seq_lens[b] += n, and *step += 1.
+ * force_n (nullable, device [batch]) overrides n (tokens emitted are then
+ * the AR argmaxes), for measurements with a prescribed acceptance.
+ */
+orthrus_status_t orthrus_commit(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, int32_t batch, int32_t K,
+                                float temperature, uint64_t seed, int64_t *step, const int32_t *force_n,
+                                int32_t *n_out, int32_t *tokens_out, int32_t *anchor_io, void *stream);
+
+/*
+ * One plain AR decoding step with the same kernels: the AR view on
+ * [anchor[b]] at position seq_lens[b], then emit the argmax (T = 0) or a
+ * Gumbel-max sample keyed by (seed, *step) (T > 0).  Writes token_out
+ * [batch], anchor_io[b] = that token, seq_lens[b] += 1, *step += 1.
+ */
+orthrus_status_t orthrus_ar_step(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, int32_t batch,
+                                 float temperature, uint64_t seed, int64_t *step, int32_t *token_out,
+                                 int32_t *anchor_io, void *stream);
+
+/*
+ * Whole generation: prefill, then cycles of draft/verify/commit (K >= 1) or
+ * plain AR steps (K == 0) until every sequence has max_new tokens.
+ * prompt: device [batch][tok_stride]; lens: HOST [batch]; out: device
+ * [batch][max_new].  Synchronises the stream once per cycle (to read how many
+ * tokens were produced); returns a pending device error, if any.
+ */
+orthrus_status_t orthrus_generate(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, const int32_t *prompt,
+                                  int32_t tok_stride, const int32_t *lens, int32_t batch, int32_t K,
+                                  int32_t max_new, float temperature, uint64_t seed, int32_t *out,
+                                  orthrus_stats_t *stats, void *stream);
+
+/*
+ * The dual-view attention on its own (paper notes §3.2 and §4.1): block of
+ * K query rows per sequence at positions t..t+K-1 (t = seq_lens[b]).
+ *   q       [batch][K][n_q][hd]
+ *   mode 0  AR verify: keys/values are cache rows [0, t+k] for row k (the
+ *           block's rows must already be in the cache at t..t+K-1);
+ *   mode 1  diffusion draft: cache rows [0, t) plus all K rows of
+ *           k_blk/v_blk [batch][K][n_kv][hd].
+ *   out     [batch][K][n_q][hd]
+ * Uses the layer-`layer` slice of the cache and the context's workspace.
+ */
+orthrus_status_t orthrus_dual_view_attention(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, int32_t layer,
+                                             int32_t mode, const void *q, const void *k_blk,
+                                             const void *v_blk, int32_t batch, int32_t K, void *out,
+                                             void *stream);
+
+/*
+ * Test and measurement hook: the logits of the last verify (which = 0) or
+ * draft (which = 1) for every block row, fp32 [batch][K][vocab], computed
+ * from the final hidden rows the step kept (one extra LM-head pass; the
+ * decode path itself never writes logits).
+ */
+orthrus_status_t orthrus_debug_logits(orthrus_ctx_t *ctx, int32_t which, int32_t batch, int32_t K,
+                                      float *logits, void *stream);
+
+/*
+ * Measurement hook.  While set, every forward of `view` (0 = AR: verify,
+ * prefill and plain AR steps; 1 = diffusion draft) records caller-owned CUDA
+ * events (cudaEvent_t passed as void*) on the launch stream around the
+ * launches of layer `layer`: starts[i] just before and stops[i] just after
+ * launch i of kernel family `family` (0 = the four projection GEMMs in the
+ * order QKV, O, gate/up, down; 1 = the attention split and combine kernels
+ * as one bracket).  Slots are used cyclically (i = hit mod n).  n = 0
+ * disables the probe.  The arrays are copied; the events must outlive the
+ * probe.  Not for use while a stream is being captured.
+ */
+orthrus_status_t orthrus_set_probe(orthrus_ctx_t *ctx, int32_t family, int32_t layer, int32_t view,
+                                   void *const *starts, void *const *stops, int32_t n);
+
+/* Number of kernel launches the context has enqueued since orthrus_create
+ * (host-side count; a CUDA-graph replay of captured calls adds nothing). */
+uint64_t orthrus_launch_count(const orthrus_ctx_t *ctx);
+
+/* Synchronises `stream`, returns and clears the device error word (*bits may
+ * be NULL). */
+orthrus_status_t orthrus_check_error(orthrus_ctx_t *ctx, void *stream, uint32_t *bits);
+
+const char *orthrus_status_string(orthrus_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ORTHRUS_H */

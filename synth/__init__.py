@@ -173,3 +173,40 @@ def make_weights(s: ModelShape, seed: int, n_layers: int | None = None,
 def make_prompt(s: ModelShape, length: int, seed: int, name: str = "prompt") -> np.ndarray:
     """Uniform random prompt over [0, vocab - 1) (the mask id never appears)."""
     return uniform_ids(length, s.vocab - 1, seed, name)
+
+
+def make_weights_torch(s: ModelShape, seed: int, device="cuda", n_layers: int | None = None):
+    """Device-side draw of the same recipe for shapes too large for the host
+    generator (the 8B shape has 9.1e9 parameters): torch's Philox generator
+    on the device, seeded per tensor from (seed, name); values drawn in fp32,
+    the diffusion copy formed in fp32 and rounded once to the model dtype.
+    The values differ from make_weights' (a different generator) but follow
+    the same distributions; tests that compare against the oracle copy the
+    pieces they need back to the host."""
+    import torch
+    L = s.n_layers if n_layers is None else n_layers
+    d, hq, hkv, hd, F, V = s.hidden, s.n_q_heads, s.n_kv_heads, s.head_dim, s.ffn, s.vocab
+    dt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
+    gen = torch.Generator(device=device)
+
+    def draw(shape, std, name):
+        gen.manual_seed((int(seed) << 32) | zlib.crc32(name.encode()))
+        return torch.randn(shape, generator=gen, device=device, dtype=torch.float32).mul_(std)
+
+    embed = draw((V, d), s.std, "embed").to(dt)
+    lm_head = embed if s.tied else draw((V, d), s.std, "lm_head").to(dt)
+    ones = torch.ones(d, device=device, dtype=dt)
+    layers = []
+    for l in range(L):
+        lw = {"attn_norm": ones, "ffn_norm": ones}
+        for key, rows in (("wq", hq * hd), ("wk", hkv * hd), ("wv", hkv * hd)):
+            base = draw((rows, d), s.std, f"L{l}.{key}")
+            lw[key] = base.to(dt)
+            lw[key + "_diff"] = base.add_(draw((rows, d), s.sigma_diff, f"L{l}.{key}_diff_noise")).to(dt)
+            del base
+        lw["wo"] = draw((d, hq * hd), s.std, f"L{l}.wo").to(dt)
+        lw["w_gate"] = draw((F, d), s.std, f"L{l}.w_gate").to(dt)
+        lw["w_up"] = draw((F, d), s.std, f"L{l}.w_up").to(dt)
+        lw["w_down"] = draw((d, F), s.std, f"L{l}.w_down").to(dt)
+        layers.append(lw)
+    return Weights(s, embed, ones, lm_head, layers)

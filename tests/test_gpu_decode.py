@@ -1,0 +1,177 @@
+"""The whole decode cycle on the GPU (paper notes §4.1-§4.3) against the CPU
+oracle and against the library's own plain AR decoding.
+
+* tiny fp32 model: token streams equal to the oracle's (greedy and T = 1,
+  seed 1); a divergence is only accepted at a decision whose oracle margin
+  is below what fp32 rounding can flip;
+* bf16 models: greedy Orthrus equals the GPU's plain AR greedy token for
+  token (paper notes §4.2, §9.1); draft and verify logits within 2e-2
+  (relative to the row's largest |logit|) of the fp64 oracle.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+FP32_MARGIN = 1e-4     # decisions closer than this may legitimately flip in fp32
+
+
+@pytest.fixture(scope="module")
+def pkg():
+    import dual_view_diffusion_b200 as p
+    p.lib()
+    return p
+
+
+def _first_diff(a, b):
+    d = np.nonzero(np.asarray(a) != np.asarray(b))[0]
+    return int(d[0]) if d.size else -1
+
+
+@pytest.fixture(scope="module")
+def tiny(pkg):
+    w = synth.make_weights(synth.TINY, 0)
+    eng = pkg.Engine(synth.TINY, w, max_batch=2, max_block=8, max_seq=160, split_tokens=64, page_size=16)
+    return w, eng
+
+
+@pytest.mark.parametrize("T,seed", [(0.0, 0), (1.0, 1)])
+def test_tiny_fp32_stream_matches_oracle(tiny, T, seed):
+    w, eng = tiny
+    prompt = synth.make_prompt(synth.TINY, 16, 0)
+    out, st = eng.generate(torch.from_numpy(prompt)[None], 4, 32, T, seed)
+    ref = oracle.Model(w).generate(prompt, 4, 32, T, seed, "orthrus")
+    got = out[0].cpu().numpy()
+    i = _first_diff(got, ref["tokens"])
+    assert i < 0 or ref["min_margin"] < FP32_MARGIN, (i, got, ref["tokens"])
+    assert st["cycles"] == ref["cycles"] or i >= 0
+    assert eng.check_error()[0] == 0
+
+
+def test_tiny_fp32_plain_ar_matches_oracle(tiny):
+    w, eng = tiny
+    prompt = synth.make_prompt(synth.TINY, 16, 0)
+    out, st = eng.generate(torch.from_numpy(prompt)[None], 0, 32, 0.0, 0)
+    ref = oracle.Model(w).generate(prompt, 4, 32, 0.0, 0, "ar")
+    assert np.array_equal(out[0].cpu().numpy(), ref["tokens"])
+    assert st["forwards"] == 32
+
+
+@pytest.mark.parametrize("K", [1, 2, 4, 8])
+def test_tiny_orthrus_equals_ar_on_gpu(tiny, K):
+    _, eng = tiny
+    prompt = torch.from_numpy(synth.make_prompt(synth.TINY, 16, 3))[None]
+    o, st = eng.generate(prompt, K, 40, 0.0, 0)
+    a, _ = eng.generate(prompt, 0, 40, 0.0, 0)
+    assert torch.equal(o, a)
+    assert st["forwards"] == 2 * st["cycles"]
+    assert 0.5 <= 40 / st["forwards"] <= K / 2 or K == 1
+
+
+def test_tiny_batch_ragged(tiny):
+    """Two sequences with different prompt lengths decode independently."""
+    w, eng = tiny
+    p0 = synth.make_prompt(synth.TINY, 16, 0)
+    p1 = synth.make_prompt(synth.TINY, 9, 7)
+    prompts = np.zeros((2, 16), np.int32)
+    prompts[0] = p0
+    prompts[1, :9] = p1
+    out, _ = eng.generate(torch.from_numpy(prompts), 4, 24, 0.0, 0, lens=[16, 9])
+    m = oracle.Model(w)
+    for b, p in enumerate((p0, p1)):
+        ref = m.generate(p, 4, 24, 0.0, 0, "orthrus")
+        i = _first_diff(out[b].cpu().numpy(), ref["tokens"])
+        assert i < 0 or ref["min_margin"] < FP32_MARGIN, (b, i)
+
+
+def test_tiny_step_api_and_cache_commit(tiny):
+    """The three-call cycle through the public entry points: committed length
+    grows by n, the committed K/V equal the plain-AR run's, and nothing past
+    the committed length + K is touched."""
+    _, eng = tiny
+    prompt = torch.from_numpy(synth.make_prompt(synth.TINY, 16, 0))[None]
+    eng.k_pages.zero_(); eng.v_pages.zero_()
+    anchor = eng.prefill(prompt)
+    eng.step.zero_()
+    total = 0
+    for _ in range(6):
+        t0 = int(eng.seq_lens[0])
+        draft = eng.draft_block(anchor, 4)
+        eng.verify_block(anchor, draft, 4)
+        n, toks = eng.commit(anchor, 4)
+        n = int(n[0])
+        assert 1 <= n <= 4 and int(eng.seq_lens[0]) == t0 + n
+        total += n
+    t = int(eng.seq_lens[0])
+    k_o = eng.k_pages.clone()
+    # untouched beyond t + K (the last verify wrote up to t_prev + K - 1)
+    ps = eng.page_size
+    flat = eng.k_pages[:, 0:eng.pages_per_seq].permute(0, 1, 3, 2, 4).reshape(eng.n_layers, -1, 2, 16)
+    assert flat[:, t + 4:].abs().sum() == 0
+    # plain AR to the same length gives the same committed K/V (bitwise)
+    eng.k_pages.zero_(); eng.v_pages.zero_()
+    anchor = eng.prefill(prompt)
+    for _ in range(total):
+        eng.ar_step(anchor)
+    flat_ar = eng.k_pages[:, 0:eng.pages_per_seq].permute(0, 1, 3, 2, 4).reshape(eng.n_layers, -1, 2, 16)
+    flat_o = k_o[:, 0:eng.pages_per_seq].permute(0, 1, 3, 2, 4).reshape(eng.n_layers, -1, 2, 16)
+    assert torch.equal(flat_ar[:, :t], flat_o[:, :t])
+
+
+def _logits_case(pkg, shape, n_layers, P, K, seed):
+    w = synth.make_weights(shape, seed, n_layers=n_layers)
+    eng = pkg.Engine(shape, w, max_batch=1, max_block=K, max_seq=P + 2 * K + 8, split_tokens=64, page_size=64)
+    prompt = synth.make_prompt(shape, P, seed)
+    anchor = eng.prefill(torch.from_numpy(prompt)[None])
+    draft = eng.draft_block(anchor, K)
+    dl = eng.debug_logits(1, 1, K)[0].cpu().numpy()
+    blk = synth.make_prompt(shape, K, seed + 1, "block")        # any ids will do for the verify check
+    eng.verify_block(anchor, torch.from_numpy(blk[None]).cuda(), K)
+    vl = eng.debug_logits(0, 1, K)[0].cpu().numpy()
+    assert eng.check_error()[0] == 0
+    m = oracle.Model(w)
+    kc, vc = m.new_cache(P + 2 * K)
+    t = m.prefill(prompt, kc, vc)
+    ref_d = m.forward(1, 1, [prompt[-1]] + [shape.mask_id] * (K - 1), t, kc.copy(), vc.copy())
+    ref_v = m.forward(0, 0, [prompt[-1]] + list(blk[:K - 1]), t, kc.copy(), vc.copy())
+    rel = lambda g, r: float((np.abs(g - r).max(axis=1) / np.abs(r).max(axis=1)).max())
+    return rel(dl, ref_d), rel(vl, ref_v), draft[0].cpu().numpy(), ref_d
+
+
+def test_bf16_logits_vs_oracle_1p7b_width(pkg):
+    """Two layers of the Qwen3-1.7B shape (full width, full vocabulary,
+    tied head), prompt 80, K = 32."""
+    s = synth.QWEN3_1_7B
+    ed, ev, draft, ref_d = _logits_case(pkg, s, 2, 80, 32, 0)
+    assert ed <= 2e-2 and ev <= 2e-2, (ed, ev)
+
+
+def test_bf16_logits_vs_oracle_ragged(pkg):
+    """A small bf16 model whose sizes leave ragged tiles everywhere."""
+    s = dataclasses.replace(synth.QWEN3_8B, n_layers=2, hidden=320, n_q_heads=4, n_kv_heads=2, ffn=704,
+                            vocab=1000)
+    ed, ev, _, _ = _logits_case(pkg, s, 2, 70, 5, 3)
+    assert ed <= 2e-2 and ev <= 2e-2, (ed, ev)
+
+
+@pytest.mark.parametrize("shape,P,N", [(synth.QWEN3_1_7B, 512, 256), (synth.QWEN3_8B, 2048, 512)])
+def test_bf16_orthrus_equals_plain_ar(pkg, shape, P, N):
+    """Full-depth random-init Qwen3 shapes, K = 32, greedy: the Orthrus
+    stream equals the GPU's own plain-AR stream token for token."""
+    w = synth.make_weights_torch(shape, 0)
+    eng = pkg.Engine(shape, w, max_batch=1, max_block=32, max_seq=P + N + 64, split_tokens=256)
+    prompt = torch.from_numpy(synth.make_prompt(shape, P, 0))[None]
+    o, st = eng.generate(prompt, 32, N, 0.0, 0)
+    a, sa = eng.generate(prompt, 0, N, 0.0, 0)
+    assert eng.check_error()[0] == 0
+    i = _first_diff(o[0].cpu().numpy(), a[0].cpu().numpy())
+    assert i < 0, (i, st)
+    assert st["forwards"] == 2 * st["cycles"] and sa["forwards"] == N
+    del eng, w
+    torch.cuda.empty_cache()
