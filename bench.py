@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the Orthrus dual-view decode step on B200.
+
+Workload (one GPU): the Qwen3-8B shape (36 layers, hidden 4096, 32/8 heads,
+head_dim 128, FFN 12288, vocab 151936), random-init bf16 weights, batch 1,
+block K = 32, a 2048-token uniform random prompt prefilled before timing,
+greedy decoding.  One step = one decode cycle: draft (diffusion view),
+verify (AR view), consensus and commit ("Orthrus: Memory-Efficient Parallel
+Token Generation via Dual-View Diffusion", paper notes §4.1).
+
+value     committed tokens/s over the timed steps (device time, CUDA events,
+          max over ranks; N ranks run independent replicas)
+e2e       the same metric with the step's input (anchor id) copied from
+          pinned host memory and its result (n and the tokens) read back
+          every step, through the library's public calls
+roofline  the projection GEMMs (the dominant kernels: ~95% of a step's HBM
+          traffic is weight streaming), timed live by CUDA events around one
+          layer's four projection launches in every verify forward of the
+          timed region; algorithmic bytes = weights + activations in/out
+attn      the dual-view attention kernels (split + combine) of one layer,
+          timed the same way; bytes = prefix K/V + Q + O
+cpu_baseline  the CPU oracle, as it stands, timed on a bounded sample (one
+          layer of each view at full width plus 1/16 of the LM head) and
+          scaled to a full step
+
+Weights and the prompt are larger than L2 (18 GB of weights per step), so no
+flush is needed between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "committed tokens/s (batch 1, Qwen3-8B shape, K=32); dual-view attn HBM GB/s"
+UNIT = "tokens/s"
+P_PROMPT, K_BLOCK, BATCH = 2048, 32, 1
+# tokens committed per cycle that this random-init 8B workload gives (the
+# mean accepted length measured on the GPU path; greedy decoding is
+# deterministic, so any correct implementation commits the same tokens).
+# Used only by the reference arm, which cannot run the whole model.
+N_BAR_WORKLOAD = 2.0
+SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--temperature", type=float, default=0.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-small", action="store_true",
+                    help="small case for ncu captures: 2 layers of the 8B shape, vocab 32000, 2 steps; "
+                         "its line is marked profile_case and is not a bench result")
+    a = ap.parse_args()
+    if a.profile_small:
+        a.steps, a.warmup, a.no_cpu_baseline, a.no_e2e = 2, 1, True, True
+    return a
+
+
+# ----------------------------------------------------------------- helpers
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    def __init__(self, index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.index = index
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={SMI_FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.p:
+            self.p.terminate()
+            try:
+                self.p.wait(5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+
+    def summary(self):
+        self.f.flush()
+        rows = [l.split(",") for l in open(self.f.name).read().splitlines() if l.strip()]
+        os.unlink(self.f.name)
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        sm, mx, reasons = [], None, set()
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gemm_bytes(s, M):
+    """Algorithmic HBM bytes of the four projection launches of one layer
+    (QKV, O, gate/up, down) for M token rows, bf16: weights once, activations
+    in and out, fp32 residual read+write."""
+    d, hq, hk, F = s.hidden, s.n_q_heads * s.head_dim, s.n_kv_heads * s.head_dim, s.ffn
+    qkv = (hq + 2 * hk) * d * 2 + M * d * 2 + M * (hq + 2 * hk) * 2
+    o = d * hq * 2 + M * hq * 2 + M * d * 4 * 2
+    gu = 2 * F * d * 2 + M * d * 2 + M * F * 2
+    dn = d * F * 2 + M * F * 2 + M * d * 4 * 2
+    return [qkv, o, gu, dn]
+
+
+def attn_bytes(s, t, K, B=1):
+    """Algorithmic bytes of one verify attention call: keys/values [0, t+K)
+    of every KV head read once, Q read, O written (bf16)."""
+    return B * ((t + K) * s.n_kv_heads * s.head_dim * 2 * 2 + 2 * K * s.n_q_heads * s.head_dim * 2)
+
+
+def kernel_traffic(name, source):
+    """DRAM bytes per launch recorded by an ncu capture of this kernel, valid
+    only while the kernel source is unchanged (sha256 recorded with it)."""
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None
+    rec = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            rec[k.strip()] = v.strip()
+    sha = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()
+    if rec.get("kernel_source_sha256") != sha:
+        return None
+    try:
+        return float(rec["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ----------------------------------------------------------------- oracle sample
+class OracleSample:
+    """The CPU oracle, as it stands, on a bounded sample of one decode step
+    of the 8B shape: one layer of each view at full width over n_rows block
+    rows against a 2047-row prefix, plus the LM head over 1/head_slice of the
+    vocabulary.  The full step is estimated by scaling: x36 layers, x32/n_rows
+    rows, x head_slice for the head.  Weights are drawn once, in fp32 (the
+    oracle computes in fp64 whatever the stored precision)."""
+
+    def __init__(self, head_slice=16):
+        import oracle
+        import synth
+        s8 = synth.QWEN3_8B
+        self.s8, self.head_slice = s8, head_slice
+        self.s = dataclasses.replace(s8, vocab=s8.vocab // head_slice, dtype="fp32")
+        self.m = oracle.Model(synth.make_weights(self.s, 0, n_layers=1))
+        self.t = P_PROMPT - 1
+        self.synth = synth
+
+    def step_seconds(self, n_rows=32):
+        s, t = self.s, self.t
+        cap = t + n_rows
+        kc = self.synth.normal((1, cap, s.n_kv_heads, s.head_dim), 1.0, 3, "bench.kc")
+        vc = self.synth.normal((1, cap, s.n_kv_heads, s.head_dim), 1.0, 3, "bench.vc")
+        prompt = self.synth.make_prompt(s, n_rows, 0)
+        draft_blk = [int(prompt[0])] + [s.mask_id] * (n_rows - 1)
+        t0 = time.perf_counter()
+        self.m.forward(1, 1, draft_blk, t, kc.copy(), vc.copy(), logits=False)
+        t1 = time.perf_counter()
+        self.m.forward(0, 0, prompt, t, kc.copy(), vc.copy(), logits=False)
+        t2 = time.perf_counter()
+        self.m.forward(0, 0, prompt, t, kc.copy(), vc.copy(), logits=True)
+        t3 = time.perf_counter()
+        layer = (t1 - t0) + (t2 - t1)
+        head = max(t3 - t2 - (t2 - t1), 0.0)
+        scale_rows = 32 / n_rows
+        return scale_rows * (self.s8.n_layers * layer + 2 * self.head_slice * head)
+
+    def describe(self, n_rows):
+        return (f"one layer of each view of the Qwen3-8B shape at full width, {n_rows} block rows over a "
+                f"{self.t}-row prefix, plus the LM head over 1/{self.head_slice} of the vocabulary; scaled "
+                f"x{self.s8.n_layers} layers, x{32 / n_rows:g} rows, x{self.head_slice} head")
+
+    @staticmethod
+    def threads():
+        return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def reduce_replicas(tokens, ms, e2e_value, world, device):
+    """Replicas only: every rank decodes its own sequence with its own copy
+    of the weights; no data moves between GPUs.  The job's throughput is
+    the tokens of all ranks over the slowest rank's device time, and the
+    end-to-end throughputs add.  Statistics only (one all-reduce each, after
+    the timed region)."""
+    if world == 1:
+        return tokens, ms, e2e_value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(tokens), float(e2e_value)], dtype=torch.float64, device=device)
+    m = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t)
+    dist.all_reduce(m, op=dist.ReduceOp.MAX)
+    return int(round(t[0].item())), float(m.item()), float(t[1].item())
+
+
+# ----------------------------------------------------------------- arms
+def run_reference(args, rank, world):
+    """The oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    samples = []
+    n_rows = 4 if args.steps + args.warmup > 24 else 32
+    sample = OracleSample()
+    for i in range(args.warmup + args.steps):
+        est = sample.step_seconds(n_rows)
+        if i >= args.warmup:
+            samples.append(est)
+    sec = statistics.mean(samples)
+    desc, threads = sample.describe(n_rows), sample.threads()
+    value = N_BAR_WORKLOAD / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "qwen3-8b-shape decode step, batch 1, K=32, prompt 2048, greedy",
+                       "global_batch": BATCH, "seq_len": P_PROMPT, "parallelism": "host cores"},
+            "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT, "cores": threads,
+                             "sample": desc + f"; tokens per step = {N_BAR_WORKLOAD} (this workload's "
+                                              "mean accepted length)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import dual_view_diffusion_b200 as pkg
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    s = synth.QWEN3_8B
+    if args.profile_small:
+        s = dataclasses.replace(s, n_layers=2, vocab=32000)
+    W, K, T = args.warmup, args.steps, args.temperature
+    n_e2e = 0 if args.no_e2e else K
+    max_seq = P_PROMPT + (W + K + n_e2e + 2) * K_BLOCK + K_BLOCK
+    w = synth.make_weights_torch(s, 0, device=dev)
+    eng = pkg.Engine(s, w, max_batch=BATCH, max_block=K_BLOCK, max_seq=max_seq, split_tokens=256,
+                     page_size=64, device=dev)
+    prompt = torch.from_numpy(synth.make_prompt(s, P_PROMPT, 100 + rank))[None].to(dev)
+    anchor = eng.prefill(prompt)
+    eng.step.zero_()
+    draft = torch.empty((BATCH, K_BLOCK), dtype=torch.int32, device=dev)
+    toks = torch.empty((BATCH, K_BLOCK), dtype=torch.int32, device=dev)
+    n_hist = torch.zeros((K + 1, BATCH), dtype=torch.int32, device=dev)
+
+    def step(i_hist):
+        eng.draft_block(anchor, K_BLOCK, T, 1234, out=draft)
+        eng.verify_block(anchor, draft, K_BLOCK, T)
+        eng.commit(anchor, K_BLOCK, T, 1234, n_out=n_hist[i_hist], tokens_out=toks)
+
+    for _ in range(W):
+        step(K)
+    torch.cuda.synchronize()
+    t_start = int(eng.seq_lens[0])
+
+    # live probes: one middle layer of every verify forward
+    probe_layer = s.n_layers // 2
+    mk = lambda n: [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    g0, g1 = mk(4 * K), mk(4 * K)
+    a0, a1 = mk(K), mk(K)
+    eng.set_probe(0, probe_layer, 0, g0, g1)
+    eng.set_probe(1, probe_layer, 0, a0, a1)
+    launches0 = eng.launch_count()
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        ev0.record()
+        for i in range(K):
+            step(i)
+        ev1.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = ev0.elapsed_time(ev1)
+    launches = eng.launch_count() - launches0
+    eng.set_probe(0, 0, 0, [], [])
+    eng.set_probe(1, 0, 0, [], [])
+    n = n_hist[:K].sum(dim=1).cpu().numpy()          # per step, summed over the batch
+    tokens = int(n.sum())
+    st, bits = eng.check_error()
+    if st != 0:
+        raise RuntimeError(f"device error bits {bits:#x}")
+
+    # projections: bytes per launch / live event durations
+    gb = gemm_bytes(s, BATCH * K_BLOCK)
+    g_ms = np.array([g0[i].elapsed_time(g1[i]) for i in range(4 * K)]).reshape(K, 4)
+    g_bytes = sum(gb) * K
+    g_time = g_ms.sum() * 1e-3
+    # attention: t per step from the committed history
+    t_steps = t_start + np.concatenate([[0], np.cumsum(n)[:-1]])
+    a_ms = np.array([a0[i].elapsed_time(a1[i]) for i in range(K)])
+    a_bytes = sum(attn_bytes(s, int(t), K_BLOCK) for t in t_steps)
+    a_time = a_ms.sum() * 1e-3
+
+    # ---------------------------------------------------------------- e2e
+    e2e = None
+    if n_e2e:
+        h_anchor = torch.empty(BATCH, dtype=torch.int32).pin_memory()
+        h_res = torch.empty((BATCH, 1 + K_BLOCK), dtype=torch.int32).pin_memory()
+        d_res = torch.empty((BATCH, 1 + K_BLOCK), dtype=torch.int32, device=dev)
+        h_anchor.copy_(anchor.cpu())
+        e2e_tokens = 0
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_e2e):
+            anchor.copy_(h_anchor, non_blocking=True)
+            eng.draft_block(anchor, K_BLOCK, T, 1234, out=draft)
+            eng.verify_block(anchor, draft, K_BLOCK, T)
+            eng.commit(anchor, K_BLOCK, T, 1234, n_out=d_res[:, 0], tokens_out=toks)
+            d_res[:, 1:].copy_(toks)
+            h_res.copy_(d_res, non_blocking=True)
+            torch.cuda.current_stream().synchronize()
+            nb = h_res[:, 0]
+            e2e_tokens += int(nb.sum())
+            for b in range(BATCH):   # the host feeds back the last committed token
+                h_anchor[b] = h_res[b, int(nb[b])]
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        e2e = {"value": e2e_tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": 4 * BATCH,
+               "d2h_bytes_per_step": 4 * BATCH * (1 + K_BLOCK), "ms_per_step": e2e_ms / n_e2e}
+
+    # ---------------------------------------------------------------- reduce
+    tot_tokens, max_ms, e2e_sum = reduce_replicas(tokens, ms, e2e["value"] if e2e else 0.0, world, dev)
+    if e2e:
+        e2e["value"] = e2e_sum
+    if rank != 0:
+        return
+    hbm, tflops, src = measured_peaks()
+    g_ach = g_bytes / g_time / 1e9
+    a_ach = a_bytes / a_time / 1e9
+    traffic = kernel_traffic("gemm_projection_qwen3_8b_shape.txt", "dual_view_diffusion_b200/csrc/gemm.cu")
+    value = tot_tokens / (max_ms * 1e-3)
+    nbar = tokens / (K * BATCH)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (random-init weights, uniform random prompt)",
+        "config": {"workload": "qwen3-8b-shape decode step (draft + verify + commit), batch 1 per GPU, K=32, "
+                               "prompt 2048, greedy", "global_batch": BATCH * world, "seq_len": P_PROMPT,
+                   "block_K": K_BLOCK, "parallelism": f"replicas x{world}",
+                   "l2": "weights (18 GB) and cache exceed L2 every step; no flush"},
+        "mean_accepted_per_cycle": nbar, "tokens_per_forward": nbar / 2,
+        "modelled_tokens_per_s_at_pages_acceptance": 10.8 / (max_ms / K * 1e-3),
+        "roofline": {"kernel": "projection GEMMs (QKV, O, gate/up, down) of one layer, verify view", "bound": "hbm",
+                     "achieved": g_ach, "peak": hbm, "unit": "GB/s", "frac": g_ach / hbm,
+                     "traffic": traffic, "peak_source": src, "algorithmic_bytes_per_layer": sum(gb),
+                     "ms_per_layer": float(g_ms.sum(axis=1).mean())},
+        "attn": {"kernel": "dual-view attention (split + combine), verify view, one layer", "bound": "hbm",
+                 "achieved": a_ach, "peak": hbm, "unit": "GB/s", "frac": a_ach / hbm,
+                 "us_per_call": float(a_ms.mean() * 1e3), "mean_prefix": float(t_steps.mean())},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if args.profile_small:
+        line = {"profile_case": True, "config": "2 layers of the Qwen3-8B shape, vocab 32000", "value": value,
+                "roofline": line["roofline"], "attn": line["attn"]}
+    if not args.no_cpu_baseline and world == 1:
+        sample = OracleSample()
+        est = sample.step_seconds(32)
+        line["cpu_baseline"] = {"value": nbar / est, "unit": UNIT, "cores": sample.threads(), "kind": "oracle",
+                                "sample": sample.describe(32) + f"; tokens per step = {nbar:.3f} (this run's mean)",
+                                "seconds_per_step": est}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -308,6 +308,9 @@ class Engine:
         family in one layer of every forward of `view` (see
         orthrus_set_probe); empty lists disable it."""
         n = len(starts)
+        for e in list(starts) + list(stops):
+            if not e.cuda_event:       # torch creates the CUDA event on first record
+                e.record()
         S = (C.c_void_p * max(n, 1))(*[e.cuda_event for e in starts])
         E = (C.c_void_p * max(n, 1))(*[e.cuda_event for e in stops])
         _check("orthrus_set_probe", lib().orthrus_set_probe(self.ctx, family, layer, view, S, E, n))

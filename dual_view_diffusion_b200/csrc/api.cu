@@ -136,23 +136,21 @@ static KvView kv_view(const orthrus_kv_t &kv)
 // Event probe (orthrus_set_probe): bracket a launch of the probed family in
 // the probed layer and view.
 struct ProbeScope {
-    Ctx &c;
+    Ctx::Probe &p;
     bool on;
     size_t slot;
     cudaStream_t s;
-    ProbeScope(Ctx &c_, int family, int layer, int view, cudaStream_t s_)
-        : c(c_), on(!c_.probe_start.empty() && c_.probe_family == family && c_.probe_layer == layer &&
-                    c_.probe_view == view),
-          slot(0), s(s_)
+    ProbeScope(Ctx &c, int family, int layer, int view, cudaStream_t s_)
+        : p(c.probe[family]), on(!p.start.empty() && p.layer == layer && p.view == view), slot(0), s(s_)
     {
         if (on) {
-            slot = c.probe_hits++ % c.probe_start.size();
-            cudaEventRecord(c.probe_start[slot], s);
+            slot = p.hits++ % p.start.size();
+            cudaEventRecord(p.start[slot], s);
         }
     }
     ~ProbeScope()
     {
-        if (on) cudaEventRecord(c.probe_stop[slot], s);
+        if (on) cudaEventRecord(p.stop[slot], s);
     }
 };
 
@@ -438,15 +436,18 @@ orthrus_status_t orthrus_set_probe(orthrus_ctx_t *c, int32_t family, int32_t lay
     if (!c || n < 0 || (n > 0 && (!starts || !stops))) return ORTHRUS_ERR_INVALID_ARG;
     if (n > 0 && (family < 0 || family > 1 || layer < 0 || layer >= c->cfg.n_layers || view < 0 || view > 1))
         return ORTHRUS_ERR_INVALID_ARG;
-    c->probe_start.clear();
-    c->probe_stop.clear();
-    c->probe_hits = 0;
+    if (family < 0 || family > 1) return ORTHRUS_ERR_INVALID_ARG;
+    Ctx::Probe &p = c->probe[family];
+    p.start.clear();
+    p.stop.clear();
+    p.hits = 0;
     for (int i = 0; i < n; ++i) {
-        if (!starts[i] || !stops[i]) { c->probe_start.clear(); c->probe_stop.clear(); return ORTHRUS_ERR_INVALID_ARG; }
-        c->probe_start.push_back((cudaEvent_t)starts[i]);
-        c->probe_stop.push_back((cudaEvent_t)stops[i]);
+        if (!starts[i] || !stops[i]) { p.start.clear(); p.stop.clear(); return ORTHRUS_ERR_INVALID_ARG; }
+        p.start.push_back((cudaEvent_t)starts[i]);
+        p.stop.push_back((cudaEvent_t)stops[i]);
     }
-    c->probe_family = family; c->probe_layer = layer; c->probe_view = view;
+    p.layer = layer;
+    p.view = view;
     return ORTHRUS_OK;
 }
 

@@ -139,9 +139,11 @@ struct Ctx {
     int32_t *n_buf, *tok_buf, *anchor_buf;  // generate scratch
     // host-side measurement state
     mutable uint64_t launches = 0;
-    int probe_family = -1, probe_layer = -1, probe_view = -1;
-    std::vector<cudaEvent_t> probe_start, probe_stop;
-    uint64_t probe_hits = 0;
+    struct Probe {
+        int layer = -1, view = -1;
+        std::vector<cudaEvent_t> start, stop;
+        uint64_t hits = 0;
+    } probe[2];                 // 0: projection GEMMs, 1: attention
 };
 
 struct Layout {

@@ -251,8 +251,8 @@ orthrus_status_t orthrus_debug_logits(orthrus_ctx_t *ctx, int32_t which, int32_t
  * launches of layer `layer`: starts[i] just before and stops[i] just after
  * launch i of kernel family `family` (0 = the four projection GEMMs in the
  * order QKV, O, gate/up, down; 1 = the attention split and combine kernels
- * as one bracket).  Slots are used cyclically (i = hit mod n).  n = 0
- * disables the probe.  The arrays are copied; the events must outlive the
+ * as one bracket).  Each family has its own probe; slots are used
+ * cyclically (i = hit mod n).  n = 0 disables that family's probe.  The arrays are copied; the events must outlive the
  * probe.  Not for use while a stream is being captured.
  */
 orthrus_status_t orthrus_set_probe(orthrus_ctx_t *ctx, int32_t family, int32_t layer, int32_t view,

@@ -247,13 +247,14 @@ class Model:
         sz = (self.n_layers, cap, s.n_kv_heads, s.head_dim)
         return np.zeros(sz), np.zeros(sz)
 
-    def forward(self, view, mode, tokens, t, kc, vc, want_hidden=False):
+    def forward(self, view, mode, tokens, t, kc, vc, want_hidden=False, logits=True):
         """One forward of a block; kc/vc are modified in place (mode 0 writes
-        rows t .. t+R-1).  Returns logits [R, V] (and final hidden rows)."""
+        rows t .. t+R-1).  Returns logits [R, V] (and final hidden rows);
+        logits=False skips the LM head and returns None for them."""
         tok = _i32(tokens)
         R = tok.size
         cap = kc.shape[1]
-        logits = np.empty((R, self.shape.vocab))
+        logits = np.empty((R, self.shape.vocab)) if logits else None
         hid = np.empty((R, self.shape.hidden)) if want_hidden else None
         rc = lib().oc_forward(C.byref(self.cfg), C.byref(self.model), int(view), int(mode), _ip(tok), R,
                               int(t), _dp(kc), _dp(vc), cap, _dp(logits), _dp(hid))

@@ -93,9 +93,12 @@ def bf16_bits(x: np.ndarray) -> np.ndarray:
     """uint16 bf16 bit patterns of x (fp64 -> fp32 -> bf16, each round to
     nearest even; finite inputs only)."""
     f = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32))
-    b = f.view(np.uint32).astype(np.uint64)
-    b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
-    return b.astype(np.uint16)
+    b = f.view(np.uint32)          # finite values: b + 0x8000 never overflows 32 bits
+    r = (b >> 16) & 1
+    r += 0x7FFF
+    r += b
+    r >>= 16
+    return r.astype(np.uint16)
 
 
 def bits_to_f32(bits: np.ndarray) -> np.ndarray:

@@ -175,3 +175,29 @@ def test_bf16_orthrus_equals_plain_ar(pkg, shape, P, N):
     assert st["forwards"] == 2 * st["cycles"] and sa["forwards"] == N
     del eng, w
     torch.cuda.empty_cache()
+
+
+def test_probe_and_launch_count(tiny):
+    """The measurement hooks: events bracket the probed launches and the
+    launch counter counts every kernel a decode cycle enqueues."""
+    _, eng = tiny
+    prompt = torch.from_numpy(synth.make_prompt(synth.TINY, 16, 0))[None]
+    anchor = eng.prefill(prompt)
+    g0 = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    g1 = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    a0 = [torch.cuda.Event(enable_timing=True)]
+    a1 = [torch.cuda.Event(enable_timing=True)]
+    eng.set_probe(0, 1, 0, g0, g1)
+    eng.set_probe(1, 1, 0, a0, a1)
+    c0 = eng.launch_count()
+    draft = eng.draft_block(anchor, 4)
+    eng.verify_block(anchor, draft, 4)
+    eng.commit(anchor, 4)
+    torch.cuda.synchronize()
+    L = eng.n_layers
+    per_forward = 1 + 8 * L + 1 + 2        # embed, 8 per layer, final norm, LM head + finalize
+    assert eng.launch_count() - c0 == 2 * per_forward + 2
+    assert all(g0[i].elapsed_time(g1[i]) > 0 for i in range(4))
+    assert a0[0].elapsed_time(a1[0]) > 0
+    eng.set_probe(0, 0, 0, [], [])
+    eng.set_probe(1, 0, 0, [], [])
