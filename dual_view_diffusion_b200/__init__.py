@@ -85,6 +85,8 @@ _SIGS = {
     "orthrus_debug_logits": [_P, _I, _I, _I, _P, _P],
     "orthrus_check_error": [_P, _P, C.POINTER(C.c_uint32)],
     "orthrus_set_probe": [_P, _I, _I, _I, C.POINTER(_P), C.POINTER(_P), _I],
+    "orthrus_dual_view_attention_noalloc": [C.POINTER(Config), C.POINTER(KV), _I, _I, _P, _P, _P, _I, _I, _P, _P,
+                                            _P],
 }
 
 

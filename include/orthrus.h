@@ -236,6 +236,36 @@ orthrus_status_t orthrus_dual_view_attention(orthrus_ctx_t *ctx, const orthrus_k
                                              void *stream);
 
 /*
+ * orthrus_dual_view_attention for callers that cannot allocate device
+ * memory.  The paper has no counterpart to this entry point; it exists for
+ * deployment.  Some callers cannot hand the library a workspace: a serving
+ * runtime that reserves the whole of HBM for its own pool at start-up (a
+ * cudaMalloc from a plugin then fails or eats memory the pool was promised),
+ * or code on a latency-critical path where cudaMalloc / cudaFree would
+ * synchronise the device.  This call needs no context and no workspace: its
+ * split partials live in a fixed 16 MiB array that the library holds on every
+ * GPU it is loaded on, until the process exits.  It allocates nothing.
+ *
+ *   cfg      model shape and limits (only the attention fields, n_layers,
+ *            dtype, max_seq and split_tokens are read); q, k_blk, v_blk, out,
+ *            kv, mode, layer, batch, K as for orthrus_dual_view_attention.
+ *   dev_err  device pointer to a uint32 the caller owns, or NULL; it is
+ *            cleared and then receives the device error bits of this call.
+ *            With NULL the bits go to a word inside the fixed array.
+ * Returns ORTHRUS_ERR_CAPACITY, launching nothing, when batch*K*n_q*
+ * ceil(max_seq/split_tokens)*(head_dim*4 + 8) bytes plus a small header do not
+ * fit in the 16 MiB.  The first call on a device also looks up the array's
+ * device address and sets the kernels' shared-memory limit; make that first
+ * call before capturing a stream.  All calls share the one array, so calls
+ * whose work overlaps on the GPU (two streams, or two threads) race and give
+ * wrong results: serialise them.
+ */
+orthrus_status_t orthrus_dual_view_attention_noalloc(const orthrus_config_t *cfg, const orthrus_kv_t *kv,
+                                                    int32_t layer, int32_t mode, const void *q, const void *k_blk,
+                                                    const void *v_blk, int32_t batch, int32_t K, void *out,
+                                                    uint32_t *dev_err, void *stream);
+
+/*
  * Test and measurement hook: the logits of the last verify (which = 0) or
  * draft (which = 1) for every block row, fp32 [batch][K][vocab], computed
  * from the final hidden rows the step kept (one extra LM-head pass; the
