@@ -128,6 +128,31 @@ static void rebase(Ctx *x, char *ws)
     fix(x->tok_buf); fix(x->anchor_buf);
 }
 
+// TMA maps for the tensor-core GEMM: every weight matrix (128-row boxes;
+// 64-row boxes for gate/up, whose tiles pair 64 gate rows with 64 up rows)
+// and every activation buffer a projection reads (32-row boxes).  A matrix
+// whose inner size is not a multiple of 64 gets no map and runs on the SIMT
+// kernel.
+static void build_tmaps(Ctx *c)
+{
+    const orthrus_config_t &f = c->cfg;
+    const int d = f.hidden, hq = f.n_q_heads * f.head_dim, hk = f.n_kv_heads * f.head_dim, F = f.ffn;
+    auto add = [&](const void *p, int rows, int cols, uint32_t box) {
+        if (!p || cols % kTileK) return;
+        CUtensorMap m;
+        if (make_tmap(&m, p, rows, cols, box)) c->tmaps[TmapKey{p, box}] = m;
+    };
+    for (const orthrus_layer_weights_t &L : c->layers) {
+        add(L.wq, hq, d, kTileN); add(L.wk, hk, d, kTileN); add(L.wv, hk, d, kTileN);
+        add(L.wq_diff, hq, d, kTileN); add(L.wk_diff, hk, d, kTileN); add(L.wv_diff, hk, d, kTileN);
+        add(L.wo, d, hq, kTileN); add(L.w_gate, F, d, 64); add(L.w_up, F, d, 64); add(L.w_down, d, F, kTileN);
+    }
+    add(c->lm_head, f.vocab, d, kTileN);
+    add(c->a, c->Rw, d, kTileM); add(c->attn_o, c->Rw, hq, kTileM); add(c->act, c->Rw, F, kTileM);
+    add(c->fin_draft, c->R, d, kTileM); add(c->fin_verify, c->R, d, kTileM);
+    add(c->res_x, 2 * f.max_batch, d, kTileM);
+}
+
 static KvView kv_view(const orthrus_kv_t &kv)
 {
     return KvView{kv.k_pages, kv.v_pages, kv.block_table, kv.num_pages, kv.page_size, kv.max_pages_per_seq};
@@ -308,10 +333,11 @@ orthrus_status_t orthrus_create(const orthrus_config_t *cfg, const orthrus_weigh
     c->layers.assign(w->layers, w->layers + cfg->n_layers);
     c->embed = w->embed; c->final_norm = w->final_norm; c->lm_head = w->lm_head;
     if (cudaGetDevice(&c->dev) != cudaSuccess || gemm_init_attributes() != cudaSuccess ||
-        attention_init_attributes() != cudaSuccess) {
+        gemm_tc_init_attributes() != cudaSuccess || attention_init_attributes() != cudaSuccess) {
         delete c;
         return ORTHRUS_ERR_CUDA;
     }
+    if (cfg->dtype == ORTHRUS_BF16) build_tmaps(c);
     std::vector<int32_t> ident(cfg->max_batch);
     for (int b = 0; b < cfg->max_batch; ++b) ident[b] = b;
     if (cudaMemset(workspace, 0, need) != cudaSuccess ||

@@ -348,7 +348,9 @@ __global__ void __launch_bounds__(128) attn_split_simt(AttnArgs a, int n_split_g
 
 // ---------------------------------------------------------------- combine
 // One warp per (block row, query head): weights 2^(m_s - M) over the splits
-// the sequence used, summed in split order.
+// the sequence used, summed in split order.  Lane s holds split s's (m, l)
+// (32 splits per round); each lane accumulates 4 output dims, loading the
+// partial rows of 8 splits before using any of them.
 template <class T>
 __global__ void __launch_bounds__(256) attn_combine(AttnArgs a)
 {
@@ -372,10 +374,35 @@ __global__ void __launch_bounds__(256) attn_combine(AttnArgs a)
     L = warp_sum(L);
     const float inv = 1.0f / L;
     const float *part = a.part + (size_t)w * a.n_splits * a.hd;
-    for (int d = lane; d < a.hd; d += 32) {
-        float acc = 0.f;
-        for (int s = 0; s < n_used; ++s) acc = fmaf(exp2f(ml[s].x - M), part[(size_t)s * a.hd + d], acc);
-        ((T *)a.out)[(size_t)w * a.hd + d] = from_f<T>(acc * inv);
+    const int c0 = lane * 4;
+    const bool mine = c0 < a.hd;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < n_used; s0 += 32) {
+        const int sl = s0 + lane;
+        const float wl = sl < n_used ? exp2f(ml[sl].x - M) : 0.f;
+        const int cnt = min(32, n_used - s0);
+        for (int j0 = 0; j0 < cnt; j0 += 8) {
+            float4 v[8];
+            float wt[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                wt[j] = __shfl_sync(0xffffffffu, wl, (j0 + j) & 31);
+                const bool ok = mine && j0 + j < cnt;
+                v[j] = ok ? *(const float4 *)(part + (size_t)(s0 + j0 + j) * a.hd + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (j0 + j < cnt) {
+                    acc.x = fmaf(wt[j], v[j].x, acc.x); acc.y = fmaf(wt[j], v[j].y, acc.y);
+                    acc.z = fmaf(wt[j], v[j].z, acc.z); acc.w = fmaf(wt[j], v[j].w, acc.w);
+                }
+            }
+        }
+    }
+    if (mine) {
+        T *o = (T *)a.out + (size_t)w * a.hd + c0;
+        o[0] = from_f<T>(acc.x * inv); o[1] = from_f<T>(acc.y * inv);
+        o[2] = from_f<T>(acc.z * inv); o[3] = from_f<T>(acc.w * inv);
     }
 }
 

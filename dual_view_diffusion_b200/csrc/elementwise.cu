@@ -32,22 +32,76 @@ __global__ void embed_kernel(const T *embed, int d, int V, int mask_id, int mode
 
 // ---------------------------------------------------------------- RMSNorm
 // out = h / sqrt(mean(h^2) + eps) * gain; fixed reduction order per row.
+// Rows of up to 8192 elements (multiple of 4) stay in registers: every load
+// is issued before the first use.
+constexpr int kNormThreads = 256, kNormVec = 8;
+
 template <class T>
-__global__ void __launch_bounds__(256) rmsnorm_kernel(const float *h, const T *gain, T *out, int d, float eps)
+__device__ __forceinline__ void store4(T *p, float a, float b, float c, float d);
+template <>
+__device__ __forceinline__ void store4<float>(float *p, float a, float b, float c, float d)
 {
-    __shared__ float red[8];
+    *(float4 *)p = make_float4(a, b, c, d);
+}
+template <>
+__device__ __forceinline__ void store4<bf16>(bf16 *p, float a, float b, float c, float d)
+{
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+    uint2 u;
+    u.x = *(uint32_t *)&lo;
+    u.y = *(uint32_t *)&hi;
+    *(uint2 *)p = u;
+}
+
+template <class T>
+__device__ __forceinline__ float4 load_gain4(const T *g, int i)
+{
+    return make_float4(to_f<T>(g[i]), to_f<T>(g[i + 1]), to_f<T>(g[i + 2]), to_f<T>(g[i + 3]));
+}
+
+template <class T>
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float *h, const T *gain, T *out, int d, float eps)
+{
+    __shared__ float red[kNormThreads / 32];
     const int row = blockIdx.x, tid = threadIdx.x;
     const float *x = h + (size_t)row * d;
     float ss = 0.f;
-    for (int i = tid; i < d; i += 256) ss = fmaf(x[i], x[i], ss);
+    const bool vec = (d & 3) == 0 && d <= kNormThreads * 4 * kNormVec;
+    float4 v[kNormVec];
+    if (vec) {
+#pragma unroll
+        for (int j = 0; j < kNormVec; ++j) {
+            const int i = (tid + j * kNormThreads) * 4;
+            v[j] = i < d ? *(const float4 *)(x + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < kNormVec; ++j) {
+            ss = fmaf(v[j].x, v[j].x, ss); ss = fmaf(v[j].y, v[j].y, ss);
+            ss = fmaf(v[j].z, v[j].z, ss); ss = fmaf(v[j].w, v[j].w, ss);
+        }
+    } else {
+        for (int i = tid; i < d; i += kNormThreads) ss = fmaf(x[i], x[i], ss);
+    }
     ss = warp_sum(ss);
     if ((tid & 31) == 0) red[tid >> 5] = ss;
     __syncthreads();
     float tot = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) tot += red[w];
+    for (int w = 0; w < kNormThreads / 32; ++w) tot += red[w];
     const float inv = 1.0f / sqrtf(tot / d + eps);
-    for (int i = tid; i < d; i += 256) out[(size_t)row * d + i] = from_f<T>(x[i] * inv * to_f<T>(gain[i]));
+    T *o = out + (size_t)row * d;
+    if (vec) {
+#pragma unroll
+        for (int j = 0; j < kNormVec; ++j) {
+            const int i = (tid + j * kNormThreads) * 4;
+            if (i < d) {
+                const float4 g = load_gain4(gain, i);
+                store4<T>(o + i, v[j].x * inv * g.x, v[j].y * inv * g.y, v[j].z * inv * g.z, v[j].w * inv * g.w);
+            }
+        }
+    } else {
+        for (int i = tid; i < d; i += kNormThreads) o[i] = from_f<T>(x[i] * inv * to_f<T>(gain[i]));
+    }
 }
 
 // ---------------------------------------------------------------- LM head
@@ -259,9 +313,9 @@ cudaError_t launch_rmsnorm(const Ctx &c, const float *h, const void *gain, void 
 {
     c.launches += 1;
     if (c.cfg.dtype == ORTHRUS_BF16)
-        rmsnorm_kernel<bf16><<<M, 256, 0, s>>>(h, (const bf16 *)gain, (bf16 *)out, c.cfg.hidden, c.cfg.rms_eps);
+        rmsnorm_kernel<bf16><<<M, kNormThreads, 0, s>>>(h, (const bf16 *)gain, (bf16 *)out, c.cfg.hidden, c.cfg.rms_eps);
     else
-        rmsnorm_kernel<float><<<M, 256, 0, s>>>(h, (const float *)gain, (float *)out, c.cfg.hidden, c.cfg.rms_eps);
+        rmsnorm_kernel<float><<<M, kNormThreads, 0, s>>>(h, (const float *)gain, (float *)out, c.cfg.hidden, c.cfg.rms_eps);
     return cudaGetLastError();
 }
 

@@ -22,14 +22,15 @@
 // bf16 uses tensor cores (mma.sync m16n8k16, fp32 accumulate); fp32 uses a
 // SIMT loop with the same tiling, scheduling and epilogues.
 #include <math.h>
+#include <stdlib.h>
 
 #include "common.cuh"
+#include "gemm_epilogue.cuh"
 #include "internal.h"
 
 namespace orthrus {
 
 constexpr int kStages = 6;
-constexpr int kTilePad = kTileN + 4;
 constexpr int kGemmThreads = 128;
 
 struct GemmShape {
@@ -199,177 +200,6 @@ __device__ void mainloop_simt(const GemmArgs &a, int mt, int nt, int k0, int k1,
     for (int m = 0; m < kTileM; ++m) tile[m][tid] = acc[m];
 }
 
-// ---------------------------------------------------------------- epilogues
-struct Best {
-    float v;
-    int i;
-    float z;
-};
-
-__device__ __forceinline__ void best_merge(Best &a, const Best &b)
-{
-    if (b.v > a.v || (b.v == a.v && b.i < a.i)) a = b;
-}
-
-__device__ __forceinline__ Best warp_best(Best b)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        Best c;
-        c.v = __shfl_xor_sync(0xffffffffu, b.v, o);
-        c.i = __shfl_xor_sync(0xffffffffu, b.i, o);
-        c.z = __shfl_xor_sync(0xffffffffu, b.z, o);
-        best_merge(b, c);
-    }
-    return b;
-}
-
-template <class T>
-__device__ void store_kv(const GemmArgs &a, bool is_k, int row, int b, int pos, int kvh, int d, float v0, float v1,
-                         int half)
-{
-    T *dst;
-    if (a.kv_to_cache) {
-        const int pidx = pos / a.kv.page_size;
-        if (pos < 0 || pidx >= a.kv.max_pages) { raise_err(a.err, ORTHRUS_DEVERR_CAPACITY); return; }
-        const int page = a.kv.block_table[(size_t)a.bt_rows[b] * a.kv.max_pages + pidx];
-        if (page < 0 || page >= a.kv.num_pages) { raise_err(a.err, ORTHRUS_DEVERR_CAPACITY); return; }
-        T *base = (T *)(is_k ? a.kv.k_pages : a.kv.v_pages);
-        dst = base + (((size_t)a.layer * a.kv.num_pages + page) * a.n_kv + kvh) * (size_t)a.kv.page_size * a.hd +
-              (size_t)(pos % a.kv.page_size) * a.hd;
-    } else {
-        T *base = (T *)(is_k ? a.k_blk : a.v_blk);
-        dst = base + (((size_t)a.layer * a.rows_max + row) * a.n_kv + kvh) * a.hd;
-    }
-    dst[d] = from_f<T>(v0);
-    dst[d + half] = from_f<T>(v1);
-}
-
-template <class T>
-__device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int nt, int n_nt)
-{
-    const int tid = threadIdx.x;
-    if (a.epi == EPI_RESID) {
-        for (int idx = tid; idx < kTileM * kTileN; idx += kGemmThreads) {
-            const int m = idx >> 7, nl = idx & 127, row = mt * kTileM + m, n = nt * kTileN + nl;
-            if (row < a.M && n < a.N) a.resid[(size_t)row * a.N + n] += tile[m][nl];
-        }
-    } else if (a.epi == EPI_SWIGLU) {
-        for (int idx = tid; idx < kTileM * 64; idx += kGemmThreads) {
-            const int m = idx >> 6, i = idx & 63, row = mt * kTileM + m, f = nt * 64 + i;
-            if (row < a.M && f < a.N) {
-                const float g = tile[m][i], u = tile[m][64 + i];
-                const float s = g / (1.0f + expf(-g));
-                ((T *)a.act)[(size_t)row * a.N + f] = from_f<T>(s * u);
-            }
-        }
-    } else if (a.epi == EPI_QKV) {
-        const int half = a.hd / 2, Nq = a.n_q * a.hd, Nk = a.n_kv * a.hd;
-        for (int idx = tid; idx < kTileM * 64; idx += kGemmThreads) {
-            const int m = idx >> 6, p = idx & 63;
-            const int nl = (p / half) * a.hd + (p % half), i = p % half;
-            const int n = nt * kTileN + nl, row = mt * kTileM + m;
-            if (row >= a.M || n >= Nq + 2 * Nk) continue;
-            const int b = row / a.K, k = row % a.K, pos = a.pos0[b] + k;
-            double x0 = tile[m][nl], x1 = tile[m][nl + half];
-            if (n < Nq + Nk) {   // rotary embedding on Q and K (rotate-half pairs)
-                const double ang = (double)pos * pow(a.rope_theta, -2.0 * i / a.hd);
-                double sn, cs;
-                sincos(ang, &sn, &cs);
-                const double r0 = x0 * cs - x1 * sn, r1 = x1 * cs + x0 * sn;
-                x0 = r0; x1 = r1;
-            }
-            if (n < Nq) {
-                T *q = (T *)a.q_out + (size_t)row * Nq;
-                q[n] = from_f<T>((float)x0);
-                q[n + half] = from_f<T>((float)x1);
-            } else {
-                const bool is_k = n < Nq + Nk;
-                const int nn = n - Nq - (is_k ? 0 : Nk);
-                store_kv<T>(a, is_k, row, b, pos, nn / a.hd, nn % a.hd, (float)x0, (float)x1, half);
-            }
-        }
-    } else if (a.epi == EPI_LMHEAD) {
-        const int lane = tid & 31, warp = tid >> 5;
-        const float it = a.inv_temp > 0.f ? a.inv_temp : 1.0f;
-        const uint32_t step = a.step ? (uint32_t)*a.step : 0u;
-        for (int ml = 0; ml < kTileM / 4; ++ml) {
-            const int m = warp * (kTileM / 4) + ml, row = mt * kTileM + m;
-            if (row >= a.M) break;
-            const int b = row / a.K, k = row % a.K;
-            const int given = a.given ? a.given[row] : -1;
-            Best zb{-INFINITY, 0x7fffffff, 0.f}, gb{-INFINITY, 0x7fffffff, 0.f};
-            float zid = NAN;
-            float zv[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int nl = lane * 4 + j, v = nt * kTileN + nl;
-                zv[j] = v < a.N ? tile[m][nl] : -INFINITY;
-                if (v < a.N) {
-                    best_merge(zb, Best{zv[j], v, zv[j]});
-                    if (v == given) zid = zv[j];
-                    if (a.lm_mode != 0 && a.inv_temp > 0.f) {
-                        const uint32_t rr = a.lm_mode == 2 ? rng_row(b, 0) : rng_row(b, k);
-                        const uint32_t pu = a.lm_mode == 2 ? PURPOSE_AR : PURPOSE_DRAFT;
-                        best_merge(gb, Best{zv[j] * a.inv_temp + gumbel(a.seed, step, rr, (uint32_t)v, pu), v, zv[j]});
-                    }
-                }
-            }
-            zb = warp_best(zb);
-            gb = warp_best(gb);
-            float s = 0.f;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (nt * kTileN + lane * 4 + j < a.N) s += expf((zv[j] - zb.v) * it);
-            s = warp_sum(s);
-            // the id's logit lives in exactly one lane (or none)
-            const unsigned has = __ballot_sync(0xffffffffu, !isnan(zid));
-            if (has) zid = __shfl_sync(0xffffffffu, zid, __ffs(has) - 1);
-            if (lane == 0) {
-                LmPart pr;
-                pr.zmax = zb.v; pr.zsum = s; pr.zarg = zb.i;
-                pr.gbest = gb.v; pr.garg = gb.i; pr.gz = gb.z; pr.zid = zid; pr.pad = 0;
-                a.lm[(size_t)row * n_nt + nt] = pr;
-            }
-        }
-    } else if (a.epi == EPI_LOGITS) {
-        for (int idx = tid; idx < kTileM * kTileN; idx += kGemmThreads) {
-            const int m = idx >> 7, nl = idx & 127, row = mt * kTileM + m, n = nt * kTileN + nl;
-            if (row < a.M && n < a.N) a.logits[(size_t)row * a.N + n] = tile[m][nl];
-        }
-    } else if (a.epi == EPI_RESAMPLE) {
-        // rows come in pairs (2b: AR view at the rejected row, 2b+1: diffusion
-        // view at the same row); score = log max(0, p - q) + Gumbel
-        const int lane = tid & 31, warp = tid >> 5;
-        const uint32_t step = a.step ? (uint32_t)*a.step : 0u;
-        for (int pl = 0; pl < kTileM / 8; ++pl) {
-            const int mp = warp * (kTileM / 8) + pl;        // pair index within tile
-            const int m = 2 * mp, row = mt * kTileM + m, b = row / 2;
-            if (row >= a.M) break;
-            const int j = a.rej_row[b];
-            if (j < 0) continue;
-            const float lp = a.lse_p[b * a.K + j], lq = a.lse_q[b * a.K + j];
-            Best gb{-INFINITY, 0x7fffffff, 0.f};
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int nl = lane * 4 + jj, v = nt * kTileN + nl;
-                if (v < a.N) {
-                    const float r = expf(tile[m][nl] * a.inv_temp - lp) - expf(tile[m + 1][nl] * a.inv_temp - lq);
-                    if (r > 0.f)
-                        best_merge(gb, Best{logf(r) + gumbel(a.seed, step, rng_row(b, j), (uint32_t)v, PURPOSE_RESIDUAL),
-                                            v, tile[m][nl]});
-                }
-            }
-            gb = warp_best(gb);
-            if (lane == 0) {
-                LmPart pr{};
-                pr.gbest = gb.v; pr.garg = gb.i; pr.gz = gb.z;
-                a.lm[(size_t)row * n_nt + nt] = pr;
-            }
-        }
-    }
-}
-
 // ---------------------------------------------------------------- kernel
 // One-dimensional grid of persistent CTAs walking (m tile, n tile, segment)
 // units in order.
@@ -394,52 +224,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(GemmArgs a, int n
             mainloop_simt<T>(a, mt, nt, c0 * kTileK, min(c1 * kTileK, a.Kd), (float *)pipe, tile);
         }
         __syncthreads();
-        if (S > 1) {
-            float *slot = a.part + ((size_t)t * S + seg) * (kTileM * kTileN);
-            for (int idx = threadIdx.x; idx < kTileM * kTileN / 4; idx += kGemmThreads) {
-                const int m = idx >> 5, c4 = (idx & 31) * 4;
-                __stcg((float4 *)(slot + m * kTileN + c4), *(float4 *)&tile[m][c4]);
-            }
-            __threadfence();
-            __syncthreads();
-            if (threadIdx.x == 0) s_last = (atomicAdd(&a.ticket[t], 1) == S - 1);
-            __syncthreads();
-            if (!s_last) continue;
-            __threadfence();
-            const float *base = a.part + (size_t)t * S * (kTileM * kTileN);
-            for (int idx = threadIdx.x; idx < kTileM * kTileN / 4; idx += kGemmThreads) {
-                const int m = idx >> 5, c4 = (idx & 31) * 4;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int s = 0; s < S; ++s) {
-                    const float4 v = __ldcg((const float4 *)(base + (size_t)s * kTileM * kTileN + m * kTileN + c4));
-                    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-                }
-                *(float4 *)&tile[m][c4] = acc;
-            }
-            if (threadIdx.x == 0) a.ticket[t] = 0;
-            __syncthreads();
-        }
-        epilogue<T>(a, tile, mt, nt, n_nt);
+        if (!split_k_gather(a, tile, t, seg, threadIdx.x, &s_last, SyncBlock{}))
+            continue;
+        epilogue<T>(a, tile, mt, nt, n_nt, threadIdx.x, SyncBlock{});
         __syncthreads();
     }
 }
 
 // ---------------------------------------------------------------- host
-// k segments per n tile: minimise waves x (chunks per segment + fill and
-// reduction overhead) over one wave of 148 persistent CTAs.  Depends on the
-// matrix shape only.
+// k segments per n tile.  A persistent CTA streams its units back to back,
+// so the time is set by the busiest CTA's chunk count; each extra segment
+// adds a partial tile to publish and reduce.  Cost = max chunks per CTA +
+// 8 chunk-equivalents per segment (fitted to the Qwen3-8B projections on a
+// B200: QKV -> 3, O -> 3, gate/up -> 2, down -> 4, LM head -> 1).  Depends on
+// the matrix shape only, never on the number of token rows.
 int choose_splits(int N, int Kd)
 {
     const int n_nt = (N + kTileN - 1) / kTileN;
     const int chunks = (Kd + kTileK - 1) / kTileK;
     int best = 1;
-    double best_cost = 1e30;
+    long best_cost = -1;
     for (int S = 1; S <= 16; ++S) {
         if (S > 1 && chunks / S < 4) break;
         const long units = (long)n_nt * S;
-        const long waves = (units + kNumSMs - 1) / kNumSMs;
-        const double cost = (double)waves * ((chunks + S - 1) / S + 2 + (S > 1 ? 1 : 0));
-        if (cost < best_cost - 1e-9) { best_cost = cost; best = S; }
+        const long per_cta = (units + kNumSMs - 1) / kNumSMs;
+        const long cost = per_cta * ((chunks + S - 1) / S) + 8L * S;
+        if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = S; }
     }
     return best;
 }
@@ -468,8 +278,12 @@ cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s)
     const long units = (long)n_mt * n_nt * a.splits;
     const int grid = (int)(units < kNumSMs ? units : kNumSMs);
     const size_t smem = gemm_smem_bytes(tc);
-    c.launches += 1;
     if (tc) {
+        const cudaError_t e = launch_gemm_tc(c, a, n_mt, n_nt, grid, s);
+        if (e != cudaErrorNotSupported) return e;
+    }
+    c.launches += 1;
+    if (tc && getenv("ORTHRUS_GEMM_MMA_SYNC")) {
         gemm_kernel<bf16, true><<<grid, kGemmThreads, smem, s>>>(a, n_mt, n_nt);
     } else if (c.cfg.dtype == ORTHRUS_BF16) {
         gemm_kernel<bf16, false><<<grid, kGemmThreads, smem, s>>>(a, n_mt, n_nt);

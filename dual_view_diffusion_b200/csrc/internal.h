@@ -2,10 +2,12 @@
 // workspace carve-up and the kernel launchers.  Not part of the C ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
 
+#include <unordered_map>
 #include <vector>
 
 #include "../../include/orthrus.h"
@@ -96,8 +98,19 @@ struct AttnArgs {
     unsigned *err;
 };
 
+// Tensor maps are looked up by (base pointer, box rows).
+struct TmapKey {
+    const void *ptr;
+    uint32_t box_rows;
+    bool operator==(const TmapKey &o) const { return ptr == o.ptr && box_rows == o.box_rows; }
+};
+struct TmapKeyHash {
+    size_t operator()(const TmapKey &k) const { return std::hash<const void *>()(k.ptr) ^ (size_t)k.box_rows * 0x9E3779B97F4A7C15ull; }
+};
+
 struct Ctx {
     orthrus_config_t cfg;
+    std::unordered_map<TmapKey, CUtensorMap, TmapKeyHash> tmaps;   // bf16 TMA maps of weights and activations
     std::vector<orthrus_layer_weights_t> layers;
     const void *embed, *final_norm, *lm_head;
     int esize;               // bytes per element of the dtype
@@ -160,6 +173,9 @@ bool use_tensor_cores(const orthrus_config_t &c);
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s);
 cudaError_t gemm_init_attributes();
+cudaError_t gemm_tc_init_attributes();
+bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, int grid, cudaStream_t s);
 cudaError_t attention_init_attributes();
 cudaError_t launch_attention(const Ctx &c, const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_embed(const Ctx &c, int mode, const int32_t *tokens, const int32_t *anchor,

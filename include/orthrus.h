@@ -63,6 +63,7 @@ typedef enum { ORTHRUS_BF16 = 0, ORTHRUS_FP32 = 1 } orthrus_dtype_t;
 #define ORTHRUS_DEVERR_TOKEN     0x1   /* token id outside [0, vocab) */
 #define ORTHRUS_DEVERR_CAPACITY  0x2   /* position beyond the sequence's pages */
 #define ORTHRUS_DEVERR_NONFINITE 0x4   /* non-finite log-sum-exp */
+#define ORTHRUS_DEVERR_TIMEOUT   0x8   /* a kernel's bounded wait ran out; it stopped early */
 
 /*
  * Model shape and run limits.  The decoder is the pages' frozen AR backbone
