@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--temperature", type=float, default=0.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--split-tokens", type=int, default=128,
+                    help="KV positions per attention split (a run-wide constant)")
     ap.add_argument("--profile-small", action="store_true",
                     help="small case for ncu captures: 2 layers of the 8B shape, vocab 32000, 2 steps; "
                          "its line is marked profile_case and is not a bench result")
@@ -276,7 +278,7 @@ def run_ours(args, rank, world, local_rank):
     n_e2e = 0 if args.no_e2e else K
     max_seq = P_PROMPT + (W + K + n_e2e + 2) * K_BLOCK + K_BLOCK
     w = synth.make_weights_torch(s, 0, device=dev)
-    eng = pkg.Engine(s, w, max_batch=BATCH, max_block=K_BLOCK, max_seq=max_seq, split_tokens=256,
+    eng = pkg.Engine(s, w, max_batch=BATCH, max_block=K_BLOCK, max_seq=max_seq, split_tokens=args.split_tokens,
                      page_size=64, device=dev)
     prompt = torch.from_numpy(synth.make_prompt(s, P_PROMPT, 100 + rank))[None].to(dev)
     anchor = eng.prefill(prompt)
@@ -385,7 +387,7 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "bf16", "data": "synthetic (random-init weights, uniform random prompt)",
         "config": {"workload": "qwen3-8b-shape decode step (draft + verify + commit), batch 1 per GPU, K=32, "
                                "prompt 2048, greedy", "global_batch": BATCH * world, "seq_len": P_PROMPT,
-                   "block_K": K_BLOCK, "parallelism": f"replicas x{world}",
+                   "block_K": K_BLOCK, "split_tokens": args.split_tokens, "parallelism": f"replicas x{world}",
                    "l2": "weights (18 GB) and cache exceed L2 every step; no flush"},
         "mean_accepted_per_cycle": nbar, "tokens_per_forward": nbar / 2,
         "modelled_tokens_per_s_at_pages_acceptance": 10.8 / (max_ms / K * 1e-3),

@@ -93,8 +93,13 @@ __global__ void __launch_bounds__(256, 1) attn_split_mma(AttnArgs a, int n_split
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     AttnSmem &sm = *(AttnSmem *)smem_raw;
-    const int s = blockIdx.x % n_split_grid, rg = blockIdx.x / n_split_grid;
-    const int kvh = blockIdx.y, b = blockIdx.z;
+    pdl_trigger();
+    pdl_wait();
+    // grid (kv head, sequence x row group, split): the split index varies
+    // slowest, so the CTAs of splits a short sequence never reaches (they
+    // exit at once) come after every working CTA
+    const int kvh = blockIdx.x, s = blockIdx.z;
+    const int rgroups = gridDim.y / a.B, b = blockIdx.y / rgroups, rg = blockIdx.y % rgroups;
     const int g = a.n_q / a.n_kv, R = a.K * g, r0 = rg * kAttnRowsMma;
     if (r0 >= R) return;
     const int t = a.seq_lens[b];
@@ -278,8 +283,10 @@ __global__ void __launch_bounds__(128) attn_split_simt(AttnArgs a, int n_split_g
     float *vs = ks + kKeyTile * hp;                     // [64][hp]
     float *ms = vs + kKeyTile * hp;                     // [32]
     float *ls = ms + kAttnRowsSimt;                     // [32]
-    const int s = blockIdx.x % n_split_grid, rg = blockIdx.x / n_split_grid;
-    const int kvh = blockIdx.y, b = blockIdx.z;
+    pdl_trigger();
+    pdl_wait();
+    const int kvh = blockIdx.x, s = blockIdx.z;
+    const int rgroups = gridDim.y / a.B, b = blockIdx.y / rgroups, rg = blockIdx.y % rgroups;
     const int g = a.n_q / a.n_kv, R = a.K * g, r0 = rg * kAttnRowsSimt;
     if (r0 >= R) return;
     const int t = a.seq_lens[b], kv_len = t + a.K;
@@ -354,6 +361,8 @@ __global__ void __launch_bounds__(128) attn_split_simt(AttnArgs a, int n_split_g
 template <class T>
 __global__ void __launch_bounds__(256) attn_combine(AttnArgs a)
 {
+    pdl_trigger();
+    pdl_wait();
     const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     const int rows = a.B * a.K * a.n_q;
     if (w >= rows) return;
@@ -432,22 +441,19 @@ cudaError_t launch_attention(const Ctx &c, const AttnArgs &a, cudaStream_t s)
     const int rgroups = (R + rows_per - 1) / rows_per;
     // splits reachable by any sequence this context serves
     const int n_split_grid = (c.cfg.max_seq + a.split_tokens - 1) / a.split_tokens;
-    dim3 grid(n_split_grid * rgroups, a.n_kv, a.B);
+    dim3 grid(a.n_kv, a.B * rgroups, n_split_grid);
     c.launches += 2;
+    cudaError_t e;
     if (tc)
-        attn_split_mma<<<grid, 256, sizeof(AttnSmem), s>>>(a, n_split_grid);
+        e = launch_k(attn_split_mma, grid, 256, sizeof(AttnSmem), s, a, n_split_grid);
     else if (c.cfg.dtype == ORTHRUS_BF16)
-        attn_split_simt<bf16><<<grid, 128, simt_smem(a.hd), s>>>(a, n_split_grid);
+        e = launch_k(attn_split_simt<bf16>, grid, 128, simt_smem(a.hd), s, a, n_split_grid);
     else
-        attn_split_simt<float><<<grid, 128, simt_smem(a.hd), s>>>(a, n_split_grid);
-    cudaError_t e = cudaGetLastError();
+        e = launch_k(attn_split_simt<float>, grid, 128, simt_smem(a.hd), s, a, n_split_grid);
     if (e != cudaSuccess) return e;
     const int rows = a.B * a.K * a.n_q;
-    if (c.cfg.dtype == ORTHRUS_BF16)
-        attn_combine<bf16><<<(rows + 7) / 8, 256, 0, s>>>(a);
-    else
-        attn_combine<float><<<(rows + 7) / 8, 256, 0, s>>>(a);
-    return cudaGetLastError();
+    if (c.cfg.dtype == ORTHRUS_BF16) return launch_k(attn_combine<bf16>, (rows + 7) / 8, 256, 0, s, a);
+    return launch_k(attn_combine<float>, (rows + 7) / 8, 256, 0, s, a);
 }
 
 }  // namespace orthrus

@@ -29,6 +29,8 @@ static std::mutex g_scratch_mu;
 
 __global__ void noalloc_identity_rows(int32_t *rows, int n)
 {
+    pdl_trigger();
+    pdl_wait();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) rows[i] = i;
 }
@@ -85,8 +87,8 @@ extern "C" orthrus_status_t orthrus_dual_view_attention_noalloc(const orthrus_co
     unsigned *err = dev_err ? (unsigned *)dev_err : (unsigned *)base;
     int32_t *bt_rows = (int32_t *)(base + off_rows);
     if (cudaMemsetAsync(err, 0, sizeof(unsigned), s) != cudaSuccess) return ORTHRUS_ERR_CUDA;
-    noalloc_identity_rows<<<(batch + 127) / 128, 128, 0, s>>>(bt_rows, batch);
-    if (cudaGetLastError() != cudaSuccess) return ORTHRUS_ERR_CUDA;
+    if (launch_k(noalloc_identity_rows, (batch + 127) / 128, 128, 0, s, bt_rows, (int)batch) != cudaSuccess)
+        return ORTHRUS_ERR_CUDA;
 
     Ctx tmp;                      // only cfg is read by the launcher
     tmp.cfg = *cfg;

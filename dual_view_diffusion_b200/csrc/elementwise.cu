@@ -16,6 +16,8 @@ __global__ void embed_kernel(const T *embed, int d, int V, int mask_id, int mode
                              const int32_t *anchor, const int32_t *draft, int K, int32_t *tok_out, float *h,
                              unsigned *err)
 {
+    pdl_trigger();
+    pdl_wait();
     const int row = blockIdx.x, b = row / K, k = row % K;
     int tok;
     if (mode == 2) tok = tokens[row];
@@ -63,6 +65,8 @@ template <class T>
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float *h, const T *gain, T *out, int d, float eps)
 {
     __shared__ float red[kNormThreads / 32];
+    pdl_trigger();
+    pdl_wait();
     const int row = blockIdx.x, tid = threadIdx.x;
     const float *x = h + (size_t)row * d;
     float ss = 0.f;
@@ -120,6 +124,8 @@ struct LmArgs {
 
 __global__ void __launch_bounds__(256) lm_finalize_kernel(LmArgs a)
 {
+    pdl_trigger();
+    pdl_wait();
     const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     const int rows = a.mode == 3 ? a.B : a.B * a.K;
     if (w >= rows) return;
@@ -203,6 +209,8 @@ struct CommitArgs {
 // needs (AR view, diffusion view).
 __global__ void commit_decide_kernel(CommitArgs a)
 {
+    pdl_trigger();
+    pdl_wait();
     const int b = blockIdx.x;
     __shared__ int s_j;
     if (threadIdx.x == 0) {
@@ -238,6 +246,8 @@ __global__ void commit_decide_kernel(CommitArgs a)
 // are already in place: paper notes §4.1 step 3), bump the step counter.
 __global__ void commit_apply_kernel(CommitArgs a)
 {
+    pdl_trigger();
+    pdl_wait();
     const int b = threadIdx.x;
     if (b < a.B) {
         const int n = a.n_out[b];
@@ -270,6 +280,8 @@ __global__ void commit_apply_kernel(CommitArgs a)
 __global__ void ar_commit_kernel(int B, const int32_t *g, int64_t *step, int32_t *token_out, int32_t *anchor_io,
                                  int32_t *seq_lens, int32_t *append_out, int32_t *produced, int stride, int amax)
 {
+    pdl_trigger();
+    pdl_wait();
     const int b = threadIdx.x;
     if (b < B) {
         const int tok = g[b];
@@ -287,11 +299,18 @@ __global__ void ar_commit_kernel(int B, const int32_t *g, int64_t *step, int32_t
 
 __global__ void set_lens_kernel(int32_t *seq_lens, int b, int value, int32_t *anchor_out, const int32_t *last_tok)
 {
+    pdl_trigger();
+    pdl_wait();
     seq_lens[b] = value;
     if (anchor_out) anchor_out[b] = *last_tok;
 }
 
-__global__ void set_int_kernel(int32_t *p, int v) { *p = v; }
+__global__ void set_int_kernel(int32_t *p, int v)
+{
+    pdl_trigger();
+    pdl_wait();
+    *p = v;
+}
 
 // ---------------------------------------------------------------- host
 cudaError_t launch_embed(const Ctx &c, int mode, const int32_t *tokens, const int32_t *anchor, const int32_t *draft,
@@ -300,23 +319,20 @@ cudaError_t launch_embed(const Ctx &c, int mode, const int32_t *tokens, const in
     const int rows = B * K;
     c.launches += 1;
     if (c.cfg.dtype == ORTHRUS_BF16)
-        embed_kernel<bf16><<<rows, 256, 0, s>>>((const bf16 *)c.embed, c.cfg.hidden, c.cfg.vocab, c.cfg.mask_token_id,
-                                                 mode, tokens, anchor, draft, K, c.tok, c.h, c.err);
-    else
-        embed_kernel<float><<<rows, 256, 0, s>>>((const float *)c.embed, c.cfg.hidden, c.cfg.vocab,
-                                                  c.cfg.mask_token_id, mode, tokens, anchor, draft, K, c.tok, c.h,
-                                                  c.err);
-    return cudaGetLastError();
+        return launch_k(embed_kernel<bf16>, rows, 256, 0, s, (const bf16 *)c.embed, c.cfg.hidden, c.cfg.vocab,
+                        c.cfg.mask_token_id, mode, tokens, anchor, draft, K, c.tok, c.h, c.err);
+    return launch_k(embed_kernel<float>, rows, 256, 0, s, (const float *)c.embed, c.cfg.hidden, c.cfg.vocab,
+                    c.cfg.mask_token_id, mode, tokens, anchor, draft, K, c.tok, c.h, c.err);
 }
 
 cudaError_t launch_rmsnorm(const Ctx &c, const float *h, const void *gain, void *out, int M, cudaStream_t s)
 {
     c.launches += 1;
     if (c.cfg.dtype == ORTHRUS_BF16)
-        rmsnorm_kernel<bf16><<<M, kNormThreads, 0, s>>>(h, (const bf16 *)gain, (bf16 *)out, c.cfg.hidden, c.cfg.rms_eps);
-    else
-        rmsnorm_kernel<float><<<M, kNormThreads, 0, s>>>(h, (const float *)gain, (float *)out, c.cfg.hidden, c.cfg.rms_eps);
-    return cudaGetLastError();
+        return launch_k(rmsnorm_kernel<bf16>, M, kNormThreads, 0, s, h, (const bf16 *)gain, (bf16 *)out, c.cfg.hidden,
+                        c.cfg.rms_eps);
+    return launch_k(rmsnorm_kernel<float>, M, kNormThreads, 0, s, h, (const float *)gain, (float *)out, c.cfg.hidden,
+                    c.cfg.rms_eps);
 }
 
 cudaError_t launch_lm_finalize_impl(const Ctx &c, int mode, int B, int K, float temperature, int32_t *tok_out,
@@ -330,8 +346,7 @@ cudaError_t launch_lm_finalize_impl(const Ctx &c, int mode, int B, int K, float 
     a.given = given; a.rej_row = c.rej_row; a.err = c.err;
     const int rows = mode == 3 ? B : B * K;
     c.launches += 1;
-    lm_finalize_kernel<<<(rows + 7) / 8, 256, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_k(lm_finalize_kernel, (rows + 7) / 8, 256, 0, s, a);
 }
 
 cudaError_t launch_lm_finalize(const Ctx &c, int mode, int B, int K, float temperature, uint64_t, const int64_t *,
@@ -364,8 +379,7 @@ cudaError_t launch_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int K, fl
     CommitArgs a = commit_args(c, kv, B, K, temperature, seed, step, force_n, n_out, tokens_out, anchor_io,
                                append_out, append_stride, append_max);
     c.launches += 2;
-    commit_decide_kernel<<<B, 128, 0, s>>>(a);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_k(commit_decide_kernel, B, 128, 0, s, a);
     if (e != cudaSuccess) return e;
     if (temperature > 0.f && !force_n) {
         // residual draw at the rejected row: one LM-head pass over the two
@@ -381,8 +395,7 @@ cudaError_t launch_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int K, fl
         e = launch_lm_finalize_impl(c, 3, B, K, temperature, nullptr, nullptr, s);
         if (e != cudaSuccess) return e;
     }
-    commit_apply_kernel<<<1, 128, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_k(commit_apply_kernel, 1, 128, 0, s, a);
 }
 
 cudaError_t launch_ar_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int64_t *step, int32_t *token_out,
@@ -390,22 +403,19 @@ cudaError_t launch_ar_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int64_
                              cudaStream_t s)
 {
     c.launches += 1;
-    ar_commit_kernel<<<1, 128, 0, s>>>(B, c.g, step, token_out, anchor_io, kv.seq_lens, append_out, c.produced,
-                                       append_stride, append_max);
-    return cudaGetLastError();
+    return launch_k(ar_commit_kernel, 1, 128, 0, s, B, (const int32_t *)c.g, step, token_out, anchor_io, kv.seq_lens,
+                    append_out, c.produced, append_stride, append_max);
 }
 
 cudaError_t launch_set_lens(const Ctx &, int32_t *seq_lens, int b, int value, int32_t *anchor_out,
                             const int32_t *last_tok, cudaStream_t s)
 {
-    set_lens_kernel<<<1, 1, 0, s>>>(seq_lens, b, value, anchor_out, last_tok);
-    return cudaGetLastError();
+    return launch_k(set_lens_kernel, 1, 1, 0, s, seq_lens, b, value, anchor_out, last_tok);
 }
 
 cudaError_t launch_set_int(int32_t *p, int v, cudaStream_t s)
 {
-    set_int_kernel<<<1, 1, 0, s>>>(p, v);
-    return cudaGetLastError();
+    return launch_k(set_int_kernel, 1, 1, 0, s, p, v);
 }
 
 cudaError_t launch_logits_dump(const Ctx &c, const void *fin, int M, float *logits, cudaStream_t s)

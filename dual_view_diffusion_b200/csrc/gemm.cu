@@ -19,10 +19,11 @@
 //     (max, argmax, log-sum-exp terms, Gumbel-max sampling) so logits never
 //     reach HBM.
 //
-// bf16 uses tensor cores (mma.sync m16n8k16, fp32 accumulate); fp32 uses a
-// SIMT loop with the same tiling, scheduling and epilogues.
+// This file holds the SIMT mainloop (fp32 models, and bf16 shapes without
+// tensor maps) and the host dispatch; the bf16 tensor-core mainloop
+// (tcgen05, TMA, TMEM) is in gemm_tc.cu.  Both share tiling, scheduling and
+// the epilogues of gemm_epilogue.cuh.
 #include <math.h>
-#include <stdlib.h>
 
 #include "common.cuh"
 #include "gemm_epilogue.cuh"
@@ -30,7 +31,6 @@
 
 namespace orthrus {
 
-constexpr int kStages = 6;
 constexpr int kGemmThreads = 128;
 
 struct GemmShape {
@@ -54,122 +54,7 @@ __device__ __forceinline__ const T *weight_row(const GemmArgs &a, int nt, int r)
     return nullptr;
 }
 
-// ---------------------------------------------------------------- mainloops
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-                 "{%0,%1,%2,%3};\n"
-                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Shared-memory image of a 64-element (128-byte) row: its eight 16-byte
-// chunks are XOR-swizzled by the row index so ldmatrix is conflict-free.
-__device__ __forceinline__ int swz(int row, int chunk) { return row * 64 + ((chunk ^ (row & 7)) << 3); }
-
-struct MmaSmem {
-    bf16 w[kStages][kTileN * kTileK];
-    bf16 x[kStages][kTileM * kTileK];
-};
-
-__device__ void mainloop_mma(const GemmArgs &a, int mt, int nt, int c0, int c1, MmaSmem &sm,
-                             float (*tile)[kTilePad])
-{
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bf16 *wp[8];
-    const bf16 *xp[2];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) wp[i] = weight_row<bf16>(a, nt, (tid >> 3) + 16 * i);
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int row = mt * kTileM + (tid >> 3) + 16 * i;
-        xp[i] = row < a.M ? (const bf16 *)a.x + (size_t)row * a.Kd : nullptr;
-    }
-    const int ch = tid & 7;
-    const bf16 *wbase = (const bf16 *)a.w[0];
-    const bf16 *xbase = (const bf16 *)a.x;
-
-    auto load = [&](int stage, int c) {
-        const uint32_t sw = smem_u32(sm.w[stage]), sx = smem_u32(sm.x[stage]);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int row = (tid >> 3) + 16 * i;
-            const bf16 *src = wp[i] ? wp[i] + (size_t)c * kTileK + ch * 8 : wbase;
-            cp_async16(sw + 2 * swz(row, ch), src, wp[i] ? 16 : 0);
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int row = (tid >> 3) + 16 * i;
-            const bf16 *src = xp[i] ? xp[i] + (size_t)c * kTileK + ch * 8 : xbase;
-            cp_async16(sx + 2 * swz(row, ch), src, xp[i] ? 16 : 0);
-        }
-    };
-
-    float acc[2][4][4];
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[i][j][k] = 0.f;
-
-    const int n = c1 - c0;
-#pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) {
-        if (s < n) load(s, c0 + s);
-        cp_async_commit();
-    }
-    for (int it = 0; it < n; ++it) {
-        cp_async_wait<kStages - 2>();
-        __syncthreads();
-        const int st = it % kStages;
-        {
-            const int nx = it + kStages - 1;
-            if (nx < n) load(nx % kStages, c0 + nx);
-            cp_async_commit();
-        }
-        const uint32_t sw = smem_u32(sm.w[st]), sx = smem_u32(sm.x[st]);
-#pragma unroll
-        for (int ks = 0; ks < kTileK / 16; ++ks) {
-            uint32_t af[2][4], bfr[4][2];
-#pragma unroll
-            for (int m2 = 0; m2 < 2; ++m2) {
-                const int row = warp * 32 + m2 * 16 + (lane & 15);
-                ldsm_x4(sw + 2 * swz(row, ks * 2 + (lane >> 4)), af[m2][0], af[m2][1], af[m2][2], af[m2][3]);
-            }
-#pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                const int mi = lane >> 3;
-                const int tok = (2 * np + (mi >> 1)) * 8 + (lane & 7);
-                ldsm_x4(sx + 2 * swz(tok, ks * 2 + (mi & 1)), bfr[2 * np][0], bfr[2 * np][1], bfr[2 * np + 1][0],
-                        bfr[2 * np + 1][1]);
-            }
-#pragma unroll
-            for (int m2 = 0; m2 < 2; ++m2)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) mma_bf16(acc[m2][j], af[m2], bfr[j][0], bfr[j][1]);
-        }
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-#pragma unroll
-    for (int m2 = 0; m2 < 2; ++m2)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int f = warp * 32 + m2 * 16 + (lane >> 2) + (i >= 2 ? 8 : 0);
-                const int m = j * 8 + (lane & 3) * 2 + (i & 1);
-                tile[m][f] = acc[m2][j][i];
-            }
-}
-
+// ---------------------------------------------------------------- mainloop
 // SIMT mainloop: thread r owns output feature r of the tile for all 32 rows.
 template <class T>
 __device__ void mainloop_simt(const GemmArgs &a, int mt, int nt, int k0, int k1, float *xs,
@@ -203,13 +88,15 @@ __device__ void mainloop_simt(const GemmArgs &a, int mt, int nt, int k0, int k1,
 // ---------------------------------------------------------------- kernel
 // One-dimensional grid of persistent CTAs walking (m tile, n tile, segment)
 // units in order.
-template <class T, bool TC>
+template <class T>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(GemmArgs a, int n_mt, int n_nt)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     float(*tile)[kTilePad] = (float(*)[kTilePad])smem_raw;
     unsigned char *pipe = smem_raw + sizeof(float) * kTileM * kTilePad;
     __shared__ int s_last;
+    pdl_trigger();
+    pdl_wait();
     if (a.epi == EPI_RESAMPLE && *a.any_flag == 0) return;
 
     const int S = a.splits;
@@ -218,11 +105,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(GemmArgs a, int n
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
         const int seg = u % S, t = u / S, mt = t % n_mt, nt = t / n_mt;
         const int c0 = (int)((long)seg * chunks / S), c1 = (int)((long)(seg + 1) * chunks / S);
-        if constexpr (TC) {
-            mainloop_mma(a, mt, nt, c0, c1, *(MmaSmem *)pipe, tile);
-        } else {
-            mainloop_simt<T>(a, mt, nt, c0 * kTileK, min(c1 * kTileK, a.Kd), (float *)pipe, tile);
-        }
+        mainloop_simt<T>(a, mt, nt, c0 * kTileK, min(c1 * kTileK, a.Kd), (float *)pipe, tile);
         __syncthreads();
         if (!split_k_gather(a, tile, t, seg, threadIdx.x, &s_last, SyncBlock{}))
             continue;
@@ -256,10 +139,7 @@ int choose_splits(int N, int Kd)
 
 bool use_tensor_cores(const orthrus_config_t &c) { return c.dtype == ORTHRUS_BF16; }
 
-size_t gemm_smem_bytes(bool tc)
-{
-    return sizeof(float) * kTileM * kTilePad + (tc ? sizeof(MmaSmem) : sizeof(float) * kTileM * kTileK);
-}
+size_t gemm_smem_bytes() { return sizeof(float) * kTileM * kTilePad + sizeof(float) * kTileM * kTileK; }
 
 cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s)
 {
@@ -277,26 +157,16 @@ cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s)
     a.err = c.err;
     const long units = (long)n_mt * n_nt * a.splits;
     const int grid = (int)(units < kNumSMs ? units : kNumSMs);
-    const size_t smem = gemm_smem_bytes(tc);
+    const size_t smem = gemm_smem_bytes();
     if (tc) {
         const cudaError_t e = launch_gemm_tc(c, a, n_mt, n_nt, grid, s);
         if (e != cudaErrorNotSupported) return e;
     }
     c.launches += 1;
-    if (tc && getenv("ORTHRUS_GEMM_MMA_SYNC")) {
-        gemm_kernel<bf16, true><<<grid, kGemmThreads, smem, s>>>(a, n_mt, n_nt);
-    } else if (c.cfg.dtype == ORTHRUS_BF16) {
-        gemm_kernel<bf16, false><<<grid, kGemmThreads, smem, s>>>(a, n_mt, n_nt);
-    } else {
-        gemm_kernel<float, false><<<grid, kGemmThreads, smem, s>>>(a, n_mt, n_nt);
-    }
-    return cudaGetLastError();
+    if (c.cfg.dtype == ORTHRUS_BF16) return launch_k(gemm_kernel<bf16>, grid, kGemmThreads, smem, s, a, n_mt, n_nt);
+    return launch_k(gemm_kernel<float>, grid, kGemmThreads, smem, s, a, n_mt, n_nt);
 }
 
-cudaError_t gemm_init_attributes()
-{
-    return cudaFuncSetAttribute(gemm_kernel<bf16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)gemm_smem_bytes(true));
-}
+cudaError_t gemm_init_attributes() { return cudaSuccess; }
 
 }  // namespace orthrus

@@ -142,7 +142,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     TcSmem &sm = *(TcSmem *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    if (a.epi == EPI_RESAMPLE && *a.any_flag == 0) return;
+    if (a.epi == EPI_RESAMPLE) {   // the flag comes from the previous kernel
+        pdl_wait();
+        if (*a.any_flag == 0) return;
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
 
@@ -168,7 +171,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
 
     if (warp == 0) {
         if (lane == 0) {   // ------------------------------------------- producer
+            // Weights never depend on earlier kernels: the first unit's first
+            // stages are requested before waiting for the predecessor grid;
+            // their activation tiles follow once it has completed.
             uint32_t stage = 0, phase = 0;
+            int deferred = 0;   // stages whose X tile is still to be requested
             for (int u = blockIdx.x; u < units && !*abort; u += gridDim.x) {
                 const int seg = u % S, t = u / S, mt = t % n_mt, nt = t / n_mt;
                 const int c0 = (int)((long)seg * chunks / S), c1 = (int)((long)(seg + 1) * chunks / S);
@@ -177,7 +184,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                 if (a.epi != EPI_SWIGLU) {
                     while (wsel < 2 && wrow >= a.wrows[wsel]) { wrow -= a.wrows[wsel]; ++wsel; }
                 }
+                const bool first = u == (int)blockIdx.x;
                 for (int c = c0; c < c1; ++c) {
+                    if (first && deferred >= 0 && c - c0 == kTcStages) {
+                        pdl_wait();
+                        for (int i = 0; i < deferred; ++i)
+                            tma_load_2d(sm.x[i], &maps.x, (c0 + i) * kTileK, mt * kTileM, &sm.full[i]);
+                        deferred = -1;
+                    }
                     if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort)) break;
                     mbar_expect_tx(&sm.full[stage], kStageWBytes + kStageXBytes);
                     if (a.epi == EPI_SWIGLU) {
@@ -186,10 +200,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                     } else {
                         tma_load_2d(sm.w[stage], &maps.w[wsel], c * kTileK, wrow, &sm.full[stage]);
                     }
-                    tma_load_2d(sm.x[stage], &maps.x, c * kTileK, mt * kTileM, &sm.full[stage]);
+                    if (first && deferred >= 0) ++deferred;
+                    else tma_load_2d(sm.x[stage], &maps.x, c * kTileK, mt * kTileM, &sm.full[stage]);
                     if (++stage == kTcStages) { stage = 0; phase ^= 1; }
                 }
+                if (first && deferred >= 0) {   // first unit shorter than the ring
+                    pdl_wait();
+                    for (int i = 0; i < deferred; ++i)
+                        tma_load_2d(sm.x[i], &maps.x, (c0 + i) * kTileK, mt * kTileM, &sm.full[i]);
+                    deferred = -1;
+                }
             }
+            if (deferred >= 0) pdl_wait();
+            pdl_trigger();   // every load of this CTA is issued
         }
         __syncwarp();   // lanes 1..31 wait for the producer lane before the block barrier
     } else if (warp == 1) {
@@ -221,6 +244,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
         }
         __syncwarp();   // lanes 1..31 wait for the MMA lane before the block barrier
     } else {   // --------------------------------------------------------- epilogue
+        pdl_wait();                                  // the epilogues read and write predecessor data
         const int et = threadIdx.x - 64;            // 0..127
         const int q = warp & 3;                      // TMEM lane quarter of this warp
         int local = 0;
@@ -311,8 +335,7 @@ cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, 
     if (it == c.tmaps.end()) return cudaErrorNotSupported;
     maps.x = it->second;
     c.launches += 1;
-    gemm_tc_kernel<<<grid, kTcThreads, gemm_tc_smem_bytes(), s>>>(maps, a, n_mt, n_nt);
-    return cudaGetLastError();
+    return launch_k(gemm_tc_kernel, grid, kTcThreads, gemm_tc_smem_bytes(), s, maps, a, n_mt, n_nt);
 }
 
 }  // namespace orthrus
