@@ -193,9 +193,11 @@ class Engine:
         self.page_size = page_size
         self.pages_per_seq = (max_seq + page_size - 1) // page_size
         num_pages = max_batch * self.pages_per_seq
-        cshape = (n_layers, num_pages, shape.n_kv_heads, page_size, shape.head_dim)
-        self.k_pages = torch.zeros(cshape, dtype=self.tdtype, device=self.device)
-        self.v_pages = torch.zeros(cshape, dtype=self.tdtype, device=self.device)
+        # K pages [slot][dim], V pages transposed [dim][slot] (see orthrus_kv_t)
+        kshape = (n_layers, num_pages, shape.n_kv_heads, page_size, shape.head_dim)
+        vshape = (n_layers, num_pages, shape.n_kv_heads, shape.head_dim, page_size)
+        self.k_pages = torch.zeros(kshape, dtype=self.tdtype, device=self.device)
+        self.v_pages = torch.zeros(vshape, dtype=self.tdtype, device=self.device)
         self.block_table = torch.arange(num_pages, dtype=torch.int32, device=self.device).view(max_batch, -1)
         self.seq_lens = torch.zeros(max_batch, dtype=torch.int32, device=self.device)
         self.kv = KV(self.k_pages.data_ptr(), self.v_pages.data_ptr(), self.block_table.data_ptr(),

@@ -73,7 +73,9 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
     const size_t R = mb * c.max_block;
     const size_t Rw = std::max(R, (size_t)kPrefillChunk);
     const size_t Rlm = std::max(R, 2 * mb);
-    const size_t n_splits = (c.max_seq + c.split_tokens - 1) / c.split_tokens;
+    // cache splits of the longest sequence plus one slot for the diffusion block
+    const size_t n_splits = (c.max_seq + c.split_tokens - 1) / c.split_tokens + 1;
+    const size_t kp = ((size_t)c.max_block + 63) / 64 * 64;
     const size_t n_vtiles = (c.vocab + kTileN - 1) / kTileN;
     size_t gfloats;
     int gtickets;
@@ -83,11 +85,15 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
     auto take = [&](size_t bytes) { size_t o = off; off += align256(bytes); return o; };
     const size_t o_h = take(Rw * d * 4), o_a = take(Rw * d * es), o_q = take(Rw * hq * es), o_o = take(Rw * hq * es);
     const size_t o_act = take(Rw * F * es);
-    const size_t o_kd = take(L * R * hk * es), o_vd = take(L * R * hk * es);
+    const size_t o_kd = take(L * mb * kp * hk * es), o_vd = take(L * mb * kp * hk * es);
+    const size_t o_bp = take(2 * mb * kp * hk * es);
     const size_t o_fd = take(R * d * es), o_fv = take(R * d * es), o_rx = take(2 * mb * d * es);
-    // attention partials: [Rw][n_q][n_splits][hd] fp32 and [Rw][n_q][n_splits] float2
-    const size_t o_part = take(Rw * c.n_q_heads * n_splits * c.head_dim * 4);
-    const size_t o_ml = take(Rw * c.n_q_heads * n_splits * 8);
+    // attention partials [Rw][n_q][n_splits][hd] fp32 and [Rw][n_q][n_splits]
+    // float2: only the SIMT attention uses them (the tensor-core attention
+    // combines its splits on chip)
+    const bool simt_attn = !(c.dtype == ORTHRUS_BF16 && c.head_dim == 128);
+    const size_t o_part = take(simt_attn ? Rw * c.n_q_heads * n_splits * c.head_dim * 4 : 0);
+    const size_t o_ml = take(simt_attn ? Rw * c.n_q_heads * n_splits * 8 : 0);
     const size_t o_gp = take(std::max(gfloats, (size_t)1) * 4), o_gt = take((size_t)gtickets * 4);
     const size_t o_lm = take(Rlm * n_vtiles * sizeof(LmPart));
     const size_t o_tok = take(Rw * 4), o_pos = take(mb * 4), o_bt = take(mb * 4), o_pr = take(4);
@@ -112,6 +118,7 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
         x->err = (unsigned *)P(o_err); x->produced = (int32_t *)P(o_prod); x->step = (int64_t *)P(o_step);
         x->n_buf = (int32_t *)P(o_nb); x->tok_buf = (int32_t *)P(o_tb); x->anchor_buf = (int32_t *)P(o_ab);
         x->R = (int)R; x->Rw = (int)Rw; x->n_splits = (int)n_splits; x->n_vtiles = (int)n_vtiles;
+        x->kp = (int)kp; x->blk_pack = P(o_bp);
         x->esize = (int)es;
     }
     return total;
@@ -120,7 +127,7 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
 static void rebase(Ctx *x, char *ws)
 {
     auto fix = [&](auto *&p) { p = (std::remove_reference_t<decltype(p)>)(ws + (size_t)(const char *)p); };
-    fix(x->h); fix(x->a); fix(x->q); fix(x->attn_o); fix(x->act); fix(x->k_diff); fix(x->v_diff);
+    fix(x->h); fix(x->a); fix(x->q); fix(x->attn_o); fix(x->act); fix(x->k_diff); fix(x->v_diff); fix(x->blk_pack);
     fix(x->fin_draft); fix(x->fin_verify); fix(x->res_x); fix(x->attn_part); fix(x->attn_ml); fix(x->gemm_part);
     fix(x->gemm_ticket); fix(x->lm_part); fix(x->tok); fix(x->pos0); fix(x->bt_rows); fix(x->prefill_row);
     fix(x->draft); fix(x->logq); fix(x->lse_q); fix(x->g); fix(x->logp); fix(x->lse_p); fix(x->rej_row);
@@ -189,7 +196,6 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
 {
     const orthrus_config_t &f = c.cfg;
     const int M = B * K, hd = f.head_dim;
-    const size_t es = c.esize;
     cudaError_t e;
     for (int l = 0; l < f.n_layers; ++l) {
         const orthrus_layer_weights_t &W = c.layers[l];
@@ -200,7 +206,7 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
         q.wrows[0] = f.n_q_heads * hd; q.wrows[1] = q.wrows[2] = f.n_kv_heads * hd;
         q.N = q.wrows[0] + 2 * q.wrows[1];
         q.epi = EPI_QKV; q.q_out = c.q; q.n_q = f.n_q_heads; q.n_kv = f.n_kv_heads; q.hd = hd; q.layer = l;
-        q.kv_to_cache = view == 0; q.k_blk = c.k_diff; q.v_blk = c.v_diff; q.rows_max = c.R;
+        q.kv_to_cache = view == 0; q.k_blk = c.k_diff; q.v_blk = c.v_diff; q.kp = c.kp; q.bmax = f.max_batch;
         q.kv = kv_view(kv); q.pos0 = pos0; q.bt_rows = bt_rows; q.K = K; q.rope_theta = (double)f.rope_theta;
         {
             ProbeScope ps(c, 0, l, view, s);
@@ -209,15 +215,15 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
 
         AttnArgs at{};
         at.q = c.q; at.out = c.attn_o;
-        const size_t lay = (size_t)l * c.R * f.n_kv_heads * hd * es;
-        at.k_blk = (const char *)c.k_diff + lay; at.v_blk = (const char *)c.v_diff + lay;
+        at.k_blk = c.k_diff; at.v_blk = c.v_diff; at.kp = c.kp; at.bmax = f.max_batch;
+        at.blk_layer = l; at.blk_layers = f.n_layers;
         at.kv = kv_view(kv); at.layer = l; at.seq_lens = pos0; at.bt_rows = bt_rows;
         at.B = B; at.K = K; at.n_q = f.n_q_heads; at.n_kv = f.n_kv_heads; at.hd = hd; at.mode = view;
         at.split_tokens = f.split_tokens; at.n_splits = c.n_splits; at.part = c.attn_part; at.ml = c.attn_ml;
         at.err = c.err;
         {
             ProbeScope ps(c, 1, l, view, s);
-            if ((e = launch_attention(c, at, s)) != cudaSuccess) return e;
+            if ((e = launch_attention(c, at, s, c.Rw)) != cudaSuccess) return e;
         }
 
         GemmArgs o{};
@@ -549,12 +555,19 @@ orthrus_status_t orthrus_dual_view_attention(orthrus_ctx_t *c, const orthrus_kv_
         layer >= c->cfg.n_layers)
         return ORTHRUS_ERR_INVALID_ARG;
     const orthrus_config_t &f = c->cfg;
+    cudaStream_t s = (cudaStream_t)stream;
     AttnArgs at{};
-    at.q = q; at.out = out; at.k_blk = k_blk; at.v_blk = v_blk; at.kv = kv_view(*kv); at.layer = layer;
+    if (mode == 1) {   // user layout [B][K][n_kv][hd] -> the kernels' transient layouts
+        const size_t half = (size_t)f.max_batch * c->kp * f.n_kv_heads * f.head_dim * c->esize;
+        CK(launch_pack_block(*c, k_blk, v_blk, c->blk_pack, (char *)c->blk_pack + half, batch, K, c->kp, s));
+        at.k_blk = c->blk_pack; at.v_blk = (char *)c->blk_pack + half;
+    }
+    at.kp = c->kp; at.bmax = f.max_batch; at.blk_layer = 0; at.blk_layers = 1;
+    at.q = q; at.out = out; at.kv = kv_view(*kv); at.layer = layer;
     at.seq_lens = kv->seq_lens; at.bt_rows = c->bt_rows; at.B = batch; at.K = K; at.n_q = f.n_q_heads;
     at.n_kv = f.n_kv_heads; at.hd = f.head_dim; at.mode = mode; at.split_tokens = f.split_tokens;
     at.n_splits = c->n_splits; at.part = c->attn_part; at.ml = c->attn_ml; at.err = c->err;
-    CK(launch_attention(*c, at, (cudaStream_t)stream));
+    CK(launch_attention(*c, at, s, batch * K));
     return ORTHRUS_OK;
 }
 

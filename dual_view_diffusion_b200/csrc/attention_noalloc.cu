@@ -60,13 +60,21 @@ extern "C" orthrus_status_t orthrus_dual_view_attention_noalloc(const orthrus_co
         return ORTHRUS_ERR_INVALID_ARG;
     if (cfg->dtype == ORTHRUS_BF16 && cfg->head_dim == 128 && kv->page_size % 64) return ORTHRUS_ERR_INVALID_ARG;
 
-    // carve: [error word][block-table rows][(m, l) per split][O partial per split]
+    // carve: [error word][block-table rows][block K][block V][(m, l) per
+    // split][O partial per split]
     const size_t rows = (size_t)batch * K;
-    const size_t n_splits = ((size_t)cfg->max_seq + cfg->split_tokens - 1) / cfg->split_tokens;
+    const size_t es = cfg->dtype == ORTHRUS_BF16 ? 2 : 4;
+    const size_t kp = ((size_t)K + 63) / 64 * 64;
+    const size_t n_splits = ((size_t)cfg->max_seq + cfg->split_tokens - 1) / cfg->split_tokens + 1;
+    const size_t blk = (size_t)batch * cfg->n_kv_heads * kp * cfg->head_dim * es;
     const size_t off_rows = 256;
-    const size_t off_ml = off_rows + up256((size_t)batch * 4);
-    const size_t off_part = off_ml + up256(rows * cfg->n_q_heads * n_splits * sizeof(float2));
-    const size_t need = off_part + rows * cfg->n_q_heads * n_splits * cfg->head_dim * sizeof(float);
+    const size_t off_kb = off_rows + up256((size_t)batch * 4);
+    const size_t off_vb = off_kb + up256(mode == 1 ? blk : 0);
+    const size_t off_ml = off_vb + up256(mode == 1 ? blk : 0);
+    // split partials: SIMT attention only (the tensor-core path combines on chip)
+    const bool simt_attn = !(cfg->dtype == ORTHRUS_BF16 && cfg->head_dim == 128);
+    const size_t off_part = off_ml + up256(simt_attn ? rows * cfg->n_q_heads * n_splits * sizeof(float2) : 0);
+    const size_t need = off_part + (simt_attn ? rows * cfg->n_q_heads * n_splits * cfg->head_dim * sizeof(float) : 0);
     if (need > kNoAllocScratchBytes) return ORTHRUS_ERR_CAPACITY;
 
     int dev = 0;
@@ -90,15 +98,21 @@ extern "C" orthrus_status_t orthrus_dual_view_attention_noalloc(const orthrus_co
     if (launch_k(noalloc_identity_rows, (batch + 127) / 128, 128, 0, s, bt_rows, (int)batch) != cudaSuccess)
         return ORTHRUS_ERR_CUDA;
 
-    Ctx tmp;                      // only cfg is read by the launcher
+    Ctx tmp;                      // only cfg (and a tensor-map cache) is used by the launchers
     tmp.cfg = *cfg;
     AttnArgs at{};
-    at.q = q; at.out = out; at.k_blk = k_blk; at.v_blk = v_blk;
+    if (mode == 1) {
+        if (launch_pack_block(tmp, k_blk, v_blk, base + off_kb, base + off_vb, batch, K, (int)kp, s) != cudaSuccess)
+            return ORTHRUS_ERR_CUDA;
+        at.k_blk = base + off_kb; at.v_blk = base + off_vb;
+    }
+    at.kp = (int)kp; at.bmax = batch; at.blk_layer = 0; at.blk_layers = 1;
+    at.q = q; at.out = out;
     at.kv = KvView{kv->k_pages, kv->v_pages, kv->block_table, kv->num_pages, kv->page_size, kv->max_pages_per_seq};
     at.layer = layer; at.seq_lens = kv->seq_lens; at.bt_rows = bt_rows;
     at.B = batch; at.K = K; at.n_q = cfg->n_q_heads; at.n_kv = cfg->n_kv_heads; at.hd = cfg->head_dim;
     at.mode = mode; at.split_tokens = cfg->split_tokens; at.n_splits = (int)n_splits;
     at.part = (float *)(base + off_part); at.ml = (float2 *)(base + off_ml); at.err = err;
-    if (launch_attention(tmp, at, s) != cudaSuccess) return ORTHRUS_ERR_CUDA;
+    if (launch_attention(tmp, at, s, batch * K) != cudaSuccess) return ORTHRUS_ERR_CUDA;
     return ORTHRUS_OK;
 }

@@ -1,0 +1,693 @@
+// Dual-view attention on the tcgen05 tensor cores (bf16, head_dim 128).
+//
+// One cluster of C CTAs per (KV head, sequence x row group).  Its M = 128
+// query rows are the block rows x the GQA group sharing the KV head, so every
+// K/V tile staged in shared memory serves all of them (paper notes §2.2-2.3:
+// both views read the one AR cache).  The keys are cut into splits aligned to
+// absolute positions; CTA r of the cluster takes splits r, r + C, ... and, per
+// 64-key tile:
+//
+//   S = Q K^T       tcgen05.mma, M 128 x N 64 x K 128, into TMEM
+//   softmax         each softmax thread owns one query row (= TMEM lane): it
+//                   reads its 64 scores with tcgen05.ld, applies the view's
+//                   mask, updates its running max / sum in log2 units, and
+//                   writes the bf16 probabilities P (128-byte swizzled) to
+//                   shared memory
+//   O += P V        tcgen05.mma, M 128 x N 128 x K 64, into a TMEM accumulator
+//
+// O is rescaled in TMEM only when a warp's running max moved (a factor of
+// exactly 1 elsewhere, so skipping it changes no bit).  K tiles come from
+// pages laid out [slot][dim], V tiles from pages laid out [dim][slot] (both
+// operands K-major), both by TMA.  For the diffusion view the block's own K/V
+// form one extra split read from the transient buffer.  The C partial states
+// are merged through distributed shared memory; nothing goes to global memory
+// but the output rows.
+//
+// Roles: warp 0 TMA producer, warp 1 MMA issuer (one thread each), warps 2..5
+// softmax and combine.  All mbarrier waits are bounded.
+#include <cuda.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace orthrus {
+
+constexpr int kAtStages = 4;
+constexpr float kRescaleSlack = 8.0f;   // log2 units a row's max may grow before O is rescaled
+constexpr int kAtMaxCluster = 8;        // portable cluster size
+constexpr int kAtPreWait = 2;           // cache tiles requested before waiting for the predecessor
+constexpr int kAtThreads = 320;   // producer warp, MMA warp, two softmax warpgroups
+constexpr int kAtRows = 128;
+constexpr int kAtKeys = 64;
+constexpr long long kAtSpinCycles = 4000000000LL;   // ~2 s at the B200 SM clock
+
+struct AtSmem {
+    alignas(1024) unsigned char q[2][kAtRows * 128];              // Q dims 0-63 / 64-127, 16 KiB each
+    alignas(1024) unsigned char k[kAtStages][2][kAtKeys * 128];   // K tile halves, 8 KiB each
+    alignas(1024) unsigned char v[kAtStages][128 * 128];          // V^T tile [128 dims][64 keys], 16 KiB
+    alignas(1024) unsigned char p[2][kAtRows * 128];              // P [128 rows][64 keys], 16 KiB, per accumulator
+    alignas(8) uint64_t q_full, full[kAtStages], empty[kAtStages], s_full[2], p_full[2], o_done[2];
+    float2 xml[2][kAtRows];   // (m, l) of each accumulator, per row
+    uint64_t ready;       // one arrival from every CTA of the cluster whose ring is free
+    uint64_t land_full;   // bytes of the partial rows pushed to this CTA
+    uint32_t tmem_base;
+    int abort;
+};
+// Once the last P.V is done, q..p (192 KiB) is reused for the combine:
+// the CTA's own merged rows and (m, l) (staging), and the rows the other
+// CTAs push to it (landing).
+constexpr uint32_t kStageO = 0, kStageMl = 64 * 1024, kLandO = 68 * 1024, kLandMl = 132 * 1024;
+static_assert(kLandMl + kAtRows * 8 <= 2 * 16384 + kAtStages * 32768 + 2 * 16384, "combine area");
+
+// TMEM columns: two O accumulators (even / odd tiles) [0, 256), S double
+// buffer [256, 384)
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemCols = 512;
+
+__device__ __forceinline__ void at_mbar_init(uint64_t *b, uint32_t n)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(b)), "r"(n));
+}
+__device__ __forceinline__ void at_expect(uint64_t *b, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void at_arrive(uint64_t *b)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(b)) : "memory");
+}
+// Bounded wait (about two seconds of SM clock); false on timeout, or when
+// another role of the CTA already gave up.
+__device__ __forceinline__ bool at_wait(uint64_t *b, uint32_t parity, volatile int *abort)
+{
+    const long long t0 = clock64();
+    for (long i = 0;; ++i) {
+        uint32_t ok;
+        asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+                     : "=r"(ok) : "r"(smem_u32(b)), "r"(parity) : "memory");
+        if (ok) return true;
+        if ((i & 255) == 255) {
+            if (*abort) return false;
+            if (clock64() - t0 > kAtSpinCycles) break;
+        }
+    }
+    *abort = 1;
+    return false;
+}
+__device__ __forceinline__ void at_tma2(void *dst, const CUtensorMap *m, int x, int y, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
+        ::"r"(smem_u32(dst)), "l"((uint64_t)m), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void at_tma4(void *dst, const CUtensorMap *m, int x, int y, int z, int w, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];\n"
+        ::"r"(smem_u32(dst)), "l"((uint64_t)m), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ uint64_t at_desc(const void *p)
+{
+    const uint32_t a = smem_u32(p);
+    return (uint64_t)((a & 0x3FFFF) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// kind::f16, fp32 accumulate, bf16 A/B, K-major, M = 128
+__host__ __device__ constexpr uint32_t idesc_n(int n) { return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | (8u << 24); }
+
+__device__ __forceinline__ void at_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc)
+{
+    asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+                 ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+__device__ __forceinline__ void at_commit(uint64_t *b)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ void at_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void at_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+
+#define AT_LD32(taddr, r)                                                                                         \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15," \
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"                     \
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), \
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),        \
+                   "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),      \
+                   "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),      \
+                   "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                                            \
+                 : "r"(taddr))
+#define AT_ST32(taddr, r)                                                                                         \
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15," \
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"                          \
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),        \
+                   "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),    \
+                   "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), \
+                   "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), \
+                   "r"(r[31]) : "memory")
+__device__ __forceinline__ void at_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void at_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+struct AtMaps {
+    CUtensorMap q;    // 4-D (dim, head in group, kv head, block row), box {64, g, 1, rows/g}
+    CUtensorMap kc;   // 2-D cache K rows [slot rows][128], box {64, 64}
+    CUtensorMap vc;   // 2-D cache V^T rows [dim rows][page_size], box {64, 128}
+    CUtensorMap kb;   // 2-D transient K [rows][128], box {64, 64}
+    CUtensorMap vb;   // 2-D transient V^T [dim rows][Kp], box {64, 128}
+};
+
+// Key range of split s for sequence b: cache splits [s*S, ...) of the cache
+// part; in the diffusion view split n_split_grid is the block's own keys.
+struct AtSplit {
+    int key0, key1, slot, ntiles;
+    bool block;
+};
+__device__ __forceinline__ AtSplit at_split(const AttnArgs &a, int s, int n_split_grid, int t)
+{
+    AtSplit r;
+    r.block = a.mode == 1 && s == n_split_grid;
+    if (r.block) {
+        r.key0 = t; r.key1 = t + a.K; r.slot = a.n_splits - 1;
+    } else {
+        r.key0 = s * a.split_tokens;
+        r.key1 = min(r.key0 + a.split_tokens, a.mode == 0 ? t + a.K : t);
+        r.slot = s;
+    }
+    r.ntiles = r.key1 > r.key0 ? (r.key1 - r.key0 + kAtKeys - 1) / kAtKeys : 0;
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t map_peer_addr(uint32_t local, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_arrive_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory"); }
+// arrive on an mbarrier of another CTA of the cluster (release at cluster scope)
+__device__ __forceinline__ void arrive_peer(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+}
+// bulk copy of this CTA's shared memory into another CTA's, completing bytes
+// on that CTA's mbarrier
+__device__ __forceinline__ void bulk_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t mbar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+                 ::"r"(dst), "r"(src), "r"(bytes), "r"(mbar) : "memory");
+}
+__device__ __forceinline__ float ex2(float x)   // 2^x, MUFU; subnormal results flush to zero
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// grid (kv head, sequence x row group, C) with clusters of C CTAs along z:
+// cluster = one (sequence, KV head, row group).  CTA r of the cluster loads
+// its Q rows once and runs the online softmax over all keys of splits r,
+// r + C, r + 2C, ... (a split's keys never depend on which block is being
+// decoded, and keys outside a row's window are exact no-ops).  Even and odd
+// tiles go to two independent accumulators (O, m, l), so the softmax of one
+// tile never waits for the P.V of the tile just before it; the two are merged
+// at the end.  The C partial states are then combined on chip: CTA q owns rows
+// [q*128/C, (q+1)*128/C); every CTA bulk-copies its merged rows to their
+// owner once the owner's ring is free, and each owner sums the C states in
+// rank order from its own shared memory.
+template <int C>
+__global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a,
+                                                                int n_split_grid)
+{
+    extern __shared__ __align__(1024) unsigned char at_raw[];
+    AtSmem &sm = *(AtSmem *)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
+    pdl_trigger();
+    const int kvh = blockIdx.x;
+    const int rgroups = gridDim.y / a.B, b = blockIdx.y / rgroups, rg = blockIdx.y % rgroups;
+    const int g = a.n_q / a.n_kv, ksub = kAtRows / g;          // block rows per row group
+    const int k_lo = rg * ksub, k_hi = min(a.K, k_lo + ksub);
+    if (k_lo >= a.K) {   // the whole cluster shares rg
+        pdl_wait();
+        return;
+    }
+    constexpr int rpc = kAtRows / C;   // rows owned per CTA
+    const int r = (int)cluster_rank();
+    const int n_total = n_split_grid + (a.mode == 1 ? 1 : 0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int *abort = &sm.abort;
+    // t, the block table and its row were written by kernels that completed
+    // before the predecessor of this one started (every launch waits on its
+    // own predecessor), so they may be read before griddepcontrol.wait
+    const int t = a.seq_lens[b];
+    const int bt_row = a.bt_rows[b];
+    // Flat tile f of this CTA is tile f % tps of split r + C * (f / tps) for
+    // every cache tile (only the last cache split can be short, and only
+    // block tiles follow it).  Warp 0 looks up the pages of 32 flat tiles at
+    // a time, one per lane.
+    const int tps = a.split_tokens / kAtKeys;
+    const int cache_lim = a.mode == 0 ? t + a.K : t;
+    auto lookup = [&](int f) {
+        const int sl = r + C * (f / tps);
+        const int key = sl * a.split_tokens + (f % tps) * kAtKeys;
+        if (sl >= n_split_grid || key >= cache_lim) return 0;
+        const int pidx = key / a.kv.page_size;
+        int page = (pidx < a.kv.max_pages) ? a.kv.block_table[(size_t)bt_row * a.kv.max_pages + pidx] : -1;
+        if (page < 0 || page >= a.kv.num_pages) { raise_err(a.err, ORTHRUS_DEVERR_CAPACITY); page = 0; }
+        return page;
+    };
+    int pg = warp == 0 ? lookup(lane) : 0;
+
+    if (threadIdx.x == 0) {
+        at_mbar_init(&sm.q_full, 1);
+        for (int i = 0; i < kAtStages; ++i) { at_mbar_init(&sm.full[i], 1); at_mbar_init(&sm.empty[i], 1); }
+        for (int i = 0; i < 2; ++i) {
+            at_mbar_init(&sm.s_full[i], 1);
+            at_mbar_init(&sm.p_full[i], 128);
+            at_mbar_init(&sm.o_done[i], 1);
+        }
+        at_mbar_init(&sm.ready, C);
+        at_mbar_init(&sm.land_full, 1);
+        sm.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        // every CTA of the cluster pushes rpc rows of O and of (m, l) here
+        at_expect(&sm.land_full, (uint32_t)C * rpc * (512u + 8u));
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&sm.tmem_base)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+    }
+    at_fence_before();
+    __syncthreads();
+    at_fence_after();
+    // the barriers of every CTA are initialised before any CTA signals another
+    cluster_arrive_relaxed();
+    const uint32_t tmem = sm.tmem_base;
+    int my_tiles = 0;
+    for (int s = r; s < n_total; s += C) my_tiles += at_split(a, s, n_split_grid, t).ntiles;
+
+    uint32_t jj = 0;
+    bool ok = true;
+    const int q4 = warp & 3, row = q4 * 32 + lane;   // softmax threads: query row = TMEM lane
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+
+    if (warp == 0) {   // ------------------------------------------------------ producer
+        // all 32 lanes walk the tiles together (page lookups); lane 0 issues.
+        // Up to kAtPreWait cache tiles below t (which the predecessor cannot
+        // be writing) are requested before waiting for it; Q right after.
+        uint32_t stage = 0, phase = 0;
+        bool waited = false, stop = false;
+        auto ensure_wait = [&]() {
+            if (waited) return;
+            pdl_wait();
+            waited = true;
+            if (my_tiles == 0) return;   // nothing will consume Q
+            const uint32_t qbytes = 2u * 128u * (uint32_t)(g * min(a.K, ksub));   // the map's box
+            at_expect(&sm.q_full, qbytes);
+            at_tma4(sm.q[0], &maps.q, 0, 0, kvh, b * a.K + k_lo, &sm.q_full);
+            at_tma4(sm.q[1], &maps.q, 64, 0, kvh, b * a.K + k_lo, &sm.q_full);
+        };
+        int f = 0;
+        for (int s = r; s < n_total && !stop; s += C) {
+            const AtSplit sp = at_split(a, s, n_split_grid, t);
+            for (int j = 0; j < sp.ntiles; ++j, ++f) {
+                if (f > 0 && (f & 31) == 0) pg = lookup(f + lane);
+                const int page = __shfl_sync(0xffffffffu, pg, f & 31);
+                int go = 1;
+                if (lane == 0) {
+                    const int p0 = sp.key0 + j * kAtKeys;
+                    if (sp.block || p0 + kAtKeys > t || f >= kAtPreWait) ensure_wait();
+                    if (!at_wait(&sm.empty[stage], phase ^ 1, abort)) {
+                        go = 0;
+                    } else {
+                        at_expect(&sm.full[stage], 2u * 8192u + 16384u);
+                        if (sp.block) {
+                            const int krow = (a.blk_layer * a.bmax + b) * a.n_kv + kvh;
+                            at_tma2(sm.k[stage][0], &maps.kb, 0, krow * a.kp + j * kAtKeys, &sm.full[stage]);
+                            at_tma2(sm.k[stage][1], &maps.kb, 64, krow * a.kp + j * kAtKeys, &sm.full[stage]);
+                            at_tma2(sm.v[stage], &maps.vb, j * kAtKeys, krow * 128, &sm.full[stage]);
+                        } else {
+                            const int off = p0 % a.kv.page_size;
+                            const int hrow = (a.layer * a.kv.num_pages + page) * a.n_kv + kvh;
+                            at_tma2(sm.k[stage][0], &maps.kc, 0, hrow * a.kv.page_size + off, &sm.full[stage]);
+                            at_tma2(sm.k[stage][1], &maps.kc, 64, hrow * a.kv.page_size + off, &sm.full[stage]);
+                            at_tma2(sm.v[stage], &maps.vc, off, hrow * 128, &sm.full[stage]);
+                        }
+                        if (++stage == kAtStages) { stage = 0; phase ^= 1; }
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, go, 0)) { stop = true; break; }
+            }
+        }
+        if (lane == 0) ensure_wait();
+        __syncwarp();
+    } else if (warp == 1) {
+        pdl_wait();
+        if (lane == 0 && my_tiles > 0) {   // ---------------------------------- MMA issuer
+            // S of tile i is issued before P.V of tile i-1; tile i uses S
+            // buffer, P buffer and O accumulator i & 1
+            bool good = at_wait(&sm.q_full, 0, abort);
+            uint32_t stage = 0, phase = 0, i = 0;
+            uint32_t pv_stage = 0;          // stage of the tile waiting for its P.V
+            bool pv_pending = false;
+            const uint32_t id_s = idesc_n(kAtKeys), id_o = idesc_n(128);
+            auto issue_pv = [&](uint32_t pi) {   // P.V of tile pi (waits for its P)
+                const uint32_t h = pi & 1;
+                if (!at_wait(&sm.p_full[h], (pi >> 1) & 1, abort)) return false;
+                at_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    at_mma(tmem + kTmemO + h * 128, at_desc(sm.p[h]) + 2 * kk, at_desc(sm.v[pv_stage]) + 2 * kk, id_o,
+                           (pi >= 2 || kk > 0) ? 1u : 0u);
+                at_commit(&sm.o_done[h]);
+                at_commit(&sm.empty[pv_stage]);
+                return true;
+            };
+            for (int s = r; s < n_total && good; s += C) {
+                const AtSplit sp = at_split(a, s, n_split_grid, t);
+                for (int j = 0; j < sp.ntiles && good; ++j, ++i) {
+                    if (!at_wait(&sm.full[stage], phase, abort)) { good = false; break; }
+                    at_fence_after();
+                    const uint32_t sbuf = kTmemS + (i & 1) * kAtKeys;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const int h = kk >> 2, o = 2 * (kk & 3);
+                        at_mma(tmem + sbuf, at_desc(sm.q[h]) + o, at_desc(sm.k[stage][h]) + o, id_s, kk > 0 ? 1u : 0u);
+                    }
+                    at_commit(&sm.s_full[i & 1]);
+                    if (pv_pending && !issue_pv(i - 1)) { good = false; break; }
+                    pv_pending = true;
+                    pv_stage = stage;
+                    if (++stage == kAtStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (good && pv_pending) issue_pv(i - 1);
+        }
+        __syncwarp();
+    } else {   // ------------------------------------------------- softmax, warpgroup h: tiles jj with jj & 1 == h
+        pdl_wait();
+        const int h = (warp - 2) >> 2;
+        const int rr = k_lo * g + row;                            // row within the sequence's K*g rows
+        const int kblk = rr / g;
+        const float scale = 1.4426950408889634f / sqrtf(128.f);
+        // exponents are taken relative to m_use, a running max that is only
+        // raised (and O rescaled) when a score exceeds it by more than
+        // kRescaleSlack: the result is the same softmax, P stays <= 2^slack
+        float m_use = -INFINITY, l_run = 0.f;
+        int last = -1;   // this warpgroup's last tile
+        for (int s = r; s < n_total && ok; s += C) {
+            const AtSplit sp = at_split(a, s, n_split_grid, t);
+            const int lim = min(sp.key1, sp.block ? sp.key1 : (a.mode == 0 ? t + kblk + 1 : sp.key1));
+            for (int j = 0; j < sp.ntiles; ++j, ++jj) {
+                if ((int)(jj & 1) != h) continue;
+                last = (int)jj;
+                ok = at_wait(&sm.s_full[h], (jj >> 1) & 1, abort);
+                if (!ok) break;
+                at_fence_after();
+                uint32_t sr[64];
+                const uint32_t sbuf = kTmemS + h * kAtKeys;
+                AT_LD32(tmem + lane_off + sbuf, sr);
+                AT_LD32(tmem + lane_off + sbuf + 32, (sr + 32));
+                at_wait_ld();
+                const int vis = lim - (sp.key0 + j * kAtKeys);   // keys of this tile the row sees
+                if (vis < kAtKeys) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (c >= vis) sr[c] = __float_as_uint(-INFINITY);
+                }
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int c = 0; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(sr[c]));
+                const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale;
+                float alpha = 1.0f;
+                if (tmax > m_use + kRescaleSlack || (m_use == -INFINITY && tmax > -INFINITY)) {
+                    alpha = m_use == -INFINITY ? 0.f : ex2(m_use - tmax);
+                    m_use = tmax;
+                }
+                const float nmu = m_use == -INFINITY ? 0.f : -m_use;
+                float rs[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float p0v = ex2(fmaf(__uint_as_float(sr[2 * c]), scale, nmu));
+                    const float p1v = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), scale, nmu));
+                    rs[c & 3] += p0v + p1v;
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0v, p1v);
+                    pk[c] = *(const uint32_t *)&h2;
+                }
+                if (jj >= 2) {   // P.V of tile jj-2 done: O_h and P_h are free
+                    ok = at_wait(&sm.o_done[h], ((jj - 2) >> 1) & 1, abort);
+                    if (!ok) break;
+                    at_fence_after();
+                    if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t orr[32];
+                            AT_LD32(tmem + lane_off + kTmemO + h * 128 + q * 32, orr);
+                            at_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+                            AT_ST32(tmem + lane_off + kTmemO + h * 128 + q * 32, orr);
+                        }
+                        at_wait_st();
+                    }
+                }
+                // P row -> shared memory, 128-byte swizzle (16-byte chunk c at c ^ (row & 7))
+                unsigned char *prow = sm.p[h] + row * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *(uint4 *)(prow + ((c ^ (row & 7)) << 4)) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                at_fence_before();
+                at_arrive(&sm.p_full[h]);
+                l_run = l_run * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+            }
+        }
+        // this warpgroup's last P.V (tcgen05 operations complete in issue order)
+        if (ok && last >= 0) ok = at_wait(&sm.o_done[h], (last >> 1) & 1, abort);
+        sm.xml[h][row] = (ok && last >= 0) ? make_float2(m_use, l_run) : make_float2(-INFINITY, 0.f);
+        at_fence_after();
+        __syncwarp();
+    }
+
+    // ------------------------------------------------------------------ combine
+    unsigned char *area = sm.q[0];
+    const uint32_t area_u = smem_u32(area);
+    cluster_wait();   // every CTA's barriers are initialised
+    if (warp >= 2) {
+        const int h = (warp - 2) >> 2;
+        asm volatile("bar.sync 1, 256;\n" ::: "memory");   // both warpgroups: every P.V is done
+        // the K/V ring, Q and P are no longer read: tell every CTA it may push here
+        if (warp == 2 && lane < C) arrive_peer(map_peer_addr(smem_u32(&sm.ready), lane));
+        __syncwarp();
+        // merge the two accumulators into (O, m, l) of this row -> staging;
+        // warpgroup h takes dims [64h, 64h + 64)
+        const float2 x0 = sm.xml[0][row], x1 = sm.xml[1][row];
+        const float M = fmaxf(x0.x, x1.x);
+        const float w0 = x0.y > 0.f ? ex2(x0.x - M) : 0.f, w1 = x1.y > 0.f ? ex2(x1.x - M) : 0.f;
+        const float l = w0 * x0.y + w1 * x1.y;
+        float *so = (float *)(area + kStageO) + row * 128;
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+            const int q = 2 * h + qq;
+            uint32_t o0[32], o1[32];
+            AT_LD32(tmem + lane_off + kTmemO + q * 32, o0);
+            AT_LD32(tmem + lane_off + kTmemO + 128 + q * 32, o1);
+            at_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float4 v;
+                float *vv = &v.x;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float y0 = w0 != 0.f ? w0 * __uint_as_float(o0[4 * c + e]) : 0.f;
+                    const float y1 = w1 != 0.f ? w1 * __uint_as_float(o1[4 * c + e]) : 0.f;
+                    vv[e] = y0 + y1;
+                }
+                *(float4 *)(so + (((q * 8 + c) ^ (row & 31)) << 2)) = v;
+            }
+        }
+        if (h == 0) ((float2 *)(area + kStageMl))[row] = l > 0.f ? make_float2(M, l) : make_float2(-INFINITY, 0.f);
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        at_fence_before();
+        __syncwarp();
+        asm volatile("bar.sync 1, 256;\n" ::: "memory");
+        if (threadIdx.x == 64) {   // push rows [q*rpc, (q+1)*rpc) to CTA q once its ring is free
+            if (at_wait(&sm.ready, 0, abort)) {
+#pragma unroll
+                for (int q = 0; q < C; ++q) {
+                    const uint32_t mbar = map_peer_addr(smem_u32(&sm.land_full), q);
+                    bulk_to_peer(map_peer_addr(area_u + kLandO + r * rpc * 512, q), area_u + kStageO + q * rpc * 512,
+                                 rpc * 512, mbar);
+                    bulk_to_peer(map_peer_addr(area_u + kLandMl + r * rpc * 8, q), area_u + kStageMl + q * rpc * 8,
+                                 rpc * 8, mbar);
+                }
+            }
+        }
+        __syncwarp();
+        // ------------------------------------------------------- owner: rows [r*rpc, (r+1)*rpc)
+        constexpr int tpr = 256 / rpc;            // threads per owned row: chunks cc, cc + tpr, ...
+        const bool landed = at_wait(&sm.land_full, 0, abort);
+        const int et = threadIdx.x - 64;
+        const int rl = et / tpr, cc = et % tpr;
+        const int orow = r * rpc + rl;
+        const float2 *lml = (const float2 *)(area + kLandMl);
+        const float *lo = (const float *)(area + kLandO);
+        float wc[C];
+        float Mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            const float2 ml = lml[c * rpc + rl];
+            if (ml.y > 0.f) Mx = fmaxf(Mx, ml.x);
+        }
+        float L = 0.f;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            const float2 ml = lml[c * rpc + rl];
+            wc[c] = ml.y > 0.f ? ex2(ml.x - Mx) : 0.f;
+            L += wc[c] * ml.y;
+        }
+        const int rrow = k_lo * g + orow, k = rrow / g, jh = rrow % g;
+        if (landed && orow < (k_hi - k_lo) * g && L > 0.f) {
+            const float inv = 1.0f / L;
+            bf16 *o = (bf16 *)a.out + ((size_t)(b * a.K + k) * a.n_q + kvh * g + jh) * 128;
+#pragma unroll
+            for (int ch = cc; ch < 32; ch += tpr) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int c = 0; c < C; ++c) {
+                    if (wc[c] == 0.f) continue;
+                    const float4 v = *(const float4 *)(lo + (size_t)(c * rpc + rl) * 128 + ((ch ^ (orow & 31)) << 2));
+                    acc.x = fmaf(wc[c], v.x, acc.x); acc.y = fmaf(wc[c], v.y, acc.y);
+                    acc.z = fmaf(wc[c], v.z, acc.z); acc.w = fmaf(wc[c], v.w, acc.w);
+                }
+                const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+                const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+                *(uint2 *)(o + ch * 4) = make_uint2(*(const uint32_t *)&lo2, *(const uint32_t *)&hi2);
+            }
+        }
+        __syncwarp();
+    }
+    // every CTA has received all its rows (so every copy out of this CTA is
+    // complete) before any CTA leaves
+    cluster_arrive_relaxed();
+    cluster_wait();
+
+    if (sm.abort && threadIdx.x == 0) raise_err(a.err, ORTHRUS_DEVERR_TIMEOUT);
+    if (warp == 1) {
+        __syncwarp();
+        at_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+// ---------------------------------------------------------------- host
+bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+bool make_tmap_box(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows);
+bool make_tmap_q4(CUtensorMap *m, const void *q, int rows_total, int n_q, int n_kv, int hd, int ksub);
+
+size_t attn_tc_smem_bytes() { return sizeof(AtSmem) + 1024; }
+
+// CTAs per (sequence, KV head, row group): a power of two up to 8 that keeps
+// one row group of the whole batch within one wave of SMs.  A function of the
+// batch and model shape only (not of the block size), so a row is reduced in
+// the same order whatever block it is in.
+int attn_cluster_size(int n_kv, int B)
+{
+    const int others = n_kv * B;
+    int C = 1;
+    while (C < kAtMaxCluster && (2 * C) * others <= kNumSMs) C *= 2;
+    return C;
+}
+
+cudaError_t attn_tc_init_attributes()
+{
+    const int bytes = (int)attn_tc_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    return e;
+}
+
+// Tensor maps for one call.  rows_total: token rows the q buffer holds.
+bool attn_tc_maps(const AttnArgs &a, int n_layers, int rows_total, AtMaps *m)
+{
+    memset(m, 0, sizeof(*m));
+    const int g = a.n_q / a.n_kv;
+    if (a.hd != 128 || kAtRows % g || a.kv.page_size % 64) return false;
+    const int ksub = std::min(a.K, kAtRows / g);
+    if (!make_tmap_q4(&m->q, a.q, rows_total, a.n_q, a.n_kv, a.hd, ksub)) return false;
+    const uint64_t heads = (uint64_t)n_layers * a.kv.num_pages * a.n_kv;
+    if (!make_tmap_box(&m->kc, a.kv.k_pages, heads * a.kv.page_size, 128, 64, 64)) return false;
+    if (!make_tmap_box(&m->vc, a.kv.v_pages, heads * 128, a.kv.page_size, 64, 128)) return false;
+    if (a.mode == 1) {
+        const uint64_t bh = (uint64_t)a.blk_layers * a.bmax * a.n_kv;
+        if (!make_tmap_box(&m->kb, a.k_blk, bh * a.kp, 128, 64, 64)) return false;
+        if (!make_tmap_box(&m->vb, a.v_blk, bh * 128, a.kp, 64, 128)) return false;
+    } else {
+        m->kb = m->kc;
+        m->vb = m->vc;
+    }
+    return true;
+}
+
+cudaError_t launch_attn_tc(const AttnArgs &a, const AtMaps &maps, int n_split_grid, cudaStream_t s);
+
+// Maps for the call, built once per distinct (buffers, shape) and kept in
+// the context.
+cudaError_t launch_attn_tc_cached(const Ctx &c, const AttnArgs &a, int n_split_grid, int q_rows, cudaStream_t s)
+{
+    const int g = a.n_q / a.n_kv;
+    if (a.hd != 128 || g < 1 || kAtRows % g || a.kv.page_size % 64) return cudaErrorNotSupported;
+    AttnMapKey key{a.q, a.kv.k_pages, a.kv.v_pages, a.k_blk, a.kv.num_pages, a.kv.page_size, a.K, a.mode, q_rows};
+    auto it = c.amaps.find(key);
+    if (it == c.amaps.end()) {
+        AtMaps m;
+        if (!attn_tc_maps(a, c.cfg.n_layers, q_rows, &m)) return cudaErrorNotSupported;
+        it = c.amaps.emplace(key, std::vector<unsigned char>((unsigned char *)&m, (unsigned char *)&m + sizeof(m))).first;
+    }
+    c.launches += 1;
+    return launch_attn_tc(a, *(const AtMaps *)it->second.data(), n_split_grid, s);
+}
+
+cudaError_t launch_attn_tc(const AttnArgs &a, const AtMaps &maps, int n_split_grid, cudaStream_t s)
+{
+    const int g = a.n_q / a.n_kv;
+    const int ksub = kAtRows / g;
+    const int rgroups = (a.K + ksub - 1) / ksub;
+    const int C = attn_cluster_size(a.n_kv, a.B);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.n_kv, a.B * rgroups, C);
+    cfg.blockDim = dim3(kAtThreads);
+    cfg.dynamicSmemBytes = attn_tc_smem_bytes();
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = C;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    switch (C) {
+    case 1: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<1>, maps, a, n_split_grid);
+    case 2: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<2>, maps, a, n_split_grid);
+    case 4: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<4>, maps, a, n_split_grid);
+    default: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<8>, maps, a, n_split_grid);
+    }
+}
+
+}  // namespace orthrus

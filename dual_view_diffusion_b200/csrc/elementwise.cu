@@ -305,6 +305,25 @@ __global__ void set_lens_kernel(int32_t *seq_lens, int b, int value, int32_t *an
     if (anchor_out) anchor_out[b] = *last_tok;
 }
 
+// Block K/V given as [B][K][n_kv][hd] -> K [B][n_kv][kp][hd] and V transposed
+// [B][n_kv][hd][kp] (rows K .. kp-1 zero).
+template <class T>
+__global__ void pack_block_kernel(const T *ks, const T *vs, T *kd, T *vd, int K, int kp, int n_kv, int hd)
+{
+    pdl_trigger();
+    pdl_wait();
+    const int b = blockIdx.y, kvh = blockIdx.x;
+    for (int idx = threadIdx.x; idx < kp * hd; idx += blockDim.x) {
+        const int k = idx / hd, d = idx % hd;
+        const T z = from_f<T>(0.f);
+        const T kv = k < K ? ks[(((size_t)b * K + k) * n_kv + kvh) * hd + d] : z;
+        const T vv = k < K ? vs[(((size_t)b * K + k) * n_kv + kvh) * hd + d] : z;
+        const size_t head = (size_t)b * n_kv + kvh;
+        kd[(head * kp + k) * hd + d] = kv;
+        vd[(head * hd + d) * kp + k] = vv;
+    }
+}
+
 __global__ void set_int_kernel(int32_t *p, int v)
 {
     pdl_trigger();
@@ -416,6 +435,18 @@ cudaError_t launch_set_lens(const Ctx &, int32_t *seq_lens, int b, int value, in
 cudaError_t launch_set_int(int32_t *p, int v, cudaStream_t s)
 {
     return launch_k(set_int_kernel, 1, 1, 0, s, p, v);
+}
+
+cudaError_t launch_pack_block(const Ctx &c, const void *k_src, const void *v_src, void *k_dst, void *v_dst, int B,
+                              int K, int kp, cudaStream_t s)
+{
+    c.launches += 1;
+    const dim3 grid(c.cfg.n_kv_heads, B);
+    if (c.cfg.dtype == ORTHRUS_BF16)
+        return launch_k(pack_block_kernel<bf16>, grid, 256, 0, s, (const bf16 *)k_src, (const bf16 *)v_src,
+                        (bf16 *)k_dst, (bf16 *)v_dst, K, kp, c.cfg.n_kv_heads, c.cfg.head_dim);
+    return launch_k(pack_block_kernel<float>, grid, 256, 0, s, (const float *)k_src, (const float *)v_src,
+                    (float *)k_dst, (float *)v_dst, K, kp, c.cfg.n_kv_heads, c.cfg.head_dim);
 }
 
 cudaError_t launch_logits_dump(const Ctx &c, const void *fin, int M, float *logits, cudaStream_t s)

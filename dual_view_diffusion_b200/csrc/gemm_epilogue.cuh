@@ -149,19 +149,24 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
             }
             const bool is_k = n < Nq + Nk;
             const int nn = n - Nq - (is_k ? 0 : Nk), kvh = nn / a.hd, d = nn % a.hd;
-            T *dst;
+            // K rows are [slot][dim]; V is stored transposed, [dim][slot]
+            size_t base, step;
             if (a.kv_to_cache) {
                 const int page = s_page[m];
                 if (page < 0) continue;
-                T *base = (T *)(is_k ? a.kv.k_pages : a.kv.v_pages);
-                dst = base + (((size_t)a.layer * a.kv.num_pages + page) * a.n_kv + kvh) * (size_t)a.kv.page_size * a.hd +
-                      (size_t)(pos % a.kv.page_size) * a.hd;
+                const size_t head = ((size_t)a.layer * a.kv.num_pages + page) * a.n_kv + kvh;
+                const int slot = pos % a.kv.page_size;
+                if (is_k) { base = (head * a.kv.page_size + slot) * a.hd + d; step = 1; }
+                else { base = (head * a.hd + d) * a.kv.page_size + slot; step = a.kv.page_size; }
             } else {
-                T *base = (T *)(is_k ? a.k_blk : a.v_blk);
-                dst = base + (((size_t)a.layer * a.rows_max + row) * a.n_kv + kvh) * a.hd;
+                const int b = row / a.K, k = row % a.K;
+                const size_t head = ((size_t)a.layer * a.bmax + b) * a.n_kv + kvh;
+                if (is_k) { base = (head * a.kp + k) * a.hd + d; step = 1; }
+                else { base = (head * a.hd + d) * a.kp + k; step = a.kp; }
             }
-            dst[d] = from_f<T>(x0);
-            dst[d + half] = from_f<T>(x1);
+            T *dst = (T *)(is_k ? (a.kv_to_cache ? a.kv.k_pages : a.k_blk) : (a.kv_to_cache ? a.kv.v_pages : a.v_blk));
+            dst[base] = from_f<T>(x0);
+            dst[base + (size_t)half * step] = from_f<T>(x1);
         }
     } else if (a.epi == EPI_LMHEAD) {
         __shared__ int s_given[kTileM];

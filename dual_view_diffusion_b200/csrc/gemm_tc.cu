@@ -34,7 +34,7 @@ constexpr int kTcThreads = 192;
 constexpr int kTcAccCols = 32;                          // TMEM columns per accumulator (N = 32)
 constexpr uint32_t kStageWBytes = kTileN * kTileK * 2;  // 16 KiB
 constexpr uint32_t kStageXBytes = kTileM * kTileK * 2;  // 4 KiB
-constexpr long kSpinLimit = 1L << 26;                  // ~seconds of polling
+constexpr long long kSpinCycles = 4000000000LL;        // ~2 s at the B200 SM clock
 
 struct TcSmem {
     alignas(1024) unsigned char w[kTcStages][kStageWBytes];
@@ -66,12 +66,17 @@ __device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity)
                  : "=r"(ok) : "r"(smem_u32(b)), "r"(parity) : "memory");
     return ok != 0;
 }
-// Bounded wait; false on timeout (or when another role already gave up).
+// Bounded wait (about two seconds of SM clock); false on timeout, or when
+// another role of the CTA already gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile int *abort)
 {
-    for (long i = 0; i < kSpinLimit; ++i) {
+    const long long t0 = clock64();
+    for (long i = 0;; ++i) {
         if (mbar_try(b, parity)) return true;
-        if ((i & 1023) == 1023 && *abort) return false;
+        if ((i & 255) == 255) {
+            if (*abort) return false;
+            if (clock64() - t0 > kSpinCycles) break;
+        }
     }
     *abort = 1;
     return false;
@@ -294,17 +299,39 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
     return fn;
 }
 
-// 2-D bf16 map over a row-major [rows][cols] matrix, box {64 cols, box_rows},
-// 128-byte swizzle, zero fill outside.
-bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows)
+// 2-D bf16 map over a row-major [rows][cols] matrix, box {box_cols, box_rows}
+// (box_cols * 2 bytes <= 128), 128-byte swizzle, zero fill outside.
+bool make_tmap_box(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows)
 {
     auto enc = get_encoder();
-    if (!enc || ((uintptr_t)ptr & 15) || (cols * 2) % 16) return false;
+    if (!enc || !ptr || ((uintptr_t)ptr & 15) || (cols * 2) % 16 || box_cols * 2 > 128) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t es[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    return make_tmap_box(m, ptr, rows, cols, 64, box_rows);
+}
+
+// 4-D view of q [rows][n_q][hd] as (dim, head in group, kv head, row), box
+// {64, g, 1, ksub}: one load brings the g heads of one KV head for ksub
+// consecutive block rows, ordered (row, head) = the attention CTA's rows.
+bool make_tmap_q4(CUtensorMap *m, const void *q, int rows_total, int n_q, int n_kv, int hd, int ksub)
+{
+    auto enc = get_encoder();
+    const int g = n_q / n_kv;
+    if (!enc || !q || ((uintptr_t)q & 15) || (hd * 2) % 16 || g > 256 || ksub > 256) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)hd, (cuuint64_t)g, (cuuint64_t)n_kv, (cuuint64_t)rows_total};
+    cuuint64_t strides[3] = {(cuuint64_t)hd * 2, (cuuint64_t)g * hd * 2, (cuuint64_t)n_q * hd * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)g, 1, (cuuint32_t)ksub};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -63,8 +63,8 @@ struct GemmArgs {
     void *q_out;             // [M][n_q*hd]
     int n_q, n_kv, hd, layer;
     int kv_to_cache;         // 1: K/V into pages at (b, pos); 0: into k_blk/v_blk
-    void *k_blk, *v_blk;     // [n_layers][rows_max][n_kv][hd] when kv_to_cache == 0
-    int rows_max;
+    void *k_blk, *v_blk;     // transient layouts of AttnArgs (kv_to_cache == 0)
+    int kp, bmax;
     KvView kv;
     const int32_t *pos0;     // [batch] position of block row 0
     const int32_t *bt_rows;  // [batch] row of block_table for each batch entry
@@ -86,13 +86,20 @@ struct GemmArgs {
 struct AttnArgs {
     const void *q;           // [B*K][n_q][hd]
     void *out;               // [B*K][n_q][hd]
-    const void *k_blk, *v_blk;  // mode 1: [B*K][n_kv][hd]
+    // mode 1: the block's transient K/V (all layers), K as
+    // [n_layers][bmax][n_kv][kp][hd] and V transposed as
+    // [n_layers][bmax][n_kv][hd][kp]; rows >= K of a slice are ignored
+    const void *k_blk, *v_blk;
+    int kp, bmax;
+    int blk_layer, blk_layers;   // layer index into, and layer count of, k_blk / v_blk
     KvView kv;
     int layer;
     const int32_t *seq_lens;  // [batch] t per sequence (positions of block row 0)
     const int32_t *bt_rows;   // [batch] block-table row
     int B, K, n_q, n_kv, hd, mode;
-    int split_tokens, n_splits;   // n_splits = buffer stride (max splits)
+    // n_splits = partial-buffer stride: cache splits of the longest sequence
+    // plus one slot (the last) for the diffusion block's own keys
+    int split_tokens, n_splits;
     float *part;             // [B*K][n_q][n_splits][hd]
     float2 *ml;              // [B*K][n_q][n_splits]
     unsigned *err;
@@ -108,8 +115,28 @@ struct TmapKeyHash {
     size_t operator()(const TmapKey &k) const { return std::hash<const void *>()(k.ptr) ^ (size_t)k.box_rows * 0x9E3779B97F4A7C15ull; }
 };
 
+// Attention tensor maps are cached per (buffers, shape).
+struct AttnMapKey {
+    const void *q, *kc, *vc, *kb;
+    int num_pages, page_size, K, mode, q_rows;
+    bool operator==(const AttnMapKey &o) const
+    {
+        return q == o.q && kc == o.kc && vc == o.vc && kb == o.kb && num_pages == o.num_pages &&
+               page_size == o.page_size && K == o.K && mode == o.mode && q_rows == o.q_rows;
+    }
+};
+struct AttnMapKeyHash {
+    size_t operator()(const AttnMapKey &k) const
+    {
+        size_t h = std::hash<const void *>()(k.q) ^ (std::hash<const void *>()(k.kc) << 1) ^
+                   (std::hash<const void *>()(k.kb) << 2);
+        return h ^ ((size_t)k.K * 131 + (size_t)k.mode * 7 + (size_t)k.num_pages * 1000003 + (size_t)k.q_rows);
+    }
+};
+
 struct Ctx {
     orthrus_config_t cfg;
+    mutable std::unordered_map<AttnMapKey, std::vector<unsigned char>, AttnMapKeyHash> amaps;
     std::unordered_map<TmapKey, CUtensorMap, TmapKeyHash> tmaps;   // bf16 TMA maps of weights and activations
     std::vector<orthrus_layer_weights_t> layers;
     const void *embed, *final_norm, *lm_head;
@@ -125,7 +152,8 @@ struct Ctx {
     void *q;                 // [Rw][n_q*hd]
     void *attn_o;            // [Rw][n_q*hd]
     void *act;               // [Rw][F]
-    void *k_diff, *v_diff;   // [n_layers][R][n_kv][hd]
+    void *k_diff, *v_diff;   // [n_layers][max_batch][n_kv][kp][hd] and [..][hd][kp] (V transposed)
+    int kp;                  // max_block rounded up to a multiple of 64
     void *fin_draft, *fin_verify;  // [R][d]
     void *res_x;             // [2*max_batch][d]
     float *attn_part;        // [Rw][n_q][n_splits][hd]
@@ -133,6 +161,7 @@ struct Ctx {
     float *gemm_part;
     size_t gemm_part_floats;
     int *gemm_ticket;
+    void *blk_pack;          // [2][max_batch][n_kv][kp][hd]: user block K/V repacked (standalone attention)
     int gemm_tickets;
     LmPart *lm_part;         // [max(R, 2*max_batch)][n_vtiles]
     int32_t *tok;            // [Rw] block tokens
@@ -175,9 +204,15 @@ cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s);
 cudaError_t gemm_init_attributes();
 cudaError_t gemm_tc_init_attributes();
 bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+bool make_tmap_box(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows);
+bool make_tmap_q4(CUtensorMap *m, const void *q, int rows_total, int n_q, int n_kv, int hd, int ksub);
+struct AtMaps;
+cudaError_t attn_tc_init_attributes();
 cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, int grid, cudaStream_t s);
 cudaError_t attention_init_attributes();
-cudaError_t launch_attention(const Ctx &c, const AttnArgs &a, cudaStream_t s);
+cudaError_t launch_attention(const Ctx &c, const AttnArgs &a, cudaStream_t s, int q_rows);
+cudaError_t launch_attn_tc_cached(const Ctx &c, const AttnArgs &a, int n_split_grid, int q_rows, cudaStream_t s);
+bool attn_tc_maps(const AttnArgs &a, int n_layers, int rows_total, AtMaps *m);
 cudaError_t launch_embed(const Ctx &c, int mode, const int32_t *tokens, const int32_t *anchor,
                          const int32_t *draft, int B, int K, cudaStream_t s);
 cudaError_t launch_rmsnorm(const Ctx &c, const float *h, const void *gain, void *out, int M, cudaStream_t s);
@@ -192,6 +227,8 @@ cudaError_t launch_ar_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int64_
                              int append_max, cudaStream_t s);
 cudaError_t launch_set_lens(const Ctx &c, int32_t *seq_lens, int b, int value, int32_t *anchor_out,
                             const int32_t *tokens, cudaStream_t s);
+cudaError_t launch_pack_block(const Ctx &c, const void *k_src, const void *v_src, void *k_dst, void *v_dst, int B,
+                              int K, int kp, cudaStream_t s);
 cudaError_t launch_logits_dump(const Ctx &c, const void *fin, int M, float *logits, cudaStream_t s);
 
 }  // namespace orthrus

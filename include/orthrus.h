@@ -106,11 +106,16 @@ typedef struct {
 /*
  * The one shared KV cache (paper notes §2.2-2.3): AR keys (after RoPE) and
  * values only, paged.
- *   k_pages, v_pages  [n_layers][num_pages][n_kv][page_size][head_dim], dtype
- *   block_table       [max_batch][max_pages_per_seq] int32 page ids
- *   seq_lens          [max_batch] int32 committed length t of each sequence
- *                     (the anchor's own K/V are not in the cache)
- * page_size must be a multiple of 16 (of 64 on the bf16 path).
+ *   k_pages      [n_layers][num_pages][n_kv][page_size][head_dim], dtype
+ *   v_pages      [n_layers][num_pages][n_kv][head_dim][page_size], dtype: V is
+ *                stored transposed inside a page, so both attention products
+ *                read their operand with the reduced dimension contiguous
+ *   block_table  [max_batch][max_pages_per_seq] int32 page ids
+ *   seq_lens     [max_batch] int32 committed length t of each sequence
+ *                (the anchor's own K/V are not in the cache)
+ * page_size must be a multiple of 16 (of 64 on the bf16 path).  Pages must
+ * hold finite values before first use (zero them once): slots beyond a
+ * sequence's length are read and then masked, and 0 * NaN would not vanish.
  */
 typedef struct {
     void *k_pages, *v_pages;

@@ -33,7 +33,7 @@ def write_cache(eng, layer, b, kc, vc, start=0):
     page = eng.block_table[b].long()[pos // ps]
     slot = pos % ps
     eng.k_pages[layer, page, :, slot, :] = kt
-    eng.v_pages[layer, page, :, slot, :] = vt
+    eng.v_pages[layer, page, :, :, slot] = vt          # V pages are [dim][slot]
 
 
 def read_cache(eng, layer, b, start, n):
@@ -42,7 +42,7 @@ def read_cache(eng, layer, b, start, n):
     page = eng.block_table[b].long()[pos // ps]
     slot = pos % ps
     return (eng.k_pages[layer, page, :, slot, :].float().cpu().numpy(),
-            eng.v_pages[layer, page, :, slot, :].float().cpu().numpy())
+            eng.v_pages[layer, page, :, :, slot].float().cpu().numpy())
 
 
 def bf16_normal(shape, seed, name):

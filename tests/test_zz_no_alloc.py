@@ -77,8 +77,10 @@ def test_noalloc_refuses_oversize_request():
     import dual_view_diffusion_b200 as pkg
     eng = attention_engine()
     cfg = pkg.Config.from_buffer_copy(eng.cfg)
-    cfg.max_seq = 1 << 20                       # far more splits than the fixed array can hold
-    q = torch.zeros((1, 32, 32, 128), dtype=torch.bfloat16, device="cuda")
+    K = 4096                                     # a block whose repacked K/V exceed the fixed array
+    cfg.max_seq = 1 << 20
+    q = torch.zeros((1, K, 32, 128), dtype=torch.bfloat16, device="cuda")
+    kb = torch.zeros((1, K, 8, 128), dtype=torch.bfloat16, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    st, _ = _noalloc(pkg, eng, cfg, 1, q, q[:, :, :8], q[:, :, :8].clone(), 1, 32, err)
+    st, _ = _noalloc(pkg, eng, cfg, 1, q, kb, kb.clone(), 1, K, err)
     assert st == 3        # ORTHRUS_ERR_CAPACITY, nothing launched
