@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <new>
 #include <type_traits>
+#include <cmath>
 #include <vector>
 
 #include "common.cuh"
@@ -59,9 +60,9 @@ static void gemm_scratch(const orthrus_config_t &c, int rows_body, int rows_lm, 
     *tickets = 1;
     for (const Shape &s : shapes) {
         const int n_mt = (s.rows + kTileM - 1) / kTileM;
-        const int S = (use_tensor_cores(c) && s.Kd % kTileK == 0) ? choose_splits(s.n_tiles * kTileN, s.Kd) : 1;
+        const int S = (use_tensor_cores(c) && s.Kd % kTileK == 0) ? sk_max_segments(s.n_tiles, s.Kd / kTileK) : 1;
         if (S > 1) *floats = std::max(*floats, (size_t)n_mt * s.n_tiles * S * kTileM * kTileN);
-        *tickets = std::max(*tickets, n_mt * s.n_tiles);
+        *tickets = std::max(*tickets, n_mt * s.n_tiles * S);
     }
 }
 
@@ -95,6 +96,9 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
     const size_t o_part = take(simt_attn ? Rw * c.n_q_heads * n_splits * c.head_dim * 4 : 0);
     const size_t o_ml = take(simt_attn ? Rw * c.n_q_heads * n_splits * 8 : 0);
     const size_t o_gp = take(std::max(gfloats, (size_t)1) * 4), o_gt = take((size_t)gtickets * 4);
+    const int rslots = std::max(resid_defer_slots(c, c.hidden, c.n_q_heads * c.head_dim), resid_defer_slots(c, c.hidden, c.ffn));
+    const size_t o_rp = take((size_t)rslots * Rw * d * 4);
+    const size_t o_invf = take((size_t)c.head_dim / 2 * 8);
     const size_t o_lm = take(Rlm * n_vtiles * sizeof(LmPart));
     const size_t o_tok = take(Rw * 4), o_pos = take(mb * 4), o_bt = take(mb * 4), o_pr = take(4);
     const size_t o_dr = take(R * 4), o_lq = take(R * 4), o_lsq = take(R * 4), o_g = take(R * 4), o_lp = take(R * 4),
@@ -110,6 +114,8 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
         x->attn_part = (float *)P(o_part); x->attn_ml = (float2 *)P(o_ml);
         x->gemm_part = (float *)P(o_gp); x->gemm_part_floats = gfloats; x->gemm_ticket = (int *)P(o_gt);
         x->gemm_tickets = gtickets; x->lm_part = (LmPart *)P(o_lm);
+        x->resid_part = (float *)P(o_rp);
+        x->rope_invf = (double *)P(o_invf);
         x->tok = (int32_t *)P(o_tok); x->pos0 = (int32_t *)P(o_pos); x->bt_rows = (int32_t *)P(o_bt);
         x->prefill_row = (int32_t *)P(o_pr);
         x->draft = (int32_t *)P(o_dr); x->logq = (float *)P(o_lq); x->lse_q = (float *)P(o_lsq);
@@ -129,7 +135,7 @@ static void rebase(Ctx *x, char *ws)
     auto fix = [&](auto *&p) { p = (std::remove_reference_t<decltype(p)>)(ws + (size_t)(const char *)p); };
     fix(x->h); fix(x->a); fix(x->q); fix(x->attn_o); fix(x->act); fix(x->k_diff); fix(x->v_diff); fix(x->blk_pack);
     fix(x->fin_draft); fix(x->fin_verify); fix(x->res_x); fix(x->attn_part); fix(x->attn_ml); fix(x->gemm_part);
-    fix(x->gemm_ticket); fix(x->lm_part); fix(x->tok); fix(x->pos0); fix(x->bt_rows); fix(x->prefill_row);
+    fix(x->gemm_ticket); fix(x->lm_part); fix(x->resid_part); fix(x->rope_invf); fix(x->tok); fix(x->pos0); fix(x->bt_rows); fix(x->prefill_row);
     fix(x->draft); fix(x->logq); fix(x->lse_q); fix(x->g); fix(x->logp); fix(x->lse_p); fix(x->rej_row);
     fix(x->res_tok); fix(x->any_reject); fix(x->err); fix(x->produced); fix(x->step); fix(x->n_buf);
     fix(x->tok_buf); fix(x->anchor_buf);
@@ -197,9 +203,12 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
     const orthrus_config_t &f = c.cfg;
     const int M = B * K, hd = f.head_dim;
     cudaError_t e;
+    // residual segments the O and down projections leave for the next RMSNorm
+    int pending = 0;
+    const int defer_o = resid_defer_slots(f, f.hidden, f.n_q_heads * hd), defer_dn = resid_defer_slots(f, f.hidden, f.ffn);
     for (int l = 0; l < f.n_layers; ++l) {
         const orthrus_layer_weights_t &W = c.layers[l];
-        if ((e = launch_rmsnorm(c, c.h, W.attn_norm, c.a, M, s)) != cudaSuccess) return e;
+        if ((e = launch_rmsnorm(c, c.h, W.attn_norm, c.a, M, pending, s)) != cudaSuccess) return e;
         GemmArgs q{};
         q.x = c.a; q.M = M; q.Kd = f.hidden;
         q.w[0] = view ? W.wq_diff : W.wq; q.w[1] = view ? W.wk_diff : W.wk; q.w[2] = view ? W.wv_diff : W.wv;
@@ -208,6 +217,7 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
         q.epi = EPI_QKV; q.q_out = c.q; q.n_q = f.n_q_heads; q.n_kv = f.n_kv_heads; q.hd = hd; q.layer = l;
         q.kv_to_cache = view == 0; q.k_blk = c.k_diff; q.v_blk = c.v_diff; q.kp = c.kp; q.bmax = f.max_batch;
         q.kv = kv_view(kv); q.pos0 = pos0; q.bt_rows = bt_rows; q.K = K; q.rope_theta = (double)f.rope_theta;
+        q.rope_invf = c.rope_invf;
         {
             ProbeScope ps(c, 0, l, view, s);
             if ((e = launch_gemm(c, q, s)) != cudaSuccess) return e;
@@ -228,13 +238,13 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
 
         GemmArgs o{};
         o.x = c.attn_o; o.M = M; o.N = f.hidden; o.Kd = f.n_q_heads * hd; o.w[0] = W.wo; o.wrows[0] = f.hidden;
-        o.epi = EPI_RESID; o.resid = c.h;
+        o.epi = EPI_RESID; o.resid = c.h; o.defer = defer_o; o.rpart = c.resid_part; o.rpart_rows = c.Rw;
         {
             ProbeScope ps(c, 0, l, view, s);
             if ((e = launch_gemm(c, o, s)) != cudaSuccess) return e;
         }
 
-        if ((e = launch_rmsnorm(c, c.h, W.ffn_norm, c.a, M, s)) != cudaSuccess) return e;
+        if ((e = launch_rmsnorm(c, c.h, W.ffn_norm, c.a, M, defer_o, s)) != cudaSuccess) return e;
         GemmArgs gu{};
         gu.x = c.a; gu.M = M; gu.N = f.ffn; gu.Kd = f.hidden; gu.w[0] = W.w_gate; gu.w[1] = W.w_up;
         gu.wrows[0] = gu.wrows[1] = f.ffn; gu.epi = EPI_SWIGLU; gu.act = c.act;
@@ -245,13 +255,14 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
 
         GemmArgs dn{};
         dn.x = c.act; dn.M = M; dn.N = f.hidden; dn.Kd = f.ffn; dn.w[0] = W.w_down; dn.wrows[0] = f.hidden;
-        dn.epi = EPI_RESID; dn.resid = c.h;
+        dn.epi = EPI_RESID; dn.resid = c.h; dn.defer = defer_dn; dn.rpart = c.resid_part; dn.rpart_rows = c.Rw;
         {
             ProbeScope ps(c, 0, l, view, s);
             if ((e = launch_gemm(c, dn, s)) != cudaSuccess) return e;
         }
+        pending = defer_dn;
     }
-    if (fin) return launch_rmsnorm(c, c.h, c.final_norm, fin, M, s);
+    if (fin) return launch_rmsnorm(c, c.h, c.final_norm, fin, M, pending, s);
     return cudaSuccess;
 }
 
@@ -346,8 +357,12 @@ orthrus_status_t orthrus_create(const orthrus_config_t *cfg, const orthrus_weigh
     if (cfg->dtype == ORTHRUS_BF16) build_tmaps(c);
     std::vector<int32_t> ident(cfg->max_batch);
     for (int b = 0; b < cfg->max_batch; ++b) ident[b] = b;
+    // rotary inverse frequencies theta^(-2i / head_dim), in double on the host
+    std::vector<double> invf(cfg->head_dim / 2);
+    for (int i = 0; i < cfg->head_dim / 2; ++i) invf[i] = std::pow((double)cfg->rope_theta, -2.0 * i / cfg->head_dim);
     if (cudaMemset(workspace, 0, need) != cudaSuccess ||
         cudaMemcpy(c->bt_rows, ident.data(), ident.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->rope_invf, invf.data(), invf.size() * 8, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess) {
         delete c;
         return ORTHRUS_ERR_CUDA;

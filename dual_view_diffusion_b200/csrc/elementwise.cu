@@ -62,13 +62,16 @@ __device__ __forceinline__ float4 load_gain4(const T *g, int i)
 }
 
 template <class T>
-__global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float *h, const T *gain, T *out, int d, float eps)
+// pending > 0: first fold the residual segments part[s][row] (s < pending,
+// in order) into h, which is written back.
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(float *h, const T *gain, T *out, int d, float eps,
+                                                               const float *part, int pending, size_t slot_stride)
 {
     __shared__ float red[kNormThreads / 32];
     pdl_trigger();
     pdl_wait();
     const int row = blockIdx.x, tid = threadIdx.x;
-    const float *x = h + (size_t)row * d;
+    float *x = h + (size_t)row * d;
     float ss = 0.f;
     const bool vec = (d & 3) == 0 && d <= kNormThreads * 4 * kNormVec;
     float4 v[kNormVec];
@@ -78,13 +81,38 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float *h, c
             const int i = (tid + j * kNormThreads) * 4;
             v[j] = i < d ? *(const float4 *)(x + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        if (pending > 0) {
+            for (int sl = 0; sl < pending; ++sl) {
+                const float *p = part + sl * slot_stride + (size_t)row * d;
+                float4 u[kNormVec];
+#pragma unroll
+                for (int j = 0; j < kNormVec; ++j) {
+                    const int i = (tid + j * kNormThreads) * 4;
+                    u[j] = i < d ? __ldcg((const float4 *)(p + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int j = 0; j < kNormVec; ++j) {
+                    v[j].x += u[j].x; v[j].y += u[j].y; v[j].z += u[j].z; v[j].w += u[j].w;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kNormVec; ++j) {
+                const int i = (tid + j * kNormThreads) * 4;
+                if (i < d) *(float4 *)(x + i) = v[j];
+            }
+        }
 #pragma unroll
         for (int j = 0; j < kNormVec; ++j) {
             ss = fmaf(v[j].x, v[j].x, ss); ss = fmaf(v[j].y, v[j].y, ss);
             ss = fmaf(v[j].z, v[j].z, ss); ss = fmaf(v[j].w, v[j].w, ss);
         }
     } else {
-        for (int i = tid; i < d; i += kNormThreads) ss = fmaf(x[i], x[i], ss);
+        for (int i = tid; i < d; i += kNormThreads) {
+            float xi = x[i];
+            for (int sl = 0; sl < pending; ++sl) xi += part[sl * slot_stride + (size_t)row * d + i];
+            if (pending > 0) x[i] = xi;
+            ss = fmaf(xi, xi, ss);
+        }
     }
     ss = warp_sum(ss);
     if ((tid & 31) == 0) red[tid >> 5] = ss;
@@ -344,14 +372,15 @@ cudaError_t launch_embed(const Ctx &c, int mode, const int32_t *tokens, const in
                     c.cfg.mask_token_id, mode, tokens, anchor, draft, K, c.tok, c.h, c.err);
 }
 
-cudaError_t launch_rmsnorm(const Ctx &c, const float *h, const void *gain, void *out, int M, cudaStream_t s)
+cudaError_t launch_rmsnorm(const Ctx &c, float *h, const void *gain, void *out, int M, int pending, cudaStream_t s)
 {
     c.launches += 1;
+    const size_t stride = (size_t)c.Rw * c.cfg.hidden;
     if (c.cfg.dtype == ORTHRUS_BF16)
         return launch_k(rmsnorm_kernel<bf16>, M, kNormThreads, 0, s, h, (const bf16 *)gain, (bf16 *)out, c.cfg.hidden,
-                        c.cfg.rms_eps);
+                        c.cfg.rms_eps, (const float *)c.resid_part, pending, stride);
     return launch_k(rmsnorm_kernel<float>, M, kNormThreads, 0, s, h, (const float *)gain, (float *)out, c.cfg.hidden,
-                    c.cfg.rms_eps);
+                    c.cfg.rms_eps, (const float *)c.resid_part, pending, stride);
 }
 
 cudaError_t launch_lm_finalize_impl(const Ctx &c, int mode, int B, int K, float temperature, int32_t *tok_out,

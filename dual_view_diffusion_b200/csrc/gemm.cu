@@ -26,6 +26,8 @@
 #include <math.h>
 
 #include "common.cuh"
+#include <algorithm>
+
 #include "gemm_epilogue.cuh"
 #include "internal.h"
 
@@ -86,58 +88,43 @@ __device__ void mainloop_simt(const GemmArgs &a, int mt, int nt, int k0, int k1,
 }
 
 // ---------------------------------------------------------------- kernel
-// One-dimensional grid of persistent CTAs walking (m tile, n tile, segment)
-// units in order.
+// One-dimensional grid of persistent CTAs walking (m tile, n tile) units in
+// order, each over the whole k range.
 template <class T>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(GemmArgs a, int n_mt, int n_nt)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     float(*tile)[kTilePad] = (float(*)[kTilePad])smem_raw;
     unsigned char *pipe = smem_raw + sizeof(float) * kTileM * kTilePad;
-    __shared__ int s_last;
     pdl_trigger();
     pdl_wait();
     if (a.epi == EPI_RESAMPLE && *a.any_flag == 0) return;
 
-    const int S = a.splits;
-    const int units = n_mt * n_nt * S;
-    const int chunks = (a.Kd + kTileK - 1) / kTileK;
+    const int units = n_mt * n_nt;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
-        const int seg = u % S, t = u / S, mt = t % n_mt, nt = t / n_mt;
-        const int c0 = (int)((long)seg * chunks / S), c1 = (int)((long)(seg + 1) * chunks / S);
-        mainloop_simt<T>(a, mt, nt, c0 * kTileK, min(c1 * kTileK, a.Kd), (float *)pipe, tile);
+        const int mt = u % n_mt, nt = u / n_mt;
+        mainloop_simt<T>(a, mt, nt, 0, a.Kd, (float *)pipe, tile);
         __syncthreads();
-        if (!split_k_gather(a, tile, t, seg, threadIdx.x, &s_last, SyncBlock{}))
-            continue;
         epilogue<T>(a, tile, mt, nt, n_nt, threadIdx.x, SyncBlock{});
         __syncthreads();
     }
 }
 
 // ---------------------------------------------------------------- host
-// k segments per n tile.  A persistent CTA streams its units back to back,
-// so the time is set by the busiest CTA's chunk count; each extra segment
-// adds a partial tile to publish and reduce.  Cost = max chunks per CTA +
-// 8 chunk-equivalents per segment (fitted to the Qwen3-8B projections on a
-// B200: QKV -> 3, O -> 3, gate/up -> 2, down -> 4, LM head -> 1).  Depends on
-// the matrix shape only, never on the number of token rows.
-int choose_splits(int N, int Kd)
-{
-    const int n_nt = (N + kTileN - 1) / kTileN;
-    const int chunks = (Kd + kTileK - 1) / kTileK;
-    int best = 1;
-    long best_cost = -1;
-    for (int S = 1; S <= 16; ++S) {
-        if (S > 1 && chunks / S < 4) break;
-        const long units = (long)n_nt * S;
-        const long per_cta = (units + kNumSMs - 1) / kNumSMs;
-        const long cost = per_cta * ((chunks + S - 1) / S) + 8L * S;
-        if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = S; }
-    }
-    return best;
-}
-
 bool use_tensor_cores(const orthrus_config_t &c) { return c.dtype == ORTHRUS_BF16; }
+
+// k segments per n tile of a residual GEMM whose sum is left to the next
+// RMSNorm: the most that keeps n_tiles x segments within one wave of SMs
+// with whole chunks per segment (0: the epilogue adds to the residual).
+// A function of the matrix shape only.
+int resid_defer_slots(const orthrus_config_t &cfg, int N, int Kd)
+{
+    if (!use_tensor_cores(cfg) || Kd % kTileK) return 0;
+    const int n_nt = (N + kTileN - 1) / kTileN, chunks = Kd / kTileK;
+    for (int S = std::min(kResidSlots, kNumSMs / std::max(n_nt, 1)); S >= 1; --S)
+        if (chunks % S == 0) return S;
+    return 0;
+}
 
 size_t gemm_smem_bytes() { return sizeof(float) * kTileM * kTilePad + sizeof(float) * kTileM * kTileK; }
 
@@ -146,22 +133,23 @@ cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s)
     const bool tc = use_tensor_cores(c.cfg) && a.Kd % kTileK == 0;
     const int n_nt = a.epi == EPI_SWIGLU ? (a.N + 63) / 64 : (a.N + kTileN - 1) / kTileN;
     const int n_mt = (a.M + kTileM - 1) / kTileM;
-    a.splits = tc ? choose_splits(n_nt * kTileN, a.Kd) : 1;
-    if (a.splits > 1) {
-        if ((size_t)n_mt * n_nt * a.splits * kTileM * kTileN > c.gemm_part_floats ||
-            n_mt * n_nt > c.gemm_tickets)
-            return cudaErrorInvalidValue;
-    }
     a.part = c.gemm_part;
     a.ticket = c.gemm_ticket;
     a.err = c.err;
-    const long units = (long)n_mt * n_nt * a.splits;
-    const int grid = (int)(units < kNumSMs ? units : kNumSMs);
-    const size_t smem = gemm_smem_bytes();
-    if (tc) {
-        const cudaError_t e = launch_gemm_tc(c, a, n_mt, n_nt, grid, s);
+    if (tc) {   // stream-K split: partial and flag slots per (token tile, n tile, segment)
+        GemmArgs t = a;
+        t.splits = t.defer > 0 ? t.defer : sk_max_segments(n_nt, a.Kd / kTileK);
+        const size_t slots = (size_t)n_mt * n_nt * t.splits;
+        if (t.splits > 1 && (slots * kTileM * kTileN > c.gemm_part_floats || slots > (size_t)c.gemm_tickets))
+            return cudaErrorInvalidValue;
+        const cudaError_t e = launch_gemm_tc(c, t, n_mt, n_nt, s);
         if (e != cudaErrorNotSupported) return e;
     }
+    if (a.defer > 0) return cudaErrorInvalidValue;   // only the tensor-core kernel defers
+    a.splits = 1;
+    const long units = (long)n_mt * n_nt;
+    const int grid = (int)(units < kNumSMs ? units : kNumSMs);
+    const size_t smem = gemm_smem_bytes();
     c.launches += 1;
     if (c.cfg.dtype == ORTHRUS_BF16) return launch_k(gemm_kernel<bf16>, grid, kGemmThreads, smem, s, a, n_mt, n_nt);
     return launch_k(gemm_kernel<float>, grid, kGemmThreads, smem, s, a, n_mt, n_nt);

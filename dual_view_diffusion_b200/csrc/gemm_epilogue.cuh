@@ -64,10 +64,116 @@ __device__ __forceinline__ void rope_sincos(int pos, double inv_freq, float &s, 
     sincosf((float)r, &s, &c);
 }
 
-template <class T, class Sync>
-__device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int nt, int n_nt, int tid, Sync sync)
+// What an epilogue can fetch before its accumulator is ready: the residual
+// rows (RESID) and the per-row destinations and rotary frequencies of a
+// head-sized QKV tile.  A warp-specialised kernel fills it while the tile's
+// last weight chunks stream in, so only arithmetic and stores remain after.
+struct QkvPre {
+    int pos[kTileM];
+    long long dst[kTileM];   // element offset of (row, dim 0); -1: skip the row
+    double invf[64];
+};
+struct EpiPre {
+    float resid[kTileM][kTilePad];
+    QkvPre qkv;
+};
+
+// E >= 0 fixes the epilogue at compile time (each tensor-core kernel carries
+// only its own epilogue's code); E < 0 dispatches on a.epi.
+template <int E> __device__ __forceinline__ int epi_kind(const GemmArgs &a) { return E >= 0 ? E : a.epi; }
+
+template <int E = -1>
+__device__ __forceinline__ bool qkv_fast(const GemmArgs &a, int es)
 {
-    if (a.epi == EPI_RESID) {
+    return epi_kind<E>(a) == EPI_QKV && es == 2 && a.hd == kTileN && (a.n_q * a.hd) % kTileN == 0;
+}
+
+// Q, K or V (0, 1, 2) and head of an n tile of a head-sized QKV projection
+__device__ __forceinline__ void qkv_kind(const GemmArgs &a, int nt, int &kind, int &head)
+{
+    const int Nq = a.n_q * kTileN, Nk = a.n_kv * kTileN, n0 = nt * kTileN;
+    kind = n0 < Nq ? 0 : (n0 < Nq + Nk ? 1 : 2);
+    head = (n0 - (kind == 0 ? 0 : (kind == 1 ? Nq : Nq + Nk))) / kTileN;
+}
+
+__device__ inline void qkv_prepare(const GemmArgs &a, QkvPre &pre, int mt, int nt, int tid)
+{
+    int kind, head;
+    qkv_kind(a, nt, kind, head);
+    if (tid < kTileM) {
+        const int row = mt * kTileM + tid;
+        int pos = -1;
+        long long dst = -1;
+        if (row < a.M) {
+            const int b = row / a.K, k = row % a.K;
+            pos = a.pos0[b] + k;
+            if (kind == 0) {
+                dst = (long long)row * a.n_q * kTileN + head * kTileN;
+            } else if (a.kv_to_cache) {
+                const int pidx = pos / a.kv.page_size;
+                int page = -1;
+                if (pos >= 0 && pidx < a.kv.max_pages) {
+                    page = a.kv.block_table[(size_t)a.bt_rows[b] * a.kv.max_pages + pidx];
+                    if (page >= a.kv.num_pages) page = -1;
+                }
+                if (page < 0) {
+                    raise_err(a.err, ORTHRUS_DEVERR_CAPACITY);
+                } else {
+                    const long long hh = ((long long)a.layer * a.kv.num_pages + page) * a.n_kv + head;
+                    const int slot = pos % a.kv.page_size;
+                    dst = kind == 1 ? (hh * a.kv.page_size + slot) * kTileN : hh * kTileN * a.kv.page_size + slot;
+                }
+            } else {
+                const long long hh = ((long long)a.layer * a.bmax + b) * a.n_kv + head;
+                dst = kind == 1 ? (hh * a.kp + k) * kTileN : hh * kTileN * a.kp + k;
+            }
+        }
+        pre.pos[tid] = pos;
+        pre.dst[tid] = dst;
+    } else if (tid >= 64) {
+        pre.invf[tid - 64] = a.rope_invf[tid - 64];
+    }
+}
+
+template <class T, int E = -1>
+__device__ void epilogue_prepare(const GemmArgs &a, EpiPre &pre, int mt, int nt, int tid)
+{
+    if (epi_kind<E>(a) == EPI_RESID && (a.N & 3) == 0) {
+        float4 v[kEpiVec];
+#pragma unroll
+        for (int j = 0; j < kEpiVec; ++j) {
+            const int c = tid + j * kEpiThreads, m = c >> 5, n = nt * kTileN + (c & 31) * 4, row = mt * kTileM + m;
+            if (row < a.M && n < a.N) v[j] = __ldcg((const float4 *)&a.resid[(size_t)row * a.N + n]);
+        }
+#pragma unroll
+        for (int j = 0; j < kEpiVec; ++j) {
+            const int c = tid + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
+            *(float4 *)&pre.resid[m][c4] = v[j];
+        }
+    } else if (qkv_fast<E>(a, sizeof(T))) {
+        qkv_prepare(a, pre.qkv, mt, nt, tid);
+    }
+}
+
+// pre: filled by epilogue_prepare for this tile (and made visible with a
+// barrier), or null to fetch everything here.
+// bf16 outputs: the same reduction, then the MUFU sine / cosine (absolute
+// error ~4e-7 on [-pi, pi], far inside bf16 rounding) in a few instructions
+__device__ __forceinline__ void rope_sincos_fast(int pos, double inv_freq, float &s, float &c)
+{
+    const double ang = (double)pos * inv_freq;
+    const double k = rint(ang * 0.15915494309189535);
+    const float r = (float)fma(-k, 6.283185307179586, ang);
+    s = __sinf(r);
+    c = __cosf(r);
+}
+
+template <class T, class Sync, int E = -1>
+__device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int nt, int n_nt, int tid, Sync sync,
+                         EpiPre *pre = nullptr)
+{
+    const int epi = epi_kind<E>(a);
+    if (epi == EPI_RESID) {
         if ((a.N & 3) == 0) {
             float4 v[kEpiVec];
             bool ok[kEpiVec];
@@ -75,7 +181,8 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
             for (int j = 0; j < kEpiVec; ++j) {
                 const int c = tid + j * kEpiThreads, m = c >> 5, n = nt * kTileN + (c & 31) * 4, row = mt * kTileM + m;
                 ok[j] = row < a.M && n < a.N;
-                if (ok[j]) v[j] = *(const float4 *)&a.resid[(size_t)row * a.N + n];
+                if (ok[j]) v[j] = pre ? *(const float4 *)&pre->resid[m][(c & 31) * 4]
+                                      : *(const float4 *)&a.resid[(size_t)row * a.N + n];
             }
 #pragma unroll
             for (int j = 0; j < kEpiVec; ++j) {
@@ -92,7 +199,27 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
                 if (row < a.M && n < a.N) a.resid[(size_t)row * a.N + n] += tile[m][nl];
             }
         }
-    } else if (a.epi == EPI_SWIGLU) {
+    } else if (epi == EPI_SWIGLU && sizeof(T) == 2 && (a.N & 7) == 0) {
+        // 8 outputs per item: gate / up float4 pairs -> one 16-byte store
+#pragma unroll
+        for (int j = 0; j < kTileM * 8 / kEpiThreads; ++j) {
+            const int item = tid + j * kEpiThreads, m = item >> 3, i0 = (item & 7) * 8;
+            const int row = mt * kTileM + m, f = nt * 64 + i0;
+            if (row >= a.M || f >= a.N) continue;
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                const float g0 = tile[m][i0 + e], g1 = tile[m][i0 + e + 1];
+                const float u0 = tile[m][64 + i0 + e], u1 = tile[m][64 + i0 + e + 1];
+                // bf16 output: the MUFU exponential and an approximate divide
+                // are well inside its rounding, and keep this path short
+                const float s0 = __fdividef(g0, 1.0f + __expf(-g0)), s1 = __fdividef(g1, 1.0f + __expf(-g1));
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(s0 * u0, s1 * u1);
+                o[e / 2] = *(const uint32_t *)&h2;
+            }
+            __stcg((uint4 *)((bf16 *)a.act + (size_t)row * a.N + f), make_uint4(o[0], o[1], o[2], o[3]));
+        }
+    } else if (epi == EPI_SWIGLU) {
 #pragma unroll 4
         for (int idx = tid; idx < kTileM * 64; idx += kEpiThreads) {
             const int m = idx >> 6, i = idx & 63, row = mt * kTileM + m, f = nt * 64 + i;
@@ -102,7 +229,78 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
                 ((T *)a.act)[(size_t)row * a.N + f] = from_f<T>(s * u);
             }
         }
-    } else if (a.epi == EPI_QKV) {
+    } else if (qkv_fast<E>(a, sizeof(T))) {
+        // one tile = one head of Q, K or V (head_dim 128).  Per-row
+        // destinations are resolved once; Q/K rows are rotated 8 dimension
+        // pairs at a time and written with 16-byte stores; V goes to its
+        // transposed layout 8 tokens at a time where they are contiguous.
+        QkvPre *qp = pre ? &pre->qkv : nullptr;
+        if (!qp) {
+            __shared__ QkvPre s_qkv;
+            qkv_prepare(a, s_qkv, mt, nt, tid);
+            sync();
+            qp = &s_qkv;
+        }
+        int kind, head;
+        qkv_kind(a, nt, kind, head);
+        const int vstride = a.kv_to_cache ? a.kv.page_size : a.kp;
+        const int *s_pos = qp->pos;
+        const long long *s_dst = qp->dst;
+        const double *s_invf = qp->invf;
+        if (kind < 2) {
+            bf16 *base = (bf16 *)(kind == 0 ? a.q_out : (a.kv_to_cache ? a.kv.k_pages : a.k_blk));
+#pragma unroll
+            for (int j = 0; j < kTileM * 8 / kEpiThreads; ++j) {
+                const int item = tid + j * kEpiThreads, m = item >> 3, i0 = (item & 7) * 8;
+                const long long dst = s_dst[m];
+                if (dst < 0) continue;
+                const int pos = s_pos[m];
+                uint32_t lo[4], hi[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    float r[4];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        float sn, cs;
+                        rope_sincos_fast(pos, s_invf[i0 + e + u], sn, cs);
+                        const float x0 = tile[m][i0 + e + u], x1 = tile[m][64 + i0 + e + u];
+                        r[u] = x0 * cs - x1 * sn;
+                        r[2 + u] = x1 * cs + x0 * sn;
+                    }
+                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(r[0], r[1]), h2 = __floats2bfloat162_rn(r[2], r[3]);
+                    lo[e / 2] = *(const uint32_t *)&l2;
+                    hi[e / 2] = *(const uint32_t *)&h2;
+                }
+                __stcg((uint4 *)(base + dst + i0), make_uint4(lo[0], lo[1], lo[2], lo[3]));
+                __stcg((uint4 *)(base + dst + 64 + i0), make_uint4(hi[0], hi[1], hi[2], hi[3]));
+            }
+        } else {
+            bf16 *base = (bf16 *)(a.kv_to_cache ? a.kv.v_pages : a.v_blk);
+#pragma unroll
+            for (int j = 0; j < kTileM * kTileN / 8 / kEpiThreads; ++j) {
+                const int item = tid + j * kEpiThreads, tg = item & 3, d = item >> 2, m0 = tg * 8;
+                const long long d0 = s_dst[m0];
+                bool run = d0 >= 0 && ((d0 + (long long)d * vstride) & 7) == 0;
+#pragma unroll
+                for (int e = 1; e < 8; ++e) run = run && s_dst[m0 + e] == d0 + e;
+                if (run) {
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(tile[m0 + e][d], tile[m0 + e + 1][d]);
+                        o[e / 2] = *(const uint32_t *)&h2;
+                    }
+                    __stcg((uint4 *)(base + d0 + (long long)d * vstride), make_uint4(o[0], o[1], o[2], o[3]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const long long de = s_dst[m0 + e];
+                        if (de >= 0) base[de + (long long)d * vstride] = __float2bfloat16_rn(tile[m0 + e][d]);
+                    }
+                }
+            }
+        }
+    } else if (epi == EPI_QKV) {
         __shared__ int s_pos[kTileM], s_page[kTileM];
         __shared__ double s_invf[64];
         const int half = a.hd / 2, Nq = a.n_q * a.hd, Nk = a.n_kv * a.hd;
@@ -124,7 +322,7 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
             s_pos[tid] = pos;
             s_page[tid] = page;
         } else if (tid >= 64 && tid - 64 < half) {
-            s_invf[tid - 64] = pow(a.rope_theta, -2.0 * (tid - 64) / a.hd);
+            s_invf[tid - 64] = a.rope_invf[tid - 64];
         }
         sync();
 #pragma unroll 4
@@ -168,7 +366,7 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
             dst[base] = from_f<T>(x0);
             dst[base + (size_t)half * step] = from_f<T>(x1);
         }
-    } else if (a.epi == EPI_LMHEAD) {
+    } else if (epi == EPI_LMHEAD) {
         __shared__ int s_given[kTileM];
         __shared__ uint32_t s_step;
         if (tid < kTileM) {
@@ -220,13 +418,13 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
                 a.lm[(size_t)row * n_nt + nt] = pr;
             }
         }
-    } else if (a.epi == EPI_LOGITS) {
+    } else if (epi == EPI_LOGITS) {
 #pragma unroll 4
         for (int idx = tid; idx < kTileM * kTileN; idx += kEpiThreads) {
             const int m = idx >> 7, nl = idx & 127, row = mt * kTileM + m, n = nt * kTileN + nl;
             if (row < a.M && n < a.N) a.logits[(size_t)row * a.N + n] = tile[m][nl];
         }
-    } else if (a.epi == EPI_RESAMPLE) {
+    } else if (epi == EPI_RESAMPLE) {
         // rows come in pairs (2b: AR view at the rejected row, 2b+1: diffusion
         // view at the same row); score = log max(0, p - q) + Gumbel
         __shared__ int s_j[kTileM / 2];
@@ -270,55 +468,6 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
             }
         }
     }
-}
-
-// Split-K: publish this unit's partial tile; the CTA that completes the
-// tile's set of segments sums them in segment order (so the sum never
-// depends on arrival order) and runs the epilogue.  `sync` is a barrier over
-// the kEpiThreads epilogue threads.  Returns true when this CTA must run the
-// epilogue.
-template <class Sync>
-__device__ bool split_k_gather(const GemmArgs &a, float (*tile)[kTilePad], int t, int seg, int tid, int *s_last,
-                               Sync sync)
-{
-    const int S = a.splits;
-    if (S == 1) return true;
-    float *slot = a.part + ((size_t)t * S + seg) * (kTileM * kTileN);
-#pragma unroll
-    for (int j = 0; j < kEpiVec; ++j) {
-        const int c = tid + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
-        __stcg((float4 *)(slot + m * kTileN + c4), *(float4 *)&tile[m][c4]);
-    }
-    __threadfence();
-    sync();
-    if (tid == 0) *s_last = (atomicAdd(&a.ticket[t], 1) == S - 1);
-    sync();
-    if (!*s_last) return false;
-    __threadfence();
-    const float *base = a.part + (size_t)t * S * (kTileM * kTileN);
-    float4 acc[kEpiVec];
-#pragma unroll
-    for (int j = 0; j < kEpiVec; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < S; ++s) {
-        float4 v[kEpiVec];
-#pragma unroll
-        for (int j = 0; j < kEpiVec; ++j) {
-            const int c = tid + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
-            v[j] = __ldcg((const float4 *)(base + (size_t)s * kTileM * kTileN + m * kTileN + c4));
-        }
-#pragma unroll
-        for (int j = 0; j < kEpiVec; ++j) {
-            acc[j].x += v[j].x; acc[j].y += v[j].y; acc[j].z += v[j].z; acc[j].w += v[j].w;
-        }
-    }
-#pragma unroll
-    for (int j = 0; j < kEpiVec; ++j) {
-        const int c = tid + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
-        *(float4 *)&tile[m][c4] = acc[j];
-    }
-    if (tid == 0) a.ticket[t] = 0;
-    sync();
-    return true;
 }
 
 }  // namespace orthrus

@@ -1,8 +1,15 @@
 // Projection GEMMs on the 5th-generation tensor cores (tcgen05) for bf16.
 //
-// Same contract as the SIMT path in gemm.cu (work units, fixed split-K per
-// matrix shape, deterministic segment-order reduction, shared epilogues), with
-// a Blackwell mainloop:
+// Work split ("stream-K"): the (n tile, 64-wide k chunk) pairs of one 32-row
+// token tile, taken n-tile-major, are cut into G = min(148, pairs) equal
+// contiguous pieces, one per CTA; token tiles repeat the same cut.  A piece
+// covers the end of one n tile, whole n tiles and the start of another, so
+// every SM streams the same number of weight bytes whatever the matrix shape.
+// An n tile cut across pieces is reduced by the piece holding its first
+// chunks: the others publish fp32 partials and a flag, and that piece sums
+// them in segment order (fixed by the shape alone, never by the token count)
+// before the fused epilogue.  The piece holding a tile's last chunks works on
+// them first, so its partial is usually published long before it is needed.
 //
 //   warp 0      producer: one thread issues TMA tile loads (W: 128 rows x 64,
 //               X: 32 token rows x 64, both 128-byte swizzled) into a ring of
@@ -11,17 +18,22 @@
 //               N = 32 tokens, K = 16 per instruction) from shared memory into a
 //               TMEM accumulator; tcgen05.commit releases each stage when the
 //               MMAs reading it are done, and publishes the accumulator at the
-//               end of a unit;
-//   warps 2..5  epilogue: drain the accumulator with tcgen05.ld (warp w reads
-//               TMEM lanes 32*(w%4) ..), stage it as fp32 in shared memory and
-//               run the split-K gather and the fused epilogue.
+//               end of a tile's chunks;
+//   warps 2..5  epilogue: fetch what the epilogue needs (residual rows, cache
+//               destinations, other pieces' partials) while the chunks stream,
+//               then drain the accumulator with tcgen05.ld (warp w reads TMEM
+//               lanes 32*(w%4) ..), stage it in shared memory and either
+//               publish it as a partial or finish the tile.
 //
-// Two accumulators (2 x 32 TMEM columns) let unit i+1's MMAs run while unit i
-// drains.  Every mbarrier wait is bounded: on timeout the kernel raises
-// ORTHRUS_DEVERR_TIMEOUT, stops issuing, and still frees its TMEM.
+// Two accumulators (2 x 32 TMEM columns) let the next tile's MMAs run while
+// one drains.  Every wait (mbarrier or flag) is bounded: on timeout the
+// kernel raises ORTHRUS_DEVERR_TIMEOUT, stops issuing, and still frees its
+// TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <string.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "gemm_epilogue.cuh"
@@ -40,6 +52,7 @@ struct TcSmem {
     alignas(1024) unsigned char w[kTcStages][kStageWBytes];
     alignas(1024) unsigned char x[kTcStages][kStageXBytes];
     float tile[kTileM][kTilePad];
+    EpiPre pre;
     alignas(8) uint64_t full[kTcStages], empty[kTcStages], tfull[2], tempty[2];
     uint32_t tmem_base;
     int abort;
@@ -136,18 +149,90 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32])
     for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
 }
 
+// ---------------------------------------------------------------- work split
+// Piece g of G covers pairs [g*P/G, (g+1)*P/G) of the P = n_nt * chunks
+// (n tile, chunk) pairs of a token tile.
+struct SkShape {
+    long P;
+    int G, chunks, n_nt, n_mt;
+};
+__host__ __device__ inline long sk_begin(const SkShape &k, int g) { return (long)g * k.P / k.G; }
+// the piece holding pair x
+__host__ __device__ inline int sk_piece(const SkShape &k, long x)
+{
+    int g = (int)((x * k.G) / k.P);
+    while (g + 1 < k.G && sk_begin(k, g + 1) <= x) ++g;
+    while (g > 0 && sk_begin(k, g) > x) --g;
+    return g;
+}
+struct SkSub {
+    int mt, nt, c0, c1, seg, nseg;
+};
+// The sub-units (token tile, n tile, chunk range) of piece g, in order.
+struct SkIter {
+    SkShape k;
+    int g, mt, nt;
+    long b, e;
+    __device__ SkIter(const SkShape &k_, int g_) : k(k_), g(g_), mt(0)
+    {
+        b = sk_begin(k, g);
+        e = sk_begin(k, g + 1);
+        nt = (int)(b / k.chunks);
+        if (g >= k.G || b >= e) mt = k.n_mt;
+    }
+    __device__ bool valid() const { return mt < k.n_mt; }
+    __device__ SkSub get() const
+    {
+        const long tb = (long)nt * k.chunks;
+        SkSub s;
+        s.mt = mt;
+        s.nt = nt;
+        s.c0 = (int)((b > tb ? b : tb) - tb);
+        s.c1 = (int)((e < tb + k.chunks ? e : tb + k.chunks) - tb);
+        const int gf = sk_piece(k, tb), gl = sk_piece(k, tb + k.chunks - 1);
+        s.seg = g - gf;
+        s.nseg = gl - gf + 1;
+        return s;
+    }
+    __device__ void advance()
+    {
+        ++nt;
+        if ((long)nt * k.chunks >= e) {
+            ++mt;
+            nt = (int)(b / k.chunks);
+        }
+    }
+};
+
 // ---------------------------------------------------------------- kernel
 struct TcMaps {
     CUtensorMap w[3];   // weight segments (QKV: Q, K, V; SwiGLU: gate, up; else w[0])
     CUtensorMap x;      // activations
 };
 
+__device__ __forceinline__ bool flag_wait(const int *f, volatile int *abort)
+{
+    const long long t0 = clock64();
+    for (long i = 0;; ++i) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(f) : "memory");
+        if (v) return true;
+        if ((i & 63) == 63) {
+            if (*abort) return false;
+            if (clock64() - t0 > kSpinCycles) break;
+        }
+    }
+    *abort = 1;
+    return false;
+}
+
+template <int E>   // the epilogue (Epi), fixed at compile time
 __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_constant__ TcMaps maps, GemmArgs a,
-                                                                 int n_mt, int n_nt)
+                                                                 SkShape sk)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     TcSmem &sm = *(TcSmem *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    if (a.epi == EPI_RESAMPLE) {   // the flag comes from the previous kernel
+    if (E == EPI_RESAMPLE) {   // the flag comes from the previous kernel
         pdl_wait();
         if (*a.any_flag == 0) return;
     }
@@ -169,54 +254,48 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-
-    const int S = a.splits;
-    const int units = n_mt * n_nt * S;
-    const int chunks = a.Kd / kTileK;
+    const int g = blockIdx.x;
 
     if (warp == 0) {
         if (lane == 0) {   // ------------------------------------------- producer
-            // Weights never depend on earlier kernels: the first unit's first
+            // Weights never depend on earlier kernels: the first kTcStages
             // stages are requested before waiting for the predecessor grid;
             // their activation tiles follow once it has completed.
             uint32_t stage = 0, phase = 0;
-            int deferred = 0;   // stages whose X tile is still to be requested
-            for (int u = blockIdx.x; u < units && !*abort; u += gridDim.x) {
-                const int seg = u % S, t = u / S, mt = t % n_mt, nt = t / n_mt;
-                const int c0 = (int)((long)seg * chunks / S), c1 = (int)((long)(seg + 1) * chunks / S);
+            int issued = 0;
+            bool waited = false;
+            int def_c[kTcStages], def_mt[kTcStages];
+            auto release_deferred = [&]() {
+                pdl_wait();
+                waited = true;
+                for (int i = 0; i < issued && i < kTcStages; ++i)
+                    tma_load_2d(sm.x[i], &maps.x, def_c[i] * kTileK, def_mt[i] * kTileM, &sm.full[i]);
+            };
+            bool stop = false;
+            for (SkIter it(sk, g); it.valid() && !stop; it.advance()) {
+                const SkSub s = it.get();
                 // weight segment of this n tile
-                int wsel = 0, wrow = nt * kTileN;
-                if (a.epi != EPI_SWIGLU) {
+                int wsel = 0, wrow = s.nt * kTileN;
+                if (E != EPI_SWIGLU) {
                     while (wsel < 2 && wrow >= a.wrows[wsel]) { wrow -= a.wrows[wsel]; ++wsel; }
                 }
-                const bool first = u == (int)blockIdx.x;
-                for (int c = c0; c < c1; ++c) {
-                    if (first && deferred >= 0 && c - c0 == kTcStages) {
-                        pdl_wait();
-                        for (int i = 0; i < deferred; ++i)
-                            tma_load_2d(sm.x[i], &maps.x, (c0 + i) * kTileK, mt * kTileM, &sm.full[i]);
-                        deferred = -1;
-                    }
-                    if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort)) break;
+                for (int c = s.c0; c < s.c1; ++c) {
+                    if (!waited && issued == kTcStages) release_deferred();
+                    if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort) || *abort) { stop = true; break; }
                     mbar_expect_tx(&sm.full[stage], kStageWBytes + kStageXBytes);
-                    if (a.epi == EPI_SWIGLU) {
-                        tma_load_2d(sm.w[stage], &maps.w[0], c * kTileK, nt * 64, &sm.full[stage]);
-                        tma_load_2d(sm.w[stage] + kStageWBytes / 2, &maps.w[1], c * kTileK, nt * 64, &sm.full[stage]);
+                    if (E == EPI_SWIGLU) {
+                        tma_load_2d(sm.w[stage], &maps.w[0], c * kTileK, s.nt * 64, &sm.full[stage]);
+                        tma_load_2d(sm.w[stage] + kStageWBytes / 2, &maps.w[1], c * kTileK, s.nt * 64, &sm.full[stage]);
                     } else {
                         tma_load_2d(sm.w[stage], &maps.w[wsel], c * kTileK, wrow, &sm.full[stage]);
                     }
-                    if (first && deferred >= 0) ++deferred;
-                    else tma_load_2d(sm.x[stage], &maps.x, c * kTileK, mt * kTileM, &sm.full[stage]);
+                    if (!waited) { def_c[issued] = c; def_mt[issued] = s.mt; }
+                    else tma_load_2d(sm.x[stage], &maps.x, c * kTileK, s.mt * kTileM, &sm.full[stage]);
+                    ++issued;
                     if (++stage == kTcStages) { stage = 0; phase ^= 1; }
                 }
-                if (first && deferred >= 0) {   // first unit shorter than the ring
-                    pdl_wait();
-                    for (int i = 0; i < deferred; ++i)
-                        tma_load_2d(sm.x[i], &maps.x, (c0 + i) * kTileK, mt * kTileM, &sm.full[i]);
-                    deferred = -1;
-                }
             }
-            if (deferred >= 0) pdl_wait();
+            if (!waited) release_deferred();
             pdl_trigger();   // every load of this CTA is issued
         }
         __syncwarp();   // lanes 1..31 wait for the producer lane before the block barrier
@@ -224,22 +303,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
         if (lane == 0) {   // ------------------------------------------- MMA issuer
             uint32_t stage = 0, phase = 0;
             int local = 0;
-            for (int u = blockIdx.x; u < units && !*abort; u += gridDim.x, ++local) {
-                const int seg = u % S;
-                const int c0 = (int)((long)seg * chunks / S), c1 = (int)((long)(seg + 1) * chunks / S);
+            for (SkIter it(sk, g); it.valid() && !*abort; it.advance(), ++local) {
+                const SkSub s = it.get();
                 const int acc = local & 1;
                 const uint32_t aphase = (local >> 1) & 1;
                 if (!mbar_wait(&sm.tempty[acc], aphase ^ 1, abort)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + acc * kTcAccCols;
                 bool ok = true;
-                for (int c = c0; c < c1; ++c) {
+                for (int c = s.c0; c < s.c1; ++c) {
                     if (!mbar_wait(&sm.full[stage], phase, abort)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t ad = smem_desc_sw128(sm.w[stage]), bd = smem_desc_sw128(sm.x[stage]);
 #pragma unroll
                     for (int k = 0; k < kTileK / 16; ++k)   // +32 bytes per k step inside the swizzle atom
-                        umma_bf16(d, ad + 2 * k, bd + 2 * k, (c > c0 || k > 0) ? 1u : 0u);
+                        umma_bf16(d, ad + 2 * k, bd + 2 * k, (c > s.c0 || k > 0) ? 1u : 0u);
                     umma_commit(&sm.empty[stage]);
                     if (++stage == kTcStages) { stage = 0; phase ^= 1; }
                 }
@@ -252,12 +330,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
         pdl_wait();                                  // the epilogues read and write predecessor data
         const int et = threadIdx.x - 64;            // 0..127
         const int q = warp & 3;                      // TMEM lane quarter of this warp
+        const int n_nt_epi = E == EPI_SWIGLU ? (a.N + 63) / 64 : (a.N + kTileN - 1) / kTileN;
         int local = 0;
-        for (int u = blockIdx.x; u < units; u += gridDim.x, ++local) {
-            const int seg = u % S, t = u / S, mt = t % n_mt, nt = t / n_mt;
+        for (SkIter it(sk, g); it.valid(); it.advance(), ++local) {
+            const SkSub s = it.get();
             const int acc = local & 1;
             const uint32_t aphase = (local >> 1) & 1;
-            const bool ok = mbar_wait(&sm.tfull[acc], aphase, abort);
+            const size_t slot0 = ((size_t)s.mt * sk.n_nt + s.nt) * a.splits;   // partial / flag slots of this tile
+            // -------- before the accumulator is ready
+            float4 rest[kEpiVec];   // segments 1.. of the tile, summed in order (reducer only)
+            bool good = !*abort;
+            const bool defer = a.defer > 0;
+            if (!defer && s.seg == 0 && s.nseg > 1) {
+                for (int sg = 1; sg < s.nseg && good; ++sg) {
+                    if (et == 0) good = flag_wait(a.ticket + slot0 + sg, abort);
+                    SyncEpilogue{}();
+                    good = good && !*abort;
+                    if (!good) break;
+                    const float *src = a.part + (slot0 + sg) * (kTileM * kTileN);
+#pragma unroll
+                    for (int j = 0; j < kEpiVec; ++j) {
+                        const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
+                        const float4 v = __ldcg((const float4 *)(src + m * kTileN + c4));
+                        if (sg == 1) rest[j] = v;
+                        else { rest[j].x += v.x; rest[j].y += v.y; rest[j].z += v.z; rest[j].w += v.w; }
+                    }
+                }
+            }
+            if (!defer && s.seg == 0) epilogue_prepare<bf16, E>(a, sm.pre, s.mt, s.nt, et);
+            // -------- the accumulator
+            const bool ok = good && mbar_wait(&sm.tfull[acc], aphase, abort);
             SyncEpilogue{}();
             if (!ok || *abort) break;
             tc_fence_after();
@@ -269,8 +371,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
 #pragma unroll
             for (int j = 0; j < kTileM; ++j) sm.tile[j][f] = r[j];
             SyncEpilogue{}();
-            if (split_k_gather(a, sm.tile, t, seg, et, &sm.s_last, SyncEpilogue{}))
-                epilogue<bf16>(a, sm.tile, mt, nt, n_nt, et, SyncEpilogue{});
+            if (defer) {   // this segment of the residual update, summed later by the RMSNorm
+#pragma unroll
+                for (int j = 0; j < kEpiVec; ++j) {
+                    const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
+                    const int row = s.mt * kTileM + m, n = s.nt * kTileN + c4;
+                    if (row < a.M && n < a.N)
+                        __stcg((float4 *)(a.rpart + ((size_t)s.seg * a.rpart_rows + row) * a.N + n),
+                               *(const float4 *)&sm.tile[m][c4]);
+                }
+                SyncEpilogue{}();
+                continue;
+            }
+            if (s.seg > 0) {   // publish this segment for the tile's reducer
+                float *dst = a.part + (slot0 + s.seg) * (kTileM * kTileN);
+#pragma unroll
+                for (int j = 0; j < kEpiVec; ++j) {
+                    const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
+                    __stcg((float4 *)(dst + m * kTileN + c4), *(const float4 *)&sm.tile[m][c4]);
+                }
+                __threadfence();
+                SyncEpilogue{}();
+                if (et == 0) asm volatile("st.release.gpu.global.b32 [%0], %1;\n" ::"l"(a.ticket + slot0 + s.seg), "r"(1) : "memory");
+                continue;
+            }
+            if (s.nseg > 1) {   // reducer: (segments 1..) + segment 0, then clear the flags
+#pragma unroll
+                for (int j = 0; j < kEpiVec; ++j) {
+                    const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
+                    float4 &o = *(float4 *)&sm.tile[m][c4];
+                    o.x = rest[j].x + o.x; o.y = rest[j].y + o.y; o.z = rest[j].z + o.z; o.w = rest[j].w + o.w;
+                }
+                if (et > 0 && et < s.nseg) a.ticket[slot0 + et] = 0;
+                SyncEpilogue{}();
+            }
+            epilogue<bf16, SyncEpilogue, E>(a, sm.tile, s.mt, s.nt, n_nt_epi, et, SyncEpilogue{}, &sm.pre);
             SyncEpilogue{}();
         }
     }
@@ -338,15 +473,44 @@ bool make_tmap_q4(CUtensorMap *m, const void *q, int rows_total, int n_q, int n_
 
 size_t gemm_tc_smem_bytes() { return sizeof(TcSmem) + 1024; }
 
+template <int E> static cudaError_t set_smem()
+{
+    return cudaFuncSetAttribute(gemm_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_tc_smem_bytes());
+}
+
 cudaError_t gemm_tc_init_attributes()
 {
-    return cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)gemm_tc_smem_bytes());
+    cudaError_t e = set_smem<EPI_QKV>();
+    if (e == cudaSuccess) e = set_smem<EPI_RESID>();
+    if (e == cudaSuccess) e = set_smem<EPI_SWIGLU>();
+    if (e == cudaSuccess) e = set_smem<EPI_LMHEAD>();
+    if (e == cudaSuccess) e = set_smem<EPI_RESAMPLE>();
+    if (e == cudaSuccess) e = set_smem<EPI_LOGITS>();
+    return e;
+}
+
+// Largest number of pieces one n tile is cut into, for n_nt tiles of
+// `chunks` k chunks (the partial and flag slots per tile).
+int sk_max_segments(int n_nt, int chunks)
+{
+    SkShape k;
+    k.P = (long)n_nt * chunks;
+    k.G = (int)std::min<long>(kNumSMs, k.P);
+    k.chunks = chunks;
+    k.n_nt = n_nt;
+    k.n_mt = 1;
+    int best = 1;
+    for (int nt = 0; nt < n_nt; ++nt) {
+        const long tb = (long)nt * chunks;
+        best = std::max(best, sk_piece(k, tb + chunks - 1) - sk_piece(k, tb) + 1);
+    }
+    return best;
 }
 
 // Launches the tcgen05 kernel when every operand has a tensor map; returns
 // cudaErrorNotSupported otherwise (the caller then uses the SIMT kernel).
-cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, int grid, cudaStream_t s)
+// a.splits must hold sk_max_segments(n_nt, Kd / 64).
+cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, cudaStream_t s)
 {
     TcMaps maps;
     memset(&maps, 0, sizeof(maps));
@@ -361,8 +525,25 @@ cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, 
     auto it = c.tmaps.find(TmapKey{a.x, (uint32_t)kTileM});
     if (it == c.tmaps.end()) return cudaErrorNotSupported;
     maps.x = it->second;
+    SkShape k;
+    k.chunks = a.Kd / kTileK;
+    k.n_nt = n_nt;
+    k.n_mt = n_mt;
+    k.P = (long)n_nt * k.chunks;
+    // deferred residual: one piece per (tile, segment), cut at whole chunks
+    k.G = a.defer > 0 ? n_nt * a.defer : (int)std::min<long>(kNumSMs, k.P);
+    if (a.defer > 0 && (k.chunks % a.defer || a.defer > kResidSlots || !a.rpart)) return cudaErrorInvalidValue;
     c.launches += 1;
-    return launch_k(gemm_tc_kernel, grid, kTcThreads, gemm_tc_smem_bytes(), s, maps, a, n_mt, n_nt);
+    const size_t smem = gemm_tc_smem_bytes();
+    switch (a.epi) {
+    case EPI_QKV: return launch_k(gemm_tc_kernel<EPI_QKV>, k.G, kTcThreads, smem, s, maps, a, k);
+    case EPI_RESID: return launch_k(gemm_tc_kernel<EPI_RESID>, k.G, kTcThreads, smem, s, maps, a, k);
+    case EPI_SWIGLU: return launch_k(gemm_tc_kernel<EPI_SWIGLU>, k.G, kTcThreads, smem, s, maps, a, k);
+    case EPI_LMHEAD: return launch_k(gemm_tc_kernel<EPI_LMHEAD>, k.G, kTcThreads, smem, s, maps, a, k);
+    case EPI_RESAMPLE: return launch_k(gemm_tc_kernel<EPI_RESAMPLE>, k.G, kTcThreads, smem, s, maps, a, k);
+    case EPI_LOGITS: return launch_k(gemm_tc_kernel<EPI_LOGITS>, k.G, kTcThreads, smem, s, maps, a, k);
+    default: return cudaErrorNotSupported;
+    }
 }
 
 }  // namespace orthrus

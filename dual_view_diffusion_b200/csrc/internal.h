@@ -19,7 +19,8 @@ constexpr int kTileM = 32;           // GEMM tile: token rows per tile
 constexpr int kTileK = 64;           // GEMM k chunk
 constexpr int kKeyTile = 64;         // attention: keys per tile
 constexpr int kPrefillChunk = 128;   // prefill rows per forward
-constexpr int kNumSMs = 148;         // B200
+constexpr int kNumSMs = 148;
+constexpr int kResidSlots = 8;   // most k segments of a deferred residual GEMM         // B200
 
 // Per-(row, vocab tile) record of the fused LM-head epilogue.
 struct LmPart {
@@ -50,13 +51,18 @@ struct GemmArgs {
     // SwiGLU epilogue, tile halves [0,64) from w[0] and [64,128) from w[1]
     const void *w[3];
     int wrows[3];
-    int splits;              // k segments per tile (fixed per matrix shape)
-    float *part;             // split partial tiles
-    int *ticket;             // per (m tile, n tile) arrival counters
+    int splits;              // partial / flag slots per (m tile, n tile): the most pieces a tile is cut into
+    float *part;             // [m tile][n tile][slot] fp32 partial tiles of a cut n tile
+    int *ticket;             // [m tile][n tile][slot] published flags (reset by the tile's reducer)
     unsigned *err;
     int epi;
     // EPI_RESID
     float *resid;            // [M][N] fp32, += result
+    // deferred residual (tensor-core path): the k segments of each tile are
+    // written to rpart[seg][row][N] and summed into resid by the next RMSNorm
+    int defer;               // segments per tile (0: add in the epilogue)
+    float *rpart;
+    int rpart_rows;
     // EPI_SWIGLU
     void *act;               // [M][N/2] dtype
     // EPI_QKV
@@ -70,6 +76,7 @@ struct GemmArgs {
     const int32_t *bt_rows;  // [batch] row of block_table for each batch entry
     int K;                   // rows per sequence in this launch
     double rope_theta;
+    const double *rope_invf; // [head_dim / 2] theta^(-2i / head_dim), computed once on the host
     // EPI_LMHEAD / EPI_RESAMPLE
     LmPart *lm;              // [M][n_vtiles]
     float inv_temp;          // 1/T (T > 0) or 0 for greedy
@@ -163,6 +170,8 @@ struct Ctx {
     int *gemm_ticket;
     void *blk_pack;          // [2][max_batch][n_kv][kp][hd]: user block K/V repacked (standalone attention)
     int gemm_tickets;
+    float *resid_part;       // [kResidSlots][Rw][hidden] deferred residual segments
+    double *rope_invf;       // [head_dim / 2] rotary inverse frequencies
     LmPart *lm_part;         // [max(R, 2*max_batch)][n_vtiles]
     int32_t *tok;            // [Rw] block tokens
     int32_t *pos0;           // [max_batch]
@@ -196,7 +205,6 @@ struct Layout {
 // workspace carve-up shared by orthrus_workspace_size and orthrus_create
 size_t plan_workspace(const orthrus_config_t &c, Ctx *ctx);
 
-int choose_splits(int N, int Kd);
 bool use_tensor_cores(const orthrus_config_t &c);
 
 // ---------------------------------------------------------------- launchers
@@ -208,14 +216,16 @@ bool make_tmap_box(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols
 bool make_tmap_q4(CUtensorMap *m, const void *q, int rows_total, int n_q, int n_kv, int hd, int ksub);
 struct AtMaps;
 cudaError_t attn_tc_init_attributes();
-cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, int grid, cudaStream_t s);
+cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, cudaStream_t s);
+int sk_max_segments(int n_nt, int chunks);
 cudaError_t attention_init_attributes();
 cudaError_t launch_attention(const Ctx &c, const AttnArgs &a, cudaStream_t s, int q_rows);
 cudaError_t launch_attn_tc_cached(const Ctx &c, const AttnArgs &a, int n_split_grid, int q_rows, cudaStream_t s);
 bool attn_tc_maps(const AttnArgs &a, int n_layers, int rows_total, AtMaps *m);
 cudaError_t launch_embed(const Ctx &c, int mode, const int32_t *tokens, const int32_t *anchor,
                          const int32_t *draft, int B, int K, cudaStream_t s);
-cudaError_t launch_rmsnorm(const Ctx &c, const float *h, const void *gain, void *out, int M, cudaStream_t s);
+cudaError_t launch_rmsnorm(const Ctx &c, float *h, const void *gain, void *out, int M, int pending, cudaStream_t s);
+int resid_defer_slots(const orthrus_config_t &cfg, int N, int Kd);
 cudaError_t launch_lm_finalize(const Ctx &c, int mode, int B, int K, float temperature, uint64_t seed,
                                const int64_t *step, int32_t *tok_out, cudaStream_t s);
 cudaError_t launch_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int K, float temperature, uint64_t seed,
