@@ -36,7 +36,7 @@ __global__ void embed_kernel(const T *embed, int d, int V, int mask_id, int mode
 // out = h / sqrt(mean(h^2) + eps) * gain; fixed reduction order per row.
 // Rows of up to 8192 elements (multiple of 4) stay in registers: every load
 // is issued before the first use.
-constexpr int kNormThreads = 256, kNormVec = 8;
+constexpr int kNormThreads = 512, kNormVec = 2;   // vector path for rows up to 4096
 
 template <class T>
 __device__ __forceinline__ void store4(T *p, float a, float b, float c, float d);
@@ -82,17 +82,23 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(float *h, const T
             v[j] = i < d ? *(const float4 *)(x + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         if (pending > 0) {
-            for (int sl = 0; sl < pending; ++sl) {
+            // every segment's loads are issued before the first add
+            float4 u[kResidSlots][kNormVec];
+#pragma unroll
+            for (int sl = 0; sl < kResidSlots; ++sl) {
                 const float *p = part + sl * slot_stride + (size_t)row * d;
-                float4 u[kNormVec];
 #pragma unroll
                 for (int j = 0; j < kNormVec; ++j) {
                     const int i = (tid + j * kNormThreads) * 4;
-                    u[j] = i < d ? __ldcg((const float4 *)(p + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    u[sl][j] = (sl < pending && i < d) ? __ldcg((const float4 *)(p + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
+            }
+#pragma unroll
+            for (int sl = 0; sl < kResidSlots; ++sl) {
+                if (sl >= pending) break;
 #pragma unroll
                 for (int j = 0; j < kNormVec; ++j) {
-                    v[j].x += u[j].x; v[j].y += u[j].y; v[j].z += u[j].z; v[j].w += u[j].w;
+                    v[j].x += u[sl][j].x; v[j].y += u[sl][j].y; v[j].z += u[sl][j].z; v[j].w += u[sl][j].w;
                 }
             }
 #pragma unroll
