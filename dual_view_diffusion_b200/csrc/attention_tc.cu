@@ -51,16 +51,14 @@ struct AtSmem {
     alignas(1024) unsigned char p[2][kAtRows * 128];              // P [128 rows][64 keys], 16 KiB, per accumulator
     alignas(8) uint64_t q_full, full[kAtStages], empty[kAtStages], s_full[2], p_full[2], o_done[2];
     float2 xml[2][kAtRows];   // (m, l) of each accumulator, per row
-    uint64_t ready;       // one arrival from every CTA of the cluster whose ring is free
-    uint64_t land_full;   // bytes of the partial rows pushed to this CTA
     uint32_t tmem_base;
     int abort;
 };
-// Once the last P.V is done, q..p (192 KiB) is reused for the combine:
-// the CTA's own merged rows and (m, l) (staging), and the rows the other
-// CTAs push to it (landing).
-constexpr uint32_t kStageO = 0, kStageMl = 64 * 1024, kLandO = 68 * 1024, kLandMl = 132 * 1024;
-static_assert(kLandMl + kAtRows * 8 <= 2 * 16384 + kAtStages * 32768 + 2 * 16384, "combine area");
+// Once the last P.V is done, q..v (160 KiB) is reused for the combine: the
+// CTA's merged rows [128][128] fp32 (16-byte chunk ch of row r at ch ^ (r & 31))
+// and (m, l) per row, read by the other CTAs of the cluster.
+constexpr uint32_t kStageO = 0, kStageMl = 64 * 1024;
+static_assert(kStageMl + kAtRows * 8 <= 2 * 16384 + kAtStages * 32768, "combine area");
 
 // TMEM columns: two O accumulators (even / odd tiles) [0, 256), S double
 // buffer [256, 384)
@@ -196,17 +194,17 @@ __device__ __forceinline__ void cluster_arrive_relaxed()
 }
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory"); }
-// arrive on an mbarrier of another CTA of the cluster (release at cluster scope)
-__device__ __forceinline__ void arrive_peer(uint32_t cluster_addr)
+__device__ __forceinline__ float4 ld_peer4(uint32_t addr)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];\n" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
 }
-// bulk copy of this CTA's shared memory into another CTA's, completing bytes
-// on that CTA's mbarrier
-__device__ __forceinline__ void bulk_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t mbar)
+__device__ __forceinline__ float2 ld_peer2(uint32_t addr)
 {
-    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
-                 ::"r"(dst), "r"(src), "r"(bytes), "r"(mbar) : "memory");
+    float2 v;
+    asm volatile("ld.shared::cluster.v2.f32 {%0,%1}, [%2];\n" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+    return v;
 }
 __device__ __forceinline__ float ex2(float x)   // 2^x, MUFU; subnormal results flush to zero
 {
@@ -222,10 +220,10 @@ __device__ __forceinline__ float ex2(float x)   // 2^x, MUFU; subnormal results 
 // decoded, and keys outside a row's window are exact no-ops).  Even and odd
 // tiles go to two independent accumulators (O, m, l), so the softmax of one
 // tile never waits for the P.V of the tile just before it; the two are merged
-// at the end.  The C partial states are then combined on chip: CTA q owns rows
-// [q*128/C, (q+1)*128/C); every CTA bulk-copies its merged rows to their
-// owner once the owner's ring is free, and each owner sums the C states in
-// rank order from its own shared memory.
+// at the end.  The C partial states are then combined on chip: every CTA
+// stages its merged rows in its own shared memory, and CTA q reads rows
+// [q*128/C, (q+1)*128/C) from all C CTAs (all loads in flight at once) and
+// sums them in rank order.
 template <int C>
 __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a,
                                                                 int n_split_grid)
@@ -276,12 +274,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
             at_mbar_init(&sm.p_full[i], 128);
             at_mbar_init(&sm.o_done[i], 1);
         }
-        at_mbar_init(&sm.ready, C);
-        at_mbar_init(&sm.land_full, 1);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-        // every CTA of the cluster pushes rpc rows of O and of (m, l) here
-        at_expect(&sm.land_full, (uint32_t)C * rpc * (512u + 8u));
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&sm.tmem_base)),
@@ -291,8 +285,6 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     at_fence_before();
     __syncthreads();
     at_fence_after();
-    // the barriers of every CTA are initialised before any CTA signals another
-    cluster_arrive_relaxed();
     const uint32_t tmem = sm.tmem_base;
     int my_tiles = 0;
     for (int s = r; s < n_total; s += C) my_tiles += at_split(a, s, n_split_grid, t).ntiles;
@@ -484,15 +476,12 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     // ------------------------------------------------------------------ combine
     unsigned char *area = sm.q[0];
     const uint32_t area_u = smem_u32(area);
-    cluster_wait();   // every CTA's barriers are initialised
     if (warp >= 2) {
         const int h = (warp - 2) >> 2;
         asm volatile("bar.sync 1, 256;\n" ::: "memory");   // both warpgroups: every P.V is done
-        // the K/V ring, Q and P are no longer read: tell every CTA it may push here
-        if (warp == 2 && lane < C) arrive_peer(map_peer_addr(smem_u32(&sm.ready), lane));
-        __syncwarp();
-        // merge the two accumulators into (O, m, l) of this row -> staging;
-        // warpgroup h takes dims [64h, 64h + 64)
+        // merge the two accumulators into (O, m, l) of this row -> staging (the
+        // K/V ring, Q and P are no longer read); warpgroup h takes dims
+        // [64h, 64h + 64)
         const float2 x0 = sm.xml[0][row], x1 = sm.xml[1][row];
         const float M = fmaxf(x0.x, x1.x);
         const float w0 = x0.y > 0.f ? ex2(x0.x - M) : 0.f, w1 = x1.y > 0.f ? ex2(x1.x - M) : 0.f;
@@ -519,58 +508,55 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
             }
         }
         if (h == 0) ((float2 *)(area + kStageMl))[row] = l > 0.f ? make_float2(M, l) : make_float2(-INFINITY, 0.f);
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         at_fence_before();
         __syncwarp();
-        asm volatile("bar.sync 1, 256;\n" ::: "memory");
-        if (threadIdx.x == 64) {   // push rows [q*rpc, (q+1)*rpc) to CTA q once its ring is free
-            if (at_wait(&sm.ready, 0, abort)) {
-#pragma unroll
-                for (int q = 0; q < C; ++q) {
-                    const uint32_t mbar = map_peer_addr(smem_u32(&sm.land_full), q);
-                    bulk_to_peer(map_peer_addr(area_u + kLandO + r * rpc * 512, q), area_u + kStageO + q * rpc * 512,
-                                 rpc * 512, mbar);
-                    bulk_to_peer(map_peer_addr(area_u + kLandMl + r * rpc * 8, q), area_u + kStageMl + q * rpc * 8,
-                                 rpc * 8, mbar);
-                }
-            }
-        }
-        __syncwarp();
-        // ------------------------------------------------------- owner: rows [r*rpc, (r+1)*rpc)
+    }
+    // every CTA's merged rows are in its shared memory (release / acquire)
+    cluster_arrive();
+    cluster_wait();
+    if (warp >= 2) {   // ----------------------------------- owner: rows [r*rpc, (r+1)*rpc), pulled from every CTA
         constexpr int tpr = 256 / rpc;            // threads per owned row: chunks cc, cc + tpr, ...
-        const bool landed = at_wait(&sm.land_full, 0, abort);
+        constexpr int cpt = 32 / tpr;             // chunks per thread
         const int et = threadIdx.x - 64;
         const int rl = et / tpr, cc = et % tpr;
         const int orow = r * rpc + rl;
-        const float2 *lml = (const float2 *)(area + kLandMl);
-        const float *lo = (const float *)(area + kLandO);
-        float wc[C];
+        uint32_t peer[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) peer[c] = map_peer_addr(area_u, c);
+        float2 ml[C];
+        float4 v[cpt][C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) ml[c] = ld_peer2(peer[c] + kStageMl + orow * 8);
+#pragma unroll
+        for (int i = 0; i < cpt; ++i) {
+            const int ch = cc + i * tpr;
+#pragma unroll
+            for (int c = 0; c < C; ++c)
+                v[i][c] = ld_peer4(peer[c] + kStageO + orow * 512 + ((ch ^ (orow & 31)) << 4));
+        }
         float Mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < C; ++c) {
-            const float2 ml = lml[c * rpc + rl];
-            if (ml.y > 0.f) Mx = fmaxf(Mx, ml.x);
-        }
-        float L = 0.f;
+        for (int c = 0; c < C; ++c)
+            if (ml[c].y > 0.f) Mx = fmaxf(Mx, ml[c].x);
+        float wc[C], L = 0.f;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            const float2 ml = lml[c * rpc + rl];
-            wc[c] = ml.y > 0.f ? ex2(ml.x - Mx) : 0.f;
-            L += wc[c] * ml.y;
+            wc[c] = ml[c].y > 0.f ? ex2(ml[c].x - Mx) : 0.f;
+            L += wc[c] * ml[c].y;
         }
         const int rrow = k_lo * g + orow, k = rrow / g, jh = rrow % g;
-        if (landed && orow < (k_hi - k_lo) * g && L > 0.f) {
+        if (!*abort && orow < (k_hi - k_lo) * g && L > 0.f) {
             const float inv = 1.0f / L;
             bf16 *o = (bf16 *)a.out + ((size_t)(b * a.K + k) * a.n_q + kvh * g + jh) * 128;
 #pragma unroll
-            for (int ch = cc; ch < 32; ch += tpr) {
+            for (int i = 0; i < cpt; ++i) {
+                const int ch = cc + i * tpr;
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < C; ++c) {
                     if (wc[c] == 0.f) continue;
-                    const float4 v = *(const float4 *)(lo + (size_t)(c * rpc + rl) * 128 + ((ch ^ (orow & 31)) << 2));
-                    acc.x = fmaf(wc[c], v.x, acc.x); acc.y = fmaf(wc[c], v.y, acc.y);
-                    acc.z = fmaf(wc[c], v.z, acc.z); acc.w = fmaf(wc[c], v.w, acc.w);
+                    acc.x = fmaf(wc[c], v[i][c].x, acc.x); acc.y = fmaf(wc[c], v[i][c].y, acc.y);
+                    acc.z = fmaf(wc[c], v[i][c].z, acc.z); acc.w = fmaf(wc[c], v[i][c].w, acc.w);
                 }
                 const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
                 const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
@@ -579,8 +565,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
         }
         __syncwarp();
     }
-    // every CTA has received all its rows (so every copy out of this CTA is
-    // complete) before any CTA leaves
+    // no CTA leaves while another may still be reading its shared memory
     cluster_arrive_relaxed();
     cluster_wait();
 
@@ -599,7 +584,8 @@ bool make_tmap_q4(CUtensorMap *m, const void *q, int rows_total, int n_q, int n_
 
 size_t attn_tc_smem_bytes() { return sizeof(AtSmem) + 1024; }
 
-// CTAs per (sequence, KV head, row group): a power of two up to 8 that keeps
+// CTAs per (sequence, KV head, row group): a power of two up to 8 (the
+// portable cluster size; 16-CTA clusters measured slower on B200) that keeps
 // one row group of the whole batch within one wave of SMs.  A function of the
 // batch and model shape only (not of the block size), so a row is reduced in
 // the same order whatever block it is in.
