@@ -139,6 +139,8 @@ cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s)
     if (tc) {   // stream-K split: partial and flag slots per (token tile, n tile, segment)
         GemmArgs t = a;
         t.splits = t.defer > 0 ? t.defer : sk_max_segments(n_nt, a.Kd / kTileK);
+        // QKV: each head tile cut in two k halves reduced inside a 2-CTA cluster
+        t.pair = (a.epi == EPI_QKV && t.defer == 0 && (a.Kd / kTileK) % 2 == 0) ? 1 : 0;
         const size_t slots = (size_t)n_mt * n_nt * t.splits;
         if (t.splits > 1 && (slots * kTileM * kTileN > c.gemm_part_floats || slots > (size_t)c.gemm_tickets))
             return cudaErrorInvalidValue;

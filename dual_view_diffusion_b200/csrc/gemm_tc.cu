@@ -52,8 +52,10 @@ struct TcSmem {
     alignas(1024) unsigned char w[kTcStages][kStageWBytes];
     alignas(1024) unsigned char x[kTcStages][kStageXBytes];
     float tile[kTileM][kTilePad];
+    float peer[kTileM][kTilePad];     // pair mode, rank 0: the other half's fp32 tile
     EpiPre pre;
     alignas(8) uint64_t full[kTcStages], empty[kTcStages], tfull[2], tempty[2];
+    uint64_t peer_full, peer_empty;   // pair mode: the second half's tile landed / was consumed
     uint32_t tmem_base;
     int abort;
     int s_last;
@@ -130,6 +132,21 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar)
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
                  : "memory");
 }
+__device__ __forceinline__ uint32_t tc_cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t tc_mapa(uint32_t local, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void tc_cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_cluster_arrive() { asm volatile("barrier.cluster.arrive;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_cluster_wait() { asm volatile("barrier.cluster.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
 
@@ -242,6 +259,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     if (threadIdx.x == 0) {
         for (int s = 0; s < kTcStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
         for (int s = 0; s < 2; ++s) { mbar_init(&sm.tfull[s], 1); mbar_init(&sm.tempty[s], kEpiThreads); }
+        mbar_init(&sm.peer_full, 1);
+        mbar_init(&sm.peer_empty, 1);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
@@ -255,6 +274,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int g = blockIdx.x;
+    // pair mode: the two CTAs of a cluster hold the two k halves of the same
+    // n tiles; rank 1 hands its fp32 tile to rank 0 through distributed shared
+    // memory.  Both CTAs' barriers are initialised before either signals the
+    // other (start of the cluster barrier; its wait comes before the first
+    // remote operation).
+    const bool pair = a.pair != 0;
+    const uint32_t crank = pair ? tc_cluster_rank() : 0u;
+    if (pair) tc_cluster_arrive_relaxed();
 
     if (warp == 0) {
         if (lane == 0) {   // ------------------------------------------- producer
@@ -328,6 +355,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
         __syncwarp();   // lanes 1..31 wait for the MMA lane before the block barrier
     } else {   // --------------------------------------------------------- epilogue
         pdl_wait();                                  // the epilogues read and write predecessor data
+        if (pair) tc_cluster_wait();
         const int et = threadIdx.x - 64;            // 0..127
         const int q = warp & 3;                      // TMEM lane quarter of this warp
         const int n_nt_epi = E == EPI_SWIGLU ? (a.N + 63) / 64 : (a.N + kTileN - 1) / kTileN;
@@ -341,7 +369,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
             float4 rest[kEpiVec];   // segments 1.. of the tile, summed in order (reducer only)
             bool good = !*abort;
             const bool defer = a.defer > 0;
-            if (!defer && s.seg == 0 && s.nseg > 1) {
+            if (pair) {
+                if (crank == 0) {
+                    if (et == 0) mbar_expect_tx(&sm.peer_full, (uint32_t)sizeof(sm.peer));
+                } else {   // the previous tile handed over has been consumed
+                    if (et == 0) good = mbar_wait(&sm.peer_empty, (local & 1) ^ 1, abort);
+                    SyncEpilogue{}();
+                    good = good && !*abort;
+                }
+            }
+            if (!pair && !defer && s.seg == 0 && s.nseg > 1) {
                 for (int sg = 1; sg < s.nseg && good; ++sg) {
                     if (et == 0) good = flag_wait(a.ticket + slot0 + sg, abort);
                     SyncEpilogue{}();
@@ -370,7 +407,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
             const int f = q * 32 + lane;             // weight row = output feature in the tile
 #pragma unroll
             for (int j = 0; j < kTileM; ++j) sm.tile[j][f] = r[j];
+            if (pair && crank == 1) {   // hand this half to rank 0
+                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                SyncEpilogue{}();
+                if (et == 0) {
+                    const uint32_t dst = tc_mapa(smem_u32(&sm.peer[0][0]), 0), bar = tc_mapa(smem_u32(&sm.peer_full), 0);
+                    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+                                 ::"r"(dst), "r"(smem_u32(&sm.tile[0][0])), "r"((uint32_t)sizeof(sm.tile)), "r"(bar) : "memory");
+                }
+                continue;
+            }
             SyncEpilogue{}();
+            if (pair) {   // rank 0: (second half) + first half, then free the landing tile
+                bool landed = true;
+                if (et == 0) landed = mbar_wait(&sm.peer_full, local & 1, abort);
+                SyncEpilogue{}();
+                if (!landed || *abort) break;
+#pragma unroll
+                for (int j = 0; j < kEpiVec; ++j) {
+                    const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
+                    float4 &o = *(float4 *)&sm.tile[m][c4];
+                    const float4 p = *(const float4 *)&sm.peer[m][c4];
+                    o.x = p.x + o.x; o.y = p.y + o.y; o.z = p.z + o.z; o.w = p.w + o.w;
+                }
+                SyncEpilogue{}();
+                if (et == 0)
+                    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n"
+                                 ::"r"(tc_mapa(smem_u32(&sm.peer_empty), 1)) : "memory");
+            }
             if (defer) {   // this segment of the residual update, summed later by the RMSNorm
 #pragma unroll
                 for (int j = 0; j < kEpiVec; ++j) {
@@ -383,7 +447,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                 SyncEpilogue{}();
                 continue;
             }
-            if (s.seg > 0) {   // publish this segment for the tile's reducer
+            if (!pair && s.seg > 0) {   // publish this segment for the tile's reducer
                 float *dst = a.part + (slot0 + s.seg) * (kTileM * kTileN);
 #pragma unroll
                 for (int j = 0; j < kEpiVec; ++j) {
@@ -395,7 +459,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                 if (et == 0) asm volatile("st.release.gpu.global.b32 [%0], %1;\n" ::"l"(a.ticket + slot0 + s.seg), "r"(1) : "memory");
                 continue;
             }
-            if (s.nseg > 1) {   // reducer: (segments 1..) + segment 0, then clear the flags
+            if (!pair && s.nseg > 1) {   // reducer: (segments 1..) + segment 0, then clear the flags
 #pragma unroll
                 for (int j = 0; j < kEpiVec; ++j) {
                     const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
@@ -412,6 +476,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
 
     tc_fence_before();
     __syncthreads();
+    if (pair) {   // no CTA leaves while the other may still signal or copy into it
+        if (warp < 2) tc_cluster_wait();
+        tc_cluster_arrive();
+        tc_cluster_wait();
+    }
     if (sm.abort && threadIdx.x == 0) raise_err(a.err, ORTHRUS_DEVERR_TIMEOUT);
     if (warp == 1) {
         __syncwarp();
@@ -533,8 +602,28 @@ cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, 
     // deferred residual: one piece per (tile, segment), cut at whole chunks
     k.G = a.defer > 0 ? n_nt * a.defer : (int)std::min<long>(kNumSMs, k.P);
     if (a.defer > 0 && (k.chunks % a.defer || a.defer > kResidSlots || !a.rpart)) return cudaErrorInvalidValue;
-    c.launches += 1;
     const size_t smem = gemm_tc_smem_bytes();
+    if (a.pair) {   // two k halves per n tile, one 2-CTA cluster per tile
+        if (a.epi != EPI_QKV || a.defer > 0 || k.chunks % 2) return cudaErrorInvalidValue;
+        k.G = 2 * n_nt;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(k.G);
+        cfg.blockDim = dim3(kTcThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = 2;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        c.launches += 1;
+        return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_QKV>, maps, a, k);
+    }
+    c.launches += 1;
     switch (a.epi) {
     case EPI_QKV: return launch_k(gemm_tc_kernel<EPI_QKV>, k.G, kTcThreads, smem, s, maps, a, k);
     case EPI_RESID: return launch_k(gemm_tc_kernel<EPI_RESID>, k.G, kTcThreads, smem, s, maps, a, k);

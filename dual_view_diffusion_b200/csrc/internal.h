@@ -61,6 +61,7 @@ struct GemmArgs {
     // deferred residual (tensor-core path): the k segments of each tile are
     // written to rpart[seg][row][N] and summed into resid by the next RMSNorm
     int defer;               // segments per tile (0: add in the epilogue)
+    int pair;                // tensor-core path: each n tile cut in two k halves by a 2-CTA cluster
     float *rpart;
     int rpart_rows;
     // EPI_SWIGLU
