@@ -29,7 +29,8 @@ static std::mutex g_scratch_mu;
 
 __global__ void noalloc_identity_rows(int32_t *rows, int n)
 {
-    pdl_trigger();
+    // no early pdl_trigger: the attention reads these rows before its
+    // griddepcontrol.wait, so it may not be scheduled until this kernel exits
     pdl_wait();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) rows[i] = i;

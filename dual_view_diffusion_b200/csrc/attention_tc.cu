@@ -244,9 +244,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     const int n_total = n_split_grid + (a.mode == 1 ? 1 : 0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
-    // t, the block table and its row were written by kernels that completed
-    // before the predecessor of this one started (every launch waits on its
-    // own predecessor), so they may be read before griddepcontrol.wait
+    // t, the block table and its row are written only by kernels that do not
+    // trigger their dependents early (commit, set-length, row-map kernels),
+    // so every kernel after them in the stream starts after they completed:
+    // they may be read before griddepcontrol.wait
     const int t = a.seq_lens[b];
     const int bt_row = a.bt_rows[b];
     // Flat tile f of this CTA is tile f % tps of split r + C * (f / tps) for

@@ -280,7 +280,8 @@ __global__ void commit_decide_kernel(CommitArgs a)
 // are already in place: paper notes §4.1 step 3), bump the step counter.
 __global__ void commit_apply_kernel(CommitArgs a)
 {
-    pdl_trigger();
+    // no early pdl_trigger: later kernels read what this one writes before
+    // their griddepcontrol.wait, so nothing may be scheduled until it exits
     pdl_wait();
     const int b = threadIdx.x;
     if (b < a.B) {
@@ -314,7 +315,8 @@ __global__ void commit_apply_kernel(CommitArgs a)
 __global__ void ar_commit_kernel(int B, const int32_t *g, int64_t *step, int32_t *token_out, int32_t *anchor_io,
                                  int32_t *seq_lens, int32_t *append_out, int32_t *produced, int stride, int amax)
 {
-    pdl_trigger();
+    // no early pdl_trigger: later kernels read what this one writes before
+    // their griddepcontrol.wait, so nothing may be scheduled until it exits
     pdl_wait();
     const int b = threadIdx.x;
     if (b < B) {
@@ -333,7 +335,8 @@ __global__ void ar_commit_kernel(int B, const int32_t *g, int64_t *step, int32_t
 
 __global__ void set_lens_kernel(int32_t *seq_lens, int b, int value, int32_t *anchor_out, const int32_t *last_tok)
 {
-    pdl_trigger();
+    // no early pdl_trigger: later kernels read what this one writes before
+    // their griddepcontrol.wait, so nothing may be scheduled until it exits
     pdl_wait();
     seq_lens[b] = value;
     if (anchor_out) anchor_out[b] = *last_tok;
@@ -360,7 +363,8 @@ __global__ void pack_block_kernel(const T *ks, const T *vs, T *kd, T *vd, int K,
 
 __global__ void set_int_kernel(int32_t *p, int v)
 {
-    pdl_trigger();
+    // no early pdl_trigger: later kernels read what this one writes before
+    // their griddepcontrol.wait, so nothing may be scheduled until it exits
     pdl_wait();
     *p = v;
 }

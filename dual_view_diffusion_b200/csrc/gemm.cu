@@ -139,8 +139,14 @@ cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s)
     if (tc) {   // stream-K split: partial and flag slots per (token tile, n tile, segment)
         GemmArgs t = a;
         t.splits = t.defer > 0 ? t.defer : sk_max_segments(n_nt, a.Kd / kTileK);
-        // QKV: each head tile cut in two k halves reduced inside a 2-CTA cluster
-        t.pair = (a.epi == EPI_QKV && t.defer == 0 && (a.Kd / kTileK) % 2 == 0) ? 1 : 0;
+        // QKV: each head tile cut in 2 k segments reduced inside a 2-CTA
+        // cluster when one cluster per tile fits one wave of SMs (a function
+        // of the matrix shape, never of the token count; 3-CTA clusters
+        // measured slower on B200)
+        t.pair = 0;
+        if (a.epi == EPI_QKV && t.defer == 0)
+            for (int S = 2; S >= 2 && !t.pair; --S)
+                if (n_nt * S <= kNumSMs && a.Kd / kTileK >= S) t.pair = S;   // the matrix shape only
         const size_t slots = (size_t)n_mt * n_nt * t.splits;
         if (t.splits > 1 && (slots * kTileM * kTileN > c.gemm_part_floats || slots > (size_t)c.gemm_tickets))
             return cudaErrorInvalidValue;

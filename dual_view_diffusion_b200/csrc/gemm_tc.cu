@@ -52,10 +52,10 @@ struct TcSmem {
     alignas(1024) unsigned char w[kTcStages][kStageWBytes];
     alignas(1024) unsigned char x[kTcStages][kStageXBytes];
     float tile[kTileM][kTilePad];
-    float peer[kTileM][kTilePad];     // pair mode, rank 0: the other half's fp32 tile
-    EpiPre pre;
+    EpiPre pre;                       // (cluster mode, rank 0: pre.resid lands rank 1's tile)
+    float peer2[kTileM][kTilePad];    // cluster mode, rank 0: rank 2's tile
     alignas(8) uint64_t full[kTcStages], empty[kTcStages], tfull[2], tempty[2];
-    uint64_t peer_full, peer_empty;   // pair mode: the second half's tile landed / was consumed
+    uint64_t peer_full, peer_empty;   // cluster mode: the other ranks' tiles landed / this rank's was consumed
     uint32_t tmem_base;
     int abort;
     int s_last;
@@ -274,12 +274,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int g = blockIdx.x;
-    // pair mode: the two CTAs of a cluster hold the two k halves of the same
-    // n tiles; rank 1 hands its fp32 tile to rank 0 through distributed shared
-    // memory.  Both CTAs' barriers are initialised before either signals the
-    // other (start of the cluster barrier; its wait comes before the first
-    // remote operation).
-    const bool pair = a.pair != 0;
+    // cluster mode (a.pair = 2 or 3 CTAs per cluster): the CTAs of a cluster
+    // hold the k segments of the same n tiles; ranks 1.. hand their fp32
+    // tiles to rank 0 through distributed shared memory.  Every CTA's barriers
+    // are initialised before any signals another (start of the cluster
+    // barrier; its wait comes before the first remote operation).
+    const bool pair = a.pair > 1;
     const uint32_t crank = pair ? tc_cluster_rank() : 0u;
     if (pair) tc_cluster_arrive_relaxed();
 
@@ -323,7 +323,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                 }
             }
             if (!waited) release_deferred();
-            pdl_trigger();   // every load of this CTA is issued
+            // the next kernel may be scheduled once every load of every CTA
+            // is issued (triggering at the start measured slower: its CTAs
+            // then compete with this grid's tail for SMs)
+            pdl_trigger();
         }
         __syncwarp();   // lanes 1..31 wait for the producer lane before the block barrier
     } else if (warp == 1) {
@@ -371,7 +374,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
             const bool defer = a.defer > 0;
             if (pair) {
                 if (crank == 0) {
-                    if (et == 0) mbar_expect_tx(&sm.peer_full, (uint32_t)sizeof(sm.peer));
+                    if (et == 0) mbar_expect_tx(&sm.peer_full, (uint32_t)((a.pair - 1) * sizeof(sm.tile)));
                 } else {   // the previous tile handed over has been consumed
                     if (et == 0) good = mbar_wait(&sm.peer_empty, (local & 1) ^ 1, abort);
                     SyncEpilogue{}();
@@ -407,18 +410,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
             const int f = q * 32 + lane;             // weight row = output feature in the tile
 #pragma unroll
             for (int j = 0; j < kTileM; ++j) sm.tile[j][f] = r[j];
-            if (pair && crank == 1) {   // hand this half to rank 0
+            if (pair && crank > 0) {   // hand this segment to rank 0
                 asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
                 SyncEpilogue{}();
                 if (et == 0) {
-                    const uint32_t dst = tc_mapa(smem_u32(&sm.peer[0][0]), 0), bar = tc_mapa(smem_u32(&sm.peer_full), 0);
+                    const float *land = crank == 1 ? &sm.pre.resid[0][0] : &sm.peer2[0][0];
+                    const uint32_t dst = tc_mapa(smem_u32(land), 0), bar = tc_mapa(smem_u32(&sm.peer_full), 0);
                     asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
                                  ::"r"(dst), "r"(smem_u32(&sm.tile[0][0])), "r"((uint32_t)sizeof(sm.tile)), "r"(bar) : "memory");
                 }
                 continue;
             }
             SyncEpilogue{}();
-            if (pair) {   // rank 0: (second half) + first half, then free the landing tile
+            if (pair) {   // rank 0: rank 2 + (rank 1 + rank 0), then free the landing tiles
                 bool landed = true;
                 if (et == 0) landed = mbar_wait(&sm.peer_full, local & 1, abort);
                 SyncEpilogue{}();
@@ -427,13 +431,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                 for (int j = 0; j < kEpiVec; ++j) {
                     const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
                     float4 &o = *(float4 *)&sm.tile[m][c4];
-                    const float4 p = *(const float4 *)&sm.peer[m][c4];
+                    const float4 p = *(const float4 *)&sm.pre.resid[m][c4];
                     o.x = p.x + o.x; o.y = p.y + o.y; o.z = p.z + o.z; o.w = p.w + o.w;
+                    if (a.pair > 2) {
+                        const float4 p2 = *(const float4 *)&sm.peer2[m][c4];
+                        o.x = p2.x + o.x; o.y = p2.y + o.y; o.z = p2.z + o.z; o.w = p2.w + o.w;
+                    }
                 }
                 SyncEpilogue{}();
-                if (et == 0)
+                if (et > 0 && et < a.pair)
                     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n"
-                                 ::"r"(tc_mapa(smem_u32(&sm.peer_empty), 1)) : "memory");
+                                 ::"r"(tc_mapa(smem_u32(&sm.peer_empty), (uint32_t)et)) : "memory");
             }
             if (defer) {   // this segment of the residual update, summed later by the RMSNorm
 #pragma unroll
@@ -603,9 +611,9 @@ cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, 
     k.G = a.defer > 0 ? n_nt * a.defer : (int)std::min<long>(kNumSMs, k.P);
     if (a.defer > 0 && (k.chunks % a.defer || a.defer > kResidSlots || !a.rpart)) return cudaErrorInvalidValue;
     const size_t smem = gemm_tc_smem_bytes();
-    if (a.pair) {   // two k halves per n tile, one 2-CTA cluster per tile
-        if (a.epi != EPI_QKV || a.defer > 0 || k.chunks % 2) return cudaErrorInvalidValue;
-        k.G = 2 * n_nt;
+    if (a.pair > 1) {   // a.pair k segments per n tile, one cluster of a.pair CTAs per tile
+        if (a.epi != EPI_QKV || a.defer > 0 || a.pair > 3 || k.chunks < a.pair) return cudaErrorInvalidValue;
+        k.G = a.pair * n_nt;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(k.G);
         cfg.blockDim = dim3(kTcThreads);
@@ -615,7 +623,7 @@ cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, 
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         attr[1].id = cudaLaunchAttributeClusterDimension;
-        attr[1].val.clusterDim.x = 2;
+        attr[1].val.clusterDim.x = a.pair;
         attr[1].val.clusterDim.y = 1;
         attr[1].val.clusterDim.z = 1;
         cfg.attrs = attr;

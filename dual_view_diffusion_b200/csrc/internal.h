@@ -61,7 +61,7 @@ struct GemmArgs {
     // deferred residual (tensor-core path): the k segments of each tile are
     // written to rpart[seg][row][N] and summed into resid by the next RMSNorm
     int defer;               // segments per tile (0: add in the epilogue)
-    int pair;                // tensor-core path: each n tile cut in two k halves by a 2-CTA cluster
+    int pair;                // tensor-core path: 2 or 3 k segments per n tile, reduced inside a cluster (0: off)
     float *rpart;
     int rpart_rows;
     // EPI_SWIGLU
