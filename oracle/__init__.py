@@ -91,14 +91,21 @@ def lib():
             l.oc_residual.argtypes = [_D, _D, C.c_int, _D]
             l.oc_draft.argtypes = [P(_Cfg), P(_Model), _D, _D, C.c_int, C.c_int, C.c_int32, C.c_int,
                                    C.c_double, C.c_uint64, C.c_uint32, _I, _D, _D, _D]
+            l.oc_draft_iter.argtypes = [P(_Cfg), P(_Model), _D, _D, C.c_int, C.c_int, C.c_int32, C.c_int,
+                                        C.c_int, C.c_double, C.c_uint64, C.c_uint32, _I, _D, _D, _D]
             l.oc_verify.argtypes = [P(_Cfg), P(_Model), _D, _D, C.c_int, C.c_int, C.c_int32, _I, C.c_int,
                                     C.c_double, _I, _D, _D, _D]
             l.oc_consensus_sample.argtypes = [_D, _D, _I, _I, C.c_int, C.c_int, C.c_uint64, C.c_uint32, _I, _D]
             l.oc_generate.argtypes = [P(_Cfg), P(_Model), _I, C.c_int, C.c_int, C.c_int, C.c_double,
                                       C.c_uint64, C.c_int, _I, _I, P(C.c_int), _D, _D, _D, P(C.c_int)]
+            l.oc_generate_iter.argtypes = [P(_Cfg), P(_Model), _I, C.c_int, C.c_int, C.c_int, C.c_double,
+                                           C.c_uint64, C.c_int, C.c_int, _I, _I, P(C.c_int), _D, _D, _D,
+                                           P(C.c_int)]
             l.oc_enumerate_ar.argtypes = [P(_Cfg), P(_Model), _I, C.c_int, C.c_int, C.c_double, _D]
             l.oc_enumerate_orthrus.argtypes = [P(_Cfg), P(_Model), _I, C.c_int, C.c_int, C.c_int,
                                                C.c_double, C.c_int, _D]
+            l.oc_enumerate_orthrus_2pass.argtypes = [P(_Cfg), P(_Model), _I, C.c_int, C.c_int, C.c_int,
+                                                     C.c_double, C.c_int, _D]
             _lib = l
     return _lib
 
@@ -270,14 +277,16 @@ class Model:
             raise RuntimeError(f"oc_prefill failed: {-t}")
         return t
 
-    def draft(self, kc, vc, t, anchor, K, T=0.0, seed=0, step=0):
+    def draft(self, kc, vc, t, anchor, K, T=0.0, seed=0, step=0, iterations=1):
+        """iterations > 1: the iterative-denoising draft (oc_draft_iter)."""
         V = self.shape.vocab
         d = np.zeros(K, np.int32)
         q = np.zeros((K, V)) if T > 0 else None
         z = np.zeros((K, V))
         mg = C.c_double(np.inf)
-        rc = lib().oc_draft(C.byref(self.cfg), C.byref(self.model), _dp(kc), _dp(vc), kc.shape[1], int(t),
-                            int(anchor), int(K), float(T), seed, step, _ip(d), _dp(q), _dp(z), C.byref(mg))
+        rc = lib().oc_draft_iter(C.byref(self.cfg), C.byref(self.model), _dp(kc), _dp(vc), kc.shape[1], int(t),
+                                 int(anchor), int(K), int(iterations), float(T), seed, step, _ip(d), _dp(q),
+                                 _dp(z), C.byref(mg))
         if rc:
             raise RuntimeError(f"oc_draft failed: {rc}")
         return d, q, z, mg.value
@@ -296,9 +305,10 @@ class Model:
             raise RuntimeError(f"oc_verify failed: {rc}")
         return g, p, z, mg.value
 
-    def generate(self, prompt, K, N, T=0.0, seed=0, method="orthrus", want_cache=False):
-        """method 'orthrus' or 'ar'.  Returns a dict with tokens, n_per_cycle,
-        cycles, min_margin, t and (optionally) the committed cache."""
+    def generate(self, prompt, K, N, T=0.0, seed=0, method="orthrus", want_cache=False, iterations=1):
+        """method 'orthrus' or 'ar'; iterations = diffusion passes per draft.
+        Returns a dict with tokens, n_per_cycle, cycles, min_margin, t and
+        (optionally) the committed cache."""
         p = _i32(prompt)
         out = np.zeros(N, np.int32)
         npc = np.zeros(N, np.int32)
@@ -309,9 +319,9 @@ class Model:
         kc = vc = None
         if want_cache:
             kc, vc = self.new_cache(cap)
-        rc = lib().oc_generate(C.byref(self.cfg), C.byref(self.model), _ip(p), p.size, int(K), int(N), float(T),
-                               seed, 1 if method == "orthrus" else 0, _ip(out), _ip(npc), C.byref(cyc),
-                               C.byref(mg), _dp(kc), _dp(vc), C.byref(tt))
+        rc = lib().oc_generate_iter(C.byref(self.cfg), C.byref(self.model), _ip(p), p.size, int(K), int(N),
+                                    float(T), seed, 1 if method == "orthrus" else 0, int(iterations), _ip(out),
+                                    _ip(npc), C.byref(cyc), C.byref(mg), _dp(kc), _dp(vc), C.byref(tt))
         if rc:
             raise RuntimeError(f"oc_generate failed: {rc}")
         res = {"tokens": out, "n_per_cycle": npc[:cyc.value], "cycles": cyc.value, "min_margin": mg.value,
@@ -329,11 +339,15 @@ class Model:
             raise RuntimeError(f"oc_enumerate_ar failed: {rc}")
         return dist
 
-    def enumerate_orthrus(self, prompt, K, N, T, planted_error=False):
+    def enumerate_orthrus(self, prompt, K, N, T, planted_error=False, passes=1):
+        """passes = 1 (single-step draft) or 2 (two-pass iterative draft)."""
         p = _i32(prompt)
         dist = np.zeros(self.shape.vocab ** N)
-        rc = lib().oc_enumerate_orthrus(C.byref(self.cfg), C.byref(self.model), _ip(p), p.size, int(K), int(N),
-                                        float(T), int(bool(planted_error)), _dp(dist))
+        fn = lib().oc_enumerate_orthrus if passes == 1 else lib().oc_enumerate_orthrus_2pass
+        if passes not in (1, 2):
+            raise ValueError("passes must be 1 or 2")
+        rc = fn(C.byref(self.cfg), C.byref(self.model), _ip(p), p.size, int(K), int(N), float(T),
+                int(bool(planted_error)), _dp(dist))
         if rc:
             raise RuntimeError(f"oc_enumerate_orthrus failed: {rc}")
         return dist

@@ -366,36 +366,52 @@ int oc_residual(const double *p, const double *q, int n, double *r)
 /* ------------------------------------------------------------------------ */
 
 /* Parallel projection (§4.1 step 1): block [anchor, mask x (K-1)] at
- * positions t .. t+K-1 through the diffusion view.  Writes the K drafts; at
- * T>0 also q_probs [K][V] = softmax(w/T) when given.  logits [K][V] may be
- * NULL. */
-int oc_draft(const oc_cfg *c, const oc_model *w, double *kc, double *vc, int cap, int t,
-             int32_t anchor, int K, double T, uint64_t seed, uint32_t step,
-             int32_t *draft, double *q_probs, double *logits, double *min_margin)
+ * positions t .. t+K-1 through the diffusion view.  With n_iter > 1 the
+ * diffusion view runs again n_iter - 1 times, each time on the block
+ * [anchor, y_1 .. y_{K-1}] of the previous pass's drafts (the iterative-
+ * denoising variant the paper-notes page compares against in §5.4.2; the
+ * page gives no procedure, this is its plainest reading).  Pass s draws its
+ * Gumbel noise with purpose DRAFT | s << 8, so pass 0 is the single-step
+ * draft.  Writes the K drafts of the last pass; at T>0 also q_probs [K][V] =
+ * softmax(w/T) of the last pass when given.  logits [K][V] may be NULL. */
+int oc_draft_iter(const oc_cfg *c, const oc_model *w, double *kc, double *vc, int cap, int t,
+                  int32_t anchor, int K, int n_iter, double T, uint64_t seed, uint32_t step,
+                  int32_t *draft, double *q_probs, double *logits, double *min_margin)
 {
+    if (n_iter < 1) return OC_ERR_ARG;
     int V = c->vocab;
     int32_t *blk = malloc(sizeof(int32_t) * K);
     double *z = malloc(sizeof(double) * (size_t)K * V);
     if (!blk || !z) { free(blk); free(z); return OC_ERR_NOMEM; }
-    blk[0] = anchor;
-    for (int k = 1; k < K; ++k) blk[k] = c->mask_id;
-    int rc = oc_forward(c, w, 1, 1, blk, K, t, kc, vc, cap, z, NULL);
-    if (rc == OC_OK) {
+    int rc = OC_OK;
+    for (int s = 0; s < n_iter && rc == OC_OK; ++s) {
+        blk[0] = anchor;
+        for (int k = 1; k < K; ++k) blk[k] = s == 0 ? c->mask_id : draft[k - 1];
+        rc = oc_forward(c, w, 1, 1, blk, K, t, kc, vc, cap, z, NULL);
+        if (rc != OC_OK) break;
+        const int last = s == n_iter - 1;
         for (int k = 0; k < K; ++k) {
             const double *zk = z + (size_t)k * V;
             double mg;
             if (T > 0.0) {
-                draft[k] = oc_sample_logits(zk, V, T, seed, step, (uint32_t)k, OC_PURPOSE_DRAFT, &mg);
-                if (q_probs) oc_softmax_t(zk, V, T, q_probs + (size_t)k * V);
+                draft[k] = oc_sample_logits(zk, V, T, seed, step, (uint32_t)k, OC_PURPOSE_DRAFT | ((uint32_t)s << 8), &mg);
+                if (last && q_probs) oc_softmax_t(zk, V, T, q_probs + (size_t)k * V);
             } else {
                 draft[k] = oc_argmax(zk, V, &mg);
             }
             if (min_margin && mg < *min_margin) *min_margin = mg;
         }
-        if (logits) memcpy(logits, z, sizeof(double) * (size_t)K * V);
+        if (last && logits) memcpy(logits, z, sizeof(double) * (size_t)K * V);
     }
     free(blk); free(z);
     return rc;
+}
+
+int oc_draft(const oc_cfg *c, const oc_model *w, double *kc, double *vc, int cap, int t,
+             int32_t anchor, int K, double T, uint64_t seed, uint32_t step,
+             int32_t *draft, double *q_probs, double *logits, double *min_margin)
+{
+    return oc_draft_iter(c, w, kc, vc, cap, t, anchor, K, 1, T, seed, step, draft, q_probs, logits, min_margin);
 }
 
 /* AR verification (§4.1 step 2): block [anchor, y_1 .. y_{K-1}] through the
@@ -466,11 +482,12 @@ int oc_consensus_sample(const double *p, const double *q, const int32_t *draft, 
  * [n_layers][cap][n_kv][hd], cap = P + N + K, rows beyond the committed length
  * zeroed.  *t_out (may be NULL) receives the final committed length.
  */
-int oc_generate(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P, int K, int N,
-                double T, uint64_t seed, int method, int32_t *out, int32_t *n_per_cycle,
-                int *n_cycles, double *min_margin, double *kc_out, double *vc_out, int *t_out)
+int oc_generate_iter(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P, int K, int N,
+                     double T, uint64_t seed, int method, int n_iter, int32_t *out, int32_t *n_per_cycle,
+                     int *n_cycles, double *min_margin, double *kc_out, double *vc_out, int *t_out)
 {
-    if (!c || !w || !prompt || P < 1 || N < 1 || K < 1 || (method != 0 && method != 1)) return OC_ERR_ARG;
+    if (!c || !w || !prompt || P < 1 || N < 1 || K < 1 || (method != 0 && method != 1) || n_iter < 1)
+        return OC_ERR_ARG;
     const int V = c->vocab;
     const int cap = P + N + K;
     const size_t kn = (size_t)c->n_kv_heads * c->head_dim;
@@ -499,7 +516,8 @@ int oc_generate(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P
             if (min_margin && mg < *min_margin) *min_margin = mg;
             n = 1;
         } else {
-            rc = oc_draft(c, w, kc, vc, cap, t, anchor, K, T, seed, (uint32_t)cycles, draft, q, NULL, min_margin);
+            rc = oc_draft_iter(c, w, kc, vc, cap, t, anchor, K, n_iter, T, seed, (uint32_t)cycles, draft, q, NULL,
+                               min_margin);
             if (rc) goto done;
             rc = oc_verify(c, w, kc, vc, cap, t, anchor, draft, K, T, g, p, NULL, min_margin);
             if (rc) goto done;
@@ -528,6 +546,14 @@ int oc_generate(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P
 done:
     free(kc); free(vc); free(draft); free(g); free(emit); free(p); free(q); free(z);
     return rc;
+}
+
+int oc_generate(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P, int K, int N,
+                double T, uint64_t seed, int method, int32_t *out, int32_t *n_per_cycle,
+                int *n_cycles, double *min_margin, double *kc_out, double *vc_out, int *t_out)
+{
+    return oc_generate_iter(c, w, prompt, P, K, N, T, seed, method, 1, out, n_per_cycle, n_cycles, min_margin,
+                            kc_out, vc_out, t_out);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -690,5 +716,133 @@ int oc_enumerate_orthrus(const oc_cfg *c, const oc_model *w, const int32_t *prom
 out:
     if (lvl) for (int e = 0; e < N; ++e) free(lvl[e]);
     free(lvl); free(seq); free(blk); free(y); free(qz); free(q); free(pz); free(p); free(r);
+    return rc;
+}
+
+/*
+ * As oc_enumerate_orthrus for the two-pass draft (oc_draft_iter, n_iter = 2):
+ * first-pass drafts x drawn independently from q1_k (mask block), second-pass
+ * drafts y drawn independently from q2_k(. | x) (block [anchor, x_1 ..
+ * x_{K-1}]), acceptance with min(1, p_k(y_k) / q2_k(y_k)), correction from
+ * norm(max(0, p_j - q2_j)).  The first pass only shapes the proposal, so the
+ * law of the emitted string must still be the AR law.  Exponential in K:
+ * micro models only.
+ */
+int oc_enumerate_orthrus_2pass(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P, int K,
+                               int N, double T, int planted_error, double *dist)
+{
+    const int V = c->vocab;
+    const long total = ipow(V, N);
+    const long ntuple = ipow(V, K), nctx = ipow(V, K - 1);
+    int rc = OC_OK;
+    double **lvl = calloc(N, sizeof(double *));
+    int32_t *seq = malloc(sizeof(int32_t) * (P + N + K));
+    int32_t *blk = malloc(sizeof(int32_t) * K);
+    int32_t *x = malloc(sizeof(int32_t) * K), *y = malloc(sizeof(int32_t) * K);
+    double *z = malloc(sizeof(double) * (size_t)K * V);
+    double *q1 = malloc(sizeof(double) * (size_t)K * V), *q2 = malloc(sizeof(double) * (size_t)K * V);
+    double *pc = malloc(sizeof(double) * (size_t)nctx * K * V);   /* verify softmax per draft context */
+    double *r = malloc(sizeof(double) * V);
+    double *kc = NULL, *vc = NULL;
+    if (!lvl || !seq || !blk || !x || !y || !z || !q1 || !q2 || !pc || !r) { rc = OC_ERR_NOMEM; goto out; }
+    for (int e = 0; e < N; ++e) {
+        lvl[e] = calloc((size_t)ipow(V, e), sizeof(double));
+        if (!lvl[e]) { rc = OC_ERR_NOMEM; goto out; }
+    }
+    memset(dist, 0, sizeof(double) * (size_t)total);
+    memcpy(seq, prompt, sizeof(int32_t) * P);
+    lvl[0][0] = 1.0;
+    const int cap = P + N + K;
+    const size_t csz = (size_t)c->n_layers * cap * c->n_kv_heads * c->head_dim;
+    kc = calloc(csz, sizeof(double));
+    vc = calloc(csz, sizeof(double));
+    if (!kc || !vc) { rc = OC_ERR_NOMEM; goto out; }
+
+    for (int e = 0; e < N && rc == OC_OK; ++e) {
+        const long cnt = ipow(V, e);
+        for (long idx = 0; idx < cnt && rc == OC_OK; ++idx) {
+            const double wstate = lvl[e][idx];
+            if (wstate == 0.0) continue;
+            long rem = idx;
+            for (int i = e - 1; i >= 0; --i) { seq[P + i] = (int32_t)(rem % V); rem /= V; }
+            const int len = P + e, t = len - 1;
+            const int32_t anchor = seq[len - 1];
+            if (t > 0) rc = oc_forward(c, w, 0, 0, seq, t, 0, kc, vc, cap, NULL, NULL);
+            if (rc) break;
+            /* verify distributions for every second-pass context y_1 .. y_{K-1} */
+            for (long ctx = 0; ctx < nctx && rc == OC_OK; ++ctx) {
+                long rr = ctx;
+                blk[0] = anchor;
+                for (int k = K - 1; k >= 1; --k) { blk[k] = (int32_t)(rr % V); rr /= V; }
+                rc = oc_forward(c, w, 0, 0, blk, K, t, kc, vc, cap, z, NULL);
+                for (int k = 0; k < K && rc == OC_OK; ++k)
+                    oc_softmax_t(z + (size_t)k * V, V, T, pc + ((size_t)ctx * K + k) * V);
+            }
+            if (rc) break;
+            /* first pass */
+            blk[0] = anchor;
+            for (int k = 1; k < K; ++k) blk[k] = c->mask_id;
+            rc = oc_forward(c, w, 1, 1, blk, K, t, kc, vc, cap, z, NULL);
+            if (rc) break;
+            for (int k = 0; k < K; ++k) oc_softmax_t(z + (size_t)k * V, V, T, q1 + (size_t)k * V);
+            long prev_x = -1;
+            for (long tx = 0; tx < ntuple && rc == OC_OK; ++tx) {
+                long rr = tx;
+                for (int k = K - 1; k >= 0; --k) { x[k] = (int32_t)(rr % V); rr /= V; }
+                double wx = 1.0;
+                for (int k = 0; k < K; ++k) wx *= q1[(size_t)k * V + x[k]];
+                if (wx == 0.0) continue;
+                if (tx / V != prev_x) {           /* the second pass sees x_1 .. x_{K-1} only */
+                    blk[0] = anchor;
+                    for (int k = 1; k < K; ++k) blk[k] = x[k - 1];
+                    rc = oc_forward(c, w, 1, 1, blk, K, t, kc, vc, cap, z, NULL);
+                    if (rc) break;
+                    for (int k = 0; k < K; ++k) oc_softmax_t(z + (size_t)k * V, V, T, q2 + (size_t)k * V);
+                    prev_x = tx / V;
+                }
+                for (long ty = 0; ty < ntuple; ++ty) {
+                    long ry = ty;
+                    for (int k = K - 1; k >= 0; --k) { y[k] = (int32_t)(ry % V); ry /= V; }
+                    double wy = 1.0;
+                    for (int k = 0; k < K; ++k) wy *= q2[(size_t)k * V + y[k]];
+                    if (wy == 0.0) continue;
+                    const double *p = pc + (size_t)(ty / V) * K * V;
+                    const double wb = wstate * wx * wy;
+                    double acc = 1.0;
+                    int j;
+                    for (j = 0; j < K; ++j) {
+                        const double *pj = p + (size_t)j * V, *qj = q2 + (size_t)j * V;
+                        double a = oc_accept_prob(pj[y[j]], qj[y[j]]);
+                        double rej = acc * (1.0 - a);
+                        if (rej > 0.0) {
+                            int none;
+                            if (planted_error) { memcpy(r, pj, sizeof(double) * V); none = 0; }
+                            else none = oc_residual(pj, qj, V, r);
+                            for (int cc = 0; cc < V; ++cc) {
+                                double pr = none ? (cc == oc_argmax(pj, V, NULL) ? 1.0 : 0.0) : r[cc];
+                                if (pr == 0.0) continue;
+                                long ne = e + j + 1, nidx = idx;
+                                int lim = ne < N ? (int)ne : N;
+                                for (int i = e; i < lim; ++i) nidx = nidx * V + (i - e < j ? y[i - e] : cc);
+                                if (ne >= N) dist[nidx] += wb * rej * pr; else lvl[ne][nidx] += wb * rej * pr;
+                            }
+                        }
+                        acc *= a;
+                        if (acc == 0.0) break;
+                    }
+                    if (j == K && acc > 0.0) {
+                        long ne = e + K, nidx = idx;
+                        int lim = ne < N ? (int)ne : N;
+                        for (int i = e; i < lim; ++i) nidx = nidx * V + y[i - e];
+                        if (ne >= N) dist[nidx] += wb * acc; else lvl[ne][nidx] += wb * acc;
+                    }
+                }
+            }
+        }
+    }
+out:
+    free(kc); free(vc);
+    if (lvl) for (int e = 0; e < N; ++e) free(lvl[e]);
+    free(lvl); free(seq); free(blk); free(x); free(y); free(z); free(q1); free(q2); free(pc); free(r);
     return rc;
 }

@@ -308,3 +308,64 @@ def test_sampler_matches_ar_law_monte_carlo():
     # p-value ~1e-4 threshold via Wilson-Hilferty
     z = ((chi2 / dof) ** (1 / 3) - (1 - 2 / (9 * dof))) / math.sqrt(2 / (9 * dof))
     assert z < 3.7, (chi2, dof)
+
+
+# ---------------------------------------------------------------- iterative denoising
+# The paper-notes page (§5.4.2) compares single-step drafting with multi-step
+# iterative denoising; the iterative variant re-runs the diffusion view on
+# its own previous drafts (oc_draft_iter).
+
+def test_iterative_draft_one_pass_is_the_draft(tiny_weights, tiny_prompt):
+    m = oracle.Model(tiny_weights)
+    kc, vc = m.new_cache(64)
+    t = m.prefill(tiny_prompt, kc, vc)
+    for T, seed in ((0.0, 0), (1.0, 3)):
+        d1, q1, z1, _ = m.draft(kc, vc, t, tiny_prompt[-1], 4, T, seed, 2)
+        di, qi, zi, _ = m.draft(kc, vc, t, tiny_prompt[-1], 4, T, seed, 2, iterations=1)
+        assert np.array_equal(d1, di) and np.array_equal(z1, zi)
+
+
+def test_iterative_draft_second_pass_sees_first_drafts(tiny_weights, tiny_prompt):
+    """Pass 2 is the diffusion view on [anchor, y1_1 .. y1_{K-1}]: retyping
+    that block by hand through the plain forward gives the same logits."""
+    m = oracle.Model(tiny_weights)
+    kc, vc = m.new_cache(64)
+    t = m.prefill(tiny_prompt, kc, vc)
+    K = 4
+    d1, _, _, _ = m.draft(kc, vc, t, tiny_prompt[-1], K)
+    d2, _, z2, _ = m.draft(kc, vc, t, tiny_prompt[-1], K, iterations=2)
+    ref = m.forward(1, 1, [tiny_prompt[-1]] + list(d1[:K - 1]), t, kc.copy(), vc.copy())
+    assert np.array_equal(z2, ref)
+    assert np.array_equal(d2, ref.argmax(axis=1))
+
+
+@pytest.mark.parametrize("iterations", [2, 3])
+@pytest.mark.parametrize("K", [2, 4])
+def test_greedy_iterative_orthrus_equals_ar(tiny_weights, tiny_prompt, K, iterations):
+    """Greedy consensus keeps the AR stream whatever the drafts."""
+    m = oracle.Model(tiny_weights)
+    a = m.generate(tiny_prompt, K, 24, 0.0, 0, "ar")
+    o = m.generate(tiny_prompt, K, 24, 0.0, 0, "orthrus", iterations=iterations)
+    assert np.array_equal(a["tokens"], o["tokens"])
+    assert (o["n_per_cycle"] >= 1).all() and (o["n_per_cycle"] <= K).all()
+
+
+@pytest.mark.parametrize("T", [1.0, 0.7])
+def test_two_pass_orthrus_is_lossless_by_enumeration(T):
+    """At T>0 the two-pass draft only changes the proposal: exact enumeration
+    over both passes' draft tuples and every accept/reject branch (micro model,
+    K = 3, first 4 tokens) gives the AR law within 1e-9; the planted residual
+    mistake breaks it."""
+    w = synth.make_weights(synth.MICRO, 0)
+    m = oracle.Model(w)
+    pr = synth.make_prompt(synth.MICRO, 3, 0)
+    pa = m.enumerate_ar(pr, 4, T)
+    p2 = m.enumerate_orthrus(pr, 3, 4, T, passes=2)
+    assert abs(p2.sum() - 1) < 1e-12
+    assert 0.5 * np.abs(pa - p2).sum() < 1e-9
+    pb = m.enumerate_orthrus(pr, 3, 4, T, planted_error=True, passes=2)
+    assert 0.5 * np.abs(pa - pb).sum() > 1e-3
+    # the two-pass proposal differs from the one-pass one (the enumeration
+    # really walks the second pass): the planted mistake lands elsewhere
+    p1b = m.enumerate_orthrus(pr, 3, 4, T, planted_error=True)
+    assert 0.5 * np.abs(pb - p1b).sum() > 1e-6
