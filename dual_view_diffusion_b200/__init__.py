@@ -76,6 +76,7 @@ _SIGS = {
     "orthrus_destroy": [_P],
     "orthrus_prefill": [_P, C.POINTER(KV), _P, _I, C.POINTER(_I), _I, _P, _P],
     "orthrus_draft_block": [_P, C.POINTER(KV), _P, _I, _I, C.c_float, C.c_uint64, _P, _P, _P],
+    "orthrus_draft_block_iterative": [_P, C.POINTER(KV), _P, _I, _I, _I, C.c_float, C.c_uint64, _P, _P, _P],
     "orthrus_verify_block": [_P, C.POINTER(KV), _P, _P, _I, _I, C.c_float, _P],
     "orthrus_commit": [_P, C.POINTER(KV), _I, _I, C.c_float, C.c_uint64, _P, _P, _P, _P, _P, _P],
     "orthrus_ar_step": [_P, C.POINTER(KV), _I, C.c_float, C.c_uint64, _P, _P, _P, _P],
@@ -241,12 +242,20 @@ class Engine:
                                                         _stream()))
         return anchor
 
-    def draft_block(self, anchor, K, temperature=0.0, seed=0, step=None, out=None):
+    def draft_block(self, anchor, K, temperature=0.0, seed=0, step=None, out=None, iterations=1):
+        """iterations > 1: the iterative-denoising draft (diffusion view re-run
+        on its own previous drafts)."""
         B = anchor.numel()
         draft = out if out is not None else self.torch.empty((B, K), dtype=self.torch.int32, device=self.device)
-        _check("orthrus_draft_block", lib().orthrus_draft_block(
-            self.ctx, C.byref(self.kv), _ptr(anchor), B, K, float(temperature), seed,
-            _ptr(self.step if step is None else step), _ptr(draft), _stream()))
+        st = self.step if step is None else step
+        if iterations == 1:
+            _check("orthrus_draft_block", lib().orthrus_draft_block(
+                self.ctx, C.byref(self.kv), _ptr(anchor), B, K, float(temperature), seed, _ptr(st), _ptr(draft),
+                _stream()))
+        else:
+            _check("orthrus_draft_block_iterative", lib().orthrus_draft_block_iterative(
+                self.ctx, C.byref(self.kv), _ptr(anchor), B, K, int(iterations), float(temperature), seed, _ptr(st),
+                _ptr(draft), _stream()))
         return draft
 
     def verify_block(self, anchor, draft, K, temperature=0.0):

@@ -267,9 +267,10 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
 }
 
 static cudaError_t lm_head(Ctx &c, const void *fin, int B, int K, int lm_mode, float temperature, uint64_t seed,
-                           const int64_t *step, const int32_t *given, cudaStream_t s)
+                           const int64_t *step, const int32_t *given, cudaStream_t s, int draft_pass = 0)
 {
     GemmArgs g{};
+    g.draft_pass = draft_pass;
     g.x = fin; g.M = B * K; g.N = c.cfg.vocab; g.Kd = c.cfg.hidden; g.w[0] = c.lm_head; g.wrows[0] = c.cfg.vocab;
     g.epi = EPI_LMHEAD; g.lm = c.lm_part; g.inv_temp = temperature > 0.f ? 1.0f / temperature : 0.f;
     g.seed = seed; g.step = step; g.lm_mode = lm_mode; g.given = given; g.K = K;
@@ -418,14 +419,25 @@ orthrus_status_t orthrus_draft_block(orthrus_ctx_t *c, const orthrus_kv_t *kv, c
                                      int32_t K, float temperature, uint64_t seed, const int64_t *step, int32_t *draft,
                                      void *stream)
 {
+    return orthrus_draft_block_iterative(c, kv, anchor, batch, K, 1, temperature, seed, step, draft, stream);
+}
+
+orthrus_status_t orthrus_draft_block_iterative(orthrus_ctx_t *c, const orthrus_kv_t *kv, const int32_t *anchor,
+                                               int32_t batch, int32_t K, int32_t iterations, float temperature,
+                                               uint64_t seed, const int64_t *step, int32_t *draft, void *stream)
+{
     orthrus_status_t st = check_step(c, kv, batch, K);
     if (st != ORTHRUS_OK) return st;
-    if (!anchor || !draft || (temperature > 0.f && !step) || temperature < 0.f) return ORTHRUS_ERR_INVALID_ARG;
+    if (!anchor || !draft || (temperature > 0.f && !step) || temperature < 0.f || iterations < 1)
+        return ORTHRUS_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
-    CK(launch_embed(*c, 0, nullptr, anchor, nullptr, batch, K, s));
-    CK(forward(*c, *kv, 1, batch, K, kv->seq_lens, c->bt_rows, c->fin_draft, s));
-    CK(lm_head(*c, c->fin_draft, batch, K, 1, temperature, seed, step, nullptr, s));
-    CK(launch_lm_finalize_impl(*c, 1, batch, K, temperature, draft, nullptr, s));
+    for (int pass = 0; pass < iterations; ++pass) {
+        // pass 0: [anchor, mask x (K-1)]; later passes: [anchor, previous drafts]
+        CK(launch_embed(*c, pass == 0 ? 0 : 1, nullptr, anchor, pass == 0 ? nullptr : draft, batch, K, s));
+        CK(forward(*c, *kv, 1, batch, K, kv->seq_lens, c->bt_rows, c->fin_draft, s));
+        CK(lm_head(*c, c->fin_draft, batch, K, 1, temperature, seed, step, nullptr, s, pass));
+        CK(launch_lm_finalize_impl(*c, 1, batch, K, temperature, draft, nullptr, s));
+    }
     return ORTHRUS_OK;
 }
 

@@ -396,7 +396,7 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
                     if (v == given) zid = zv[j];
                     if (sampling) {
                         const uint32_t rr = a.lm_mode == 2 ? rng_row(b, 0) : rng_row(b, k);
-                        const uint32_t pu = a.lm_mode == 2 ? PURPOSE_AR : PURPOSE_DRAFT;
+                        const uint32_t pu = a.lm_mode == 2 ? PURPOSE_AR : (PURPOSE_DRAFT | ((uint32_t)a.draft_pass << 8));
                         best_merge(gb, Best{zv[j] * a.inv_temp + gumbel(a.seed, step, rr, (uint32_t)v, pu), v, zv[j]});
                     }
                 }

@@ -84,6 +84,7 @@ struct GemmArgs {
     uint64_t seed;
     const int64_t *step;
     int lm_mode;             // 0 verify (zid from given ids), 1 draft (Gumbel), 2 AR sample
+    int draft_pass;          // lm_mode 1: pass of an iterative draft (Gumbel purpose DRAFT | pass << 8)
     const int32_t *given;    // [M] id whose logit is wanted (verify), or null
     const float *lse_p, *lse_q;   // EPI_RESAMPLE: per (b, k) row
     const int32_t *rej_row;  // EPI_RESAMPLE: [batch] j or -1

@@ -177,6 +177,23 @@ orthrus_status_t orthrus_draft_block(orthrus_ctx_t *ctx, const orthrus_kv_t *kv,
                                      const int64_t *step, int32_t *draft, void *stream);
 
 /*
+ * Iterative-denoising draft: the multi-step variant the paper-notes page
+ * compares with single-step drafting (§5.4.2; the page gives no procedure).
+ * Pass 0 is orthrus_draft_block; each further pass s (< iterations) runs the
+ * diffusion view again on the block [anchor[b], draft[b][0] .. draft[b][K-2]]
+ * of the previous pass's drafts (same positions, same mask) and overwrites
+ * draft with its own argmaxes or samples; pass s keys its Gumbel noise with
+ * (seed, *step, row, purpose DRAFT | s << 8).  The acceptance test that
+ * follows uses the last pass's distribution, so sampled decoding stays
+ * lossless.  iterations = 1 is orthrus_draft_block exactly; iterations < 1
+ * returns ORTHRUS_ERR_INVALID_ARG.  Each pass is one diffusion forward and
+ * one LM-head pass; the cache is never written.
+ */
+orthrus_status_t orthrus_draft_block_iterative(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, const int32_t *anchor,
+                                               int32_t batch, int32_t K, int32_t iterations, float temperature,
+                                               uint64_t seed, const int64_t *step, int32_t *draft, void *stream);
+
+/*
  * AR verification (paper notes §4.1 step 2): per sequence, the block
  * [anchor, draft[0..K-2]] at positions t..t+K-1 through the AR view, causal
  * (row k sees cache rows [0, t+k]).  Its K/V are written into cache slots
