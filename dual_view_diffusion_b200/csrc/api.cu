@@ -95,6 +95,13 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
     const bool simt_attn = !(c.dtype == ORTHRUS_BF16 && c.head_dim == 128);
     const size_t o_part = take(simt_attn ? Rw * c.n_q_heads * n_splits * c.head_dim * 4 : 0);
     const size_t o_ml = take(simt_attn ? Rw * c.n_q_heads * n_splits * 8 : 0);
+    // long contexts: the tensor-core attention spreads a row group over up
+    // to kAttnMaxClusters clusters and merges them through these (one
+    // ticket per owner CTA)
+    const bool attn_x2 = !simt_attn && c.max_seq >= kAttnTwoClusterSeq;
+    const size_t o_xo = take(attn_x2 ? kAttnMaxClusters * Rw * c.n_q_heads * c.head_dim * 4 : 0);
+    const size_t o_xml = take(attn_x2 ? kAttnMaxClusters * Rw * c.n_q_heads * 8 : 0);
+    const size_t o_xc = take(attn_x2 ? Rw * c.n_kv_heads * 8 * 4 : 0);
     const size_t o_gp = take(std::max(gfloats, (size_t)1) * 4), o_gt = take((size_t)gtickets * 4);
     const int rslots = std::max(resid_defer_slots(c, c.hidden, c.n_q_heads * c.head_dim), resid_defer_slots(c, c.hidden, c.ffn));
     const size_t o_rp = take((size_t)rslots * Rw * d * 4);
@@ -112,6 +119,8 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
         x->h = (float *)P(o_h); x->a = P(o_a); x->q = P(o_q); x->attn_o = P(o_o); x->act = P(o_act);
         x->k_diff = P(o_kd); x->v_diff = P(o_vd); x->fin_draft = P(o_fd); x->fin_verify = P(o_fv); x->res_x = P(o_rx);
         x->attn_part = (float *)P(o_part); x->attn_ml = (float2 *)P(o_ml);
+        x->attn_xo = attn_x2 ? (float *)P(o_xo) : nullptr; x->attn_xml = attn_x2 ? (float2 *)P(o_xml) : nullptr;
+        x->attn_xcnt = attn_x2 ? (int *)P(o_xc) : nullptr; x->attn_xz = attn_x2 ? kAttnMaxClusters : 1;
         x->gemm_part = (float *)P(o_gp); x->gemm_part_floats = gfloats; x->gemm_ticket = (int *)P(o_gt);
         x->gemm_tickets = gtickets; x->lm_part = (LmPart *)P(o_lm);
         x->resid_part = (float *)P(o_rp);
@@ -139,6 +148,7 @@ static void rebase(Ctx *x, char *ws)
     fix(x->draft); fix(x->logq); fix(x->lse_q); fix(x->g); fix(x->logp); fix(x->lse_p); fix(x->rej_row);
     fix(x->res_tok); fix(x->any_reject); fix(x->err); fix(x->produced); fix(x->step); fix(x->n_buf);
     fix(x->tok_buf); fix(x->anchor_buf);
+    if (x->attn_xz > 1) { fix(x->attn_xo); fix(x->attn_xml); fix(x->attn_xcnt); }
 }
 
 // TMA maps for the tensor-core GEMM: every weight matrix (128-row boxes;
@@ -230,6 +240,8 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
         at.kv = kv_view(kv); at.layer = l; at.seq_lens = pos0; at.bt_rows = bt_rows;
         at.B = B; at.K = K; at.n_q = f.n_q_heads; at.n_kv = f.n_kv_heads; at.hd = hd; at.mode = view;
         at.split_tokens = f.split_tokens; at.n_splits = c.n_splits; at.part = c.attn_part; at.ml = c.attn_ml;
+        at.xo = c.attn_xo; at.xml = c.attn_xml; at.xcnt = c.attn_xcnt; at.xrows = c.Rw * f.n_q_heads;
+        at.xz = c.attn_xz;
         at.err = c.err;
         {
             ProbeScope ps(c, 1, l, view, s);
@@ -594,6 +606,8 @@ orthrus_status_t orthrus_dual_view_attention(orthrus_ctx_t *c, const orthrus_kv_
     at.seq_lens = kv->seq_lens; at.bt_rows = c->bt_rows; at.B = batch; at.K = K; at.n_q = f.n_q_heads;
     at.n_kv = f.n_kv_heads; at.hd = f.head_dim; at.mode = mode; at.split_tokens = f.split_tokens;
     at.n_splits = c->n_splits; at.part = c->attn_part; at.ml = c->attn_ml; at.err = c->err;
+    at.xo = c->attn_xo; at.xml = c->attn_xml; at.xcnt = c->attn_xcnt; at.xrows = c->Rw * f.n_q_heads;
+    at.xz = c->attn_xz;
     CK(launch_attention(*c, at, s, batch * K));
     return ORTHRUS_OK;
 }

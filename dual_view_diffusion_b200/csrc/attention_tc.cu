@@ -5,15 +5,22 @@
 // K/V tile staged in shared memory serves all of them (paper notes §2.2-2.3:
 // both views read the one AR cache).  The keys are cut into splits aligned to
 // absolute positions; CTA r of the cluster takes splits r, r + C, ... and, per
-// 64-key tile:
+// 128-key tile:
 //
-//   S = Q K^T       tcgen05.mma, M 128 x N 64 x K 128, into TMEM
+//   S = Q K^T       tcgen05.mma, M 128 x N 128 x K 128 (A = Q, kept in TMEM
+//                   for the whole kernel), into TMEM
 //   softmax         each softmax thread owns one query row (= TMEM lane): it
-//                   reads its 64 scores with tcgen05.ld, applies the view's
-//                   mask, updates its running max / sum in log2 units, and
-//                   writes the bf16 probabilities P (128-byte swizzled) to
-//                   shared memory
-//   O += P V        tcgen05.mma, M 128 x N 128 x K 64, into a TMEM accumulator
+//                   reads its 128 scores with tcgen05.ld (which frees S for
+//                   the next tile), applies the view's mask, updates its
+//                   running max / sum in log2 units, and writes the bf16
+//                   probabilities P back to TMEM
+//   O += P V        tcgen05.mma, M 128 x N 128 x K 128 (A = P from TMEM), into
+//                   a TMEM accumulator
+//
+// A tcgen05.mma instruction costs the tensor pipe about the same time for any
+// N up to 128 (measured on B200: ~130 SM cycles each for M 128, K 16), so the
+// tile is as wide as TMEM allows: 16 instructions per 128 keys, against 24
+// for two 64-key tiles.
 //
 // O is rescaled in TMEM only when a warp's running max moved (a factor of
 // exactly 1 elsewhere, so skipping it changes no bit).  K tiles come from
@@ -23,8 +30,12 @@
 // are merged through distributed shared memory; nothing goes to global memory
 // but the output rows.
 //
-// Roles: warp 0 TMA producer, warp 1 MMA issuer (one thread each), warps 2..5
-// softmax and combine.  All mbarrier waits are bounded.
+// Roles: warp 0 K producer and warp 2 V producer (TMA, one issuing thread
+// each, separate rings: a K tile is free once S is computed, a V tile only
+// after its P.V), warp 1 MMA issuer (one thread), warps 4..11 softmax (two
+// warpgroups taking alternate tiles) and combine.  A tile's keys are two
+// 64-key subtiles, each from its own page.  All mbarrier waits are
+// bounded.
 #include <cuda.h>
 #include <string.h>
 
@@ -35,34 +46,44 @@
 
 namespace orthrus {
 
-constexpr int kAtStages = 4;
+constexpr int kAtKStages = 3;   // K tiles are released as soon as S = Q K^T is done
+constexpr int kAtVStages = 3;   // V tiles live until their P.V
 constexpr float kRescaleSlack = 8.0f;   // log2 units a row's max may grow before O is rescaled
 constexpr int kAtMaxCluster = 8;        // portable cluster size
+constexpr int kAtMaxZ = 4;              // clusters per row group (long contexts)
+constexpr int kAtZCluster = 4;          // their size
 constexpr int kAtPreWait = 2;           // cache tiles requested before waiting for the predecessor
-constexpr int kAtThreads = 320;   // producer warp, MMA warp, two softmax warpgroups
+constexpr int kAtThreads = 384;   // producer warpgroup (K, MMA, V, spare), two softmax warpgroups
+constexpr int kAtVWarp = 2;       // the V producer warp
+constexpr int kAtSoftWarp0 = 4;   // first softmax warp
 constexpr int kAtRows = 128;
-constexpr int kAtKeys = 64;
+constexpr int kAtKeys = 128;      // keys per tile
+constexpr int kAtSub = 64;        // keys per subtile (one page box)
 constexpr long long kAtSpinCycles = 4000000000LL;   // ~2 s at the B200 SM clock
 
 struct AtSmem {
-    alignas(1024) unsigned char q[2][kAtRows * 128];              // Q dims 0-63 / 64-127, 16 KiB each
-    alignas(1024) unsigned char k[kAtStages][2][kAtKeys * 128];   // K tile halves, 8 KiB each
-    alignas(1024) unsigned char v[kAtStages][128 * 128];          // V^T tile [128 dims][64 keys], 16 KiB
-    alignas(1024) unsigned char p[2][kAtRows * 128];              // P [128 rows][64 keys], 16 KiB, per accumulator
-    alignas(8) uint64_t q_full, full[kAtStages], empty[kAtStages], s_full[2], p_full[2], o_done[2];
+    alignas(1024) unsigned char k[kAtKStages][2][kAtKeys * 128];  // K tile [128 keys] x dims 0-63 / 64-127, 16 KiB each
+    alignas(1024) unsigned char v[kAtVStages][2][128 * 128];      // V^T subtiles [128 dims][64 keys], 16 KiB each
+    alignas(8) uint64_t q_ready, kfull[kAtKStages], kempty[kAtKStages], vfull[kAtVStages], vempty[kAtVStages];
+    uint64_t s_full[2], s_free, p_full[2], o_done[2];
     float2 xml[2][kAtRows];   // (m, l) of each accumulator, per row
     uint32_t tmem_base;
     int abort;
+    int xticket;   // this cluster's arrival order at the cross-cluster combine
 };
-// Once the last P.V is done, q..v (160 KiB) is reused for the combine: the
+// Once the last P.V is done, k..v (192 KiB) is reused for the combine: the
 // CTA's merged rows [128][128] fp32 (16-byte chunk ch of row r at ch ^ (r & 31))
 // and (m, l) per row, read by the other CTAs of the cluster.
 constexpr uint32_t kStageO = 0, kStageMl = 64 * 1024;
-static_assert(kStageMl + kAtRows * 8 <= 2 * 16384 + kAtStages * 32768, "combine area");
+static_assert(kStageMl + kAtRows * 8 <= kAtKStages * 32768 + kAtVStages * 32768, "combine area");
 
-// TMEM columns: two O accumulators (even / odd tiles) [0, 256), S double
-// buffer [256, 384)
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemCols = 512;
+// TMEM columns: two O accumulators (even / odd tiles) [0, 256), S [256, 384)
+// (one buffer: the softmax frees it as soon as it has read its scores), P
+// [384, 448) and Q [448, 512) (bf16 pairs: the A operands of P.V and of
+// Q K^T read straight from TMEM).  One P buffer suffices: P of tile i is
+// written once the P.V of tile i-1 is done, which is no later than the
+// softmax of tile i needs it.
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 384, kTmemQ = 448, kTmemCols = 512;
 
 __device__ __forceinline__ void at_mbar_init(uint64_t *b, uint32_t n)
 {
@@ -120,6 +141,12 @@ __device__ __forceinline__ void at_mma(uint32_t d, uint64_t a, uint64_t b, uint3
     asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
                  ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
 }
+// D (TMEM) += A (TMEM) * B (shared memory descriptor)
+__device__ __forceinline__ void at_mma_ta(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc)
+{
+    asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
+                 ::"r"(d), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
 __device__ __forceinline__ void at_commit(uint64_t *b)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(b)) : "memory");
@@ -144,11 +171,16 @@ __device__ __forceinline__ void at_fence_after() { asm volatile("tcgen05.fence::
                    "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), \
                    "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), \
                    "r"(r[31]) : "memory")
+#define AT_ST16(taddr, r)                                                                                         \
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15," \
+                 "%16};\n"                                                                                          \
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),        \
+                   "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),    \
+                   "r"(r[15]) : "memory")
 __device__ __forceinline__ void at_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void at_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
 struct AtMaps {
-    CUtensorMap q;    // 4-D (dim, head in group, kv head, block row), box {64, g, 1, rows/g}
     CUtensorMap kc;   // 2-D cache K rows [slot rows][128], box {64, 64}
     CUtensorMap vc;   // 2-D cache V^T rows [dim rows][page_size], box {64, 128}
     CUtensorMap kb;   // 2-D transient K [rows][128], box {64, 64}
@@ -241,6 +273,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     }
     constexpr int rpc = kAtRows / C;   // rows owned per CTA
     const int r = (int)cluster_rank();
+    // Z clusters of C CTAs share the (sequence, KV head, row group): CTA ci
+    // of the Ctot takes splits ci, ci + Ctot, ...
+    const int Z = a.xz, zc = (int)blockIdx.z / C, ci = zc * C + r, Ctot = C * Z;
     const int n_total = n_split_grid + (a.mode == 1 ? 1 : 0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
@@ -248,28 +283,38 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     // trigger their dependents early (commit, set-length, row-map kernels),
     // so every kernel after them in the stream starts after they completed:
     // they may be read before griddepcontrol.wait
+    if (threadIdx.x == 0) {   // the first TMA of each map need not wait for its descriptor
+        asm volatile("prefetch.tensormap [%0];\n" ::"l"((uint64_t)&maps.kc) : "memory");
+        asm volatile("prefetch.tensormap [%0];\n" ::"l"((uint64_t)&maps.vc) : "memory");
+        if (a.mode == 1) {
+            asm volatile("prefetch.tensormap [%0];\n" ::"l"((uint64_t)&maps.kb) : "memory");
+            asm volatile("prefetch.tensormap [%0];\n" ::"l"((uint64_t)&maps.vb) : "memory");
+        }
+    }
     const int t = a.seq_lens[b];
     const int bt_row = a.bt_rows[b];
-    // Flat tile f of this CTA is tile f % tps of split r + C * (f / tps) for
-    // every cache tile (only the last cache split can be short, and only
-    // block tiles follow it).  Warp 0 looks up the pages of 32 flat tiles at
-    // a time, one per lane.
-    const int tps = a.split_tokens / kAtKeys;
+    // Flat subtile f of this CTA is subtile f % tps of split ci + Ctot * (f / tps)
+    // for every cache subtile (only the last cache split can be short, and
+    // only block tiles follow it).  Each producer warp looks up the pages of
+    // 32 flat subtiles at a time, one per lane.
+    const int tps = a.split_tokens / kAtSub;
     const int cache_lim = a.mode == 0 ? t + a.K : t;
     auto lookup = [&](int f) {
-        const int sl = r + C * (f / tps);
-        const int key = sl * a.split_tokens + (f % tps) * kAtKeys;
+        const int sl = ci + Ctot * (f / tps);
+        const int key = sl * a.split_tokens + (f % tps) * kAtSub;
         if (sl >= n_split_grid || key >= cache_lim) return 0;
         const int pidx = key / a.kv.page_size;
         int page = (pidx < a.kv.max_pages) ? a.kv.block_table[(size_t)bt_row * a.kv.max_pages + pidx] : -1;
         if (page < 0 || page >= a.kv.num_pages) { raise_err(a.err, ORTHRUS_DEVERR_CAPACITY); page = 0; }
         return page;
     };
-    int pg = warp == 0 ? lookup(lane) : 0;
+    int pg = (warp == 0 || warp == kAtVWarp) ? lookup(lane) : 0;
 
     if (threadIdx.x == 0) {
-        at_mbar_init(&sm.q_full, 1);
-        for (int i = 0; i < kAtStages; ++i) { at_mbar_init(&sm.full[i], 1); at_mbar_init(&sm.empty[i], 1); }
+        at_mbar_init(&sm.q_ready, 128);
+        for (int i = 0; i < kAtKStages; ++i) { at_mbar_init(&sm.kfull[i], 1); at_mbar_init(&sm.kempty[i], 1); }
+        for (int i = 0; i < kAtVStages; ++i) { at_mbar_init(&sm.vfull[i], 1); at_mbar_init(&sm.vempty[i], 1); }
+        at_mbar_init(&sm.s_free, 128);
         for (int i = 0; i < 2; ++i) {
             at_mbar_init(&sm.s_full[i], 1);
             at_mbar_init(&sm.p_full[i], 128);
@@ -288,56 +333,88 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     at_fence_after();
     const uint32_t tmem = sm.tmem_base;
     int my_tiles = 0;
-    for (int s = r; s < n_total; s += C) my_tiles += at_split(a, s, n_split_grid, t).ntiles;
+    for (int s = ci; s < n_total; s += Ctot) my_tiles += at_split(a, s, n_split_grid, t).ntiles;
 
     uint32_t jj = 0;
     bool ok = true;
     const int q4 = warp & 3, row = q4 * 32 + lane;   // softmax threads: query row = TMEM lane
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
-    if (warp == 0) {   // ------------------------------------------------------ producer
-        // all 32 lanes walk the tiles together (page lookups); lane 0 issues.
-        // Up to kAtPreWait cache tiles below t (which the predecessor cannot
-        // be writing) are requested before waiting for it; Q right after.
-        uint32_t stage = 0, phase = 0;
+    if (warp == 0 || warp == kAtVWarp) {   // ------------------------ K / V producers
+        // Two producer warps, one per ring, so V tiles run as far ahead as
+        // their deeper ring allows instead of trailing the K issue.  All 32
+        // lanes of a producer walk the subtiles together (page lookups); lane
+        // 0 issues.  A tile is two 64-key subtiles; where the second lies past
+        // the split's end the first is loaded again in its place (finite data,
+        // masked out by the softmax).  Up to kAtPreWait cache tiles below t
+        // (which the predecessor cannot be writing) are requested before
+        // waiting for it.
+        const bool kprod = warp == 0;
+        uint32_t ks = 0, kph = 0, vs = 0, vph = 0;
         bool waited = false, stop = false;
         auto ensure_wait = [&]() {
             if (waited) return;
             pdl_wait();
             waited = true;
-            if (my_tiles == 0) return;   // nothing will consume Q
-            const uint32_t qbytes = 2u * 128u * (uint32_t)(g * min(a.K, ksub));   // the map's box
-            at_expect(&sm.q_full, qbytes);
-            at_tma4(sm.q[0], &maps.q, 0, 0, kvh, b * a.K + k_lo, &sm.q_full);
-            at_tma4(sm.q[1], &maps.q, 64, 0, kvh, b * a.K + k_lo, &sm.q_full);
         };
-        int f = 0;
-        for (int s = r; s < n_total && !stop; s += C) {
+        int f = 0, ft = 0;   // cache subtiles, tiles walked so far
+        for (int s = ci; s < n_total && !stop; s += Ctot) {
             const AtSplit sp = at_split(a, s, n_split_grid, t);
-            for (int j = 0; j < sp.ntiles; ++j, ++f) {
-                if (f > 0 && (f & 31) == 0) pg = lookup(f + lane);
-                const int page = __shfl_sync(0xffffffffu, pg, f & 31);
+            for (int j = 0; j < sp.ntiles; ++j, ++ft) {
+                const int p0 = sp.key0 + j * kAtKeys;
+                const bool two = p0 + kAtSub < sp.key1;
+                int page[2] = {0, 0};
+                if (!sp.block) {
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        if (u == 1 && !two) break;
+                        if (f > 0 && (f & 31) == 0) pg = lookup(f + lane);
+                        page[u] = __shfl_sync(0xffffffffu, pg, f & 31);
+                        ++f;
+                    }
+                }
                 int go = 1;
                 if (lane == 0) {
-                    const int p0 = sp.key0 + j * kAtKeys;
-                    if (sp.block || p0 + kAtKeys > t || f >= kAtPreWait) ensure_wait();
-                    if (!at_wait(&sm.empty[stage], phase ^ 1, abort)) {
-                        go = 0;
-                    } else {
-                        at_expect(&sm.full[stage], 2u * 8192u + 16384u);
-                        if (sp.block) {
-                            const int krow = (a.blk_layer * a.bmax + b) * a.n_kv + kvh;
-                            at_tma2(sm.k[stage][0], &maps.kb, 0, krow * a.kp + j * kAtKeys, &sm.full[stage]);
-                            at_tma2(sm.k[stage][1], &maps.kb, 64, krow * a.kp + j * kAtKeys, &sm.full[stage]);
-                            at_tma2(sm.v[stage], &maps.vb, j * kAtKeys, krow * 128, &sm.full[stage]);
+                    if (sp.block || min(p0 + kAtKeys, sp.key1) > t || ft >= kAtPreWait) ensure_wait();
+                    const int krow = (a.blk_layer * a.bmax + b) * a.n_kv + kvh;
+                    int off[2], hrow[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int uu = (u == 1 && two) ? 1 : 0;
+                        off[u] = (p0 + uu * kAtSub) % a.kv.page_size;
+                        hrow[u] = (a.layer * a.kv.num_pages + page[uu]) * a.n_kv + kvh;
+                    }
+                    const int brow0 = j * kAtKeys, brow1 = two ? brow0 + kAtSub : brow0;
+                    if (kprod) {
+                        if (!at_wait(&sm.kempty[ks], kph ^ 1, abort)) {
+                            go = 0;
                         } else {
-                            const int off = p0 % a.kv.page_size;
-                            const int hrow = (a.layer * a.kv.num_pages + page) * a.n_kv + kvh;
-                            at_tma2(sm.k[stage][0], &maps.kc, 0, hrow * a.kv.page_size + off, &sm.full[stage]);
-                            at_tma2(sm.k[stage][1], &maps.kc, 64, hrow * a.kv.page_size + off, &sm.full[stage]);
-                            at_tma2(sm.v[stage], &maps.vc, off, hrow * 128, &sm.full[stage]);
+                            at_expect(&sm.kfull[ks], 4u * 8192u);
+#pragma unroll
+                            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                                for (int hh = 0; hh < 2; ++hh) {
+                                    if (sp.block)
+                                        at_tma2(sm.k[ks][hh] + u * 8192, &maps.kb, hh * 64, krow * a.kp + (u ? brow1 : brow0),
+                                                &sm.kfull[ks]);
+                                    else
+                                        at_tma2(sm.k[ks][hh] + u * 8192, &maps.kc, hh * 64, hrow[u] * a.kv.page_size + off[u],
+                                                &sm.kfull[ks]);
+                                }
+                            if (++ks == kAtKStages) { ks = 0; kph ^= 1; }
                         }
-                        if (++stage == kAtStages) { stage = 0; phase ^= 1; }
+                    } else {
+                        if (!at_wait(&sm.vempty[vs], vph ^ 1, abort)) {
+                            go = 0;
+                        } else {
+                            at_expect(&sm.vfull[vs], 2u * 16384u);
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                if (sp.block) at_tma2(sm.v[vs][u], &maps.vb, u ? brow1 : brow0, krow * 128, &sm.vfull[vs]);
+                                else at_tma2(sm.v[vs][u], &maps.vc, off[u], hrow[u] * 128, &sm.vfull[vs]);
+                            }
+                            if (++vs == kAtVStages) { vs = 0; vph ^= 1; }
+                        }
                     }
                 }
                 if (!__shfl_sync(0xffffffffu, go, 0)) { stop = true; break; }
@@ -348,49 +425,49 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     } else if (warp == 1) {
         pdl_wait();
         if (lane == 0 && my_tiles > 0) {   // ---------------------------------- MMA issuer
-            // S of tile i is issued before P.V of tile i-1; tile i uses S
-            // buffer, P buffer and O accumulator i & 1
-            bool good = at_wait(&sm.q_full, 0, abort);
-            uint32_t stage = 0, phase = 0, i = 0;
-            uint32_t pv_stage = 0;          // stage of the tile waiting for its P.V
+            // S of tile i is issued (once the softmax has read S of tile i-1)
+            // before P.V of tile i-1; tile i accumulates into O_(i & 1)
+            bool good = at_wait(&sm.q_ready, 0, abort);
+            uint32_t ks = 0, kph = 0, vs = 0, vph = 0, i = 0;
             bool pv_pending = false;
-            const uint32_t id_s = idesc_n(kAtKeys), id_o = idesc_n(128);
-            auto issue_pv = [&](uint32_t pi) {   // P.V of tile pi (waits for its P)
+            const uint32_t id = idesc_n(128);
+            auto issue_pv = [&](uint32_t pi) {   // P.V of tile pi (waits for its P and its V tile)
                 const uint32_t h = pi & 1;
                 if (!at_wait(&sm.p_full[h], (pi >> 1) & 1, abort)) return false;
+                if (!at_wait(&sm.vfull[vs], vph, abort)) return false;
                 at_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    at_mma(tmem + kTmemO + h * 128, at_desc(sm.p[h]) + 2 * kk, at_desc(sm.v[pv_stage]) + 2 * kk, id_o,
-                           (pi >= 2 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 8; ++kk)   // A = P_h in TMEM, 16 keys (8 columns) per step
+                    at_mma_ta(tmem + kTmemO + h * 128, tmem + kTmemP + kk * 8,
+                              at_desc(sm.v[vs][kk >> 2]) + 2 * (kk & 3), id, (pi >= 2 || kk > 0) ? 1u : 0u);
                 at_commit(&sm.o_done[h]);
-                at_commit(&sm.empty[pv_stage]);
+                at_commit(&sm.vempty[vs]);
+                if (++vs == kAtVStages) { vs = 0; vph ^= 1; }
                 return true;
             };
-            for (int s = r; s < n_total && good; s += C) {
+            for (int s = ci; s < n_total && good; s += Ctot) {
                 const AtSplit sp = at_split(a, s, n_split_grid, t);
                 for (int j = 0; j < sp.ntiles && good; ++j, ++i) {
-                    if (!at_wait(&sm.full[stage], phase, abort)) { good = false; break; }
+                    if (!at_wait(&sm.kfull[ks], kph, abort)) { good = false; break; }
+                    if (i > 0 && !at_wait(&sm.s_free, (i - 1) & 1, abort)) { good = false; break; }
                     at_fence_after();
-                    const uint32_t sbuf = kTmemS + (i & 1) * kAtKeys;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const int h = kk >> 2, o = 2 * (kk & 3);
-                        at_mma(tmem + sbuf, at_desc(sm.q[h]) + o, at_desc(sm.k[stage][h]) + o, id_s, kk > 0 ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < 8; ++kk)   // A = Q in TMEM, 16 dims (8 columns) per step
+                        at_mma_ta(tmem + kTmemS, tmem + kTmemQ + kk * 8, at_desc(sm.k[ks][kk >> 2]) + 2 * (kk & 3), id,
+                                  kk > 0 ? 1u : 0u);
                     at_commit(&sm.s_full[i & 1]);
+                    at_commit(&sm.kempty[ks]);
+                    if (++ks == kAtKStages) { ks = 0; kph ^= 1; }
                     if (pv_pending && !issue_pv(i - 1)) { good = false; break; }
                     pv_pending = true;
-                    pv_stage = stage;
-                    if (++stage == kAtStages) { stage = 0; phase ^= 1; }
                 }
             }
             if (good && pv_pending) issue_pv(i - 1);
         }
         __syncwarp();
-    } else {   // ------------------------------------------------- softmax, warpgroup h: tiles jj with jj & 1 == h
+    } else if (warp >= kAtSoftWarp0) {   // ---------------------------- softmax, warpgroup h: tiles jj with jj & 1 == h
         pdl_wait();
-        const int h = (warp - 2) >> 2;
+        const int h = (warp - kAtSoftWarp0) >> 2;
         const int rr = k_lo * g + row;                            // row within the sequence's K*g rows
         const int kblk = rr / g;
         const float scale = 1.4426950408889634f / sqrtf(128.f);
@@ -399,7 +476,27 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
         // kRescaleSlack: the result is the same softmax, P stays <= 2^slack
         float m_use = -INFINITY, l_run = 0.f;
         int last = -1;   // this warpgroup's last tile
-        for (int s = r; s < n_total && ok; s += C) {
+        if (h == 0) {   // Q row -> TMEM lane row (bf16 pairs); rows past the block are zero
+            uint32_t qr[64];
+            if (kblk < k_hi) {
+                const uint4 *src = (const uint4 *)((const bf16 *)a.q +
+                                                   ((size_t)(b * a.K + kblk) * a.n_q + kvh * g + rr % g) * 128);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const uint4 v = src[c];
+                    qr[4 * c] = v.x; qr[4 * c + 1] = v.y; qr[4 * c + 2] = v.z; qr[4 * c + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) qr[c] = 0u;
+            }
+            AT_ST32(tmem + lane_off + kTmemQ, qr);
+            AT_ST32(tmem + lane_off + kTmemQ + 32, (qr + 32));
+            at_wait_st();
+            at_fence_before();
+            at_arrive(&sm.q_ready);
+        }
+        for (int s = ci; s < n_total && ok; s += Ctot) {
             const AtSplit sp = at_split(a, s, n_split_grid, t);
             const int lim = min(sp.key1, sp.block ? sp.key1 : (a.mode == 0 ? t + kblk + 1 : sp.key1));
             for (int j = 0; j < sp.ntiles; ++j, ++jj) {
@@ -408,20 +505,21 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
                 ok = at_wait(&sm.s_full[h], (jj >> 1) & 1, abort);
                 if (!ok) break;
                 at_fence_after();
-                uint32_t sr[64];
-                const uint32_t sbuf = kTmemS + h * kAtKeys;
-                AT_LD32(tmem + lane_off + sbuf, sr);
-                AT_LD32(tmem + lane_off + sbuf + 32, (sr + 32));
+                uint32_t sr[128];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) AT_LD32(tmem + lane_off + kTmemS + q * 32, (sr + q * 32));
                 at_wait_ld();
+                at_fence_before();
+                at_arrive(&sm.s_free);   // S may be overwritten by the next tile
                 const int vis = lim - (sp.key0 + j * kAtKeys);   // keys of this tile the row sees
                 if (vis < kAtKeys) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
+                    for (int c = 0; c < kAtKeys; ++c)
                         if (c >= vis) sr[c] = __float_as_uint(-INFINITY);
                 }
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int c = 0; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(sr[c]));
+                for (int c = 0; c < kAtKeys; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(sr[c]));
                 const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale;
                 float alpha = 1.0f;
                 if (tmax > m_use + kRescaleSlack || (m_use == -INFINITY && tmax > -INFINITY)) {
@@ -429,39 +527,38 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
                     m_use = tmax;
                 }
                 const float nmu = m_use == -INFINITY ? 0.f : -m_use;
+                // P row: 64 bf16 pairs (the P.V A operand), computed while the
+                // P.V of tile jj-1 may still be reading P
                 float rs[4] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t pk[32];
+                uint32_t pk[kAtKeys / 2];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
+                for (int c = 0; c < kAtKeys / 2; ++c) {
                     const float p0v = ex2(fmaf(__uint_as_float(sr[2 * c]), scale, nmu));
                     const float p1v = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), scale, nmu));
                     rs[c & 3] += p0v + p1v;
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0v, p1v);
                     pk[c] = *(const uint32_t *)&h2;
                 }
-                if (jj >= 2) {   // P.V of tile jj-2 done: O_h and P_h are free
-                    ok = at_wait(&sm.o_done[h], ((jj - 2) >> 1) & 1, abort);
+                if (jj >= 1) {   // P.V of tile jj-1 done (so that of tile jj-2 too): P and O_h are free
+                    ok = at_wait(&sm.o_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, abort);
                     if (!ok) break;
                     at_fence_after();
-                    if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+                }
+                // P row -> TMEM lane row
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t orr[32];
-                            AT_LD32(tmem + lane_off + kTmemO + h * 128 + q * 32, orr);
-                            at_wait_ld();
+                for (int q = 0; q < 4; ++q) AT_ST16(tmem + lane_off + kTmemP + q * 16, (pk + 16 * q));
+                if (jj >= 2 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-                            AT_ST32(tmem + lane_off + kTmemO + h * 128 + q * 32, orr);
-                        }
-                        at_wait_st();
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t orr[32];
+                        AT_LD32(tmem + lane_off + kTmemO + h * 128 + q * 32, orr);
+                        at_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+                        AT_ST32(tmem + lane_off + kTmemO + h * 128 + q * 32, orr);
                     }
                 }
-                // P row -> shared memory, 128-byte swizzle (16-byte chunk c at c ^ (row & 7))
-                unsigned char *prow = sm.p[h] + row * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *(uint4 *)(prow + ((c ^ (row & 7)) << 4)) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                at_wait_st();
                 at_fence_before();
                 at_arrive(&sm.p_full[h]);
                 l_run = l_run * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
@@ -475,10 +572,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     }
 
     // ------------------------------------------------------------------ combine
-    unsigned char *area = sm.q[0];
+    unsigned char *area = sm.k[0][0];
     const uint32_t area_u = smem_u32(area);
-    if (warp >= 2) {
-        const int h = (warp - 2) >> 2;
+    if (warp >= kAtSoftWarp0) {
+        const int h = (warp - kAtSoftWarp0) >> 2;
         asm volatile("bar.sync 1, 256;\n" ::: "memory");   // both warpgroups: every P.V is done
         // merge the two accumulators into (O, m, l) of this row -> staging (the
         // K/V ring, Q and P are no longer read); warpgroup h takes dims
@@ -515,10 +612,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     // every CTA's merged rows are in its shared memory (release / acquire)
     cluster_arrive();
     cluster_wait();
-    if (warp >= 2) {   // ----------------------------------- owner: rows [r*rpc, (r+1)*rpc), pulled from every CTA
+    if (warp >= kAtSoftWarp0) {   // ---------------- owner: rows [r*rpc, (r+1)*rpc), pulled from every CTA
         constexpr int tpr = 256 / rpc;            // threads per owned row: chunks cc, cc + tpr, ...
         constexpr int cpt = 32 / tpr;             // chunks per thread
-        const int et = threadIdx.x - 64;
+        const int et = threadIdx.x - 32 * kAtSoftWarp0;
         const int rl = et / tpr, cc = et % tpr;
         const int orow = r * rpc + rl;
         uint32_t peer[C];
@@ -546,22 +643,88 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
             L += wc[c] * ml[c].y;
         }
         const int rrow = k_lo * g + orow, k = rrow / g, jh = rrow % g;
-        if (!*abort && orow < (k_hi - k_lo) * g && L > 0.f) {
-            const float inv = 1.0f / L;
-            bf16 *o = (bf16 *)a.out + ((size_t)(b * a.K + k) * a.n_q + kvh * g + jh) * 128;
+        const bool vrow = orow < (k_hi - k_lo) * g;
+        float4 acc[cpt];   // sum over the cluster's CTAs, in rank order, relative to Mx
 #pragma unroll
-            for (int i = 0; i < cpt; ++i) {
-                const int ch = cc + i * tpr;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < cpt; ++i) {
+            acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int c = 0; c < C; ++c) {
-                    if (wc[c] == 0.f) continue;
-                    acc.x = fmaf(wc[c], v[i][c].x, acc.x); acc.y = fmaf(wc[c], v[i][c].y, acc.y);
-                    acc.z = fmaf(wc[c], v[i][c].z, acc.z); acc.w = fmaf(wc[c], v[i][c].w, acc.w);
+            for (int c = 0; c < C; ++c) {
+                if (wc[c] == 0.f) continue;
+                acc[i].x = fmaf(wc[c], v[i][c].x, acc[i].x); acc[i].y = fmaf(wc[c], v[i][c].y, acc[i].y);
+                acc[i].z = fmaf(wc[c], v[i][c].z, acc[i].z); acc[i].w = fmaf(wc[c], v[i][c].w, acc[i].w);
+            }
+        }
+        const size_t orow_g = (size_t)(b * a.K + k) * a.n_q + kvh * g + jh;   // (token, query head) of the row
+        bf16 *o = (bf16 *)a.out + orow_g * 128;
+        auto store = [&](int i, float4 y, float inv) {
+            const int ch = cc + i * tpr;
+            const __nv_bfloat162 lo2 = __floats2bfloat162_rn(y.x * inv, y.y * inv);
+            const __nv_bfloat162 hi2 = __floats2bfloat162_rn(y.z * inv, y.w * inv);
+            *(uint2 *)(o + ch * 4) = make_uint2(*(const uint32_t *)&lo2, *(const uint32_t *)&hi2);
+        };
+        if (Z == 1) {
+            if (!*abort && vrow && L > 0.f) {
+                const float inv = 1.0f / L;
+#pragma unroll
+                for (int i = 0; i < cpt; ++i) store(i, acc[i], inv);
+            }
+        } else {
+            // Z clusters: each leaves its (acc, Mx, L) in global memory; the
+            // last of them (an atomic ticket) merges all Z in cluster order,
+            // so the result does not depend on the order they finished in
+            const size_t xs = (size_t)a.xrows;
+            if (vrow) {
+                float4 *xo = (float4 *)(a.xo + ((size_t)zc * xs + orow_g) * 128);
+#pragma unroll
+                for (int i = 0; i < cpt; ++i) __stcg(xo + cc + i * tpr, acc[i]);
+                if (cc == 0) __stcg(a.xml + (size_t)zc * xs + orow_g, make_float2(Mx, L));
+            }
+            asm volatile("bar.sync 1, 256;\n" ::: "memory");
+            const int cidx = ((b * rgroups + rg) * a.n_kv + kvh) * C + r;
+            if (et == 0) {
+                __threadfence();
+                sm.xticket = atomicAdd(a.xcnt + cidx, 1);
+            }
+            asm volatile("bar.sync 1, 256;\n" ::: "memory");
+            if (sm.xticket == Z - 1) {
+                __threadfence();
+                if (vrow) {
+                    float2 mlz[kAtMaxZ];
+                    float Mf = -INFINITY;
+#pragma unroll
+                    for (int z = 0; z < kAtMaxZ; ++z) {
+                        if (z >= Z) break;
+                        mlz[z] = z == zc ? make_float2(Mx, L) : __ldcg(a.xml + (size_t)z * xs + orow_g);
+                        if (mlz[z].y > 0.f) Mf = fmaxf(Mf, mlz[z].x);
+                    }
+                    float wz[kAtMaxZ], Lf = 0.f;
+#pragma unroll
+                    for (int z = 0; z < kAtMaxZ; ++z) {
+                        if (z >= Z) break;
+                        wz[z] = mlz[z].y > 0.f ? ex2(mlz[z].x - Mf) : 0.f;
+                        Lf = fmaf(wz[z], mlz[z].y, Lf);
+                    }
+                    if (!*abort && Lf > 0.f) {
+                        const float inv = 1.0f / Lf;
+#pragma unroll
+                        for (int i = 0; i < cpt; ++i) {
+                            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                            for (int z = 0; z < kAtMaxZ; ++z) {
+                                if (z >= Z) break;
+                                if (wz[z] == 0.f) continue;
+                                const float4 az = z == zc ? acc[i]
+                                                          : __ldcg((const float4 *)(a.xo + ((size_t)z * xs + orow_g) * 128) +
+                                                                   cc + i * tpr);
+                                y.x = fmaf(wz[z], az.x, y.x); y.y = fmaf(wz[z], az.y, y.y);
+                                y.z = fmaf(wz[z], az.z, y.z); y.w = fmaf(wz[z], az.w, y.w);
+                            }
+                            store(i, y, inv);
+                        }
+                    }
                 }
-                const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-                const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-                *(uint2 *)(o + ch * 4) = make_uint2(*(const uint32_t *)&lo2, *(const uint32_t *)&hi2);
+                if (et == 0) a.xcnt[cidx] = 0;   // ready for the next call
             }
         }
         __syncwarp();
@@ -581,41 +744,66 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
 // ---------------------------------------------------------------- host
 bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
 bool make_tmap_box(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows);
-bool make_tmap_q4(CUtensorMap *m, const void *q, int rows_total, int n_q, int n_kv, int hd, int ksub);
 
 size_t attn_tc_smem_bytes() { return sizeof(AtSmem) + 1024; }
 
-// CTAs per (sequence, KV head, row group): a power of two up to 8 (the
-// portable cluster size; 16-CTA clusters measured slower on B200) that keeps
-// one row group of the whole batch within one wave of SMs.  A function of the
-// batch and model shape only (not of the block size), so a row is reduced in
-// the same order whatever block it is in.
+// CTAs of this kernel in C-CTA clusters that the GPU holds at once (one CTA
+// per SM), for C = 1, 2, 4, 8: measured by attn_tc_init_attributes; the
+// defaults are B200's (148 SMs, clusters confined to a GPC).
+static int g_cluster_ctas[4] = {148, 148, 132, 120};
+static int cluster_ctas(int C) { return g_cluster_ctas[C >= 8 ? 3 : C >= 4 ? 2 : C >= 2 ? 1 : 0]; }
+
+// CTAs per (sequence, KV head, row group): the largest power of two up to 8
+// (the portable cluster size; 16-CTA clusters measured slower on B200: fewer
+// than eight of them fit on the GPU at once) that keeps one row group of the
+// whole batch within one wave.  A function of the batch and model shape only
+// (not of the block size), so a row is reduced in the same order whatever
+// block it is in.
 int attn_cluster_size(int n_kv, int B)
 {
     const int others = n_kv * B;
     int C = 1;
-    while (C < kAtMaxCluster && (2 * C) * others <= kNumSMs) C *= 2;
+    while (C < kAtMaxCluster && (2 * C) * others <= cluster_ctas(2 * C)) C *= 2;
     return C;
+}
+
+template <int C> static cudaError_t at_prepare(int bytes, int *ctas)
+{
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, C);
+    cfg.blockDim = dim3(kAtThreads);
+    cfg.dynamicSmemBytes = bytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = C;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel<C>, &cfg);
+    if (e == cudaSuccess && n > 0) *ctas = std::min(n * C, kNumSMs);
+    return e;
 }
 
 cudaError_t attn_tc_init_attributes()
 {
     const int bytes = (int)attn_tc_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaError_t e = at_prepare<1>(bytes, &g_cluster_ctas[0]);
+    if (e == cudaSuccess) e = at_prepare<2>(bytes, &g_cluster_ctas[1]);
+    if (e == cudaSuccess) e = at_prepare<4>(bytes, &g_cluster_ctas[2]);
+    if (e == cudaSuccess) e = at_prepare<8>(bytes, &g_cluster_ctas[3]);
     return e;
 }
 
-// Tensor maps for one call.  rows_total: token rows the q buffer holds.
-bool attn_tc_maps(const AttnArgs &a, int n_layers, int rows_total, AtMaps *m)
+// Tensor maps for one call (Q rows are read with plain 16-byte loads).
+bool attn_tc_maps(const AttnArgs &a, int n_layers, AtMaps *m)
 {
     memset(m, 0, sizeof(*m));
     const int g = a.n_q / a.n_kv;
-    if (a.hd != 128 || kAtRows % g || a.kv.page_size % 64) return false;
-    const int ksub = std::min(a.K, kAtRows / g);
-    if (!make_tmap_q4(&m->q, a.q, rows_total, a.n_q, a.n_kv, a.hd, ksub)) return false;
+    if (a.hd != 128 || kAtRows % g || a.kv.page_size % 64 || ((uintptr_t)a.q & 15)) return false;
     const uint64_t heads = (uint64_t)n_layers * a.kv.num_pages * a.n_kv;
     if (!make_tmap_box(&m->kc, a.kv.k_pages, heads * a.kv.page_size, 128, 64, 64)) return false;
     if (!make_tmap_box(&m->vc, a.kv.v_pages, heads * 128, a.kv.page_size, 64, 128)) return false;
@@ -642,7 +830,7 @@ cudaError_t launch_attn_tc_cached(const Ctx &c, const AttnArgs &a, int n_split_g
     auto it = c.amaps.find(key);
     if (it == c.amaps.end()) {
         AtMaps m;
-        if (!attn_tc_maps(a, c.cfg.n_layers, q_rows, &m)) return cudaErrorNotSupported;
+        if (!attn_tc_maps(a, c.cfg.n_layers, &m)) return cudaErrorNotSupported;
         it = c.amaps.emplace(key, std::vector<unsigned char>((unsigned char *)&m, (unsigned char *)&m + sizeof(m))).first;
     }
     c.launches += 1;
@@ -654,9 +842,19 @@ cudaError_t launch_attn_tc(const AttnArgs &a, const AtMaps &maps, int n_split_gr
     const int g = a.n_q / a.n_kv;
     const int ksub = kAtRows / g;
     const int rgroups = (a.K + ksub - 1) / ksub;
-    const int C = attn_cluster_size(a.n_kv, a.B);
+    int C = attn_cluster_size(a.n_kv, a.B);
+    AttnArgs x = a;
+    x.xz = 1;
+    if (a.xz > 1 && a.xo && a.xml && a.xcnt) {
+        // long contexts: Z clusters of 4 per row group, all of them within
+        // one wave of four-CTA clusters
+        const int Cz = std::min(C, kAtZCluster);
+        int Z = 1;
+        while (Z < std::min(a.xz, kAtMaxZ) && 2 * Z * Cz * a.n_kv * a.B <= cluster_ctas(Cz)) Z *= 2;
+        if (Z > 1) { C = Cz; x.xz = Z; }
+    }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.n_kv, a.B * rgroups, C);
+    cfg.gridDim = dim3(a.n_kv, a.B * rgroups, C * x.xz);
     cfg.blockDim = dim3(kAtThreads);
     cfg.dynamicSmemBytes = attn_tc_smem_bytes();
     cfg.stream = s;
@@ -670,10 +868,10 @@ cudaError_t launch_attn_tc(const AttnArgs &a, const AtMaps &maps, int n_split_gr
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     switch (C) {
-    case 1: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<1>, maps, a, n_split_grid);
-    case 2: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<2>, maps, a, n_split_grid);
-    case 4: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<4>, maps, a, n_split_grid);
-    default: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<8>, maps, a, n_split_grid);
+    case 1: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<1>, maps, x, n_split_grid);
+    case 2: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<2>, maps, x, n_split_grid);
+    case 4: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<4>, maps, x, n_split_grid);
+    default: return cudaLaunchKernelEx(&cfg, attn_tc_kernel<8>, maps, x, n_split_grid);
     }
 }
 

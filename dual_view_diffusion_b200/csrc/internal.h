@@ -20,7 +20,11 @@ constexpr int kTileK = 64;           // GEMM k chunk
 constexpr int kKeyTile = 64;         // attention: keys per tile
 constexpr int kPrefillChunk = 128;   // prefill rows per forward
 constexpr int kNumSMs = 148;
-constexpr int kResidSlots = 8;   // most k segments of a deferred residual GEMM         // B200
+// Contexts this long spread each attention row group over up to
+// kAttnMaxClusters clusters.
+constexpr int kAttnTwoClusterSeq = 8192;
+constexpr int kAttnMaxClusters = 4;
+constexpr int kResidSlots = 8;   // most k segments of a deferred residual GEMM
 
 // Per-(row, vocab tile) record of the fused LM-head epilogue.
 struct LmPart {
@@ -111,6 +115,14 @@ struct AttnArgs {
     int split_tokens, n_splits;
     float *part;             // [B*K][n_q][n_splits][hd]
     float2 *ml;              // [B*K][n_q][n_splits]
+    // tensor-core path, xz > 1: up to xz clusters per (sequence, KV head,
+    // row group) merged through [xz][xrows][hd] fp32 partial rows,
+    // [xz][xrows] (m, l) and a ticket per owner CTA (zero between calls);
+    // xrows = row capacity x n_q.  xz == 1 (or no buffers): one cluster.
+    float *xo;
+    float2 *xml;
+    int *xcnt;
+    int xrows, xz;
     unsigned *err;
 };
 
@@ -167,6 +179,10 @@ struct Ctx {
     void *res_x;             // [2*max_batch][d]
     float *attn_part;        // [Rw][n_q][n_splits][hd]
     float2 *attn_ml;         // [Rw][n_q][n_splits]
+    float *attn_xo;          // [kAttnMaxClusters][Rw][n_q][hd] (long contexts only, else null)
+    float2 *attn_xml;        // [kAttnMaxClusters][Rw][n_q]
+    int *attn_xcnt;          // [Rw][n_kv][8] tickets
+    int attn_xz;             // most clusters per attention row group (1: short contexts)
     float *gemm_part;
     size_t gemm_part_floats;
     int *gemm_ticket;
