@@ -19,8 +19,8 @@ roofline  the projection GEMMs (the dominant kernels: ~95% of a step's HBM
           timed region; algorithmic bytes = weights + activations in/out
 attn      the dual-view attention kernel of one layer, timed the same way;
           bytes = prefix K/V + Q + O
-attn_long_context  the attention entry point alone at L = 8K and 32K (both
-          views), each call timed after an L2 flush
+attn_long_context  the attention entry point alone at L = 8K, 32K and 128K
+          (both views), each call timed after an L2 flush
 cpu_baseline  the CPU oracle, as it stands, timed on a bounded sample (one
           layer of each view at full width plus 1/16 of the LM head) and
           scaled to a full step
@@ -71,6 +71,10 @@ def parse():
     ap.add_argument("--profile-small", action="store_true",
                     help="small case for ncu captures: 2 layers of the 8B shape, vocab 32000, 2 steps; "
                          "its line is marked profile_case and is not a bench result")
+    ap.add_argument("--profile-attn", type=int, default=0, metavar="L",
+                    help="small case for ncu captures of the attention kernel: the attention entry point "
+                         "alone at prefix length L (both views, 2 calls each); its line is marked "
+                         "profile_case and is not a bench result")
     a = ap.parse_args()
     if a.profile_small:
         a.steps, a.warmup, a.no_cpu_baseline, a.no_e2e = 2, 1, True, True
@@ -184,12 +188,15 @@ def kernel_traffic(name, sources, key="dram_bytes_per_layer"):
         return None
 
 
-def attn_long_context(hbm, split_tokens, lengths=(8192, 32768), reps=10):
+def attn_long_context(hbm, split_tokens, lengths=(8192, 32768, 131072), reps=10):
     """The dual-view attention entry point alone at long context (the
     attention layer shape of the 8B model: 32/8 heads, head_dim 128, block
     K = 32, batch 1), both views, on N(0,1) bf16 inputs.  Each call is timed
-    by CUDA events around the call only, after a 256 MiB write that flushes
-    L2.  Bytes = prefix K/V + block K/V + Q + O."""
+    by CUDA events around the call only, after a 256 MiB read that flushes
+    L2 (a read leaves clean lines: no write-back lands inside the timed
+    call) and a short device-side wait that lets the host enqueue the call
+    before the start event is reached (so host submission time is not
+    counted as device time).  Bytes = prefix K/V + block K/V + Q + O."""
     import torch
     import synth
     import dual_view_diffusion_b200 as pkg
@@ -204,7 +211,8 @@ def attn_long_context(hbm, split_tokens, lengths=(8192, 32768), reps=10):
     q = torch.randn((1, K, n_q, hd), generator=g, device="cuda").to(torch.bfloat16)
     kb = torch.randn((1, K, n_kv, hd), generator=g, device="cuda").to(torch.bfloat16)
     vb = torch.randn((1, K, n_kv, hd), generator=g, device="cuda").to(torch.bfloat16)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = torch.ones(64 << 20, dtype=torch.float32, device="cuda")   # 256 MiB, read to flush L2
+    sink = torch.empty((), dtype=torch.float32, device="cuda")
     out = []
     for L in lengths:
         eng.seq_lens[0] = L
@@ -213,7 +221,8 @@ def attn_long_context(hbm, split_tokens, lengths=(8192, 32768), reps=10):
                 eng.attention(0, mode, q, kb, vb, 1, K)
             ms = []
             for _ in range(reps):
-                flush.zero_()
+                torch.sum(flush, dim=0, out=sink)
+                torch.cuda._sleep(200000)   # ~0.1 ms of device time: the host gets ahead of the GPU
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record()
                 eng.attention(0, mode, q, kb, vb, 1, K)
@@ -227,7 +236,8 @@ def attn_long_context(hbm, split_tokens, lengths=(8192, 32768), reps=10):
     assert eng.check_error()[0] == 0
     del eng
     torch.cuda.empty_cache()
-    return {"unit": "GB/s", "peak": hbm, "how": "isolated calls, L2 flushed before each, median of " + str(reps),
+    return {"unit": "GB/s", "peak": hbm, "how": "isolated calls, L2 flushed by a 256 MiB read before each, "
+            "host enqueue hidden behind a device-side wait, median of " + str(reps),
             "points": out}
 
 
@@ -486,6 +496,11 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.profile_attn:
+        hbm, _, _ = measured_peaks()
+        res = attn_long_context(hbm, args.split_tokens, lengths=(args.profile_attn,), reps=2)
+        print(json.dumps({"profile_case": "attention entry point alone", "attn_long_context": res}), flush=True)
         return
     if world > 1:
         import datetime

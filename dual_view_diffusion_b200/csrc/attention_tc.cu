@@ -37,6 +37,7 @@
 // 64-key subtiles, each from its own page.  All mbarrier waits are
 // bounded.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <string.h>
 
 #include <algorithm>
@@ -72,10 +73,11 @@ struct AtSmem {
     int xticket;   // this cluster's arrival order at the cross-cluster combine
 };
 // Once the last P.V is done, k..v (192 KiB) is reused for the combine: the
-// CTA's merged rows [128][128] fp32 (16-byte chunk ch of row r at ch ^ (r & 31))
-// and (m, l) per row, read by the other CTAs of the cluster.
-constexpr uint32_t kStageO = 0, kStageMl = 64 * 1024;
-static_assert(kStageMl + kAtRows * 8 <= kAtKStages * 32768 + kAtVStages * 32768, "combine area");
+// CTA's normalised rows [128][128] as fp16 scaled per half row (16-byte chunk
+// ch of row r at ch ^ (r & 15)) and (m, l, scale, scale) per row, read by the
+// other CTAs of the cluster.
+constexpr uint32_t kStageO = 0, kStageMl = 32 * 1024;
+static_assert(kStageMl + kAtRows * 16 <= kAtKStages * 32768 + kAtVStages * 32768, "combine area");
 
 // TMEM columns: two O accumulators (even / odd tiles) [0, 256), S [256, 384)
 // (one buffer: the softmax frees it as soon as it has read its scores), P
@@ -230,6 +232,12 @@ __device__ __forceinline__ float4 ld_peer4(uint32_t addr)
 {
     float4 v;
     asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];\n" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint4 ld_peer4u(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
     return v;
 }
 __device__ __forceinline__ float2 ld_peer2(uint32_t addr)
@@ -577,35 +585,47 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     if (warp >= kAtSoftWarp0) {
         const int h = (warp - kAtSoftWarp0) >> 2;
         asm volatile("bar.sync 1, 256;\n" ::: "memory");   // both warpgroups: every P.V is done
-        // merge the two accumulators into (O, m, l) of this row -> staging (the
-        // K/V ring, Q and P are no longer read); warpgroup h takes dims
-        // [64h, 64h + 64)
+        // merge the two accumulators into the normalised row o = O / l and
+        // stage it (the K/V ring is no longer read) as fp16 scaled by the
+        // largest |o| of each half row, so every staged value lies in
+        // [-1, 1]; warpgroup h takes dims [64h, 64h + 64)
         const float2 x0 = sm.xml[0][row], x1 = sm.xml[1][row];
         const float M = fmaxf(x0.x, x1.x);
         const float w0 = x0.y > 0.f ? ex2(x0.x - M) : 0.f, w1 = x1.y > 0.f ? ex2(x1.x - M) : 0.f;
         const float l = w0 * x0.y + w1 * x1.y;
-        float *so = (float *)(area + kStageO) + row * 128;
+        float y[64];
 #pragma unroll
         for (int qq = 0; qq < 2; ++qq) {
-            const int q = 2 * h + qq;
             uint32_t o0[32], o1[32];
-            AT_LD32(tmem + lane_off + kTmemO + q * 32, o0);
-            AT_LD32(tmem + lane_off + kTmemO + 128 + q * 32, o1);
+            AT_LD32(tmem + lane_off + kTmemO + (2 * h + qq) * 32, o0);
+            AT_LD32(tmem + lane_off + kTmemO + 128 + (2 * h + qq) * 32, o1);
             at_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float4 v;
-                float *vv = &v.x;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float y0 = w0 != 0.f ? w0 * __uint_as_float(o0[4 * c + e]) : 0.f;
-                    const float y1 = w1 != 0.f ? w1 * __uint_as_float(o1[4 * c + e]) : 0.f;
-                    vv[e] = y0 + y1;
-                }
-                *(float4 *)(so + (((q * 8 + c) ^ (row & 31)) << 2)) = v;
+            for (int e = 0; e < 32; ++e) {
+                const float y0 = w0 != 0.f ? w0 * __uint_as_float(o0[e]) : 0.f;
+                const float y1 = w1 != 0.f ? w1 * __uint_as_float(o1[e]) : 0.f;
+                y[32 * qq + e] = y0 + y1;
             }
         }
-        if (h == 0) ((float2 *)(area + kStageMl))[row] = l > 0.f ? make_float2(M, l) : make_float2(-INFINITY, 0.f);
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) amax = fmaxf(amax, fabsf(y[e]));
+        const float sc = l > 0.f ? amax / l : 0.f;             // max |o| over the half row
+        const float r = amax > 0.f ? 1.0f / amax : 0.f;        // o / sc = y / amax
+        unsigned char *so = area + kStageO + row * 256;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t u[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const __half2 h2 = __floats2half2_rn(y[8 * c + 2 * e] * r, y[8 * c + 2 * e + 1] * r);
+                u[e] = *(const uint32_t *)&h2;
+            }
+            *(uint4 *)(so + (((8 * h + c) ^ (row & 15)) << 4)) = make_uint4(u[0], u[1], u[2], u[3]);
+        }
+        float *ml = (float *)(area + kStageMl) + row * 4;   // (m, l, scale of dims 0-63, scale of dims 64-127)
+        if (h == 0) { ml[0] = l > 0.f ? M : -INFINITY; ml[1] = l > 0.f ? l : 0.f; }
+        ml[2 + h] = sc;
         at_fence_before();
         __syncwarp();
     }
@@ -614,70 +634,86 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     cluster_wait();
     if (warp >= kAtSoftWarp0) {   // ---------------- owner: rows [r*rpc, (r+1)*rpc), pulled from every CTA
         constexpr int tpr = 256 / rpc;            // threads per owned row: chunks cc, cc + tpr, ...
-        constexpr int cpt = 32 / tpr;             // chunks per thread
+        constexpr int cpt = 16 / tpr;             // 8-dim chunks per thread
+        static_assert(cpt >= 1, "cluster too large for the owner split");
         const int et = threadIdx.x - 32 * kAtSoftWarp0;
         const int rl = et / tpr, cc = et % tpr;
         const int orow = r * rpc + rl;
         uint32_t peer[C];
 #pragma unroll
         for (int c = 0; c < C; ++c) peer[c] = map_peer_addr(area_u, c);
-        float2 ml[C];
-        float4 v[cpt][C];
+        float4 mls[C];
+        uint4 hv[cpt][C];
 #pragma unroll
-        for (int c = 0; c < C; ++c) ml[c] = ld_peer2(peer[c] + kStageMl + orow * 8);
+        for (int c = 0; c < C; ++c) mls[c] = ld_peer4(peer[c] + kStageMl + orow * 16);
 #pragma unroll
         for (int i = 0; i < cpt; ++i) {
             const int ch = cc + i * tpr;
 #pragma unroll
-            for (int c = 0; c < C; ++c)
-                v[i][c] = ld_peer4(peer[c] + kStageO + orow * 512 + ((ch ^ (orow & 31)) << 4));
+            for (int c = 0; c < C; ++c) hv[i][c] = ld_peer4u(peer[c] + kStageO + orow * 256 + ((ch ^ (orow & 15)) << 4));
         }
         float Mx = -INFINITY;
 #pragma unroll
         for (int c = 0; c < C; ++c)
-            if (ml[c].y > 0.f) Mx = fmaxf(Mx, ml[c].x);
+            if (mls[c].y > 0.f) Mx = fmaxf(Mx, mls[c].x);
         float wc[C], L = 0.f;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            wc[c] = ml[c].y > 0.f ? ex2(ml[c].x - Mx) : 0.f;
-            L += wc[c] * ml[c].y;
+            wc[c] = mls[c].y > 0.f ? ex2(mls[c].x - Mx) * mls[c].y : 0.f;   // weight x row sum
+            L += wc[c];
         }
+        const float invL = L > 0.f ? 1.0f / L : 0.f;
         const int rrow = k_lo * g + orow, k = rrow / g, jh = rrow % g;
         const bool vrow = orow < (k_hi - k_lo) * g;
-        float4 acc[cpt];   // sum over the cluster's CTAs, in rank order, relative to Mx
+        float yo[cpt][8];   // the cluster's normalised row, dims 8 ch .. 8 ch + 7, CTAs in rank order
 #pragma unroll
         for (int i = 0; i < cpt; ++i) {
-            acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int ch = cc + i * tpr;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) yo[i][e] = 0.f;
 #pragma unroll
             for (int c = 0; c < C; ++c) {
                 if (wc[c] == 0.f) continue;
-                acc[i].x = fmaf(wc[c], v[i][c].x, acc[i].x); acc[i].y = fmaf(wc[c], v[i][c].y, acc[i].y);
-                acc[i].z = fmaf(wc[c], v[i][c].z, acc[i].z); acc[i].w = fmaf(wc[c], v[i][c].w, acc[i].w);
+                const float f = wc[c] * invL * (ch < 8 ? mls[c].z : mls[c].w);
+                const __half2 *h2 = (const __half2 *)&hv[i][c];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 v = __half22float2(h2[e]);
+                    yo[i][2 * e] = fmaf(f, v.x, yo[i][2 * e]);
+                    yo[i][2 * e + 1] = fmaf(f, v.y, yo[i][2 * e + 1]);
+                }
             }
         }
         const size_t orow_g = (size_t)(b * a.K + k) * a.n_q + kvh * g + jh;   // (token, query head) of the row
         bf16 *o = (bf16 *)a.out + orow_g * 128;
-        auto store = [&](int i, float4 y, float inv) {
-            const int ch = cc + i * tpr;
-            const __nv_bfloat162 lo2 = __floats2bfloat162_rn(y.x * inv, y.y * inv);
-            const __nv_bfloat162 hi2 = __floats2bfloat162_rn(y.z * inv, y.w * inv);
-            *(uint2 *)(o + ch * 4) = make_uint2(*(const uint32_t *)&lo2, *(const uint32_t *)&hi2);
+        auto store = [&](int i, const float *v) {
+            uint32_t u[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+                u[e] = *(const uint32_t *)&b2;
+            }
+            *(uint4 *)(o + (cc + i * tpr) * 8) = make_uint4(u[0], u[1], u[2], u[3]);
         };
         if (Z == 1) {
             if (!*abort && vrow && L > 0.f) {
-                const float inv = 1.0f / L;
 #pragma unroll
-                for (int i = 0; i < cpt; ++i) store(i, acc[i], inv);
+                for (int i = 0; i < cpt; ++i) store(i, yo[i]);
             }
-        } else {
-            // Z clusters: each leaves its (acc, Mx, L) in global memory; the
-            // last of them (an atomic ticket) merges all Z in cluster order,
-            // so the result does not depend on the order they finished in
+        } else if constexpr (C >= kAtZCluster) {   // (the host picks Z > 1 only with C >= 4)
+            // Z clusters: each leaves its normalised row and (Mx, L) in global
+            // memory; the last of them (an atomic ticket) merges all Z in
+            // cluster order, so the result does not depend on the order they
+            // finished in
             const size_t xs = (size_t)a.xrows;
             if (vrow) {
                 float4 *xo = (float4 *)(a.xo + ((size_t)zc * xs + orow_g) * 128);
 #pragma unroll
-                for (int i = 0; i < cpt; ++i) __stcg(xo + cc + i * tpr, acc[i]);
+                for (int i = 0; i < cpt; ++i) {
+                    const int ch = cc + i * tpr;
+                    __stcg(xo + 2 * ch, make_float4(yo[i][0], yo[i][1], yo[i][2], yo[i][3]));
+                    __stcg(xo + 2 * ch + 1, make_float4(yo[i][4], yo[i][5], yo[i][6], yo[i][7]));
+                }
                 if (cc == 0) __stcg(a.xml + (size_t)zc * xs + orow_g, make_float2(Mx, L));
             }
             asm volatile("bar.sync 1, 256;\n" ::: "memory");
@@ -690,37 +726,56 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
             if (sm.xticket == Z - 1) {
                 __threadfence();
                 if (vrow) {
+                    // every other cluster's row, all loads in flight at once
                     float2 mlz[kAtMaxZ];
-                    float Mf = -INFINITY;
+                    float4 az[kAtMaxZ][cpt][2];
 #pragma unroll
                     for (int z = 0; z < kAtMaxZ; ++z) {
-                        if (z >= Z) break;
-                        mlz[z] = z == zc ? make_float2(Mx, L) : __ldcg(a.xml + (size_t)z * xs + orow_g);
-                        if (mlz[z].y > 0.f) Mf = fmaxf(Mf, mlz[z].x);
+                        if (z < Z && z != zc) {
+                            mlz[z] = __ldcg(a.xml + (size_t)z * xs + orow_g);
+                            const float4 *xq = (const float4 *)(a.xo + ((size_t)z * xs + orow_g) * 128);
+#pragma unroll
+                            for (int i = 0; i < cpt; ++i) {
+                                const int ch = cc + i * tpr;
+                                az[z][i][0] = __ldcg(xq + 2 * ch);
+                                az[z][i][1] = __ldcg(xq + 2 * ch + 1);
+                            }
+                        } else {
+                            mlz[z] = make_float2(Mx, L);
+#pragma unroll
+                            for (int i = 0; i < cpt; ++i) {
+                                az[z][i][0] = make_float4(yo[i][0], yo[i][1], yo[i][2], yo[i][3]);
+                                az[z][i][1] = make_float4(yo[i][4], yo[i][5], yo[i][6], yo[i][7]);
+                            }
+                        }
                     }
+                    float Mf = -INFINITY;
+#pragma unroll
+                    for (int z = 0; z < kAtMaxZ; ++z)
+                        if (z < Z && mlz[z].y > 0.f) Mf = fmaxf(Mf, mlz[z].x);
                     float wz[kAtMaxZ], Lf = 0.f;
 #pragma unroll
                     for (int z = 0; z < kAtMaxZ; ++z) {
-                        if (z >= Z) break;
-                        wz[z] = mlz[z].y > 0.f ? ex2(mlz[z].x - Mf) : 0.f;
-                        Lf = fmaf(wz[z], mlz[z].y, Lf);
+                        wz[z] = (z < Z && mlz[z].y > 0.f) ? ex2(mlz[z].x - Mf) * mlz[z].y : 0.f;
+                        Lf += wz[z];
                     }
                     if (!*abort && Lf > 0.f) {
                         const float inv = 1.0f / Lf;
 #pragma unroll
                         for (int i = 0; i < cpt; ++i) {
-                            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+                            float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                             for (int z = 0; z < kAtMaxZ; ++z) {
-                                if (z >= Z) break;
                                 if (wz[z] == 0.f) continue;
-                                const float4 az = z == zc ? acc[i]
-                                                          : __ldcg((const float4 *)(a.xo + ((size_t)z * xs + orow_g) * 128) +
-                                                                   cc + i * tpr);
-                                y.x = fmaf(wz[z], az.x, y.x); y.y = fmaf(wz[z], az.y, y.y);
-                                y.z = fmaf(wz[z], az.z, y.z); y.w = fmaf(wz[z], az.w, y.w);
+                                const float f = wz[z] * inv;
+                                const float *s0 = &az[z][i][0].x, *s1 = &az[z][i][1].x;
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    v[e] = fmaf(f, s0[e], v[e]);
+                                    v[4 + e] = fmaf(f, s1[e], v[4 + e]);
+                                }
                             }
-                            store(i, y, inv);
+                            store(i, v);
                         }
                     }
                 }
@@ -850,7 +905,8 @@ cudaError_t launch_attn_tc(const AttnArgs &a, const AtMaps &maps, int n_split_gr
         // one wave of four-CTA clusters
         const int Cz = std::min(C, kAtZCluster);
         int Z = 1;
-        while (Z < std::min(a.xz, kAtMaxZ) && 2 * Z * Cz * a.n_kv * a.B <= cluster_ctas(Cz)) Z *= 2;
+        // (clusters smaller than 4 mean a batch too wide for two of them)
+        while (Cz == kAtZCluster && Z < std::min(a.xz, kAtMaxZ) && 2 * Z * Cz * a.n_kv * a.B <= cluster_ctas(Cz)) Z *= 2;
         if (Z > 1) { C = Cz; x.xz = Z; }
     }
     cudaLaunchConfig_t cfg = {};

@@ -343,21 +343,30 @@ __global__ void set_lens_kernel(int32_t *seq_lens, int b, int value, int32_t *an
 }
 
 // Block K/V given as [B][K][n_kv][hd] -> K [B][n_kv][kp][hd] and V transposed
-// [B][n_kv][hd][kp] (rows K .. kp-1 zero).
+// [B][n_kv][hd][kp] (rows K .. kp-1 zero).  Grid (n_kv, B, kp / 16), 256
+// threads: 16 rows x 16 runs of 8 dims, every load of a thread in flight at
+// once.
 template <class T>
 __global__ void pack_block_kernel(const T *ks, const T *vs, T *kd, T *vd, int K, int kp, int n_kv, int hd)
 {
     pdl_trigger();
     pdl_wait();
     const int b = blockIdx.y, kvh = blockIdx.x;
-    for (int idx = threadIdx.x; idx < kp * hd; idx += blockDim.x) {
-        const int k = idx / hd, d = idx % hd;
-        const T z = from_f<T>(0.f);
-        const T kv = k < K ? ks[(((size_t)b * K + k) * n_kv + kvh) * hd + d] : z;
-        const T vv = k < K ? vs[(((size_t)b * K + k) * n_kv + kvh) * hd + d] : z;
-        const size_t head = (size_t)b * n_kv + kvh;
-        kd[(head * kp + k) * hd + d] = kv;
-        vd[(head * hd + d) * kp + k] = vv;
+    const int k = blockIdx.z * 16 + (int)threadIdx.x / 16, d0 = ((int)threadIdx.x % 16) * 8;
+    if (k >= kp || d0 >= hd) return;
+    const T z = from_f<T>(0.f);
+    T kv[8], vv[8];
+    const size_t src = (((size_t)b * K + k) * n_kv + kvh) * hd + d0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        kv[e] = k < K ? ks[src + e] : z;
+        vv[e] = k < K ? vs[src + e] : z;
+    }
+    const size_t head = (size_t)b * n_kv + kvh;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        kd[(head * kp + k) * hd + d0 + e] = kv[e];
+        vd[(head * hd + d0 + e) * kp + k] = vv[e];
     }
 }
 
@@ -480,7 +489,7 @@ cudaError_t launch_pack_block(const Ctx &c, const void *k_src, const void *v_src
                               int K, int kp, cudaStream_t s)
 {
     c.launches += 1;
-    const dim3 grid(c.cfg.n_kv_heads, B);
+    const dim3 grid(c.cfg.n_kv_heads, B, (kp + 15) / 16);
     if (c.cfg.dtype == ORTHRUS_BF16)
         return launch_k(pack_block_kernel<bf16>, grid, 256, 0, s, (const bf16 *)k_src, (const bf16 *)v_src,
                         (bf16 *)k_dst, (bf16 *)v_dst, K, kp, c.cfg.n_kv_heads, c.cfg.head_dim);
