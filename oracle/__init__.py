@@ -6,8 +6,9 @@ imports it, and it never imports the product package.
 
 The C source follows the paper-notes page on "Orthrus: Memory-Efficient
 Parallel Token Generation via Dual-View Diffusion" (§2.1 dual-view layer,
-§3.2 diffusion mask, §4.1-4.3 the decode cycle and its consensus); each C
-function cites the passage it restates.
+§3.2 diffusion mask, §4.1-4.3 the decode cycle and its consensus; §3.1-3.3
+the training-side block mask and forward KL); each C function cites the
+passage it restates.
 """
 from __future__ import annotations
 
@@ -106,6 +107,9 @@ def lib():
                                                C.c_double, C.c_int, _D]
             l.oc_enumerate_orthrus_2pass.argtypes = [P(_Cfg), P(_Model), _I, C.c_int, C.c_int, C.c_int,
                                                      C.c_double, C.c_int, _D]
+            l.oc_block_mask_attention.argtypes = [_D, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _D, _D,
+                                                  C.c_int, _D, _D, _I, _D]
+            l.oc_kl_rows.argtypes = [_D, _D, C.c_int, C.c_int, _F, C.c_int, _D, _D, _D]
             _lib = l
     return _lib
 
@@ -171,6 +175,36 @@ def attention(q, kc, vc, kb, vb, mode):
     o = np.empty_like(q)
     lib().oc_attention(_dp(q), R, nq, nkv, hd, _dp(kc), _dp(vc), t, _dp(kb), _dp(vb), int(mode), _dp(o))
     return o
+
+
+def block_mask_attention(q, kctx, vctx, kblk, vblk, anchors, K):
+    """Diffusion-pass attention of one packed training sequence under the
+    dual-pass block mask.  q [n_blocks*K, n_q, hd]; kctx/vctx [L, n_kv, hd]
+    (clean context, AR view); kblk/vblk [n_blocks*K, n_kv, hd] (the blocks'
+    diffusion K/V); anchors [n_blocks].  Returns o [n_blocks*K, n_q, hd]."""
+    q, kblk, vblk = _f64(q), _f64(kblk), _f64(vblk)
+    rows, nq, hd = q.shape
+    nkv = kblk.shape[1]
+    L = 0 if kctx is None else kctx.shape[0]
+    kctx = _f64(kctx) if L else np.zeros((1, nkv, hd))
+    vctx = _f64(vctx) if L else np.zeros((1, nkv, hd))
+    a = _i32(anchors)
+    nb = a.size
+    assert rows == nb * K
+    o = np.empty_like(q)
+    lib().oc_block_mask_attention(_dp(q), nb, K, nq, nkv, hd, _dp(kctx), _dp(vctx), L, _dp(kblk), _dp(vblk),
+                                  _ip(a), _dp(o))
+    return o
+
+
+def kl_rows(hA, hD, W):
+    """Forward KL(softmax(W hA) || softmax(W hD)) per row, and both
+    log-sum-exps.  hA/hD [rows, d] (final-normed hidden rows), W [V, d]."""
+    hA, hD, W = _f64(np.atleast_2d(hA)), _f64(np.atleast_2d(hD)), _f32(W)
+    rows, d = hA.shape
+    kl, la, ld = np.empty(rows), np.empty(rows), np.empty(rows)
+    lib().oc_kl_rows(_dp(hA), _dp(hD), rows, d, _fp(W), W.shape[0], _dp(kl), _dp(la), _dp(ld))
+    return kl, la, ld
 
 
 def philox4x32_10(ctr, key):

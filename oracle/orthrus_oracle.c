@@ -13,7 +13,11 @@
  * anchor plus bidirectional attention inside the block), §4.1 (the cycle:
  * parallel projection, AR verification, consensus and cache truncation),
  * §4.2 (greedy consensus), §4.3 (rejection sampling at T>0).  The
- * hotdry.top engineering page ("推理机制") restates the same cycle.
+ * hotdry.top engineering page ("推理机制") restates the same cycle.  The
+ * training-side pieces follow §3.1-3.3 of the paper-notes page (packed
+ * sequences of anchor blocks, the dual-pass block mask, forward KL against
+ * the frozen AR view) and the hotdry.top page's training section
+ * ("训练策略：双通块掩码与前向 KL 蒸馏").
  *
  * Arithmetic is fp64 throughout.  Weights arrive as fp32 arrays holding the
  * exact model values (bf16 values are exactly representable in fp32).  Every
@@ -845,4 +849,123 @@ out:
     if (lvl) for (int e = 0; e < N; ++e) free(lvl[e]);
     free(lvl); free(seq); free(blk); free(x); free(y); free(z); free(q1); free(q2); free(pc); free(r);
     return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Training-side pieces (paper notes §3.1-3.3): the dual-pass block mask and  */
+/* the forward KL against the frozen AR view.                                 */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Block-masked attention of the diffusion pass over one packed training
+ * sequence (paper notes §3.1-3.2: a packed sequence of L clean tokens holds
+ * n_blocks anchor blocks of K positions; block b starts at anchor position
+ * a_b).  The key set is the packed layout itself: the L clean context
+ * positions (their AR K/V) followed by every block's K rows (its diffusion
+ * K/V).  Query row k of block b may see
+ *   - context position p        iff p < a_b  (causal up to, not including,
+ *                                             its anchor: the anchor is the
+ *                                             block's own row 0),
+ *   - row k' of block b'         iff b' == b  (bidirectional inside the
+ *                                             block; blocks never see one
+ *                                             another).
+ *   q            [n_blocks*K][n_q][hd]
+ *   kctx, vctx   [L][n_kv][hd]
+ *   kblk, vblk   [n_blocks*K][n_kv][hd]
+ *   anchors      [n_blocks], 0 <= a_b <= L
+ *   o            [n_blocks*K][n_q][hd]
+ * The mask is evaluated for every key of the packed layout (L + n_blocks*K
+ * of them), so this is a plain masked softmax written out, independent of
+ * oc_attention's per-sequence key walk.
+ */
+void oc_block_mask_attention(const double *q, int n_blocks, int K, int n_q, int n_kv, int hd,
+                             const double *kctx, const double *vctx, int L,
+                             const double *kblk, const double *vblk, const int32_t *anchors, double *o)
+{
+    int g = n_q / n_kv;
+    long nkeys = (long)L + (long)n_blocks * K;
+    double scale = 1.0 / sqrt((double)hd);
+    #pragma omp parallel for schedule(static) collapse(2) if ((long)n_blocks * K * n_q * nkeys * hd > 1000000)
+    for (int row = 0; row < n_blocks * K; ++row)
+        for (int h = 0; h < n_q; ++h) {
+            int b = row / K, kvh = h / g;
+            const double *qv = q + ((size_t)row * n_q + h) * hd;
+            double *s = (double *)malloc(sizeof(double) * (size_t)nkeys);
+            char *vis = (char *)malloc((size_t)nkeys);
+            double m = -INFINITY;
+            for (long j = 0; j < nkeys; ++j) {
+                int visible;
+                const double *kv;
+                if (j < L) {
+                    visible = j < anchors[b];
+                    kv = kctx + ((size_t)j * n_kv + kvh) * hd;
+                } else {
+                    long jb = j - L;
+                    visible = (int)(jb / K) == b;
+                    kv = kblk + ((size_t)jb * n_kv + kvh) * hd;
+                }
+                vis[j] = (char)visible;
+                if (!visible) continue;
+                double d = 0.0;
+                for (int i = 0; i < hd; ++i) d += qv[i] * kv[i];
+                s[j] = d * scale;
+                if (s[j] > m) m = s[j];
+            }
+            double l = 0.0;
+            for (long j = 0; j < nkeys; ++j)
+                if (vis[j]) { s[j] = exp(s[j] - m); l += s[j]; }
+            double *ov = o + ((size_t)row * n_q + h) * hd;
+            for (int i = 0; i < hd; ++i) ov[i] = 0.0;
+            for (long j = 0; j < nkeys; ++j) {
+                if (!vis[j]) continue;
+                const double *vv = (j < L) ? vctx + ((size_t)j * n_kv + kvh) * hd
+                                           : vblk + ((size_t)(j - L) * n_kv + kvh) * hd;
+                double p = s[j] / l;
+                for (int i = 0; i < hd; ++i) ov[i] += p * vv[i];
+            }
+            free(vis);
+            free(s);
+        }
+}
+
+/*
+ * Forward KL of the distillation loss (paper notes §3.3): for each row r,
+ * z_A = W h_A[r] (frozen AR view) and z_D = W h_D[r] (diffusion view) over
+ * the whole vocabulary (the shared LM head W [V][d]; h are the final-normed
+ * hidden rows), p = softmax(z) and
+ *     KL(p_A || p_D) = sum_v p_A(v) (log p_A(v) - log p_D(v)).
+ * Also returns both log-sum-exps.
+ */
+void oc_kl_rows(const double *hA, const double *hD, int rows, int d, const float *W, int V,
+                double *kl, double *lseA, double *lseD)
+{
+    #pragma omp parallel for schedule(static) if ((long)rows * V * d > 1000000)
+    for (int r = 0; r < rows; ++r) {
+        double *zA = (double *)malloc(sizeof(double) * (size_t)V);
+        double *zD = (double *)malloc(sizeof(double) * (size_t)V);
+        double mA = -INFINITY, mD = -INFINITY;
+        for (int v = 0; v < V; ++v) {
+            const float *w = W + (size_t)v * d;
+            double a = 0.0, b = 0.0;
+            for (int i = 0; i < d; ++i) {
+                a += (double)w[i] * hA[(size_t)r * d + i];
+                b += (double)w[i] * hD[(size_t)r * d + i];
+            }
+            zA[v] = a; zD[v] = b;
+            if (a > mA) mA = a;
+            if (b > mD) mD = b;
+        }
+        double sA = 0.0, sD = 0.0;
+        for (int v = 0; v < V; ++v) { sA += exp(zA[v] - mA); sD += exp(zD[v] - mD); }
+        double la = mA + log(sA), ld = mD + log(sD), acc = 0.0;
+        for (int v = 0; v < V; ++v) {
+            double lpa = zA[v] - la, lpd = zD[v] - ld;
+            acc += exp(lpa) * (lpa - lpd);
+        }
+        kl[r] = acc;
+        if (lseA) lseA[r] = la;
+        if (lseD) lseD[r] = ld;
+        free(zA);
+        free(zD);
+    }
 }

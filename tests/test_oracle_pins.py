@@ -4,8 +4,9 @@ known-answer vectors and exact enumeration of the sampled decode.
 
 Passages restated by the oracle: the paper-notes page on "Orthrus:
 Memory-Efficient Parallel Token Generation via Dual-View Diffusion", §2.1
-(dual-view layer), §3.2 (diffusion mask), §4.1-§4.3 (cycle, greedy and
-sampled consensus), §5.1 (TPF bounds), §9.1 (losslessness).
+(dual-view layer), §3.1-§3.3 (packed anchor blocks, dual-pass block mask,
+forward KL), §3.2 (diffusion mask), §4.1-§4.3 (cycle, greedy and sampled
+consensus), §5.1 (TPF bounds), §9.1 (losslessness).
 """
 import math
 import os
@@ -369,3 +370,103 @@ def test_two_pass_orthrus_is_lossless_by_enumeration(T):
     # really walks the second pass): the planted mistake lands elsewhere
     p1b = m.enumerate_orthrus(pr, 3, 4, T, planted_error=True)
     assert 0.5 * np.abs(pb - p1b).sum() > 1e-6
+
+
+# ------------------------------------------------------------------ training-side pieces (§3.1-§3.3)
+def _bm_case(rng, n_blocks=3, K=4, L=12, nq=4, nkv=2, hd=16, anchors=None):
+    q = rng.standard_normal((n_blocks * K, nq, hd))
+    kc, vc = rng.standard_normal((L, nkv, hd)), rng.standard_normal((L, nkv, hd))
+    kb, vb = rng.standard_normal((n_blocks * K, nkv, hd)), rng.standard_normal((n_blocks * K, nkv, hd))
+    if anchors is None:
+        anchors = rng.integers(0, L + 1, n_blocks)
+    return q, kc, vc, kb, vb, np.asarray(anchors, np.int32)
+
+
+def test_block_mask_equals_per_block_diffusion_attention():
+    # each block under the packed mask == the diffusion-view attention of
+    # that block alone over the context prefix before its anchor (the
+    # oracle's per-sequence formulation, a separate code path)
+    rng = np.random.default_rng(11)
+    K = 4
+    q, kc, vc, kb, vb, a = _bm_case(rng, n_blocks=4, K=K, anchors=[0, 5, 12, 7])
+    o = oracle.block_mask_attention(q, kc, vc, kb, vb, a, K)
+    for b in range(4):
+        s = slice(b * K, (b + 1) * K)
+        t = int(a[b])
+        ref = oracle.attention(q[s], kc[:t] if t else None, vc[:t] if t else None, kb[s], vb[s], 1)
+        assert np.allclose(o[s], ref, rtol=0, atol=1e-12)
+
+
+def test_block_mask_uniform_scores_average_the_visible_values():
+    # every visible key equal -> uniform softmax -> output = mean of the
+    # visible value rows (context [0, a_b) and the block's K rows)
+    rng = np.random.default_rng(12)
+    K, L, nq, nkv, hd = 4, 10, 4, 2, 8
+    q, kc, vc, kb, vb, a = _bm_case(rng, n_blocks=3, K=K, L=L, nq=nq, nkv=nkv, hd=hd, anchors=[0, 3, 10])
+    k0 = rng.standard_normal(hd)
+    kc[:] = k0
+    kb[:] = k0
+    o = oracle.block_mask_attention(q, kc, vc, kb, vb, a, K)
+    g = nq // nkv
+    for b in range(3):
+        t = int(a[b])
+        for h in range(nq):
+            vis = np.concatenate([vc[:t, h // g], vb[b * K:(b + 1) * K, h // g]])
+            for k in range(K):
+                assert np.allclose(o[b * K + k, h], vis.mean(0), atol=1e-12)
+
+
+def test_block_mask_blocks_are_mutually_invisible_and_anchor_excluded():
+    rng = np.random.default_rng(13)
+    K = 4
+    q, kc, vc, kb, vb, a = _bm_case(rng, n_blocks=2, K=K, anchors=[6, 9])
+    o = oracle.block_mask_attention(q, kc, vc, kb, vb, a, K)
+    kb2, vb2 = kb.copy(), vb.copy()
+    kb2[K:] += 3.0
+    vb2[K:] -= 2.0
+    o2 = oracle.block_mask_attention(q, kc, vc, kb2, vb2, a, K)
+    assert np.array_equal(o[:K], o2[:K])            # block 1 changed, block 0 untouched
+    assert not np.allclose(o[K:], o2[K:])
+    kc3, vc3 = kc.copy(), vc.copy()
+    kc3[6:] += 5.0                                  # at or after block 0's anchor
+    vc3[6:] += 5.0
+    o3 = oracle.block_mask_attention(q, kc3, vc3, kb, vb, a, K)
+    assert np.array_equal(o[:K], o3[:K])
+    kc3[5] += 5.0                                   # the last context row before the anchor
+    vc3[5] += 5.0
+    o4 = oracle.block_mask_attention(q, kc3, vc3, kb, vb, a, K)
+    assert not np.allclose(o[:K], o4[:K])
+
+
+def test_kl_rows_matches_library_relative_entropy():
+    from scipy.stats import entropy
+    rng = np.random.default_rng(14)
+    V, d = 300, 24
+    W = rng.standard_normal((V, d)).astype(np.float32)
+    hA = rng.standard_normal((5, d))
+    hD = hA + 0.4 * rng.standard_normal((5, d))
+    kl, la, ld = oracle.kl_rows(hA, hD, W)
+    zA, zD = hA @ W.T.astype(np.float64), hD @ W.T.astype(np.float64)
+    for r in range(5):
+        pA = torch.softmax(torch.from_numpy(zA[r]), 0).numpy()
+        pD = torch.softmax(torch.from_numpy(zD[r]), 0).numpy()
+        assert math.isclose(kl[r], entropy(pA, pD), rel_tol=1e-10)        # forward KL(p_A || p_D)
+        assert math.isclose(la[r], float(torch.logsumexp(torch.from_numpy(zA[r]), 0)), rel_tol=1e-12)
+        assert math.isclose(ld[r], float(torch.logsumexp(torch.from_numpy(zD[r]), 0)), rel_tol=1e-12)
+        assert not math.isclose(kl[r], entropy(pD, pA), rel_tol=1e-6)     # the reverse direction differs
+
+
+def test_kl_rows_closed_forms():
+    rng = np.random.default_rng(15)
+    W = rng.standard_normal((40, 6)).astype(np.float32)
+    h = rng.standard_normal((3, 6))
+    kl, _, _ = oracle.kl_rows(h, h, W)
+    assert np.all(np.abs(kl) < 1e-12)                # identical views
+    # two-token vocabulary: KL = p log(p/q) + (1-p) log((1-p)/(1-q))
+    W2 = np.array([[1.0, 0.0], [0.0, 1.0]], np.float32)
+    hA, hD = np.array([[0.7, -0.4]]), np.array([[-0.2, 0.5]])
+    p = 1 / (1 + math.exp(-(0.7 + 0.4)))
+    qq = 1 / (1 + math.exp(-(-0.2 - 0.5)))
+    want = p * math.log(p / qq) + (1 - p) * math.log((1 - p) / (1 - qq))
+    kl2, _, _ = oracle.kl_rows(hA, hD, W2)
+    assert math.isclose(kl2[0], want, rel_tol=1e-12)
