@@ -83,6 +83,8 @@ _SIGS = {
     "orthrus_generate": [_P, C.POINTER(KV), _P, _I, C.POINTER(_I), _I, _I, _I, C.c_float, C.c_uint64, _P,
                          C.POINTER(Stats), _P],
     "orthrus_dual_view_attention": [_P, C.POINTER(KV), _I, _I, _P, _P, _P, _I, _I, _P, _P],
+    "orthrus_block_mask_attention": [_P, C.POINTER(KV), _I, _P, _P, _P, _P, _I, _I, _P, _P],
+    "orthrus_kl_lm_head": [_P, _P, _P, _I, _P, _P, _P, _P],
     "orthrus_debug_logits": [_P, _I, _I, _I, _P, _P],
     "orthrus_check_error": [_P, _P, C.POINTER(C.c_uint32)],
     "orthrus_set_probe": [_P, _I, _I, _I, C.POINTER(_P), C.POINTER(_P), _I],
@@ -305,6 +307,28 @@ class Engine:
             self.ctx, C.byref(self.kv), layer, mode, _ptr(q), _ptr(k_blk), _ptr(v_blk), B, K, _ptr(out),
             _stream()))
         return out
+
+    def block_mask_attention(self, layer, q, k_blk, v_blk, anchors, K):
+        """Training-side block-masked attention of one packed sequence:
+        block b (rows [b*K, (b+1)*K) of q) sees context positions
+        [0, anchors[b]) of block-table row 0 and its own K rows.
+        anchors: device int32 [n_blocks]."""
+        n_blocks = int(anchors.numel())
+        out = self.torch.empty_like(q)
+        _check("orthrus_block_mask_attention", lib().orthrus_block_mask_attention(
+            self.ctx, C.byref(self.kv), layer, _ptr(q), _ptr(k_blk), _ptr(v_blk), _ptr(anchors), n_blocks, K,
+            _ptr(out), _stream()))
+        return out
+
+    def kl_lm_head(self, h_ar, h_diff):
+        """Forward KL(softmax(W h_ar) || softmax(W h_diff)) per row through the
+        LM head, with both log-sum-exps: three fp32 [rows] tensors."""
+        rows = int(h_ar.shape[0])
+        kl = self.torch.empty(rows, dtype=self.torch.float32, device=self.device)
+        la, ld = self.torch.empty_like(kl), self.torch.empty_like(kl)
+        _check("orthrus_kl_lm_head", lib().orthrus_kl_lm_head(
+            self.ctx, _ptr(h_ar), _ptr(h_diff), rows, _ptr(kl), _ptr(la), _ptr(ld), _stream()))
+        return kl, la, ld
 
     def debug_logits(self, which, B, K):
         out = self.torch.empty((B, K, self.shape.vocab), dtype=self.torch.float32, device=self.device)

@@ -108,6 +108,7 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
     const size_t o_invf = take((size_t)c.head_dim / 2 * 8);
     const size_t o_lm = take(Rlm * n_vtiles * sizeof(LmPart));
     const size_t o_tok = take(Rw * 4), o_pos = take(mb * 4), o_bt = take(mb * 4), o_pr = take(4);
+    const size_t o_bz = take(mb * 4);   // zeros, never written
     const size_t o_dr = take(R * 4), o_lq = take(R * 4), o_lsq = take(R * 4), o_g = take(R * 4), o_lp = take(R * 4),
                  o_lsp = take(R * 4);
     const size_t o_rj = take(mb * 4), o_rt = take(mb * 4), o_any = take(4), o_err = take(4), o_prod = take(mb * 4),
@@ -126,6 +127,7 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
         x->resid_part = (float *)P(o_rp);
         x->rope_invf = (double *)P(o_invf);
         x->tok = (int32_t *)P(o_tok); x->pos0 = (int32_t *)P(o_pos); x->bt_rows = (int32_t *)P(o_bt);
+        x->bt_zero = (int32_t *)P(o_bz);
         x->prefill_row = (int32_t *)P(o_pr);
         x->draft = (int32_t *)P(o_dr); x->logq = (float *)P(o_lq); x->lse_q = (float *)P(o_lsq);
         x->g = (int32_t *)P(o_g); x->logp = (float *)P(o_lp); x->lse_p = (float *)P(o_lsp);
@@ -144,7 +146,7 @@ static void rebase(Ctx *x, char *ws)
     auto fix = [&](auto *&p) { p = (std::remove_reference_t<decltype(p)>)(ws + (size_t)(const char *)p); };
     fix(x->h); fix(x->a); fix(x->q); fix(x->attn_o); fix(x->act); fix(x->k_diff); fix(x->v_diff); fix(x->blk_pack);
     fix(x->fin_draft); fix(x->fin_verify); fix(x->res_x); fix(x->attn_part); fix(x->attn_ml); fix(x->gemm_part);
-    fix(x->gemm_ticket); fix(x->lm_part); fix(x->resid_part); fix(x->rope_invf); fix(x->tok); fix(x->pos0); fix(x->bt_rows); fix(x->prefill_row);
+    fix(x->gemm_ticket); fix(x->lm_part); fix(x->resid_part); fix(x->rope_invf); fix(x->tok); fix(x->pos0); fix(x->bt_rows); fix(x->bt_zero); fix(x->prefill_row);
     fix(x->draft); fix(x->logq); fix(x->lse_q); fix(x->g); fix(x->logp); fix(x->lse_p); fix(x->rej_row);
     fix(x->res_tok); fix(x->any_reject); fix(x->err); fix(x->produced); fix(x->step); fix(x->n_buf);
     fix(x->tok_buf); fix(x->anchor_buf);
@@ -609,6 +611,52 @@ orthrus_status_t orthrus_dual_view_attention(orthrus_ctx_t *c, const orthrus_kv_
     at.xo = c->attn_xo; at.xml = c->attn_xml; at.xcnt = c->attn_xcnt; at.xrows = c->Rw * f.n_q_heads;
     at.xz = c->attn_xz;
     CK(launch_attention(*c, at, s, batch * K));
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_block_mask_attention(orthrus_ctx_t *c, const orthrus_kv_t *kv, int32_t layer,
+                                              const void *q, const void *k_blk, const void *v_blk,
+                                              const int32_t *anchors, int32_t n_blocks, int32_t K, void *out,
+                                              void *stream)
+{
+    if (!c || !kv || !q || !k_blk || !v_blk || !anchors || !out) return ORTHRUS_ERR_INVALID_ARG;
+    const orthrus_config_t &f = c->cfg;
+    if (n_blocks < 1 || K < 1 || K > f.max_block || layer < 0 || layer >= f.n_layers) return ORTHRUS_ERR_INVALID_ARG;
+    {   // kv->seq_lens is not read here: the block lengths are the anchors
+        orthrus_kv_t k2 = *kv;
+        k2.seq_lens = const_cast<int32_t *>(anchors);
+        if (!kv_ok(c, &k2)) return ORTHRUS_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    // the diffusion view with one sequence per block: length = the block's
+    // anchor, every block on block-table row 0 (the packed context); blocks
+    // are independent, so they go max_batch at a time
+    const size_t half = (size_t)f.max_batch * c->kp * f.n_kv_heads * f.head_dim * c->esize;
+    const size_t qrow = (size_t)K * f.n_q_heads * f.head_dim * c->esize, kvrow = (size_t)K * f.n_kv_heads * f.head_dim * c->esize;
+    for (int b0 = 0; b0 < n_blocks; b0 += f.max_batch) {
+        const int nb = std::min(f.max_batch, n_blocks - b0);
+        CK(launch_pack_block(*c, (const char *)k_blk + b0 * kvrow, (const char *)v_blk + b0 * kvrow, c->blk_pack,
+                             (char *)c->blk_pack + half, nb, K, c->kp, s));
+        AttnArgs at{};
+        at.k_blk = c->blk_pack; at.v_blk = (char *)c->blk_pack + half;
+        at.kp = c->kp; at.bmax = f.max_batch; at.blk_layer = 0; at.blk_layers = 1;
+        at.q = (const char *)q + b0 * qrow; at.out = (char *)out + b0 * qrow; at.kv = kv_view(*kv); at.layer = layer;
+        at.seq_lens = anchors + b0; at.bt_rows = c->bt_zero; at.B = nb; at.K = K; at.n_q = f.n_q_heads;
+        at.n_kv = f.n_kv_heads; at.hd = f.head_dim; at.mode = 1; at.split_tokens = f.split_tokens;
+        at.n_splits = c->n_splits; at.part = c->attn_part; at.ml = c->attn_ml; at.err = c->err;
+        at.xo = c->attn_xo; at.xml = c->attn_xml; at.xcnt = c->attn_xcnt; at.xrows = c->Rw * f.n_q_heads;
+        at.xz = c->attn_xz;
+        CK(launch_attention(*c, at, s, nb * K));
+    }
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_kl_lm_head(orthrus_ctx_t *c, const void *h_ar, const void *h_diff, int32_t rows,
+                                    float *kl, float *lse_ar, float *lse_diff, void *stream)
+{
+    if (!c || !h_ar || !h_diff || !kl || rows < 1) return ORTHRUS_ERR_INVALID_ARG;
+    if (2 * (size_t)rows > (size_t)c->cfg.max_batch * c->cfg.max_block) return ORTHRUS_ERR_CAPACITY;
+    CK(launch_kl_lm_head(*c, h_ar, h_diff, rows, kl, lse_ar, lse_diff, (cudaStream_t)stream));
     return ORTHRUS_OK;
 }
 

@@ -370,6 +370,67 @@ __global__ void pack_block_kernel(const T *ks, const T *vs, T *kd, T *vd, int K,
     }
 }
 
+// Rows of two views into one interleaved activation buffer: out[2r] =
+// a[r], out[2r+1] = b[r] (the row pairs of the forward-KL LM-head GEMM).
+template <class T>
+__global__ void interleave_rows_kernel(const T *ra, const T *rb, T *out, int d)
+{
+    pdl_trigger();
+    pdl_wait();
+    const int r = blockIdx.x;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+        out[(size_t)(2 * r) * d + i] = ra[(size_t)r * d + i];
+        out[(size_t)(2 * r + 1) * d + i] = rb[(size_t)r * d + i];
+    }
+}
+
+// Forward KL per row pair from the per-tile records of EPI_KL (paper notes
+// §3.3): with M = max over tiles, S = sum_t s_t exp(m_t - M) for each view
+// and T = sum_t t_t exp(ma_t - M_AR),
+//     LSE = M + log S,   KL(p_AR || p_diff) = T / S_AR - (LSE_AR - LSE_diff).
+struct KlArgs {
+    const KlPart *part;
+    int n_vtiles, rows;
+    float *kl, *lse_a, *lse_d;
+    unsigned *err;
+};
+
+__global__ void __launch_bounds__(256) kl_finalize_kernel(KlArgs a)
+{
+    pdl_trigger();
+    pdl_wait();
+    const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (w >= a.rows) return;
+    const KlPart *p = a.part + (size_t)w * a.n_vtiles;
+    float Ma = -INFINITY, Md = -INFINITY;
+    for (int i = lane; i < a.n_vtiles; i += 32) {
+        Ma = fmaxf(Ma, p[i].ma);
+        Md = fmaxf(Md, p[i].md);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        Ma = fmaxf(Ma, __shfl_xor_sync(0xffffffffu, Ma, o));
+        Md = fmaxf(Md, __shfl_xor_sync(0xffffffffu, Md, o));
+    }
+    float Sa = 0.f, Ta = 0.f, Sd = 0.f;
+    for (int i = lane; i < a.n_vtiles; i += 32) {
+        const float fa = expf(p[i].ma - Ma);
+        Sa = fmaf(p[i].sa, fa, Sa);
+        Ta = fmaf(p[i].ta, fa, Ta);
+        Sd = fmaf(p[i].sd, expf(p[i].md - Md), Sd);
+    }
+    Sa = warp_sum(Sa);
+    Ta = warp_sum(Ta);
+    Sd = warp_sum(Sd);
+    if (lane != 0) return;
+    const float la = Ma + logf(Sa), ld = Md + logf(Sd);
+    const float kl = Ta / Sa - (la - ld);
+    if (!isfinite(kl)) raise_err(a.err, ORTHRUS_DEVERR_NONFINITE);
+    a.kl[w] = kl;
+    if (a.lse_a) a.lse_a[w] = la;
+    if (a.lse_d) a.lse_d[w] = ld;
+}
+
 __global__ void set_int_kernel(int32_t *p, int v)
 {
     // no early pdl_trigger: later kernels read what this one writes before
@@ -495,6 +556,30 @@ cudaError_t launch_pack_block(const Ctx &c, const void *k_src, const void *v_src
                         (bf16 *)k_dst, (bf16 *)v_dst, K, kp, c.cfg.n_kv_heads, c.cfg.head_dim);
     return launch_k(pack_block_kernel<float>, grid, 256, 0, s, (const float *)k_src, (const float *)v_src,
                     (float *)k_dst, (float *)v_dst, K, kp, c.cfg.n_kv_heads, c.cfg.head_dim);
+}
+
+cudaError_t launch_kl_lm_head(const Ctx &c, const void *h_a, const void *h_d, int rows, float *kl, float *lse_a,
+                              float *lse_d, cudaStream_t s)
+{
+    const int d = c.cfg.hidden;
+    c.launches += 1;
+    cudaError_t e = c.cfg.dtype == ORTHRUS_BF16
+                        ? launch_k(interleave_rows_kernel<bf16>, rows, 256, 0, s, (const bf16 *)h_a, (const bf16 *)h_d,
+                                   (bf16 *)c.a, d)
+                        : launch_k(interleave_rows_kernel<float>, rows, 256, 0, s, (const float *)h_a,
+                                   (const float *)h_d, (float *)c.a, d);
+    if (e != cudaSuccess) return e;
+    GemmArgs g{};
+    g.x = c.a; g.M = 2 * rows; g.N = c.cfg.vocab; g.Kd = d;
+    g.w[0] = c.lm_head; g.wrows[0] = c.cfg.vocab;
+    g.epi = EPI_KL; g.kl = (KlPart *)c.lm_part;
+    e = launch_gemm(c, g, s);
+    if (e != cudaSuccess) return e;
+    KlArgs k;
+    k.part = (const KlPart *)c.lm_part; k.n_vtiles = c.n_vtiles; k.rows = rows;
+    k.kl = kl; k.lse_a = lse_a; k.lse_d = lse_d; k.err = c.err;
+    c.launches += 1;
+    return launch_k(kl_finalize_kernel, (rows + 7) / 8, 256, 0, s, k);
 }
 
 cudaError_t launch_logits_dump(const Ctx &c, const void *fin, int M, float *logits, cudaStream_t s)

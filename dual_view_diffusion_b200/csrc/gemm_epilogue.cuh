@@ -424,6 +424,50 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
             const int m = idx >> 7, nl = idx & 127, row = mt * kTileM + m, n = nt * kTileN + nl;
             if (row < a.M && n < a.N) a.logits[(size_t)row * a.N + n] = tile[m][nl];
         }
+    } else if (epi == EPI_KL) {
+        // rows come in pairs (2i: AR view, 2i+1: diffusion view of the same
+        // position, paper notes §3.3); per pair and vocabulary tile: each
+        // view's max and sum of exponentials, and the AR-weighted sum of
+        // z_AR - z_diff (the forward-KL numerator)
+        const int lane = tid & 31, warp = tid >> 5;
+        for (int pl = 0; pl < kTileM / 8; ++pl) {
+            const int mp = warp * (kTileM / 8) + pl;        // pair index within tile
+            const int m = 2 * mp, row = mt * kTileM + m;
+            if (row >= a.M) break;
+            float za[4], zd[4];
+            float ma = -INFINITY, md = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int nl = lane * 4 + j;
+                const bool ok = nt * kTileN + nl < a.N;
+                za[j] = ok ? tile[m][nl] : -INFINITY;
+                zd[j] = ok ? tile[m + 1][nl] : -INFINITY;
+                ma = fmaxf(ma, za[j]);
+                md = fmaxf(md, zd[j]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, o));
+                md = fmaxf(md, __shfl_xor_sync(0xffffffffu, md, o));
+            }
+            float sa = 0.f, ta = 0.f, sd = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (nt * kTileN + lane * 4 + j >= a.N) continue;
+                const float ea = expf(za[j] - ma);
+                sa += ea;
+                ta = fmaf(ea, za[j] - zd[j], ta);
+                sd += expf(zd[j] - md);
+            }
+            sa = warp_sum(sa);
+            ta = warp_sum(ta);
+            sd = warp_sum(sd);
+            if (lane == 0) {
+                KlPart pr{};
+                pr.ma = ma; pr.sa = sa; pr.ta = ta; pr.md = md; pr.sd = sd;
+                a.kl[(size_t)(row / 2) * n_nt + nt] = pr;
+            }
+        }
     } else if (epi == EPI_RESAMPLE) {
         // rows come in pairs (2b: AR view at the rejected row, 2b+1: diffusion
         // view at the same row); score = log max(0, p - q) + Gumbel

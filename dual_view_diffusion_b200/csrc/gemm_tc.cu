@@ -563,6 +563,7 @@ cudaError_t gemm_tc_init_attributes()
     if (e == cudaSuccess) e = set_smem<EPI_LMHEAD>();
     if (e == cudaSuccess) e = set_smem<EPI_RESAMPLE>();
     if (e == cudaSuccess) e = set_smem<EPI_LOGITS>();
+    if (e == cudaSuccess) e = set_smem<EPI_KL>();
     return e;
 }
 
@@ -639,6 +640,7 @@ cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, 
     case EPI_LMHEAD: return launch_k(gemm_tc_kernel<EPI_LMHEAD>, k.G, kTcThreads, smem, s, maps, a, k);
     case EPI_RESAMPLE: return launch_k(gemm_tc_kernel<EPI_RESAMPLE>, k.G, kTcThreads, smem, s, maps, a, k);
     case EPI_LOGITS: return launch_k(gemm_tc_kernel<EPI_LOGITS>, k.G, kTcThreads, smem, s, maps, a, k);
+    case EPI_KL: return launch_k(gemm_tc_kernel<EPI_KL>, k.G, kTcThreads, smem, s, maps, a, k);
     default: return cudaErrorNotSupported;
     }
 }

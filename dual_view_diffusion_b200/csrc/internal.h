@@ -38,7 +38,20 @@ struct LmPart {
     int pad;
 };
 
-enum Epi : int { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_LMHEAD = 3, EPI_RESAMPLE = 4, EPI_LOGITS = 5 };
+// Per-(row pair, vocab tile) record of the fused forward-KL epilogue: rows
+// 2i (AR view) and 2i+1 (diffusion view) of the same position.
+struct KlPart {
+    float ma;    // max AR logit in the tile
+    float sa;    // sum over the tile of exp(z_AR - ma)
+    float ta;    // sum over the tile of exp(z_AR - ma) (z_AR - z_diff)
+    float md;    // max diffusion logit in the tile
+    float sd;    // sum over the tile of exp(z_diff - md)
+    int pad[3];
+};
+static_assert(sizeof(KlPart) == sizeof(LmPart), "KL records share the LM-head record buffer");
+
+enum Epi : int { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_LMHEAD = 3, EPI_RESAMPLE = 4, EPI_LOGITS = 5,
+                 EPI_KL = 6 };
 
 // Where an attention / QKV call reads positions and writes K/V.
 struct KvView {
@@ -94,6 +107,7 @@ struct GemmArgs {
     const int32_t *rej_row;  // EPI_RESAMPLE: [batch] j or -1
     const int *any_flag;     // EPI_RESAMPLE: skip everything when 0
     float *logits;           // EPI_LOGITS: [M][N] fp32
+    KlPart *kl;              // EPI_KL: [M / 2][n_vtiles]
 };
 
 struct AttnArgs {
@@ -194,6 +208,7 @@ struct Ctx {
     int32_t *tok;            // [Rw] block tokens
     int32_t *pos0;           // [max_batch]
     int32_t *bt_rows;        // [max_batch] identity rows 0..max_batch-1
+    int32_t *bt_zero;        // [max_batch] zeros (every entry reads block-table row 0)
     int32_t *prefill_row;    // [1]
     int32_t *draft;          // [R]
     float *logq, *lse_q;     // [R]
@@ -258,5 +273,7 @@ cudaError_t launch_set_lens(const Ctx &c, int32_t *seq_lens, int b, int value, i
 cudaError_t launch_pack_block(const Ctx &c, const void *k_src, const void *v_src, void *k_dst, void *v_dst, int B,
                               int K, int kp, cudaStream_t s);
 cudaError_t launch_logits_dump(const Ctx &c, const void *fin, int M, float *logits, cudaStream_t s);
+cudaError_t launch_kl_lm_head(const Ctx &c, const void *h_a, const void *h_d, int rows, float *kl, float *lse_a,
+                              float *lse_d, cudaStream_t s);
 
 }  // namespace orthrus

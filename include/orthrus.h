@@ -289,6 +289,54 @@ orthrus_status_t orthrus_dual_view_attention_noalloc(const orthrus_config_t *cfg
                                                     uint32_t *dev_err, void *stream);
 
 /*
+ * Training-side dual-pass block-masked attention (paper notes §3.1-3.2; the
+ * hotdry.top page's training section): one packed training sequence of L
+ * clean positions holds n_blocks anchor blocks of K positions each; block b
+ * starts at anchor position anchors[b].  Query row k of block b sees the
+ * clean context positions [0, anchors[b]) (their AR K/V) and all K rows of
+ * its own block (their diffusion K/V, bidirectional); blocks never see one
+ * another.  This is the diffusion-view kernel with one "sequence" per block,
+ * all reading the same context pages.
+ *   kv        block_table row 0 lists the packed context's pages, in order;
+ *             its layer-`layer` slice holds the context K/V (rows [0, L));
+ *             kv->seq_lens is not read.
+ *   q         device [n_blocks][K][n_q][hd] (context dtype)
+ *   k_blk,
+ *   v_blk     device [n_blocks][K][n_kv][hd], the blocks' diffusion K/V
+ *   anchors   DEVICE int32 [n_blocks], 0 <= anchors[b]; positions past the
+ *             pages block_table row 0 covers raise ORTHRUS_DEVERR_CAPACITY
+ *   out       device [n_blocks][K][n_q][hd]
+ * Requires n_blocks >= 1 and 1 <= K <= max_block; blocks are independent
+ * and are processed max_batch at a time.  Ownership and errors as for
+ * orthrus_dual_view_attention.
+ */
+orthrus_status_t orthrus_block_mask_attention(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, int32_t layer,
+                                              const void *q, const void *k_blk, const void *v_blk,
+                                              const int32_t *anchors, int32_t n_blocks, int32_t K, void *out,
+                                              void *stream);
+
+/*
+ * Forward KL of the distillation loss (paper notes §3.3): for each row r,
+ * with the shared LM head W,
+ *     KL(p_AR || p_diff) = sum_v p_AR(v) (log p_AR(v) - log p_diff(v)),
+ *     p_AR = softmax(W h_ar[r]),  p_diff = softmax(W h_diff[r]),
+ * over the whole vocabulary, fused into the LM-head GEMM: the logits never
+ * reach memory (per vocabulary tile the epilogue keeps both views' max and
+ * sum of exponentials and sum exp(z_AR - max)(z_AR - z_diff); a second
+ * kernel merges the tiles).
+ *   h_ar, h_diff  device [rows][hidden] (context dtype): final-normed hidden
+ *                 rows of the two views at the same positions
+ *   kl            device fp32 [rows]
+ *   lse_ar,
+ *   lse_diff      device fp32 [rows] log-sum-exps of the two views, or NULL
+ * Requires 1 <= rows and 2 * rows <= max_batch * max_block.  Uses the
+ * context's workspace (its activation rows and LM-head records), so it must
+ * not overlap a decode call of the same context on the GPU.
+ */
+orthrus_status_t orthrus_kl_lm_head(orthrus_ctx_t *ctx, const void *h_ar, const void *h_diff, int32_t rows,
+                                    float *kl, float *lse_ar, float *lse_diff, void *stream);
+
+/*
  * Test and measurement hook: the logits of the last verify (which = 0) or
  * draft (which = 1) for every block row, fp32 [batch][K][vocab], computed
  * from the final hidden rows the step kept (one extra LM-head pass; the
