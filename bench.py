@@ -21,6 +21,10 @@ attn      the dual-view attention kernel of one layer, timed the same way;
           bytes = prefix K/V + Q + O
 attn_long_context  the attention entry point alone at L = 8K, 32K and 128K
           (both views), each call timed after an L2 flush
+train_kernels  the training-side kernels (block-masked attention of a packed
+          2048-position sequence with 256 anchor blocks; the forward-KL
+          LM-head epilogue over the full vocabulary), each timed alone beside
+          the oracle on a sample
 cpu_baseline  the CPU oracle, as it stands, timed on a bounded sample (one
           layer of each view at full width plus 1/16 of the LM head) and
           scaled to a full step
@@ -239,6 +243,99 @@ def attn_long_context(hbm, split_tokens, lengths=(8192, 32768, 131072), reps=10)
     return {"unit": "GB/s", "peak": hbm, "how": "isolated calls, L2 flushed by a 256 MiB read before each, "
             "host enqueue hidden behind a device-side wait, median of " + str(reps),
             "points": out}
+
+
+def _timed(fn, reps, flush, sink):
+    """Median device time (us) of fn() over reps calls, each after a 256 MiB
+    read that flushes L2 and a device-side wait that hides host enqueue."""
+    import torch
+    for _ in range(2):
+        fn()
+    ms = []
+    for _ in range(reps):
+        torch.sum(flush, dim=0, out=sink)
+        torch.cuda._sleep(200000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    return statistics.median(ms) * 1e3
+
+
+def train_kernels(hbm, tflops, eng, reps=10):
+    """The training-side kernels of the pages (§3.1-3.3), each timed alone
+    (flushed L2, median of reps) beside the CPU oracle on a sample.
+    block_mask_attention: one packed training sequence, 256 anchor blocks of
+    K = 32 over 2048 positions (anchors uniform in [0, 2016], seed 4), the 8B
+    attention shape, N(0,1) bf16; bound tensor: useful FLOPs = 4 hd x the
+    keys each (row, query head) sees.  kl_lm_head: 16 row pairs (N(0, 3^2)
+    bf16 hidden rows, diffusion = AR + N(0, 1.8^2)) through the 8B LM head
+    (151936 x 4096, the decode engine's); bound HBM: the head's bytes + rows."""
+    import numpy as np
+    import torch
+    import oracle
+    import synth
+    import dual_view_diffusion_b200 as pkg
+    flush = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+    sink = torch.empty((), dtype=torch.float32, device="cuda")
+    out = {}
+    # ---- block-masked attention
+    nb, K, L = 256, K_BLOCK, 2048
+    s = dataclasses.replace(synth.QWEN3_8B, n_layers=1, hidden=64, ffn=64, vocab=256)
+    w = synth.make_weights(s, 0, n_layers=1)
+    ae = pkg.Engine(s, w, max_batch=128, max_block=K, max_seq=L + 64, split_tokens=128)
+    g = torch.Generator(device="cuda").manual_seed(4)
+    n_q, n_kv, hd = s.n_q_heads, s.n_kv_heads, s.head_dim
+    for pg in (ae.k_pages, ae.v_pages):
+        pg.copy_(torch.randn(pg.shape, generator=g, device="cuda").to(pg.dtype))
+    q = torch.randn((nb, K, n_q, hd), generator=g, device="cuda").to(torch.bfloat16)
+    kb = torch.randn((nb, K, n_kv, hd), generator=g, device="cuda").to(torch.bfloat16)
+    vb = torch.randn((nb, K, n_kv, hd), generator=g, device="cuda").to(torch.bfloat16)
+    anchors = np.random.default_rng(4).integers(0, L - K + 1, nb).astype(np.int32)
+    ad = torch.from_numpy(anchors).cuda()
+    us = _timed(lambda: ae.block_mask_attention(0, q, kb, vb, ad, K), reps, flush, sink)
+    flops = float(4 * hd * K * n_q * (anchors.astype(np.int64) + K).sum())
+    byts = 2 * nb * K * n_q * hd * 2 + 2 * nb * K * n_kv * hd * 2 + 2 * L * n_kv * hd * 2
+    t0 = time.perf_counter()
+    qh, kbh, vbh = (x.float().cpu().numpy() for x in (q[:2], kb[:2], vb[:2]))
+    kc = ae.k_pages[0, :L // ae.page_size].float().permute(0, 2, 1, 3).reshape(L, n_kv, hd).cpu().numpy()
+    vc = ae.v_pages[0, :L // ae.page_size].float().permute(0, 3, 1, 2).reshape(L, n_kv, hd).cpu().numpy()
+    t_prep = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    for b in range(2):
+        oracle.block_mask_attention(qh[b], kc, vc, kbh[b], vbh[b], anchors[b:b + 1], K)
+    t_cpu = (time.perf_counter() - t0) / float(anchors[:2].astype(np.int64).sum() + 2 * K) * \
+        float(anchors.astype(np.int64).sum() + nb * K)
+    ach = flops / us / 1e6
+    out["block_mask_attention"] = {
+        "workload": "256 anchor blocks x K=32 in one packed 2048-position sequence, 32/8 heads, head_dim 128",
+        "us": us, "bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s", "frac": ach / tflops,
+        "hbm_gbs": byts / us / 1e3, "algorithmic_flops": flops, "algorithmic_bytes": byts,
+        "cpu_baseline": {"seconds": t_cpu, "cores": OracleSample.threads(), "kind": "oracle",
+                         "sample": "2 of the 256 blocks, scaled by visible keys"}}
+    del ae
+    torch.cuda.empty_cache()
+    # ---- forward-KL LM head on the decode engine's 8B head
+    rows, d, V = 16, eng.shape.hidden, eng.shape.vocab
+    gk = torch.Generator(device="cuda").manual_seed(5)
+    hA = (3.0 * torch.randn((rows, d), generator=gk, device="cuda")).to(torch.bfloat16)
+    hD = (hA.float() + 1.8 * torch.randn((rows, d), generator=gk, device="cuda")).to(torch.bfloat16)
+    us = _timed(lambda: eng.kl_lm_head(hA, hD), reps, flush, sink)
+    byts = V * d * 2 + 2 * rows * d * 2 + rows * 12
+    Vs = 8192
+    Wh = eng.lm_head[:Vs].float().cpu().numpy()
+    t0 = time.perf_counter()
+    oracle.kl_rows(hA[:1].float().cpu().numpy(), hD[:1].float().cpu().numpy(), Wh)
+    t_cpu = (time.perf_counter() - t0) * rows * V / Vs
+    ach = byts / us / 1e3
+    out["kl_lm_head"] = {
+        "workload": "16 row pairs through the 151936 x 4096 LM head", "us": us, "bound": "hbm",
+        "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "algorithmic_bytes": byts,
+        "cpu_baseline": {"seconds": t_cpu, "cores": OracleSample.threads(), "kind": "oracle",
+                         "sample": f"1 row pair over the first {Vs} vocabulary ids, scaled"}}
+    return out
 
 
 # ----------------------------------------------------------------- oracle sample
@@ -477,6 +574,7 @@ def run_ours(args, rank, world, local_rank):
         line["e2e"] = e2e
     if not args.profile_small:
         line["attn_long_context"] = attn_long_context(hbm, args.split_tokens)
+        line["train_kernels"] = train_kernels(hbm, tflops, eng)
     if args.profile_small:
         line = {"profile_case": True, "config": "2 layers of the Qwen3-8B shape, vocab 32000", "value": value,
                 "roofline": line["roofline"], "attn": line["attn"]}
