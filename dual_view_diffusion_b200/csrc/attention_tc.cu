@@ -607,6 +607,23 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
                 y[32 * qq + e] = y0 + y1;
             }
         }
+        if (C == 1 && Z == 1) {   // a lone CTA: this row is final, write it from registers
+            const int rr1 = k_lo * g + row, k1 = rr1 / g;
+            if (!*abort && k1 < k_hi && l > 0.f) {
+                const float inv = 1.0f / l;
+                bf16 *o = (bf16 *)a.out + ((size_t)(b * a.K + k1) * a.n_q + kvh * g + rr1 % g) * 128 + 64 * h;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t u[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[8 * c + 2 * e] * inv, y[8 * c + 2 * e + 1] * inv);
+                        u[e] = *(const uint32_t *)&b2;
+                    }
+                    *(uint4 *)(o + 8 * c) = make_uint4(u[0], u[1], u[2], u[3]);
+                }
+            }
+        } else {
         float amax = 0.f;
 #pragma unroll
         for (int e = 0; e < 64; ++e) amax = fmaxf(amax, fabsf(y[e]));
@@ -627,12 +644,13 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
         if (h == 0) { ml[0] = l > 0.f ? M : -INFINITY; ml[1] = l > 0.f ? l : 0.f; }
         ml[2 + h] = sc;
         at_fence_before();
+        }
         __syncwarp();
     }
     // every CTA's merged rows are in its shared memory (release / acquire)
     cluster_arrive();
     cluster_wait();
-    if (warp >= kAtSoftWarp0) {   // ---------------- owner: rows [r*rpc, (r+1)*rpc), pulled from every CTA
+    if (warp >= kAtSoftWarp0 && !(C == 1 && Z == 1)) {   // ------- owner: rows [r*rpc, (r+1)*rpc), pulled from every CTA
         constexpr int tpr = 256 / rpc;            // threads per owned row: chunks cc, cc + tpr, ...
         constexpr int cpt = 16 / tpr;             // 8-dim chunks per thread
         static_assert(cpt >= 1, "cluster too large for the owner split");

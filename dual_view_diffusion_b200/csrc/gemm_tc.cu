@@ -97,6 +97,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile
     return false;
 }
 
+// Weight tiles are read once per forward: they are loaded with an L2
+// evict-first policy so that the weight stream does not push activations,
+// cache pages and the other kernels' code out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar,
+                                                 uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;\n"
+        ::"r"(smem_u32(dst)), "l"((uint64_t)map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
 {
     asm volatile(
@@ -291,6 +309,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
             uint32_t stage = 0, phase = 0;
             int issued = 0;
             bool waited = false;
+            const uint64_t wpol = l2_evict_first();
             int def_c[kTcStages], def_mt[kTcStages];
             auto release_deferred = [&]() {
                 pdl_wait();
@@ -311,10 +330,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                     if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort) || *abort) { stop = true; break; }
                     mbar_expect_tx(&sm.full[stage], kStageWBytes + kStageXBytes);
                     if (E == EPI_SWIGLU) {
-                        tma_load_2d(sm.w[stage], &maps.w[0], c * kTileK, s.nt * 64, &sm.full[stage]);
-                        tma_load_2d(sm.w[stage] + kStageWBytes / 2, &maps.w[1], c * kTileK, s.nt * 64, &sm.full[stage]);
+                        tma_load_2d_hint(sm.w[stage], &maps.w[0], c * kTileK, s.nt * 64, &sm.full[stage], wpol);
+                        tma_load_2d_hint(sm.w[stage] + kStageWBytes / 2, &maps.w[1], c * kTileK, s.nt * 64,
+                                         &sm.full[stage], wpol);
                     } else {
-                        tma_load_2d(sm.w[stage], &maps.w[wsel], c * kTileK, wrow, &sm.full[stage]);
+                        tma_load_2d_hint(sm.w[stage], &maps.w[wsel], c * kTileK, wrow, &sm.full[stage], wpol);
                     }
                     if (!waited) { def_c[issued] = c; def_mt[issued] = s.mt; }
                     else tma_load_2d(sm.x[stage], &maps.x, c * kTileK, s.mt * kTileM, &sm.full[stage]);
