@@ -123,6 +123,15 @@ __device__ __forceinline__ void at_tma2(void *dst, const CUtensorMap *m, int x, 
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
         ::"r"(smem_u32(dst)), "l"((uint64_t)m), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
 }
+// cache tiles are read once per view: loaded evict-first, they leave the
+// rest of L2 (activations, code, block tables) in place
+__device__ __forceinline__ void at_tma2_ef(void *dst, const CUtensorMap *m, int x, int y, uint64_t *bar, uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;\n"
+        ::"r"(smem_u32(dst)), "l"((uint64_t)m), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol) : "memory");
+}
 __device__ __forceinline__ void at_tma4(void *dst, const CUtensorMap *m, int x, int y, int z, int w, uint64_t *bar)
 {
     asm volatile(
@@ -358,6 +367,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
         // (which the predecessor cannot be writing) are requested before
         // waiting for it.
         const bool kprod = warp == 0;
+        uint64_t pol;
+        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
         uint32_t ks = 0, kph = 0, vs = 0, vph = 0;
         bool waited = false, stop = false;
         auto ensure_wait = [&]() {
@@ -406,8 +417,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
                                         at_tma2(sm.k[ks][hh] + u * 8192, &maps.kb, hh * 64, krow * a.kp + (u ? brow1 : brow0),
                                                 &sm.kfull[ks]);
                                     else
-                                        at_tma2(sm.k[ks][hh] + u * 8192, &maps.kc, hh * 64, hrow[u] * a.kv.page_size + off[u],
-                                                &sm.kfull[ks]);
+                                        at_tma2_ef(sm.k[ks][hh] + u * 8192, &maps.kc, hh * 64, hrow[u] * a.kv.page_size + off[u],
+                                                &sm.kfull[ks], pol);
                                 }
                             if (++ks == kAtKStages) { ks = 0; kph ^= 1; }
                         }
@@ -419,7 +430,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
                                 if (sp.block) at_tma2(sm.v[vs][u], &maps.vb, u ? brow1 : brow0, krow * 128, &sm.vfull[vs]);
-                                else at_tma2(sm.v[vs][u], &maps.vc, off[u], hrow[u] * 128, &sm.vfull[vs]);
+                                else at_tma2_ef(sm.v[vs][u], &maps.vc, off[u], hrow[u] * 128, &sm.vfull[vs], pol);
                             }
                             if (++vs == kAtVStages) { vs = 0; vph ^= 1; }
                         }
