@@ -146,3 +146,27 @@ def test_kl_lm_head_identical_views_is_zero():
     torch.cuda.synchronize()
     assert np.all(kl.cpu().numpy() == 0.0)
     assert torch.equal(la, ld)
+
+
+def test_block_mask_attention_ragged_shapes():
+    # short blocks (K = 8: one partial subtile), a context that is not a
+    # multiple of the tile (L = 300), anchors at 0 and at L, more blocks than
+    # one launch holds (7 blocks, max_batch 5: launches of 5 and 2)
+    n_blocks, K, L, n_q, n_kv, hd = 7, 8, 300, 16, 4, 128
+    q, kc, vc, kb, vb, a = _block_case(24, n_blocks, K, L, n_q, n_kv, hd, anchors=[300, 0, 64, 65, 127, 128, 299])
+    eng = attention_engine(n_q=n_q, n_kv=n_kv, hd=hd, max_batch=5, max_block=16, max_seq=L + 64, split_tokens=128)
+    got = _run_block_mask(eng, q, kc, vc, kb, vb, a, K)
+    want = oracle.block_mask_attention(q, kc, vc, kb, vb, a, K)
+    assert np.abs(got - want).max() < ATOL_ATTN
+
+
+def test_kl_lm_head_single_row_ragged_vocab():
+    # one row pair, a vocabulary of 129 ids (a full tile plus one id)
+    eng, W = _kl_engine(129, 256)
+    hA, hD = _kl_rows(34, 1, 256)
+    kl, la, ld = eng.kl_lm_head(_dev(hA, eng), _dev(hD, eng))
+    torch.cuda.synchronize()
+    kl_o, la_o, ld_o = oracle.kl_rows(hA, hD, W)
+    assert abs(float(kl[0]) - kl_o[0]) <= 2e-2 * kl_o[0] + 2e-3
+    assert np.allclose(la.cpu().numpy(), la_o, rtol=1e-4, atol=1e-3)
+    assert np.allclose(ld.cpu().numpy(), ld_o, rtol=1e-4, atol=1e-3)
