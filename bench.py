@@ -19,8 +19,9 @@ roofline  the projection GEMMs (the dominant kernels: ~95% of a step's HBM
           timed region; algorithmic bytes = weights + activations in/out
 attn      the dual-view attention kernel of one layer, timed the same way;
           bytes = prefix K/V + Q + O
-attn_long_context  the attention entry point alone at L = 8K, 32K and 128K
-          (both views), each call timed after an L2 flush
+attn_long_context  the attention entry point alone at L = 4K (the single-layer
+          attention workload: 32/8 heads, head_dim 128, K = 32, batch 1),
+          8K, 32K and 128K (both views), each call timed after an L2 flush
 train_kernels  the training-side kernels (block-masked attention of a packed
           2048-position sequence with 256 anchor blocks; the forward-KL
           LM-head epilogue over the full vocabulary), each timed alone beside
@@ -192,7 +193,7 @@ def kernel_traffic(name, sources, key="dram_bytes_per_layer"):
         return None
 
 
-def attn_long_context(hbm, split_tokens, lengths=(8192, 32768, 131072), reps=10):
+def attn_long_context(hbm, split_tokens, lengths=(4096, 8192, 32768, 131072), reps=10):
     """The dual-view attention entry point alone at long context (the
     attention layer shape of the 8B model: 32/8 heads, head_dim 128, block
     K = 32, batch 1), both views, on N(0,1) bf16 inputs.  Each call is timed
