@@ -252,15 +252,16 @@ def attn_long_context(hbm, split_tokens, lengths=(4096, 8192, 32768, 131072), re
             "points": out}
 
 
-def _timed(fn, reps, flush, sink):
-    """Median device time (us) of fn() over reps calls, each after a 256 MiB
-    read that flushes L2 and a device-side wait that hides host enqueue."""
+def _timed(fn, reps):
+    """Median device time (us) of fn() over reps calls, each after a
+    device-side wait that hides host enqueue (the callers' inputs exceed L2,
+    so no flush is needed)."""
     import torch
     for _ in range(2):
         fn()
     ms = []
     for _ in range(reps):
-        torch.sum(flush, dim=0, out=sink)
+        torch.cuda.synchronize()
         torch.cuda._sleep(200000)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
@@ -273,7 +274,8 @@ def _timed(fn, reps, flush, sink):
 
 def train_kernels(hbm, tflops, eng, reps=10):
     """The training-side kernels of the pages (§3.1-3.3), each timed alone
-    (flushed L2, median of reps) beside the CPU oracle on a sample.
+    (median of reps; each reads more than L2 holds: 176 MB of queries,
+    outputs and K/V, and the 1.24 GB head) beside the CPU oracle on a sample.
     block_mask_attention: one packed training sequence, 256 anchor blocks of
     K = 32 over 2048 positions (anchors uniform in [0, 2016], seed 4), the 8B
     attention shape, N(0,1) bf16; bound tensor: useful FLOPs = 4 hd x the
@@ -285,8 +287,6 @@ def train_kernels(hbm, tflops, eng, reps=10):
     import oracle
     import synth
     import dual_view_diffusion_b200 as pkg
-    flush = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
-    sink = torch.empty((), dtype=torch.float32, device="cuda")
     out = {}
     # ---- block-masked attention
     nb, K, L = 256, K_BLOCK, 2048
@@ -302,7 +302,7 @@ def train_kernels(hbm, tflops, eng, reps=10):
     vb = torch.randn((nb, K, n_kv, hd), generator=g, device="cuda").to(torch.bfloat16)
     anchors = np.random.default_rng(4).integers(0, L - K + 1, nb).astype(np.int32)
     ad = torch.from_numpy(anchors).cuda()
-    us = _timed(lambda: ae.block_mask_attention(0, q, kb, vb, ad, K), reps, flush, sink)
+    us = _timed(lambda: ae.block_mask_attention(0, q, kb, vb, ad, K), reps)
     flops = float(4 * hd * K * n_q * (anchors.astype(np.int64) + K).sum())
     byts = 2 * nb * K * n_q * hd * 2 + 2 * nb * K * n_kv * hd * 2 + 2 * L * n_kv * hd * 2
     t0 = time.perf_counter()
@@ -329,7 +329,7 @@ def train_kernels(hbm, tflops, eng, reps=10):
     gk = torch.Generator(device="cuda").manual_seed(5)
     hA = (3.0 * torch.randn((rows, d), generator=gk, device="cuda")).to(torch.bfloat16)
     hD = (hA.float() + 1.8 * torch.randn((rows, d), generator=gk, device="cuda")).to(torch.bfloat16)
-    us = _timed(lambda: eng.kl_lm_head(hA, hD), reps, flush, sink)
+    us = _timed(lambda: eng.kl_lm_head(hA, hD), reps)
     byts = V * d * 2 + 2 * rows * d * 2 + rows * 12
     Vs = 8192
     Wh = eng.lm_head[:Vs].float().cpu().numpy()
