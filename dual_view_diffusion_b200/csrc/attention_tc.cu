@@ -132,12 +132,6 @@ __device__ __forceinline__ void at_tma2_ef(void *dst, const CUtensorMap *m, int 
         " [%0], [%1, {%2, %3}], [%4], %5;\n"
         ::"r"(smem_u32(dst)), "l"((uint64_t)m), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol) : "memory");
 }
-__device__ __forceinline__ void at_tma4(void *dst, const CUtensorMap *m, int x, int y, int z, int w, uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];\n"
-        ::"r"(smem_u32(dst)), "l"((uint64_t)m), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)) : "memory");
-}
 __device__ __forceinline__ uint64_t at_desc(const void *p)
 {
     const uint32_t a = smem_u32(p);
@@ -247,12 +241,6 @@ __device__ __forceinline__ uint4 ld_peer4u(uint32_t addr)
 {
     uint4 v;
     asm volatile("ld.shared::cluster.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
-}
-__device__ __forceinline__ float2 ld_peer2(uint32_t addr)
-{
-    float2 v;
-    asm volatile("ld.shared::cluster.v2.f32 {%0,%1}, [%2];\n" : "=f"(v.x), "=f"(v.y) : "r"(addr));
     return v;
 }
 __device__ __forceinline__ float ex2(float x)   // 2^x, MUFU; subnormal results flush to zero

@@ -551,23 +551,6 @@ bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, ui
     return make_tmap_box(m, ptr, rows, cols, 64, box_rows);
 }
 
-// 4-D view of q [rows][n_q][hd] as (dim, head in group, kv head, row), box
-// {64, g, 1, ksub}: one load brings the g heads of one KV head for ksub
-// consecutive block rows, ordered (row, head) = the attention CTA's rows.
-bool make_tmap_q4(CUtensorMap *m, const void *q, int rows_total, int n_q, int n_kv, int hd, int ksub)
-{
-    auto enc = get_encoder();
-    const int g = n_q / n_kv;
-    if (!enc || !q || ((uintptr_t)q & 15) || (hd * 2) % 16 || g > 256 || ksub > 256) return false;
-    cuuint64_t dims[4] = {(cuuint64_t)hd, (cuuint64_t)g, (cuuint64_t)n_kv, (cuuint64_t)rows_total};
-    cuuint64_t strides[3] = {(cuuint64_t)hd * 2, (cuuint64_t)g * hd * 2, (cuuint64_t)n_q * hd * 2};
-    cuuint32_t box[4] = {64, (cuuint32_t)g, 1, (cuuint32_t)ksub};
-    cuuint32_t es[4] = {1, 1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 size_t gemm_tc_smem_bytes() { return sizeof(TcSmem) + 1024; }
 
 template <int E> static cudaError_t set_smem()

@@ -246,7 +246,6 @@ cudaError_t gemm_init_attributes();
 cudaError_t gemm_tc_init_attributes();
 bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
 bool make_tmap_box(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows);
-bool make_tmap_q4(CUtensorMap *m, const void *q, int rows_total, int n_q, int n_kv, int hd, int ksub);
 struct AtMaps;
 cudaError_t attn_tc_init_attributes();
 cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, cudaStream_t s);
