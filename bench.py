@@ -13,10 +13,12 @@ value     committed tokens/s over the timed steps (device time, CUDA events,
 e2e       the same metric with the step's input (anchor id) copied from
           pinned host memory and its result (n and the tokens) read back
           every step, through the library's public calls
-roofline  the projection GEMMs (the dominant kernels: ~95% of a step's HBM
-          traffic is weight streaming), timed live by CUDA events around one
-          layer's four projection launches in every verify forward of the
-          timed region; algorithmic bytes = weights + activations in/out
+roofline  the gate/up GEMM with its fused SwiGLU (the step's largest kernel by
+          device time; ~95% of a step's HBM traffic is weight streaming),
+          timed live by CUDA events around its launch in one layer of every
+          verify forward of the timed region; algorithmic bytes = weights +
+          activations in/out.  layer_gemms: the same for the layer's four
+          projection GEMMs together, with each one's time
 attn      the dual-view attention kernel of one layer, timed the same way;
           bytes = prefix K/V + Q + O
 attn_long_context  the attention entry point alone at L = 4K (the single-layer
@@ -554,6 +556,9 @@ def run_ours(args, rank, world, local_rank):
     g_ach = g_bytes / g_time / 1e9
     a_ach = a_bytes / a_time / 1e9
     traffic = kernel_traffic("gemm_projection_qwen3_8b_shape.txt", GEMM_SOURCES)
+    gu_traffic = kernel_traffic("gemm_projection_qwen3_8b_shape.txt", GEMM_SOURCES, "dram_bytes_gate_up")
+    gu_us = float(g_ms[:, 2].mean() * 1e3)
+    gu_ach = gb[2] / (gu_us * 1e-6) / 1e9
     a_traffic = kernel_traffic("attention_qwen3_8b_shape.txt", ATTN_SOURCES, "dram_bytes_per_launch")
     value = tot_tokens / (max_ms * 1e-3)
     nbar = tokens / (K * BATCH)
@@ -567,10 +572,17 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "weights (18 GB) and cache exceed L2 every step; no flush"},
         "mean_accepted_per_cycle": nbar, "tokens_per_forward": nbar / 2,
         "modelled_tokens_per_s_at_pages_acceptance": 10.8 / (max_ms / K * 1e-3),
-        "roofline": {"kernel": "projection GEMMs (QKV, O, gate/up, down) of one layer, verify view", "bound": "hbm",
-                     "achieved": g_ach, "peak": hbm, "unit": "GB/s", "frac": g_ach / hbm,
-                     "traffic": traffic, "peak_source": src, "algorithmic_bytes_per_layer": sum(gb),
-                     "ms_per_layer": float(g_ms.sum(axis=1).mean())},
+        "roofline": {"kernel": "gate/up projection GEMM with the fused SwiGLU epilogue (gemm_tc_kernel<EPI_SWIGLU>, "
+                               "the step's largest kernel by device time), one verify-view layer",
+                     "bound": "hbm", "achieved": gu_ach, "peak": hbm, "unit": "GB/s", "frac": gu_ach / hbm,
+                     "traffic": gu_traffic, "peak_source": src, "algorithmic_bytes": gb[2], "us_per_launch": gu_us,
+                     "layer_gemms": {"kernel": "the four projection GEMMs (QKV, O, gate/up, down) of one layer",
+                                     "achieved": g_ach, "frac": g_ach / hbm, "traffic": traffic,
+                                     "algorithmic_bytes_per_layer": sum(gb),
+                                     "ms_per_layer": float(g_ms.sum(axis=1).mean()),
+                                     "per_gemm": {n: {"us": float(g_ms[:, i].mean() * 1e3),
+                                                      "achieved_gbs": gb[i] / float(g_ms[:, i].mean() * 1e-3) / 1e9}
+                                                  for i, n in enumerate(("qkv", "o", "gate_up", "down"))}}},
         "attn": {"kernel": "dual-view attention (cluster split + on-chip combine), verify view, one layer",
                  "bound": "hbm", "achieved": a_ach, "peak": hbm, "unit": "GB/s", "frac": a_ach / hbm,
                  "traffic": a_traffic, "us_per_call": float(a_ms.mean() * 1e3), "mean_prefix": float(t_steps.mean())},
