@@ -170,3 +170,31 @@ def test_kl_lm_head_single_row_ragged_vocab():
     assert abs(float(kl[0]) - kl_o[0]) <= 2e-2 * kl_o[0] + 2e-3
     assert np.allclose(la.cpu().numpy(), la_o, rtol=1e-4, atol=1e-3)
     assert np.allclose(ld.cpu().numpy(), ld_o, rtol=1e-4, atol=1e-3)
+
+
+def test_training_entry_points_fp32_tiny():
+    # the same two entry points on the fp32 tiny shape (4/2 heads, head_dim 16,
+    # vocab 256): the SIMT attention and SIMT GEMM paths
+    import dual_view_diffusion_b200 as pkg
+    s = synth.TINY
+    w = synth.make_weights(s, 0)
+    eng = pkg.Engine(s, w, max_batch=4, max_block=8, max_seq=128, split_tokens=64, page_size=16)
+    n_blocks, K, L = 6, 4, 40
+    rng = np.random.default_rng(25)
+    q = rng.standard_normal((n_blocks * K, s.n_q_heads, s.head_dim)).astype(np.float32)
+    kc = rng.standard_normal((L, s.n_kv_heads, s.head_dim)).astype(np.float32)
+    vc = rng.standard_normal((L, s.n_kv_heads, s.head_dim)).astype(np.float32)
+    kb = rng.standard_normal((n_blocks * K, s.n_kv_heads, s.head_dim)).astype(np.float32)
+    vb = rng.standard_normal((n_blocks * K, s.n_kv_heads, s.head_dim)).astype(np.float32)
+    a = np.array([0, 5, 16, 17, 39, 40], np.int32)
+    got = _run_block_mask(eng, q, kc, vc, kb, vb, a, K)
+    want = oracle.block_mask_attention(q, kc, vc, kb, vb, a, K)
+    assert np.abs(got - want).max() < 1e-4
+    hA = 2.0 * rng.standard_normal((3, s.hidden)).astype(np.float32)
+    hD = (hA + 1.0 * rng.standard_normal((3, s.hidden))).astype(np.float32)
+    kl, la, ld = eng.kl_lm_head(_dev(hA, eng), _dev(hD, eng))
+    torch.cuda.synchronize()
+    kl_o, la_o, ld_o = oracle.kl_rows(hA, hD, w.lm_head)
+    assert np.allclose(kl.cpu().numpy(), kl_o, rtol=1e-4, atol=1e-6)
+    assert np.allclose(la.cpu().numpy(), la_o, rtol=1e-5, atol=1e-5)
+    assert np.allclose(ld.cpu().numpy(), ld_o, rtol=1e-5, atol=1e-5)
