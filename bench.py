@@ -19,8 +19,10 @@ roofline  the gate/up GEMM with its fused SwiGLU (the step's largest kernel by
           verify forward of the timed region; algorithmic bytes = weights +
           activations in/out.  layer_gemms: the same for the layer's four
           projection GEMMs together, with each one's time
-attn      the dual-view attention kernel of one layer, timed the same way;
-          bytes = prefix K/V + Q + O
+attn      the dual-view attention entry point on the single-layer workload
+          (L = 4096, K = 32, batch 1), timed as attn_long_context does;
+          in_step: the attention kernel of one layer inside the decode
+          step, timed like the roofline GEMM; bytes = prefix K/V + Q + O
 attn_long_context  the attention entry point alone at L = 4K (the single-layer
           attention workload: 32/8 heads, head_dim 128, K = 32, batch 1),
           8K, 32K and 128K (both views), timed over runs of calls on
@@ -592,7 +594,23 @@ def run_ours(args, rank, world, local_rank):
     if e2e:
         line["e2e"] = e2e
     if not args.profile_small:
-        line["attn_long_context"] = attn_long_context(hbm, args.split_tokens)
+        lc = attn_long_context(hbm, args.split_tokens)
+        line["attn_long_context"] = lc
+        # the single-layer attention workload (L = 4096, K = 32, batch 1):
+        # its verify-view point is the attn headline, the step's own
+        # attention (timed inside the decode step) stays beside it
+        p4 = [p for p in lc["points"] if p["L"] == 4096]
+        if p4:
+            v, dv = p4[0], (p4[1] if len(p4) > 1 else None)
+            in_step = line["attn"]
+            line["attn"] = {
+                "kernel": "dual-view attention entry point, the single-layer workload (L = 4096 + K = 32, batch 1, "
+                          "32/8 heads, head_dim 128), verify view",
+                "bound": "hbm", "achieved": v["achieved"], "peak": hbm, "unit": "GB/s", "frac": v["frac"],
+                "traffic": kernel_traffic("attention_l4k_single_layer.txt", ATTN_SOURCES, "dram_bytes_per_launch"),
+                "us_per_call": v["us"], "how": lc["how"],
+                "draft_view": {"achieved": dv["achieved"], "frac": dv["frac"], "us_per_call": dv["us"]} if dv else None,
+                "in_step": in_step}
         line["train_kernels"] = train_kernels(hbm, tflops, eng)
     if args.profile_small:
         line = {"profile_case": True, "config": "2 layers of the Qwen3-8B shape, vocab 32000", "value": value,
