@@ -43,6 +43,7 @@ from __future__ import annotations
 import argparse
 import dataclasses
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -166,10 +167,34 @@ def attn_bytes(s, t, K, B=1):
     return B * ((t + K) * s.n_kv_heads * s.head_dim * 2 * 2 + 2 * K * s.n_q_heads * s.head_dim * 2)
 
 
+def _code_only(text):
+    """C++/CUDA source without comments, blank lines or trailing blanks: a
+    profile stays valid across comment-only edits of its kernel."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = []
+    for line in text.splitlines():
+        # drop a // comment unless it sits inside a string literal
+        out, in_str = [], False
+        i = 0
+        while i < len(line):
+            c = line[i]
+            if c == '"' and (i == 0 or line[i - 1] != "\\"):
+                in_str = not in_str
+            if not in_str and line.startswith("//", i):
+                break
+            out.append(c)
+            i += 1
+        s = "".join(out).rstrip()
+        if s:
+            lines.append(s)
+    return "\n".join(lines)
+
+
 def source_sha(sources):
+    """sha256 of the kernel sources' code (comments and blank lines removed)."""
     h = hashlib.sha256()
     for s in sources:
-        h.update(open(os.path.join(ROOT, s), "rb").read())
+        h.update(_code_only(open(os.path.join(ROOT, s), encoding="utf-8").read()).encode())
     return h.hexdigest()
 
 

@@ -1,11 +1,12 @@
 // Dual-view attention on the tcgen05 tensor cores (bf16, head_dim 128).
 //
-// One cluster of C CTAs per (KV head, sequence x row group).  Its M = 128
-// query rows are the block rows x the GQA group sharing the KV head, so every
-// K/V tile staged in shared memory serves all of them (paper notes §2.2-2.3:
-// both views read the one AR cache).  The keys are cut into splits aligned to
-// absolute positions; CTA r of the cluster takes splits r, r + C, ... and, per
-// 128-key tile:
+// Z clusters of C CTAs per (KV head, sequence x row group) — one cluster
+// normally, four 4-CTA clusters for long contexts at small batch.  Its M =
+// 128 query rows are the block rows x the GQA group sharing the KV head, so
+// every K/V tile staged in shared memory serves all of them (paper notes
+// §2.2-2.3: both views read the one AR cache).  The keys are cut into splits
+// aligned to absolute positions; CTA i of the Z * C takes splits i, i + ZC,
+// ... and, per 128-key tile:
 //
 //   S = Q K^T       tcgen05.mma, M 128 x N 128 x K 128 (A = Q, kept in TMEM
 //                   for the whole kernel), into TMEM
@@ -25,10 +26,13 @@
 // O is rescaled in TMEM only when a warp's running max moved (a factor of
 // exactly 1 elsewhere, so skipping it changes no bit).  K tiles come from
 // pages laid out [slot][dim], V tiles from pages laid out [dim][slot] (both
-// operands K-major), both by TMA.  For the diffusion view the block's own K/V
-// form one extra split read from the transient buffer.  The C partial states
-// are merged through distributed shared memory; nothing goes to global memory
-// but the output rows.
+// operands K-major), both by TMA with an L2 evict-first hint (a cache tile is
+// read once per view).  For the diffusion view the block's own K/V form one
+// extra split read from the transient buffer.  A cluster's C partial states
+// are merged through distributed shared memory (fp16 rows scaled per half
+// row); with Z > 1 each cluster leaves its merged rows in L2 and the last
+// cluster to finish (an atomic ticket) merges all Z in cluster order.  A lone
+// CTA (C = Z = 1) writes its rows straight from registers.
 //
 // Roles: warp 0 K producer and warp 2 V producer (TMA, one issuing thread
 // each, separate rings: a K tile is free once S is computed, a V tile only
