@@ -27,6 +27,7 @@ attn_long_context  the attention entry point alone at L = 4K (the single-layer
           attention workload: 32/8 heads, head_dim 128, K = 32, batch 1),
           8K, 32K and 128K (both views), timed over runs of calls on
           distinct layers' caches that together exceed L2 (K/V from HBM)
+iterative_draft  the same decode step with a two-pass iterative-denoising draft
 train_kernels  the training-side kernels (block-masked attention of a packed
           2048-position sequence with 256 anchor blocks; the forward-KL
           LM-head epilogue over the full vocabulary), each timed alone beside
@@ -58,6 +59,7 @@ sys.path.insert(0, ROOT)
 METRIC = "committed tokens/s (batch 1, Qwen3-8B shape, K=32); dual-view attn HBM GB/s"
 UNIT = "tokens/s"
 P_PROMPT, K_BLOCK, BATCH = 2048, 32, 1
+ITER_STEPS = 20   # decode steps timed with the two-pass iterative draft
 # tokens committed per cycle that this random-init 8B workload gives (the
 # mean accepted length measured on the GPU path, 1.00-1.03 over runs: the
 # random-init diffusion view almost never agrees with the AR view).  Used
@@ -480,7 +482,8 @@ def run_ours(args, rank, world, local_rank):
         s = dataclasses.replace(s, n_layers=2, vocab=32000)
     W, K, T = args.warmup, args.steps, args.temperature
     n_e2e = 0 if args.no_e2e else K
-    max_seq = P_PROMPT + (W + K + n_e2e + 2) * K_BLOCK + K_BLOCK
+    n_iter = 0 if args.profile_small else 3 + ITER_STEPS   # the iterative-draft measurement
+    max_seq = P_PROMPT + (W + K + n_e2e + n_iter + 2) * K_BLOCK + K_BLOCK
     w = synth.make_weights_torch(s, 0, device=dev)
     eng = pkg.Engine(s, w, max_batch=BATCH, max_block=K_BLOCK, max_seq=max_seq, split_tokens=args.split_tokens,
                      page_size=64, device=dev)
@@ -573,6 +576,32 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": e2e_tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": 4 * BATCH,
                "d2h_bytes_per_step": 4 * BATCH * (1 + K_BLOCK), "ms_per_step": e2e_ms / n_e2e}
 
+    # ---------------------------------------------------------------- iterative draft (next row f1)
+    it_line = None
+    if n_iter:
+        n_it = torch.zeros((ITER_STEPS, BATCH), dtype=torch.int32, device=dev)
+
+        def step_it(j):
+            eng.draft_block(anchor, K_BLOCK, T, 1234, out=draft, iterations=2)
+            eng.verify_block(anchor, draft, K_BLOCK, T)
+            eng.commit(anchor, K_BLOCK, T, 1234, n_out=n_it[j], tokens_out=toks)
+
+        for j in range(3):
+            step_it(j)
+        torch.cuda.synchronize()
+        e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2.record()
+        for j in range(ITER_STEPS):
+            step_it(j)
+        e3.record()
+        torch.cuda.synchronize()
+        it_ms = e2.elapsed_time(e3)
+        it_tok = int(n_it.sum())
+        it_line = {"iterations": 2, "steps": ITER_STEPS, "ms_per_step": it_ms / ITER_STEPS,
+                   "value": it_tok / (it_ms * 1e-3), "unit": UNIT,
+                   "how": "the same decode step with a two-pass iterative-denoising draft (the diffusion view "
+                          "re-run on its own drafts), CUDA events around the steps"}
+
     # ---------------------------------------------------------------- reduce
     tot_tokens, max_ms, e2e_sum = reduce_replicas(tokens, ms, e2e["value"] if e2e else 0.0, world, dev)
     if e2e:
@@ -618,6 +647,8 @@ def run_ours(args, rank, world, local_rank):
     }
     if e2e:
         line["e2e"] = e2e
+    if it_line:
+        line["iterative_draft"] = it_line
     if not args.profile_small:
         lc = attn_long_context(hbm, args.split_tokens)
         line["attn_long_context"] = lc
