@@ -25,8 +25,10 @@ attn      the dual-view attention entry point on the single-layer workload
           step, timed like the roofline GEMM; bytes = prefix K/V + Q + O
 attn_long_context  the attention entry point alone at L = 4K (the single-layer
           attention workload: 32/8 heads, head_dim 128, K = 32, batch 1),
-          8K, 32K and 128K (both views), timed over runs of calls on
-          distinct layers' caches that together exceed L2 (K/V from HBM)
+          8K, 32K and 128K (both views), and at batch 4 and 16 for L = 8K
+          and 32K (cells of the long-context sweep), timed over runs of
+          calls on distinct layers' caches that together exceed L2 (K/V
+          from HBM)
 iterative_draft  the same decode step with a two-pass iterative-denoising draft
 train_kernels  the training-side kernels (block-masked attention of a packed
           2048-position sequence with 256 anchor blocks; the forward-KL
@@ -225,10 +227,16 @@ def kernel_traffic(name, sources, key="dram_bytes_per_layer"):
         return None
 
 
-def attn_long_context(hbm, split_tokens, lengths=(4096, 8192, 32768, 131072), reps=5):
+LONG_CONTEXT_BATCHED = ((8192, 4), (8192, 16), (32768, 4), (32768, 16))
+
+
+def attn_long_context(hbm, split_tokens, lengths=(4096, 8192, 32768, 131072), batched=LONG_CONTEXT_BATCHED,
+                      reps=5):
     """The dual-view attention entry point alone (the attention layer shape
-    of the 8B model: 32/8 heads, head_dim 128, block K = 32, batch 1), both
-    views, on N(0,1) bf16 inputs, timed the way a forward meets it: a run of
+    of the 8B model: 32/8 heads, head_dim 128, block K = 32), at batch 1 for
+    each of `lengths` and at the (L, batch) cells of `batched` (every
+    sequence of a batch at prefix L), both views, on N(0,1) bf16 inputs,
+    timed the way a forward meets it: a run of
     calls over n distinct layers' caches, back to back, whose caches
     together exceed 2.5x L2, so every call reads its K/V from HBM (inputs
     larger than L2: no flush) while code and block tables stay where a
@@ -243,22 +251,23 @@ def attn_long_context(hbm, split_tokens, lengths=(4096, 8192, 32768, 131072), re
     K = K_BLOCK
     n_q, n_kv, hd = synth.QWEN3_8B.n_q_heads, synth.QWEN3_8B.n_kv_heads, synth.QWEN3_8B.head_dim
     out = []
-    for L in lengths:
-        byts = (L + K) * n_kv * hd * 2 * 2 + 2 * K * n_q * hd * 2
+    for L, B in [(L, 1) for L in lengths] + list(batched):
+        byts = B * ((L + K) * n_kv * hd * 2 * 2 + 2 * K * n_q * hd * 2)
         nl = max(2, math.ceil(2.5 * 126e6 / byts))
         s = dataclasses.replace(synth.QWEN3_8B, n_layers=nl, hidden=64, ffn=64, vocab=256)
         w = synth.make_weights(s, 0, n_layers=nl)
-        eng = pkg.Engine(s, w, max_batch=1, max_block=K, max_seq=L + K + 64, split_tokens=split_tokens)
+        eng = pkg.Engine(s, w, max_batch=B, max_block=K, max_seq=L + K + 64, split_tokens=split_tokens)
         g = torch.Generator(device="cuda").manual_seed(2)
         for pg in (eng.k_pages, eng.v_pages):
-            pg.copy_(torch.randn(pg.shape, generator=g, device="cuda").to(pg.dtype))
-        q = torch.randn((1, K, n_q, hd), generator=g, device="cuda").to(torch.bfloat16)
-        kb = torch.randn((1, K, n_kv, hd), generator=g, device="cuda").to(torch.bfloat16)
-        vb = torch.randn((1, K, n_kv, hd), generator=g, device="cuda").to(torch.bfloat16)
-        eng.seq_lens[0] = L
+            for i in range(pg.shape[0]):   # one layer at a time: bounded fp32 scratch
+                pg[i].copy_(torch.randn(pg[i].shape, generator=g, device="cuda").to(pg.dtype))
+        q = torch.randn((B, K, n_q, hd), generator=g, device="cuda").to(torch.bfloat16)
+        kb = torch.randn((B, K, n_kv, hd), generator=g, device="cuda").to(torch.bfloat16)
+        vb = torch.randn((B, K, n_kv, hd), generator=g, device="cuda").to(torch.bfloat16)
+        eng.seq_lens[:B] = L
         for mode in (0, 1):
             for layer in range(nl):
-                eng.attention(layer, mode, q, kb, vb, 1, K)
+                eng.attention(layer, mode, q, kb, vb, B, K)
             ms = []
             for _ in range(reps):
                 torch.cuda.synchronize()
@@ -266,12 +275,13 @@ def attn_long_context(hbm, split_tokens, lengths=(4096, 8192, 32768, 131072), re
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record()
                 for layer in range(nl):
-                    eng.attention(layer, mode, q, kb, vb, 1, K)
+                    eng.attention(layer, mode, q, kb, vb, B, K)
                 e1.record()
                 torch.cuda.synchronize()
                 ms.append(e0.elapsed_time(e1) / nl)
             us = statistics.median(ms) * 1e3
-            out.append({"L": L, "view": "draft (mode 1)" if mode else "verify (mode 0)", "us": us, "layers": nl,
+            out.append({"L": L, "batch": B, "view": "draft (mode 1)" if mode else "verify (mode 0)", "us": us,
+                        "layers": nl,
                         "achieved": byts / us / 1e3, "frac": byts / us / 1e3 / hbm})
         assert eng.check_error()[0] == 0
         del eng
@@ -655,7 +665,7 @@ def run_ours(args, rank, world, local_rank):
         # the single-layer attention workload (L = 4096, K = 32, batch 1):
         # its verify-view point is the attn headline, the step's own
         # attention (timed inside the decode step) stays beside it
-        p4 = [p for p in lc["points"] if p["L"] == 4096]
+        p4 = [p for p in lc["points"] if p["L"] == 4096 and p["batch"] == 1]
         if p4:
             v, dv = p4[0], (p4[1] if len(p4) > 1 else None)
             in_step = line["attn"]
@@ -690,7 +700,7 @@ def main():
         return
     if args.profile_attn:
         hbm, _, _ = measured_peaks()
-        res = attn_long_context(hbm, args.split_tokens, lengths=(args.profile_attn,), reps=1)
+        res = attn_long_context(hbm, args.split_tokens, lengths=(args.profile_attn,), batched=(), reps=1)
         print(json.dumps({"profile_case": "attention entry point alone", "attn_long_context": res}), flush=True)
         return
     if world > 1:
