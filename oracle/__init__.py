@@ -7,8 +7,8 @@ imports it, and it never imports the product package.
 The C source follows the paper-notes page on "Orthrus: Memory-Efficient
 Parallel Token Generation via Dual-View Diffusion" (§2.1 dual-view layer,
 §3.2 diffusion mask, §4.1-4.3 the decode cycle and its consensus; §3.1-3.3
-the training-side block mask and forward KL); each C function cites the
-passage it restates.
+the training-side block mask and forward KL; §7.5 / §9.6 tree verification
+of one draft's marginals); each C function cites the passage it restates.
 """
 from __future__ import annotations
 
@@ -110,6 +110,14 @@ def lib():
             l.oc_block_mask_attention.argtypes = [_D, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _D, _D,
                                                   C.c_int, _D, _D, _I, _D]
             l.oc_kl_rows.argtypes = [_D, _D, C.c_int, C.c_int, _F, C.c_int, _D, _D, _D]
+            l.oc_attention_tree.argtypes = [_D, C.c_int, C.c_int, C.c_int, C.c_int, _D, _D, C.c_int, _D, _D, _I,
+                                            _D]
+            l.oc_forward_tree.argtypes = [P(_Cfg), P(_Model), _I, _I, C.c_int, C.c_int, _D, _D, C.c_int, _D]
+            l.oc_tree_build.argtypes = [_D, C.c_int, C.c_int, C.c_int, C.c_int, _I, _I, _I, _D]
+            l.oc_tree_accept.argtypes = [_I, _I, C.c_int, _I, _I, _I]
+            l.oc_tree_commit_kv.argtypes = [_D, _D, C.c_int, C.c_int, C.c_int, C.c_int, _I, C.c_int]
+            l.oc_generate_tree.argtypes = [P(_Cfg), P(_Model), _I, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                           _I, _I, P(C.c_int), _D, _D, P(C.c_int)]
             _lib = l
     return _lib
 
@@ -205,6 +213,54 @@ def kl_rows(hA, hD, W):
     kl, la, ld = np.empty(rows), np.empty(rows), np.empty(rows)
     lib().oc_kl_rows(_dp(hA), _dp(hD), rows, d, _fp(W), W.shape[0], _dp(kl), _dp(la), _dp(ld))
     return kl, la, ld
+
+
+def attention_tree(q, kc, vc, kb, vb, parent):
+    """Tree-masked attention: row r sees the cache and the rows of its own
+    root path (parent[0] = -1, parent[r] < r).  Shapes as attention()."""
+    q, kb, vb, par = _f64(q), _f64(kb), _f64(vb), _i32(parent)
+    R, nq, hd = q.shape
+    nkv = kb.shape[1]
+    t = 0 if kc is None else kc.shape[0]
+    kc = _f64(kc) if t else np.zeros((1, nkv, hd))
+    vc = _f64(vc) if t else np.zeros((1, nkv, hd))
+    o = np.empty_like(q)
+    lib().oc_attention_tree(_dp(q), R, nq, nkv, hd, _dp(kc), _dp(vc), t, _dp(kb), _dp(vb), _ip(par), _dp(o))
+    return o
+
+
+def tree_build(logp, W, N):
+    """Best-first draft tree over logp [D, V] (row d: log-probabilities of
+    the token at depth d + 1), W candidates per depth, N prefixes.  Returns
+    (parent, token, depth, score) of the root plus the chosen nodes, in
+    selection order."""
+    lp = _f64(np.atleast_2d(logp))
+    D, V = lp.shape
+    par, tok, dep = (np.zeros(N + 1, np.int32) for _ in range(3))
+    sc = np.zeros(N + 1)
+    n = lib().oc_tree_build(_dp(lp), D, V, int(W), int(N), _ip(par), _ip(tok), _ip(dep), _dp(sc))
+    if n < 0:
+        raise ValueError(f"oc_tree_build failed: {-n}")
+    return par[:n], tok[:n], dep[:n], sc[:n]
+
+
+def tree_accept(parent, token, g):
+    """Greedy walk of a verified tree: returns (n, emitted tokens, path rows)."""
+    par, tok, g = _i32(parent), _i32(token), _i32(g)
+    R = par.size
+    emit, path = np.zeros(R, np.int32), np.zeros(R, np.int32)
+    n = lib().oc_tree_accept(_ip(par), _ip(tok), R, _ip(g), _ip(emit), _ip(path))
+    return n, emit[:n], path[:n]
+
+
+def tree_commit_kv(kc, vc, t, path):
+    """In place: path row path[i]'s K/V (slot t + path[i]) to slot t + i.
+    kc/vc [n_layers, cap, n_kv, hd] float64 C-contiguous."""
+    assert kc.dtype == np.float64 and kc.flags.c_contiguous and vc.flags.c_contiguous
+    p = _i32(path)
+    nl, cap = kc.shape[:2]
+    kn = int(np.prod(kc.shape[2:]))
+    lib().oc_tree_commit_kv(_dp(kc), _dp(vc), nl, cap, kn, int(t), _ip(p), p.size - 1)
 
 
 def philox4x32_10(ctr, key):
@@ -360,6 +416,40 @@ class Model:
             raise RuntimeError(f"oc_generate failed: {rc}")
         res = {"tokens": out, "n_per_cycle": npc[:cyc.value], "cycles": cyc.value, "min_margin": mg.value,
                "t": tt.value}
+        if want_cache:
+            res["k_cache"], res["v_cache"] = kc, vc
+        return res
+
+    def forward_tree(self, tokens, parent, t, kc, vc):
+        """AR forward of a draft tree (rows = nodes, parent[0] = -1); K/V
+        written at slots t .. t+R-1 of kc/vc (in place).  Returns logits."""
+        tok, par = _i32(tokens), _i32(parent)
+        z = np.empty((tok.size, self.shape.vocab))
+        rc = lib().oc_forward_tree(C.byref(self.cfg), C.byref(self.model), _ip(tok), _ip(par), tok.size, int(t),
+                                   _dp(kc), _dp(vc), kc.shape[1], _dp(z))
+        if rc:
+            raise RuntimeError(f"oc_forward_tree failed: {rc}")
+        return z
+
+    def generate_tree(self, prompt, K, W, nodes, N, want_cache=False):
+        """Greedy decoding with best-first tree verification (W candidates
+        per depth, `nodes` prefixes per cycle).  Returns a dict like
+        generate()."""
+        p = _i32(prompt)
+        out = np.zeros(N, np.int32)
+        npc = np.zeros(N, np.int32)
+        cyc = C.c_int()
+        tt = C.c_int()
+        cap = p.size + N + nodes + 1
+        kc = vc = None
+        if want_cache:
+            kc, vc = self.new_cache(cap)
+        rc = lib().oc_generate_tree(C.byref(self.cfg), C.byref(self.model), _ip(p), p.size, int(K), int(W),
+                                    int(nodes), int(N), _ip(out), _ip(npc), C.byref(cyc), _dp(kc), _dp(vc),
+                                    C.byref(tt))
+        if rc:
+            raise RuntimeError(f"oc_generate_tree failed: {rc}")
+        res = {"tokens": out, "n_per_cycle": npc[:cyc.value], "cycles": cyc.value, "t": tt.value}
         if want_cache:
             res["k_cache"], res["v_cache"] = kc, vc
         return res

@@ -17,7 +17,10 @@
  * training-side pieces follow §3.1-3.3 of the paper-notes page (packed
  * sequences of anchor blocks, the dual-pass block mask, forward KL against
  * the frozen AR view) and the hotdry.top page's training section
- * ("训练策略：双通块掩码与前向 KL 蒸馏").
+ * ("训练策略：双通块掩码与前向 KL 蒸馏").  Tree verification follows the
+ * paper-notes page's §7.5 (DDTree: a best-first tree of the top prefixes of
+ * one diffusion forward's marginals, verified by one tree-attention pass)
+ * and §9.6 (the same proposed for Orthrus's K marginals); greedy only.
  *
  * Arithmetic is fp64 throughout.  Weights arrive as fp32 arrays holding the
  * exact model values (bf16 values are exactly representable in fp32).  Every
@@ -160,6 +163,60 @@ void oc_attention(const double *q, int R, int n_q, int n_kv, int hd,
         }
 }
 
+/*
+ * Tree-masked attention for the verification of a draft tree (the DDTree
+ * comparison of the paper-notes page, §7.5, and its suggestion in §9.6: one
+ * diffusion forward's marginals expanded best-first into a tree that one AR
+ * forward verifies with a tree mask).  Block row r is a tree node; parent[r]
+ * is its parent row (parent[0] = -1: the root, the anchor; 0 <= parent[r] <
+ * r otherwise).  Row r sees cache rows [0, t) and the block rows on its own
+ * root path (its ancestors and itself), in row order.  A chain (parent[r] =
+ * r - 1) is mode 0 of oc_attention key for key.
+ */
+void oc_attention_tree(const double *q, int R, int n_q, int n_kv, int hd,
+                       const double *kc, const double *vc, int t,
+                       const double *kb, const double *vb, const int32_t *parent, double *o)
+{
+    int g = n_q / n_kv;
+    double scale = 1.0 / sqrt((double)hd);
+    #pragma omp parallel for schedule(static) collapse(2) if ((long)R * n_q * (t + R) * hd > 1000000)
+    for (int r = 0; r < R; ++r)
+        for (int h = 0; h < n_q; ++h) {
+            int kvh = h / g;
+            char *on_path = (char *)calloc((size_t)R, 1);
+            for (int a = r; a >= 0; a = parent[a]) on_path[a] = 1;
+            const double *qv = q + ((size_t)r * n_q + h) * hd;
+            double *s = (double *)malloc(sizeof(double) * (size_t)(t + R));
+            double m = -INFINITY;
+            for (int j = 0; j < t + R; ++j) {
+                if (j >= t && !on_path[j - t]) continue;
+                const double *kv = (j < t) ? kc + ((size_t)j * n_kv + kvh) * hd
+                                           : kb + ((size_t)(j - t) * n_kv + kvh) * hd;
+                double d = 0.0;
+                for (int i = 0; i < hd; ++i) d += qv[i] * kv[i];
+                s[j] = d * scale;
+                if (s[j] > m) m = s[j];
+            }
+            double l = 0.0;
+            for (int j = 0; j < t + R; ++j) {
+                if (j >= t && !on_path[j - t]) continue;
+                s[j] = exp(s[j] - m);
+                l += s[j];
+            }
+            double *ov = o + ((size_t)r * n_q + h) * hd;
+            for (int i = 0; i < hd; ++i) ov[i] = 0.0;
+            for (int j = 0; j < t + R; ++j) {
+                if (j >= t && !on_path[j - t]) continue;
+                const double *vv = (j < t) ? vc + ((size_t)j * n_kv + kvh) * hd
+                                           : vb + ((size_t)(j - t) * n_kv + kvh) * hd;
+                double p = s[j] / l;
+                for (int i = 0; i < hd; ++i) ov[i] += p * vv[i];
+            }
+            free(s);
+            free(on_path);
+        }
+}
+
 /* ------------------------------------------------------------------------ */
 /* One forward of either view over a block of R rows.                         */
 /* ------------------------------------------------------------------------ */
@@ -177,10 +234,41 @@ void oc_attention(const double *q, int R, int n_q, int n_kv, int hd,
  * logits [R][vocab] and final_hidden [R][hidden] (after the final norm) may
  * be NULL.
  */
+static int forward_rows(const oc_cfg *c, const oc_model *w, int view, int mode,
+                        const int32_t *tokens, const int32_t *parent, int R, int t,
+                        double *kc, double *vc, int cap,
+                        double *logits, double *final_hidden);
+
 int oc_forward(const oc_cfg *c, const oc_model *w, int view, int mode,
                const int32_t *tokens, int R, int t,
                double *kc, double *vc, int cap,
                double *logits, double *final_hidden)
+{
+    return forward_rows(c, w, view, mode, tokens, NULL, R, t, kc, vc, cap, logits, final_hidden);
+}
+
+/*
+ * AR forward of a draft tree (paper notes §7.5 / §9.6, tree verification):
+ * row r is a node with token tokens[r] and parent parent[r] (see
+ * oc_attention_tree), at position t + depth(r) (depth(0) = 0, depth(r) =
+ * depth(parent[r]) + 1); the rows' K/V are written into cache slots t ..
+ * t+R-1 in row order and every row attends to the cache and its own root
+ * path.  A node's logits are those of a plain causal forward of its root
+ * path.
+ */
+int oc_forward_tree(const oc_cfg *c, const oc_model *w, const int32_t *tokens, const int32_t *parent, int R,
+                    int t, double *kc, double *vc, int cap, double *logits)
+{
+    if (!parent || R <= 0 || parent[0] != -1) return OC_ERR_ARG;
+    for (int r = 1; r < R; ++r)
+        if (parent[r] < 0 || parent[r] >= r) return OC_ERR_ARG;
+    return forward_rows(c, w, 0, 0, tokens, parent, R, t, kc, vc, cap, logits, NULL);
+}
+
+static int forward_rows(const oc_cfg *c, const oc_model *w, int view, int mode,
+                        const int32_t *tokens, const int32_t *parent, int R, int t,
+                        double *kc, double *vc, int cap,
+                        double *logits, double *final_hidden)
 {
     if (!c || !w || !tokens || R <= 0 || t < 0 || (view != 0 && view != 1) || (mode != 0 && mode != 1))
         return OC_ERR_ARG;
@@ -201,8 +289,11 @@ int oc_forward(const oc_cfg *c, const oc_model *w, int view, int mode,
     double *y = calloc((size_t)R * d, sizeof(double));
     double *gt = calloc((size_t)R * F, sizeof(double));
     double *up = calloc((size_t)R * F, sizeof(double));
+    int *pos = calloc((size_t)R, sizeof(int));
     int rc = OC_OK;
-    if (!h || !a || !q || !k || !v || !o || !y || !gt || !up) { rc = OC_ERR_NOMEM; goto done; }
+    if (!h || !a || !q || !k || !v || !o || !y || !gt || !up || !pos) { rc = OC_ERR_NOMEM; goto done; }
+    for (int r = 0; r < R; ++r)   /* a chain sits at t + r; a tree node one past its parent */
+        pos[r] = !parent ? t + r : (r == 0 ? t : pos[parent[r]] + 1);
 
     for (int r = 0; r < R; ++r)
         for (int i = 0; i < d; ++i) h[(size_t)r * d + i] = (double)w->embed[(size_t)tokens[r] * d + i];
@@ -215,13 +306,16 @@ int oc_forward(const oc_cfg *c, const oc_model *w, int view, int mode,
         oc_linear(a, R, d, view ? L->wk_diff : L->wk, nkv * hd, k);
         oc_linear(a, R, d, view ? L->wv_diff : L->wv, nkv * hd, v);
         for (int r = 0; r < R; ++r) {
-            oc_rope(q + r * qn, nq, hd, t + r, c->rope_theta);
-            oc_rope(k + r * kn, nkv, hd, t + r, c->rope_theta);
+            oc_rope(q + r * qn, nq, hd, pos[r], c->rope_theta);
+            oc_rope(k + r * kn, nkv, hd, pos[r], c->rope_theta);
         }
         if (mode == 0) {
             memcpy(kcl + (size_t)t * kn, k, sizeof(double) * R * kn);
             memcpy(vcl + (size_t)t * kn, v, sizeof(double) * R * kn);
-            oc_attention(q, R, nq, nkv, hd, kcl, vcl, t, kcl + (size_t)t * kn, vcl + (size_t)t * kn, 0, o);
+            if (parent)
+                oc_attention_tree(q, R, nq, nkv, hd, kcl, vcl, t, kcl + (size_t)t * kn, vcl + (size_t)t * kn, parent, o);
+            else
+                oc_attention(q, R, nq, nkv, hd, kcl, vcl, t, kcl + (size_t)t * kn, vcl + (size_t)t * kn, 0, o);
         } else {
             oc_attention(q, R, nq, nkv, hd, kcl, vcl, t, k, v, 1, o);
         }
@@ -238,7 +332,7 @@ int oc_forward(const oc_cfg *c, const oc_model *w, int view, int mode,
     if (final_hidden) memcpy(final_hidden, a, sizeof(double) * R * d);
     if (logits) oc_linear(a, R, d, w->lm_head, V, logits);
 done:
-    free(h); free(a); free(q); free(k); free(v); free(o); free(y); free(gt); free(up);
+    free(h); free(a); free(q); free(k); free(v); free(o); free(y); free(gt); free(up); free(pos);
     return rc;
 }
 
@@ -968,4 +1062,215 @@ void oc_kl_rows(const double *hA, const double *hD, int rows, int d, const float
         free(zA);
         free(zD);
     }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Tree verification (paper notes §7.5 and §9.6: DDTree's best-first tree    */
+/* over one diffusion forward's marginals, verified by one tree-masked AR    */
+/* forward).  Greedy (T = 0) only: the pages give no sampling rule for it.   */
+/* ------------------------------------------------------------------------ */
+
+/* Lexicographic order of rank sequences, a prefix before its extensions. */
+static int rankseq_less(const int32_t *a, int la, const int32_t *b, int lb)
+{
+    for (int i = 0; i < la && i < lb; ++i)
+        if (a[i] != b[i]) return a[i] < b[i];
+    return la < lb;
+}
+
+/*
+ * Best-first draft tree.  logp [D][V]: log-probabilities of the token at
+ * depth d + 1 (the draft row d's distribution at T = 1).  At every depth
+ * the candidates are the W most probable ids of that row (ties: lowest id),
+ * ranked 0 .. W-1.  A prefix y_1 .. y_d scores sum_i logp[i-1][y_i]; the
+ * tree is the root (the anchor, row 0) plus the N best prefixes of depth
+ * 1 .. D, ordered by score and then by their rank sequences (so a prefix
+ * always precedes its extensions, and the chosen set is closed under
+ * prefixes).  They are found the best-first way: a pool holding, for every
+ * chosen node, its best child and its next sibling, from which the best
+ * entry is taken N times.  Outputs (N + 1 rows, in selection order, so a
+ * parent's row is below its children's): parent (-1 for the root), token
+ * (-1 for the root), depth, score.  Returns the number of rows (fewer than
+ * N + 1 when fewer prefixes exist), or -OC_ERR_* on bad arguments.
+ */
+int oc_tree_build(const double *logp, int D, int V, int W, int N, int32_t *parent, int32_t *token,
+                  int32_t *depth, double *score)
+{
+    if (D < 0 || V < 1 || W < 1 || W > V || N < 0 || !parent || !token || !depth || !score) return -OC_ERR_ARG;
+    if (D > 0 && !logp) return -OC_ERR_ARG;
+    int32_t *cand = malloc(sizeof(int32_t) * (size_t)(D > 0 ? D : 1) * W);   /* [D][W] ranked ids */
+    int32_t *rseq = malloc(sizeof(int32_t) * (size_t)(N + 1) * (D > 0 ? D : 1));   /* node rank sequences */
+    int pool_cap = 2 * N + 2;
+    int32_t *pp = malloc(sizeof(int32_t) * pool_cap), *pr = malloc(sizeof(int32_t) * pool_cap);
+    double *ps = malloc(sizeof(double) * pool_cap);
+    int32_t *tmp = malloc(sizeof(int32_t) * (size_t)(D > 0 ? D : 1) + sizeof(int32_t));
+    int32_t *tmp2 = malloc(sizeof(int32_t) * (size_t)(D > 0 ? D : 1) + sizeof(int32_t));
+    if (!cand || !rseq || !pp || !pr || !ps || !tmp || !tmp2) {
+        free(cand); free(rseq); free(pp); free(pr); free(ps); free(tmp); free(tmp2);
+        return -OC_ERR_NOMEM;
+    }
+    for (int d = 0; d < D; ++d) {   /* W rounds of "largest not yet taken, lowest id on ties" */
+        const double *row = logp + (size_t)d * V;
+        for (int r = 0; r < W; ++r) {
+            int best = -1;
+            for (int v = 0; v < V; ++v) {
+                int taken = 0;
+                for (int u = 0; u < r; ++u) taken |= cand[d * W + u] == v;
+                if (!taken && (best < 0 || row[v] > row[best])) best = v;
+            }
+            cand[d * W + r] = best;
+        }
+    }
+    parent[0] = -1; token[0] = -1; depth[0] = 0; score[0] = 0.0;
+    int n = 1, np = 0;
+    if (D > 0 && N > 0) { pp[0] = 0; pr[0] = 0; ps[0] = logp[cand[0]]; np = 1; }
+    while (n <= N && np > 0) {
+        /* the best pool entry: largest score, then smallest rank sequence */
+        int bi = 0;
+        for (int i = 1; i < np; ++i) {
+            if (ps[i] > ps[bi]) { bi = i; continue; }
+            if (ps[i] < ps[bi]) continue;
+            int li = depth[pp[i]] + 1, lb = depth[pp[bi]] + 1;
+            memcpy(tmp, rseq + (size_t)pp[i] * D, sizeof(int32_t) * (li - 1)); tmp[li - 1] = pr[i];
+            memcpy(tmp2, rseq + (size_t)pp[bi] * D, sizeof(int32_t) * (lb - 1)); tmp2[lb - 1] = pr[bi];
+            if (rankseq_less(tmp, li, tmp2, lb)) bi = i;
+        }
+        const int par = pp[bi], rk = pr[bi];
+        const double sc = ps[bi];
+        pp[bi] = pp[np - 1]; pr[bi] = pr[np - 1]; ps[bi] = ps[np - 1]; --np;
+        const int d = depth[par] + 1;
+        parent[n] = par; depth[n] = d; score[n] = sc; token[n] = cand[(d - 1) * W + rk];
+        memcpy(rseq + (size_t)n * D, rseq + (size_t)par * D, sizeof(int32_t) * (d - 1));
+        rseq[(size_t)n * D + d - 1] = rk;
+        if (rk + 1 < W) {   /* next sibling */
+            pp[np] = par; pr[np] = rk + 1; ps[np] = score[par] + logp[(size_t)(d - 1) * V + cand[(d - 1) * W + rk + 1]];
+            ++np;
+        }
+        if (d < D) {   /* best child */
+            pp[np] = n; pr[np] = 0; ps[np] = sc + logp[(size_t)d * V + cand[d * W]];
+            ++np;
+        }
+        ++n;
+    }
+    free(cand); free(rseq); free(pp); free(pr); free(ps); free(tmp); free(tmp2);
+    return n;
+}
+
+/*
+ * Greedy acceptance on a verified tree: from the root, follow the child
+ * whose token equals the AR argmax g of the current node while one exists
+ * (siblings hold distinct tokens); emit the followed tokens and then g of
+ * the last node reached.  path[0 .. m] = the rows of the accepted root path
+ * (path[0] = 0); emit[0 .. m] the tokens.  Returns n = m + 1 in [1, depth
+ * + 1].  A chain reduces to oc_consensus_greedy.
+ */
+int oc_tree_accept(const int32_t *parent, const int32_t *token, int R, const int32_t *g, int32_t *emit,
+                   int32_t *path)
+{
+    int cur = 0, m = 0;
+    path[0] = 0;
+    for (;;) {
+        int next = -1;
+        for (int c = cur + 1; c < R && next < 0; ++c)
+            if (parent[c] == cur && token[c] == g[cur]) next = c;
+        if (next < 0) break;
+        emit[m++] = token[next];
+        path[m] = next;
+        cur = next;
+    }
+    emit[m] = g[cur];
+    return m + 1;
+}
+
+/* Commit of an accepted tree path: the K/V of path row path[i] (cache slot
+ * t + path[i]) move to slot t + i, for i = 1 .. m, in every layer.  path[i]
+ * >= i and increasing, so ascending i never overwrites a slot still to be
+ * read. */
+void oc_tree_commit_kv(double *kc, double *vc, int n_layers, int cap, int kn, int t, const int32_t *path, int m)
+{
+    for (int l = 0; l < n_layers; ++l) {
+        double *kl = kc + (size_t)l * cap * kn, *vl = vc + (size_t)l * cap * kn;
+        for (int i = 1; i <= m; ++i) {
+            memmove(kl + (size_t)(t + i) * kn, kl + (size_t)(t + path[i]) * kn, sizeof(double) * kn);
+            memmove(vl + (size_t)(t + i) * kn, vl + (size_t)(t + path[i]) * kn, sizeof(double) * kn);
+        }
+    }
+}
+
+/*
+ * Greedy decoding with tree verification: every cycle one diffusion draft
+ * of K rows (oc_draft at T = 0), log-softmax of its rows 0 .. K-2 (the
+ * tokens at depths 1 .. K-1), a best-first tree of `nodes` prefixes with W
+ * candidates per depth, one tree-masked AR forward of the root plus the
+ * nodes, oc_tree_accept and the K/V compaction; the committed length grows
+ * by n.  With W = 1 and nodes = K - 1 the tree is the draft chain and every
+ * cycle equals oc_generate's.  out / n_per_cycle / cycles / t as there;
+ * kc_out, vc_out (may be NULL): the cache, rows >= t zeroed, with capacity
+ * P + N + nodes + 1.
+ */
+int oc_generate_tree(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P, int K, int W, int nodes,
+                     int N, int32_t *out, int32_t *n_per_cycle, int *n_cycles, double *kc_out, double *vc_out,
+                     int *t_out)
+{
+    if (!c || !w || !prompt || P < 1 || N < 1 || K < 1 || W < 1 || W > c->vocab || nodes < 0) return OC_ERR_ARG;
+    const int V = c->vocab, D = K - 1;
+    const int cap = P + N + nodes + 1;
+    const size_t kn = (size_t)c->n_kv_heads * c->head_dim;
+    const size_t csz = (size_t)c->n_layers * cap * kn;
+    double *kc = calloc(csz, sizeof(double)), *vc = calloc(csz, sizeof(double));
+    int32_t *draft = malloc(sizeof(int32_t) * K);
+    double *z = malloc(sizeof(double) * (size_t)K * V);
+    double *lp = malloc(sizeof(double) * (size_t)(D > 0 ? D : 1) * V);
+    int32_t *par = malloc(sizeof(int32_t) * (nodes + 1)), *tok = malloc(sizeof(int32_t) * (nodes + 1));
+    int32_t *dep = malloc(sizeof(int32_t) * (nodes + 1)), *g = malloc(sizeof(int32_t) * (nodes + 1));
+    int32_t *emit = malloc(sizeof(int32_t) * (nodes + 1)), *path = malloc(sizeof(int32_t) * (nodes + 1));
+    double *sc = malloc(sizeof(double) * (nodes + 1));
+    double *zt = malloc(sizeof(double) * (size_t)(nodes + 1) * V);
+    int rc = OC_OK;
+    if (!kc || !vc || !draft || !z || !lp || !par || !tok || !dep || !g || !emit || !path || !sc || !zt) {
+        rc = OC_ERR_NOMEM;
+        goto done;
+    }
+    int t = oc_prefill(c, w, prompt, P, kc, vc, cap);
+    if (t < 0) { rc = -t; goto done; }
+    int32_t anchor = prompt[P - 1];
+    int produced = 0, cycles = 0;
+    while (produced < N) {
+        rc = oc_draft(c, w, kc, vc, cap, t, anchor, K, 0.0, 0, 0, draft, NULL, z, NULL);
+        if (rc) goto done;
+        for (int d = 0; d < D; ++d) {   /* log-softmax at T = 1 */
+            const double *zr = z + (size_t)d * V;
+            double m = -INFINITY, s = 0.0;
+            for (int v = 0; v < V; ++v) if (zr[v] > m) m = zr[v];
+            for (int v = 0; v < V; ++v) s += exp(zr[v] - m);
+            for (int v = 0; v < V; ++v) lp[(size_t)d * V + v] = zr[v] - m - log(s);
+        }
+        const int R = oc_tree_build(lp, D, V, W, nodes, par, tok, dep, sc);
+        if (R < 0) { rc = -R; goto done; }
+        tok[0] = anchor;
+        rc = oc_forward_tree(c, w, tok, par, R, t, kc, vc, cap, zt);
+        if (rc) goto done;
+        for (int r = 0; r < R; ++r) g[r] = oc_argmax(zt + (size_t)r * V, V, NULL);
+        const int n = oc_tree_accept(par, tok, R, g, emit, path);
+        oc_tree_commit_kv(kc, vc, c->n_layers, cap, (int)kn, t, path, n - 1);
+        t += n;
+        anchor = emit[n - 1];
+        for (int i = 0; i < n && produced < N; ++i) out[produced++] = emit[i];
+        if (n_per_cycle) n_per_cycle[cycles] = n;
+        ++cycles;
+    }
+    if (n_cycles) *n_cycles = cycles;
+    if (t_out) *t_out = t;
+    if (kc_out || vc_out) {
+        for (int l = 0; l < c->n_layers; ++l) {
+            memset(kc + ((size_t)l * cap + t) * kn, 0, sizeof(double) * (size_t)(cap - t) * kn);
+            memset(vc + ((size_t)l * cap + t) * kn, 0, sizeof(double) * (size_t)(cap - t) * kn);
+        }
+        if (kc_out) memcpy(kc_out, kc, sizeof(double) * csz);
+        if (vc_out) memcpy(vc_out, vc, sizeof(double) * csz);
+    }
+done:
+    free(kc); free(vc); free(draft); free(z); free(lp); free(par); free(tok); free(dep); free(g); free(emit);
+    free(path); free(sc); free(zt);
+    return rc;
 }
