@@ -344,29 +344,37 @@ __global__ void set_lens_kernel(int32_t *seq_lens, int b, int value, int32_t *an
 
 // Block K/V given as [B][K][n_kv][hd] -> K [B][n_kv][kp][hd] and V transposed
 // [B][n_kv][hd][kp] (rows K .. kp-1 zero).  Grid (n_kv, B, kp / 16), 256
-// threads: 16 rows x 16 runs of 8 dims, every load of a thread in flight at
-// once.
+// threads, 16 rows per CTA: K is copied row by row, V is staged in shared
+// memory and written out a dim at a time (16 consecutive rows), so the
+// loads and stores of a warp touch consecutive elements; every load of a
+// thread is in flight at once (hd <= 128).
 template <class T>
-__global__ void pack_block_kernel(const T *ks, const T *vs, T *kd, T *vd, int K, int kp, int n_kv, int hd)
+__global__ void __launch_bounds__(256) pack_block_kernel(const T *__restrict__ ks, const T *__restrict__ vs,
+                                                         T *__restrict__ kd, T *__restrict__ vd, int K, int kp,
+                                                         int n_kv, int hd)
 {
+    constexpr int kRows = 16;
+    constexpr int kPad = 4 / (int)sizeof(T);   // a 32-bit word per row: a column read walks the banks
+    __shared__ T tile[kRows][128 + kPad];
     pdl_trigger();
     pdl_wait();
-    const int b = blockIdx.y, kvh = blockIdx.x;
-    const int k = blockIdx.z * 16 + (int)threadIdx.x / 16, d0 = ((int)threadIdx.x % 16) * 8;
-    if (k >= kp || d0 >= hd) return;
-    const T z = from_f<T>(0.f);
-    T kv[8], vv[8];
-    const size_t src = (((size_t)b * K + k) * n_kv + kvh) * hd + d0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        kv[e] = k < K ? ks[src + e] : z;
-        vv[e] = k < K ? vs[src + e] : z;
-    }
+    const int kvh = blockIdx.x, b = blockIdx.y, k0 = blockIdx.z * kRows;
     const size_t head = (size_t)b * n_kv + kvh;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        kd[(head * kp + k) * hd + d0 + e] = kv[e];
-        vd[(head * hd + d0 + e) * kp + k] = vv[e];
+    const T z = from_f<T>(0.f);
+    const int n = kRows * hd;
+#pragma unroll 8
+    for (int i = threadIdx.x; i < n; i += 256) {
+        const int r = i / hd, d = i % hd, k = k0 + r;
+        const size_t src = (((size_t)b * K + k) * n_kv + kvh) * hd + d;
+        const bool in = k < K;
+        kd[(head * kp + k) * hd + d] = in ? ks[src] : z;
+        tile[r][d] = in ? vs[src] : z;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int i = threadIdx.x; i < n; i += 256) {
+        const int d = i / kRows, r = i % kRows;
+        vd[(head * hd + d) * kp + k0 + r] = tile[r][d];
     }
 }
 
@@ -550,7 +558,8 @@ cudaError_t launch_pack_block(const Ctx &c, const void *k_src, const void *v_src
                               int K, int kp, cudaStream_t s)
 {
     c.launches += 1;
-    const dim3 grid(c.cfg.n_kv_heads, B, (kp + 15) / 16);
+    if (kp % 16 || c.cfg.head_dim > 128) return cudaErrorInvalidValue;
+    const dim3 grid(c.cfg.n_kv_heads, B, kp / 16);
     if (c.cfg.dtype == ORTHRUS_BF16)
         return launch_k(pack_block_kernel<bf16>, grid, 256, 0, s, (const bf16 *)k_src, (const bf16 *)v_src,
                         (bf16 *)k_dst, (bf16 *)v_dst, K, kp, c.cfg.n_kv_heads, c.cfg.head_dim);

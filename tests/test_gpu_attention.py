@@ -19,9 +19,9 @@ def eng():
     return attention_engine()
 
 
-def _case(eng, ts, K, mode, seed=2, tag=""):
-    """ts: committed length per sequence.  Returns max-abs error over all
-    sequences and the GPU output."""
+def _case(eng, ts, K, mode, seed=2, tag="", check=None):
+    """ts: committed length per sequence.  Returns max-abs error over the
+    sequences in `check` (default all) and the GPU output."""
     B = len(ts)
     nq, nkv, hd = 32, 8, 128
     q = bf16_normal((B, K, nq, hd), seed, f"q{tag}")
@@ -42,6 +42,8 @@ def _case(eng, ts, K, mode, seed=2, tag=""):
     assert st == 0, bits
     err = 0.0
     for b, t in enumerate(ts):
+        if check is not None and b not in check:
+            continue
         ref = oracle.attention(q[b], kcs[b] if t else None, vcs[b] if t else None, kb[b], vb[b], mode)
         err = max(err, float(np.abs(out[b] - ref).max()))
     return err, out
@@ -65,6 +67,24 @@ def test_edges(eng, mode, t, K):
 @pytest.mark.parametrize("mode", [0, 1])
 def test_ragged_batch(eng, mode):
     err, _ = _case(eng, [100, 1000, 257], 16, mode, tag="rag")
+    assert err <= TOL, err
+
+
+@pytest.fixture(scope="module")
+def eng16():
+    e = attention_engine(max_batch=16, max_seq=8192 + 32 + 64, split_tokens=128)
+    yield e
+    del e
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_batch16_long_context(eng16, mode):
+    """The benchmark's batched long-context cell in its launch configuration:
+    16 sequences at L = 8192 with K = 32 (split 128: one CTA per sequence
+    and KV head); the first, a middle and the last sequence are checked
+    against the oracle, so a per-sequence offset error shows."""
+    err, _ = _case(eng16, [8192] * 16, 32, mode, tag="b16", check=(0, 7, 15))
     assert err <= TOL, err
 
 
