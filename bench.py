@@ -90,6 +90,10 @@ def parse():
                     help="small case for ncu captures of the attention kernel: the attention entry point "
                          "alone at prefix length L (both views, 2 calls each); its line is marked "
                          "profile_case and is not a bench result")
+    ap.add_argument("--profile-train", action="store_true",
+                    help="small case for ncu captures of the training-side kernels: train_kernels alone (one "
+                         "timed call each, no CPU oracle) on a one-layer engine with the 8B LM head; its line "
+                         "is marked profile_case and is not a bench result")
     a = ap.parse_args()
     if a.profile_small:
         a.steps, a.warmup, a.no_cpu_baseline, a.no_e2e = 2, 1, True, True
@@ -313,7 +317,7 @@ def _timed(fn, reps):
     return statistics.median(ms) * 1e3
 
 
-def train_kernels(hbm, tflops, eng, reps=10):
+def train_kernels(hbm, tflops, eng, reps=10, cpu=True):
     """The training-side kernels of the pages (§3.1-3.3), each timed alone
     (median of reps; each reads more than L2 holds: 176 MB of queries,
     outputs and K/V, and the 1.24 GB head) beside the CPU oracle on a sample.
@@ -322,7 +326,9 @@ def train_kernels(hbm, tflops, eng, reps=10):
     attention shape, N(0,1) bf16; bound tensor: useful FLOPs = 4 hd x the
     keys each (row, query head) sees.  kl_lm_head: 16 row pairs (N(0, 3^2)
     bf16 hidden rows, diffusion = AR + N(0, 1.8^2)) through the 8B LM head
-    (151936 x 4096, the decode engine's); bound HBM: the head's bytes + rows."""
+    (151936 x 4096, the decode engine's, or a one-layer engine's when eng is
+    None); bound HBM: the head's bytes + rows.  cpu=False skips the oracle
+    samples."""
     import numpy as np
     import torch
     import oracle
@@ -346,44 +352,63 @@ def train_kernels(hbm, tflops, eng, reps=10):
     us = _timed(lambda: ae.block_mask_attention(0, q, kb, vb, ad, K), reps)
     flops = float(4 * hd * K * n_q * (anchors.astype(np.int64) + K).sum())
     byts = 2 * nb * K * n_q * hd * 2 + 2 * nb * K * n_kv * hd * 2 + 2 * L * n_kv * hd * 2
-    t0 = time.perf_counter()
-    qh, kbh, vbh = (x.float().cpu().numpy() for x in (q[:2], kb[:2], vb[:2]))
-    kc = ae.k_pages[0, :L // ae.page_size].float().permute(0, 2, 1, 3).reshape(L, n_kv, hd).cpu().numpy()
-    vc = ae.v_pages[0, :L // ae.page_size].float().permute(0, 3, 1, 2).reshape(L, n_kv, hd).cpu().numpy()
-    t_prep = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    for b in range(2):
-        oracle.block_mask_attention(qh[b], kc, vc, kbh[b], vbh[b], anchors[b:b + 1], K)
-    t_cpu = (time.perf_counter() - t0) / float(anchors[:2].astype(np.int64).sum() + 2 * K) * \
-        float(anchors.astype(np.int64).sum() + nb * K)
     ach = flops / us / 1e6
     out["block_mask_attention"] = {
         "workload": "256 anchor blocks x K=32 in one packed 2048-position sequence, 32/8 heads, head_dim 128",
         "us": us, "bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s", "frac": ach / tflops,
         "hbm_gbs": byts / us / 1e3, "algorithmic_flops": flops, "algorithmic_bytes": byts,
-        "cpu_baseline": {"seconds": t_cpu, "cores": OracleSample.threads(), "kind": "oracle",
-                         "sample": "2 of the 256 blocks, scaled by visible keys"}}
+        "ncu_dram_bytes_first_launch": kernel_traffic("block_mask_attention_training.txt", ATTN_SOURCES,
+                                                      "dram_bytes_per_launch")}
+    if cpu:
+        _block_mask_cpu(out["block_mask_attention"], ae, q, kb, vb, anchors, nb, K, L)
     del ae
     torch.cuda.empty_cache()
     # ---- forward-KL LM head on the decode engine's 8B head
+    own = eng is None
+    if own:
+        s8 = dataclasses.replace(synth.QWEN3_8B, n_layers=1)
+        eng = pkg.Engine(s8, synth.make_weights_torch(s8, 0, n_layers=1), max_batch=1, max_block=K_BLOCK,
+                         max_seq=256, split_tokens=128)
     rows, d, V = 16, eng.shape.hidden, eng.shape.vocab
     gk = torch.Generator(device="cuda").manual_seed(5)
     hA = (3.0 * torch.randn((rows, d), generator=gk, device="cuda")).to(torch.bfloat16)
     hD = (hA.float() + 1.8 * torch.randn((rows, d), generator=gk, device="cuda")).to(torch.bfloat16)
     us = _timed(lambda: eng.kl_lm_head(hA, hD), reps)
     byts = V * d * 2 + 2 * rows * d * 2 + rows * 12
-    Vs = 8192
-    Wh = eng.lm_head[:Vs].float().cpu().numpy()
-    t0 = time.perf_counter()
-    oracle.kl_rows(hA[:1].float().cpu().numpy(), hD[:1].float().cpu().numpy(), Wh)
-    t_cpu = (time.perf_counter() - t0) * rows * V / Vs
     ach = byts / us / 1e3
     out["kl_lm_head"] = {
         "workload": "16 row pairs through the 151936 x 4096 LM head", "us": us, "bound": "hbm",
         "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "algorithmic_bytes": byts,
-        "cpu_baseline": {"seconds": t_cpu, "cores": OracleSample.threads(), "kind": "oracle",
-                         "sample": f"1 row pair over the first {Vs} vocabulary ids, scaled"}}
+        "traffic": kernel_traffic("kl_lm_head_qwen3_8b_head.txt", GEMM_SOURCES, "dram_bytes_per_launch")}
+    if cpu:
+        Vs = 8192
+        Wh = eng.lm_head[:Vs].float().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.kl_rows(hA[:1].float().cpu().numpy(), hD[:1].float().cpu().numpy(), Wh)
+        t_cpu = (time.perf_counter() - t0) * rows * V / Vs
+        out["kl_lm_head"]["cpu_baseline"] = {"seconds": t_cpu, "cores": OracleSample.threads(), "kind": "oracle",
+                                             "sample": f"1 row pair over the first {Vs} vocabulary ids, scaled"}
+    if own:
+        del eng
+        torch.cuda.empty_cache()
     return out
+
+
+def _block_mask_cpu(rec, ae, q, kb, vb, anchors, nb, K, L):
+    """The oracle on 2 of the blocks, scaled by visible keys to all of them."""
+    import numpy as np
+    import oracle
+    n_kv, hd = ae.shape.n_kv_heads, ae.shape.head_dim
+    qh, kbh, vbh = (x.float().cpu().numpy() for x in (q[:2], kb[:2], vb[:2]))
+    kc = ae.k_pages[0, :L // ae.page_size].float().permute(0, 2, 1, 3).reshape(L, n_kv, hd).cpu().numpy()
+    vc = ae.v_pages[0, :L // ae.page_size].float().permute(0, 3, 1, 2).reshape(L, n_kv, hd).cpu().numpy()
+    t0 = time.perf_counter()
+    for b in range(2):
+        oracle.block_mask_attention(qh[b], kc, vc, kbh[b], vbh[b], anchors[b:b + 1], K)
+    t_cpu = (time.perf_counter() - t0) / float(anchors[:2].astype(np.int64).sum() + 2 * K) * \
+        float(anchors.astype(np.int64).sum() + nb * K)
+    rec["cpu_baseline"] = {"seconds": t_cpu, "cores": OracleSample.threads(), "kind": "oracle",
+                           "sample": "2 of the 256 blocks, scaled by visible keys"}
 
 
 # ----------------------------------------------------------------- oracle sample
@@ -697,6 +722,11 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.profile_train:
+        hbm, tflops, _ = measured_peaks()
+        res = train_kernels(hbm, tflops, None, reps=1, cpu=False)
+        print(json.dumps({"profile_case": "training-side kernels alone", "train_kernels": res}), flush=True)
         return
     if args.profile_attn:
         hbm, _, _ = measured_peaks()
