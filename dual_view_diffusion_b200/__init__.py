@@ -85,6 +85,9 @@ _SIGS = {
     "orthrus_dual_view_attention": [_P, C.POINTER(KV), _I, _I, _P, _P, _P, _I, _I, _P, _P],
     "orthrus_block_mask_attention": [_P, C.POINTER(KV), _I, _P, _P, _P, _P, _I, _I, _P, _P],
     "orthrus_kl_lm_head": [_P, _P, _P, _I, _P, _P, _P, _P],
+    "orthrus_tree_topw": [_P, _P, _I, _I, _P, _P, _P, _P],
+    "orthrus_tree_build": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P],
+    "orthrus_tree_commit": [_P, C.POINTER(KV), _I, _I, _P, _P, _P, _P, _P, _P, _P, _P],
     "orthrus_debug_logits": [_P, _I, _I, _I, _P, _P],
     "orthrus_check_error": [_P, _P, C.POINTER(C.c_uint32)],
     "orthrus_set_probe": [_P, _I, _I, _I, C.POINTER(_P), C.POINTER(_P), _I],
@@ -329,6 +332,45 @@ class Engine:
         _check("orthrus_kl_lm_head", lib().orthrus_kl_lm_head(
             self.ctx, _ptr(h_ar), _ptr(h_diff), rows, _ptr(kl), _ptr(la), _ptr(ld), _stream()))
         return kl, la, ld
+
+    def tree_topw(self, logits, width):
+        """The `width` best ids and logits of each fp32 logits row, and the
+        row's log-sum-exp: (ids int32 [rows, width], vals fp32, lse fp32)."""
+        t = self.torch
+        z = logits.reshape(-1, logits.shape[-1])
+        rows = int(z.shape[0])
+        ids = t.empty((rows, width), dtype=t.int32, device=self.device)
+        vals = t.empty((rows, width), dtype=t.float32, device=self.device)
+        lse = t.empty(rows, dtype=t.float32, device=self.device)
+        _check("orthrus_tree_topw", lib().orthrus_tree_topw(self.ctx, _ptr(z), rows, width, _ptr(ids), _ptr(vals),
+                                                            _ptr(lse), _stream()))
+        return ids, vals, lse
+
+    def tree_build(self, ids, vals, lse, nodes):
+        """Best-first draft trees from per-depth candidates ids/vals [B, D, W]
+        and lse [B, D]: (parent, token, depth, score [B, nodes + 1], n_rows [B])."""
+        t = self.torch
+        B, D, W = (int(x) for x in ids.shape)
+        par, tok, dep = (t.empty((B, nodes + 1), dtype=t.int32, device=self.device) for _ in range(3))
+        sc = t.empty((B, nodes + 1), dtype=t.float64, device=self.device)
+        nr = t.empty(B, dtype=t.int32, device=self.device)
+        _check("orthrus_tree_build", lib().orthrus_tree_build(
+            self.ctx, _ptr(ids), _ptr(vals), _ptr(lse), B, D, W, nodes, _ptr(par), _ptr(tok), _ptr(dep), _ptr(sc),
+            _ptr(nr), _stream()))
+        return par, tok, dep, sc, nr
+
+    def tree_commit(self, parent, token, n_rows, g, anchor):
+        """Greedy acceptance on verified trees [B, rows] and the commit of the
+        accepted paths' K/V; anchor [B] is updated in place.  Returns
+        (n [B], emitted tokens [B, rows])."""
+        t = self.torch
+        B, R = (int(x) for x in parent.shape)
+        n = t.empty(B, dtype=t.int32, device=self.device)
+        emit = t.full((B, R), -1, dtype=t.int32, device=self.device)
+        _check("orthrus_tree_commit", lib().orthrus_tree_commit(
+            self.ctx, C.byref(self.kv), B, R, _ptr(parent), _ptr(token), _ptr(n_rows), _ptr(g), _ptr(n), _ptr(emit),
+            _ptr(anchor), _stream()))
+        return n, emit
 
     def debug_logits(self, which, B, K):
         out = self.torch.empty((B, K, self.shape.vocab), dtype=self.torch.float32, device=self.device)

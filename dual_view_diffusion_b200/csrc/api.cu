@@ -660,6 +660,50 @@ orthrus_status_t orthrus_kl_lm_head(orthrus_ctx_t *c, const void *h_ar, const vo
     return ORTHRUS_OK;
 }
 
+orthrus_status_t orthrus_tree_topw(orthrus_ctx_t *c, const float *logits, int32_t rows, int32_t width,
+                                   int32_t *ids, float *vals, float *lse, void *stream)
+{
+    if (!c || !logits || !ids || !vals || !lse || rows < 1 || width < 1 || width > 8 || width > c->cfg.vocab)
+        return ORTHRUS_ERR_INVALID_ARG;
+    CK(launch_tree_topw(*c, logits, rows, width, ids, vals, lse, (cudaStream_t)stream));
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_tree_build(orthrus_ctx_t *c, const int32_t *ids, const float *vals, const float *lse,
+                                    int32_t batch, int32_t depth, int32_t width, int32_t nodes, int32_t *parent,
+                                    int32_t *token, int32_t *node_depth, double *score, int32_t *n_rows,
+                                    void *stream)
+{
+    if (!c || !parent || !token || !node_depth || !score || !n_rows || batch < 1 || depth < 0 || depth >= 128 ||
+        width < 1 || width > 8 || nodes < 0 || nodes >= 128 || (depth > 0 && (!ids || !vals || !lse)))
+        return ORTHRUS_ERR_INVALID_ARG;
+    if (batch > c->cfg.max_batch) return ORTHRUS_ERR_CAPACITY;
+    TreeBuildArgs a{};
+    a.ids = ids; a.vals = vals; a.lse = lse; a.D = depth; a.W = width; a.N = nodes;
+    a.parent = parent; a.token = token; a.depth = node_depth; a.score = score; a.n_rows = n_rows;
+    CK(launch_tree_build(*c, a, batch, (cudaStream_t)stream));
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_tree_commit(orthrus_ctx_t *c, const orthrus_kv_t *kv, int32_t batch, int32_t rows,
+                                     const int32_t *parent, const int32_t *token, const int32_t *n_rows,
+                                     const int32_t *g, int32_t *n_out, int32_t *emit, int32_t *anchor,
+                                     void *stream)
+{
+    orthrus_status_t st = check_step(c, kv, batch, rows);
+    if (st != ORTHRUS_OK) return st;
+    if (!parent || !token || !n_rows || !g || !n_out || !emit || !anchor) return ORTHRUS_ERR_INVALID_ARG;
+    if (rows > 128) return ORTHRUS_ERR_CAPACITY;
+    const orthrus_config_t &f = c->cfg;
+    TreeCommitArgs a{};
+    a.kv = kv_view(*kv); a.seq_lens = kv->seq_lens;
+    a.rows = rows; a.n_layers = f.n_layers; a.n_kv = f.n_kv_heads; a.hd = f.head_dim; a.vocab = f.vocab;
+    a.parent = parent; a.token = token; a.g = g; a.n_rows = n_rows;
+    a.n_out = n_out; a.emit = emit; a.anchor = anchor; a.err = c->err;
+    CK(launch_tree_commit(*c, a, batch, (cudaStream_t)stream));
+    return ORTHRUS_OK;
+}
+
 orthrus_status_t orthrus_debug_logits(orthrus_ctx_t *c, int32_t which, int32_t batch, int32_t K, float *logits,
                                       void *stream)
 {

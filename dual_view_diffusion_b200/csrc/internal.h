@@ -272,6 +272,31 @@ cudaError_t launch_set_lens(const Ctx &c, int32_t *seq_lens, int b, int value, i
 cudaError_t launch_pack_block(const Ctx &c, const void *k_src, const void *v_src, void *k_dst, void *v_dst, int B,
                               int K, int kp, cudaStream_t s);
 cudaError_t launch_logits_dump(const Ctx &c, const void *fin, int M, float *logits, cudaStream_t s);
+// Tree verification (tree.cu): the draft tree's builder and its commit.
+struct TreeBuildArgs {   // one best-first tree per sequence
+    const int32_t *ids;      // [B][D][W] candidate ids, best first
+    const float *vals;       // [B][D][W] their logits
+    const float *lse;        // [B][D]
+    int D, W, N;
+    int32_t *parent, *token, *depth;   // [B][N+1]
+    double *score;                     // [B][N+1]
+    int32_t *n_rows;                   // [B]
+};
+
+struct TreeCommitArgs {
+    KvView kv;
+    int32_t *seq_lens;
+    int rows, n_layers, n_kv, hd, vocab;
+    const int32_t *parent, *token, *g;   // [B][rows]
+    const int32_t *n_rows;               // [B]
+    int32_t *n_out, *emit, *anchor;      // [B], [B][rows], [B]
+    unsigned *err;
+};
+
+cudaError_t launch_tree_topw(const Ctx &c, const float *logits, int rows, int W, int32_t *ids, float *vals,
+                             float *lse, cudaStream_t s);
+cudaError_t launch_tree_build(const Ctx &c, const TreeBuildArgs &a, int B, cudaStream_t s);
+cudaError_t launch_tree_commit(const Ctx &c, const TreeCommitArgs &a, int B, cudaStream_t s);
 cudaError_t launch_kl_lm_head(const Ctx &c, const void *h_a, const void *h_d, int rows, float *kl, float *lse_a,
                               float *lse_d, cudaStream_t s);
 

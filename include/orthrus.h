@@ -337,6 +337,69 @@ orthrus_status_t orthrus_kl_lm_head(orthrus_ctx_t *ctx, const void *h_ar, const 
                                     float *kl, float *lse_ar, float *lse_diff, void *stream);
 
 /*
+ * Tree verification, the parts that do not change a forward (paper notes
+ * §7.5: DDTree expands one diffusion forward's marginals best-first into a
+ * tree of the top prefixes and verifies it with tree attention in one pass;
+ * §9.6: the same proposed for Orthrus).  Greedy only.  A tree of R rows
+ * keeps row 0 as the root (the anchor) and every other row r as a node
+ * with parent[r] in [0, r) and its draft token; node r sits at position
+ * t + depth(r).  The tree-masked verify forward that fills cache slots
+ * t .. t+R-1 and the AR argmax g of every row is not part of this library
+ * yet.
+ *
+ * orthrus_tree_topw: for each of `rows` rows of fp32 logits (device,
+ * [rows][vocab]) the `width` largest logits, best first (ties: lowest id),
+ * ids [rows][width] int32 and vals [rows][width] fp32, and the row's
+ * log-sum-exp lse [rows] fp32 (T = 1).  Requires 1 <= width <= 8 and
+ * width <= vocab.  A non-finite log-sum-exp raises ORTHRUS_DEVERR_NONFINITE.
+ */
+orthrus_status_t orthrus_tree_topw(orthrus_ctx_t *ctx, const float *logits, int32_t rows, int32_t width,
+                                   int32_t *ids, float *vals, float *lse, void *stream);
+
+/*
+ * orthrus_tree_build: per sequence b, the best-first draft tree.  Inputs
+ * (device): ids, vals [batch][depth][width] and lse [batch][depth] as
+ * orthrus_tree_topw writes them for the draft rows 0 .. depth-1 (row d
+ * gives the candidates for depth d + 1, log q = val - lse).  A prefix
+ * scores the fp64 sum of its log q; the tree is the root plus the `nodes`
+ * best prefixes of depth <= `depth`, ordered by score and then by their
+ * rank sequences, rows in that order.  Outputs (device) [batch][nodes + 1]:
+ * parent (-1 for the root and unused rows), token (-1 likewise),
+ * node_depth, score (fp64, -inf on unused rows); n_rows [batch] = rows used
+ * (fewer than nodes + 1 when fewer prefixes exist).  Requires 1 <= batch <=
+ * max_batch, 0 <= depth < 128, 1 <= width <= 8, 0 <= nodes < 128.
+ */
+orthrus_status_t orthrus_tree_build(orthrus_ctx_t *ctx, const int32_t *ids, const float *vals, const float *lse,
+                                    int32_t batch, int32_t depth, int32_t width, int32_t nodes, int32_t *parent,
+                                    int32_t *token, int32_t *node_depth, double *score, int32_t *n_rows,
+                                    void *stream);
+
+/*
+ * orthrus_tree_commit: greedy acceptance on a verified tree and the commit
+ * of its accepted path.  Per sequence b (t = kv->seq_lens[b] on entry):
+ * from the root, follow the lowest row whose parent is the current row and
+ * whose token equals the current row's AR argmax g; emit the followed
+ * tokens and then g of the last row reached (n = path length + 1); the
+ * K/V of the i-th accepted node move from cache slot t + row to slot t + i
+ * in every layer and KV head; kv->seq_lens[b] += n; anchor[b] = the last
+ * emitted token.
+ *   parent, token, g  device int32 [batch][rows] (g: the AR argmax of each
+ *                     tree row's logits)
+ *   n_rows            device int32 [batch]: valid rows of each tree
+ *   n_out             device int32 [batch]
+ *   emit              device int32 [batch][rows]: tokens 0 .. n-1
+ *   anchor            device int32 [batch], written
+ * Requires 1 <= batch <= max_batch and 1 <= rows <= min(max_block, 128).
+ * A parent outside [0, r) or a g outside [0, vocab) raises
+ * ORTHRUS_DEVERR_TOKEN; slots beyond the sequence's pages raise
+ * ORTHRUS_DEVERR_CAPACITY (those rows are not moved).
+ */
+orthrus_status_t orthrus_tree_commit(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, int32_t batch, int32_t rows,
+                                     const int32_t *parent, const int32_t *token, const int32_t *n_rows,
+                                     const int32_t *g, int32_t *n_out, int32_t *emit, int32_t *anchor,
+                                     void *stream);
+
+/*
  * Test and measurement hook: the logits of the last verify (which = 0) or
  * draft (which = 1) for every block row, fp32 [batch][K][vocab], computed
  * from the final hidden rows the step kept (one extra LM-head pass; the

@@ -113,6 +113,7 @@ def lib():
             l.oc_attention_tree.argtypes = [_D, C.c_int, C.c_int, C.c_int, C.c_int, _D, _D, C.c_int, _D, _D, _I,
                                             _D]
             l.oc_forward_tree.argtypes = [P(_Cfg), P(_Model), _I, _I, C.c_int, C.c_int, _D, _D, C.c_int, _D]
+            l.oc_topw.argtypes = [_D, C.c_int, C.c_int, _I, _D]
             l.oc_tree_build.argtypes = [_D, C.c_int, C.c_int, C.c_int, C.c_int, _I, _I, _I, _D]
             l.oc_tree_accept.argtypes = [_I, _I, C.c_int, _I, _I, _I]
             l.oc_tree_commit_kv.argtypes = [_D, _D, C.c_int, C.c_int, C.c_int, C.c_int, _I, C.c_int]
@@ -227,6 +228,20 @@ def attention_tree(q, kc, vc, kb, vb, parent):
     o = np.empty_like(q)
     lib().oc_attention_tree(_dp(q), R, nq, nkv, hd, _dp(kc), _dp(vc), t, _dp(kb), _dp(vb), _ip(par), _dp(o))
     return o
+
+
+def topw(z, W):
+    """The W largest entries of each row of z (ties: lowest id) and each
+    row's log-sum-exp: (ids int32 [rows, W], lse [rows])."""
+    z = _f64(np.atleast_2d(z))
+    rows, V = z.shape
+    ids = np.zeros((rows, W), np.int32)
+    lse = np.zeros(rows)
+    for r in range(rows):
+        out = C.c_double()
+        lib().oc_topw(_dp(z[r]), V, int(W), _ip(ids[r]), C.byref(out))
+        lse[r] = out.value
+    return ids, lse
 
 
 def tree_build(logp, W, N):

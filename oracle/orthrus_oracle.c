@@ -1070,6 +1070,28 @@ void oc_kl_rows(const double *hA, const double *hD, int rows, int d, const float
 /* forward).  Greedy (T = 0) only: the pages give no sampling rule for it.   */
 /* ------------------------------------------------------------------------ */
 
+/* The W largest entries of z [V], best first, ties to the lowest id (W
+ * rounds of "largest not yet taken"), and, if lse is not NULL, the
+ * log-sum-exp log sum_v exp(z_v) = m + log sum_v exp(z_v - m), m = max z. */
+void oc_topw(const double *z, int V, int W, int32_t *ids, double *lse)
+{
+    for (int r = 0; r < W; ++r) {
+        int best = -1;
+        for (int v = 0; v < V; ++v) {
+            int taken = 0;
+            for (int u = 0; u < r; ++u) taken |= ids[u] == v;
+            if (!taken && (best < 0 || z[v] > z[best])) best = v;
+        }
+        ids[r] = best;
+    }
+    if (lse) {
+        double m = -INFINITY, s = 0.0;
+        for (int v = 0; v < V; ++v) if (z[v] > m) m = z[v];
+        for (int v = 0; v < V; ++v) s += exp(z[v] - m);
+        *lse = m + log(s);
+    }
+}
+
 /* Lexicographic order of rank sequences, a prefix before its extensions. */
 static int rankseq_less(const int32_t *a, int la, const int32_t *b, int lb)
 {
@@ -1109,18 +1131,7 @@ int oc_tree_build(const double *logp, int D, int V, int W, int N, int32_t *paren
         free(cand); free(rseq); free(pp); free(pr); free(ps); free(tmp); free(tmp2);
         return -OC_ERR_NOMEM;
     }
-    for (int d = 0; d < D; ++d) {   /* W rounds of "largest not yet taken, lowest id on ties" */
-        const double *row = logp + (size_t)d * V;
-        for (int r = 0; r < W; ++r) {
-            int best = -1;
-            for (int v = 0; v < V; ++v) {
-                int taken = 0;
-                for (int u = 0; u < r; ++u) taken |= cand[d * W + u] == v;
-                if (!taken && (best < 0 || row[v] > row[best])) best = v;
-            }
-            cand[d * W + r] = best;
-        }
-    }
+    for (int d = 0; d < D; ++d) oc_topw(logp + (size_t)d * V, V, W, cand + d * W, NULL);
     parent[0] = -1; token[0] = -1; depth[0] = 0; score[0] = 0.0;
     int n = 1, np = 0;
     if (D > 0 && N > 0) { pp[0] = 0; pr[0] = 0; ps[0] = logp[cand[0]]; np = 1; }

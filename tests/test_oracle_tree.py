@@ -72,6 +72,17 @@ def test_tree_build_matches_brute_force(D, V, W, N, kind):
     assert list(sc[1:]) == [s for _, s in want]        # same sums in the same order: exact
 
 
+def test_topw_matches_numpy_and_scipy():
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(31)
+    for z in (rng.standard_normal((4, 300)) * 3.0, rng.integers(-2, 3, size=(4, 50)).astype(np.float64)):
+        ids, lse = oracle.topw(z, 6)
+        for r in range(z.shape[0]):
+            want = np.lexsort((np.arange(z.shape[1]), -z[r]))[:6]    # by value, then lowest id
+            assert list(ids[r]) == list(want)
+            assert math.isclose(lse[r], float(logsumexp(z[r])), rel_tol=1e-14)
+
+
 def test_tree_structure_invariants():
     rng = np.random.default_rng(3)
     lp = _log_softmax(rng.standard_normal((6, 11)))
