@@ -30,6 +30,9 @@ attn_long_context  the attention entry point alone at L = 4K (the single-layer
           calls on distinct layers' caches that together exceed L2 (K/V
           from HBM)
 iterative_draft  the same decode step with a two-pass iterative-denoising draft
+tree_kernels  the tree-verification kernels built so far (top-W of the draft
+          rows, the best-first build, the walk and K/V compaction), each
+          timed alone
 train_kernels  the training-side kernels (block-masked attention of a packed
           2048-position sequence with 256 anchor blocks; the forward-KL
           LM-head epilogue over the full vocabulary), each timed alone beside
@@ -394,6 +397,59 @@ def train_kernels(hbm, tflops, eng, reps=10, cpu=True):
     return out
 
 
+def tree_kernels(hbm, reps=20):
+    """The tree-verification kernels that exist so far (paper notes §7.5 /
+    §9.6), each timed alone (median of reps, device time) at the decode
+    workload's sizes: top-W (W = 4) and log-sum-exp of the K - 1 = 31 draft
+    rows' fp32 logits over the 151936-id vocabulary (HBM: 31 x 151936 x 4 B
+    read; no flush between reps, so the 18.8 MB may be L2 hits); the
+    best-first build of 31 nodes over depth 31; the walk and the K/V
+    compaction of a 32-row tree whose accepted path has 8 nodes, in the
+    36-layer, 8-KV-head, head_dim-128 bf16 cache.  Latency-bound except
+    top-W."""
+    import numpy as np
+    import torch
+    import synth
+    import dual_view_diffusion_b200 as pkg
+    K, W, V = K_BLOCK, 4, synth.QWEN3_8B.vocab
+    s = dataclasses.replace(synth.QWEN3_8B, hidden=64, ffn=64)
+    eng = pkg.Engine(s, synth.make_weights_torch(s, 0), max_batch=1, max_block=K, max_seq=P_PROMPT + 2 * K,
+                     split_tokens=128)
+    g = torch.Generator(device="cuda").manual_seed(7)
+    z = 3.0 * torch.randn((K - 1, V), generator=g, device="cuda")
+    ids, vals, lse = eng.tree_topw(z, W)
+    us_topw = _timed(lambda: eng.tree_topw(z, W), reps)
+    D = K - 1
+    us_build = _timed(lambda: eng.tree_build(ids.view(1, D, W), vals.view(1, D, W), lse.view(1, D), K - 1), reps)
+    # a 32-row tree: 23 leaves under the root (rows 1..23), then a chain of 8 nodes (rows 24..31) that
+    # the AR argmaxes accept, so its K/V move from slots t+24..t+31 to t+1..t+8
+    par = np.array([-1] + [0] * 23 + [0] + list(range(24, 31)), np.int32)
+    tok = np.array([-1] + [1000 + i for i in range(23)] + [100 + i for i in range(8)], np.int32)
+    gg = np.full(K, 7, np.int32)
+    gg[0] = 100
+    gg[24:31] = np.arange(101, 108)
+    dev = lambda a: torch.from_numpy(a[None]).cuda()
+    pd, td, gd, nr = dev(par), dev(tok), dev(gg), torch.tensor([K], dtype=torch.int32, device="cuda")
+    anchor = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def commit():
+        eng.seq_lens[0] = P_PROMPT
+        eng.tree_commit(pd, td, nr, gd, anchor)
+    commit()
+    n_acc = int(eng.seq_lens[0].item()) - P_PROMPT
+    us_commit = _timed(commit, reps)   # includes the one-element length reset (a copy kernel)
+    assert eng.check_error()[0] == 0
+    byts = (K - 1) * V * 4
+    out = {"topw": {"rows": K - 1, "width": W, "us": us_topw, "bound": "hbm", "achieved": byts / us_topw / 1e3,
+                    "peak": hbm, "unit": "GB/s", "frac": byts / us_topw / 1e3 / hbm, "algorithmic_bytes": byts},
+           "build": {"nodes": K - 1, "depth": D, "width": W, "us": us_build, "bound": "latency"},
+           "commit": {"rows": K, "accepted": n_acc, "layers": s.n_layers, "us": us_commit, "bound": "latency",
+                      "moved_bytes": 2 * (n_acc - 1) * s.n_layers * s.n_kv_heads * s.head_dim * 2}}
+    del eng
+    torch.cuda.empty_cache()
+    return out
+
+
 def _block_mask_cpu(rec, ae, q, kb, vb, anchors, nb, K, L):
     """The oracle on 2 of the blocks, scaled by visible keys to all of them."""
     import numpy as np
@@ -703,6 +759,7 @@ def run_ours(args, rank, world, local_rank):
                 "draft_view": {"achieved": dv["achieved"], "frac": dv["frac"], "us_per_call": dv["us"]} if dv else None,
                 "in_step": in_step}
         line["train_kernels"] = train_kernels(hbm, tflops, eng)
+        line["tree_kernels"] = tree_kernels(hbm)
     if args.profile_small:
         line = {"profile_case": True, "config": "2 layers of the Qwen3-8B shape, vocab 32000", "value": value,
                 "roofline": line["roofline"], "attn": line["attn"]}

@@ -665,6 +665,7 @@ orthrus_status_t orthrus_tree_topw(orthrus_ctx_t *c, const float *logits, int32_
 {
     if (!c || !logits || !ids || !vals || !lse || rows < 1 || width < 1 || width > 8 || width > c->cfg.vocab)
         return ORTHRUS_ERR_INVALID_ARG;
+    if (rows > 65535) return ORTHRUS_ERR_CAPACITY;
     CK(launch_tree_topw(*c, logits, rows, width, ids, vals, lse, (cudaStream_t)stream));
     return ORTHRUS_OK;
 }

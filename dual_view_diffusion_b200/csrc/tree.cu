@@ -3,8 +3,9 @@
 // tree of the top prefixes and verifies it with tree attention in one pass;
 // §9.6: the same proposed for Orthrus's K marginals).  Greedy only.
 //
-//   tree_topw_kernel     per row of fp32 logits: the W best ids (ties: lowest
-//                        id) with their logits, and the row's log-sum-exp
+//   tree_topw_kernel     per row of fp32 logits (one 8-CTA cluster): the W
+//                        best ids (ties: lowest id) with their logits, and
+//                        the row's log-sum-exp
 //   tree_build_kernel    one warp per sequence: the root plus the N best
 //                        prefixes of depth <= D, scores = sums of log q in
 //                        fp64, ordered by score and then by rank sequence
@@ -22,6 +23,7 @@ namespace orthrus {
 constexpr int kTreeMaxW = 8;        // candidates per depth
 constexpr int kTreeMaxRows = 128;   // rows of one tree (root + nodes)
 constexpr int kTreeTopwThreads = 256;
+constexpr int kTreeTopwSplit = 8;     // CTAs (one cluster) per logits row
 
 __device__ __forceinline__ bool tw_better(float va, int ia, float vb, int ib)
 {
@@ -58,39 +60,120 @@ __device__ __forceinline__ void tw_warp_merge(float (&v)[kTreeMaxW], int (&i)[kT
     }
 }
 
-// Grid rows, kTreeTopwThreads threads.  z [rows][V] fp32.
+// A logit into a thread's sorted top list (the common case is one compare).
+__device__ __forceinline__ void tw_insert(float x, int v, float (&tv)[kTreeMaxW], int (&ti)[kTreeMaxW])
+{
+    if (tw_better(x, v, tv[kTreeMaxW - 1], ti[kTreeMaxW - 1])) {
+        tv[kTreeMaxW - 1] = x;
+        ti[kTreeMaxW - 1] = v;
+#pragma unroll
+        for (int j = kTreeMaxW - 1; j > 0; --j)
+            if (tw_better(tv[j], ti[j], tv[j - 1], ti[j - 1])) {
+                const float a = tv[j]; tv[j] = tv[j - 1]; tv[j - 1] = a;
+                const int b = ti[j]; ti[j] = ti[j - 1]; ti[j - 1] = b;
+            }
+    }
+}
+
+// Up to four logits (x[0 .. n-1]) into a thread's running (max, sum of
+// exp(x - max)): one rescale per group, the exponentials independent.
+__device__ __forceinline__ void tw_lse4(const float (&x)[4], int n, float &m, float &s)
+{
+    float mc = x[0];
+#pragma unroll
+    for (int e = 1; e < 4; ++e)
+        if (e < n) mc = fmaxf(mc, x[e]);
+    if (mc > m) { s *= expf(m - mc); m = mc; }
+    float add = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        if (e < n) add += expf(x[e] - m);
+    s += add;
+}
+
+__device__ __forceinline__ uint32_t tw_smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ uint32_t tw_mapa(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float tw_ld_peer_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ int tw_ld_peer_s32(uint32_t addr)
+{
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];\n" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void tw_cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+// Grid (kTreeTopwSplit, rows), clusters of kTreeTopwSplit CTAs along x: CTA
+// s of a row's cluster takes ids [s * chunk, (s + 1) * chunk) (chunk a
+// multiple of 4), each thread a sorted top list and a running (max, sum),
+// merged across the CTA's warps; then CTA 0 pulls every CTA's list and
+// (max, sum) from distributed shared memory and merges them.  VEC (V a
+// multiple of 4, z 16-byte aligned): 16-byte loads, four in flight.
+template <bool VEC>
 __global__ void __launch_bounds__(kTreeTopwThreads) tree_topw_kernel(const float *__restrict__ z, int V, int W,
-                                                                     int32_t *ids, float *vals, float *lse,
-                                                                     unsigned *err)
+                                                                     int chunk, int32_t *ids, float *vals,
+                                                                     float *lse, unsigned *err)
 {
     pdl_trigger();
     pdl_wait();
-    __shared__ float wv[kTreeTopwThreads / 32][kTreeMaxW];
-    __shared__ int wi[kTreeTopwThreads / 32][kTreeMaxW];
-    __shared__ float wm[kTreeTopwThreads / 32], ws[kTreeTopwThreads / 32];
-    const int row = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int nw = kTreeTopwThreads / 32;
+    __shared__ float wv[nw][kTreeMaxW];
+    __shared__ int wi[nw][kTreeMaxW];
+    __shared__ float wm[nw], ws[nw];
+    __shared__ float cv[kTreeMaxW];   // this CTA's result, read by CTA 0 of the cluster
+    __shared__ int ci[kTreeMaxW];
+    __shared__ float cms[2];
+    const int split = blockIdx.x, row = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lo = split * chunk, hi = min(V, lo + chunk);
     const float *zr = z + (size_t)row * V;
     float tv[kTreeMaxW];
     int ti[kTreeMaxW];
 #pragma unroll
     for (int j = 0; j < kTreeMaxW; ++j) { tv[j] = -INFINITY; ti[j] = INT_MAX; }
     float m = -INFINITY, s = 0.f;   // running max and sum of exp(x - m)
-    for (int v = threadIdx.x; v < V; v += kTreeTopwThreads) {
-        const float x = zr[v];
-        if (x > m) { s = s * expf(m - x) + 1.f; m = x; }
-        else s += expf(x - m);
-        if (tw_better(x, v, tv[kTreeMaxW - 1], ti[kTreeMaxW - 1])) {   // insert, keep the list sorted
-            tv[kTreeMaxW - 1] = x;
-            ti[kTreeMaxW - 1] = v;
+    if (VEC) {
+        constexpr int U = 4;
+        const int q0 = lo / 4, q1 = (hi + 3) / 4;   // hi is V or a multiple of 4; V % 4 == 0 here
+        const float4 *z4 = (const float4 *)zr;
+        for (int i0 = q0 + threadIdx.x; i0 < q1; i0 += kTreeTopwThreads * U) {
+            float4 x4[U];
 #pragma unroll
-            for (int j = kTreeMaxW - 1; j > 0; --j)
-                if (tw_better(tv[j], ti[j], tv[j - 1], ti[j - 1])) {
-                    const float a = tv[j]; tv[j] = tv[j - 1]; tv[j - 1] = a;
-                    const int b = ti[j]; ti[j] = ti[j - 1]; ti[j - 1] = b;
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + u * kTreeTopwThreads;
+                x4[u] = i < q1 ? z4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + u * kTreeTopwThreads;
+                if (i < q1) {
+                    const float x[4] = {x4[u].x, x4[u].y, x4[u].z, x4[u].w};
+                    tw_lse4(x, 4, m, s);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) tw_insert(x[e], 4 * i + e, tv, ti);
                 }
+            }
+        }
+    } else {
+        for (int v = lo + threadIdx.x; v < hi; v += kTreeTopwThreads) {
+            const float x[4] = {zr[v], 0.f, 0.f, 0.f};
+            tw_lse4(x, 1, m, s);
+            tw_insert(x[0], v, tv, ti);
         }
     }
-    // log-sum-exp: (m, s) pairs merged across the warp, then across warps
+    // this CTA: (m, s) across the warp, then across warps; lists likewise
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
         const float m2 = __shfl_xor_sync(0xffffffffu, m, off), s2 = __shfl_xor_sync(0xffffffffu, s, off);
@@ -109,7 +192,6 @@ __global__ void __launch_bounds__(kTreeTopwThreads) tree_topw_kernel(const float
     }
     __syncthreads();
     if (warp == 0) {
-        constexpr int nw = kTreeTopwThreads / 32;
 #pragma unroll
         for (int j = 0; j < kTreeMaxW; ++j) {
             tv[j] = lane < nw ? wv[lane][j] : -INFINITY;
@@ -119,8 +201,36 @@ __global__ void __launch_bounds__(kTreeTopwThreads) tree_topw_kernel(const float
         if (lane == 0) {
             float M = -INFINITY, S = 0.f;
             for (int w = 0; w < nw; ++w) M = fmaxf(M, wm[w]);
-            for (int w = 0; w < nw; ++w) S += ws[w] * expf(wm[w] - M);
-            const float l = M + logf(S);
+            if (M != -INFINITY)
+                for (int w = 0; w < nw; ++w) S += ws[w] * expf(wm[w] - M);
+            cms[0] = M;
+            cms[1] = S;
+#pragma unroll
+            for (int j = 0; j < kTreeMaxW; ++j) { cv[j] = mv[j]; ci[j] = mi[j]; }
+        }
+    }
+    tw_cluster_sync();   // every CTA's result is in its shared memory
+    if (split == 0 && warp == 0) {
+        // lane c < kTreeTopwSplit holds CTA c's list; the same warp merge
+        const bool on = lane < kTreeTopwSplit;
+        const uint32_t pv = tw_mapa(tw_smem_u32(cv), on ? lane : 0), pi = tw_mapa(tw_smem_u32(ci), on ? lane : 0);
+#pragma unroll
+        for (int j = 0; j < kTreeMaxW; ++j) {
+            tv[j] = on ? tw_ld_peer_f32(pv + 4 * j) : -INFINITY;
+            ti[j] = on ? tw_ld_peer_s32(pi + 4 * j) : INT_MAX;
+        }
+        const uint32_t pm = tw_mapa(tw_smem_u32(cms), on ? lane : 0);
+        float m1 = on ? tw_ld_peer_f32(pm) : -INFINITY, s1 = on ? tw_ld_peer_f32(pm + 4) : 0.f;
+        tw_warp_merge(tv, ti, mv, mi);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m1, off), s2 = __shfl_xor_sync(0xffffffffu, s1, off);
+            const float M = fmaxf(m1, m2);
+            s1 = (M == -INFINITY) ? 0.f : s1 * expf(m1 - M) + s2 * expf(m2 - M);
+            m1 = M;
+        }
+        if (lane == 0) {
+            const float l = m1 + logf(s1);
             if (!isfinite(l)) raise_err(err, ORTHRUS_DEVERR_NONFINITE);
             lse[row] = l;
             for (int j = 0; j < W; ++j) {
@@ -129,6 +239,7 @@ __global__ void __launch_bounds__(kTreeTopwThreads) tree_topw_kernel(const float
             }
         }
     }
+    tw_cluster_sync();   // no CTA leaves while CTA 0 may still read its shared memory
 }
 
 // ------------------------------------------------------------------ builder
@@ -220,22 +331,34 @@ __global__ void __launch_bounds__(32) tree_build_kernel(TreeBuildArgs a)
 
 // ------------------------------------------------------------------- commit
 
-// The greedy walk (shared by both kernels): from the root follow the lowest
+// One sequence's tree rows staged in shared memory by the whole CTA (the walk
+// then reads no global memory).  Returns R, the rows in use.
+__device__ int tree_stage(const TreeCommitArgs &a, int b, int32_t *par, int32_t *tok, int32_t *g)
+{
+    const int R = min(max(a.n_rows[b], 1), a.rows);
+    for (int r = threadIdx.x; r < R; r += blockDim.x) {
+        par[r] = a.parent[(size_t)b * a.rows + r];
+        tok[r] = a.token[(size_t)b * a.rows + r];
+        g[r] = a.g[(size_t)b * a.rows + r];
+    }
+    __syncthreads();
+    return R;
+}
+
+// The greedy walk (both kernels, one thread): from the root follow the lowest
 // row whose parent is the current row and whose token is the current row's
 // argmax g; path[0..m] = rows visited.  Returns m; a malformed parent entry
 // raises ORTHRUS_DEVERR_TOKEN and ends the walk there.
-__device__ int tree_walk(const TreeCommitArgs &a, int b, int32_t *path)
+__device__ int tree_walk(const int32_t *par, const int32_t *tok, const int32_t *g, int R, unsigned *err,
+                         int32_t *path)
 {
-    const int R = min(max(a.n_rows[b], 1), a.rows);
-    const int32_t *par = a.parent + (size_t)b * a.rows, *tok = a.token + (size_t)b * a.rows;
-    const int32_t *g = a.g + (size_t)b * a.rows;
     int cur = 0, m = 0;
     path[0] = 0;
     for (;;) {
         int next = -1;
         for (int c = cur + 1; c < R && next < 0; ++c) {
             const int p = par[c];
-            if (p < 0 || p >= c) { raise_err(a.err, ORTHRUS_DEVERR_TOKEN); return m; }
+            if (p < 0 || p >= c) { raise_err(err, ORTHRUS_DEVERR_TOKEN); return m; }
             if (p == cur && tok[c] == g[cur]) next = c;
         }
         if (next < 0) return m;
@@ -251,12 +374,13 @@ __device__ int tree_walk(const TreeCommitArgs &a, int b, int32_t *path)
 template <class T>
 __global__ void __launch_bounds__(128) tree_compact_kernel(TreeCommitArgs a)
 {
-    __shared__ int32_t path[kTreeMaxRows];
+    __shared__ int32_t path[kTreeMaxRows], s_par[kTreeMaxRows], s_tok[kTreeMaxRows], s_g[kTreeMaxRows];
     __shared__ int m_s, t_s;
     __shared__ T kbuf[32][128], vbuf[32][128];
     pdl_wait();   // no early trigger: tree_finish_kernel writes seq_lens, read here
     const int b = blockIdx.y, layer = blockIdx.x / a.n_kv, kvh = blockIdx.x % a.n_kv, hd = a.hd;
-    if (threadIdx.x == 0) { m_s = tree_walk(a, b, path); t_s = a.seq_lens[b]; }
+    const int R = tree_stage(a, b, s_par, s_tok, s_g);
+    if (threadIdx.x == 0) { m_s = tree_walk(s_par, s_tok, s_g, R, a.err, path); t_s = a.seq_lens[b]; }
     __syncthreads();
     const int m = m_s, t = t_s;
     const T *kp = (const T *)a.kv.k_pages;
@@ -292,17 +416,17 @@ __global__ void __launch_bounds__(128) tree_compact_kernel(TreeCommitArgs a)
     }
 }
 
-// Grid 1, B threads (B <= max_batch): emitted tokens, n, anchor, seq_len.
-__global__ void tree_finish_kernel(TreeCommitArgs a, int B)
+// Grid B, 128 threads: emitted tokens, n, anchor, seq_len of sequence b.
+__global__ void __launch_bounds__(128) tree_finish_kernel(TreeCommitArgs a)
 {
+    __shared__ int32_t path[kTreeMaxRows], s_par[kTreeMaxRows], s_tok[kTreeMaxRows], s_g[kTreeMaxRows];
     pdl_wait();
-    const int b = threadIdx.x;
-    if (b >= B) return;
-    int32_t path[kTreeMaxRows];
-    const int m = tree_walk(a, b, path);
-    const int32_t *tok = a.token + (size_t)b * a.rows, *g = a.g + (size_t)b * a.rows;
-    for (int i = 1; i <= m; ++i) a.emit[(size_t)b * a.rows + i - 1] = tok[path[i]];
-    int last = g[path[m]];
+    const int b = blockIdx.x;
+    const int R = tree_stage(a, b, s_par, s_tok, s_g);
+    if (threadIdx.x != 0) return;
+    const int m = tree_walk(s_par, s_tok, s_g, R, a.err, path);
+    for (int i = 1; i <= m; ++i) a.emit[(size_t)b * a.rows + i - 1] = s_tok[path[i]];
+    int last = s_g[path[m]];
     if (last < 0 || last >= a.vocab) { raise_err(a.err, ORTHRUS_DEVERR_TOKEN); last = 0; }
     a.emit[(size_t)b * a.rows + m] = last;
     a.n_out[b] = m + 1;
@@ -313,8 +437,25 @@ __global__ void tree_finish_kernel(TreeCommitArgs a, int B)
 cudaError_t launch_tree_topw(const Ctx &c, const float *logits, int rows, int W, int32_t *ids, float *vals,
                              float *lse, cudaStream_t s)
 {
+    const int V = c.cfg.vocab;
+    const bool vec = V % 4 == 0 && ((uintptr_t)logits & 15) == 0;
+    const int chunk = ((V + 4 * kTreeTopwSplit - 1) / (4 * kTreeTopwSplit)) * 4;   // a multiple of 4
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kTreeTopwSplit, rows);
+    cfg.blockDim = dim3(kTreeTopwThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = kTreeTopwSplit;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     c.launches += 1;
-    return launch_k(tree_topw_kernel, rows, kTreeTopwThreads, 0, s, logits, c.cfg.vocab, W, ids, vals, lse, c.err);
+    if (vec) return cudaLaunchKernelEx(&cfg, tree_topw_kernel<true>, logits, V, W, chunk, ids, vals, lse, c.err);
+    return cudaLaunchKernelEx(&cfg, tree_topw_kernel<false>, logits, V, W, chunk, ids, vals, lse, c.err);
 }
 
 cudaError_t launch_tree_build(const Ctx &c, const TreeBuildArgs &a, int B, cudaStream_t s)
@@ -327,13 +468,13 @@ cudaError_t launch_tree_build(const Ctx &c, const TreeBuildArgs &a, int B, cudaS
 
 cudaError_t launch_tree_commit(const Ctx &c, const TreeCommitArgs &a, int B, cudaStream_t s)
 {
-    if (a.hd > 128 || a.rows > kTreeMaxRows || B > 1024) return cudaErrorInvalidValue;
+    if (a.hd > 128 || a.rows > kTreeMaxRows || B > 65535) return cudaErrorInvalidValue;
     c.launches += 2;
     const dim3 grid(a.n_layers * a.n_kv, B);
     cudaError_t e = c.cfg.dtype == ORTHRUS_BF16 ? launch_k(tree_compact_kernel<bf16>, grid, 128, 0, s, a)
                                                 : launch_k(tree_compact_kernel<float>, grid, 128, 0, s, a);
     if (e != cudaSuccess) return e;
-    return launch_k(tree_finish_kernel, 1, B, 0, s, a, B);
+    return launch_k(tree_finish_kernel, B, 128, 0, s, a);
 }
 
 }  // namespace orthrus

@@ -350,8 +350,9 @@ orthrus_status_t orthrus_kl_lm_head(orthrus_ctx_t *ctx, const void *h_ar, const 
  * orthrus_tree_topw: for each of `rows` rows of fp32 logits (device,
  * [rows][vocab]) the `width` largest logits, best first (ties: lowest id),
  * ids [rows][width] int32 and vals [rows][width] fp32, and the row's
- * log-sum-exp lse [rows] fp32 (T = 1).  Requires 1 <= width <= 8 and
- * width <= vocab.  A non-finite log-sum-exp raises ORTHRUS_DEVERR_NONFINITE.
+ * log-sum-exp lse [rows] fp32 (T = 1).  Requires 1 <= width <= 8,
+ * width <= vocab and rows <= 65535 (ORTHRUS_ERR_CAPACITY beyond).  A
+ * non-finite log-sum-exp raises ORTHRUS_DEVERR_NONFINITE.
  */
 orthrus_status_t orthrus_tree_topw(orthrus_ctx_t *ctx, const float *logits, int32_t rows, int32_t width,
                                    int32_t *ids, float *vals, float *lse, void *stream);

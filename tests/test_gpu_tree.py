@@ -62,6 +62,21 @@ def test_topw_matches_oracle(eng_full_vocab, kind, W):
     assert (np.abs(lse - want_lse) <= 1e-5 * np.maximum(1.0, np.abs(want_lse))).all()
 
 
+def test_topw_scalar_path():
+    """A vocabulary that is not a multiple of 4 takes the kernel's scalar
+    loads (the 16-byte path needs whole float4s per row)."""
+    eng = _engine(1001)
+    z = _f32((3, 1001), 43, "topw_odd", 2.0)
+    ids, vals, lse = eng.tree_topw(torch.from_numpy(z).cuda(), 5)
+    assert eng.check_error()[0] == 0
+    want_ids, want_lse = oracle.topw(z.astype(np.float64), 5)
+    assert np.array_equal(ids.cpu().numpy(), want_ids)
+    assert np.array_equal(vals.cpu().numpy(), np.take_along_axis(z, want_ids, axis=1))
+    assert (np.abs(lse.cpu().numpy() - want_lse) <= 1e-5 * np.maximum(1.0, np.abs(want_lse))).all()
+    del eng
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("D,W,N", [(7, 2, 7), (7, 4, 20), (31, 3, 31), (5, 8, 60), (3, 2, 40)])
 def test_tree_build_matches_oracle(eng_small, D, W, N):
     """Candidates from the GPU top-W kernel (pinned exact above); the
