@@ -152,6 +152,12 @@ def make_config(shape, dtype, max_batch, max_block, max_seq, split_tokens=256) -
                   max_block, max_seq, split_tokens, shape.rope_theta, shape.rms_eps)
 
 
+def _need(x, dtype, name):
+    """Marshalling check: a contiguous device tensor of the dtype the C call reads."""
+    if x.dtype != dtype or not x.is_cuda or not x.is_contiguous():
+        raise TypeError(f"{name}: expected a contiguous CUDA {dtype} tensor, got {x.dtype} on {x.device}")
+
+
 class Engine:
     """One model on one CUDA device: weights, a paged KV cache and a
     context.  `weights` is either host arrays (attributes embed, final_norm,
@@ -337,7 +343,10 @@ class Engine:
         """The `width` best ids and logits of each fp32 logits row, and the
         row's log-sum-exp: (ids int32 [rows, width], vals fp32, lse fp32)."""
         t = self.torch
-        z = logits.reshape(-1, logits.shape[-1])
+        _need(logits, t.float32, "logits")
+        z = logits.reshape(-1, logits.shape[-1]).contiguous()
+        if int(z.shape[1]) != self.shape.vocab:
+            raise ValueError(f"logits rows must have {self.shape.vocab} entries")
         rows = int(z.shape[0])
         ids = t.empty((rows, width), dtype=t.int32, device=self.device)
         vals = t.empty((rows, width), dtype=t.float32, device=self.device)
@@ -350,6 +359,8 @@ class Engine:
         """Best-first draft trees from per-depth candidates ids/vals [B, D, W]
         and lse [B, D]: (parent, token, depth, score [B, nodes + 1], n_rows [B])."""
         t = self.torch
+        for name, x, dt in (("ids", ids, t.int32), ("vals", vals, t.float32), ("lse", lse, t.float32)):
+            _need(x, dt, name)
         B, D, W = (int(x) for x in ids.shape)
         par, tok, dep = (t.empty((B, nodes + 1), dtype=t.int32, device=self.device) for _ in range(3))
         sc = t.empty((B, nodes + 1), dtype=t.float64, device=self.device)
@@ -364,6 +375,8 @@ class Engine:
         accepted paths' K/V; anchor [B] is updated in place.  Returns
         (n [B], emitted tokens [B, rows])."""
         t = self.torch
+        for name, x in (("parent", parent), ("token", token), ("n_rows", n_rows), ("g", g), ("anchor", anchor)):
+            _need(x, t.int32, name)
         B, R = (int(x) for x in parent.shape)
         n = t.empty(B, dtype=t.int32, device=self.device)
         emit = t.full((B, R), -1, dtype=t.int32, device=self.device)
