@@ -8,7 +8,8 @@ The C source follows the paper-notes page on "Orthrus: Memory-Efficient
 Parallel Token Generation via Dual-View Diffusion" (§2.1 dual-view layer,
 §3.2 diffusion mask, §4.1-4.3 the decode cycle and its consensus; §3.1-3.3
 the training-side block mask and forward KL; §7.5 / §9.6 tree verification
-of one draft's marginals); each C function cites the passage it restates.
+of one draft's marginals and the adaptive block length); each C function
+cites the passage it restates.
 """
 from __future__ import annotations
 
@@ -114,6 +115,11 @@ def lib():
                                             _D]
             l.oc_forward_tree.argtypes = [P(_Cfg), P(_Model), _I, _I, C.c_int, C.c_int, _D, _D, C.c_int, _D]
             l.oc_topw.argtypes = [_D, C.c_int, C.c_int, _I, _D]
+            l.oc_entropy.argtypes = [_D, C.c_int]
+            l.oc_entropy.restype = C.c_double
+            l.oc_adaptive_len.argtypes = [_D, C.c_int, C.c_double]
+            l.oc_generate_adaptive.argtypes = [P(_Cfg), P(_Model), _I, C.c_int, C.c_int, C.c_double, C.c_int, _I,
+                                               _I, _I, P(C.c_int), _D, _D, P(C.c_int)]
             l.oc_tree_build.argtypes = [_D, C.c_int, C.c_int, C.c_int, C.c_int, _I, _I, _I, _D]
             l.oc_tree_accept.argtypes = [_I, _I, C.c_int, _I, _I, _I]
             l.oc_tree_commit_kv.argtypes = [_D, _D, C.c_int, C.c_int, C.c_int, C.c_int, _I, C.c_int]
@@ -242,6 +248,18 @@ def topw(z, W):
         lib().oc_topw(_dp(z[r]), V, int(W), _ip(ids[r]), C.byref(out))
         lse[r] = out.value
     return ids, lse
+
+
+def entropy(z):
+    """Entropy (nats) of softmax(z) at T = 1."""
+    z = _f64(z)
+    return lib().oc_entropy(_dp(z), z.size)
+
+
+def adaptive_len(H, h_max):
+    """The adaptive verify length for draft-row entropies H [K]."""
+    H = _f64(H)
+    return lib().oc_adaptive_len(_dp(H), H.size, float(h_max))
 
 
 def tree_build(logp, W, N):
@@ -465,6 +483,30 @@ class Model:
         if rc:
             raise RuntimeError(f"oc_generate_tree failed: {rc}")
         res = {"tokens": out, "n_per_cycle": npc[:cyc.value], "cycles": cyc.value, "t": tt.value}
+        if want_cache:
+            res["k_cache"], res["v_cache"] = kc, vc
+        return res
+
+    def generate_adaptive(self, prompt, K, h_max, N, want_cache=False):
+        """Greedy decoding whose cycles verify only the drafted tokens whose
+        draft rows have entropy <= h_max (at most K rows).  Returns a dict
+        like generate() plus k_per_cycle."""
+        p = _i32(prompt)
+        out = np.zeros(N, np.int32)
+        npc = np.zeros(N, np.int32)
+        kpc = np.zeros(N, np.int32)
+        cyc = C.c_int()
+        tt = C.c_int()
+        kc = vc = None
+        if want_cache:
+            kc, vc = self.new_cache(p.size + N + K)
+        rc = lib().oc_generate_adaptive(C.byref(self.cfg), C.byref(self.model), _ip(p), p.size, int(K), float(h_max),
+                                        int(N), _ip(out), _ip(npc), _ip(kpc), C.byref(cyc), _dp(kc), _dp(vc),
+                                        C.byref(tt))
+        if rc:
+            raise RuntimeError(f"oc_generate_adaptive failed: {rc}")
+        res = {"tokens": out, "n_per_cycle": npc[:cyc.value], "k_per_cycle": kpc[:cyc.value], "cycles": cyc.value,
+               "t": tt.value}
         if want_cache:
             res["k_cache"], res["v_cache"] = kc, vc
         return res

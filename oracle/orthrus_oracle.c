@@ -1285,3 +1285,90 @@ done:
     free(path); free(sc); free(zt);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Adaptive block length (paper notes §7.4 and §9.6: SV's information-gain   */
+/* signal deciding how many drafted tokens to verify, suggested for Orthrus; */
+/* no rule is given).  Reading: the entropy of each draft row's distribution */
+/* is the signal; a cycle verifies the drafted tokens while their rows'      */
+/* entropies stay at or below a threshold.  Greedy only.                     */
+/* ------------------------------------------------------------------------ */
+
+/* Entropy (nats) of softmax(z) at T = 1: H = LSE - sum_v p_v z_v. */
+double oc_entropy(const double *z, int V)
+{
+    double m = -INFINITY, s = 0.0, e = 0.0;
+    for (int v = 0; v < V; ++v) if (z[v] > m) m = z[v];
+    for (int v = 0; v < V; ++v) s += exp(z[v] - m);
+    const double lse = m + log(s);
+    for (int v = 0; v < V; ++v) e += exp(z[v] - lse) * z[v];
+    return lse - e;
+}
+
+/* The verify length for one cycle: 1 + the number of leading drafted tokens
+ * y_1, y_2, ... (y_k comes from draft row k-1) whose rows have entropy <=
+ * h_max, at most K.  H [K]: the draft rows' entropies. */
+int oc_adaptive_len(const double *H, int K, double h_max)
+{
+    int k = 1;
+    while (k < K && H[k - 1] <= h_max) ++k;
+    return k;
+}
+
+/*
+ * Greedy decoding with an adaptive block length: every cycle drafts K rows
+ * (oc_draft, T = 0), takes Kt = oc_adaptive_len(entropies, K, h_max), runs
+ * the AR verification of [anchor, y_1 .. y_{Kt-1}] and the greedy consensus
+ * over those Kt rows.  Writes out / n_per_cycle / k_per_cycle (the Kt of
+ * each cycle) / cycles / t; kc_out, vc_out as oc_generate_iter's (capacity
+ * P + N + K).  h_max = +inf is the fixed-K cycle; h_max < 0 verifies the
+ * anchor alone (plain AR).
+ */
+int oc_generate_adaptive(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P, int K, double h_max,
+                         int N, int32_t *out, int32_t *n_per_cycle, int32_t *k_per_cycle, int *n_cycles,
+                         double *kc_out, double *vc_out, int *t_out)
+{
+    if (!c || !w || !prompt || P < 1 || N < 1 || K < 1) return OC_ERR_ARG;
+    const int V = c->vocab;
+    const int cap = P + N + K;
+    const size_t kn = (size_t)c->n_kv_heads * c->head_dim;
+    const size_t csz = (size_t)c->n_layers * cap * kn;
+    double *kc = calloc(csz, sizeof(double)), *vc = calloc(csz, sizeof(double));
+    int32_t *draft = malloc(sizeof(int32_t) * K), *g = malloc(sizeof(int32_t) * K);
+    int32_t *emit = malloc(sizeof(int32_t) * K);
+    double *z = malloc(sizeof(double) * (size_t)K * V), *H = malloc(sizeof(double) * K);
+    int rc = OC_OK;
+    if (!kc || !vc || !draft || !g || !emit || !z || !H) { rc = OC_ERR_NOMEM; goto done; }
+    int t = oc_prefill(c, w, prompt, P, kc, vc, cap);
+    if (t < 0) { rc = -t; goto done; }
+    int32_t anchor = prompt[P - 1];
+    int produced = 0, cycles = 0;
+    while (produced < N) {
+        rc = oc_draft(c, w, kc, vc, cap, t, anchor, K, 0.0, 0, 0, draft, NULL, z, NULL);
+        if (rc) goto done;
+        for (int k = 0; k < K; ++k) H[k] = oc_entropy(z + (size_t)k * V, V);
+        const int Kt = oc_adaptive_len(H, K, h_max);
+        rc = oc_verify(c, w, kc, vc, cap, t, anchor, draft, Kt, 0.0, g, NULL, NULL, NULL);
+        if (rc) goto done;
+        const int n = oc_consensus_greedy(draft, g, Kt, emit);
+        t += n;
+        anchor = emit[n - 1];
+        for (int i = 0; i < n && produced < N; ++i) out[produced++] = emit[i];
+        if (n_per_cycle) n_per_cycle[cycles] = n;
+        if (k_per_cycle) k_per_cycle[cycles] = Kt;
+        ++cycles;
+    }
+    if (n_cycles) *n_cycles = cycles;
+    if (t_out) *t_out = t;
+    if (kc_out || vc_out) {
+        for (int l = 0; l < c->n_layers; ++l) {
+            memset(kc + ((size_t)l * cap + t) * kn, 0, sizeof(double) * (size_t)(cap - t) * kn);
+            memset(vc + ((size_t)l * cap + t) * kn, 0, sizeof(double) * (size_t)(cap - t) * kn);
+        }
+        if (kc_out) memcpy(kc_out, kc, sizeof(double) * csz);
+        if (vc_out) memcpy(vc_out, vc, sizeof(double) * csz);
+    }
+done:
+    free(kc); free(vc); free(draft); free(g); free(emit); free(z); free(H);
+    return rc;
+}
