@@ -18,7 +18,12 @@
  * orthrus_prefill builds the shared cache with the AR view (§2.2);
  * orthrus_ar_step is one step of plain AR decoding with the same kernels
  * (the baseline the method must reproduce exactly at T = 0, §4.2, §9.1);
- * orthrus_generate drives the whole loop.
+ * orthrus_generate drives the whole loop.  Beyond the cycle:
+ * orthrus_draft_block_iterative (multi-pass denoising draft, §5.4.2),
+ * orthrus_block_mask_attention and orthrus_kl_lm_head (the training-side
+ * dual-pass block mask and forward KL, §3.1-3.3), and orthrus_tree_topw /
+ * orthrus_tree_build / orthrus_tree_commit (tree verification's draft tree
+ * and commit, §7.5, §9.6; its tree-masked verify forward is not here yet).
  *
  * Conventions for every entry point:
  *   - Every pointer to tensor data is a DEVICE pointer owned by the caller
