@@ -445,9 +445,41 @@ def tree_kernels(hbm, reps=20):
            "build": {"nodes": K - 1, "depth": D, "width": W, "us": us_build, "bound": "latency"},
            "commit": {"rows": K, "accepted": n_acc, "layers": s.n_layers, "us": us_commit, "bound": "latency",
                       "moved_bytes": 2 * (n_acc - 1) * s.n_layers * s.n_kv_heads * s.head_dim * 2}}
+    _tree_cpu(out, z[:2].cpu().numpy(), W, K, s.n_layers, s.n_kv_heads, s.head_dim, par, tok, gg)
     del eng
     torch.cuda.empty_cache()
     return out
+
+
+def _tree_cpu(out, z2, W, K, n_layers, n_kv, hd, par, tok, gg):
+    """The oracle beside each tree kernel: top-W + log-sum-exp of 2 of the
+    31 logits rows (scaled to 31), the best-first build of the same tree
+    (D = K - 1 rows of log q over the vocabulary), and the walk plus the
+    K/V moves of the same path in an fp64 cache of the same layers and
+    heads (capacity K, t = 0)."""
+    import numpy as np
+    import oracle
+    rows = K - 1
+    t0 = time.perf_counter()
+    ids, lse = oracle.topw(z2.astype(np.float64), W)
+    t_topw = (time.perf_counter() - t0) * rows / z2.shape[0]
+    logp = np.repeat(z2[:1].astype(np.float64) - lse[0], rows, axis=0)
+    t0 = time.perf_counter()
+    oracle.tree_build(logp, W, rows)
+    t_build = time.perf_counter() - t0
+    kc = np.zeros((n_layers, K, n_kv, hd))
+    vc = np.zeros_like(kc)
+    t0 = time.perf_counter()
+    _, _, path = oracle.tree_accept(par, tok, gg)
+    oracle.tree_commit_kv(kc, vc, 0, path)
+    t_commit = time.perf_counter() - t0
+    cores = OracleSample.threads()
+    out["topw"]["cpu_baseline"] = {"seconds": t_topw, "cores": cores, "kind": "oracle",
+                                   "sample": f"2 of the {rows} rows, scaled"}
+    out["build"]["cpu_baseline"] = {"seconds": t_build, "cores": cores, "kind": "oracle",
+                                    "sample": "the whole build (one logits row repeated for every depth)"}
+    out["commit"]["cpu_baseline"] = {"seconds": t_commit, "cores": cores, "kind": "oracle",
+                                     "sample": "the whole walk and the moves of the same path"}
 
 
 def _block_mask_cpu(rec, ae, q, kb, vb, anchors, nb, K, L):
