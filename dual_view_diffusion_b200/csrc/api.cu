@@ -92,7 +92,9 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
     // attention partials [Rw][n_q][n_splits][hd] fp32 and [Rw][n_q][n_splits]
     // float2: only the SIMT attention uses them (the tensor-core attention
     // combines its splits on chip)
-    const bool simt_attn = !(c.dtype == ORTHRUS_BF16 && c.head_dim == 128);
+    // (pages of a multiple of 64 slots are required of the bf16 head_dim-128
+    // path, so they do not decide it here)
+    const bool simt_attn = !attn_tc_shape_ok(c.dtype, c.head_dim, c.n_q_heads, c.n_kv_heads, 64);
     const size_t o_part = take(simt_attn ? Rw * c.n_q_heads * n_splits * c.head_dim * 4 : 0);
     const size_t o_ml = take(simt_attn ? Rw * c.n_q_heads * n_splits * 8 : 0);
     // long contexts: the tensor-core attention spreads a row group over up
@@ -120,6 +122,7 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
         x->h = (float *)P(o_h); x->a = P(o_a); x->q = P(o_q); x->attn_o = P(o_o); x->act = P(o_act);
         x->k_diff = P(o_kd); x->v_diff = P(o_vd); x->fin_draft = P(o_fd); x->fin_verify = P(o_fv); x->res_x = P(o_rx);
         x->attn_part = (float *)P(o_part); x->attn_ml = (float2 *)P(o_ml);
+        x->attn_simt_rows = simt_attn ? (int)Rw : 0;
         x->attn_xo = attn_x2 ? (float *)P(o_xo) : nullptr; x->attn_xml = attn_x2 ? (float2 *)P(o_xml) : nullptr;
         x->attn_xcnt = attn_x2 ? (int *)P(o_xc) : nullptr; x->attn_xz = attn_x2 ? kAttnMaxClusters : 1;
         x->gemm_part = (float *)P(o_gp); x->gemm_part_floats = gfloats; x->gemm_ticket = (int *)P(o_gt);
@@ -247,7 +250,7 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
         at.err = c.err;
         {
             ProbeScope ps(c, 1, l, view, s);
-            if ((e = launch_attention(c, at, s, c.Rw)) != cudaSuccess) return e;
+            if ((e = launch_attention(c, at, s, c.Rw, c.attn_simt_rows)) != cudaSuccess) return e;
         }
 
         GemmArgs o{};
@@ -295,16 +298,21 @@ static cudaError_t lm_head(Ctx &c, const void *fin, int B, int K, int lm_mode, f
 
 using namespace orthrus;
 
-#define CK(x)                                     \
-    do {                                          \
-        cudaError_t e_ = (x);                     \
-        if (e_ != cudaSuccess) return ORTHRUS_ERR_CUDA; \
+// cudaErrorNotSupported: a launcher found no kernel for these arguments
+// (e.g. the attention's buffers admit no tensor maps and the context holds no
+// room for the SIMT kernel's partials); nothing was launched.
+#define CK(x)                                                                              \
+    do {                                                                                   \
+        cudaError_t e_ = (x);                                                              \
+        if (e_ == cudaErrorNotSupported) return ORTHRUS_ERR_UNSUPPORTED;                   \
+        if (e_ != cudaSuccess) return ORTHRUS_ERR_CUDA;                                    \
     } while (0)
 
 static bool kv_ok(const orthrus_ctx_t *c, const orthrus_kv_t *kv)
 {
     if (!kv || !kv->k_pages || !kv->v_pages || !kv->block_table || !kv->seq_lens) return false;
     if (kv->num_pages < 1 || kv->max_pages_per_seq < 1) return false;
+    if ((uintptr_t)kv->k_pages % 16 || (uintptr_t)kv->v_pages % 16) return false;
     const int ps_mult = (c->cfg.dtype == ORTHRUS_BF16 && c->cfg.head_dim == 128) ? 64 : 16;
     if (kv->page_size < ps_mult || kv->page_size % ps_mult) return false;
     return true;
@@ -610,7 +618,7 @@ orthrus_status_t orthrus_dual_view_attention(orthrus_ctx_t *c, const orthrus_kv_
     at.n_splits = c->n_splits; at.part = c->attn_part; at.ml = c->attn_ml; at.err = c->err;
     at.xo = c->attn_xo; at.xml = c->attn_xml; at.xcnt = c->attn_xcnt; at.xrows = c->Rw * f.n_q_heads;
     at.xz = c->attn_xz;
-    CK(launch_attention(*c, at, s, batch * K));
+    CK(launch_attention(*c, at, s, batch * K, c->attn_simt_rows));
     return ORTHRUS_OK;
 }
 
@@ -646,7 +654,7 @@ orthrus_status_t orthrus_block_mask_attention(orthrus_ctx_t *c, const orthrus_kv
         at.n_splits = c->n_splits; at.part = c->attn_part; at.ml = c->attn_ml; at.err = c->err;
         at.xo = c->attn_xo; at.xml = c->attn_xml; at.xcnt = c->attn_xcnt; at.xrows = c->Rw * f.n_q_heads;
         at.xz = c->attn_xz;
-        CK(launch_attention(*c, at, s, nb * K));
+        CK(launch_attention(*c, at, s, nb * K, c->attn_simt_rows));
     }
     return ORTHRUS_OK;
 }

@@ -238,29 +238,45 @@ cudaError_t attention_init_attributes()
                                 (int)simt_smem(128));
 }
 
-// q_rows: token rows the q buffer holds (its tensor map's extent).
-cudaError_t launch_attention(const Ctx &c, const AttnArgs &a, cudaStream_t s, int q_rows)
+bool attn_tc_shape_ok(int dtype, int hd, int n_q, int n_kv, int page_size)
+{
+    if (dtype != ORTHRUS_BF16 || hd != 128 || n_kv < 1 || n_q % n_kv) return false;
+    const int g = n_q / n_kv;
+    return g >= 1 && 128 % g == 0 && page_size % 64 == 0;
+}
+
+cudaError_t launch_attention_simt(const Ctx &c, const AttnArgs &a, cudaStream_t s)
 {
     const int n_split_grid = (c.cfg.max_seq + a.split_tokens - 1) / a.split_tokens;
-    cudaError_t e = cudaErrorNotSupported;
-    // tensor-core path: one launch, the cluster combines and writes the output
-    if (c.cfg.dtype == ORTHRUS_BF16) e = launch_attn_tc_cached(c, a, n_split_grid, q_rows, s);
-    if (e != cudaErrorNotSupported) return e;
-    {
-        const int g = a.n_q / a.n_kv, R = a.K * g;
-        const int rgroups = (R + kAttnRowsSimt - 1) / kAttnRowsSimt;
-        dim3 grid(a.n_kv, a.B * rgroups, n_split_grid + (a.mode == 1 ? 1 : 0));
-        if (c.cfg.dtype == ORTHRUS_BF16)
-            e = launch_k(attn_split_simt<bf16>, grid, 128, simt_smem(a.hd), s, a, n_split_grid);
-        else
-            e = launch_k(attn_split_simt<float>, grid, 128, simt_smem(a.hd), s, a, n_split_grid);
-        c.launches += 1;
-    }
+    const int g = a.n_q / a.n_kv, R = a.K * g;
+    const int rgroups = (R + kAttnRowsSimt - 1) / kAttnRowsSimt;
+    dim3 grid(a.n_kv, a.B * rgroups, n_split_grid + (a.mode == 1 ? 1 : 0));
+    cudaError_t e;
+    if (c.cfg.dtype == ORTHRUS_BF16)
+        e = launch_k(attn_split_simt<bf16>, grid, 128, simt_smem(a.hd), s, a, n_split_grid);
+    else
+        e = launch_k(attn_split_simt<float>, grid, 128, simt_smem(a.hd), s, a, n_split_grid);
+    c.launches += 1;
     if (e != cudaSuccess) return e;
     c.launches += 1;
     const int rows = a.B * a.K * a.n_q;
     if (c.cfg.dtype == ORTHRUS_BF16) return launch_k(attn_combine<bf16>, (rows + 7) / 8, 256, 0, s, a);
     return launch_k(attn_combine<float>, (rows + 7) / 8, 256, 0, s, a);
+}
+
+// q_rows: token rows the q buffer holds (its tensor map's extent).
+cudaError_t launch_attention(const Ctx &c, const AttnArgs &a, cudaStream_t s, int q_rows, int simt_rows)
+{
+    const int n_split_grid = (c.cfg.max_seq + a.split_tokens - 1) / a.split_tokens;
+    // tensor-core path: one launch, the cluster combines and writes the output
+    if (attn_tc_shape_ok(c.cfg.dtype, a.hd, a.n_q, a.n_kv, a.kv.page_size)) {
+        const cudaError_t e = launch_attn_tc_cached(c, a, n_split_grid, q_rows, s);
+        if (e != cudaErrorNotSupported) return e;
+    }
+    // the SIMT kernel writes [B*K][n_q][n_splits] partials: only into room
+    // the caller reserved for them
+    if (a.B * a.K > simt_rows || !a.part || !a.ml || a.n_splits < n_split_grid + 1) return cudaErrorNotSupported;
+    return launch_attention_simt(c, a, s);
 }
 
 }  // namespace orthrus

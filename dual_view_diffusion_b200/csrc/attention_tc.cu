@@ -189,12 +189,6 @@ __device__ __forceinline__ void at_fence_after() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void at_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void at_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
-struct AtMaps {
-    CUtensorMap kc;   // 2-D cache K rows [slot rows][128], box {64, 64}
-    CUtensorMap vc;   // 2-D cache V^T rows [dim rows][page_size], box {64, 128}
-    CUtensorMap kb;   // 2-D transient K [rows][128], box {64, 64}
-    CUtensorMap vb;   // 2-D transient V^T [dim rows][Kp], box {64, 128}
-};
 
 // Key range of split s for sequence b: cache splits [s*S, ...) of the cache
 // part; in the diffusion view split n_split_grid is the block's own keys.
@@ -894,14 +888,11 @@ bool attn_tc_maps(const AttnArgs &a, int n_layers, AtMaps *m)
     return true;
 }
 
-cudaError_t launch_attn_tc(const AttnArgs &a, const AtMaps &maps, int n_split_grid, cudaStream_t s);
-
 // Maps for the call, built once per distinct (buffers, shape) and kept in
 // the context.
 cudaError_t launch_attn_tc_cached(const Ctx &c, const AttnArgs &a, int n_split_grid, int q_rows, cudaStream_t s)
 {
-    const int g = a.n_q / a.n_kv;
-    if (a.hd != 128 || g < 1 || kAtRows % g || a.kv.page_size % 64) return cudaErrorNotSupported;
+    if (!attn_tc_shape_ok(c.cfg.dtype, a.hd, a.n_q, a.n_kv, a.kv.page_size)) return cudaErrorNotSupported;
     AttnMapKey key{a.q, a.kv.k_pages, a.kv.v_pages, a.k_blk, a.kv.num_pages, a.kv.page_size, a.K, a.mode, q_rows};
     auto it = c.amaps.find(key);
     if (it == c.amaps.end()) {

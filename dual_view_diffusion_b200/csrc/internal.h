@@ -193,6 +193,7 @@ struct Ctx {
     void *res_x;             // [2*max_batch][d]
     float *attn_part;        // [Rw][n_q][n_splits][hd]
     float2 *attn_ml;         // [Rw][n_q][n_splits]
+    int attn_simt_rows;      // token rows attn_part / attn_ml hold (0: none; the tensor-core attention needs none)
     float *attn_xo;          // [kAttnMaxClusters][Rw][n_q][hd] (long contexts only, else null)
     float2 *attn_xml;        // [kAttnMaxClusters][Rw][n_q]
     int *attn_xcnt;          // [Rw][n_kv][8] tickets
@@ -246,14 +247,30 @@ cudaError_t gemm_init_attributes();
 cudaError_t gemm_tc_init_attributes();
 bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
 bool make_tmap_box(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows);
-struct AtMaps;
+// Tensor maps of one tensor-core attention call.
+struct AtMaps {
+    CUtensorMap kc;   // 2-D cache K rows [slot rows][128], box {64, 64}
+    CUtensorMap vc;   // 2-D cache V^T rows [dim rows][page_size], box {64, 128}
+    CUtensorMap kb;   // 2-D transient K [rows][128], box {64, 64}
+    CUtensorMap vb;   // 2-D transient V^T [dim rows][Kp], box {64, 128}
+};
 cudaError_t attn_tc_init_attributes();
 cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, cudaStream_t s);
 int sk_max_segments(int n_nt, int chunks);
 cudaError_t attention_init_attributes();
-cudaError_t launch_attention(const Ctx &c, const AttnArgs &a, cudaStream_t s, int q_rows);
+// The attention of one call: the tensor-core kernel when the shape and the
+// buffers allow it (attn_tc_shape_ok and tensor maps that encode), else the
+// SIMT split kernel and its combine.  Their partials (a.part / a.ml, stride
+// a.n_splits) hold simt_rows token rows; a call of more rows than that
+// (simt_rows = 0: none reserved) launches nothing and returns
+// cudaErrorNotSupported instead of falling back.
+cudaError_t launch_attention(const Ctx &c, const AttnArgs &a, cudaStream_t s, int q_rows, int simt_rows);
+cudaError_t launch_attention_simt(const Ctx &c, const AttnArgs &a, cudaStream_t s);
+// bf16, head_dim 128, GQA group dividing 128, pages of a multiple of 64 slots
+bool attn_tc_shape_ok(int dtype, int hd, int n_q, int n_kv, int page_size);
 cudaError_t launch_attn_tc_cached(const Ctx &c, const AttnArgs &a, int n_split_grid, int q_rows, cudaStream_t s);
-bool attn_tc_maps(const AttnArgs &a, int n_layers, int rows_total, AtMaps *m);
+cudaError_t launch_attn_tc(const AttnArgs &a, const AtMaps &maps, int n_split_grid, cudaStream_t s);
+bool attn_tc_maps(const AttnArgs &a, int n_layers, AtMaps *m);
 cudaError_t launch_embed(const Ctx &c, int mode, const int32_t *tokens, const int32_t *anchor,
                          const int32_t *draft, int B, int K, cudaStream_t s);
 cudaError_t launch_rmsnorm(const Ctx &c, float *h, const void *gain, void *out, int M, int pending, cudaStream_t s);

@@ -84,6 +84,7 @@ __device__ __forceinline__ void tw_lse4(const float (&x)[4], int n, float &m, fl
     for (int e = 1; e < 4; ++e)
         if (e < n) mc = fmaxf(mc, x[e]);
     if (mc > m) { s *= expf(m - mc); m = mc; }
+    if (m == -INFINITY) return;   // every logit so far is -inf (a masked id): nothing to add
     float add = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e)

@@ -257,6 +257,11 @@ orthrus_status_t orthrus_generate(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, co
  *           k_blk/v_blk [batch][K][n_kv][hd].
  *   out     [batch][K][n_q][hd]
  * Uses the layer-`layer` slice of the cache and the context's workspace.
+ * On a bf16 head_dim-128 context whose GQA group divides 128 the tensor-core
+ * kernel runs and needs q 16-byte aligned; otherwise (or when its tensor maps
+ * cannot be encoded over these buffers) the call returns
+ * ORTHRUS_ERR_UNSUPPORTED without launching anything, since such a context
+ * holds no room for the SIMT kernel's split partials.
  */
 orthrus_status_t orthrus_dual_view_attention(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, int32_t layer,
                                              int32_t mode, const void *q, const void *k_blk,
@@ -271,8 +276,12 @@ orthrus_status_t orthrus_dual_view_attention(orthrus_ctx_t *ctx, const orthrus_k
  * cudaMalloc from a plugin then fails or eats memory the pool was promised),
  * or code on a latency-critical path where cudaMalloc / cudaFree would
  * synchronise the device.  This call needs no context and no workspace: its
- * split partials live in a fixed 16 MiB array that the library holds on every
- * GPU it is loaded on, until the process exits.  It allocates nothing.
+ * scratch lives in a fixed 16 MiB array that the library holds on every GPU
+ * it is loaded on, until the process exits.  It allocates nothing.  It runs
+ * the kernels, launch shapes and summation orders that
+ * orthrus_dual_view_attention runs for the same config, so its output is
+ * bit-identical to that entry point's (long contexts included: from max_seq
+ * >= 8192 both spread a row group over several clusters).
  *
  *   cfg      model shape and limits (only the attention fields, n_layers,
  *            dtype, max_seq and split_tokens are read); q, k_blk, v_blk, out,
@@ -280,13 +289,24 @@ orthrus_status_t orthrus_dual_view_attention(orthrus_ctx_t *ctx, const orthrus_k
  *   dev_err  device pointer to a uint32 the caller owns, or NULL; it is
  *            cleared and then receives the device error bits of this call.
  *            With NULL the bits go to a word inside the fixed array.
- * Returns ORTHRUS_ERR_CAPACITY, launching nothing, when batch*K*n_q*
- * ceil(max_seq/split_tokens)*(head_dim*4 + 8) bytes plus a small header do not
- * fit in the 16 MiB.  The first call on a device also looks up the array's
- * device address and sets the kernels' shared-memory limit; make that first
- * call before capturing a stream.  All calls share the one array, so calls
- * whose work overlaps on the GPU (two streams, or two threads) race and give
- * wrong results: serialise them.
+ *
+ * Capacity.  With rows = batch*K, kp = K rounded up to 64, es = 2 (bf16) or
+ * 4 (fp32), S = ceil(max_seq / split_tokens) + 1 and up(x) = x rounded up to
+ * 256, the call needs
+ *     256 + up(4 * batch)
+ *   + (mode 1 only) 2 * up(batch * n_kv * kp * head_dim * es)   (block K, V^T)
+ *   + tensor-core path, max_seq >= 8192 only:
+ *       up(4 * rows * n_q * head_dim * 4) + up(4 * rows * n_q * 8) + rows * n_kv * 32
+ *   + SIMT path: up(rows * n_q * S * 8) + rows * n_q * S * head_dim * 4
+ * bytes, and returns ORTHRUS_ERR_CAPACITY, launching nothing, when that
+ * exceeds 16 MiB.  The tensor-core path is taken for bf16, head_dim 128, a
+ * GQA group dividing 128, q 16-byte aligned and buffers whose tensor maps
+ * encode; every other call takes the SIMT path, whose split partials are
+ * then counted.  The first call on a device also looks up the array's device
+ * address and sets the kernels' shared-memory limit; make that first call
+ * before capturing a stream.  All calls share the one array, which keeps the
+ * last call's contents, so calls whose work overlaps on the GPU (two
+ * streams, or two threads) race and give wrong results: serialise them.
  */
 orthrus_status_t orthrus_dual_view_attention_noalloc(const orthrus_config_t *cfg, const orthrus_kv_t *kv,
                                                     int32_t layer, int32_t mode, const void *q, const void *k_blk,

@@ -62,6 +62,28 @@ def test_topw_matches_oracle(eng_full_vocab, kind, W):
     assert (np.abs(lse - want_lse) <= 1e-5 * np.maximum(1.0, np.abs(want_lse))).all()
 
 
+def test_topw_masked_ids(eng_full_vocab):
+    """Masked vocabulary entries (-inf logits, a normal input) leave the
+    top-W and a finite log-sum-exp: rows whose leading ids, scattered ids,
+    or all but a few ids are -inf (so many threads meet only -inf logits
+    before their first finite one)."""
+    eng = eng_full_vocab
+    V = eng.shape.vocab
+    z = _f32((3, V), 44, "topw_masked", 3.0)
+    z[0, : V // 2] = -np.inf
+    z[1, ::3] = -np.inf
+    keep = np.zeros(V, bool)
+    keep[[5, 70000, V - 1]] = True
+    z[2, ~keep] = -np.inf
+    ids, vals, lse = eng.tree_topw(torch.from_numpy(z).cuda(), 3)
+    assert eng.check_error()[0] == 0
+    want_ids, want_lse = oracle.topw(z.astype(np.float64), 3)
+    assert np.array_equal(ids.cpu().numpy(), want_ids)
+    assert np.array_equal(vals.cpu().numpy(), np.take_along_axis(z, want_ids, axis=1))
+    assert np.isfinite(lse.cpu().numpy()).all()
+    assert (np.abs(lse.cpu().numpy() - want_lse) <= 1e-5 * np.maximum(1.0, np.abs(want_lse))).all()
+
+
 def test_topw_scalar_path():
     """A vocabulary that is not a multiple of 4 takes the kernel's scalar
     loads (the 16-byte path needs whole float4s per row)."""
