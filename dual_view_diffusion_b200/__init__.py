@@ -89,6 +89,7 @@ _SIGS = {
     "orthrus_tree_build": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P],
     "orthrus_tree_commit": [_P, C.POINTER(KV), _I, _I, _P, _P, _P, _P, _P, _P, _P, _P],
     "orthrus_debug_logits": [_P, _I, _I, _I, _P, _P],
+    "orthrus_debug_rows": [_P, _I, _I, _I, _P, _P, _P, _P],
     "orthrus_check_error": [_P, _P, C.POINTER(C.c_uint32)],
     "orthrus_set_probe": [_P, _I, _I, _I, C.POINTER(_P), C.POINTER(_P), _I],
     "orthrus_dual_view_attention_noalloc": [C.POINTER(Config), C.POINTER(KV), _I, _I, _P, _P, _P, _I, _I, _P, _P,
@@ -389,6 +390,18 @@ class Engine:
         out = self.torch.empty((B, K, self.shape.vocab), dtype=self.torch.float32, device=self.device)
         _check("orthrus_debug_logits", lib().orthrus_debug_logits(self.ctx, which, B, K, _ptr(out), _stream()))
         return out
+
+    def debug_rows(self, which, B, K):
+        """(tokens int32, log-probability of the row's token, log-sum-exp)
+        [B, K] of the last verify (which = 0: AR argmax, log p(y_k)) or draft
+        (which = 1: drafted token, log q(y_k))."""
+        t = self.torch
+        tok = t.empty((B, K), dtype=t.int32, device=self.device)
+        lp, lse = t.empty((B, K), dtype=t.float32, device=self.device), t.empty((B, K), dtype=t.float32,
+                                                                              device=self.device)
+        _check("orthrus_debug_rows", lib().orthrus_debug_rows(self.ctx, which, B, K, _ptr(tok), _ptr(lp), _ptr(lse),
+                                                              _stream()))
+        return tok, lp, lse
 
     def check_error(self):
         bits = C.c_uint32()

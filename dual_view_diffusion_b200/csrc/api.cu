@@ -713,6 +713,19 @@ orthrus_status_t orthrus_tree_commit(orthrus_ctx_t *c, const orthrus_kv_t *kv, i
     return ORTHRUS_OK;
 }
 
+orthrus_status_t orthrus_debug_rows(orthrus_ctx_t *c, int32_t which, int32_t batch, int32_t K, int32_t *tok,
+                                    float *logprob, float *lse, void *stream)
+{
+    if (!c || (which != 0 && which != 1) || batch < 1 || K < 1) return ORTHRUS_ERR_INVALID_ARG;
+    if (batch * K > c->R) return ORTHRUS_ERR_CAPACITY;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t n = (size_t)batch * K * 4;
+    if (tok) CK(cudaMemcpyAsync(tok, which ? c->draft : c->g, n, cudaMemcpyDeviceToDevice, s));
+    if (logprob) CK(cudaMemcpyAsync(logprob, which ? c->logq : c->logp, n, cudaMemcpyDeviceToDevice, s));
+    if (lse) CK(cudaMemcpyAsync(lse, which ? c->lse_q : c->lse_p, n, cudaMemcpyDeviceToDevice, s));
+    return ORTHRUS_OK;
+}
+
 orthrus_status_t orthrus_debug_logits(orthrus_ctx_t *c, int32_t which, int32_t batch, int32_t K, float *logits,
                                       void *stream)
 {

@@ -435,6 +435,21 @@ orthrus_status_t orthrus_debug_logits(orthrus_ctx_t *ctx, int32_t which, int32_t
                                       float *logits, void *stream);
 
 /*
+ * Test hook: the per-row results the last verify (which = 0) or draft
+ * (which = 1) left for consensus, for batch x K rows in [b][k] order —
+ *   which = 0: tok = the AR argmax g_k, logprob = log p_k(y_k) of the
+ *              verified token (log softmax(z/T) at T > 0, of z at T = 0),
+ *              lse = log-sum-exp of z/T (of z at T = 0);
+ *   which = 1: tok = the drafted token y_k (argmax, or the Gumbel-max
+ *              sample at T > 0), logprob = log q_k(y_k), lse likewise of
+ *              the diffusion view's logits.
+ * tok (int32), logprob and lse (fp32) are device [batch][K]; any may be
+ * NULL.  Device-to-device copies on the stream, no arithmetic.
+ */
+orthrus_status_t orthrus_debug_rows(orthrus_ctx_t *ctx, int32_t which, int32_t batch, int32_t K, int32_t *tok,
+                                    float *logprob, float *lse, void *stream);
+
+/*
  * Measurement hook.  While set, every forward of `view` (0 = AR: verify,
  * prefill and plain AR steps; 1 = diffusion draft) records caller-owned CUDA
  * events (cudaEvent_t passed as void*) on the launch stream around the

@@ -83,6 +83,7 @@ def lib():
             l.oc_uniform.restype = C.c_double
             l.oc_gumbel.argtypes = l.oc_uniform.argtypes
             l.oc_gumbel.restype = C.c_double
+            l.oc_gumbel_vec.argtypes = [C.c_uint64, C.c_uint32, C.c_uint32, C.c_uint32, C.c_int, _D]
             l.oc_argmax.argtypes = [_D, C.c_int, _D]
             l.oc_softmax_t.argtypes = [_D, C.c_int, C.c_double, _D]
             l.oc_sample_logits.argtypes = [_D, C.c_int, C.c_double, C.c_uint64, C.c_uint32, C.c_uint32,
@@ -102,7 +103,7 @@ def lib():
                                       C.c_uint64, C.c_int, _I, _I, P(C.c_int), _D, _D, _D, P(C.c_int)]
             l.oc_generate_iter.argtypes = [P(_Cfg), P(_Model), _I, C.c_int, C.c_int, C.c_int, C.c_double,
                                            C.c_uint64, C.c_int, C.c_int, _I, _I, P(C.c_int), _D, _D, _D,
-                                           P(C.c_int)]
+                                           P(C.c_int), _D]
             l.oc_enumerate_ar.argtypes = [P(_Cfg), P(_Model), _I, C.c_int, C.c_int, C.c_double, _D]
             l.oc_enumerate_orthrus.argtypes = [P(_Cfg), P(_Model), _I, C.c_int, C.c_int, C.c_int,
                                                C.c_double, C.c_int, _D]
@@ -312,6 +313,13 @@ def gumbel(seed, step, row, id_, purpose):
     return lib().oc_gumbel(seed, step, row, id_, purpose)
 
 
+def gumbel_vec(seed, step, row, purpose, n):
+    """gumbel(seed, step, row, i, purpose) for i = 0 .. n-1."""
+    g = np.empty(n)
+    lib().oc_gumbel_vec(seed, step, row, purpose, int(n), _dp(g))
+    return g
+
+
 def argmax(x):
     x = _f64(x); m = C.c_double()
     i = lib().oc_argmax(_dp(x), x.size, C.byref(m))
@@ -430,11 +438,13 @@ class Model:
 
     def generate(self, prompt, K, N, T=0.0, seed=0, method="orthrus", want_cache=False, iterations=1):
         """method 'orthrus' or 'ar'; iterations = diffusion passes per draft.
-        Returns a dict with tokens, n_per_cycle, cycles, min_margin, t and
+        Returns a dict with tokens, n_per_cycle, cycles, min_margin,
+        cycle_margin (the smallest decision margin of each cycle), t and
         (optionally) the committed cache."""
         p = _i32(prompt)
         out = np.zeros(N, np.int32)
         npc = np.zeros(N, np.int32)
+        cmg = np.zeros(N)
         cyc = C.c_int()
         mg = C.c_double()
         tt = C.c_int()
@@ -444,11 +454,11 @@ class Model:
             kc, vc = self.new_cache(cap)
         rc = lib().oc_generate_iter(C.byref(self.cfg), C.byref(self.model), _ip(p), p.size, int(K), int(N),
                                     float(T), seed, 1 if method == "orthrus" else 0, int(iterations), _ip(out),
-                                    _ip(npc), C.byref(cyc), C.byref(mg), _dp(kc), _dp(vc), C.byref(tt))
+                                    _ip(npc), C.byref(cyc), C.byref(mg), _dp(kc), _dp(vc), C.byref(tt), _dp(cmg))
         if rc:
             raise RuntimeError(f"oc_generate failed: {rc}")
         res = {"tokens": out, "n_per_cycle": npc[:cyc.value], "cycles": cyc.value, "min_margin": mg.value,
-               "t": tt.value}
+               "cycle_margin": cmg[:cyc.value], "t": tt.value}
         if want_cache:
             res["k_cache"], res["v_cache"] = kc, vc
         return res

@@ -386,6 +386,13 @@ double oc_gumbel(uint64_t seed, uint32_t step, uint32_t row, uint32_t id, uint32
     return -log(-log(oc_uniform(seed, step, row, id, purpose)));
 }
 
+/* The Gumbel noise of ids 0 .. n-1 of one (step, row, purpose): g[i] =
+ * oc_gumbel(seed, step, row, i, purpose). */
+void oc_gumbel_vec(uint64_t seed, uint32_t step, uint32_t row, uint32_t purpose, int n, double *g)
+{
+    for (int i = 0; i < n; ++i) g[i] = oc_gumbel(seed, step, row, (uint32_t)i, purpose);
+}
+
 /* Lowest index of the maximum; *margin (if given) = best - second best. */
 int oc_argmax(const double *x, int n, double *margin)
 {
@@ -559,6 +566,7 @@ int oc_consensus_sample(const double *p, const double *q, const int32_t *draft, 
             for (int i = 0; i < V; ++i) lr[i] = r[i] > 0.0 ? log(r[i]) : -INFINITY;
             double mg;
             emit[k] = oc_sample_logits(lr, V, 1.0, seed, step, (uint32_t)k, OC_PURPOSE_RESIDUAL, &mg);
+            if (min_margin && mg < *min_margin) *min_margin = mg;
         } else {
             emit[k] = g[k];
         }
@@ -575,14 +583,18 @@ int oc_consensus_sample(const double *p, const double *q, const int32_t *draft, 
  * Stops once N tokens are out; out[N].  n_per_cycle (may be NULL) receives
  * the tokens emitted by each cycle and *n_cycles their count.  *min_margin
  * (may be NULL) receives the smallest argmax / acceptance decision margin
- * seen, so callers can tell a decision that fp32 rounding could flip.
+ * seen, so callers can tell a decision that fp32 rounding could flip, and
+ * cycle_margin[c] (may be NULL; N entries) the smallest margin among the
+ * decisions of cycle c alone (draft argmaxes or samples, verify argmaxes at
+ * T = 0, acceptance tests and the residual draw at T > 0).
  * kc_out / vc_out (may be NULL) receive the final committed cache
  * [n_layers][cap][n_kv][hd], cap = P + N + K, rows beyond the committed length
  * zeroed.  *t_out (may be NULL) receives the final committed length.
  */
 int oc_generate_iter(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P, int K, int N,
                      double T, uint64_t seed, int method, int n_iter, int32_t *out, int32_t *n_per_cycle,
-                     int *n_cycles, double *min_margin, double *kc_out, double *vc_out, int *t_out)
+                     int *n_cycles, double *min_margin, double *kc_out, double *vc_out, int *t_out,
+                     double *cycle_margin)
 {
     if (!c || !w || !prompt || P < 1 || N < 1 || K < 1 || (method != 0 && method != 1) || n_iter < 1)
         return OC_ERR_ARG;
@@ -605,23 +617,24 @@ int oc_generate_iter(const oc_cfg *c, const oc_model *w, const int32_t *prompt, 
     int produced = 0, cycles = 0;
     while (produced < N) {
         int n;
+        double cm = INFINITY;   /* smallest decision margin of this cycle */
         if (method == 0) {
             rc = oc_forward(c, w, 0, 0, &anchor, 1, t, kc, vc, cap, z, NULL);
             if (rc) goto done;
-            double mg;
-            emit[0] = (T > 0.0) ? oc_sample_logits(z, V, T, seed, (uint32_t)produced, 0, OC_PURPOSE_AR, &mg)
-                                : oc_argmax(z, V, &mg);
-            if (min_margin && mg < *min_margin) *min_margin = mg;
+            emit[0] = (T > 0.0) ? oc_sample_logits(z, V, T, seed, (uint32_t)produced, 0, OC_PURPOSE_AR, &cm)
+                                : oc_argmax(z, V, &cm);
             n = 1;
         } else {
             rc = oc_draft_iter(c, w, kc, vc, cap, t, anchor, K, n_iter, T, seed, (uint32_t)cycles, draft, q, NULL,
-                               min_margin);
+                               &cm);
             if (rc) goto done;
-            rc = oc_verify(c, w, kc, vc, cap, t, anchor, draft, K, T, g, p, NULL, min_margin);
+            rc = oc_verify(c, w, kc, vc, cap, t, anchor, draft, K, T, g, p, NULL, &cm);
             if (rc) goto done;
-            n = (T > 0.0) ? oc_consensus_sample(p, q, draft, g, K, V, seed, (uint32_t)cycles, emit, min_margin)
+            n = (T > 0.0) ? oc_consensus_sample(p, q, draft, g, K, V, seed, (uint32_t)cycles, emit, &cm)
                           : oc_consensus_greedy(draft, g, K, emit);
         }
+        if (min_margin && cm < *min_margin) *min_margin = cm;
+        if (cycle_margin) cycle_margin[cycles] = cm;
         /* commit (§4.1 step 3): keep cache rows t .. t+n-1 (already written by
          * the AR forward for the accepted inputs), discard the rest. */
         t += n;
@@ -651,7 +664,7 @@ int oc_generate(const oc_cfg *c, const oc_model *w, const int32_t *prompt, int P
                 int *n_cycles, double *min_margin, double *kc_out, double *vc_out, int *t_out)
 {
     return oc_generate_iter(c, w, prompt, P, K, N, T, seed, method, 1, out, n_per_cycle, n_cycles, min_margin,
-                            kc_out, vc_out, t_out);
+                            kc_out, vc_out, t_out, NULL);
 }
 
 /* ------------------------------------------------------------------------ */

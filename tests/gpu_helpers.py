@@ -47,3 +47,44 @@ def read_cache(eng, layer, b, start, n):
 
 def bf16_normal(shape, seed, name):
     return synth.round_bf16(synth.normal(shape, 1.0, seed, name))
+
+
+def step_cycles(eng, prompts, lens, K, N, T, seed, iterations=1):
+    """Drive decode cycles through the public step calls (draft, verify,
+    commit) until every sequence has N tokens.  prompts: int array [B, S];
+    lens: per-sequence prompt lengths.  Returns, per sequence, the list of
+    (n, emitted tokens) of each cycle."""
+    p = torch.from_numpy(np.ascontiguousarray(prompts, dtype=np.int32))
+    B = p.shape[0]
+    eng.step.zero_()
+    anchor = eng.prefill(p, lens)
+    cycles = [[] for _ in range(B)]
+    done = [0] * B
+    while min(done) < N:
+        draft = eng.draft_block(anchor, K, temperature=T, seed=seed, iterations=iterations)
+        eng.verify_block(anchor, draft, K, temperature=T)
+        n, toks = eng.commit(anchor, K, temperature=T, seed=seed)
+        n, toks = n.cpu().numpy(), toks.cpu().numpy()
+        for b in range(B):
+            cycles[b].append((int(n[b]), toks[b, :n[b]].tolist()))
+            done[b] += int(n[b])
+    return cycles
+
+
+def first_divergent_cycle(cycles, ref, N):
+    """The first cycle whose (n, emitted tokens) differ from the oracle's
+    run (ref: Model.generate's dict), or -1.  Before that cycle both sides
+    emitted the same tokens, so their caches, anchors and step counters were
+    identical: a divergence there is decided by that cycle's own decisions,
+    whose smallest oracle margin is ref["cycle_margin"][c]."""
+    pos = 0
+    for c, (n, toks) in enumerate(cycles):
+        if pos >= N:
+            break
+        if c >= ref["cycles"]:
+            return c
+        m = min(n, N - pos)
+        if n != int(ref["n_per_cycle"][c]) or list(toks[:m]) != [int(x) for x in ref["tokens"][pos:pos + m]]:
+            return c
+        pos += n
+    return -1

@@ -1,9 +1,10 @@
 """The whole decode cycle on the GPU (paper notes §4.1-§4.3) against the CPU
 oracle and against the library's own plain AR decoding.
 
-* tiny fp32 model: token streams equal to the oracle's (greedy and T = 1,
-  seed 1); a divergence is only accepted at a decision whose oracle margin
-  is below what fp32 rounding can flip;
+* tiny fp32 model: every cycle's accepted length and tokens equal the
+  oracle's (greedy, T = 1 and T = 0.7); a divergence is only accepted in a
+  cycle one of whose own decisions has an oracle margin below what fp32
+  rounding can flip;
 * bf16 models: greedy Orthrus equals the GPU's plain AR greedy token for
   token (paper notes §4.2, §9.1); draft and verify logits within 2e-2
   (relative to the row's largest |logit|) of the fp64 oracle.
@@ -16,6 +17,7 @@ import torch
 
 import oracle
 import synth
+from gpu_helpers import first_divergent_cycle, step_cycles
 
 pytestmark = pytest.mark.gpu
 
@@ -41,16 +43,23 @@ def tiny(pkg):
     return w, eng
 
 
-@pytest.mark.parametrize("T,seed", [(0.0, 0), (1.0, 1)])
+@pytest.mark.parametrize("T,seed", [(0.0, 0), (1.0, 1), (0.7, 5)])
 def test_tiny_fp32_stream_matches_oracle(tiny, T, seed):
+    """Cycle by cycle through the step calls: every cycle's (n, tokens)
+    equals the oracle's, unless the first cycle that differs holds a
+    decision whose oracle margin is below what fp32 rounding can flip; the
+    whole-generation entry point gives the step calls' stream."""
     w, eng = tiny
     prompt = synth.make_prompt(synth.TINY, 16, 0)
-    out, st = eng.generate(torch.from_numpy(prompt)[None], 4, 32, T, seed)
-    ref = oracle.Model(w).generate(prompt, 4, 32, T, seed, "orthrus")
-    got = out[0].cpu().numpy()
-    i = _first_diff(got, ref["tokens"])
-    assert i < 0 or ref["min_margin"] < FP32_MARGIN, (i, got, ref["tokens"])
-    assert st["cycles"] == ref["cycles"] or i >= 0
+    N = 32
+    cyc = step_cycles(eng, prompt[None], [16], 4, N, T, seed)[0]
+    ref = oracle.Model(w).generate(prompt, 4, N, T, seed, "orthrus")
+    c = first_divergent_cycle(cyc, ref, N)
+    assert c < 0 or ref["cycle_margin"][c] < FP32_MARGIN, (c, cyc, ref["tokens"], ref["cycle_margin"])
+    stream = [x for _, toks in cyc for x in toks][:N]
+    out, st = eng.generate(torch.from_numpy(prompt)[None], 4, N, T, seed)
+    assert out[0].cpu().tolist() == stream
+    assert st["cycles"] == len(cyc)
     assert eng.check_error()[0] == 0
 
 
@@ -82,12 +91,14 @@ def test_tiny_batch_ragged(tiny):
     prompts = np.zeros((2, 16), np.int32)
     prompts[0] = p0
     prompts[1, :9] = p1
+    cyc = step_cycles(eng, prompts, [16, 9], 4, 24, 0.0, 0)
     out, _ = eng.generate(torch.from_numpy(prompts), 4, 24, 0.0, 0, lens=[16, 9])
     m = oracle.Model(w)
     for b, p in enumerate((p0, p1)):
         ref = m.generate(p, 4, 24, 0.0, 0, "orthrus")
-        i = _first_diff(out[b].cpu().numpy(), ref["tokens"])
-        assert i < 0 or ref["min_margin"] < FP32_MARGIN, (b, i)
+        c = first_divergent_cycle(cyc[b], ref, 24)
+        assert c < 0 or ref["cycle_margin"][c] < FP32_MARGIN, (b, c)
+        assert out[b].cpu().tolist() == [x for _, toks in cyc[b] for x in toks][:24]
 
 
 def test_tiny_step_api_and_cache_commit(tiny):

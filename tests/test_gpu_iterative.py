@@ -4,9 +4,9 @@ its own previous drafts, through orthrus_draft_block_iterative.
 
 * tiny fp32 model: the drafts of every pass count (2 and 3 passes, greedy and
   T = 1) equal the oracle's, and a whole sampled decode driven through the
-  step API with two-pass drafts equals the oracle's two-pass stream; a
-  divergence is only accepted at a decision whose oracle margin is below
-  what fp32 rounding can flip;
+  step API with two-pass drafts equals the oracle's two-pass stream cycle by
+  cycle; a divergence is only accepted in a draft (or a cycle) one of whose
+  own decisions has an oracle margin below what fp32 rounding can flip;
 * bf16, two layers of the Qwen3-1.7B shape: greedy decoding with two-pass
   drafts emits exactly the GPU's own plain-AR stream.
 """
@@ -16,6 +16,7 @@ import torch
 
 import oracle
 import synth
+from gpu_helpers import first_divergent_cycle, step_cycles
 
 pytestmark = pytest.mark.gpu
 
@@ -58,18 +59,10 @@ def test_tiny_two_pass_sampled_stream_matches_oracle(tiny):
     w, eng = tiny
     prompt = synth.make_prompt(synth.TINY, 16, 2)
     K, N, T, seed = 4, 24, 1.0, 7
-    eng.step.zero_()
-    anchor = eng.prefill(torch.from_numpy(prompt)[None])
-    got = []
-    while len(got) < N:
-        draft = eng.draft_block(anchor, K, temperature=T, seed=seed, iterations=2)
-        eng.verify_block(anchor, draft, K, temperature=T)
-        n, toks = eng.commit(anchor, K, temperature=T, seed=seed)
-        got += toks[0, :int(n[0])].tolist()
-    got = np.array(got[:N], np.int32)
+    cyc = step_cycles(eng, prompt[None], [prompt.size], K, N, T, seed, iterations=2)[0]
     ref = oracle.Model(w).generate(prompt, K, N, T, seed, "orthrus", iterations=2)
-    i = int(np.nonzero(got != ref["tokens"])[0][0]) if (got != ref["tokens"]).any() else -1
-    assert i < 0 or ref["min_margin"] < FP32_MARGIN, (i, got, ref["tokens"])
+    c = first_divergent_cycle(cyc, ref, N)
+    assert c < 0 or ref["cycle_margin"][c] < FP32_MARGIN, (c, cyc, ref["tokens"])
     assert eng.check_error()[0] == 0
 
 
