@@ -88,8 +88,11 @@ _SIGS = {
     "orthrus_tree_topw": [_P, _P, _I, _I, _P, _P, _P, _P],
     "orthrus_tree_build": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P],
     "orthrus_tree_commit": [_P, C.POINTER(KV), _I, _I, _P, _P, _P, _P, _P, _P, _P, _P],
+    "orthrus_verify_tree": [_P, C.POINTER(KV), _P, _P, _P, _I, _I, _P, _P],
     "orthrus_debug_logits": [_P, _I, _I, _I, _P, _P],
     "orthrus_debug_rows": [_P, _I, _I, _I, _P, _P, _P, _P],
+    "orthrus_adaptive_len": [_P, _I, _I, C.c_float, _P, _P, _P],
+    "orthrus_commit_adaptive": [_P, C.POINTER(KV), _I, _I, _P, _P, _P, _P, _P, _P],
     "orthrus_check_error": [_P, _P, C.POINTER(C.c_uint32)],
     "orthrus_set_probe": [_P, _I, _I, _I, C.POINTER(_P), C.POINTER(_P), _I],
     "orthrus_dual_view_attention_noalloc": [C.POINTER(Config), C.POINTER(KV), _I, _I, _P, _P, _P, _I, _I, _P, _P,
@@ -286,6 +289,29 @@ class Engine:
                                                       _ptr(n), _ptr(toks), _ptr(anchor), _stream()))
         return n, toks
 
+    def adaptive_len(self, B, K, h_max, kt=None, entropy=False):
+        """Per-sequence verify length after a greedy draft (rows whose
+        entropy is at most h_max extend it).  Returns kt [B] (and the draft
+        rows' entropies [B, K] when entropy=True)."""
+        t = self.torch
+        kt = kt if kt is not None else t.empty(B, dtype=t.int32, device=self.device)
+        ent = t.empty((B, K), dtype=t.float32, device=self.device) if entropy else None
+        _check("orthrus_adaptive_len", lib().orthrus_adaptive_len(self.ctx, B, K, float(h_max), _ptr(kt), _ptr(ent),
+                                                                  _stream()))
+        return (kt, ent) if entropy else kt
+
+    def commit_adaptive(self, anchor, K, kt, step=None, n_out=None, tokens_out=None):
+        """Greedy consensus over the first kt[b] verified rows + commit;
+        anchor is updated in place.  Returns (n, tokens)."""
+        B = anchor.numel()
+        t = self.torch
+        n = n_out if n_out is not None else t.empty(B, dtype=t.int32, device=self.device)
+        toks = tokens_out if tokens_out is not None else t.empty((B, K), dtype=t.int32, device=self.device)
+        _check("orthrus_commit_adaptive", lib().orthrus_commit_adaptive(
+            self.ctx, C.byref(self.kv), B, K, _ptr(kt), _ptr(self.step if step is None else step), _ptr(n),
+            _ptr(toks), _ptr(anchor), _stream()))
+        return n, toks
+
     def ar_step(self, anchor, temperature=0.0, seed=0, step=None, token_out=None):
         B = anchor.numel()
         t = self.torch
@@ -370,6 +396,18 @@ class Engine:
             self.ctx, _ptr(ids), _ptr(vals), _ptr(lse), B, D, W, nodes, _ptr(par), _ptr(tok), _ptr(dep), _ptr(sc),
             _ptr(nr), _stream()))
         return par, tok, dep, sc, nr
+
+    def verify_tree(self, anchor, parent, token):
+        """Tree-masked AR verification of trees parent/token [B, rows] (row 0
+        the anchor): returns each row's AR argmax g [B, rows]."""
+        t = self.torch
+        for name, x in (("anchor", anchor), ("parent", parent), ("token", token)):
+            _need(x, t.int32, name)
+        B, R = (int(x) for x in parent.shape)
+        g = t.empty((B, R), dtype=t.int32, device=self.device)
+        _check("orthrus_verify_tree", lib().orthrus_verify_tree(self.ctx, C.byref(self.kv), _ptr(anchor), _ptr(parent),
+                                                                _ptr(token), B, R, _ptr(g), _stream()))
+        return g
 
     def tree_commit(self, parent, token, n_rows, g, anchor):
         """Greedy acceptance on verified trees [B, rows] and the commit of the

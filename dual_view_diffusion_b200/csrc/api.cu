@@ -110,9 +110,10 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
     const size_t o_invf = take((size_t)c.head_dim / 2 * 8);
     const size_t o_lm = take(Rlm * n_vtiles * sizeof(LmPart));
     const size_t o_tok = take(Rw * 4), o_pos = take(mb * 4), o_bt = take(mb * 4), o_pr = take(4);
+    const size_t o_ttok = take(R * 4), o_tdep = take(R * 4), o_tmask = take(R * 16);
     const size_t o_bz = take(mb * 4);   // zeros, never written
     const size_t o_dr = take(R * 4), o_lq = take(R * 4), o_lsq = take(R * 4), o_g = take(R * 4), o_lp = take(R * 4),
-                 o_lsp = take(R * 4);
+                 o_lsp = take(R * 4), o_ent = take(R * 4);
     const size_t o_rj = take(mb * 4), o_rt = take(mb * 4), o_any = take(4), o_err = take(4), o_prod = take(mb * 4),
                  o_step = take(8), o_nb = take(mb * 4), o_tb = take(R * 4), o_ab = take(mb * 4);
     const size_t total = off;
@@ -131,8 +132,10 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
         x->rope_invf = (double *)P(o_invf);
         x->tok = (int32_t *)P(o_tok); x->pos0 = (int32_t *)P(o_pos); x->bt_rows = (int32_t *)P(o_bt);
         x->bt_zero = (int32_t *)P(o_bz);
+        x->tree_tok = (int32_t *)P(o_ttok); x->tree_depth = (int32_t *)P(o_tdep); x->tree_mask = (uint32_t *)P(o_tmask);
         x->prefill_row = (int32_t *)P(o_pr);
         x->draft = (int32_t *)P(o_dr); x->logq = (float *)P(o_lq); x->lse_q = (float *)P(o_lsq);
+        x->ent = (float *)P(o_ent);
         x->g = (int32_t *)P(o_g); x->logp = (float *)P(o_lp); x->lse_p = (float *)P(o_lsp);
         x->rej_row = (int32_t *)P(o_rj); x->res_tok = (int32_t *)P(o_rt); x->any_reject = (int *)P(o_any);
         x->err = (unsigned *)P(o_err); x->produced = (int32_t *)P(o_prod); x->step = (int64_t *)P(o_step);
@@ -150,7 +153,8 @@ static void rebase(Ctx *x, char *ws)
     fix(x->h); fix(x->a); fix(x->q); fix(x->attn_o); fix(x->act); fix(x->k_diff); fix(x->v_diff); fix(x->blk_pack);
     fix(x->fin_draft); fix(x->fin_verify); fix(x->res_x); fix(x->attn_part); fix(x->attn_ml); fix(x->gemm_part);
     fix(x->gemm_ticket); fix(x->lm_part); fix(x->resid_part); fix(x->rope_invf); fix(x->tok); fix(x->pos0); fix(x->bt_rows); fix(x->bt_zero); fix(x->prefill_row);
-    fix(x->draft); fix(x->logq); fix(x->lse_q); fix(x->g); fix(x->logp); fix(x->lse_p); fix(x->rej_row);
+    fix(x->tree_tok); fix(x->tree_depth); fix(x->tree_mask);
+    fix(x->draft); fix(x->logq); fix(x->lse_q); fix(x->ent); fix(x->g); fix(x->logp); fix(x->lse_p); fix(x->rej_row);
     fix(x->res_tok); fix(x->any_reject); fix(x->err); fix(x->produced); fix(x->step); fix(x->n_buf);
     fix(x->tok_buf); fix(x->anchor_buf);
     if (x->attn_xz > 1) { fix(x->attn_xo); fix(x->attn_xml); fix(x->attn_xcnt); }
@@ -212,8 +216,11 @@ struct ProbeScope {
 //   view 1: diffusion W^diff, K/V into the transient buffer, block
 //           bidirectional (mode 1)
 // fin (nullable): final-norm rows for the LM head.
+// rope_pos / tree_mask (view 0 only, nullable): the tree-masked verify's
+// per-row rotary positions (depths) and ancestor masks.
 static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int K, const int32_t *pos0,
-                           const int32_t *bt_rows, void *fin, cudaStream_t s)
+                           const int32_t *bt_rows, void *fin, cudaStream_t s, const int32_t *rope_pos = nullptr,
+                           const uint32_t *tree_mask = nullptr)
 {
     const orthrus_config_t &f = c.cfg;
     const int M = B * K, hd = f.head_dim;
@@ -232,7 +239,7 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
         q.epi = EPI_QKV; q.q_out = c.q; q.n_q = f.n_q_heads; q.n_kv = f.n_kv_heads; q.hd = hd; q.layer = l;
         q.kv_to_cache = view == 0; q.k_blk = c.k_diff; q.v_blk = c.v_diff; q.kp = c.kp; q.bmax = f.max_batch;
         q.kv = kv_view(kv); q.pos0 = pos0; q.bt_rows = bt_rows; q.K = K; q.rope_theta = (double)f.rope_theta;
-        q.rope_invf = c.rope_invf;
+        q.rope_invf = c.rope_invf; q.rope_pos = view == 0 ? rope_pos : nullptr;
         {
             ProbeScope ps(c, 0, l, view, s);
             if ((e = launch_gemm(c, q, s)) != cudaSuccess) return e;
@@ -247,6 +254,7 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
         at.split_tokens = f.split_tokens; at.n_splits = c.n_splits; at.part = c.attn_part; at.ml = c.attn_ml;
         at.xo = c.attn_xo; at.xml = c.attn_xml; at.xcnt = c.attn_xcnt; at.xrows = c.Rw * f.n_q_heads;
         at.xz = c.attn_xz;
+        at.tree_mask = view == 0 ? tree_mask : nullptr;
         at.err = c.err;
         {
             ProbeScope ps(c, 1, l, view, s);
@@ -489,6 +497,27 @@ orthrus_status_t orthrus_commit(orthrus_ctx_t *c, const orthrus_kv_t *kv, int32_
     return ORTHRUS_OK;
 }
 
+orthrus_status_t orthrus_adaptive_len(orthrus_ctx_t *c, int32_t batch, int32_t K, float h_max, int32_t *kt,
+                                      float *entropy, void *stream)
+{
+    if (!c || !kt || batch < 1 || K < 1 || h_max != h_max) return ORTHRUS_ERR_INVALID_ARG;
+    if (batch > c->cfg.max_batch || K > c->cfg.max_block) return ORTHRUS_ERR_CAPACITY;
+    CK(launch_adaptive_len(*c, batch, K, h_max, kt, entropy, (cudaStream_t)stream));
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_commit_adaptive(orthrus_ctx_t *c, const orthrus_kv_t *kv, int32_t batch, int32_t K,
+                                         const int32_t *kt, int64_t *step, int32_t *n_out, int32_t *tokens_out,
+                                         int32_t *anchor_io, void *stream)
+{
+    orthrus_status_t st = check_step(c, kv, batch, K);
+    if (st != ORTHRUS_OK) return st;
+    if (!kt || !step || !n_out || !anchor_io) return ORTHRUS_ERR_INVALID_ARG;
+    CK(launch_commit(*c, *kv, batch, K, 0.f, 0, step, nullptr, n_out, tokens_out, anchor_io, nullptr, 0, 0,
+                     (cudaStream_t)stream, kt));
+    return ORTHRUS_OK;
+}
+
 static orthrus_status_t ar_step_impl(orthrus_ctx_t *c, const orthrus_kv_t *kv, int batch, float temperature,
                                      uint64_t seed, int64_t *step, int32_t *token_out, int32_t *anchor_io,
                                      int32_t *append, int stride, int amax, cudaStream_t s)
@@ -691,6 +720,24 @@ orthrus_status_t orthrus_tree_build(orthrus_ctx_t *c, const int32_t *ids, const 
     a.ids = ids; a.vals = vals; a.lse = lse; a.D = depth; a.W = width; a.N = nodes;
     a.parent = parent; a.token = token; a.depth = node_depth; a.score = score; a.n_rows = n_rows;
     CK(launch_tree_build(*c, a, batch, (cudaStream_t)stream));
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_verify_tree(orthrus_ctx_t *c, const orthrus_kv_t *kv, const int32_t *anchor,
+                                     const int32_t *parent, const int32_t *token, int32_t batch, int32_t rows,
+                                     int32_t *g, void *stream)
+{
+    orthrus_status_t st = check_step(c, kv, batch, rows);
+    if (st != ORTHRUS_OK) return st;
+    if (!anchor || !parent || !token || !g) return ORTHRUS_ERR_INVALID_ARG;
+    if (rows > 128) return ORTHRUS_ERR_CAPACITY;
+    cudaStream_t s = (cudaStream_t)stream;
+    CK(launch_tree_prep(*c, anchor, parent, token, batch, rows, s));
+    CK(launch_embed(*c, 2, c->tree_tok, nullptr, nullptr, batch, rows, s));
+    CK(forward(*c, *kv, 0, batch, rows, kv->seq_lens, c->bt_rows, c->fin_verify, s, c->tree_depth, c->tree_mask));
+    CK(lm_head(*c, c->fin_verify, batch, rows, 0, 0.f, 0, nullptr, nullptr, s));
+    CK(launch_lm_finalize_impl(*c, 0, batch, rows, 0.f, nullptr, nullptr, s));
+    CK(cudaMemcpyAsync(g, c->g, (size_t)batch * rows * 4, cudaMemcpyDeviceToDevice, s));
     return ORTHRUS_OK;
 }
 

@@ -116,14 +116,20 @@ __global__ void __launch_bounds__(128) attn_split_simt(AttnArgs a, int n_split_g
         __syncthreads();
         for (int r = warp; r < nr; r += 4) {
             const int k = (r0 + r) / g;
-            const int lim = (a.mode == 0 && !block) ? t + k + 1 : key1;
+            const bool tree = a.mode == 0 && a.tree_mask != nullptr;
+            const int lim = (a.mode == 0 && !block && !tree) ? t + k + 1 : key1;
             float sv[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int j = lane + 32 * h, p = p0 + j;
                 float acc = 0.f;
                 for (int d = 0; d < hd; ++d) acc = fmaf(qs[r * hd + d], ks[j * hp + d], acc);
-                sv[h] = (p < lim && p < key1) ? acc * scale : -INFINITY;
+                bool see = p < lim && p < key1;
+                if (tree && see && p >= t) {   // a block key: the row's ancestors and itself only
+                    const int jb = p - t;
+                    see = jb < 128 && ((a.tree_mask[(size_t)(b * a.K + k) * 4 + (jb >> 5)] >> (jb & 31)) & 1u);
+                }
+                sv[h] = see ? acc * scale : -INFINITY;
             }
             float tmax = fmaxf(sv[0], sv[1]);
 #pragma unroll

@@ -241,6 +241,19 @@ __device__ __forceinline__ uint4 ld_peer4u(uint32_t addr)
     asm volatile("ld.shared::cluster.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
     return v;
 }
+// Tree verify: 32 visibility bits of block indices j0 .. j0+31 for one query
+// row (bit b <-> block index j0 + b): a negative index is a cache key
+// (visible), 0 .. 127 the row's ancestor bits m, beyond the block nothing.
+__device__ __forceinline__ uint32_t tree_window(const uint32_t (&m)[4], int j0)
+{
+    const int w = j0 >> 5, sh = j0 & 31;   // floor division: j0 may be negative
+    auto word = [&](int i) -> uint32_t {
+        return i < 0 ? 0xffffffffu : i == 0 ? m[0] : i == 1 ? m[1] : i == 2 ? m[2] : i == 3 ? m[3] : 0u;
+    };
+    const uint32_t lo = word(w), hi = word(w + 1);
+    return sh ? (lo >> sh) | (hi << (32 - sh)) : lo;
+}
+
 __device__ __forceinline__ float ex2(float x)   // 2^x, MUFU; subnormal results flush to zero
 {
     float y;
@@ -481,6 +494,14 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
         // kRescaleSlack: the result is the same softmax, P stays <= 2^slack
         float m_use = -INFINITY, l_run = 0.f;
         int last = -1;   // this warpgroup's last tile
+        // tree verify: this row's ancestor bits (rows past the block see nothing
+        // of it; they are never written)
+        const bool tree = a.mode == 0 && a.tree_mask != nullptr;
+        uint32_t tm[4] = {0u, 0u, 0u, 0u};
+        if (tree && kblk < k_hi) {
+            const uint4 v = *(const uint4 *)(a.tree_mask + (size_t)(b * a.K + kblk) * 4);
+            tm[0] = v.x; tm[1] = v.y; tm[2] = v.z; tm[3] = v.w;
+        }
         if (h == 0) {   // Q row -> TMEM lane row (bf16 pairs); rows past the block are zero
             uint32_t qr[64];
             if (kblk < k_hi) {
@@ -503,7 +524,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
         }
         for (int s = ci; s < n_total && ok; s += Ctot) {
             const AtSplit sp = at_split(a, s, n_split_grid, t);
-            const int lim = min(sp.key1, sp.block ? sp.key1 : (a.mode == 0 ? t + kblk + 1 : sp.key1));
+            const int lim = min(sp.key1, (sp.block || tree) ? sp.key1 : (a.mode == 0 ? t + kblk + 1 : sp.key1));
             for (int j = 0; j < sp.ntiles; ++j, ++jj) {
                 if ((int)(jj & 1) != h) continue;
                 last = (int)jj;
@@ -521,6 +542,15 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
 #pragma unroll
                     for (int c = 0; c < kAtKeys; ++c)
                         if (c >= vis) sr[c] = __float_as_uint(-INFINITY);
+                }
+                const int j0 = sp.key0 + j * kAtKeys - t;          // block index of this tile's first key
+                if (tree && j0 + kAtKeys > 0) {                    // the tile reaches the block
+                    uint32_t wv[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) wv[i] = tree_window(tm, j0 + 32 * i);
+#pragma unroll
+                    for (int c = 0; c < kAtKeys; ++c)
+                        if (!((wv[c >> 5] >> (c & 31)) & 1u)) sr[c] = __float_as_uint(-INFINITY);
                 }
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll

@@ -152,6 +152,7 @@ struct LmArgs {
     float inv_temp;
     int32_t *draft, *draft_user, *g, *res_tok;
     float *logq, *lse_q, *logp, *lse_p;
+    float *ent;
     const int32_t *given, *rej_row;
     unsigned *err;
 };
@@ -197,9 +198,14 @@ __global__ void __launch_bounds__(256) lm_finalize_kernel(LmArgs a)
     const unsigned has = __ballot_sync(0xffffffffu, !isnan(zid));
     if (has) zid = __shfl_sync(0xffffffffu, zid, __ffs(has) - 1);
     const float it = a.inv_temp > 0.f ? a.inv_temp : 1.0f;
-    float s = 0.f;
-    for (int i = lane; i < a.n_vtiles; i += 32) s += p[i].zsum * expf((p[i].zmax - zm) * it);
+    float s = 0.f, ez = 0.f;
+    for (int i = lane; i < a.n_vtiles; i += 32) {
+        const float f = expf((p[i].zmax - zm) * it);
+        s += p[i].zsum * f;
+        if (a.mode == 1) ez = fmaf(p[i].zez, f, ez);
+    }
     s = warp_sum(s);
+    if (a.mode == 1) ez = warp_sum(ez);
     const float lse = zm * it + logf(s);
     if (lane != 0) return;
     if (!isfinite(lse)) raise_err(a.err, ORTHRUS_DEVERR_NONFINITE);
@@ -214,6 +220,8 @@ __global__ void __launch_bounds__(256) lm_finalize_kernel(LmArgs a)
         if (a.draft_user) a.draft_user[w] = tok;
         a.lse_q[w] = lse;
         a.logq[w] = (a.inv_temp > 0.f ? gz : zm) * it - lse;
+        // entropy of softmax(z / T): LSE(z / T) - E[z] / T
+        if (a.ent) a.ent[w] = lse - it * (ez / s);
     } else {
         a.g[w] = a.inv_temp > 0.f ? ga : za;
     }
@@ -226,6 +234,7 @@ struct CommitArgs {
     uint64_t seed;
     int64_t *step;
     const int32_t *force_n;
+    const int32_t *kt;       // greedy: per-sequence verify length (consensus over its first kt rows), or null
     const int32_t *draft, *g, *res_tok;
     const float *logp, *logq;
     int32_t *rej_row;
@@ -252,7 +261,9 @@ __global__ void commit_decide_kernel(CommitArgs a)
         if (a.force_n) {
             n = min(max(a.force_n[b], 1), a.K);
         } else if (a.inv_temp <= 0.f) {
-            for (int k = 0; k < a.K; ++k)
+            const int kt = a.kt ? min(max(a.kt[b], 1), a.K) : a.K;
+            n = kt;
+            for (int k = 0; k < kt; ++k)
                 if (a.draft[b * a.K + k] != a.g[b * a.K + k]) { n = k + 1; break; }
         } else {
             const uint32_t step = (uint32_t)*a.step;
@@ -331,6 +342,22 @@ __global__ void ar_commit_kernel(int B, const int32_t *g, int64_t *step, int32_t
     }
     __syncthreads();
     if (threadIdx.x == 0) *step += 1;
+}
+
+// Adaptive block length (reading of the paper-notes page §7.4 / §9.6): per
+// sequence, 1 + the number of leading drafted tokens y_1, y_2, ... (y_k from
+// draft row k-1) whose rows' entropies are at most h_max, at most K.
+__global__ void adaptive_len_kernel(const float *ent, int B, int K, float h_max, int32_t *kt, float *ent_out)
+{
+    pdl_trigger();
+    pdl_wait();
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= B) return;
+    int k = 1;
+    while (k < K && ent[b * K + k - 1] <= h_max) ++k;
+    kt[b] = k;
+    if (ent_out)
+        for (int i = 0; i < K; ++i) ent_out[b * K + i] = ent[b * K + i];
 }
 
 __global__ void set_lens_kernel(int32_t *seq_lens, int b, int value, int32_t *anchor_out, const int32_t *last_tok)
@@ -479,7 +506,7 @@ cudaError_t launch_lm_finalize_impl(const Ctx &c, int mode, int B, int K, float 
     a.inv_temp = temperature > 0.f ? 1.0f / temperature : 0.f;
     a.draft = c.draft; a.draft_user = tok_out; a.g = c.g; a.res_tok = c.res_tok;
     a.logq = c.logq; a.lse_q = c.lse_q; a.logp = c.logp; a.lse_p = c.lse_p;
-    a.given = given; a.rej_row = c.rej_row; a.err = c.err;
+    a.given = given; a.rej_row = c.rej_row; a.err = c.err; a.ent = c.ent;
     const int rows = mode == 3 ? B : B * K;
     c.launches += 1;
     return launch_k(lm_finalize_kernel, (rows + 7) / 8, 256, 0, s, a);
@@ -497,7 +524,7 @@ static CommitArgs commit_args(const Ctx &c, const orthrus_kv_t &kv, int B, int K
 {
     CommitArgs a;
     a.B = B; a.K = K; a.inv_temp = temperature > 0.f ? 1.0f / temperature : 0.f;
-    a.seed = seed; a.step = step; a.force_n = force_n;
+    a.seed = seed; a.step = step; a.force_n = force_n; a.kt = nullptr;
     a.draft = c.draft; a.g = c.g; a.res_tok = c.res_tok; a.logp = c.logp; a.logq = c.logq;
     a.rej_row = c.rej_row; a.any_reject = c.any_reject;
     a.fin_verify = c.fin_verify; a.fin_draft = c.fin_draft; a.res_x = c.res_x;
@@ -510,10 +537,11 @@ static CommitArgs commit_args(const Ctx &c, const orthrus_kv_t &kv, int B, int K
 cudaError_t launch_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int K, float temperature, uint64_t seed,
                           int64_t *step, const int32_t *force_n, int32_t *n_out, int32_t *tokens_out,
                           int32_t *anchor_io, int32_t *append_out, int append_stride, int append_max,
-                          cudaStream_t s)
+                          cudaStream_t s, const int32_t *kt)
 {
     CommitArgs a = commit_args(c, kv, B, K, temperature, seed, step, force_n, n_out, tokens_out, anchor_io,
                                append_out, append_stride, append_max);
+    a.kt = kt;
     c.launches += 2;
     cudaError_t e = launch_k(commit_decide_kernel, B, 128, 0, s, a);
     if (e != cudaSuccess) return e;
@@ -547,6 +575,12 @@ cudaError_t launch_set_lens(const Ctx &, int32_t *seq_lens, int b, int value, in
                             const int32_t *last_tok, cudaStream_t s)
 {
     return launch_k(set_lens_kernel, 1, 1, 0, s, seq_lens, b, value, anchor_out, last_tok);
+}
+
+cudaError_t launch_adaptive_len(const Ctx &c, int B, int K, float h_max, int32_t *kt, float *ent_out, cudaStream_t s)
+{
+    c.launches += 1;
+    return launch_k(adaptive_len_kernel, (B + 127) / 128, 128, 0, s, (const float *)c.ent, B, K, h_max, kt, ent_out);
 }
 
 cudaError_t launch_set_int(int32_t *p, int v, cudaStream_t s)

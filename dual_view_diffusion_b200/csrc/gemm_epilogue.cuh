@@ -106,13 +106,14 @@ __device__ inline void qkv_prepare(const GemmArgs &a, QkvPre &pre, int mt, int n
         long long dst = -1;
         if (row < a.M) {
             const int b = row / a.K, k = row % a.K;
-            pos = a.pos0[b] + k;
+            const int spos = a.pos0[b] + k;                              // cache slot
+            pos = a.rope_pos ? a.pos0[b] + a.rope_pos[row] : spos;       // rotary position
             if (kind == 0) {
                 dst = (long long)row * a.n_q * kTileN + head * kTileN;
             } else if (a.kv_to_cache) {
-                const int pidx = pos / a.kv.page_size;
+                const int pidx = spos / a.kv.page_size;
                 int page = -1;
-                if (pos >= 0 && pidx < a.kv.max_pages) {
+                if (spos >= 0 && pidx < a.kv.max_pages) {
                     page = a.kv.block_table[(size_t)a.bt_rows[b] * a.kv.max_pages + pidx];
                     if (page >= a.kv.num_pages) page = -1;
                 }
@@ -120,7 +121,7 @@ __device__ inline void qkv_prepare(const GemmArgs &a, QkvPre &pre, int mt, int n
                     raise_err(a.err, ORTHRUS_DEVERR_CAPACITY);
                 } else {
                     const long long hh = ((long long)a.layer * a.kv.num_pages + page) * a.n_kv + head;
-                    const int slot = pos % a.kv.page_size;
+                    const int slot = spos % a.kv.page_size;
                     dst = kind == 1 ? (hh * a.kv.page_size + slot) * kTileN : hh * kTileN * a.kv.page_size + slot;
                 }
             } else {
@@ -301,18 +302,19 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
             }
         }
     } else if (epi == EPI_QKV) {
-        __shared__ int s_pos[kTileM], s_page[kTileM];
+        __shared__ int s_pos[kTileM], s_page[kTileM], s_slot[kTileM];
         __shared__ double s_invf[64];
         const int half = a.hd / 2, Nq = a.n_q * a.hd, Nk = a.n_kv * a.hd;
         if (tid < kTileM) {
             const int row = mt * kTileM + tid;
-            int pos = -1, page = -1;
+            int pos = -1, page = -1, spos = -1;
             if (row < a.M) {
                 const int b = row / a.K, k = row % a.K;
-                pos = a.pos0[b] + k;
+                spos = a.pos0[b] + k;                                  // cache slot
+                pos = a.rope_pos ? a.pos0[b] + a.rope_pos[row] : spos; // rotary position
                 if (a.kv_to_cache) {
-                    const int pidx = pos / a.kv.page_size;
-                    if (pos >= 0 && pidx < a.kv.max_pages) {
+                    const int pidx = spos / a.kv.page_size;
+                    if (spos >= 0 && pidx < a.kv.max_pages) {
                         page = a.kv.block_table[(size_t)a.bt_rows[b] * a.kv.max_pages + pidx];
                         if (page >= a.kv.num_pages) page = -1;
                     }
@@ -321,6 +323,7 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
             }
             s_pos[tid] = pos;
             s_page[tid] = page;
+            s_slot[tid] = spos;
         } else if (tid >= 64 && tid - 64 < half) {
             s_invf[tid - 64] = a.rope_invf[tid - 64];
         }
@@ -353,7 +356,7 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
                 const int page = s_page[m];
                 if (page < 0) continue;
                 const size_t head = ((size_t)a.layer * a.kv.num_pages + page) * a.n_kv + kvh;
-                const int slot = pos % a.kv.page_size;
+                const int slot = s_slot[m] % a.kv.page_size;
                 if (is_k) { base = (head * a.kv.page_size + slot) * a.hd + d; step = 1; }
                 else { base = (head * a.hd + d) * a.kv.page_size + slot; step = a.kv.page_size; }
             } else {
@@ -403,18 +406,26 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
             }
             zb = warp_best(zb);
             if (sampling) gb = warp_best(gb);
-            float s = 0.f;
+            // sum of exp((z - max) / T), and for draft rows the same weights
+            // times z (the mean logit of the row's distribution, for its
+            // entropy)
+            float s = 0.f, ez = 0.f;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                if (nt * kTileN + lane * 4 + j < a.N) s += expf((zv[j] - zb.v) * it);
+                if (nt * kTileN + lane * 4 + j < a.N) {
+                    const float ex = expf((zv[j] - zb.v) * it);
+                    s += ex;
+                    ez = fmaf(ex, zv[j], ez);
+                }
             s = warp_sum(s);
+            if (a.lm_mode == 1) ez = warp_sum(ez);
             // the id's logit lives in exactly one lane (or none)
             const unsigned has = __ballot_sync(0xffffffffu, !isnan(zid));
             if (has) zid = __shfl_sync(0xffffffffu, zid, __ffs(has) - 1);
             if (lane == 0) {
                 LmPart pr;
                 pr.zmax = zb.v; pr.zsum = s; pr.zarg = zb.i;
-                pr.gbest = gb.v; pr.garg = gb.i; pr.gz = gb.z; pr.zid = zid; pr.pad = 0;
+                pr.gbest = gb.v; pr.garg = gb.i; pr.gz = gb.z; pr.zid = zid; pr.zez = ez;
                 a.lm[(size_t)row * n_nt + nt] = pr;
             }
         }

@@ -35,7 +35,7 @@ struct LmPart {
     int garg;     // its index
     float gz;     // logit at garg
     float zid;    // logit at the row's given id, NaN if the id is not in the tile
-    int pad;
+    float zez;    // draft rows: sum over the tile of exp((z - zmax) / T) * z (the entropy's mean logit)
 };
 
 // Per-(row pair, vocab tile) record of the fused forward-KL epilogue: rows
@@ -93,6 +93,10 @@ struct GemmArgs {
     const int32_t *pos0;     // [batch] position of block row 0
     const int32_t *bt_rows;  // [batch] row of block_table for each batch entry
     int K;                   // rows per sequence in this launch
+    // tree verify: row (b, k) is rotated for position pos0[b] + rope_pos[b*K + k]
+    // (its depth in the tree) while its K/V still go to slot pos0[b] + k; null:
+    // position = slot
+    const int32_t *rope_pos;
     double rope_theta;
     const double *rope_invf; // [head_dim / 2] theta^(-2i / head_dim), computed once on the host
     // EPI_LMHEAD / EPI_RESAMPLE
@@ -137,6 +141,10 @@ struct AttnArgs {
     float2 *xml;
     int *xcnt;
     int xrows, xz;
+    // mode 0 tree verify (K <= 128): bit j of tree_mask[(b*K + k)*4 + j/32]
+    // set when block row j is row k's ancestor or row k itself; row k then
+    // sees cache keys [0, t) and exactly those block keys.  Null: causal.
+    const uint32_t *tree_mask;
     unsigned *err;
 };
 
@@ -207,12 +215,15 @@ struct Ctx {
     double *rope_invf;       // [head_dim / 2] rotary inverse frequencies
     LmPart *lm_part;         // [max(R, 2*max_batch)][n_vtiles]
     int32_t *tok;            // [Rw] block tokens
+    int32_t *tree_tok, *tree_depth;   // [R] tree verify: row tokens and depths
+    uint32_t *tree_mask;     // [R][4] tree verify: ancestor bit masks
     int32_t *pos0;           // [max_batch]
     int32_t *bt_rows;        // [max_batch] identity rows 0..max_batch-1
     int32_t *bt_zero;        // [max_batch] zeros (every entry reads block-table row 0)
     int32_t *prefill_row;    // [1]
     int32_t *draft;          // [R]
     float *logq, *lse_q;     // [R]
+    float *ent;              // [R] entropy of each draft row's distribution
     int32_t *g;              // [R]
     float *logp, *lse_p;     // [R]
     int32_t *rej_row;        // [max_batch]
@@ -280,7 +291,8 @@ cudaError_t launch_lm_finalize(const Ctx &c, int mode, int B, int K, float tempe
 cudaError_t launch_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int K, float temperature, uint64_t seed,
                           int64_t *step, const int32_t *force_n, int32_t *n_out, int32_t *tokens_out,
                           int32_t *anchor_io, int32_t *append_out, int append_stride, int append_max,
-                          cudaStream_t s);
+                          cudaStream_t s, const int32_t *kt = nullptr);
+cudaError_t launch_adaptive_len(const Ctx &c, int B, int K, float h_max, int32_t *kt, float *ent_out, cudaStream_t s);
 cudaError_t launch_ar_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int64_t *step,
                              int32_t *token_out, int32_t *anchor_io, int32_t *append_out, int append_stride,
                              int append_max, cudaStream_t s);
@@ -310,6 +322,8 @@ struct TreeCommitArgs {
     unsigned *err;
 };
 
+cudaError_t launch_tree_prep(const Ctx &c, const int32_t *anchor, const int32_t *parent, const int32_t *token, int B,
+                             int R, cudaStream_t s);
 cudaError_t launch_tree_topw(const Ctx &c, const float *logits, int rows, int W, int32_t *ids, float *vals,
                              float *lse, cudaStream_t s);
 cudaError_t launch_tree_build(const Ctx &c, const TreeBuildArgs &a, int B, cudaStream_t s);

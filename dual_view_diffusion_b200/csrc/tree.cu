@@ -435,6 +435,64 @@ __global__ void __launch_bounds__(128) tree_finish_kernel(TreeCommitArgs a)
     a.seq_lens[b] += m + 1;
 }
 
+// Inputs of the tree-masked verify forward, per sequence b and tree row r
+// (grid B, kTreeMaxRows threads): the row's token (the anchor for the
+// root), its depth (the rotary position is t + depth) and its ancestor bit
+// mask (bit j set for every row j on its root path, itself included).  A
+// row r > 0 with parent -1 is unused (a tree smaller than the block): it
+// gets the anchor, depth 0 and only its own bit.  A parent outside [0, r)
+// raises ORTHRUS_DEVERR_TOKEN and leaves the row unused, as does a token
+// outside [0, vocab).
+__global__ void __launch_bounds__(kTreeMaxRows) tree_prep_kernel(const int32_t *anchor, const int32_t *parent,
+                                                                 const int32_t *token, int R, int vocab,
+                                                                 int32_t *tok, int32_t *depth, uint32_t *mask,
+                                                                 unsigned *err)
+{
+    __shared__ int32_t s_par[kTreeMaxRows];
+    pdl_trigger();
+    pdl_wait();
+    const int b = blockIdx.x, r = threadIdx.x;
+    if (r < R) s_par[r] = r == 0 ? -1 : parent[(size_t)b * R + r];
+    __syncthreads();
+    if (r >= R) return;
+    int tk = anchor[b], dep = 0;
+    uint32_t m[4] = {0u, 0u, 0u, 0u};
+    m[r >> 5] |= 1u << (r & 31);
+    if (r > 0 && s_par[r] != -1) {
+        const int t0 = token[(size_t)b * R + r];
+        bool ok = t0 >= 0 && t0 < vocab;
+        int cur = r;
+        while (ok && cur > 0) {   // at most r steps: parents strictly decrease
+            const int p = s_par[cur];
+            if (p < 0 || p >= cur) { ok = false; break; }
+            m[p >> 5] |= 1u << (p & 31);
+            ++dep;
+            cur = p;
+        }
+        if (ok) {
+            tk = t0;
+        } else {
+            raise_err(err, ORTHRUS_DEVERR_TOKEN);
+            dep = 0;
+            m[0] = m[1] = m[2] = m[3] = 0u;
+            m[r >> 5] = 1u << (r & 31);
+        }
+    }
+    const size_t row = (size_t)b * R + r;
+    tok[row] = tk;
+    depth[row] = dep;
+    *(uint4 *)(mask + row * 4) = make_uint4(m[0], m[1], m[2], m[3]);
+}
+
+cudaError_t launch_tree_prep(const Ctx &c, const int32_t *anchor, const int32_t *parent, const int32_t *token, int B,
+                             int R, cudaStream_t s)
+{
+    if (R < 1 || R > kTreeMaxRows) return cudaErrorInvalidValue;
+    c.launches += 1;
+    return launch_k(tree_prep_kernel, B, kTreeMaxRows, 0, s, anchor, parent, token, R, c.cfg.vocab, c.tree_tok,
+                    c.tree_depth, c.tree_mask, c.err);
+}
+
 cudaError_t launch_tree_topw(const Ctx &c, const float *logits, int rows, int W, int32_t *ids, float *vals,
                              float *lse, cudaStream_t s)
 {

@@ -21,9 +21,11 @@
  * orthrus_generate drives the whole loop.  Beyond the cycle:
  * orthrus_draft_block_iterative (multi-pass denoising draft, §5.4.2),
  * orthrus_block_mask_attention and orthrus_kl_lm_head (the training-side
- * dual-pass block mask and forward KL, §3.1-3.3), and orthrus_tree_topw /
- * orthrus_tree_build / orthrus_tree_commit (tree verification's draft tree
- * and commit, §7.5, §9.6; its tree-masked verify forward is not here yet).
+ * dual-pass block mask and forward KL, §3.1-3.3), orthrus_tree_topw /
+ * orthrus_tree_build / orthrus_verify_tree / orthrus_tree_commit (tree
+ * verification over the draft's marginals, §7.5, §9.6), and
+ * orthrus_adaptive_len / orthrus_commit_adaptive (a verify length set by the
+ * draft rows' entropies, §7.4, §9.6).
  *
  * Conventions for every entry point:
  *   - Every pointer to tensor data is a DEVICE pointer owned by the caller
@@ -226,6 +228,39 @@ orthrus_status_t orthrus_commit(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, int3
                                 int32_t *n_out, int32_t *tokens_out, int32_t *anchor_io, void *stream);
 
 /*
+ * Adaptive block length (paper notes §7.4: a verify length set by the
+ * draft's own uncertainty, SV's signal, named as complementary to Orthrus;
+ * §9.6: a dynamic K; neither gives a rule).  Reading taken: after a draft
+ * of K rows, sequence b verifies kt[b] = 1 + the number of leading drafted
+ * tokens y_1, y_2, ... whose draft rows have entropy at most h_max (y_k is
+ * drafted by row k-1), so 1 <= kt[b] <= K; h_max = +inf is the fixed-K
+ * cycle and h_max < 0 plain AR.  Greedy decoding only: the entropy is that
+ * of the row's softmax(z) at T = 1, in nats, computed inside the draft's
+ * LM-head epilogue (no logits are written).
+ *   kt       device int32 [batch], written
+ *   entropy  device fp32 [batch][K] (nullable): the rows' entropies
+ * Call after orthrus_draft_block (temperature 0) with the same batch and K;
+ * then orthrus_verify_block (temperature 0, block K) and
+ * orthrus_commit_adaptive.  h_max NaN returns ORTHRUS_ERR_INVALID_ARG.
+ */
+orthrus_status_t orthrus_adaptive_len(orthrus_ctx_t *ctx, int32_t batch, int32_t K, float h_max, int32_t *kt,
+                                      float *entropy, void *stream);
+
+/*
+ * Greedy consensus and commit over the first kt[b] rows of the verified
+ * block (kt as orthrus_adaptive_len writes it, clamped to [1, K]): accept
+ * drafted tokens while they equal the AR argmax within those rows, at the
+ * first mismatch emit the AR argmax, else emit all kt[b]; n_out, tokens_out,
+ * anchor_io, seq_lens and *step as orthrus_commit at temperature 0.  The
+ * verify rows kt[b] .. K-1 do not change rows below them (causal mask); their
+ * K/V lie beyond the committed length and are overwritten later, so the
+ * result equals a verify of kt[b] rows.
+ */
+orthrus_status_t orthrus_commit_adaptive(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, int32_t batch, int32_t K,
+                                         const int32_t *kt, int64_t *step, int32_t *n_out, int32_t *tokens_out,
+                                         int32_t *anchor_io, void *stream);
+
+/*
  * One plain AR decoding step with the same kernels: the AR view on
  * [anchor[b]] at position seq_lens[b], then emit the argmax (T = 0) or a
  * Gumbel-max sample keyed by (seed, *step) (T > 0).  Writes token_out
@@ -368,9 +403,10 @@ orthrus_status_t orthrus_kl_lm_head(orthrus_ctx_t *ctx, const void *h_ar, const 
  * §9.6: the same proposed for Orthrus).  Greedy only.  A tree of R rows
  * keeps row 0 as the root (the anchor) and every other row r as a node
  * with parent[r] in [0, r) and its draft token; node r sits at position
- * t + depth(r).  The tree-masked verify forward that fills cache slots
- * t .. t+R-1 and the AR argmax g of every row is not part of this library
- * yet.
+ * t + depth(r).  A tree cycle is: the draft (orthrus_draft_block), the top-W
+ * candidates of its rows (orthrus_tree_topw), the tree
+ * (orthrus_tree_build), its tree-masked AR forward (orthrus_verify_tree)
+ * and the walk plus commit (orthrus_tree_commit).
  *
  * orthrus_tree_topw: for each of `rows` rows of fp32 logits (device,
  * [rows][vocab]) the `width` largest logits, best first (ties: lowest id),
@@ -399,6 +435,26 @@ orthrus_status_t orthrus_tree_build(orthrus_ctx_t *ctx, const int32_t *ids, cons
                                     int32_t batch, int32_t depth, int32_t width, int32_t nodes, int32_t *parent,
                                     int32_t *token, int32_t *node_depth, double *score, int32_t *n_rows,
                                     void *stream);
+
+/*
+ * orthrus_verify_tree: the tree-masked AR verification of one tree per
+ * sequence (paper notes §7.5: all the tree's nodes in one forward with tree
+ * attention).  Row 0 is the anchor, row r > 0 the node with parent[r] in
+ * [0, r) and token[r], as orthrus_tree_build writes them (rows with parent
+ * -1 past the tree's end are unused).  Row r is rotated for position
+ * t + depth(r) (t = seq_lens[b]) but its AR K/V are written to cache slot
+ * t + r; it attends to cache rows [0, t) and to the block rows on its own
+ * root path (its ancestors and itself), so every node's logits equal those
+ * of a plain causal forward of its root path.  Writes g [batch][rows]
+ * int32: each row's AR argmax (the consensus input of orthrus_tree_commit).
+ * The pages for t + rows positions must exist.  Requires 1 <= rows <=
+ * min(max_block, 128); a parent outside [0, r) or a token outside
+ * [0, vocab) raises ORTHRUS_DEVERR_TOKEN (that row is then treated as
+ * unused).  Greedy only.
+ */
+orthrus_status_t orthrus_verify_tree(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, const int32_t *anchor,
+                                     const int32_t *parent, const int32_t *token, int32_t batch, int32_t rows,
+                                     int32_t *g, void *stream);
 
 /*
  * orthrus_tree_commit: greedy acceptance on a verified tree and the commit
