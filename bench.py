@@ -65,11 +65,15 @@ METRIC = "committed tokens/s (batch 1, Qwen3-8B shape, K=32); dual-view attn HBM
 UNIT = "tokens/s"
 P_PROMPT, K_BLOCK, BATCH = 2048, 32, 1
 ITER_STEPS = 20   # decode steps timed with the two-pass iterative draft
+VARIANT_STEPS = 20   # decode steps timed for each of the other decode loops (sampled, tree, adaptive)
 # tokens committed per cycle that this random-init 8B workload gives (the
 # mean accepted length measured on the GPU path, 1.00-1.03 over runs: the
 # random-init diffusion view almost never agrees with the AR view).  Used
 # only by the reference arm, which cannot run the whole model.
 N_BAR_WORKLOAD = 1.0
+# block rows of the oracle's bounded sample (both CPU legs: the reference arm
+# and cpu_baseline), scaled to the 32 rows of a step
+ORACLE_ROWS = 8
 SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -84,6 +88,11 @@ def parse():
     ap.add_argument("--temperature", type=float, default=0.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", choices=["reduced", "full", "none"], default="reduced",
+                    help="long-context step sweep: L at batch 1, K at L = 2K, batch at L = 8K (reduced), every "
+                         "(L, batch, K) cell that fits (full), or none")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the other decode loops (sampled, plain AR, tree, adaptive) and the 1.7B config")
     ap.add_argument("--split-tokens", type=int, default=128,
                     help="KV positions per attention split (a run-wide constant)")
     ap.add_argument("--profile-small", action="store_true",
@@ -99,7 +108,7 @@ def parse():
                          "is marked profile_case and is not a bench result")
     a = ap.parse_args()
     if a.profile_small:
-        a.steps, a.warmup, a.no_cpu_baseline, a.no_e2e = 2, 1, True, True
+        a.steps, a.warmup, a.no_cpu_baseline, a.no_e2e, a.sweep, a.no_variants = 2, 1, True, True, "none", True
     return a
 
 
@@ -499,6 +508,239 @@ def _block_mask_cpu(rec, ae, q, kb, vb, anchors, nb, K, L):
                            "sample": "2 of the 256 blocks, scaled by visible keys"}
 
 
+def _time_steps(fn, n):
+    """Device time (ms) of n calls of fn(i), CUDA events around the run on the
+    current stream."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(n):
+        fn(i)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def decode_variants(eng, anchor, draft, toks, value, ms_step, steps=VARIANT_STEPS):
+    """Other decode loops on the benchmark's engine (the 8B shape, batch 1,
+    K = 32), each warmed up three steps and then timed over `steps` steps
+    with CUDA events:
+      sampled   the Orthrus step at T = 1.0 with rejection sampling (paper
+                notes §4.3): draft samples, acceptance test, residual draw
+      plain_ar  one AR forward per token (the same kernels, K = 1): the
+                baseline whose greedy stream Orthrus reproduces (§4.2)
+      tree      a tree-verified step (§7.5 / §9.6): draft, its rows' logits,
+                top-4 candidates per depth, a best-first tree of 31 nodes,
+                the tree-masked verify forward (32 rows, as the chain's) and
+                the walk plus K/V compaction
+      adaptive  the adaptive block length (§7.4 / §9.6, reading R23): the
+                verify length from the draft rows' entropies, threshold the
+                median entropy of a warm-up draft"""
+    import numpy as np
+    import torch
+    B, K, dev = BATCH, K_BLOCK, anchor.device
+    out = {}
+    # ---- sampled T = 1.0
+    n_s = torch.zeros((steps + 3, B), dtype=torch.int32, device=dev)
+
+    def st_sampled(j):
+        eng.draft_block(anchor, K, 1.0, 4321, out=draft)
+        eng.verify_block(anchor, draft, K, 1.0)
+        eng.commit(anchor, K, 1.0, 4321, n_out=n_s[j], tokens_out=toks)
+    for j in range(3):
+        st_sampled(steps + j)
+    ms = _time_steps(st_sampled, steps)
+    tok = int(n_s[:steps].sum())
+    out["sampled"] = {"temperature": 1.0, "steps": steps, "ms_per_step": ms / steps,
+                      "value": tok / (ms * 1e-3), "unit": UNIT, "mean_accepted_per_cycle": tok / (steps * B),
+                      "how": "draft samples (Gumbel-max), acceptance u < p/q, residual draw from max(0, p - q) at "
+                             "the first rejection (one extra LM-head pass over two rows); CUDA events"}
+    # ---- plain AR
+    ar_tok = torch.empty(B, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        eng.ar_step(anchor, token_out=ar_tok)
+    n_ar = 4 * steps
+    ms = _time_steps(lambda i: eng.ar_step(anchor, token_out=ar_tok), n_ar)
+    ar_val = n_ar * B / (ms * 1e-3)
+    out["plain_ar"] = {"steps": n_ar, "ms_per_token": ms / n_ar, "value": ar_val, "unit": UNIT,
+                       "orthrus_over_ar": value / ar_val,
+                       "modelled_orthrus_over_ar_at_pages_acceptance": 10.8 / (ms_step * 1e-3) / ar_val,
+                       "how": "orthrus_ar_step (AR view on one row, argmax, commit 1) back to back; the ratio is "
+                              "the greedy decode step's tokens/s (measured acceptance) over this; the modelled "
+                              "ratio uses the pages' 10.8 tokens per cycle"}
+    # ---- tree-verified step (greedy)
+    W, nodes, D = 4, K - 1, K - 1
+    zbuf = torch.empty((B, K, eng.shape.vocab), dtype=torch.float32, device=dev)
+    n_t = torch.zeros((steps + 3, B), dtype=torch.int32, device=dev)
+
+    def st_tree(j):
+        eng.draft_block(anchor, K, out=draft)
+        eng.debug_logits(1, B, K, out=zbuf)
+        ids, vals, lse = eng.tree_topw(zbuf[:, :D], W)
+        par, tk, _, _, nr = eng.tree_build(ids.view(B, D, W), vals.view(B, D, W), lse.view(B, D), nodes)
+        g = eng.verify_tree(anchor, par, tk)
+        n, _ = eng.tree_commit(par, tk, nr, g, anchor)
+        n_t[j].copy_(n)
+    for j in range(3):
+        st_tree(steps + j)
+    ms = _time_steps(st_tree, steps)
+    tok = int(n_t[:steps].sum())
+    out["tree"] = {"width": W, "nodes": nodes, "steps": steps, "ms_per_step": ms / steps,
+                   "value": tok / (ms * 1e-3), "unit": UNIT, "mean_accepted_per_cycle": tok / (steps * B),
+                   "how": "draft, the draft rows' fp32 logits (one extra LM-head pass written to memory), top-W, "
+                          "best-first build, tree-masked verify forward, walk + K/V compaction; greedy"}
+    # ---- adaptive block length (greedy)
+    kt = torch.empty(B, dtype=torch.int32, device=dev)
+    eng.draft_block(anchor, K, out=draft)
+    _, ent = eng.adaptive_len(B, K, float("inf"), kt=kt, entropy=True)
+    h_max = float(ent.float().median())
+    n_a = torch.zeros((steps + 3, B), dtype=torch.int32, device=dev)
+    k_a = torch.zeros((steps + 3, B), dtype=torch.int32, device=dev)
+
+    def st_adaptive(j):
+        eng.draft_block(anchor, K, out=draft)
+        eng.adaptive_len(B, K, h_max, kt=kt)
+        eng.verify_block(anchor, draft, K)
+        eng.commit_adaptive(anchor, K, kt, n_out=n_a[j], tokens_out=toks)
+        k_a[j].copy_(kt)
+    for j in range(3):
+        st_adaptive(steps + j)
+    ms = _time_steps(st_adaptive, steps)
+    tok = int(n_a[:steps].sum())
+    out["adaptive"] = {"h_max": h_max, "steps": steps, "ms_per_step": ms / steps, "value": tok / (ms * 1e-3),
+                       "unit": UNIT, "mean_accepted_per_cycle": tok / (steps * B),
+                       "mean_verify_rows": float(k_a[:steps].float().mean()),
+                       "how": "draft, per-sequence verify length from the draft rows' entropies (threshold: the "
+                              "median entropy of a warm-up draft), verify of the block, greedy consensus over the "
+                              "first kt rows; the verify forward still runs 32 rows (its cost is weight streaming)"}
+    return out
+
+
+def config_1p7b(split_tokens, steps=VARIANT_STEPS):
+    """The Qwen3-1.7B-shaped random-init model (28 layers, hidden 2048, 16/8
+    heads, FFN 6144, tied head), prompt 512, K = 32, batch 1, greedy: the
+    decode step and plain AR, each timed over `steps` (AR: 4x) steps after
+    three warm-up steps."""
+    import torch
+    import synth
+    import dual_view_diffusion_b200 as pkg
+    s = synth.QWEN3_1_7B
+    P, K, B = 512, K_BLOCK, 1
+    w = synth.make_weights_torch(s, 0)
+    eng = pkg.Engine(s, w, max_batch=B, max_block=K, max_seq=P + (2 * steps + 12) * K + 4 * steps + 64,
+                     split_tokens=split_tokens)
+    prompt = torch.from_numpy(synth.make_prompt(s, P, 0))[None].cuda()
+    anchor = eng.prefill(prompt)
+    eng.step.zero_()
+    draft = torch.empty((B, K), dtype=torch.int32, device="cuda")
+    toks = torch.empty((B, K), dtype=torch.int32, device="cuda")
+    n_h = torch.zeros((steps + 3, B), dtype=torch.int32, device="cuda")
+
+    def st(j):
+        eng.draft_block(anchor, K, out=draft)
+        eng.verify_block(anchor, draft, K)
+        eng.commit(anchor, K, n_out=n_h[j], tokens_out=toks)
+    for j in range(3):
+        st(steps + j)
+    ms = _time_steps(st, steps)
+    tok = int(n_h[:steps].sum())
+    ar_tok = torch.empty(B, dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        eng.ar_step(anchor, token_out=ar_tok)
+    ms_ar = _time_steps(lambda i: eng.ar_step(anchor, token_out=ar_tok), 4 * steps)
+    assert eng.check_error()[0] == 0
+    val, ar_val = tok / (ms * 1e-3), 4 * steps / (ms_ar * 1e-3)
+    del eng, w
+    torch.cuda.empty_cache()
+    return {"workload": "qwen3-1.7b-shape decode step, batch 1, K=32, prompt 512, greedy", "steps": steps,
+            "ms_per_step": ms / steps, "value": val, "unit": UNIT, "mean_accepted_per_cycle": tok / steps,
+            "plain_ar": {"ms_per_token": ms_ar / (4 * steps), "value": ar_val}, "orthrus_over_ar": val / ar_val}
+
+
+SWEEP_L = (2048, 8192, 32768, 131072)
+SWEEP_B = (1, 4, 16)
+SWEEP_K = (4, 8, 16, 32)
+
+
+def sweep_cells(full):
+    """The long-context sweep's (L, batch, K) cells: all of them when full,
+    else L at batch 1 and K = 32, K at L = 2K and batch 1, batch at L = 8K
+    and K = 32."""
+    if full:
+        return [(L, B, K) for L in SWEEP_L for B in SWEEP_B for K in SWEEP_K]
+    cells = [(L, 1, 32) for L in SWEEP_L] + [(2048, 1, K) for K in SWEEP_K[:-1]] + [(8192, B, 32) for B in SWEEP_B[1:]]
+    return cells
+
+
+def step_sweep(w, s, split_tokens, cells, steps=4, warm=2, hbm=None):
+    """One 8B-shape decode step (draft + verify + commit) per (L, batch, K)
+    cell: every sequence's cache filled with N(0, 1) bf16 K/V (seed 3) up to
+    prefix L (no prefill), anchors uniform ids, the accepted length of each
+    sequence and step drawn uniformly from 1..K (seed 3, orthrus_commit's
+    force_n); `warm` steps, then `steps` timed with CUDA events.  Bytes per
+    step: both views' weights (the decode engine's) + every sequence's K/V
+    prefix read twice (draft and verify).  A cell whose cache would not fit
+    next to the weights with 16 GB to spare is skipped and listed."""
+    import numpy as np
+    import torch
+    import dual_view_diffusion_b200 as pkg
+    free, _ = torch.cuda.mem_get_info()
+    kv_tok = s.n_layers * s.n_kv_heads * s.head_dim * 2 * 2
+    wbytes = sum(x * 2 for x in gemm_bytes_weights(s)) * s.n_layers + 2 * s.vocab * s.hidden * 2
+    out, skipped = [], []
+    for L, B, K in cells:
+        max_seq = L + (warm + steps + 1) * K + 64
+        need = B * ((max_seq + 63) // 64 * 64) * kv_tok
+        if need > free - 16e9:
+            skipped.append({"L": L, "batch": B, "K": K, "kv_bytes": need,
+                            "why": f"the paged cache ({need / 2**30:.0f} GiB) does not fit beside the weights"})
+            continue
+        eng = pkg.Engine(s, w, max_batch=B, max_block=K, max_seq=max_seq, split_tokens=split_tokens, page_size=64)
+        g = torch.Generator(device="cuda").manual_seed(3)
+        for pg in (eng.k_pages, eng.v_pages):
+            for i in range(pg.shape[0]):
+                pg[i].normal_(generator=g)
+        rng = np.random.Generator(np.random.Philox(key=3))
+        anchor = torch.from_numpy(rng.integers(0, s.vocab - 1, B).astype(np.int32)).cuda()
+        fn = torch.from_numpy(rng.integers(1, K + 1, (warm + steps, B)).astype(np.int32)).cuda()
+        eng.seq_lens[:B] = L
+        eng.step.zero_()
+        draft = torch.empty((B, K), dtype=torch.int32, device="cuda")
+        toks = torch.empty((B, K), dtype=torch.int32, device="cuda")
+        nbuf = torch.empty(B, dtype=torch.int32, device="cuda")
+
+        def st(j):
+            eng.draft_block(anchor, K, out=draft)
+            eng.verify_block(anchor, draft, K)
+            eng.commit(anchor, K, force_n=fn[j], n_out=nbuf, tokens_out=toks)
+        for j in range(warm):
+            st(j)
+        ms = _time_steps(lambda i: st(warm + i), steps)
+        assert eng.check_error()[0] == 0
+        tok = int(fn[warm:].sum())
+        mean_t = L + float(fn[:warm].sum()) / B + float(fn[warm:].sum()) / (2 * B)
+        byts = wbytes + 2 * B * (mean_t + K) * kv_tok
+        rec = {"L": L, "batch": B, "K": K, "ms_per_step": ms / steps, "tokens_per_s": tok / (ms * 1e-3),
+               "workspace_bytes": eng.ws_bytes, "achieved_gbs": byts / (ms / steps * 1e-3) / 1e9}
+        if hbm:
+            rec["frac"] = rec["achieved_gbs"] / hbm
+        out.append(rec)
+        del eng
+        torch.cuda.empty_cache()
+    return {"how": "one decode step per cell, cache filled synthetically (N(0,1) bf16, seed 3), accepted length "
+                   "forced uniform over 1..K (seed 3), CUDA events over the timed steps; bytes = weights of both "
+                   "views + K/V prefix read by both views", "cells": out, "skipped": skipped}
+
+
+def gemm_bytes_weights(s):
+    """Parameters one decode step reads per layer for each projection (QKV,
+    O, gate/up, down), both views together: each view reads its own QKV and
+    the shared O and FFN once."""
+    d, hq, hk, F = s.hidden, s.n_q_heads * s.head_dim, s.n_kv_heads * s.head_dim, s.ffn
+    return [2 * (hq + 2 * hk) * d, 2 * d * hq, 2 * 2 * F * d, 2 * d * F]
+
+
 # ----------------------------------------------------------------- oracle sample
 class OracleSample:
     """The CPU oracle, as it stands, on a bounded sample of one decode step
@@ -569,18 +811,22 @@ def run_reference(args, rank, world):
     """The oracle as the reference arm (rank 0 only)."""
     if rank != 0:
         return
-    samples = []
-    n_rows = 4 if args.steps + args.warmup > 24 else 32
+    samples, walls = [], []
     sample = OracleSample()
     for i in range(args.warmup + args.steps):
-        est = sample.step_seconds(n_rows)
+        t0 = time.perf_counter()
+        est = sample.step_seconds(ORACLE_ROWS)
         if i >= args.warmup:
             samples.append(est)
+            walls.append(time.perf_counter() - t0)
     sec = statistics.mean(samples)
-    desc, threads = sample.describe(n_rows), sample.threads()
+    desc, threads = sample.describe(ORACLE_ROWS), sample.threads()
     value = N_BAR_WORKLOAD / sec
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(walls) * 1e3,
+            "ms_per_step_is": "the measured wall time of one step's bounded oracle sample; value is extrapolated "
+                              "from it to a whole decode step (extrapolated_ms_per_full_step)",
+            "extrapolated_ms_per_full_step": sec * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "qwen3-8b-shape decode step, batch 1, K=32, prompt 2048, greedy",
                        "global_batch": BATCH, "seq_len": P_PROMPT, "parallelism": "host cores"},
@@ -606,7 +852,10 @@ def run_ours(args, rank, world, local_rank):
     W, K, T = args.warmup, args.steps, args.temperature
     n_e2e = 0 if args.no_e2e else K
     n_iter = 0 if args.profile_small else 3 + ITER_STEPS   # the iterative-draft measurement
-    max_seq = P_PROMPT + (W + K + n_e2e + n_iter + 2) * K_BLOCK + K_BLOCK
+    # the other decode loops: sampled, tree and adaptive steps (<= K tokens
+    # each), plain AR (1 token each)
+    n_var = 0 if args.no_variants else 3 * (VARIANT_STEPS + 4) * K_BLOCK + 4 * VARIANT_STEPS + 8
+    max_seq = P_PROMPT + (W + K + n_e2e + n_iter + 2) * K_BLOCK + K_BLOCK + n_var
     w = synth.make_weights_torch(s, 0, device=dev)
     eng = pkg.Engine(s, w, max_batch=BATCH, max_block=K_BLOCK, max_seq=max_seq, split_tokens=args.split_tokens,
                      page_size=64, device=dev)
@@ -725,6 +974,14 @@ def run_ours(args, rank, world, local_rank):
                    "how": "the same decode step with a two-pass iterative-denoising draft (the diffusion view "
                           "re-run on its own drafts), CUDA events around the steps"}
 
+    # ---------------------------------------------------------------- other decode loops
+    variants = None
+    if not args.no_variants:
+        variants = decode_variants(eng, anchor, draft, toks, tokens / (ms * 1e-3), ms / K)
+        st, bits = eng.check_error()
+        if st != 0:
+            raise RuntimeError(f"device error bits {bits:#x}")
+
     # ---------------------------------------------------------------- reduce
     tot_tokens, max_ms, e2e_sum = reduce_replicas(tokens, ms, e2e["value"] if e2e else 0.0, world, dev)
     if e2e:
@@ -758,6 +1015,10 @@ def run_ours(args, rank, world, local_rank):
                      "layer_gemms": {"kernel": "the four projection GEMMs (QKV, O, gate/up, down) of one layer",
                                      "achieved": g_ach, "frac": g_ach / hbm, "traffic": traffic,
                                      "algorithmic_bytes_per_layer": sum(gb),
+                                     "note": "each GEMM is bracketed by its own CUDA events; under programmatic "
+                                             "dependent launch a kernel starts while its predecessor drains, so "
+                                             "the brackets overlap and are not disjoint times (their sum exceeds "
+                                             "the step)",
                                      "ms_per_layer": float(g_ms.sum(axis=1).mean()),
                                      "per_gemm": {n: {"us": float(g_ms[:, i].mean() * 1e3),
                                                       "achieved_gbs": gb[i] / float(g_ms[:, i].mean() * 1e-3) / 1e9}
@@ -772,6 +1033,8 @@ def run_ours(args, rank, world, local_rank):
         line["e2e"] = e2e
     if it_line:
         line["iterative_draft"] = it_line
+    if variants:
+        line.update(variants)
     if not args.profile_small:
         lc = attn_long_context(hbm, args.split_tokens)
         line["attn_long_context"] = lc
@@ -792,14 +1055,20 @@ def run_ours(args, rank, world, local_rank):
                 "in_step": in_step}
         line["train_kernels"] = train_kernels(hbm, tflops, eng)
         line["tree_kernels"] = tree_kernels(hbm)
+    if args.sweep != "none" and world == 1:
+        line["step_sweep"] = step_sweep(w, s, args.split_tokens, sweep_cells(args.sweep == "full"), hbm=hbm)
+    if not args.no_variants and world == 1:
+        line["config_1p7b"] = config_1p7b(args.split_tokens)
     if args.profile_small:
         line = {"profile_case": True, "config": "2 layers of the Qwen3-8B shape, vocab 32000", "value": value,
                 "roofline": line["roofline"], "attn": line["attn"]}
     if not args.no_cpu_baseline and world == 1:
         sample = OracleSample()
-        est = sample.step_seconds(32)
+        ests = [sample.step_seconds(ORACLE_ROWS) for _ in range(3)]
+        est = statistics.mean(ests[1:])     # the first sample is the warm-up, as in the reference arm
         line["cpu_baseline"] = {"value": nbar / est, "unit": UNIT, "cores": sample.threads(), "kind": "oracle",
-                                "sample": sample.describe(32) + f"; tokens per step = {nbar:.3f} (this run's mean)",
+                                "sample": sample.describe(ORACLE_ROWS) + f"; mean of 2 samples after 1 warm-up; "
+                                          f"tokens per step = {nbar:.3f} (this run's mean)",
                                 "seconds_per_step": est}
     print(json.dumps(line), flush=True)
 

@@ -424,8 +424,12 @@ class Engine:
             _ptr(anchor), _stream()))
         return n, emit
 
-    def debug_logits(self, which, B, K):
-        out = self.torch.empty((B, K, self.shape.vocab), dtype=self.torch.float32, device=self.device)
+    def debug_logits(self, which, B, K, out=None):
+        """fp32 logits [B, K, vocab] of the last verify (which = 0) or draft
+        (which = 1), from the final hidden rows they kept."""
+        if out is None:
+            out = self.torch.empty((B, K, self.shape.vocab), dtype=self.torch.float32, device=self.device)
+        _need(out, self.torch.float32, "out")
         _check("orthrus_debug_logits", lib().orthrus_debug_logits(self.ctx, which, B, K, _ptr(out), _stream()))
         return out
 
