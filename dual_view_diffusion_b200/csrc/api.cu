@@ -59,10 +59,24 @@ static void gemm_scratch(const orthrus_config_t &c, int rows_body, int rows_lm, 
     *floats = 0;
     *tickets = 1;
     for (const Shape &s : shapes) {
-        const int n_mt = (s.rows + kTileM - 1) / kTileM;
         const int S = (use_tensor_cores(c) && s.Kd % kTileK == 0) ? sk_max_segments(s.n_tiles, s.Kd / kTileK) : 1;
-        if (S > 1) *floats = std::max(*floats, (size_t)n_mt * s.n_tiles * S * kTileM * kTileN);
-        *tickets = std::max(*tickets, n_mt * s.n_tiles * S);
+        // the largest token tiles x tile rows any M up to s.rows uses
+        size_t rows_mt = 0, n_mt_max = 0;
+        for (int M = 1; M <= s.rows; M += (M < 256 ? 1 : 32)) {
+            int n_mt, tm;
+            gemm_token_tile(M, &n_mt, &tm);
+            rows_mt = std::max(rows_mt, (size_t)n_mt * tm);
+            n_mt_max = std::max(n_mt_max, (size_t)n_mt);
+        }
+        {
+            int n_mt, tm;
+            gemm_token_tile(s.rows, &n_mt, &tm);
+            rows_mt = std::max(rows_mt, (size_t)n_mt * tm);
+            n_mt_max = std::max(n_mt_max, (size_t)n_mt);
+        }
+        const size_t n_mt32 = (s.rows + kTileM - 1) / kTileM;
+        if (S > 1) *floats = std::max(*floats, rows_mt * s.n_tiles * S * kTileN);
+        *tickets = std::max(*tickets, (int)(std::max(n_mt32, n_mt_max) * s.n_tiles * S));
     }
 }
 
@@ -174,15 +188,19 @@ static void build_tmaps(Ctx *c)
         CUtensorMap m;
         if (make_tmap(&m, p, rows, cols, box)) c->tmaps[TmapKey{p, box}] = m;
     };
+    // activation buffers: one map per token-tile height the GEMM may use
+    auto add_x = [&](const void *p, int rows, int cols) {
+        for (uint32_t box = kTileM; box <= (uint32_t)kTcTokenTileMax; box += kTileM) add(p, rows, cols, box);
+    };
     for (const orthrus_layer_weights_t &L : c->layers) {
         add(L.wq, hq, d, kTileN); add(L.wk, hk, d, kTileN); add(L.wv, hk, d, kTileN);
         add(L.wq_diff, hq, d, kTileN); add(L.wk_diff, hk, d, kTileN); add(L.wv_diff, hk, d, kTileN);
         add(L.wo, d, hq, kTileN); add(L.w_gate, F, d, 64); add(L.w_up, F, d, 64); add(L.w_down, d, F, kTileN);
     }
     add(c->lm_head, f.vocab, d, kTileN);
-    add(c->a, c->Rw, d, kTileM); add(c->attn_o, c->Rw, hq, kTileM); add(c->act, c->Rw, F, kTileM);
-    add(c->fin_draft, c->R, d, kTileM); add(c->fin_verify, c->R, d, kTileM);
-    add(c->res_x, 2 * f.max_batch, d, kTileM);
+    add_x(c->a, c->Rw, d); add_x(c->attn_o, c->Rw, hq); add_x(c->act, c->Rw, F);
+    add_x(c->fin_draft, c->R, d); add_x(c->fin_verify, c->R, d);
+    add_x(c->res_x, 2 * f.max_batch, d);
 }
 
 static KvView kv_view(const orthrus_kv_t &kv)

@@ -137,20 +137,24 @@ cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s)
     a.ticket = c.gemm_ticket;
     a.err = c.err;
     if (tc) {   // stream-K split: partial and flag slots per (token tile, n tile, segment)
+        int n_mt_tc, tm;
+        gemm_token_tile(a.M, &n_mt_tc, &tm);
         GemmArgs t = a;
         t.splits = t.defer > 0 ? t.defer : sk_max_segments(n_nt, a.Kd / kTileK);
         // QKV: each head tile cut in 2 k segments reduced inside a 2-CTA
         // cluster when one cluster per tile fits one wave of SMs (a function
         // of the matrix shape, never of the token count; 3-CTA clusters
-        // measured slower on B200)
+        // measured slower on B200).  Token tiles of TM rows (all the rows of
+        // a step up to 256) ride on each weight tile; the summation order of
+        // a row never depends on TM.
         t.pair = 0;
         if (a.epi == EPI_QKV && t.defer == 0)
             for (int S = 2; S >= 2 && !t.pair; --S)
                 if (n_nt * S <= kNumSMs && a.Kd / kTileK >= S) t.pair = S;   // the matrix shape only
-        const size_t slots = (size_t)n_mt * n_nt * t.splits;
-        if (t.splits > 1 && (slots * kTileM * kTileN > c.gemm_part_floats || slots > (size_t)c.gemm_tickets))
+        const size_t slots = (size_t)n_mt_tc * n_nt * t.splits;
+        if (t.splits > 1 && (slots * tm * kTileN > c.gemm_part_floats || slots > (size_t)c.gemm_tickets))
             return cudaErrorInvalidValue;
-        const cudaError_t e = launch_gemm_tc(c, t, n_mt, n_nt, s);
+        const cudaError_t e = launch_gemm_tc(c, t, n_mt_tc, tm, n_nt, s);
         if (e != cudaErrorNotSupported) return e;
     }
     if (a.defer > 0) return cudaErrorInvalidValue;   // only the tensor-core kernel defers

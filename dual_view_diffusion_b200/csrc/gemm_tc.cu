@@ -1,8 +1,11 @@
 // Projection GEMMs on the 5th-generation tensor cores (tcgen05) for bf16.
 //
-// Work split ("stream-K"): the (n tile, 64-wide k chunk) pairs of one 32-row
-// token tile, taken n-tile-major, are cut into G = min(148, pairs) equal
-// contiguous pieces, one per CTA; token tiles repeat the same cut.  A piece
+// Work split ("stream-K"): the (n tile, 64-wide k chunk) pairs of one token
+// tile, taken n-tile-major, are cut into G = min(148, pairs) equal contiguous
+// pieces, one per CTA; token tiles repeat the same cut.  A token tile holds
+// TM rows, a multiple of 32 up to 256 (one MMA's N): every token row of a
+// step of up to 256 rows rides on each weight tile, so the weights stream
+// from HBM once whatever the batch.  A piece
 // covers the end of one n tile, whole n tiles and the start of another, so
 // every SM streams the same number of weight bytes whatever the matrix shape.
 // An n tile cut across pieces is reduced by the piece holding its first
@@ -12,20 +15,22 @@
 // them first, so its partial is usually published long before it is needed.
 //
 //   warp 0      producer: one thread issues TMA tile loads (W: 128 rows x 64,
-//               X: 32 token rows x 64, both 128-byte swizzled) into a ring of
-//               shared-memory stages, signalling an mbarrier per stage;
+//               X: TM token rows x 64, both 128-byte swizzled) into a ring of
+//               shared-memory stages (8 for TM = 32, fewer for wider token
+//               tiles), signalling an mbarrier per stage;
 //   warp 1      MMA issuer: one thread issues tcgen05.mma (M = 128 weight rows,
-//               N = 32 tokens, K = 16 per instruction) from shared memory into a
+//               N = TM tokens, K = 16 per instruction) from shared memory into a
 //               TMEM accumulator; tcgen05.commit releases each stage when the
 //               MMAs reading it are done, and publishes the accumulator at the
 //               end of a tile's chunks;
 //   warps 2..5  epilogue: fetch what the epilogue needs (residual rows, cache
 //               destinations, other pieces' partials) while the chunks stream,
-//               then drain the accumulator with tcgen05.ld (warp w reads TMEM
-//               lanes 32*(w%4) ..), stage it in shared memory and either
-//               publish it as a partial or finish the tile.
+//               then drain the accumulator 32 token rows at a time with
+//               tcgen05.ld (warp w reads TMEM lanes 32*(w%4) ..), stage each
+//               32-row chunk in shared memory and either publish it as a
+//               partial or finish it.
 //
-// Two accumulators (2 x 32 TMEM columns) let the next tile's MMAs run while
+// Two accumulators (2 x TM TMEM columns) let the next tile's MMAs run while
 // one drains.  Every wait (mbarrier or flag) is bounded: on timeout the
 // kernel raises ORTHRUS_DEVERR_TIMEOUT, stops issuing, and still frees its
 // TMEM.
@@ -41,16 +46,17 @@
 
 namespace orthrus {
 
-constexpr int kTcStages = 8;
+constexpr int kTcStages = 8;                             // most ring stages (TM = 32)
 constexpr int kTcThreads = 192;
-constexpr int kTcAccCols = 32;                          // TMEM columns per accumulator (N = 32)
+constexpr int kTcMaxTM = 256;                           // token rows per tile: one MMA's largest N
 constexpr uint32_t kStageWBytes = kTileN * kTileK * 2;  // 16 KiB
-constexpr uint32_t kStageXBytes = kTileM * kTileK * 2;  // 4 KiB
 constexpr long long kSpinCycles = 4000000000LL;        // ~2 s at the B200 SM clock
+constexpr size_t kTcSmemBudget = 227 * 1024;            // dynamic shared memory of one CTA
 
+// The fixed part of the shared memory; the stage ring (kStageWBytes weight
+// tiles, then TM x 128-byte token tiles, stages of each) follows it at a
+// 1024-byte boundary, sized per launch.
 struct TcSmem {
-    alignas(1024) unsigned char w[kTcStages][kStageWBytes];
-    alignas(1024) unsigned char x[kTcStages][kStageXBytes];
     float tile[kTileM][kTilePad];
     EpiPre pre;                       // (cluster mode, rank 0: pre.resid lands rank 1's tile)
     float peer2[kTileM][kTilePad];    // cluster mode, rank 0: rank 2's tile
@@ -60,6 +66,23 @@ struct TcSmem {
     int abort;
     int s_last;
 };
+constexpr size_t kTcRingOffset = (sizeof(TcSmem) + 1023) / 1024 * 1024;
+
+// Ring stages for token tiles of tm rows: as many as fit beside the fixed
+// part, at most kTcStages.
+__host__ __device__ inline int tc_stages(int tm)
+{
+    const size_t per = kStageWBytes + (size_t)tm * kTileK * 2;
+    const size_t n = (kTcSmemBudget - 1024 - kTcRingOffset) / per;
+    return (int)(n < (size_t)kTcStages ? n : (size_t)kTcStages);
+}
+// TMEM columns of the two accumulators (a power of two, at least 32)
+__host__ __device__ inline uint32_t tc_tmem_cols(int tm)
+{
+    uint32_t c = 32;
+    while (c < 2u * (uint32_t)tm) c <<= 1;
+    return c;
+}
 
 // ---------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count)
@@ -134,15 +157,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(const void *p)
 }
 
 // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both
-// K-major, N = 32, M = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTileM >> 3) << 17) |
-                            ((uint32_t)(kTileN >> 4) << 24);
+// K-major, N = tm token rows, M = 128 weight rows.
+__device__ __forceinline__ uint32_t tc_idesc(int tm)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(tm >> 3) << 17) | ((uint32_t)(kTileN >> 4) << 24);
+}
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
 {
     asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
                  " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
-                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
                  : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint64_t *bar)
@@ -190,6 +216,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32])
 struct SkShape {
     long P;
     int G, chunks, n_nt, n_mt;
+    int tm;       // token rows per token tile (a multiple of 32, at most kTcMaxTM)
+    int stages;   // ring stages (tc_stages(tm))
 };
 __host__ __device__ inline long sk_begin(const SkShape &k, int g) { return (long)g * k.P / k.G; }
 // the piece holding pair x
@@ -266,16 +294,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                                                                  SkShape sk)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    TcSmem &sm = *(TcSmem *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    unsigned char *base = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    TcSmem &sm = *(TcSmem *)base;
     if (E == EPI_RESAMPLE) {   // the flag comes from the previous kernel
         pdl_wait();
         if (*a.any_flag == 0) return;
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
+    const int tm = sk.tm, nch = tm / kTileM, stages = sk.stages;
+    const uint32_t xbytes = (uint32_t)tm * kTileK * 2;
+    unsigned char *ring_w = base + kTcRingOffset, *ring_x = ring_w + (size_t)stages * kStageWBytes;
+    const uint32_t tcols = tc_tmem_cols(tm);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kTcStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
+        for (int s = 0; s < stages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
         for (int s = 0; s < 2; ++s) { mbar_init(&sm.tfull[s], 1); mbar_init(&sm.tempty[s], kEpiThreads); }
         mbar_init(&sm.peer_full, 1);
         mbar_init(&sm.peer_empty, 1);
@@ -284,7 +317,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&sm.tmem_base)),
-                     "r"(2 * kTcAccCols));
+                     "r"(tcols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
     }
     tc_fence_before();
@@ -294,17 +327,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     const int g = blockIdx.x;
     // cluster mode (a.pair = 2 or 3 CTAs per cluster): the CTAs of a cluster
     // hold the k segments of the same n tiles; ranks 1.. hand their fp32
-    // tiles to rank 0 through distributed shared memory.  Every CTA's barriers
-    // are initialised before any signals another (start of the cluster
-    // barrier; its wait comes before the first remote operation).
+    // tiles to rank 0 through distributed shared memory, one 32-row chunk at
+    // a time.  Every CTA's barriers are initialised before any signals
+    // another (start of the cluster barrier; its wait comes before the first
+    // remote operation).
     const bool pair = a.pair > 1;
     const uint32_t crank = pair ? tc_cluster_rank() : 0u;
     if (pair) tc_cluster_arrive_relaxed();
 
     if (warp == 0) {
         if (lane == 0) {   // ------------------------------------------- producer
-            // Weights never depend on earlier kernels: the first kTcStages
-            // stages are requested before waiting for the predecessor grid;
+            // Weights never depend on earlier kernels: the first stages of
+            // the ring are requested before waiting for the predecessor grid;
             // their activation tiles follow once it has completed.
             uint32_t stage = 0, phase = 0;
             int issued = 0;
@@ -314,8 +348,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
             auto release_deferred = [&]() {
                 pdl_wait();
                 waited = true;
-                for (int i = 0; i < issued && i < kTcStages; ++i)
-                    tma_load_2d(sm.x[i], &maps.x, def_c[i] * kTileK, def_mt[i] * kTileM, &sm.full[i]);
+                for (int i = 0; i < issued && i < stages; ++i)
+                    tma_load_2d(ring_x + (size_t)i * xbytes, &maps.x, def_c[i] * kTileK, def_mt[i] * tm, &sm.full[i]);
             };
             bool stop = false;
             for (SkIter it(sk, g); it.valid() && !stop; it.advance()) {
@@ -326,20 +360,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                     while (wsel < 2 && wrow >= a.wrows[wsel]) { wrow -= a.wrows[wsel]; ++wsel; }
                 }
                 for (int c = s.c0; c < s.c1; ++c) {
-                    if (!waited && issued == kTcStages) release_deferred();
+                    if (!waited && issued == stages) release_deferred();
                     if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort) || *abort) { stop = true; break; }
-                    mbar_expect_tx(&sm.full[stage], kStageWBytes + kStageXBytes);
+                    mbar_expect_tx(&sm.full[stage], kStageWBytes + xbytes);
+                    unsigned char *wdst = ring_w + (size_t)stage * kStageWBytes;
                     if (E == EPI_SWIGLU) {
-                        tma_load_2d_hint(sm.w[stage], &maps.w[0], c * kTileK, s.nt * 64, &sm.full[stage], wpol);
-                        tma_load_2d_hint(sm.w[stage] + kStageWBytes / 2, &maps.w[1], c * kTileK, s.nt * 64,
-                                         &sm.full[stage], wpol);
+                        tma_load_2d_hint(wdst, &maps.w[0], c * kTileK, s.nt * 64, &sm.full[stage], wpol);
+                        tma_load_2d_hint(wdst + kStageWBytes / 2, &maps.w[1], c * kTileK, s.nt * 64, &sm.full[stage], wpol);
                     } else {
-                        tma_load_2d_hint(sm.w[stage], &maps.w[wsel], c * kTileK, wrow, &sm.full[stage], wpol);
+                        tma_load_2d_hint(wdst, &maps.w[wsel], c * kTileK, wrow, &sm.full[stage], wpol);
                     }
                     if (!waited) { def_c[issued] = c; def_mt[issued] = s.mt; }
-                    else tma_load_2d(sm.x[stage], &maps.x, c * kTileK, s.mt * kTileM, &sm.full[stage]);
+                    else tma_load_2d(ring_x + (size_t)stage * xbytes, &maps.x, c * kTileK, s.mt * tm, &sm.full[stage]);
                     ++issued;
-                    if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+                    if (++stage == (uint32_t)stages) { stage = 0; phase ^= 1; }
                 }
             }
             if (!waited) release_deferred();
@@ -353,23 +387,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
         if (lane == 0) {   // ------------------------------------------- MMA issuer
             uint32_t stage = 0, phase = 0;
             int local = 0;
+            const uint32_t idesc = tc_idesc(tm);
             for (SkIter it(sk, g); it.valid() && !*abort; it.advance(), ++local) {
                 const SkSub s = it.get();
                 const int acc = local & 1;
                 const uint32_t aphase = (local >> 1) & 1;
                 if (!mbar_wait(&sm.tempty[acc], aphase ^ 1, abort)) break;
                 tc_fence_after();
-                const uint32_t d = tmem + acc * kTcAccCols;
+                const uint32_t d = tmem + acc * tm;
                 bool ok = true;
                 for (int c = s.c0; c < s.c1; ++c) {
                     if (!mbar_wait(&sm.full[stage], phase, abort)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t ad = smem_desc_sw128(sm.w[stage]), bd = smem_desc_sw128(sm.x[stage]);
+                    const uint64_t ad = smem_desc_sw128(ring_w + (size_t)stage * kStageWBytes);
+                    const uint64_t bd = smem_desc_sw128(ring_x + (size_t)stage * xbytes);
 #pragma unroll
                     for (int k = 0; k < kTileK / 16; ++k)   // +32 bytes per k step inside the swizzle atom
-                        umma_bf16(d, ad + 2 * k, bd + 2 * k, (c > s.c0 || k > 0) ? 1u : 0u);
+                        umma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (c > s.c0 || k > 0) ? 1u : 0u);
                     umma_commit(&sm.empty[stage]);
-                    if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+                    if (++stage == (uint32_t)stages) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
                 umma_commit(&sm.tfull[acc]);
@@ -382,32 +418,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
         const int et = threadIdx.x - 64;            // 0..127
         const int q = warp & 3;                      // TMEM lane quarter of this warp
         const int n_nt_epi = E == EPI_SWIGLU ? (a.N + 63) / 64 : (a.N + kTileN - 1) / kTileN;
+        const size_t tile_f = (size_t)tm * kTileN;   // floats of one partial tile
         int local = 0;
+        uint32_t hc = 0;   // cluster mode: chunk handovers so far
         for (SkIter it(sk, g); it.valid(); it.advance(), ++local) {
             const SkSub s = it.get();
             const int acc = local & 1;
             const uint32_t aphase = (local >> 1) & 1;
             const size_t slot0 = ((size_t)s.mt * sk.n_nt + s.nt) * a.splits;   // partial / flag slots of this tile
+            // 32-row chunks of the token tile that hold rows below M
+            const int nvalid = min(nch, (a.M - s.mt * tm + kTileM - 1) / kTileM);
             // -------- before the accumulator is ready
-            float4 rest[kEpiVec];   // segments 1.. of the tile, summed in order (reducer only)
             bool good = !*abort;
             const bool defer = a.defer > 0;
-            if (pair) {
-                if (crank == 0) {
-                    if (et == 0) mbar_expect_tx(&sm.peer_full, (uint32_t)((a.pair - 1) * sizeof(sm.tile)));
-                } else {   // the previous tile handed over has been consumed
-                    if (et == 0) good = mbar_wait(&sm.peer_empty, (local & 1) ^ 1, abort);
-                    SyncEpilogue{}();
-                    good = good && !*abort;
-                }
-            }
-            if (!pair && !defer && s.seg == 0 && s.nseg > 1) {
+            const bool reducer = !pair && !defer && s.seg == 0 && s.nseg > 1;
+            if (reducer) {   // the other segments' partials must be published first
                 for (int sg = 1; sg < s.nseg && good; ++sg) {
                     if (et == 0) good = flag_wait(a.ticket + slot0 + sg, abort);
                     SyncEpilogue{}();
                     good = good && !*abort;
-                    if (!good) break;
-                    const float *src = a.part + (slot0 + sg) * (kTileM * kTileN);
+                }
+            }
+            // segments 1.. of chunk 0, summed in order (reducer only)
+            float4 rest[kEpiVec];
+            auto load_rest = [&](int ch) {
+#pragma unroll
+                for (int j = 0; j < kEpiVec; ++j) rest[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int sg = 1; sg < s.nseg; ++sg) {
+                    const float *src = a.part + (slot0 + sg) * tile_f + (size_t)ch * kTileM * kTileN;
 #pragma unroll
                     for (int j = 0; j < kEpiVec; ++j) {
                         const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
@@ -416,88 +454,120 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                         else { rest[j].x += v.x; rest[j].y += v.y; rest[j].z += v.z; rest[j].w += v.w; }
                     }
                 }
-            }
-            if (!defer && s.seg == 0) epilogue_prepare<bf16, E>(a, sm.pre, s.mt, s.nt, et);
+            };
+            if (reducer && good) load_rest(0);
+            if (!defer && s.seg == 0) epilogue_prepare<bf16, E>(a, sm.pre, s.mt * nch, s.nt, et);
             // -------- the accumulator
             const bool ok = good && mbar_wait(&sm.tfull[acc], aphase, abort);
             SyncEpilogue{}();
             if (!ok || *abort) break;
             tc_fence_after();
-            float r[32];
-            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + acc * kTcAccCols, r);
-            tc_fence_before();
-            mbar_arrive(&sm.tempty[acc]);
-            const int f = q * 32 + lane;             // weight row = output feature in the tile
-#pragma unroll
-            for (int j = 0; j < kTileM; ++j) sm.tile[j][f] = r[j];
-            if (pair && crank > 0) {   // hand this segment to rank 0
-                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-                SyncEpilogue{}();
-                if (et == 0) {
-                    const float *land = crank == 1 ? &sm.pre.resid[0][0] : &sm.peer2[0][0];
-                    const uint32_t dst = tc_mapa(smem_u32(land), 0), bar = tc_mapa(smem_u32(&sm.peer_full), 0);
-                    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
-                                 ::"r"(dst), "r"(smem_u32(&sm.tile[0][0])), "r"((uint32_t)sizeof(sm.tile)), "r"(bar) : "memory");
+            bool stop = false;
+            for (int ch = 0; ch < nch; ++ch) {
+                const int mt32 = s.mt * nch + ch;   // this chunk's 32-row tile index
+                const bool last = ch == nch - 1;
+                if (ch >= nvalid) {   // rows past M: nothing to read or write
+                    if (last) { tc_fence_before(); mbar_arrive(&sm.tempty[acc]); }
+                    continue;
                 }
-                continue;
-            }
-            SyncEpilogue{}();
-            if (pair) {   // rank 0: rank 2 + (rank 1 + rank 0), then free the landing tiles
-                bool landed = true;
-                if (et == 0) landed = mbar_wait(&sm.peer_full, local & 1, abort);
-                SyncEpilogue{}();
-                if (!landed || *abort) break;
-#pragma unroll
-                for (int j = 0; j < kEpiVec; ++j) {
-                    const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
-                    float4 &o = *(float4 *)&sm.tile[m][c4];
-                    const float4 p = *(const float4 *)&sm.pre.resid[m][c4];
-                    o.x = p.x + o.x; o.y = p.y + o.y; o.z = p.z + o.z; o.w = p.w + o.w;
-                    if (a.pair > 2) {
-                        const float4 p2 = *(const float4 *)&sm.peer2[m][c4];
-                        o.x = p2.x + o.x; o.y = p2.y + o.y; o.z = p2.z + o.z; o.w = p2.w + o.w;
+                float r[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + acc * tm + ch * kTileM, r);
+                if (last || ch + 1 >= nvalid) {   // the accumulator is drained
+                    tc_fence_before();
+                    if (last) mbar_arrive(&sm.tempty[acc]);
+                }
+                const int f = q * 32 + lane;             // weight row = output feature in the tile
+                if (ch > 0) SyncEpilogue{}();            // the previous chunk's readers are done with the tile
+                if (pair) {   // handover hc of this cluster: one per 32-row chunk, in the same order on every rank
+                    if (crank == 0) {
+                        if (et == 0) mbar_expect_tx(&sm.peer_full, (uint32_t)((a.pair - 1) * sizeof(sm.tile)));
+                    } else {   // rank 0 has consumed the previous handover (so its copy out of sm.tile is done)
+                        bool freed = true;
+                        if (et == 0) freed = mbar_wait(&sm.peer_empty, (hc & 1) ^ 1, abort);
+                        SyncEpilogue{}();
+                        if (!freed || *abort) { stop = true; break; }
                     }
                 }
-                SyncEpilogue{}();
-                if (et > 0 && et < a.pair)
-                    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n"
-                                 ::"r"(tc_mapa(smem_u32(&sm.peer_empty), (uint32_t)et)) : "memory");
-            }
-            if (defer) {   // this segment of the residual update, summed later by the RMSNorm
 #pragma unroll
-                for (int j = 0; j < kEpiVec; ++j) {
-                    const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
-                    const int row = s.mt * kTileM + m, n = s.nt * kTileN + c4;
-                    if (row < a.M && n < a.N)
-                        __stcg((float4 *)(a.rpart + ((size_t)s.seg * a.rpart_rows + row) * a.N + n),
-                               *(const float4 *)&sm.tile[m][c4]);
+                for (int j = 0; j < kTileM; ++j) sm.tile[j][f] = r[j];
+                if (pair && crank > 0) {   // hand this chunk's segment to rank 0
+                    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                    SyncEpilogue{}();
+                    if (et == 0) {
+                        const float *land = crank == 1 ? &sm.pre.resid[0][0] : &sm.peer2[0][0];
+                        const uint32_t dst = tc_mapa(smem_u32(land), 0), bar = tc_mapa(smem_u32(&sm.peer_full), 0);
+                        asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+                                     ::"r"(dst), "r"(smem_u32(&sm.tile[0][0])), "r"((uint32_t)sizeof(sm.tile)), "r"(bar) : "memory");
+                    }
+                    ++hc;
+                    continue;
                 }
                 SyncEpilogue{}();
-                continue;
-            }
-            if (!pair && s.seg > 0) {   // publish this segment for the tile's reducer
-                float *dst = a.part + (slot0 + s.seg) * (kTileM * kTileN);
+                if (pair) {   // rank 0: rank 2 + (rank 1 + rank 0), then free the landing tiles
+                    bool landed = true;
+                    if (et == 0) landed = mbar_wait(&sm.peer_full, hc & 1, abort);
+                    ++hc;
+                    SyncEpilogue{}();
+                    if (!landed || *abort) { stop = true; break; }
 #pragma unroll
-                for (int j = 0; j < kEpiVec; ++j) {
-                    const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
-                    __stcg((float4 *)(dst + m * kTileN + c4), *(const float4 *)&sm.tile[m][c4]);
+                    for (int j = 0; j < kEpiVec; ++j) {
+                        const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
+                        float4 &o = *(float4 *)&sm.tile[m][c4];
+                        const float4 p = *(const float4 *)&sm.pre.resid[m][c4];
+                        o.x = p.x + o.x; o.y = p.y + o.y; o.z = p.z + o.z; o.w = p.w + o.w;
+                        if (a.pair > 2) {
+                            const float4 p2 = *(const float4 *)&sm.peer2[m][c4];
+                            o.x = p2.x + o.x; o.y = p2.y + o.y; o.z = p2.z + o.z; o.w = p2.w + o.w;
+                        }
+                    }
+                    SyncEpilogue{}();
+                    if (et > 0 && et < a.pair)
+                        asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n"
+                                     ::"r"(tc_mapa(smem_u32(&sm.peer_empty), (uint32_t)et)) : "memory");
                 }
+                if (defer) {   // this segment of the residual update, summed later by the RMSNorm
+#pragma unroll
+                    for (int j = 0; j < kEpiVec; ++j) {
+                        const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
+                        const int row = mt32 * kTileM + m, n = s.nt * kTileN + c4;
+                        if (row < a.M && n < a.N)
+                            __stcg((float4 *)(a.rpart + ((size_t)s.seg * a.rpart_rows + row) * a.N + n),
+                                   *(const float4 *)&sm.tile[m][c4]);
+                    }
+                    continue;
+                }
+                if (!pair && s.seg > 0) {   // publish this segment's chunk for the tile's reducer
+                    float *dst = a.part + (slot0 + s.seg) * tile_f + (size_t)ch * kTileM * kTileN;
+#pragma unroll
+                    for (int j = 0; j < kEpiVec; ++j) {
+                        const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
+                        __stcg((float4 *)(dst + m * kTileN + c4), *(const float4 *)&sm.tile[m][c4]);
+                    }
+                    continue;
+                }
+                if (reducer) {   // (segments 1..) + segment 0
+                    if (ch > 0) load_rest(ch);
+#pragma unroll
+                    for (int j = 0; j < kEpiVec; ++j) {
+                        const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
+                        float4 &o = *(float4 *)&sm.tile[m][c4];
+                        o.x = rest[j].x + o.x; o.y = rest[j].y + o.y; o.z = rest[j].z + o.z; o.w = rest[j].w + o.w;
+                    }
+                    SyncEpilogue{}();
+                }
+                if (ch > 0 && !defer && s.seg == 0) {   // chunk 0's was fetched while the chunks streamed
+                    epilogue_prepare<bf16, E>(a, sm.pre, mt32, s.nt, et);
+                    SyncEpilogue{}();
+                }
+                epilogue<bf16, SyncEpilogue, E>(a, sm.tile, mt32, s.nt, n_nt_epi, et, SyncEpilogue{}, &sm.pre);
+            }
+            if (stop) break;
+            if (!pair && !defer && s.seg > 0) {   // every chunk of this segment is out: raise its flag
                 __threadfence();
                 SyncEpilogue{}();
                 if (et == 0) asm volatile("st.release.gpu.global.b32 [%0], %1;\n" ::"l"(a.ticket + slot0 + s.seg), "r"(1) : "memory");
-                continue;
             }
-            if (!pair && s.nseg > 1) {   // reducer: (segments 1..) + segment 0, then clear the flags
-#pragma unroll
-                for (int j = 0; j < kEpiVec; ++j) {
-                    const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
-                    float4 &o = *(float4 *)&sm.tile[m][c4];
-                    o.x = rest[j].x + o.x; o.y = rest[j].y + o.y; o.z = rest[j].z + o.z; o.w = rest[j].w + o.w;
-                }
-                if (et > 0 && et < s.nseg) a.ticket[slot0 + et] = 0;
-                SyncEpilogue{}();
-            }
-            epilogue<bf16, SyncEpilogue, E>(a, sm.tile, s.mt, s.nt, n_nt_epi, et, SyncEpilogue{}, &sm.pre);
+            if (reducer && et > 0 && et < s.nseg) a.ticket[slot0 + et] = 0;   // flags ready for the next call
             SyncEpilogue{}();
         }
     }
@@ -513,7 +583,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(2 * kTcAccCols));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(tcols));
     }
 }
 
@@ -551,11 +621,24 @@ bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, ui
     return make_tmap_box(m, ptr, rows, cols, 64, box_rows);
 }
 
-size_t gemm_tc_smem_bytes() { return sizeof(TcSmem) + 1024; }
+// Dynamic shared memory of a launch with token tiles of tm rows (the fixed
+// part, its ring, and slack for the 1024-byte alignment of the base).
+size_t gemm_tc_smem_bytes(int tm)
+{
+    return 1024 + kTcRingOffset + (size_t)tc_stages(tm) * (kStageWBytes + (size_t)tm * kTileK * 2);
+}
+
+void gemm_token_tile(int M, int *n_mt, int *tm)
+{
+    const int n = (M + kTcMaxTM - 1) / kTcMaxTM;
+    const int per = (M + n - 1) / n;
+    *n_mt = n;
+    *tm = (per + kTileM - 1) / kTileM * kTileM;
+}
 
 template <int E> static cudaError_t set_smem()
 {
-    return cudaFuncSetAttribute(gemm_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_tc_smem_bytes());
+    return cudaFuncSetAttribute(gemm_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBudget);
 }
 
 cudaError_t gemm_tc_init_attributes()
@@ -590,9 +673,11 @@ int sk_max_segments(int n_nt, int chunks)
 
 // Launches the tcgen05 kernel when every operand has a tensor map; returns
 // cudaErrorNotSupported otherwise (the caller then uses the SIMT kernel).
-// a.splits must hold sk_max_segments(n_nt, Kd / 64).
-cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, cudaStream_t s)
+// a.splits must hold sk_max_segments(n_nt, Kd / 64); n_mt token tiles of tm
+// rows (gemm_token_tile).
+cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int tm, int n_nt, cudaStream_t s)
 {
+    if (tm < kTileM || tm > kTcMaxTM || tm % kTileM) return cudaErrorInvalidValue;
     TcMaps maps;
     memset(&maps, 0, sizeof(maps));
     const int nseg = a.epi == EPI_SWIGLU ? 2 : 3;
@@ -603,18 +688,20 @@ cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, 
         maps.w[i] = it->second;
         if (a.epi != EPI_SWIGLU && i < 2 && a.wrows[i + 1] > 0 && a.wrows[i] % kTileN) return cudaErrorNotSupported;
     }
-    auto it = c.tmaps.find(TmapKey{a.x, (uint32_t)kTileM});
+    auto it = c.tmaps.find(TmapKey{a.x, (uint32_t)tm});
     if (it == c.tmaps.end()) return cudaErrorNotSupported;
     maps.x = it->second;
     SkShape k;
     k.chunks = a.Kd / kTileK;
     k.n_nt = n_nt;
     k.n_mt = n_mt;
+    k.tm = tm;
+    k.stages = tc_stages(tm);
     k.P = (long)n_nt * k.chunks;
     // deferred residual: one piece per (tile, segment), cut at whole chunks
     k.G = a.defer > 0 ? n_nt * a.defer : (int)std::min<long>(kNumSMs, k.P);
     if (a.defer > 0 && (k.chunks % a.defer || a.defer > kResidSlots || !a.rpart)) return cudaErrorInvalidValue;
-    const size_t smem = gemm_tc_smem_bytes();
+    const size_t smem = gemm_tc_smem_bytes(tm);
     if (a.pair > 1) {   // a.pair k segments per n tile, one cluster of a.pair CTAs per tile
         if (a.epi != EPI_QKV || a.defer > 0 || a.pair > 3 || k.chunks < a.pair) return cudaErrorInvalidValue;
         k.G = a.pair * n_nt;

@@ -266,7 +266,11 @@ struct AtMaps {
     CUtensorMap vb;   // 2-D transient V^T [dim rows][Kp], box {64, 128}
 };
 cudaError_t attn_tc_init_attributes();
-cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int n_nt, cudaStream_t s);
+cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int tm, int n_nt, cudaStream_t s);
+// Token tiles of the tensor-core GEMM for M token rows: n_mt tiles of tm rows
+// (a multiple of 32, at most 256, as even as the multiple allows).
+void gemm_token_tile(int M, int *n_mt, int *tm);
+constexpr int kTcTokenTileMax = 256;
 int sk_max_segments(int n_nt, int chunks);
 cudaError_t attention_init_attributes();
 // The attention of one call: the tensor-core kernel when the shape and the
