@@ -51,7 +51,9 @@ constexpr int kTcThreads = 192;
 constexpr int kTcMaxTM = 256;                           // token rows per tile: one MMA's largest N
 constexpr uint32_t kStageWBytes = kTileN * kTileK * 2;  // 16 KiB
 constexpr long long kSpinCycles = 4000000000LL;        // ~2 s at the B200 SM clock
-constexpr size_t kTcSmemBudget = 227 * 1024;            // dynamic shared memory of one CTA
+// dynamic shared memory of one CTA: the 227 KiB a block may opt in to, less
+// the epilogues' static shared arrays (at most 1 KiB) and 1 KiB of slack
+constexpr size_t kTcSmemBudget = 225 * 1024;
 
 // The fixed part of the shared memory; the stage ring (kStageWBytes weight
 // tiles, then TM x 128-byte token tiles, stages of each) follows it at a
