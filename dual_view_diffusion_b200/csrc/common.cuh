@@ -41,19 +41,29 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k)
 
 enum Purpose : uint32_t { PURPOSE_DRAFT = 1, PURPOSE_ACCEPT = 2, PURPOSE_RESIDUAL = 3, PURPOSE_AR = 4 };
 
-// Uniform in (0,1) from counter (id, row, step, purpose) and key = seed:
-// top 24 bits of the first output word, centred in their cell.
-__device__ __forceinline__ float uniform01(uint64_t seed, uint32_t step, uint32_t row, uint32_t id,
-                                           uint32_t purpose)
+// The uniform u = (k + 1/2) / 2^24 in (0, 1), k = the top 24 bits of the
+// first output word of Philox4x32-10 at counter (id, row, step, purpose) and
+// key = seed, is only ever used through -log(u), returned here.  u itself is
+// not an fp32 number once k >= 2^23 (k + 1/2 then needs 25 bits), and
+// rounding it would move -log(u) by up to 2^-25 / (1 - u) relative: for the
+// draws nearest 1, which decide Gumbel-max winners, that is ~1e-3.  So for
+// u > 1/2 the exact complement 1 - u = (2^24 - 1 - k + 1/2) / 2^24 (fewer
+// than 24 significant bits) goes through log1p.
+__device__ __forceinline__ float neg_log_uniform(uint64_t seed, uint32_t step, uint32_t row, uint32_t id,
+                                                 uint32_t purpose)
 {
     const uint4 o = philox4x32_10(make_uint4(id, row, step, purpose),
                                   make_uint2((uint32_t)seed, (uint32_t)(seed >> 32)));
-    return ((float)(o.x >> 8) + 0.5f) * (1.0f / 16777216.0f);
+    const uint32_t k = o.x >> 8;
+    constexpr float kInv24 = 1.0f / 16777216.0f;
+    if (k < (1u << 23)) return -logf(((float)k + 0.5f) * kInv24);
+    return -log1pf(-(((float)((1u << 24) - 1u - k) + 0.5f) * kInv24));
 }
 
+// Gumbel noise -log(-log u) of the same uniform.
 __device__ __forceinline__ float gumbel(uint64_t seed, uint32_t step, uint32_t row, uint32_t id, uint32_t purpose)
 {
-    return -logf(-logf(uniform01(seed, step, row, id, purpose)));
+    return -logf(neg_log_uniform(seed, step, row, id, purpose));
 }
 
 // Row id used in the RNG counter: sequence b, block row k.

@@ -270,8 +270,8 @@ __global__ void commit_decide_kernel(CommitArgs a)
         } else {
             const uint32_t step = (uint32_t)*a.step;
             for (int k = 0; k < a.K; ++k) {
-                const float u = uniform01(a.seed, step, rng_row(b, k), 0, PURPOSE_ACCEPT);
-                if (!(logf(u) < a.logp[b * a.K + k] - a.logq[b * a.K + k])) { j = k; n = k + 1; break; }
+                const float log_u = -neg_log_uniform(a.seed, step, rng_row(b, k), 0, PURPOSE_ACCEPT);
+                if (!(log_u < a.logp[b * a.K + k] - a.logq[b * a.K + k])) { j = k; n = k + 1; break; }
             }
         }
         a.n_out[b] = n;
