@@ -241,11 +241,7 @@ struct CommitArgs {
     int *any_reject;
     const void *fin_verify, *fin_draft;
     void *res_x;
-    // fused final norm (null: not fused): partial sums of squares of the fin
-    // rows ([row][ss_tiles]); the staged rows' 1/rms go to res_inv
-    const float *ss_verify, *ss_draft;
-    int ss_tiles;
-    float eps;
+    const float *inv_verify, *inv_draft;   // fused final norm: 1/rms of the fin rows (null: not fused)
     float *res_inv;
     int d, esize;
     int32_t *n_out, *tokens_out, *anchor_io, *seq_lens;
@@ -290,11 +286,9 @@ __global__ void commit_decide_kernel(CommitArgs a)
         const char *sd = (const char *)a.fin_draft + (size_t)(b * a.K + s_j) * bytes;
         char *dv = (char *)a.res_x + (size_t)(2 * b) * bytes;
         for (size_t i = threadIdx.x; i < bytes; i += blockDim.x) { dv[i] = sv[i]; dv[bytes + i] = sd[i]; }
-        if (a.ss_verify && threadIdx.x < 2) {   // summed in tile order, as the projections do
-            const float *p = (threadIdx.x == 0 ? a.ss_verify : a.ss_draft) + (size_t)(b * a.K + s_j) * a.ss_tiles;
-            float ss = 0.f;
-            for (int t = 0; t < a.ss_tiles; ++t) ss += p[t];
-            a.res_inv[2 * b + threadIdx.x] = 1.0f / sqrtf(ss / a.d + a.eps);
+        if (a.inv_verify && threadIdx.x == 0) {
+            a.res_inv[2 * b] = a.inv_verify[b * a.K + s_j];
+            a.res_inv[2 * b + 1] = a.inv_draft[b * a.K + s_j];
         }
     }
 }
@@ -540,8 +534,8 @@ static CommitArgs commit_args(const Ctx &c, const orthrus_kv_t &kv, int B, int K
     a.draft = c.draft; a.g = c.g; a.res_tok = c.res_tok; a.logp = c.logp; a.logq = c.logq;
     a.rej_row = c.rej_row; a.any_reject = c.any_reject;
     a.fin_verify = c.fin_verify; a.fin_draft = c.fin_draft; a.res_x = c.res_x;
-    a.ss_verify = c.fused_norm ? c.norm_ss_fin[0] : nullptr; a.ss_draft = c.fused_norm ? c.norm_ss_fin[1] : nullptr;
-    a.ss_tiles = (c.cfg.hidden + kTileN - 1) / kTileN; a.eps = c.cfg.rms_eps; a.res_inv = c.res_inv;
+    a.inv_verify = c.fused_norm ? c.inv_fin[0] : nullptr; a.inv_draft = c.fused_norm ? c.inv_fin[1] : nullptr;
+    a.res_inv = c.res_inv;
     a.d = c.cfg.hidden; a.esize = c.esize;
     a.n_out = n_out; a.tokens_out = tokens_out; a.anchor_io = anchor_io; a.seq_lens = kv.seq_lens;
     a.append_out = append_out; a.produced = c.produced; a.append_stride = append_stride; a.append_max = append_max;
@@ -640,11 +634,11 @@ cudaError_t launch_kl_lm_head(const Ctx &c, const void *h_a, const void *h_d, in
     return launch_k(kl_finalize_kernel, (rows + 7) / 8, 256, 0, s, k);
 }
 
-cudaError_t launch_logits_dump(const Ctx &c, const void *fin, const float *row_ss, int M, float *logits,
+cudaError_t launch_logits_dump(const Ctx &c, const void *fin, const float *row_scale, int M, float *logits,
                                cudaStream_t s)
 {
     GemmArgs g{};
-    if (row_ss) set_row_ss(g, c, row_ss);
+    g.row_scale = row_scale;
     g.x = fin; g.M = M; g.N = c.cfg.vocab; g.Kd = c.cfg.hidden;
     g.w[0] = c.lm_head; g.wrows[0] = c.cfg.vocab;
     g.epi = EPI_LOGITS; g.logits = logits;

@@ -159,7 +159,7 @@ cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s)
     }
     // only the tensor-core kernel defers residual segments and scales rows by
     // a fused norm's 1/rms: never fall back to the SIMT kernel with them
-    if (a.defer > 0 || a.row_scale || a.row_ss || a.norm_cnt) return cudaErrorInvalidValue;
+    if (a.defer > 0 || a.row_scale || a.norm_cnt) return cudaErrorInvalidValue;
     a.splits = 1;
     const long units = (long)n_mt * n_nt;
     const int grid = (int)(units < kNumSMs ? units : kNumSMs);

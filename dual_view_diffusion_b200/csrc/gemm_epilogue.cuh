@@ -162,39 +162,36 @@ __device__ void epilogue_prepare(const GemmArgs &a, EpiPre &pre, int mt, int nt,
 // fenced): h += segments 0 .. defer-1 in segment order (the order the
 // unfused RMSNorm kernel folds them in), then, with a norm gain, the bf16
 // operand x = h * gain of the next projection and each row's sum of squares
-// over the tile's 128 columns.  The next projection sums those partials in
-// tile order into 1/rms = 1/sqrt(mean(h^2) + eps) and scales its
-// accumulator rows by it, so the normalised operand RMSNorm(h) = 1/rms *
-// (h * gain) is never formed: y = 1/rms * ((h * gain) . W^T).
-__device__ inline void resid_fold_norm(const GemmArgs &a, int mt, int nt, int n_nt, int tid)
+// over the tile's 128 columns; the last n tile of the 32-row tile to finish
+// sums those partials in n-tile order into inv = 1/sqrt(mean(h^2) + eps).
+// The next projection scales its accumulator rows by inv, so the normalised
+// operand RMSNorm(h) = inv * (h * gain) never has to be formed: y = inv *
+// ((h * gain) . W^T).  flag: a shared int the 128 threads use to agree on
+// the row-tile ticket.
+template <class Sync>
+__device__ void resid_fold_norm(const GemmArgs &a, int mt, int nt, int n_nt, int tid, Sync sync, int *flag)
 {
     const int S = a.defer;
-    float4 v[kEpiVec], u[2][kEpiVec];
+    float4 v[kEpiVec];
     bool ok[kEpiVec];
-    // h and the first two segments in one round of loads, then pairs
 #pragma unroll
     for (int j = 0; j < kEpiVec; ++j) {
         const int c = tid + j * kEpiThreads, m = c >> 5, n = nt * kTileN + (c & 31) * 4, row = mt * kTileM + m;
         ok[j] = row < a.M && n < a.N;
-        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-        v[j] = ok[j] ? __ldcg((const float4 *)&a.resid[(size_t)row * a.N + n]) : z;
+        v[j] = ok[j] ? __ldcg((const float4 *)&a.resid[(size_t)row * a.N + n]) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // segments two at a time, every load of a pair in flight before its adds
+    for (int s0 = 0; s0 < S; s0 += 2) {
+        float4 u[2][kEpiVec];
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl)
-            u[sl][j] = (sl < S && ok[j]) ? __ldcg((const float4 *)(a.rpart + ((size_t)sl * a.rpart_rows + row) * a.N + n))
-                                         : z;
-    }
-    for (int s0 = 0; s0 < S; s0 += 2) {
-        if (s0 > 0) {
 #pragma unroll
-            for (int sl = 0; sl < 2; ++sl)
-#pragma unroll
-                for (int j = 0; j < kEpiVec; ++j) {
-                    const int c = tid + j * kEpiThreads, m = c >> 5, n = nt * kTileN + (c & 31) * 4, row = mt * kTileM + m;
-                    u[sl][j] = (s0 + sl < S && ok[j])
-                                   ? __ldcg((const float4 *)(a.rpart + ((size_t)(s0 + sl) * a.rpart_rows + row) * a.N + n))
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-        }
+            for (int j = 0; j < kEpiVec; ++j) {
+                const int c = tid + j * kEpiThreads, m = c >> 5, n = nt * kTileN + (c & 31) * 4, row = mt * kTileM + m;
+                u[sl][j] = (s0 + sl < S && ok[j])
+                               ? __ldcg((const float4 *)(a.rpart + ((size_t)(s0 + sl) * a.rpart_rows + row) * a.N + n))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl) {
             if (s0 + sl >= S) break;
@@ -229,31 +226,22 @@ __device__ inline void resid_fold_norm(const GemmArgs &a, int mt, int nt, int n_
     }
     // ready for the next launch: this tile's arrivals are all in
     if (tid == 0) a.norm_cnt[(size_t)mt * n_nt + nt] = 0;
-}
-
-// 1/rms of rows row0 .. row0 + n - 1 from a fused norm's partial sums
-// (row_ss, summed in tile order) into out[0 .. n), n <= 2 * kEpiThreads.
-__device__ inline void rows_inv_from_ss(const GemmArgs &a, int row0, int n, int tid, float *out)
-{
-    for (int r = tid; r < n; r += kEpiThreads) {
-        const int row = row0 + r;
-        float inv = 0.f;
+    if (!a.norm_gain) return;
+    __threadfence();
+    sync();
+    if (tid == 0) *flag = atomicAdd(a.norm_cnt + a.norm_cnt_tiles + mt, 1);
+    sync();
+    if (*flag != n_nt - 1) return;
+    __threadfence();
+    if (tid < kTileM) {   // the last n tile of this 32-row tile: every row's 1/rms
+        const int row = mt * kTileM + tid;
         if (row < a.M) {
-            const float *p = a.row_ss + (size_t)row * a.row_ss_tiles;
             float ss = 0.f;
-            int t = 0;
-            for (; t + 8 <= a.row_ss_tiles; t += 8) {   // eight loads in flight, summed in tile order
-                float x[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = __ldcg(p + t + e);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ss += x[e];
-            }
-            for (; t < a.row_ss_tiles; ++t) ss += __ldcg(p + t);
-            inv = 1.0f / sqrtf(ss / a.row_ss_cols + a.row_ss_eps);
+            for (int t = 0; t < n_nt; ++t) ss += __ldcg(a.norm_ss + (size_t)row * n_nt + t);
+            a.norm_inv[row] = 1.0f / sqrtf(ss / a.N + a.norm_eps);
         }
-        out[r] = inv;
     }
+    if (tid == 0) a.norm_cnt[a.norm_cnt_tiles + mt] = 0;
 }
 
 // pre: filled by epilogue_prepare for this tile (and made visible with a

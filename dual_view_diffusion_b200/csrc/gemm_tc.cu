@@ -49,7 +49,6 @@ namespace orthrus {
 constexpr int kTcStages = 8;                             // most ring stages (TM = 32)
 constexpr int kTcThreads = 192;
 constexpr int kTcMaxTM = 256;                           // token rows per tile: one MMA's largest N
-constexpr int kTcMaxTMFixed = kTcMaxTM;
 constexpr uint32_t kStageWBytes = kTileN * kTileK * 2;  // 16 KiB
 constexpr long long kSpinCycles = 4000000000LL;        // ~2 s at the B200 SM clock
 // dynamic shared memory of one CTA: the 227 KiB a block may opt in to, less
@@ -68,7 +67,6 @@ struct TcSmem {
     uint32_t tmem_base;
     int abort;
     int s_last;
-    float inv[kTcMaxTMFixed];         // 1/rms of the token tile's rows (fused norm consumers)
 };
 constexpr size_t kTcRingOffset = (sizeof(TcSmem) + 1023) / 1024 * 1024;
 
@@ -425,7 +423,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
         const size_t tile_f = (size_t)tm * kTileN;   // floats of one partial tile
         int local = 0;
         uint32_t hc = 0;   // cluster mode: chunk handovers so far
-        int inv_mt = -1;   // token tile whose 1/rms rows sm.inv holds
         for (SkIter it(sk, g); it.valid(); it.advance(), ++local) {
             const SkSub s = it.get();
             const int acc = local & 1;
@@ -461,11 +458,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                 }
             };
             if (reducer && good) load_rest(0);
-            if (a.row_ss && s.mt != inv_mt) {   // this token tile's 1/rms, while its chunks stream
-                SyncEpilogue{}();                 // the previous tile's readers are done with sm.inv
-                rows_inv_from_ss(a, s.mt * tm, tm, et, sm.inv);
-                inv_mt = s.mt;
-            }
             if (!defer && s.seg == 0) epilogue_prepare<bf16, E>(a, sm.pre, s.mt * nch, s.nt, et);
             // -------- the accumulator
             const bool ok = good && mbar_wait(&sm.tfull[acc], aphase, abort);
@@ -551,7 +543,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                         SyncEpilogue{}();
                         if (sm.s_last == a.defer - 1) {
                             __threadfence();
-                            resid_fold_norm(a, mt32, s.nt, n_nt_epi, et);
+                            resid_fold_norm(a, mt32, s.nt, n_nt_epi, et, SyncEpilogue{}, &sm.s_last);
                         }
                         SyncEpilogue{}();
                     }
@@ -580,11 +572,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                     epilogue_prepare<bf16, E>(a, sm.pre, mt32, s.nt, et);
                     SyncEpilogue{}();
                 }
-                if (a.row_scale || a.row_ss) {   // a fused RMSNorm's 1/rms of each token row
+                if (a.row_scale) {   // a fused RMSNorm's 1/rms of each token row
 #pragma unroll
                     for (int j = 0; j < kEpiVec; ++j) {
                         const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4, row = mt32 * kTileM + m;
-                        const float sc = row >= a.M ? 0.f : a.row_ss ? sm.inv[ch * kTileM + m] : __ldcg(a.row_scale + row);
+                        const float sc = row < a.M ? __ldcg(a.row_scale + row) : 0.f;
                         float4 &o = *(float4 *)&sm.tile[m][c4];
                         o.x *= sc; o.y *= sc; o.z *= sc; o.w *= sc;
                     }

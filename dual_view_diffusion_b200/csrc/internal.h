@@ -115,22 +115,22 @@ struct GemmArgs {
     // Fused residual fold and RMSNorm (EPI_RESID with defer > 0, tensor-core
     // path, norm_cnt non-null): the last of the defer segments of a (32-row
     // tile, n tile) to arrive adds h and the segments in segment order into
-    // h, and with a norm gain writes norm_x = bf16(h * norm_gain) and each
-    // row's sum of squares over the tile's columns to norm_ss[row][n tile].
-    // norm_cnt[mt32 * n_nt + nt]: arrival counters, zero between launches
-    // (each last arriver resets its own).
+    // h, writes norm_x = bf16(h * norm_gain) (norm_gain non-null) and each
+    // row's sum of squares over the tile's columns to norm_ss; the last n
+    // tile of a 32-row tile to arrive turns those into norm_inv[row] =
+    // 1/sqrt(mean(h^2) + norm_eps).  Counters: norm_cnt[mt32 * n_nt + nt]
+    // per tile, then norm_cnt[n_mt32 * n_nt + mt32] per 32-row tile, zero
+    // between launches (each last arriver resets its own).
     const void *norm_gain;
     void *norm_x;            // [M][N] bf16
+    float *norm_inv;         // [M]
     float *norm_ss;          // [M][n_nt]
     int *norm_cnt;
-    // consumers of a fused norm: accumulator row r is multiplied by its
-    // 1/rms, either given (row_scale[r]) or formed from the folding GEMM's
-    // partial sums (row_ss[r][0 .. row_ss_tiles), summed in tile order:
-    // 1/sqrt(sum / row_ss_cols + row_ss_eps)); both null: no scaling
+    int norm_cnt_tiles;      // n_mt32 * n_nt: offset of the per-row-tile counters
+    float norm_eps;
+    // consumers of a fused norm: accumulator row r is multiplied by
+    // row_scale[r] before the epilogue (null: no scaling)
     const float *row_scale;
-    const float *row_ss;
-    int row_ss_tiles, row_ss_cols;
-    float row_ss_eps;
 };
 
 struct AttnArgs {
@@ -248,10 +248,9 @@ struct Ctx {
     // draft), of the residual-draw rows (res_inv); partial sums of squares
     // and arrival counters of the folding GEMMs
     bool fused_norm;
-    float *res_inv;          // [2 * max_batch] 1/rms of the residual-draw rows
-    float *norm_ss;          // [Rw][ceil(hidden / 128)] partial sums of squares of c.a's rows
-    float *norm_ss_fin[2];   // [R][ceil(hidden / 128)] the same for fin_verify (0) and fin_draft (1)
-    int *norm_cnt;           // [Rw / 32][ceil(hidden / 128)] arrival counters
+    float *inv, *inv_fin[2], *res_inv;   // [Rw], [R] x 2, [2 * max_batch]
+    float *norm_ss;          // [Rw][ceil(hidden / 128)]
+    int *norm_cnt;           // [Rw / 32][ceil(hidden / 128) + 1]
     int32_t *g;              // [R]
     float *logp, *lse_p;     // [R]
     int32_t *rej_row;        // [max_batch]
@@ -332,9 +331,8 @@ cudaError_t launch_set_lens(const Ctx &c, int32_t *seq_lens, int b, int value, i
                             const int32_t *tokens, cudaStream_t s);
 cudaError_t launch_pack_block(const Ctx &c, const void *k_src, const void *v_src, void *k_dst, void *v_dst, int B,
                               int K, int kp, cudaStream_t s);
-cudaError_t launch_logits_dump(const Ctx &c, const void *fin, const float *row_ss, int M, float *logits,
+cudaError_t launch_logits_dump(const Ctx &c, const void *fin, const float *row_scale, int M, float *logits,
                                cudaStream_t s);
-void set_row_ss(GemmArgs &g, const Ctx &c, const float *ss);
 // Tree verification (tree.cu): the draft tree's builder and its commit.
 struct TreeBuildArgs {   // one best-first tree per sequence
     const int32_t *ids;      // [B][D][W] candidate ids, best first
