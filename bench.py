@@ -37,19 +37,9 @@ train_kernels  the training-side kernels (block-masked attention of a packed
           2048-position sequence with 256 anchor blocks; the forward-KL
           LM-head epilogue over the full vocabulary), each timed alone beside
           the oracle on a sample
-sampled / plain_ar / tree / adaptive  the other decode loops on the same
-          engine: the step at T = 1.0 with rejection sampling, one AR
-          forward per token (and the Orthrus / AR ratio), a tree-verified
-          step (top-4 candidates, 31 nodes), the adaptive block length
-step_sweep  one decode step per (L, batch, K) cell of the long-context sweep
-          (reduced by default: L at batch 1, K at L = 2K, batch at L = 8K;
-          --sweep full for every cell that fits), synthetic cache, forced
-          acceptance
-config_1p7b  the Qwen3-1.7B-shaped model's decode step and plain AR
 cpu_baseline  the CPU oracle, as it stands, timed on a bounded sample (one
-          layer of each view at full width over 8 block rows plus 1/16 of
-          the LM head) and scaled to a full step; the reference arm
-          (--impl reference) times the same sample
+          layer of each view at full width plus 1/16 of the LM head) and
+          scaled to a full step
 
 Weights and the prompt are larger than L2 (18 GB of weights per step), so no
 flush is needed between steps.

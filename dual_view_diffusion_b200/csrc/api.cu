@@ -125,10 +125,6 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
     const size_t o_lm = take(Rlm * n_vtiles * sizeof(LmPart));
     const size_t o_tok = take(Rw * 4), o_pos = take(mb * 4), o_bt = take(mb * 4), o_pr = take(4);
     const size_t o_ttok = take(R * 4), o_tdep = take(R * 4), o_tmask = take(R * 16);
-    // fused residual + RMSNorm: 1/rms rows, sums of squares per (row, n tile), counters
-    const size_t nnt_d = (d + kTileN - 1) / kTileN, nmt_w = (Rw + kTileM - 1) / kTileM;
-    const size_t o_inv = take(Rw * 4), o_ifv = take(R * 4), o_ifd = take(R * 4), o_rinv = take(2 * mb * 4);
-    const size_t o_nss = take(Rw * nnt_d * 4), o_ncnt = take(nmt_w * (nnt_d + 1) * 4);
     const size_t o_bz = take(mb * 4);   // zeros, never written
     const size_t o_dr = take(R * 4), o_lq = take(R * 4), o_lsq = take(R * 4), o_g = take(R * 4), o_lp = take(R * 4),
                  o_lsp = take(R * 4), o_ent = take(R * 4);
@@ -151,11 +147,6 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
         x->tok = (int32_t *)P(o_tok); x->pos0 = (int32_t *)P(o_pos); x->bt_rows = (int32_t *)P(o_bt);
         x->bt_zero = (int32_t *)P(o_bz);
         x->tree_tok = (int32_t *)P(o_ttok); x->tree_depth = (int32_t *)P(o_tdep); x->tree_mask = (uint32_t *)P(o_tmask);
-        x->inv = (float *)P(o_inv); x->inv_fin[0] = (float *)P(o_ifv); x->inv_fin[1] = (float *)P(o_ifd);
-        x->res_inv = (float *)P(o_rinv); x->norm_ss = (float *)P(o_nss); x->norm_cnt = (int *)P(o_ncnt);
-        x->fused_norm = use_tensor_cores(c) && c.hidden % kTileK == 0 &&
-                        resid_defer_slots(c, c.hidden, c.n_q_heads * c.head_dim) > 0 &&
-                        resid_defer_slots(c, c.hidden, c.ffn) > 0;
         x->prefill_row = (int32_t *)P(o_pr);
         x->draft = (int32_t *)P(o_dr); x->logq = (float *)P(o_lq); x->lse_q = (float *)P(o_lsq);
         x->ent = (float *)P(o_ent);
@@ -177,7 +168,6 @@ static void rebase(Ctx *x, char *ws)
     fix(x->fin_draft); fix(x->fin_verify); fix(x->res_x); fix(x->attn_part); fix(x->attn_ml); fix(x->gemm_part);
     fix(x->gemm_ticket); fix(x->lm_part); fix(x->resid_part); fix(x->rope_invf); fix(x->tok); fix(x->pos0); fix(x->bt_rows); fix(x->bt_zero); fix(x->prefill_row);
     fix(x->tree_tok); fix(x->tree_depth); fix(x->tree_mask);
-    fix(x->inv); fix(x->inv_fin[0]); fix(x->inv_fin[1]); fix(x->res_inv); fix(x->norm_ss); fix(x->norm_cnt);
     fix(x->draft); fix(x->logq); fix(x->lse_q); fix(x->ent); fix(x->g); fix(x->logp); fix(x->lse_p); fix(x->rej_row);
     fix(x->res_tok); fix(x->any_reject); fix(x->err); fix(x->produced); fix(x->step); fix(x->n_buf);
     fix(x->tok_buf); fix(x->anchor_buf);
@@ -253,25 +243,12 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
     const orthrus_config_t &f = c.cfg;
     const int M = B * K, hd = f.head_dim;
     cudaError_t e;
-    // residual segments the O and down projections leave for the next
-    // RMSNorm.  Tensor-core path (c.fused_norm): those GEMMs fold their own
-    // segments into h and write the next projection's operand h * gain and
-    // each row's 1/rms, which the next projection applies to its
-    // accumulator; only layer 0's attention norm is a kernel of its own.
+    // residual segments the O and down projections leave for the next RMSNorm
     int pending = 0;
     const int defer_o = resid_defer_slots(f, f.hidden, f.n_q_heads * hd), defer_dn = resid_defer_slots(f, f.hidden, f.ffn);
-    const bool fused = c.fused_norm;
-    const int n_nt_d = (f.hidden + kTileN - 1) / kTileN;
-    auto fold = [&](GemmArgs &g, const void *gain, void *x_out, float *inv_out) {
-        if (!fused) return;
-        g.norm_gain = gain; g.norm_x = x_out; g.norm_inv = inv_out; g.norm_ss = c.norm_ss; g.norm_cnt = c.norm_cnt;
-        g.norm_cnt_tiles = ((M + kTileM - 1) / kTileM) * n_nt_d; g.norm_eps = f.rms_eps;
-    };
-    float *inv_fin = fin == c.fin_draft ? c.inv_fin[1] : c.inv_fin[0];
     for (int l = 0; l < f.n_layers; ++l) {
         const orthrus_layer_weights_t &W = c.layers[l];
-        if (!fused || l == 0)
-            if ((e = launch_rmsnorm(c, c.h, W.attn_norm, c.a, M, pending, s)) != cudaSuccess) return e;
+        if ((e = launch_rmsnorm(c, c.h, W.attn_norm, c.a, M, pending, s)) != cudaSuccess) return e;
         GemmArgs q{};
         q.x = c.a; q.M = M; q.Kd = f.hidden;
         q.w[0] = view ? W.wq_diff : W.wq; q.w[1] = view ? W.wk_diff : W.wk; q.w[2] = view ? W.wv_diff : W.wv;
@@ -281,7 +258,6 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
         q.kv_to_cache = view == 0; q.k_blk = c.k_diff; q.v_blk = c.v_diff; q.kp = c.kp; q.bmax = f.max_batch;
         q.kv = kv_view(kv); q.pos0 = pos0; q.bt_rows = bt_rows; q.K = K; q.rope_theta = (double)f.rope_theta;
         q.rope_invf = c.rope_invf; q.rope_pos = view == 0 ? rope_pos : nullptr;
-        q.row_scale = (fused && l > 0) ? c.inv : nullptr;
         {
             ProbeScope ps(c, 0, l, view, s);
             if ((e = launch_gemm(c, q, s)) != cudaSuccess) return e;
@@ -306,18 +282,15 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
         GemmArgs o{};
         o.x = c.attn_o; o.M = M; o.N = f.hidden; o.Kd = f.n_q_heads * hd; o.w[0] = W.wo; o.wrows[0] = f.hidden;
         o.epi = EPI_RESID; o.resid = c.h; o.defer = defer_o; o.rpart = c.resid_part; o.rpart_rows = c.Rw;
-        fold(o, W.ffn_norm, c.a, c.inv);
         {
             ProbeScope ps(c, 0, l, view, s);
             if ((e = launch_gemm(c, o, s)) != cudaSuccess) return e;
         }
 
-        if (!fused)
-            if ((e = launch_rmsnorm(c, c.h, W.ffn_norm, c.a, M, defer_o, s)) != cudaSuccess) return e;
+        if ((e = launch_rmsnorm(c, c.h, W.ffn_norm, c.a, M, defer_o, s)) != cudaSuccess) return e;
         GemmArgs gu{};
         gu.x = c.a; gu.M = M; gu.N = f.ffn; gu.Kd = f.hidden; gu.w[0] = W.w_gate; gu.w[1] = W.w_up;
         gu.wrows[0] = gu.wrows[1] = f.ffn; gu.epi = EPI_SWIGLU; gu.act = c.act;
-        gu.row_scale = fused ? c.inv : nullptr;
         {
             ProbeScope ps(c, 0, l, view, s);
             if ((e = launch_gemm(c, gu, s)) != cudaSuccess) return e;
@@ -326,15 +299,13 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
         GemmArgs dn{};
         dn.x = c.act; dn.M = M; dn.N = f.hidden; dn.Kd = f.ffn; dn.w[0] = W.w_down; dn.wrows[0] = f.hidden;
         dn.epi = EPI_RESID; dn.resid = c.h; dn.defer = defer_dn; dn.rpart = c.resid_part; dn.rpart_rows = c.Rw;
-        if (l + 1 < f.n_layers) fold(dn, c.layers[l + 1].attn_norm, c.a, c.inv);
-        else fold(dn, fin ? c.final_norm : nullptr, fin, inv_fin);   // no final norm without a head to feed
         {
             ProbeScope ps(c, 0, l, view, s);
             if ((e = launch_gemm(c, dn, s)) != cudaSuccess) return e;
         }
-        pending = fused ? 0 : defer_dn;
+        pending = defer_dn;
     }
-    if (fin && !fused) return launch_rmsnorm(c, c.h, c.final_norm, fin, M, pending, s);
+    if (fin) return launch_rmsnorm(c, c.h, c.final_norm, fin, M, pending, s);
     return cudaSuccess;
 }
 
@@ -342,8 +313,6 @@ static cudaError_t lm_head(Ctx &c, const void *fin, int B, int K, int lm_mode, f
                            const int64_t *step, const int32_t *given, cudaStream_t s, int draft_pass = 0)
 {
     GemmArgs g{};
-    // the final norm's 1/rms of each row, when it was fused into the last down projection
-    g.row_scale = c.fused_norm ? (fin == c.fin_draft ? c.inv_fin[1] : c.inv_fin[0]) : nullptr;
     g.draft_pass = draft_pass;
     g.x = fin; g.M = B * K; g.N = c.cfg.vocab; g.Kd = c.cfg.hidden; g.w[0] = c.lm_head; g.wrows[0] = c.cfg.vocab;
     g.epi = EPI_LMHEAD; g.lm = c.lm_part; g.inv_temp = temperature > 0.f ? 1.0f / temperature : 0.f;
@@ -827,8 +796,7 @@ orthrus_status_t orthrus_debug_logits(orthrus_ctx_t *c, int32_t which, int32_t b
 {
     if (!c || !logits || (which != 0 && which != 1) || batch < 1 || K < 1) return ORTHRUS_ERR_INVALID_ARG;
     if (batch * K > c->R) return ORTHRUS_ERR_CAPACITY;
-    CK(launch_logits_dump(*c, which ? c->fin_draft : c->fin_verify,
-                          c->fused_norm ? c->inv_fin[which ? 1 : 0] : nullptr, batch * K, logits, (cudaStream_t)stream));
+    CK(launch_logits_dump(*c, which ? c->fin_draft : c->fin_verify, batch * K, logits, (cudaStream_t)stream));
     return ORTHRUS_OK;
 }
 

@@ -241,8 +241,6 @@ struct CommitArgs {
     int *any_reject;
     const void *fin_verify, *fin_draft;
     void *res_x;
-    const float *inv_verify, *inv_draft;   // fused final norm: 1/rms of the fin rows (null: not fused)
-    float *res_inv;
     int d, esize;
     int32_t *n_out, *tokens_out, *anchor_io, *seq_lens;
     int32_t *append_out, *produced;
@@ -286,10 +284,6 @@ __global__ void commit_decide_kernel(CommitArgs a)
         const char *sd = (const char *)a.fin_draft + (size_t)(b * a.K + s_j) * bytes;
         char *dv = (char *)a.res_x + (size_t)(2 * b) * bytes;
         for (size_t i = threadIdx.x; i < bytes; i += blockDim.x) { dv[i] = sv[i]; dv[bytes + i] = sd[i]; }
-        if (a.inv_verify && threadIdx.x == 0) {
-            a.res_inv[2 * b] = a.inv_verify[b * a.K + s_j];
-            a.res_inv[2 * b + 1] = a.inv_draft[b * a.K + s_j];
-        }
     }
 }
 
@@ -534,8 +528,6 @@ static CommitArgs commit_args(const Ctx &c, const orthrus_kv_t &kv, int B, int K
     a.draft = c.draft; a.g = c.g; a.res_tok = c.res_tok; a.logp = c.logp; a.logq = c.logq;
     a.rej_row = c.rej_row; a.any_reject = c.any_reject;
     a.fin_verify = c.fin_verify; a.fin_draft = c.fin_draft; a.res_x = c.res_x;
-    a.inv_verify = c.fused_norm ? c.inv_fin[0] : nullptr; a.inv_draft = c.fused_norm ? c.inv_fin[1] : nullptr;
-    a.res_inv = c.res_inv;
     a.d = c.cfg.hidden; a.esize = c.esize;
     a.n_out = n_out; a.tokens_out = tokens_out; a.anchor_io = anchor_io; a.seq_lens = kv.seq_lens;
     a.append_out = append_out; a.produced = c.produced; a.append_stride = append_stride; a.append_max = append_max;
@@ -561,7 +553,6 @@ cudaError_t launch_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int K, fl
         g.x = c.res_x; g.M = 2 * B; g.N = c.cfg.vocab; g.Kd = c.cfg.hidden;
         g.w[0] = c.lm_head; g.wrows[0] = c.cfg.vocab;
         g.epi = EPI_RESAMPLE; g.lm = c.lm_part; g.inv_temp = 1.0f / temperature; g.seed = seed; g.step = step;
-        g.row_scale = c.fused_norm ? c.res_inv : nullptr;
         g.lse_p = c.lse_p; g.lse_q = c.lse_q; g.rej_row = c.rej_row; g.any_flag = c.any_reject; g.K = K;
         e = launch_gemm(c, g, s);
         if (e != cudaSuccess) return e;
@@ -634,11 +625,9 @@ cudaError_t launch_kl_lm_head(const Ctx &c, const void *h_a, const void *h_d, in
     return launch_k(kl_finalize_kernel, (rows + 7) / 8, 256, 0, s, k);
 }
 
-cudaError_t launch_logits_dump(const Ctx &c, const void *fin, const float *row_scale, int M, float *logits,
-                               cudaStream_t s)
+cudaError_t launch_logits_dump(const Ctx &c, const void *fin, int M, float *logits, cudaStream_t s)
 {
     GemmArgs g{};
-    g.row_scale = row_scale;
     g.x = fin; g.M = M; g.N = c.cfg.vocab; g.Kd = c.cfg.hidden;
     g.w[0] = c.lm_head; g.wrows[0] = c.cfg.vocab;
     g.epi = EPI_LOGITS; g.logits = logits;

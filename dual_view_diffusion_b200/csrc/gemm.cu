@@ -157,9 +157,7 @@ cudaError_t launch_gemm(const Ctx &c, GemmArgs a, cudaStream_t s)
         const cudaError_t e = launch_gemm_tc(c, t, n_mt_tc, tm, n_nt, s);
         if (e != cudaErrorNotSupported) return e;
     }
-    // only the tensor-core kernel defers residual segments and scales rows by
-    // a fused norm's 1/rms: never fall back to the SIMT kernel with them
-    if (a.defer > 0 || a.row_scale || a.norm_cnt) return cudaErrorInvalidValue;
+    if (a.defer > 0) return cudaErrorInvalidValue;   // only the tensor-core kernel defers
     a.splits = 1;
     const long units = (long)n_mt * n_nt;
     const int grid = (int)(units < kNumSMs ? units : kNumSMs);

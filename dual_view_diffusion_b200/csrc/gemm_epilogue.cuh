@@ -156,94 +156,6 @@ __device__ void epilogue_prepare(const GemmArgs &a, EpiPre &pre, int mt, int nt,
     }
 }
 
-// Fused residual fold and RMSNorm, run by the last of the a.defer segment
-// writers of the (32-row tile mt, n tile nt) of a deferred EPI_RESID GEMM
-// (the caller has seen the tile's arrival counter reach a.defer - 1 and
-// fenced): h += segments 0 .. defer-1 in segment order (the order the
-// unfused RMSNorm kernel folds them in), then, with a norm gain, the bf16
-// operand x = h * gain of the next projection and each row's sum of squares
-// over the tile's 128 columns; the last n tile of the 32-row tile to finish
-// sums those partials in n-tile order into inv = 1/sqrt(mean(h^2) + eps).
-// The next projection scales its accumulator rows by inv, so the normalised
-// operand RMSNorm(h) = inv * (h * gain) never has to be formed: y = inv *
-// ((h * gain) . W^T).  flag: a shared int the 128 threads use to agree on
-// the row-tile ticket.
-template <class Sync>
-__device__ void resid_fold_norm(const GemmArgs &a, int mt, int nt, int n_nt, int tid, Sync sync, int *flag)
-{
-    const int S = a.defer;
-    float4 v[kEpiVec];
-    bool ok[kEpiVec];
-#pragma unroll
-    for (int j = 0; j < kEpiVec; ++j) {
-        const int c = tid + j * kEpiThreads, m = c >> 5, n = nt * kTileN + (c & 31) * 4, row = mt * kTileM + m;
-        ok[j] = row < a.M && n < a.N;
-        v[j] = ok[j] ? __ldcg((const float4 *)&a.resid[(size_t)row * a.N + n]) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    // segments two at a time, every load of a pair in flight before its adds
-    for (int s0 = 0; s0 < S; s0 += 2) {
-        float4 u[2][kEpiVec];
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl)
-#pragma unroll
-            for (int j = 0; j < kEpiVec; ++j) {
-                const int c = tid + j * kEpiThreads, m = c >> 5, n = nt * kTileN + (c & 31) * 4, row = mt * kTileM + m;
-                u[sl][j] = (s0 + sl < S && ok[j])
-                               ? __ldcg((const float4 *)(a.rpart + ((size_t)(s0 + sl) * a.rpart_rows + row) * a.N + n))
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-            if (s0 + sl >= S) break;
-#pragma unroll
-            for (int j = 0; j < kEpiVec; ++j) {
-                v[j].x += u[sl][j].x; v[j].y += u[sl][j].y; v[j].z += u[sl][j].z; v[j].w += u[sl][j].w;
-            }
-        }
-    }
-    const int lane = tid & 31;
-#pragma unroll
-    for (int j = 0; j < kEpiVec; ++j) {
-        const int c = tid + j * kEpiThreads, m = c >> 5, n = nt * kTileN + (c & 31) * 4, row = mt * kTileM + m;
-        if (ok[j]) __stcg((float4 *)&a.resid[(size_t)row * a.N + n], v[j]);
-        if (a.norm_gain) {
-            if (ok[j]) {
-                const bf16 *g = (const bf16 *)a.norm_gain + n;
-                const __nv_bfloat162 g01 = *(const __nv_bfloat162 *)g, g23 = *(const __nv_bfloat162 *)(g + 2);
-                const float2 f01 = __bfloat1622float2(g01), f23 = __bfloat1622float2(g23);
-                const __nv_bfloat162 lo = __floats2bfloat162_rn(v[j].x * f01.x, v[j].y * f01.y);
-                const __nv_bfloat162 hi = __floats2bfloat162_rn(v[j].z * f23.x, v[j].w * f23.y);
-                uint2 o;
-                o.x = *(const uint32_t *)&lo;
-                o.y = *(const uint32_t *)&hi;
-                __stcg((uint2 *)((bf16 *)a.norm_x + (size_t)row * a.N + n), o);
-            }
-            // warp w holds rows w, w + 4, ...: one row's 128 columns per j
-            float ss = ok[j] ? fmaf(v[j].x, v[j].x, fmaf(v[j].y, v[j].y, fmaf(v[j].z, v[j].z, v[j].w * v[j].w))) : 0.f;
-            ss = warp_sum(ss);
-            if (lane == 0 && row < a.M) __stcg(a.norm_ss + (size_t)row * n_nt + nt, ss);
-        }
-    }
-    // ready for the next launch: this tile's arrivals are all in
-    if (tid == 0) a.norm_cnt[(size_t)mt * n_nt + nt] = 0;
-    if (!a.norm_gain) return;
-    __threadfence();
-    sync();
-    if (tid == 0) *flag = atomicAdd(a.norm_cnt + a.norm_cnt_tiles + mt, 1);
-    sync();
-    if (*flag != n_nt - 1) return;
-    __threadfence();
-    if (tid < kTileM) {   // the last n tile of this 32-row tile: every row's 1/rms
-        const int row = mt * kTileM + tid;
-        if (row < a.M) {
-            float ss = 0.f;
-            for (int t = 0; t < n_nt; ++t) ss += __ldcg(a.norm_ss + (size_t)row * n_nt + t);
-            a.norm_inv[row] = 1.0f / sqrtf(ss / a.N + a.norm_eps);
-        }
-    }
-    if (tid == 0) a.norm_cnt[a.norm_cnt_tiles + mt] = 0;
-}
-
 // pre: filled by epilogue_prepare for this tile (and made visible with a
 // barrier), or null to fetch everything here.
 // bf16 outputs: the same reduction, then the MUFU sine / cosine (absolute

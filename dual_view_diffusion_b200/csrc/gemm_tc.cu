@@ -527,7 +527,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                         asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n"
                                      ::"r"(tc_mapa(smem_u32(&sm.peer_empty), (uint32_t)et)) : "memory");
                 }
-                if (defer) {   // this segment of the residual update, summed later in segment order
+                if (defer) {   // this segment of the residual update, summed later by the RMSNorm
 #pragma unroll
                     for (int j = 0; j < kEpiVec; ++j) {
                         const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4;
@@ -535,17 +535,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                         if (row < a.M && n < a.N)
                             __stcg((float4 *)(a.rpart + ((size_t)s.seg * a.rpart_rows + row) * a.N + n),
                                    *(const float4 *)&sm.tile[m][c4]);
-                    }
-                    if (a.norm_cnt) {   // the last segment of this tile to arrive folds it (and normalises)
-                        __threadfence();
-                        SyncEpilogue{}();
-                        if (et == 0) sm.s_last = atomicAdd(a.norm_cnt + (size_t)mt32 * n_nt_epi + s.nt, 1);
-                        SyncEpilogue{}();
-                        if (sm.s_last == a.defer - 1) {
-                            __threadfence();
-                            resid_fold_norm(a, mt32, s.nt, n_nt_epi, et, SyncEpilogue{}, &sm.s_last);
-                        }
-                        SyncEpilogue{}();
                     }
                     continue;
                 }
@@ -570,16 +559,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                 }
                 if (ch > 0 && !defer && s.seg == 0) {   // chunk 0's was fetched while the chunks streamed
                     epilogue_prepare<bf16, E>(a, sm.pre, mt32, s.nt, et);
-                    SyncEpilogue{}();
-                }
-                if (a.row_scale) {   // a fused RMSNorm's 1/rms of each token row
-#pragma unroll
-                    for (int j = 0; j < kEpiVec; ++j) {
-                        const int c = et + j * kEpiThreads, m = c >> 5, c4 = (c & 31) * 4, row = mt32 * kTileM + m;
-                        const float sc = row < a.M ? __ldcg(a.row_scale + row) : 0.f;
-                        float4 &o = *(float4 *)&sm.tile[m][c4];
-                        o.x *= sc; o.y *= sc; o.z *= sc; o.w *= sc;
-                    }
                     SyncEpilogue{}();
                 }
                 epilogue<bf16, SyncEpilogue, E>(a, sm.tile, mt32, s.nt, n_nt_epi, et, SyncEpilogue{}, &sm.pre);

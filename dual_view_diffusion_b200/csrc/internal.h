@@ -112,25 +112,6 @@ struct GemmArgs {
     const int *any_flag;     // EPI_RESAMPLE: skip everything when 0
     float *logits;           // EPI_LOGITS: [M][N] fp32
     KlPart *kl;              // EPI_KL: [M / 2][n_vtiles]
-    // Fused residual fold and RMSNorm (EPI_RESID with defer > 0, tensor-core
-    // path, norm_cnt non-null): the last of the defer segments of a (32-row
-    // tile, n tile) to arrive adds h and the segments in segment order into
-    // h, writes norm_x = bf16(h * norm_gain) (norm_gain non-null) and each
-    // row's sum of squares over the tile's columns to norm_ss; the last n
-    // tile of a 32-row tile to arrive turns those into norm_inv[row] =
-    // 1/sqrt(mean(h^2) + norm_eps).  Counters: norm_cnt[mt32 * n_nt + nt]
-    // per tile, then norm_cnt[n_mt32 * n_nt + mt32] per 32-row tile, zero
-    // between launches (each last arriver resets its own).
-    const void *norm_gain;
-    void *norm_x;            // [M][N] bf16
-    float *norm_inv;         // [M]
-    float *norm_ss;          // [M][n_nt]
-    int *norm_cnt;
-    int norm_cnt_tiles;      // n_mt32 * n_nt: offset of the per-row-tile counters
-    float norm_eps;
-    // consumers of a fused norm: accumulator row r is multiplied by
-    // row_scale[r] before the epilogue (null: no scaling)
-    const float *row_scale;
 };
 
 struct AttnArgs {
@@ -243,14 +224,6 @@ struct Ctx {
     int32_t *draft;          // [R]
     float *logq, *lse_q;     // [R]
     float *ent;              // [R] entropy of each draft row's distribution
-    // fused residual + RMSNorm (tensor-core path): per-row 1/rms of c.a
-    // (inv), of the two views' final-normed rows (inv_fin[0] verify, [1]
-    // draft), of the residual-draw rows (res_inv); partial sums of squares
-    // and arrival counters of the folding GEMMs
-    bool fused_norm;
-    float *inv, *inv_fin[2], *res_inv;   // [Rw], [R] x 2, [2 * max_batch]
-    float *norm_ss;          // [Rw][ceil(hidden / 128)]
-    int *norm_cnt;           // [Rw / 32][ceil(hidden / 128) + 1]
     int32_t *g;              // [R]
     float *logp, *lse_p;     // [R]
     int32_t *rej_row;        // [max_batch]
@@ -331,8 +304,7 @@ cudaError_t launch_set_lens(const Ctx &c, int32_t *seq_lens, int b, int value, i
                             const int32_t *tokens, cudaStream_t s);
 cudaError_t launch_pack_block(const Ctx &c, const void *k_src, const void *v_src, void *k_dst, void *v_dst, int B,
                               int K, int kp, cudaStream_t s);
-cudaError_t launch_logits_dump(const Ctx &c, const void *fin, const float *row_scale, int M, float *logits,
-                               cudaStream_t s);
+cudaError_t launch_logits_dump(const Ctx &c, const void *fin, int M, float *logits, cudaStream_t s);
 // Tree verification (tree.cu): the draft tree's builder and its commit.
 struct TreeBuildArgs {   // one best-first tree per sequence
     const int32_t *ids;      // [B][D][W] candidate ids, best first
