@@ -72,14 +72,14 @@ constexpr size_t kTcRingOffset = (sizeof(TcSmem) + 1023) / 1024 * 1024;
 
 // Ring stages for token tiles of tm rows: as many as fit beside the fixed
 // part, at most kTcStages.
-__host__ __device__ inline int tc_stages(int tm)
+__host__ __device__ constexpr int tc_stages(int tm)
 {
     const size_t per = kStageWBytes + (size_t)tm * kTileK * 2;
     const size_t n = (kTcSmemBudget - 1024 - kTcRingOffset) / per;
     return (int)(n < (size_t)kTcStages ? n : (size_t)kTcStages);
 }
 // TMEM columns of the two accumulators (a power of two, at least 32)
-__host__ __device__ inline uint32_t tc_tmem_cols(int tm)
+__host__ __device__ constexpr uint32_t tc_tmem_cols(int tm)
 {
     uint32_t c = 32;
     while (c < 2u * (uint32_t)tm) c <<= 1;
@@ -291,7 +291,11 @@ __device__ __forceinline__ bool flag_wait(const int *f, volatile int *abort)
     return false;
 }
 
-template <int E>   // the epilogue (Epi), fixed at compile time
+// E: the epilogue (Epi), fixed at compile time.  TMF: the token tile's rows
+// when fixed at compile time (32: one token tile of a decode step at batch
+// 1, where the ring and the chunk loop fold to constants), or 0 for a tile
+// size taken from sk.tm.
+template <int E, int TMF>
 __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_constant__ TcMaps maps, GemmArgs a,
                                                                  SkShape sk)
 {
@@ -304,7 +308,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
-    const int tm = sk.tm, nch = tm / kTileM, stages = sk.stages;
+    const int tm = TMF ? TMF : sk.tm, nch = tm / kTileM, stages = TMF ? tc_stages(TMF) : sk.stages;
     const uint32_t xbytes = (uint32_t)tm * kTileK * 2;
     unsigned char *ring_w = base + kTcRingOffset, *ring_x = ring_w + (size_t)stages * kStageWBytes;
     const uint32_t tcols = tc_tmem_cols(tm);
@@ -640,7 +644,18 @@ void gemm_token_tile(int M, int *n_mt, int *tm)
 
 template <int E> static cudaError_t set_smem()
 {
-    return cudaFuncSetAttribute(gemm_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBudget);
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<E, kTileM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kTcSmemBudget);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(gemm_tc_kernel<E, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBudget);
+}
+
+template <int E>
+static cudaError_t launch_tc_e(int G, size_t smem, cudaStream_t s, const TcMaps &maps, const GemmArgs &a,
+                               const SkShape &k)
+{
+    if (k.tm == kTileM) return launch_k(gemm_tc_kernel<E, kTileM>, G, kTcThreads, smem, s, maps, a, k);
+    return launch_k(gemm_tc_kernel<E, 0>, G, kTcThreads, smem, s, maps, a, k);
 }
 
 cudaError_t gemm_tc_init_attributes()
@@ -722,17 +737,18 @@ cudaError_t launch_gemm_tc(const Ctx &c, const GemmArgs &a, int n_mt, int tm, in
         cfg.attrs = attr;
         cfg.numAttrs = 2;
         c.launches += 1;
-        return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_QKV>, maps, a, k);
+        if (tm == kTileM) return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_QKV, kTileM>, maps, a, k);
+        return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_QKV, 0>, maps, a, k);
     }
     c.launches += 1;
     switch (a.epi) {
-    case EPI_QKV: return launch_k(gemm_tc_kernel<EPI_QKV>, k.G, kTcThreads, smem, s, maps, a, k);
-    case EPI_RESID: return launch_k(gemm_tc_kernel<EPI_RESID>, k.G, kTcThreads, smem, s, maps, a, k);
-    case EPI_SWIGLU: return launch_k(gemm_tc_kernel<EPI_SWIGLU>, k.G, kTcThreads, smem, s, maps, a, k);
-    case EPI_LMHEAD: return launch_k(gemm_tc_kernel<EPI_LMHEAD>, k.G, kTcThreads, smem, s, maps, a, k);
-    case EPI_RESAMPLE: return launch_k(gemm_tc_kernel<EPI_RESAMPLE>, k.G, kTcThreads, smem, s, maps, a, k);
-    case EPI_LOGITS: return launch_k(gemm_tc_kernel<EPI_LOGITS>, k.G, kTcThreads, smem, s, maps, a, k);
-    case EPI_KL: return launch_k(gemm_tc_kernel<EPI_KL>, k.G, kTcThreads, smem, s, maps, a, k);
+    case EPI_QKV: return launch_tc_e<EPI_QKV>(k.G, smem, s, maps, a, k);
+    case EPI_RESID: return launch_tc_e<EPI_RESID>(k.G, smem, s, maps, a, k);
+    case EPI_SWIGLU: return launch_tc_e<EPI_SWIGLU>(k.G, smem, s, maps, a, k);
+    case EPI_LMHEAD: return launch_tc_e<EPI_LMHEAD>(k.G, smem, s, maps, a, k);
+    case EPI_RESAMPLE: return launch_tc_e<EPI_RESAMPLE>(k.G, smem, s, maps, a, k);
+    case EPI_LOGITS: return launch_tc_e<EPI_LOGITS>(k.G, smem, s, maps, a, k);
+    case EPI_KL: return launch_tc_e<EPI_KL>(k.G, smem, s, maps, a, k);
     default: return cudaErrorNotSupported;
     }
 }
