@@ -171,6 +171,39 @@ def test_bf16_logits_vs_oracle_ragged(pkg):
     assert ed <= 2e-2 and ev <= 2e-2, (ed, ev)
 
 
+def test_bf16_logits_vs_oracle_full_depth_1p7b(pkg):
+    """The whole 28-layer Qwen3-1.7B shape (tied head, 151936 ids): the draft
+    and verify logits of two decode cycles against the fp64 oracle at the
+    same positions, within 2e-2 of each row's largest |logit|; the oracle
+    follows the GPU's accepted tokens."""
+    s = synth.QWEN3_1_7B
+    w = synth.make_weights(s, 0)
+    K, P = 8, 64
+    eng = pkg.Engine(s, w, max_batch=1, max_block=K, max_seq=P + 4 * K, split_tokens=64)
+    prompt = synth.make_prompt(s, P, 6)
+    m = oracle.Model(w)
+    kc, vc = m.new_cache(P + 4 * K)
+    t = m.prefill(prompt, kc, vc)
+    anchor = eng.prefill(torch.from_numpy(prompt)[None])
+    a = int(prompt[-1])
+    rel = lambda g, r: float((np.abs(g - r).max(axis=1) / np.abs(r).max(axis=1)).max())
+    for _ in range(2):
+        draft = eng.draft_block(anchor, K)
+        dl = eng.debug_logits(1, 1, K)[0].cpu().numpy()
+        ref_d = m.forward(1, 1, [a] + [s.mask_id] * (K - 1), t, kc.copy(), vc.copy())
+        eng.verify_block(anchor, draft, K)
+        vl = eng.debug_logits(0, 1, K)[0].cpu().numpy()
+        ref_v = m.forward(0, 0, [a] + draft[0, :K - 1].cpu().tolist(), t, kc, vc)
+        assert rel(dl, ref_d) <= 2e-2 and rel(vl, ref_v) <= 2e-2, (rel(dl, ref_d), rel(vl, ref_v))
+        n, toks = eng.commit(anchor, K)
+        n = int(n[0])
+        t += n
+        a = int(toks[0, n - 1])
+    assert eng.check_error()[0] == 0
+    del eng, w
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("shape,P,N,split", [(synth.QWEN3_1_7B, 512, 256, 256), (synth.QWEN3_8B, 2048, 512, 128)])
 def test_bf16_orthrus_equals_plain_ar(pkg, shape, P, N, split):
     """Full-depth random-init Qwen3 shapes, K = 32, greedy: the Orthrus
