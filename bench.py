@@ -530,10 +530,10 @@ def decode_variants(eng, anchor, draft, toks, value, ms_step, steps=VARIANT_STEP
                 notes §4.3): draft samples, acceptance test, residual draw
       plain_ar  one AR forward per token (the same kernels, K = 1): the
                 baseline whose greedy stream Orthrus reproduces (§4.2)
-      tree      a tree-verified step (§7.5 / §9.6): draft, its rows' logits,
-                top-4 candidates per depth, a best-first tree of 31 nodes,
-                the tree-masked verify forward (32 rows, as the chain's) and
-                the walk plus K/V compaction
+      tree      a tree-verified step (§7.5 / §9.6): draft with the top-4
+                candidates of its rows from the LM-head pass, a best-first
+                tree of 31 nodes, the tree-masked verify forward (32 rows, as
+                the chain's) and the walk plus K/V compaction
       adaptive  the adaptive block length (§7.4 / §9.6, reading R23): the
                 verify length from the draft rows' entropies, threshold the
                 median entropy of a warm-up draft"""
@@ -571,14 +571,11 @@ def decode_variants(eng, anchor, draft, toks, value, ms_step, steps=VARIANT_STEP
                               "ratio uses the pages' 10.8 tokens per cycle"}
     # ---- tree-verified step (greedy)
     W, nodes, D = 4, K - 1, K - 1
-    zbuf = torch.empty((B, K, eng.shape.vocab), dtype=torch.float32, device=dev)
     n_t = torch.zeros((steps + 3, B), dtype=torch.int32, device=dev)
 
     def st_tree(j):
-        eng.draft_block(anchor, K, out=draft)
-        eng.debug_logits(1, B, K, out=zbuf)
-        ids, vals, lse = eng.tree_topw(zbuf[:, :D], W)
-        par, tk, _, _, nr = eng.tree_build(ids.view(B, D, W), vals.view(B, D, W), lse.view(B, D), nodes)
+        _, ids, vals, lse = eng.draft_block_topw(anchor, K, W, D, out=draft)
+        par, tk, _, _, nr = eng.tree_build(ids, vals, lse, nodes)
         g = eng.verify_tree(anchor, par, tk)
         n, _ = eng.tree_commit(par, tk, nr, g, anchor)
         n_t[j].copy_(n)
@@ -588,8 +585,8 @@ def decode_variants(eng, anchor, draft, toks, value, ms_step, steps=VARIANT_STEP
     tok = int(n_t[:steps].sum())
     out["tree"] = {"width": W, "nodes": nodes, "steps": steps, "ms_per_step": ms / steps,
                    "value": tok / (ms * 1e-3), "unit": UNIT, "mean_accepted_per_cycle": tok / (steps * B),
-                   "how": "draft, the draft rows' fp32 logits (one extra LM-head pass written to memory), top-W, "
-                          "best-first build, tree-masked verify forward, walk + K/V compaction; greedy"}
+                   "how": "draft with the top-W of its rows taken inside the LM-head pass, best-first build, "
+                          "tree-masked verify forward, walk + K/V compaction; greedy"}
     # ---- adaptive block length (greedy)
     kt = torch.empty(B, dtype=torch.int32, device=dev)
     eng.draft_block(anchor, K, out=draft)

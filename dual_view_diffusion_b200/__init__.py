@@ -89,6 +89,7 @@ _SIGS = {
     "orthrus_tree_build": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P],
     "orthrus_tree_commit": [_P, C.POINTER(KV), _I, _I, _P, _P, _P, _P, _P, _P, _P, _P],
     "orthrus_verify_tree": [_P, C.POINTER(KV), _P, _P, _P, _I, _I, _P, _P],
+    "orthrus_draft_block_topw": [_P, C.POINTER(KV), _P, _I, _I, _I, _I, _P, _P, _P, _P, _P],
     "orthrus_debug_logits": [_P, _I, _I, _I, _P, _P],
     "orthrus_debug_rows": [_P, _I, _I, _I, _P, _P, _P, _P],
     "orthrus_adaptive_len": [_P, _I, _I, C.c_float, _P, _P, _P],
@@ -272,6 +273,23 @@ class Engine:
                 self.ctx, C.byref(self.kv), _ptr(anchor), B, K, int(iterations), float(temperature), seed, _ptr(st),
                 _ptr(draft), _stream()))
         return draft
+
+    def draft_block_topw(self, anchor, K, width, depth=None, out=None):
+        """Greedy draft plus, for draft rows k < depth (default K - 1), the
+        `width` best ids and logits and each row's log-sum-exp, taken inside
+        the LM-head pass: (draft [B, K], ids [B, depth, width], vals, lse
+        [B, depth])."""
+        t = self.torch
+        B = anchor.numel()
+        depth = K - 1 if depth is None else depth
+        draft = out if out is not None else t.empty((B, K), dtype=t.int32, device=self.device)
+        ids = t.empty((B, depth, width), dtype=t.int32, device=self.device)
+        vals = t.empty((B, depth, width), dtype=t.float32, device=self.device)
+        lse = t.empty((B, depth), dtype=t.float32, device=self.device)
+        _check("orthrus_draft_block_topw", lib().orthrus_draft_block_topw(
+            self.ctx, C.byref(self.kv), _ptr(anchor), B, K, int(width), int(depth), _ptr(draft), _ptr(ids),
+            _ptr(vals), _ptr(lse), _stream()))
+        return draft, ids, vals, lse
 
     def verify_block(self, anchor, draft, K, temperature=0.0):
         B = anchor.numel()

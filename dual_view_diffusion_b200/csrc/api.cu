@@ -123,6 +123,7 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
     const size_t o_rp = take((size_t)rslots * Rw * d * 4);
     const size_t o_invf = take((size_t)c.head_dim / 2 * 8);
     const size_t o_lm = take(Rlm * n_vtiles * sizeof(LmPart));
+    const size_t o_top = take(R * n_vtiles * kTopWMax * sizeof(TopRec));
     const size_t o_tok = take(Rw * 4), o_pos = take(mb * 4), o_bt = take(mb * 4), o_pr = take(4);
     const size_t o_ttok = take(R * 4), o_tdep = take(R * 4), o_tmask = take(R * 16);
     const size_t o_bz = take(mb * 4);   // zeros, never written
@@ -141,7 +142,7 @@ size_t plan_workspace(const orthrus_config_t &c, Ctx *x)
         x->attn_xo = attn_x2 ? (float *)P(o_xo) : nullptr; x->attn_xml = attn_x2 ? (float2 *)P(o_xml) : nullptr;
         x->attn_xcnt = attn_x2 ? (int *)P(o_xc) : nullptr; x->attn_xz = attn_x2 ? kAttnMaxClusters : 1;
         x->gemm_part = (float *)P(o_gp); x->gemm_part_floats = gfloats; x->gemm_ticket = (int *)P(o_gt);
-        x->gemm_tickets = gtickets; x->lm_part = (LmPart *)P(o_lm);
+        x->gemm_tickets = gtickets; x->lm_part = (LmPart *)P(o_lm); x->top_part = (TopRec *)P(o_top);
         x->resid_part = (float *)P(o_rp);
         x->rope_invf = (double *)P(o_invf);
         x->tok = (int32_t *)P(o_tok); x->pos0 = (int32_t *)P(o_pos); x->bt_rows = (int32_t *)P(o_bt);
@@ -166,7 +167,7 @@ static void rebase(Ctx *x, char *ws)
     auto fix = [&](auto *&p) { p = (std::remove_reference_t<decltype(p)>)(ws + (size_t)(const char *)p); };
     fix(x->h); fix(x->a); fix(x->q); fix(x->attn_o); fix(x->act); fix(x->k_diff); fix(x->v_diff); fix(x->blk_pack);
     fix(x->fin_draft); fix(x->fin_verify); fix(x->res_x); fix(x->attn_part); fix(x->attn_ml); fix(x->gemm_part);
-    fix(x->gemm_ticket); fix(x->lm_part); fix(x->resid_part); fix(x->rope_invf); fix(x->tok); fix(x->pos0); fix(x->bt_rows); fix(x->bt_zero); fix(x->prefill_row);
+    fix(x->gemm_ticket); fix(x->lm_part); fix(x->top_part); fix(x->resid_part); fix(x->rope_invf); fix(x->tok); fix(x->pos0); fix(x->bt_rows); fix(x->bt_zero); fix(x->prefill_row);
     fix(x->tree_tok); fix(x->tree_depth); fix(x->tree_mask);
     fix(x->draft); fix(x->logq); fix(x->lse_q); fix(x->ent); fix(x->g); fix(x->logp); fix(x->lse_p); fix(x->rej_row);
     fix(x->res_tok); fix(x->any_reject); fix(x->err); fix(x->produced); fix(x->step); fix(x->n_buf);
@@ -310,9 +311,10 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
 }
 
 static cudaError_t lm_head(Ctx &c, const void *fin, int B, int K, int lm_mode, float temperature, uint64_t seed,
-                           const int64_t *step, const int32_t *given, cudaStream_t s, int draft_pass = 0)
+                           const int64_t *step, const int32_t *given, cudaStream_t s, int draft_pass = 0, int topw = 0)
 {
     GemmArgs g{};
+    g.topw = topw; g.top = c.top_part;
     g.draft_pass = draft_pass;
     g.x = fin; g.M = B * K; g.N = c.cfg.vocab; g.Kd = c.cfg.hidden; g.w[0] = c.lm_head; g.wrows[0] = c.cfg.vocab;
     g.epi = EPI_LMHEAD; g.lm = c.lm_part; g.inv_temp = temperature > 0.f ? 1.0f / temperature : 0.f;
@@ -486,6 +488,24 @@ orthrus_status_t orthrus_draft_block_iterative(orthrus_ctx_t *c, const orthrus_k
         CK(lm_head(*c, c->fin_draft, batch, K, 1, temperature, seed, step, nullptr, s, pass));
         CK(launch_lm_finalize_impl(*c, 1, batch, K, temperature, draft, nullptr, s));
     }
+    return ORTHRUS_OK;
+}
+
+orthrus_status_t orthrus_draft_block_topw(orthrus_ctx_t *c, const orthrus_kv_t *kv, const int32_t *anchor,
+                                          int32_t batch, int32_t K, int32_t width, int32_t depth, int32_t *draft,
+                                          int32_t *ids, float *vals, float *lse, void *stream)
+{
+    orthrus_status_t st = check_step(c, kv, batch, K);
+    if (st != ORTHRUS_OK) return st;
+    if (!anchor || !draft || !ids || !vals || !lse || width < 1 || width > kTopWMax || width > c->cfg.vocab ||
+        depth < 1 || depth > K)
+        return ORTHRUS_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    CK(launch_embed(*c, 0, nullptr, anchor, nullptr, batch, K, s));
+    CK(forward(*c, *kv, 1, batch, K, kv->seq_lens, c->bt_rows, c->fin_draft, s));
+    CK(lm_head(*c, c->fin_draft, batch, K, 1, 0.f, 0, nullptr, nullptr, s, 0, width));
+    CK(launch_lm_finalize_impl(*c, 1, batch, K, 0.f, draft, nullptr, s));
+    CK(launch_topw_finalize(*c, batch, K, depth, width, ids, vals, lse, s));
     return ORTHRUS_OK;
 }
 

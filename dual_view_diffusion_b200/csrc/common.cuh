@@ -3,6 +3,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <limits.h>
 #include <stdint.h>
 
 #include "../../include/orthrus.h"
@@ -90,6 +91,61 @@ __device__ __forceinline__ void warp_argmax(float &v, int &i)
         const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
         const int i2 = __shfl_xor_sync(0xffffffffu, i, o);
         argmax_merge(v, i, v2, i2);
+    }
+}
+
+// ---------------------------------------------------------------- top-W lists
+// Sorted (best first) lists of the kTopWMax largest (value, id) pairs; ties
+// go to the lowest id.  Unused entries hold (-inf, INT_MAX).
+constexpr int kTopWMax = 8;
+
+__device__ __forceinline__ bool tw_better(float va, int ia, float vb, int ib)
+{
+    return va > vb || (va == vb && ia < ib);
+}
+
+// One lane's sorted list (best first) gives up its head.
+__device__ __forceinline__ void tw_pop(float (&v)[kTopWMax], int (&i)[kTopWMax])
+{
+#pragma unroll
+    for (int j = 0; j + 1 < kTopWMax; ++j) { v[j] = v[j + 1]; i[j] = i[j + 1]; }
+    v[kTopWMax - 1] = -INFINITY;
+    i[kTopWMax - 1] = INT_MAX;
+}
+
+// The warp's kTopWMax best entries over all lanes' sorted lists, best
+// first, into ov/oi (every lane gets the same result).  Ids are distinct
+// across lanes, so the winner of a round is one lane.
+__device__ __forceinline__ void tw_warp_merge(float (&v)[kTopWMax], int (&i)[kTopWMax], float *ov, int *oi)
+{
+#pragma unroll 1
+    for (int r = 0; r < kTopWMax; ++r) {
+        float bv = v[0];
+        int bi = i[0];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov2 = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi2 = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (tw_better(ov2, oi2, bv, bi)) { bv = ov2; bi = oi2; }
+        }
+        if (i[0] == bi && bi != INT_MAX) tw_pop(v, i);
+        ov[r] = bv;
+        oi[r] = bi;
+    }
+}
+
+// A logit into a thread's sorted top list (the common case is one compare).
+__device__ __forceinline__ void tw_insert(float x, int v, float (&tv)[kTopWMax], int (&ti)[kTopWMax])
+{
+    if (tw_better(x, v, tv[kTopWMax - 1], ti[kTopWMax - 1])) {
+        tv[kTopWMax - 1] = x;
+        ti[kTopWMax - 1] = v;
+#pragma unroll
+        for (int j = kTopWMax - 1; j > 0; --j)
+            if (tw_better(tv[j], ti[j], tv[j - 1], ti[j - 1])) {
+                const float a = tv[j]; tv[j] = tv[j - 1]; tv[j - 1] = a;
+                const int b = ti[j]; ti[j] = ti[j - 1]; ti[j - 1] = b;
+            }
     }
 }
 

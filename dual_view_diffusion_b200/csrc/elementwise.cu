@@ -227,6 +227,44 @@ __global__ void __launch_bounds__(256) lm_finalize_kernel(LmArgs a)
     }
 }
 
+// The draft rows' top-W candidates (tree verification) from the LM-head
+// epilogue's per-tile records: one warp per (sequence, row < depth), each
+// lane a sorted top-W of the tiles it scans, merged across the warp (ties
+// to the lowest id), with the row's log-sum-exp (T = 1: the draft is
+// greedy).
+__global__ void __launch_bounds__(256) topw_finalize_kernel(const TopRec *top, const float *lse_q, int n_vtiles, int B,
+                                                            int K, int depth, int W, int32_t *ids, float *vals,
+                                                            float *lse)
+{
+    pdl_trigger();
+    pdl_wait();
+    const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (w >= B * depth) return;
+    const int b = w / depth, k = w % depth, row = b * K + k;
+    float tv[kTopWMax];
+    int ti[kTopWMax];
+#pragma unroll
+    for (int j = 0; j < kTopWMax; ++j) { tv[j] = -INFINITY; ti[j] = INT_MAX; }
+    for (int t = lane; t < n_vtiles; t += 32) {
+        const TopRec *p = top + ((size_t)row * n_vtiles + t) * kTopWMax;
+        for (int r = 0; r < W; ++r) {
+            const TopRec q = p[r];
+            if (!tw_better(q.z, q.id, tv[kTopWMax - 1], ti[kTopWMax - 1])) break;   // the tile's list is sorted
+            tw_insert(q.z, q.id, tv, ti);
+        }
+    }
+    float ov[kTopWMax];
+    int oi[kTopWMax];
+    tw_warp_merge(tv, ti, ov, oi);
+    if (lane == 0) {
+        for (int r = 0; r < W; ++r) {
+            ids[(size_t)w * W + r] = oi[r];
+            vals[(size_t)w * W + r] = ov[r];
+        }
+        lse[w] = lse_q[row];
+    }
+}
+
 // ---------------------------------------------------------------- commit
 struct CommitArgs {
     int B, K;
@@ -516,6 +554,14 @@ cudaError_t launch_lm_finalize(const Ctx &c, int mode, int B, int K, float tempe
                                int32_t *tok_out, cudaStream_t s)
 {
     return launch_lm_finalize_impl(c, mode, B, K, temperature, tok_out, mode == 0 ? tok_out : nullptr, s);
+}
+
+cudaError_t launch_topw_finalize(const Ctx &c, int B, int K, int depth, int W, int32_t *ids, float *vals, float *lse,
+                                 cudaStream_t s)
+{
+    c.launches += 1;
+    return launch_k(topw_finalize_kernel, (B * depth + 7) / 8, 256, 0, s, (const TopRec *)c.top_part,
+                    (const float *)c.lse_q, c.n_vtiles, B, K, depth, W, ids, vals, lse);
 }
 
 static CommitArgs commit_args(const Ctx &c, const orthrus_kv_t &kv, int B, int K, float temperature, uint64_t seed,

@@ -419,6 +419,40 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
                 }
             s = warp_sum(s);
             if (a.lm_mode == 1) ez = warp_sum(ez);
+            if (a.topw > 0) {   // this tile's topw best (z, id), best first, ties to the lowest id
+                float tv[4];
+                int ti[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int v = nt * kTileN + lane * 4 + j;
+                    tv[j] = v < a.N ? zv[j] : -INFINITY;
+                    ti[j] = v < a.N ? v : INT_MAX;
+                }
+#pragma unroll
+                for (int i = 0; i < 3; ++i)   // a lane's four, sorted
+#pragma unroll
+                    for (int j = 0; j < 3 - i; ++j)
+                        if (tw_better(tv[j + 1], ti[j + 1], tv[j], ti[j])) {
+                            const float x = tv[j]; tv[j] = tv[j + 1]; tv[j + 1] = x;
+                            const int y = ti[j]; ti[j] = ti[j + 1]; ti[j + 1] = y;
+                        }
+                TopRec *out = a.top + ((size_t)row * n_nt + nt) * kTopWMax;
+                for (int r = 0; r < a.topw; ++r) {
+                    float bv = tv[0];
+                    int bi = ti[0];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                        if (tw_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+                    }
+                    if (ti[0] == bi && bi != INT_MAX) {   // the owning lane gives up its head
+                        tv[0] = tv[1]; tv[1] = tv[2]; tv[2] = tv[3]; tv[3] = -INFINITY;
+                        ti[0] = ti[1]; ti[1] = ti[2]; ti[2] = ti[3]; ti[3] = INT_MAX;
+                    }
+                    if (lane == 0) out[r] = TopRec{bv, bi};
+                }
+            }
             // the id's logit lives in exactly one lane (or none)
             const unsigned has = __ballot_sync(0xffffffffu, !isnan(zid));
             if (has) zid = __shfl_sync(0xffffffffu, zid, __ffs(has) - 1);

@@ -38,6 +38,13 @@ struct LmPart {
     float zez;    // draft rows: sum over the tile of exp((z - zmax) / T) * z (the entropy's mean logit)
 };
 
+// One of the kTopWMax best logits of a (row, vocab tile), for the draft's
+// top-W candidates (tree verification).
+struct TopRec {
+    float z;
+    int id;
+};
+
 // Per-(row pair, vocab tile) record of the fused forward-KL epilogue: rows
 // 2i (AR view) and 2i+1 (diffusion view) of the same position.
 struct KlPart {
@@ -106,6 +113,8 @@ struct GemmArgs {
     const int64_t *step;
     int lm_mode;             // 0 verify (zid from given ids), 1 draft (Gumbel), 2 AR sample
     int draft_pass;          // lm_mode 1: pass of an iterative draft (Gumbel purpose DRAFT | pass << 8)
+    int topw;                // lm_mode 1: keep each (row, tile)'s topw best logits in top (0: off)
+    TopRec *top;             // [M][n_vtiles][kTopWMax]
     const int32_t *given;    // [M] id whose logit is wanted (verify), or null
     const float *lse_p, *lse_q;   // EPI_RESAMPLE: per (b, k) row
     const int32_t *rej_row;  // EPI_RESAMPLE: [batch] j or -1
@@ -214,6 +223,7 @@ struct Ctx {
     float *resid_part;       // [kResidSlots][Rw][hidden] deferred residual segments
     double *rope_invf;       // [head_dim / 2] rotary inverse frequencies
     LmPart *lm_part;         // [max(R, 2*max_batch)][n_vtiles]
+    TopRec *top_part;        // [R][n_vtiles][kTopWMax] the draft rows' per-tile top-W
     int32_t *tok;            // [Rw] block tokens
     int32_t *tree_tok, *tree_depth;   // [R] tree verify: row tokens and depths
     uint32_t *tree_mask;     // [R][4] tree verify: ancestor bit masks
@@ -292,6 +302,10 @@ cudaError_t launch_rmsnorm(const Ctx &c, float *h, const void *gain, void *out, 
 int resid_defer_slots(const orthrus_config_t &cfg, int N, int Kd);
 cudaError_t launch_lm_finalize(const Ctx &c, int mode, int B, int K, float temperature, uint64_t seed,
                                const int64_t *step, int32_t *tok_out, cudaStream_t s);
+// The draft rows' top-W from the per-tile records: rows k < depth of each
+// sequence to ids / vals [B][depth][W] and their log-sum-exps to lse [B][depth].
+cudaError_t launch_topw_finalize(const Ctx &c, int B, int K, int depth, int W, int32_t *ids, float *vals, float *lse,
+                                 cudaStream_t s);
 cudaError_t launch_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int K, float temperature, uint64_t seed,
                           int64_t *step, const int32_t *force_n, int32_t *n_out, int32_t *tokens_out,
                           int32_t *anchor_io, int32_t *append_out, int append_stride, int append_max,

@@ -20,60 +20,10 @@
 
 namespace orthrus {
 
-constexpr int kTreeMaxW = 8;        // candidates per depth
+constexpr int kTreeMaxW = kTopWMax;   // candidates per depth
 constexpr int kTreeMaxRows = 128;   // rows of one tree (root + nodes)
 constexpr int kTreeTopwThreads = 256;
 constexpr int kTreeTopwSplit = 8;     // CTAs (one cluster) per logits row
-
-__device__ __forceinline__ bool tw_better(float va, int ia, float vb, int ib)
-{
-    return va > vb || (va == vb && ia < ib);
-}
-
-// One lane's sorted list (best first) gives up its head.
-__device__ __forceinline__ void tw_pop(float (&v)[kTreeMaxW], int (&i)[kTreeMaxW])
-{
-#pragma unroll
-    for (int j = 0; j + 1 < kTreeMaxW; ++j) { v[j] = v[j + 1]; i[j] = i[j + 1]; }
-    v[kTreeMaxW - 1] = -INFINITY;
-    i[kTreeMaxW - 1] = INT_MAX;
-}
-
-// The warp's kTreeMaxW best entries over all lanes' sorted lists, best
-// first, into ov/oi (every lane gets the same result).  Ids are distinct
-// across lanes, so the winner of a round is one lane.
-__device__ __forceinline__ void tw_warp_merge(float (&v)[kTreeMaxW], int (&i)[kTreeMaxW], float *ov, int *oi)
-{
-#pragma unroll 1
-    for (int r = 0; r < kTreeMaxW; ++r) {
-        float bv = v[0];
-        int bi = i[0];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov2 = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oi2 = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (tw_better(ov2, oi2, bv, bi)) { bv = ov2; bi = oi2; }
-        }
-        if (i[0] == bi && bi != INT_MAX) tw_pop(v, i);
-        ov[r] = bv;
-        oi[r] = bi;
-    }
-}
-
-// A logit into a thread's sorted top list (the common case is one compare).
-__device__ __forceinline__ void tw_insert(float x, int v, float (&tv)[kTreeMaxW], int (&ti)[kTreeMaxW])
-{
-    if (tw_better(x, v, tv[kTreeMaxW - 1], ti[kTreeMaxW - 1])) {
-        tv[kTreeMaxW - 1] = x;
-        ti[kTreeMaxW - 1] = v;
-#pragma unroll
-        for (int j = kTreeMaxW - 1; j > 0; --j)
-            if (tw_better(tv[j], ti[j], tv[j - 1], ti[j - 1])) {
-                const float a = tv[j]; tv[j] = tv[j - 1]; tv[j - 1] = a;
-                const int b = ti[j]; ti[j] = ti[j - 1]; ti[j - 1] = b;
-            }
-    }
-}
 
 // Up to four logits (x[0 .. n-1]) into a thread's running (max, sum of
 // exp(x - max)): one rescale per group, the exponentials independent.

@@ -403,8 +403,9 @@ orthrus_status_t orthrus_kl_lm_head(orthrus_ctx_t *ctx, const void *h_ar, const 
  * §9.6: the same proposed for Orthrus).  Greedy only.  A tree of R rows
  * keeps row 0 as the root (the anchor) and every other row r as a node
  * with parent[r] in [0, r) and its draft token; node r sits at position
- * t + depth(r).  A tree cycle is: the draft (orthrus_draft_block), the top-W
- * candidates of its rows (orthrus_tree_topw), the tree
+ * t + depth(r).  A tree cycle is: the draft with the top-W candidates of its
+ * rows (orthrus_draft_block_topw; or orthrus_draft_block and
+ * orthrus_tree_topw over materialised logits), the tree
  * (orthrus_tree_build), its tree-masked AR forward (orthrus_verify_tree)
  * and the walk plus commit (orthrus_tree_commit).
  *
@@ -417,6 +418,22 @@ orthrus_status_t orthrus_kl_lm_head(orthrus_ctx_t *ctx, const void *h_ar, const 
  */
 orthrus_status_t orthrus_tree_topw(orthrus_ctx_t *ctx, const float *logits, int32_t rows, int32_t width,
                                    int32_t *ids, float *vals, float *lse, void *stream);
+
+/*
+ * orthrus_draft_block_topw: the greedy draft (orthrus_draft_block at
+ * temperature 0: writes draft [batch][K]) that also returns, for draft rows
+ * k < depth of every sequence, the `width` largest logits best first (ties:
+ * lowest id) as ids [batch][depth][width] int32 and vals fp32, and each
+ * row's log-sum-exp lse [batch][depth] fp32 (T = 1) — orthrus_tree_topw's
+ * outputs for those rows, taken inside the LM-head pass (each vocabulary
+ * tile keeps its best width logits; a second kernel merges the tiles) so the
+ * logits never reach memory.  depth = K - 1 gives the candidates
+ * orthrus_tree_build takes for a tree that fits a K-row block.  Requires
+ * 1 <= width <= 8, width <= vocab and 1 <= depth <= K.
+ */
+orthrus_status_t orthrus_draft_block_topw(orthrus_ctx_t *ctx, const orthrus_kv_t *kv, const int32_t *anchor,
+                                          int32_t batch, int32_t K, int32_t width, int32_t depth, int32_t *draft,
+                                          int32_t *ids, float *vals, float *lse, void *stream);
 
 /*
  * orthrus_tree_build: per sequence b, the best-first draft tree.  Inputs

@@ -3,10 +3,11 @@ cycles (the paper-notes page on "Orthrus", §7.5: DDTree verifies a
 best-first tree of one draft's top prefixes with tree attention in one
 forward; §9.6: the same proposed for Orthrus; greedy only).
 
-Each cycle runs the library's own pieces: the draft (orthrus_draft_block),
-its rows' logits, top-W (orthrus_tree_topw), the tree (orthrus_tree_build),
-the tree-masked AR forward (orthrus_verify_tree) and the walk plus commit
-(orthrus_tree_commit).  The oracle mirrors each cycle on the tree the GPU
+Each cycle runs the library's own pieces: the draft with the top-W of its
+rows taken in the LM-head pass (orthrus_draft_block_topw; or the draft, its
+materialised logits and orthrus_tree_topw, which the first test shows to
+give the same candidates), the tree (orthrus_tree_build), the tree-masked AR
+forward (orthrus_verify_tree) and the walk plus commit (orthrus_tree_commit).  The oracle mirrors each cycle on the tree the GPU
 built (the builder itself is pinned exactly in test_gpu_tree.py):
 
 * tiny fp32 model: every node's logits within 1e-4 of the row's largest
@@ -35,14 +36,18 @@ pytestmark = pytest.mark.gpu
 SHAPE = dataclasses.replace(synth.TINY, std=0.2, sigma_diff=0.05)   # peaky: trees of varied depth
 
 
-def _tree_cycle(eng, anchor, K, W, nodes):
-    """One tree-verified decode cycle through the C ABI.  Returns the tree
-    (parent, token, n_rows), the GPU's g, its node logits, n and the emitted
-    tokens (sequence 0)."""
+def _tree_cycle(eng, anchor, K, W, nodes, epilogue_topw=True):
+    """One tree-verified decode cycle through the C ABI (the draft's top-W
+    from its LM-head epilogue, or from its materialised logits).  Returns
+    the tree (parent, token, n_rows), the GPU's g, its node logits, n and the
+    emitted tokens (sequence 0)."""
     D = K - 1
-    eng.draft_block(anchor, K)
-    z = eng.debug_logits(1, 1, K)[0, :D].contiguous()
-    ids, vals, lse = eng.tree_topw(z, W)
+    if epilogue_topw:
+        _, ids, vals, lse = eng.draft_block_topw(anchor, K, W, D)
+    else:
+        eng.draft_block(anchor, K)
+        z = eng.debug_logits(1, 1, K)[0, :D].contiguous()
+        ids, vals, lse = eng.tree_topw(z, W)
     par, tok, _, _, nr = eng.tree_build(ids.view(1, D, W), vals.view(1, D, W), lse.view(1, D), nodes)
     g = eng.verify_tree(anchor, par, tok)
     zt = eng.debug_logits(0, 1, nodes + 1)[0].cpu().numpy().astype(np.float64)
@@ -79,6 +84,35 @@ def tiny():
     return w, eng
 
 
+@pytest.mark.parametrize("vocab_shape", ["tiny", "bf16"])
+def test_draft_topw_from_epilogue_equals_materialised(tiny, vocab_shape):
+    """orthrus_draft_block_topw (top-W inside the LM-head pass) against the
+    greedy draft's materialised logits through orthrus_tree_topw: the same
+    drafts, ids and logits exactly, log-sum-exps within 1e-5 relative; on
+    the tiny fp32 model and on two bf16 layers of the 1.7B shape (151936
+    ids, ties included by the integer-valued logits of no row: random)."""
+    import dual_view_diffusion_b200 as pkg
+    if vocab_shape == "tiny":
+        w, eng = tiny
+        s, P, K = SHAPE, 16, 8
+    else:
+        s, P, K = synth.QWEN3_1_7B, 40, 16
+        w = synth.make_weights(s, 0, n_layers=2)
+        eng = pkg.Engine(s, w, max_batch=1, max_block=K, max_seq=128, split_tokens=64)
+    prompt = synth.make_prompt(s, P, 9)
+    for W, D in ((1, K - 1), (4, K - 1), (8, K // 2)):
+        anchor = eng.prefill(torch.from_numpy(prompt)[None])
+        d1, ids1, vals1, lse1 = eng.draft_block_topw(anchor, K, W, D)
+        d2 = eng.draft_block(anchor, K)
+        z = eng.debug_logits(1, 1, K)[0, :D].contiguous()
+        ids2, vals2, lse2 = eng.tree_topw(z, W)
+        assert eng.check_error()[0] == 0
+        assert torch.equal(d1, d2)
+        assert torch.equal(ids1[0], ids2) and torch.equal(vals1[0], vals2), W
+        l1, l2 = lse1[0].cpu().numpy(), lse2.cpu().numpy()
+        assert (np.abs(l1 - l2) <= 1e-5 * np.maximum(1.0, np.abs(l2))).all(), (l1, l2)
+
+
 @pytest.mark.parametrize("K,W,nodes", [(8, 3, 12), (6, 2, 15), (4, 4, 9)])
 def test_tiny_tree_cycles_match_oracle(tiny, K, W, nodes):
     w, eng = tiny
@@ -93,7 +127,7 @@ def test_tiny_tree_cycles_match_oracle(tiny, K, W, nodes):
     got, mirror, depths = [], True, []
     while len(got) < N:
         a = int(anchor[0])
-        par, tok, R, g, zt, n, emit = _tree_cycle(eng, anchor, K, W, nodes)
+        par, tok, R, g, zt, n, emit = _tree_cycle(eng, anchor, K, W, nodes, epilogue_topw=(W != 2))
         depths.append(int(n))
         got += emit
         if not mirror:
