@@ -175,10 +175,11 @@ def test_bf16_logits_vs_oracle_full_depth_1p7b(pkg):
     """The whole 28-layer Qwen3-1.7B shape (tied head, 151936 ids): the draft
     and verify logits of two decode cycles against the fp64 oracle at the
     same positions; the oracle follows the GPU's accepted tokens.  At this
-    depth the bf16 roundings of 28 layers add up: each row's relative L2
-    error ||dz|| / ||z|| is held to 2e-2, and its largest |dz| (2.0-2.1 % of
-    the row's largest |logit| on these seeds, against < 1 % at two layers)
-    to 3e-2."""
+    depth the bf16 operand roundings of 28 layers add up to ~2 % by
+    themselves (test_bf16_floor.py emulates them on the CPU: 1.9 % of the
+    row's largest |logit|, 2.0 % relative L2, on this seed), so each row's
+    largest |dz| over its largest |logit| and its relative L2 error are
+    bounded by that test's FULL_DEPTH_BOUND, 2.5e-2."""
     s = synth.QWEN3_1_7B
     w = synth.make_weights(s, 0)
     K, P = 8, 64
@@ -200,7 +201,7 @@ def test_bf16_logits_vs_oracle_full_depth_1p7b(pkg):
         ref_v = m.forward(0, 0, [a] + draft[0, :K - 1].cpu().tolist(), t, kc, vc)
         errs = (rel_l2(dl, ref_d), rel_l2(vl, ref_v), rel_max(dl, ref_d), rel_max(vl, ref_v))
         print("full-depth 1.7B logits: relative L2 draft %.2e verify %.2e, max/row-max draft %.2e verify %.2e" % errs)
-        assert errs[0] <= 2e-2 and errs[1] <= 2e-2 and errs[2] <= 3e-2 and errs[3] <= 3e-2, errs
+        assert max(errs) <= 2.5e-2, errs
         n, toks = eng.commit(anchor, K)
         n = int(n[0])
         t += n
