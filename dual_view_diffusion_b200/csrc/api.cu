@@ -283,6 +283,10 @@ static cudaError_t forward(Ctx &c, const orthrus_kv_t &kv, int view, int B, int 
         GemmArgs o{};
         o.x = c.attn_o; o.M = M; o.N = f.hidden; o.Kd = f.n_q_heads * hd; o.w[0] = W.wo; o.wrows[0] = f.hidden;
         o.epi = EPI_RESID; o.resid = c.h; o.defer = defer_o; o.rpart = c.resid_part; o.rpart_rows = c.Rw;
+        // the attention before it is latency-bound: a full ring of weight
+        // requests (16 MiB over the grid) issued while it runs delays its
+        // own loads more than it saves here (measured on the 8B decode step)
+        o.prewait_stages = 2;
         {
             ProbeScope ps(c, 0, l, view, s);
             if ((e = launch_gemm(c, o, s)) != cudaSuccess) return e;

@@ -51,8 +51,8 @@
 
 namespace orthrus {
 
-constexpr int kAtKStages = 3;   // K tiles are released as soon as S = Q K^T is done
-constexpr int kAtVStages = 3;   // V tiles live until their P.V
+constexpr int kAtKStages = 2;   // K tiles are released as soon as S = Q K^T is done
+constexpr int kAtVStages = 2;   // V tiles live until their P.V
 constexpr float kRescaleSlack = 8.0f;   // log2 units a row's max may grow before O is rescaled
 constexpr int kAtMaxCluster = 8;        // portable cluster size
 constexpr int kAtMaxZ = 4;              // clusters per row group (long contexts)

@@ -350,6 +350,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
             int issued = 0;
             bool waited = false;
             const uint64_t wpol = l2_evict_first();
+            const int prewait = a.prewait_stages > 0 ? min(stages, a.prewait_stages) : stages;
             int def_c[kTcStages], def_mt[kTcStages];
             auto release_deferred = [&]() {
                 pdl_wait();
@@ -366,7 +367,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                     while (wsel < 2 && wrow >= a.wrows[wsel]) { wrow -= a.wrows[wsel]; ++wsel; }
                 }
                 for (int c = s.c0; c < s.c1; ++c) {
-                    if (!waited && issued == stages) release_deferred();
+                    if (!waited && issued == prewait) release_deferred();
                     if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort) || *abort) { stop = true; break; }
                     mbar_expect_tx(&sm.full[stage], kStageWBytes + xbytes);
                     unsigned char *wdst = ring_w + (size_t)stage * kStageWBytes;

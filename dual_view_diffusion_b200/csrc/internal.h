@@ -86,6 +86,9 @@ struct GemmArgs {
     // written to rpart[seg][row][N] and summed into resid by the next RMSNorm
     int defer;               // segments per tile (0: add in the epilogue)
     int pair;                // tensor-core path: 2 or 3 k segments per n tile, reduced inside a cluster (0: off)
+    // tensor-core path: ring stages whose weight tiles are requested before
+    // waiting for the predecessor grid (0: the whole ring)
+    int prewait_stages;
     float *rpart;
     int rpart_rows;
     // EPI_SWIGLU
