@@ -277,27 +277,38 @@ __device__ void epilogue(const GemmArgs &a, float (*tile)[kTilePad], int mt, int
             }
         } else {
             bf16 *base = (bf16 *)(a.kv_to_cache ? a.kv.v_pages : a.v_blk);
+            // every 8-row group's slots consecutive and 16-byte aligned (a
+            // block starting at a multiple of 8, inside one page): one 16-byte
+            // store per (group, dim); otherwise (a decode block at any
+            // position) each warp writes 32 consecutive slots of one dim row
+            // per store instruction, lane = row
+            bool vec = (vstride & 7) == 0;
 #pragma unroll
-            for (int j = 0; j < kTileM * kTileN / 8 / kEpiThreads; ++j) {
-                const int item = tid + j * kEpiThreads, tg = item & 3, d = item >> 2, m0 = tg * 8;
-                const long long d0 = s_dst[m0];
-                bool run = d0 >= 0 && ((d0 + (long long)d * vstride) & 7) == 0;
+            for (int tg = 0; tg < kTileM / 8; ++tg) {
+                const long long d0 = s_dst[tg * 8];
+                vec = vec && d0 >= 0 && (d0 & 7) == 0;
 #pragma unroll
-                for (int e = 1; e < 8; ++e) run = run && s_dst[m0 + e] == d0 + e;
-                if (run) {
+                for (int e = 1; e < 8; ++e) vec = vec && s_dst[tg * 8 + e] == d0 + e;
+            }
+            if (vec) {
+#pragma unroll
+                for (int j = 0; j < kTileM * kTileN / 8 / kEpiThreads; ++j) {
+                    const int item = tid + j * kEpiThreads, tg = item & 3, d = item >> 2, m0 = tg * 8;
                     uint32_t o[4];
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
                         const __nv_bfloat162 h2 = __floats2bfloat162_rn(tile[m0 + e][d], tile[m0 + e + 1][d]);
                         o[e / 2] = *(const uint32_t *)&h2;
                     }
-                    __stcg((uint4 *)(base + d0 + (long long)d * vstride), make_uint4(o[0], o[1], o[2], o[3]));
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const long long de = s_dst[m0 + e];
-                        if (de >= 0) base[de + (long long)d * vstride] = __float2bfloat16_rn(tile[m0 + e][d]);
-                    }
+                    __stcg((uint4 *)(base + s_dst[m0] + (long long)d * vstride), make_uint4(o[0], o[1], o[2], o[3]));
+                }
+            } else {
+                const int m = tid & 31, w = tid >> 5;
+                const long long de = s_dst[m];
+#pragma unroll 8
+                for (int dd = 0; dd < kTileN / (kEpiThreads / 32); ++dd) {
+                    const int d = w * (kTileN / (kEpiThreads / 32)) + dd;
+                    if (de >= 0) base[de + (long long)d * vstride] = __float2bfloat16_rn(tile[m][d]);
                 }
             }
         }
