@@ -42,6 +42,73 @@ __device__ __forceinline__ void tw_lse4(const float (&x)[4], int n, float &m, fl
     s += add;
 }
 
+// The warp keeps one sorted list (every lane holds the same copy): the
+// lanes' candidates (n values each, ids ascending within a lane) enter one
+// at a time in (lane, element) order, each insertion the same on every lane,
+// and a candidate is dropped as soon as the list's last entry passes it.  A
+// warp meets about W ln(N / W) insertions over N logits, so almost every
+// step is one compare per value and a ballot.  Every lane must call it.
+__device__ __forceinline__ void tw_warp_insert(const float *x, const int *id, int n, float (&tv)[kTopWMax],
+                                               int (&ti)[kTopWMax])
+{
+    const int lane = threadIdx.x & 31;
+    if (ti[kTopWMax - 1] == INT_MAX) {
+        // the list is not full yet (the first steps, warp-uniform): every
+        // lane's candidates and one entry of the list each go into a private
+        // list, and the warp merges them all at once
+        float pv[kTopWMax];
+        int pi[kTopWMax];
+#pragma unroll
+        for (int j = 0; j < kTopWMax; ++j) { pv[j] = -INFINITY; pi[j] = INT_MAX; }
+        float cv = -INFINITY;
+        int cid = INT_MAX;
+#pragma unroll
+        for (int j = 0; j < kTopWMax; ++j)
+            if (j == lane) { cv = tv[j]; cid = ti[j]; }
+        if (cid != INT_MAX) tw_insert(cv, cid, pv, pi);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (k < n) tw_insert(x[k], id[k], pv, pi);
+#pragma unroll
+        for (int r = 0; r < kTopWMax; ++r) {   // round r: the warp's best remaining head
+            float bv = pv[0];
+            int bi = pi[0];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                if (tw_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+            }
+            if (pi[0] == bi && bi != INT_MAX) tw_pop(pv, pi);
+            tv[r] = bv;
+            ti[r] = bi;
+        }
+        return;
+    }
+    uint32_t cm = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        if (k < n && tw_better(x[k], id[k], tv[kTopWMax - 1], ti[kTopWMax - 1])) cm |= 1u << k;
+    for (;;) {
+        const uint32_t any = __ballot_sync(0xffffffffu, cm != 0);
+        if (!any) break;
+        const int src = __ffs(any) - 1;
+        const int e = __ffs(__shfl_sync(0xffffffffu, cm, src)) - 1;
+        float xv = x[0];
+        int xi = id[0];
+#pragma unroll
+        for (int k = 1; k < 4; ++k)
+            if (k < n && k == e) { xv = x[k]; xi = id[k]; }
+        xv = __shfl_sync(0xffffffffu, xv, src);
+        xi = __shfl_sync(0xffffffffu, xi, src);
+        tw_insert(xv, xi, tv, ti);
+        if (lane == src) cm &= ~(1u << e);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (((cm >> k) & 1u) && !tw_better(x[k], id[k], tv[kTopWMax - 1], ti[kTopWMax - 1])) cm &= ~(1u << k);
+    }
+}
+
 __device__ __forceinline__ uint32_t tw_smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 __device__ __forceinline__ uint32_t tw_mapa(uint32_t addr, uint32_t rank)
 {
@@ -95,33 +162,39 @@ __global__ void __launch_bounds__(kTreeTopwThreads) tree_topw_kernel(const float
 #pragma unroll
     for (int j = 0; j < kTreeMaxW; ++j) { tv[j] = -INFINITY; ti[j] = INT_MAX; }
     float m = -INFINITY, s = 0.f;   // running max and sum of exp(x - m)
+    // lanes walk the range in warp-uniform steps (the list is shared by the
+    // warp); lanes past the end offer nothing
     if (VEC) {
         constexpr int U = 4;
         const int q0 = lo / 4, q1 = (hi + 3) / 4;   // hi is V or a multiple of 4; V % 4 == 0 here
         const float4 *z4 = (const float4 *)zr;
-        for (int i0 = q0 + threadIdx.x; i0 < q1; i0 += kTreeTopwThreads * U) {
+        for (int b0 = q0 + (threadIdx.x & ~31); b0 < q1; b0 += kTreeTopwThreads * U) {
             float4 x4[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int i = i0 + u * kTreeTopwThreads;
+                const int i = b0 + lane + u * kTreeTopwThreads;
                 x4[u] = i < q1 ? z4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int i = i0 + u * kTreeTopwThreads;
-                if (i < q1) {
-                    const float x[4] = {x4[u].x, x4[u].y, x4[u].z, x4[u].w};
-                    tw_lse4(x, 4, m, s);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) tw_insert(x[e], 4 * i + e, tv, ti);
-                }
+                const int i = b0 + lane + u * kTreeTopwThreads;
+                const bool in = i < q1;
+                const float x[4] = {in ? x4[u].x : -INFINITY, in ? x4[u].y : -INFINITY,
+                                    in ? x4[u].z : -INFINITY, in ? x4[u].w : -INFINITY};
+                const int id[4] = {in ? 4 * i : INT_MAX, in ? 4 * i + 1 : INT_MAX, in ? 4 * i + 2 : INT_MAX,
+                                   in ? 4 * i + 3 : INT_MAX};
+                if (in) tw_lse4(x, 4, m, s);
+                tw_warp_insert(x, id, 4, tv, ti);
             }
         }
     } else {
-        for (int v = lo + threadIdx.x; v < hi; v += kTreeTopwThreads) {
-            const float x[4] = {zr[v], 0.f, 0.f, 0.f};
-            tw_lse4(x, 1, m, s);
-            tw_insert(x[0], v, tv, ti);
+        for (int b = lo + (threadIdx.x & ~31); b < hi; b += kTreeTopwThreads) {
+            const int v = b + lane;
+            const bool in = v < hi;
+            const float x[4] = {in ? zr[v] : -INFINITY, 0.f, 0.f, 0.f};
+            const int id[4] = {in ? v : INT_MAX, 0, 0, 0};
+            if (in) tw_lse4(x, 1, m, s);
+            tw_warp_insert(x, id, 1, tv, ti);
         }
     }
     // this CTA: (m, s) across the warp, then across warps; lists likewise
@@ -134,7 +207,8 @@ __global__ void __launch_bounds__(kTreeTopwThreads) tree_topw_kernel(const float
     }
     float mv[kTreeMaxW];
     int mi[kTreeMaxW];
-    tw_warp_merge(tv, ti, mv, mi);
+#pragma unroll
+    for (int j = 0; j < kTreeMaxW; ++j) { mv[j] = tv[j]; mi[j] = ti[j]; }   // the warp's list (every lane's copy)
     if (lane == 0) {
         wm[warp] = m;
         ws[warp] = s;
