@@ -29,7 +29,33 @@ __global__ void embed_kernel(const T *embed, int d, int V, int mask_id, int mode
     }
     if (threadIdx.x == 0) tok_out[row] = tok;
     const T *src = embed + (size_t)tok * d;
-    for (int i = threadIdx.x; i < d; i += blockDim.x) h[(size_t)row * d + i] = to_f<T>(src[i]);
+    float *dst = h + (size_t)row * d;
+    constexpr int E = 16 / (int)sizeof(T);   // elements per 16-byte chunk
+    if (d % E == 0 && ((uintptr_t)src & 15) == 0 && ((uintptr_t)dst & 15) == 0) {
+        // every chunk of the row in flight at once (one round trip to the table)
+        constexpr int Q = 4;
+        const int nc = d / E;
+        for (int c0 = threadIdx.x; c0 < nc; c0 += Q * blockDim.x) {
+            uint4 u[Q];
+#pragma unroll
+            for (int q = 0; q < Q; ++q) {
+                const int c = c0 + q * blockDim.x;
+                if (c < nc) u[q] = ((const uint4 *)src)[c];
+            }
+#pragma unroll
+            for (int q = 0; q < Q; ++q) {
+                const int c = c0 + q * blockDim.x;
+                if (c >= nc) continue;
+                const T *e = (const T *)&u[q];
+#pragma unroll
+                for (int k4 = 0; k4 < E; k4 += 4)
+                    *(float4 *)(dst + (size_t)c * E + k4) =
+                        make_float4(to_f<T>(e[k4]), to_f<T>(e[k4 + 1]), to_f<T>(e[k4 + 2]), to_f<T>(e[k4 + 3]));
+            }
+        }
+    } else {
+        for (int i = threadIdx.x; i < d; i += blockDim.x) dst[i] = to_f<T>(src[i]);
+    }
 }
 
 // ---------------------------------------------------------------- RMSNorm
@@ -69,11 +95,21 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(float *h, const T
 {
     __shared__ float red[kNormThreads / 32];
     pdl_trigger();
-    pdl_wait();
     const int row = blockIdx.x, tid = threadIdx.x;
+    const bool vec = (d & 3) == 0 && d <= kNormThreads * 4 * kNormVec;
+    // the gain is a weight (no predecessor writes it): fetched before the
+    // wait, so the output loop does not wait on a second round trip
+    float4 gv[kNormVec];
+    if (vec) {
+#pragma unroll
+        for (int j = 0; j < kNormVec; ++j) {
+            const int i = (tid + j * kNormThreads) * 4;
+            gv[j] = i < d ? load_gain4(gain, i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    pdl_wait();
     float *x = h + (size_t)row * d;
     float ss = 0.f;
-    const bool vec = (d & 3) == 0 && d <= kNormThreads * 4 * kNormVec;
     float4 v[kNormVec];
     if (vec) {
 #pragma unroll
@@ -133,7 +169,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(float *h, const T
         for (int j = 0; j < kNormVec; ++j) {
             const int i = (tid + j * kNormThreads) * 4;
             if (i < d) {
-                const float4 g = load_gain4(gain, i);
+                const float4 g = gv[j];
                 store4<T>(o + i, v[j].x * inv * g.x, v[j].y * inv * g.y, v[j].z * inv * g.z, v[j].w * inv * g.w);
             }
         }
