@@ -315,16 +315,29 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_tc_kernel(const __grid_con
     // 32 flat subtiles at a time, one per lane.
     const int tps = a.split_tokens / kAtSub;
     const int cache_lim = a.mode == 0 ? t + a.K : t;
-    auto lookup = [&](int f) {
+    // (row = the sequence's block-table row; `got` = that row's entry when
+    // already fetched)
+    auto page_of = [&](int f, int row, bool have, int got) {
         const int sl = ci + Ctot * (f / tps);
         const int key = sl * a.split_tokens + (f % tps) * kAtSub;
         if (sl >= n_split_grid || key >= cache_lim) return 0;
         const int pidx = key / a.kv.page_size;
-        int page = (pidx < a.kv.max_pages) ? a.kv.block_table[(size_t)bt_row * a.kv.max_pages + pidx] : -1;
+        int page = pidx < a.kv.max_pages ? (have ? got : a.kv.block_table[(size_t)row * a.kv.max_pages + pidx]) : -1;
         if (page < 0 || page >= a.kv.num_pages) { raise_err(a.err, ORTHRUS_DEVERR_CAPACITY); page = 0; }
         return page;
     };
-    int pg = (warp == 0 || warp == kAtVWarp) ? lookup(lane) : 0;
+    auto lookup = [&](int f) { return page_of(f, bt_row, false, 0); };
+    int pg = 0;
+    if (warp == 0 || warp == kAtVWarp) {
+        // the first pages are read from row b, the usual row map, together
+        // with t and the map itself (one round trip instead of two); only a
+        // sequence mapped elsewhere reads its own row afterwards
+        const int sl = ci + Ctot * (lane / tps);
+        const int pidx = (sl * a.split_tokens + (lane % tps) * kAtSub) / a.kv.page_size;
+        const int guess = (sl < n_split_grid && pidx < a.kv.max_pages)
+                              ? a.kv.block_table[(size_t)b * a.kv.max_pages + pidx] : 0;
+        pg = page_of(lane, bt_row, bt_row == b, guess);
+    }
 
     if (threadIdx.x == 0) {
         at_mbar_init(&sm.q_ready, 128);
