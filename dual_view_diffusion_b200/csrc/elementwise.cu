@@ -217,6 +217,8 @@ __global__ void __launch_bounds__(256) lm_finalize_kernel(LmArgs a)
     float gb = -INFINITY, gz = 0.f;
     int ga = 0x7fffffff;
     float zid = NAN;
+    // (unrolled: the tiles' records are independent loads, in flight together)
+#pragma unroll 4
     for (int i = lane; i < a.n_vtiles; i += 32) {
         const LmPart q = p[i];
         argmax_merge(zm, za, q.zmax, q.zarg);
@@ -235,6 +237,7 @@ __global__ void __launch_bounds__(256) lm_finalize_kernel(LmArgs a)
     if (has) zid = __shfl_sync(0xffffffffu, zid, __ffs(has) - 1);
     const float it = a.inv_temp > 0.f ? a.inv_temp : 1.0f;
     float s = 0.f, ez = 0.f;
+#pragma unroll 4
     for (int i = lane; i < a.n_vtiles; i += 32) {
         const float f = expf((p[i].zmax - zm) * it);
         s += p[i].zsum * f;
@@ -328,28 +331,39 @@ __global__ void commit_decide_kernel(CommitArgs a)
 {
     pdl_trigger();
     pdl_wait();
-    const int b = blockIdx.x;
+    const int b = blockIdx.x, lane = threadIdx.x & 31;
     __shared__ int s_j;
-    if (threadIdx.x == 0) {
+    if (threadIdx.x < 32) {   // warp 0: rows k = lane, lane + 32, ... tested at once, the first failure wins
         int n = a.K, j = -1;
         if (a.force_n) {
             n = min(max(a.force_n[b], 1), a.K);
         } else if (a.inv_temp <= 0.f) {
             const int kt = a.kt ? min(max(a.kt[b], 1), a.K) : a.K;
             n = kt;
-            for (int k = 0; k < kt; ++k)
-                if (a.draft[b * a.K + k] != a.g[b * a.K + k]) { n = k + 1; break; }
+            for (int k0 = 0; k0 < kt; k0 += 32) {
+                const int k = k0 + lane;
+                const unsigned miss = __ballot_sync(0xffffffffu, k < kt && a.draft[b * a.K + k] != a.g[b * a.K + k]);
+                if (miss) { n = k0 + __ffs(miss); break; }
+            }
         } else {
             const uint32_t step = (uint32_t)*a.step;
-            for (int k = 0; k < a.K; ++k) {
-                const float log_u = -neg_log_uniform(a.seed, step, rng_row(b, k), 0, PURPOSE_ACCEPT);
-                if (!(log_u < a.logp[b * a.K + k] - a.logq[b * a.K + k])) { j = k; n = k + 1; break; }
+            for (int k0 = 0; k0 < a.K; k0 += 32) {
+                const int k = k0 + lane;
+                bool rej = false;
+                if (k < a.K) {
+                    const float log_u = -neg_log_uniform(a.seed, step, rng_row(b, k), 0, PURPOSE_ACCEPT);
+                    rej = !(log_u < a.logp[b * a.K + k] - a.logq[b * a.K + k]);
+                }
+                const unsigned r = __ballot_sync(0xffffffffu, rej);
+                if (r) { j = k0 + __ffs(r) - 1; n = j + 1; break; }
             }
         }
-        a.n_out[b] = n;
-        if (a.rej_row) a.rej_row[b] = j;
-        if (j >= 0) atomicOr(a.any_reject, 1);
-        s_j = j;
+        if (lane == 0) {
+            a.n_out[b] = n;
+            if (a.rej_row) a.rej_row[b] = j;
+            if (j >= 0) atomicOr(a.any_reject, 1);
+            s_j = j;
+        }
     }
     __syncthreads();
     if (s_j >= 0 && a.res_x) {
@@ -368,29 +382,28 @@ __global__ void commit_apply_kernel(CommitArgs a)
     // no early pdl_trigger: later kernels read what this one writes before
     // their griddepcontrol.wait, so nothing may be scheduled until it exits
     pdl_wait();
-    const int b = threadIdx.x;
+    // one warp per sequence, a lane per emitted token
+    const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (b < a.B) {
         const int n = a.n_out[b];
         const int j = a.rej_row ? a.rej_row[b] : -1;
         const bool sampled = a.inv_temp > 0.f && !a.force_n;
-        int last = 0;
-        for (int i = 0; i < n; ++i) {
+        const int p0 = a.append_out ? a.produced[b] : 0;
+        for (int i = lane; i < n; i += 32) {
             int tok;
             if (!sampled) tok = a.g[b * a.K + i];
             else tok = (i == j) ? a.res_tok[b] : a.draft[b * a.K + i];
             if (a.tokens_out) a.tokens_out[b * a.K + i] = tok;
-            if (a.append_out) {
-                const int pos = a.produced[b] + i;
-                if (pos < a.append_max) a.append_out[(size_t)b * a.append_stride + pos] = tok;
-            }
-            last = tok;
+            if (a.append_out && p0 + i < a.append_max) a.append_out[(size_t)b * a.append_stride + p0 + i] = tok;
+            if (i == n - 1) a.anchor_io[b] = tok;
         }
-        if (a.append_out) a.produced[b] += n;
-        a.anchor_io[b] = last;
-        a.seq_lens[b] += n;
+        __syncwarp();   // every lane has read produced[b]
+        if (lane == 0) {
+            if (a.append_out) a.produced[b] = p0 + n;
+            a.seq_lens[b] += n;
+        }
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {   // nothing in this kernel reads them
         *a.step += 1;
         if (a.any_reject) *a.any_reject = 0;
     }
@@ -641,7 +654,7 @@ cudaError_t launch_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int K, fl
         e = launch_lm_finalize_impl(c, 3, B, K, temperature, nullptr, nullptr, s);
         if (e != cudaSuccess) return e;
     }
-    return launch_k(commit_apply_kernel, 1, 128, 0, s, a);
+    return launch_k(commit_apply_kernel, (B + 3) / 4, 128, 0, s, a);
 }
 
 cudaError_t launch_ar_commit(const Ctx &c, const orthrus_kv_t &kv, int B, int64_t *step, int32_t *token_out,
