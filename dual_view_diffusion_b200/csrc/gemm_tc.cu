@@ -577,15 +577,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
             if (reducer && et > 0 && et < s.nseg) a.ticket[slot0 + et] = 0;   // flags ready for the next call
             SyncEpilogue{}();
         }
+        // cluster mode, ranks 1..: rank 0's last signal (its arrive after
+        // consuming the last handover) lands before this CTA leaves; rank 0
+        // itself waited for every copy into it, so no cluster barrier is
+        // needed at the end
+        if (pair && crank > 0 && hc > 0) {
+            if (et == 0) mbar_wait(&sm.peer_empty, (hc - 1) & 1, abort);
+            SyncEpilogue{}();
+        }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (pair) {   // no CTA leaves while the other may still signal or copy into it
-        if (warp < 2) tc_cluster_wait();
-        tc_cluster_arrive();
-        tc_cluster_wait();
-    }
+    if (pair && warp < 2) tc_cluster_wait();   // (their arrive at the start)
     if (sm.abort && threadIdx.x == 0) raise_err(a.err, ORTHRUS_DEVERR_TIMEOUT);
     if (warp == 1) {
         __syncwarp();
