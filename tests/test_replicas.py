@@ -36,7 +36,7 @@ def _worker(rank, world, port, out):
 
 
 def test_two_rank_reduction():
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()   # no fork of a multi-threaded parent
     out = mgr.dict()
     port = _free_port()
     mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
