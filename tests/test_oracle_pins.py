@@ -57,6 +57,22 @@ def test_gumbel_max_samples_softmax():
     assert chi2 < 25.0          # 5 dof: p-value ~1e-4
 
 
+def test_softmax_t_matches_torch():
+    z = np.random.default_rng(9).standard_normal(50) * 3.0
+    for T in (0.3, 0.7, 1.0, 2.5):
+        want = torch.softmax(torch.from_numpy(z) / T, 0).numpy()
+        assert np.allclose(oracle.softmax_t(z, T), want, rtol=1e-13, atol=1e-17)
+
+
+def test_argmax_lowest_index_and_margin():
+    # ties go to the lowest index (the order the greedy decode commits to);
+    # the margin is best minus second best, 0 at a tie
+    assert oracle.argmax([1.0, 3.0, 3.0, 2.0]) == (1, 0.0)
+    assert oracle.argmax([0.5, 2.0, -1.0, 1.5]) == (1, 0.5)
+    assert oracle.argmax([4.0, 4.0]) == (0, 0.0)
+    assert oracle.argmax([-2.0, -3.0, -1.0]) == (2, 1.0)
+
+
 # ------------------------------------------------------------------ blocks
 def test_rmsnorm_closed_form_and_torch():
     for c in (0.5, -3.0, 1e-4):
@@ -178,6 +194,69 @@ def test_ar_forward_matches_hf_llama():
     assert np.abs(z - ref).max() < 1e-6 * max(1.0, np.abs(ref).max())
 
 
+def test_ar_greedy_stream_matches_hf_llama():
+    """The oracle's plain AR decode (prefill of all but the last prompt token,
+    that token as the first anchor, then one cached row per token) emits the
+    tokens of a greedy loop over HuggingFace full-sequence forwards.  The
+    loop's smallest argmax margin is asserted to stay far above the 1e-6 the
+    two models' logits may differ by, so equality is a strict test."""
+    w = synth.make_weights(synth.TINY, 0, random_gains=True)
+    pr = synth.make_prompt(synth.TINY, 16, 0)
+    hf = _hf_llama(w)
+    seq, want, margins = [int(x) for x in pr], [], []
+    with torch.no_grad():
+        for _ in range(24):
+            z = hf(torch.tensor([seq], dtype=torch.int64)).logits[0, -1].numpy()
+            top2 = np.sort(z)[-2:]
+            margins.append(top2[1] - top2[0])
+            want.append(int(np.argmax(z)))
+            seq.append(want[-1])
+    assert min(margins) > 1e-4
+    a = oracle.Model(w).generate(pr, 1, 24, 0.0, 0, "ar")
+    assert a["tokens"].tolist() == want
+
+
+def test_ar_law_matches_hf_llama():
+    """The exact AR law of the first two tokens at T = 0.7 (the enumeration
+    the losslessness pins compare against) is the product of HuggingFace's
+    softmax(logits / T) after the prompt and after the prompt plus the first
+    token."""
+    w = synth.make_weights(synth.MICRO, 0)
+    pr = synth.make_prompt(synth.MICRO, 3, 0)
+    T, V = 0.7, synth.MICRO.vocab
+    hf = _hf_llama(w)
+
+    def p_next(seq):
+        with torch.no_grad():
+            z = hf(torch.tensor([list(seq)], dtype=torch.int64)).logits[0, -1]
+        return torch.softmax(z / T, 0).numpy()
+
+    p1 = p_next(pr)
+    want = np.concatenate([p1[x] * p_next(list(pr) + [x]) for x in range(V)])
+    got = oracle.Model(w).enumerate_ar(pr, 2, T)
+    assert np.allclose(got, want, rtol=0, atol=1e-6)
+
+
+def test_diffusion_view_is_the_network_with_its_own_projections(tiny_weights, tiny_prompt):
+    """Notes §2.1: the diffusion view is the frozen network with only W_Q,
+    W_K, W_V replaced by the diffusion copies.  Its forward over a block
+    equals the AR-view code path, under the same (bidirectional) mask, of a
+    model whose W_Q/W_K/W_V are those copies; with the original model's AR
+    weights the result differs."""
+    import dataclasses
+    w = tiny_weights
+    swapped = dataclasses.replace(w, layers=[dict(lw, wq=lw["wq_diff"], wk=lw["wk_diff"], wv=lw["wv_diff"])
+                                             for lw in w.layers])
+    m, m2 = oracle.Model(w), oracle.Model(swapped)
+    kc, vc = m.new_cache(64)
+    t = m.prefill(tiny_prompt, kc, vc)
+    mask = synth.TINY.mask_id
+    blk = [int(tiny_prompt[-1]), mask, 17, mask, mask]
+    a = m.forward(1, 1, blk, t, kc.copy(), vc.copy())
+    assert np.array_equal(a, m2.forward(0, 1, blk, t, kc.copy(), vc.copy()))
+    assert not np.allclose(a, m.forward(0, 1, blk, t, kc.copy(), vc.copy()), rtol=0, atol=1e-9)
+
+
 def test_block_rows_equal_single_rows(tiny_weights, tiny_prompt):
     """Row k of a causal block equals the same row run alone after the rows
     before it were committed (bitwise: rows are computed independently)."""
@@ -216,6 +295,41 @@ def test_draft_does_not_touch_cache(tiny_weights, tiny_prompt):
     k0, v0 = kc.copy(), vc.copy()
     m.draft(kc, vc, t, tiny_prompt[-1], 4)
     assert np.array_equal(kc, k0) and np.array_equal(vc, v0)
+
+
+def test_draft_is_the_diffusion_view_of_anchor_and_masks(tiny_weights, tiny_prompt):
+    """Notes §4.1 step 1: the draft is one diffusion-view forward of the block
+    [anchor, m, ..., m] at positions t .. t+K-1; row k's token is its argmax
+    (T = 0) or the Gumbel-max draw of row k's noise (T > 0, which also
+    returns q = softmax(z / T)).  Retyping the block through the plain
+    forward gives the same logits."""
+    m = oracle.Model(tiny_weights)
+    kc, vc = m.new_cache(64)
+    t = m.prefill(tiny_prompt, kc, vc)
+    K, a = 5, int(tiny_prompt[-1])
+    ref = m.forward(1, 1, [a] + [synth.TINY.mask_id] * (K - 1), t, kc.copy(), vc.copy())
+    d, _, z, _ = m.draft(kc, vc, t, a, K)
+    assert np.array_equal(z, ref) and np.array_equal(d, ref.argmax(axis=1))
+    T, seed, step = 0.8, 5, 3
+    d2, q2, _, _ = m.draft(kc, vc, t, a, K, T, seed, step)
+    assert [int(x) for x in d2] == [oracle.sample_logits(ref[k], T, seed, step, k, oracle.PURPOSE_DRAFT)[0]
+                                    for k in range(K)]
+    assert np.allclose(q2, torch.softmax(torch.from_numpy(ref) / T, 1).numpy(), rtol=1e-12, atol=1e-15)
+
+
+def test_verify_is_the_ar_view_of_anchor_and_drafts(tiny_weights, tiny_prompt):
+    """Notes §4.1 step 2: verification is one causal AR-view forward of
+    [anchor, y_1 .. y_{K-1}] at positions t .. t+K-1 that writes those rows'
+    K/V into the cache; g_k is row k's argmax."""
+    m = oracle.Model(tiny_weights)
+    kc, vc = m.new_cache(64)
+    t = m.prefill(tiny_prompt, kc, vc)
+    a, y = int(tiny_prompt[-1]), [40, 3, 200, 77, 9]
+    k2, v2 = kc.copy(), vc.copy()
+    ref = m.forward(0, 0, [a] + y[:-1], t, k2, v2)
+    g, _, z, _ = m.verify(kc, vc, t, a, y)
+    assert np.array_equal(z, ref) and np.array_equal(g, ref.argmax(axis=1))
+    assert np.array_equal(kc, k2) and np.array_equal(vc, v2)
 
 
 # ------------------------------------------------------------------ consensus
