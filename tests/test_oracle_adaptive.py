@@ -77,3 +77,35 @@ def test_adaptive_decoding_equals_ar(model, h_max):
     t = min(ar["t"], a["t"])
     assert np.array_equal(ar["k_cache"][:, :t], a["k_cache"][:, :t])
     assert np.array_equal(ar["v_cache"][:, :t], a["v_cache"][:, :t])
+
+
+def test_adaptive_cycle_is_its_retyped_steps(model):
+    """An adaptive cycle is: the draft at T = 0, scipy's entropy of each
+    draft row's softmax, the length rule, one AR verify of [anchor, y_1 ..
+    y_{Kt-1}] and the greedy consensus over those Kt rows.  Retyping four
+    cycles from those pinned pieces gives generate_adaptive's lengths and
+    tokens (no entropy within 1e-9 of the threshold, so the rule cannot flip
+    on rounding)."""
+    from scipy.special import softmax
+    from scipy.stats import entropy
+    m, p = model
+    K, h_max = 8, 4.4
+    kc, vc = m.new_cache(len(p) + 64)
+    t = m.prefill(p, kc, vc)
+    anchor, out, ns, ks = int(p[-1]), [], [], []
+    for _ in range(4):
+        d, _, z, _ = m.draft(kc, vc, t, anchor, K)
+        H = [float(entropy(softmax(z[k]))) for k in range(K)]
+        assert min(abs(h - h_max) for h in H) > 1e-9
+        kt = oracle.adaptive_len(H, h_max)
+        g, _, _, _ = m.verify(kc, vc, t, anchor, d[:kt])
+        n, emit = oracle.consensus_greedy(d[:kt], g)
+        t += n
+        anchor = int(emit[-1])
+        out += [int(x) for x in emit]
+        ns.append(int(n))
+        ks.append(int(kt))
+    assert len(set(ks)) >= 2                            # the threshold does vary the length
+    r = m.generate_adaptive(p, K, h_max, len(out))
+    assert r["k_per_cycle"][:4].tolist() == ks and r["n_per_cycle"][:4].tolist() == ns
+    assert r["tokens"].tolist() == out

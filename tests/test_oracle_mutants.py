@@ -142,15 +142,32 @@ MUTANTS = (
            "if (j >= t && j - t > r) continue;", ("tree_sdpa",), count=3),
     Mutant("tree rows at their row positions", "forward_rows", "(r == 0 ? t : pos[parent[r]] + 1)", "t + r",
            ("tree_forward",)),
+    Mutant("tree scores from unnormalised logits", "oc_generate_tree", "lp[(size_t)d * V + v] = zr[v] - m - log(s);",
+           "lp[(size_t)d * V + v] = zr[v] - m;", ("tree_cycle",)),
+    Mutant("tree depths from the next draft row", "oc_generate_tree", "const double *zr = z + (size_t)d * V;",
+           "const double *zr = z + (size_t)(d + 1) * V;", ("tree_cycle",)),
+    Mutant("tree root is the first draft, not the anchor", "oc_generate_tree", "tok[0] = anchor;",
+           "tok[0] = draft[0];", ("tree_eq_ar", "tree_cycle")),
     # adaptive block length (notes §7.4, §9.6)
     Mutant("entropy sign", "oc_entropy", "return lse - e;", "return e - lse;", ("entropy",)),
     Mutant("threshold made strict", "oc_adaptive_len", "H[k - 1] <= h_max", "H[k - 1] < h_max", ("adaptive_len",)),
     Mutant("length rule reads the next row", "oc_adaptive_len", "H[k - 1] <= h_max", "H[k] <= h_max",
            ("adaptive_len",)),
+    Mutant("every row's entropy taken from row 0", "oc_generate_adaptive",
+           "H[k] = oc_entropy(z + (size_t)k * V, V);", "H[k] = oc_entropy(z, V);", ("adaptive_cycle",)),
+    # the iterative draft (notes §5.4.2) and the exact law of the sampled cycle (notes §4.3)
+    Mutant("second pass reads the drafts one row late", "oc_draft_iter", "s == 0 ? c->mask_id : draft[k - 1]",
+           "s == 0 ? c->mask_id : draft[k]", ("iterative_pass2",)),
+    Mutant("enumeration forgets the acceptance so far", "oc_enumerate_orthrus", "double rej = acc * (1.0 - a);",
+           "double rej = 1.0 - a;", ("lossless_enum",)),
 )
 
 SDPA_CASES = ((0, 1, 0), (0, 5, 1), (37, 4, 0), (37, 4, 1))
 TREE_CASES = ((3, 7, 3, 10, "normal"), (4, 5, 3, 20, "integer ties"))
+
+
+def _adaptive_model():
+    return oracle.Model(synth.make_weights(AD.SHAPE, 0)), synth.make_prompt(AD.SHAPE, 16, 0)
 
 
 def _pins(tw, tp):
@@ -184,6 +201,11 @@ def _pins(tw, tp):
         "tree_commit": TR.test_tree_commit_kv_moves_the_path,
         "tree_sdpa": TR.test_attention_tree_matches_sdpa_and_chain,
         "tree_forward": lambda: TR.test_forward_tree_rows_equal_root_path_forwards(tw, tp),
+        "tree_cycle": lambda: TR.test_tree_cycle_is_its_retyped_steps(tw, tp),
+        "tree_eq_ar": lambda: TR.test_greedy_tree_decoding_equals_ar(tw, tp, 8, 4, 20),
+        "iterative_pass2": lambda: P.test_iterative_draft_second_pass_sees_first_drafts(tw, tp),
+        "lossless_enum": lambda: P.test_sampled_orthrus_is_lossless_by_enumeration(0.7),
+        "adaptive_cycle": lambda: AD.test_adaptive_cycle_is_its_retyped_steps(_adaptive_model()),
         "entropy": AD.test_entropy_matches_scipy_and_closed_forms,
         "adaptive_len": AD.test_adaptive_len_worked_examples,
     }

@@ -235,3 +235,31 @@ def test_greedy_tree_decoding_equals_ar(tiny_weights, tiny_prompt, K, W, nodes):
     t = min(a["t"], tr["t"])
     assert np.array_equal(a["k_cache"][:, :t], tr["k_cache"][:, :t])
     assert np.array_equal(a["v_cache"][:, :t], tr["v_cache"][:, :t])
+
+
+def test_tree_cycle_is_its_retyped_steps(tiny_weights, tiny_prompt):
+    """A tree-verified cycle is: the draft at T = 0, numpy's log-softmax of
+    its rows 0 .. K-2 (the tokens at depths 1 .. K-1), the best-first tree
+    over them, one tree-masked AR forward of the anchor (the root) and the
+    nodes, the greedy walk and the K/V compaction.  Retyping four cycles from
+    those pinned pieces gives generate_tree's lengths and tokens."""
+    m = oracle.Model(tiny_weights)
+    K, W, nodes = 6, 3, 10
+    kc, vc = m.new_cache(len(tiny_prompt) + 64)
+    t = m.prefill(tiny_prompt, kc, vc)
+    anchor, out, ns = int(tiny_prompt[-1]), [], []
+    for _ in range(4):
+        _, _, z, _ = m.draft(kc, vc, t, anchor, K)
+        par, tok, _, _ = oracle.tree_build(_log_softmax(z[:K - 1]), W, nodes)
+        tok = tok.copy()
+        tok[0] = anchor
+        g = m.forward_tree(tok, par, t, kc, vc).argmax(axis=1)
+        n, emit, path = oracle.tree_accept(par, tok, g)
+        oracle.tree_commit_kv(kc, vc, t, path)
+        t += n
+        anchor = int(emit[-1])
+        out += [int(x) for x in emit]
+        ns.append(int(n))
+    assert max(ns) >= 2                                 # the walk and the compaction do run
+    r = m.generate_tree(tiny_prompt, K, W, nodes, len(out))
+    assert r["n_per_cycle"][:4].tolist() == ns and r["tokens"].tolist() == out
