@@ -71,10 +71,10 @@ def test_tokens_past_n_are_not_compared():
     pos = sum(n for n, _ in cyc[:-1])
     n, toks = cyc[-1]
     kept = 13 - pos
-    assert kept < n
-    cyc[-1] = (n, toks[:kept] + [(t + 1) % synth.TINY.vocab for t in toks[kept:]])
+    assert 0 < kept < n and len(toks) == kept          # the oracle keeps only the tokens up to N
+    cyc[-1] = (n, toks + [7] * (n - kept))             # a GPU cycle emits all n; the rest is free
     assert first_divergent_cycle(cyc, ref13, 13) == -1
-    cyc[-1] = (n, [(toks[0] + 1) % synth.TINY.vocab] + toks[1:])
+    cyc[-1] = (n, [(toks[0] + 1) % synth.TINY.vocab] + toks[1:] + [7] * (n - kept))
     assert first_divergent_cycle(cyc, ref13, 13) == len(cyc) - 1
 
 
