@@ -177,6 +177,8 @@ class Engine:
         self.dtype_name = dtype or shape.dtype
         self.tdtype = torch.bfloat16 if self.dtype_name == "bf16" else torch.float32
         self.device = torch.device(device)
+        if self.device.type != "cuda":
+            raise ValueError(f"Engine runs on a CUDA device only (got {self.device}); the library has no CPU path")
         n_layers = len(weights.layers)
         shape_l = type("S", (), {k: getattr(shape, k) for k in ("hidden", "n_q_heads", "n_kv_heads", "head_dim",
                                                                   "ffn", "vocab", "rope_theta", "rms_eps")})()

@@ -99,3 +99,16 @@ def test_null_arguments_rejected(pkg):
     assert lib.orthrus_verify_block(None, None, None, None, 1, 4, 0.0, None) == 1
     assert lib.orthrus_commit(None, None, 1, 4, 0.0, 0, None, None, None, None, None, None) == 1
     assert lib.orthrus_check_error(None, None, None) == 1
+
+
+def test_no_cpu_path(pkg, monkeypatch):
+    """The product path fails loudly instead of falling back: an engine on a
+    CPU device is refused before anything is allocated, and a missing
+    library raises instead of loading anything else."""
+    w = synth.make_weights(synth.TINY, 0)
+    with pytest.raises(ValueError, match="CUDA device only"):
+        pkg.Engine(synth.TINY, w, device="cpu")
+    monkeypatch.setattr(pkg, "_lib", None)
+    monkeypatch.setattr(pkg, "_LIB_PATH", os.path.join(ROOT, "no_such_dir", "liborthrus.so"))
+    with pytest.raises(ImportError, match="missing"):
+        pkg.lib()
