@@ -158,6 +158,8 @@ MUTANTS = (
     # the iterative draft (notes §5.4.2) and the exact law of the sampled cycle (notes §4.3)
     Mutant("second pass reads the drafts one row late", "oc_draft_iter", "s == 0 ? c->mask_id : draft[k - 1]",
            "s == 0 ? c->mask_id : draft[k]", ("iterative_pass2",)),
+    Mutant("two-pass proposal taken from the first pass", "oc_draft_iter", "if (last && q_probs) oc_softmax_t(",
+           "if (s == 0 && q_probs) oc_softmax_t(", ("proposal_last_pass", "sampler_mc_2pass")),
     Mutant("enumeration forgets the acceptance so far", "oc_enumerate_orthrus", "double rej = acc * (1.0 - a);",
            "double rej = 1.0 - a;", ("lossless_enum",)),
 )
@@ -191,7 +193,9 @@ def _pins(tw, tp):
         "greedy_examples": P.test_consensus_greedy_examples,
         "accept_residual": P.test_accept_and_residual,
         "greedy_eq_ar": lambda: [P.test_greedy_orthrus_equals_ar(tw, tp, K) for K in (1, 2, 4, 8)],
-        "sampler_mc": P.test_sampler_matches_ar_law_monte_carlo,
+        "sampler_mc": lambda: P.test_sampler_matches_ar_law_monte_carlo(1),
+        "sampler_mc_2pass": lambda: P.test_sampler_matches_ar_law_monte_carlo(2),
+        "proposal_last_pass": lambda: P.test_sampled_draft_proposal_is_the_last_pass(tw, tp),
         "block_mask_per_block": P.test_block_mask_equals_per_block_diffusion_attention,
         "block_mask_invisible": P.test_block_mask_blocks_are_mutually_invisible_and_anchor_excluded,
         "kl_scipy": P.test_kl_rows_matches_library_relative_entropy,

@@ -403,10 +403,12 @@ def test_sampled_orthrus_is_lossless_by_enumeration(T):
     assert 0.5 * np.abs(pa - m.enumerate_orthrus(pr, 1, 4, T)).sum() < 1e-9
 
 
-def test_sampler_matches_ar_law_monte_carlo():
+@pytest.mark.parametrize("iterations", [1, 2])
+def test_sampler_matches_ar_law_monte_carlo(iterations):
     """The oracle's real sampled decode (Philox uniforms, Gumbel drafts,
-    acceptance test, residual draw) against the exact AR law of the first two
-    tokens: chi-square over 6000 seeds on the micro model."""
+    acceptance test, residual draw; one draft pass or two) against the exact
+    AR law of the first two tokens: chi-square over 6000 seeds on the micro
+    model."""
     w = synth.make_weights(synth.MICRO, 0)
     m = oracle.Model(w)
     pr = synth.make_prompt(synth.MICRO, 3, 0)
@@ -414,7 +416,7 @@ def test_sampler_matches_ar_law_monte_carlo():
     n = 6000
     cnt = np.zeros(64)
     for s in range(n):
-        o = m.generate(pr, 3, 2, 1.0, s + 1, "orthrus")
+        o = m.generate(pr, 3, 2, 1.0, s + 1, "orthrus", iterations=iterations)
         cnt[o["tokens"][0] * 8 + o["tokens"][1]] += 1
     e = n * pa
     keep = e >= 5
@@ -429,6 +431,21 @@ def test_sampler_matches_ar_law_monte_carlo():
 # The paper-notes page (§5.4.2) compares single-step drafting with multi-step
 # iterative denoising; the iterative variant re-runs the diffusion view on
 # its own previous drafts (oc_draft_iter).
+
+def test_sampled_draft_proposal_is_the_last_pass(tiny_weights, tiny_prompt):
+    """At T > 0 the proposal q the acceptance test divides by is softmax(z/T)
+    of the pass whose drafts are proposed: the last one, whose logits the
+    draft returns (retyped through the plain forward on the previous pass's
+    drafts)."""
+    m = oracle.Model(tiny_weights)
+    kc, vc = m.new_cache(64)
+    t = m.prefill(tiny_prompt, kc, vc)
+    K, T, seed, step, a = 4, 0.9, 7, 1, int(tiny_prompt[-1])
+    d1, _, _, _ = m.draft(kc, vc, t, a, K, T, seed, step)
+    d2, q2, z2, _ = m.draft(kc, vc, t, a, K, T, seed, step, iterations=2)
+    assert np.array_equal(z2, m.forward(1, 1, [a] + list(d1[:K - 1]), t, kc.copy(), vc.copy()))
+    assert np.allclose(q2, torch.softmax(torch.from_numpy(z2) / T, 1).numpy(), rtol=1e-12, atol=1e-15)
+
 
 def test_iterative_draft_one_pass_is_the_draft(tiny_weights, tiny_prompt):
     m = oracle.Model(tiny_weights)
